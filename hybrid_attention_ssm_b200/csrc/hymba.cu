@@ -1,0 +1,874 @@
+// libhymba.so: the C ABI declared in include/hymba.h.  Host code validates arguments,
+// carves the workspace, encodes TMA tensor maps and enqueues the sm_100a kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/hymba.h"
+#include "attn.cuh"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "misc.cuh"
+#include "ssm.cuh"
+
+using namespace hymba;
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+#define HY_CUDA(call)                                                                     \
+  do {                                                                                    \
+    cudaError_t e_ = (call);                                                              \
+    if (e_ != cudaSuccess) return fail(HYMBA_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+#define HY_TRY(expr)            \
+  do {                          \
+    int rc_ = (expr);           \
+    if (rc_ != HYMBA_OK) return rc_; \
+  } while (0)
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ----------------------------------------------------------------------------------------
+// device properties and TMA descriptor encoding
+// ----------------------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct DeviceInfo {
+  int sms = 0;
+  int major = 0;
+  bool ok = false;
+};
+DeviceInfo g_dev[64];
+std::mutex g_mu;
+EncodeTiledFn g_encode = nullptr;
+
+int device_info(DeviceInfo** out) {
+  int dev = 0;
+  HY_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(HYMBA_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ok) {
+    HY_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+    HY_CUDA(cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev));
+    d.ok = true;
+  }
+  if (d.major != 10) return fail(HYMBA_ERR_UNSUPPORTED, "needs an sm_100 device (found major %d)", d.major);
+  if (g_encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    HY_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+    if (fn == nullptr || q != cudaDriverEntryPointSuccess)
+      return fail(HYMBA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  *out = &d;
+  return HYMBA_OK;
+}
+
+// A 2-D or 3-D tiled map with 128-byte swizzle; dims/strides innermost first, strides in
+// bytes for dims 1.. ; box inner extent must be 128 bytes.
+int make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int rank, const uint64_t* dims,
+             const uint64_t* strides_bytes, const uint32_t* box) {
+  if (!aligned16(base)) return fail(HYMBA_ERR_INVALID_ARG, "tensor base %p not 16-byte aligned", base);
+  cuuint64_t d[3], s[2];
+  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+  }
+  for (int i = 0; i < rank - 1; ++i) {
+    s[i] = strides_bytes[i];
+    if (s[i] % 16 != 0) return fail(HYMBA_ERR_INVALID_ARG, "tensor stride %llu not a multiple of 16", (unsigned long long)s[i]);
+  }
+  CUresult r = g_encode(m, dt, rank, const_cast<void*>(base), d, s, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(HYMBA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return HYMBA_OK;
+}
+
+// ----------------------------------------------------------------------------------------
+// GEMM launcher
+// ----------------------------------------------------------------------------------------
+struct GemmCall {
+  // A source 0 (optional): [rows0, K] row stride lda0 elements
+  const void* a0 = nullptr;
+  int rows0 = 0;
+  long long lda0 = 0;
+  // A source 1: [nb1, rows1, K], row stride lda1, batch stride a1_bstride (elements)
+  const void* a1 = nullptr;
+  int nb1 = 1, rows1 = 0;
+  long long lda1 = 0, a1_bstride = 0;
+  // B: [N, K] row stride ldb
+  const void* b = nullptr;
+  int N = 0;
+  long long ldb = 0;
+  int K = 0;
+  bool tf32 = false;
+  int bn = 256;
+  int split_k = 1;
+  GemmParams p{};
+};
+
+template <int BN, int STAGES, bool TF32>
+int launch_gemm_inst(const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& mb, const GemmParams& p,
+                     int grid, cudaStream_t st) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  constexpr int smem = GemmSmem<BN, STAGES>::TOTAL;
+  auto kern = gemm_tc_kernel<BN, STAGES, TF32>;
+  if (!attr_set[dev & 63]) {
+    HY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    attr_set[dev & 63] = true;
+  }
+  kern<<<grid, GEMM_THREADS, smem, st>>>(m0, m1, mb, p);
+  HY_CUDA(cudaGetLastError());
+  return HYMBA_OK;
+}
+
+int run_gemm(GemmCall& c, const DeviceInfo& dev, cudaStream_t st) {
+  const CUtensorMapDataType dt = c.tf32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const int esz = c.tf32 ? 4 : 2;
+  const uint32_t kbox = c.tf32 ? 32 : 64;
+  CUtensorMap m0, m1, mb;
+  {
+    const uint64_t dims[3] = {(uint64_t)c.K, (uint64_t)c.rows1, (uint64_t)c.nb1};
+    const uint64_t str[2] = {(uint64_t)c.lda1 * esz, (uint64_t)c.a1_bstride * esz};
+    const uint32_t box[3] = {kbox, (uint32_t)GEMM_BM, 1};
+    HY_TRY(make_map(&m1, c.a1, dt, 3, dims, str, box));
+  }
+  if (c.a0 != nullptr && c.rows0 > 0) {
+    const uint64_t dims[2] = {(uint64_t)c.K, (uint64_t)c.rows0};
+    const uint64_t str[1] = {(uint64_t)c.lda0 * esz};
+    const uint32_t box[2] = {kbox, (uint32_t)GEMM_BM};
+    HY_TRY(make_map(&m0, c.a0, dt, 2, dims, str, box));
+  } else {
+    m0 = m1;
+  }
+  {
+    const uint64_t dims[2] = {(uint64_t)c.K, (uint64_t)c.N};
+    const uint64_t str[1] = {(uint64_t)c.ldb * esz};
+    const uint32_t box[2] = {kbox, (uint32_t)c.bn};
+    HY_TRY(make_map(&mb, c.b, dt, 2, dims, str, box));
+  }
+  GemmParams& p = c.p;
+  p.tiles0 = (c.a0 != nullptr && c.rows0 > 0) ? cdiv(c.rows0, GEMM_BM) : 0;
+  p.rows0 = c.rows0;
+  p.nb1 = c.nb1;
+  p.rows1 = c.rows1;
+  p.tiles1 = cdiv(c.rows1, GEMM_BM);
+  p.N = c.N;
+  p.K = c.K;
+  p.n_tiles_n = cdiv(c.N, c.bn);
+  p.k_blocks = cdiv(c.K, kbox);
+  p.split_k = c.split_k < 1 ? 1 : (c.split_k > p.k_blocks ? p.k_blocks : c.split_k);
+  p.m_tiles = p.tiles0 + c.nb1 * p.tiles1;
+  p.total_tiles = p.m_tiles * p.n_tiles_n * p.split_k;
+  if (p.total_tiles <= 0) return HYMBA_OK;
+  const int grid = p.total_tiles < dev.sms ? p.total_tiles : dev.sms;
+  if (c.tf32) {
+    if (c.bn == 256) return launch_gemm_inst<256, 4, true>(m0, m1, mb, p, grid, st);
+    if (c.bn == 128) return launch_gemm_inst<128, 6, true>(m0, m1, mb, p, grid, st);
+  } else {
+    if (c.bn == 256) return launch_gemm_inst<256, 4, false>(m0, m1, mb, p, grid, st);
+    if (c.bn == 160) return launch_gemm_inst<160, 5, false>(m0, m1, mb, p, grid, st);
+    if (c.bn == 128) return launch_gemm_inst<128, 6, false>(m0, m1, mb, p, grid, st);
+    if (c.bn == 64) return launch_gemm_inst<64, 8, false>(m0, m1, mb, p, grid, st);
+  }
+  return fail(HYMBA_ERR_UNSUPPORTED, "no GEMM tile width %d", c.bn);
+}
+
+// smallest supported tile width covering n (for skinny N), else 256
+int pick_bn_cover(int n) {
+  if (n <= 64) return 64;
+  if (n <= 128) return 128;
+  if (n <= 160) return 160;
+  return 256;
+}
+// tile width for a wide N: 256 unless that leaves most SMs idle
+int pick_bn_wide(int m_tiles, int N, int sms) {
+  return (long long)m_tiles * cdiv(N, 256) >= sms ? 256 : 128;
+}
+
+void fill_rope_theta(double* theta, float base) {
+  for (int j = 0; j < 32; ++j) theta[j] = std::pow((double)base, -2.0 * j / 64.0);
+}
+
+// ----------------------------------------------------------------------------------------
+// validation and workspace layout
+// ----------------------------------------------------------------------------------------
+int check_cfg(const hymba_layer_cfg* c) {
+  if (c == nullptr) return fail(HYMBA_ERR_INVALID_ARG, "cfg is NULL");
+  if (c->head_dim != 64) return fail(HYMBA_ERR_UNSUPPORTED, "head_dim %d (only 64)", c->head_dim);
+  if (c->d_state != 16) return fail(HYMBA_ERR_UNSUPPORTED, "d_state %d (only 16)", c->d_state);
+  if (c->d_conv != 4) return fail(HYMBA_ERR_UNSUPPORTED, "d_conv %d (only 4)", c->d_conv);
+  if (c->d_model < 8 || c->d_model % 8) return fail(HYMBA_ERR_UNSUPPORTED, "d_model %d (multiple of 8)", c->d_model);
+  if (c->d_inner < 64 || c->d_inner % 64) return fail(HYMBA_ERR_UNSUPPORTED, "d_inner %d (multiple of 64)", c->d_inner);
+  if (c->n_q_heads < 1 || c->n_kv_heads < 1 || c->n_q_heads % c->n_kv_heads)
+    return fail(HYMBA_ERR_UNSUPPORTED, "heads %d/%d", c->n_q_heads, c->n_kv_heads);
+  if (c->n_q_heads / c->n_kv_heads > DEC_MAXG)
+    return fail(HYMBA_ERR_UNSUPPORTED, "more than %d query heads per KV head", DEC_MAXG);
+  if (c->dt_rank < 4 || c->dt_rank % 4 || c->dt_rank + 2 * c->d_state > 256)
+    return fail(HYMBA_ERR_UNSUPPORTED, "dt_rank %d", c->dt_rank);
+  if (c->window < 1 || c->n_meta < 0) return fail(HYMBA_ERR_INVALID_ARG, "window %d / n_meta %d", c->window, c->n_meta);
+  if (c->kv_role < 0 || c->kv_role > 2) return fail(HYMBA_ERR_INVALID_ARG, "kv_role %d", c->kv_role);
+  if (c->kv_role == HYMBA_KV_CONSUMER && c->is_global)
+    return fail(HYMBA_ERR_INVALID_ARG, "a global layer cannot consume a shared SWA cache");
+  if (!(c->rope_base > 1.f) || !(c->norm_eps >= 0.f)) return fail(HYMBA_ERR_INVALID_ARG, "rope_base/norm_eps");
+  return HYMBA_OK;
+}
+
+struct Dims {
+  int d, Hq, Hkv, D, Di, S, R, M, W;
+  int qw, kvw, P, xz_off, uw, ld_xbc;
+};
+Dims dims_of(const hymba_layer_cfg* c) {
+  Dims x;
+  x.d = c->d_model; x.Hq = c->n_q_heads; x.Hkv = c->n_kv_heads; x.D = c->head_dim; x.Di = c->d_inner;
+  x.S = c->d_state; x.R = c->dt_rank; x.M = c->n_meta; x.W = c->window;
+  x.qw = x.Hq * x.D;
+  x.kvw = x.Hkv * x.D;
+  const bool kv = c->kv_role != HYMBA_KV_CONSUMER;
+  x.P = x.qw + (kv ? 2 * x.kvw : 0) + 2 * x.Di;
+  x.xz_off = x.qw + (kv ? 2 * x.kvw : 0);
+  x.uw = x.qw + x.Di;
+  x.ld_xbc = (x.R + 2 * x.S + 3) & ~3;
+  return x;
+}
+
+struct PrefillWs {
+  size_t q, xz, xc, xcT, xbc, dT, y, o, u, sstate, cstate, total;
+  int T, Tp;
+};
+PrefillWs prefill_layout(const Dims& m, int B, int n_tokens, int x_has_meta) {
+  PrefillWs w;
+  w.T = x_has_meta ? n_tokens : m.M + n_tokens;
+  w.Tp = (w.T + 7) & ~7;
+  const size_t rows = (size_t)B * w.T;
+  size_t off = 256;
+  auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
+  w.q = take(rows * m.qw * 2);
+  w.xz = take(rows * 2 * m.Di * 2);
+  w.xc = take(rows * m.Di * 2);
+  w.xcT = take((size_t)B * m.Di * w.Tp * 2);
+  w.xbc = take(rows * m.ld_xbc * 4);
+  w.dT = take((size_t)B * m.Di * w.Tp * 4);
+  w.y = take(rows * m.Di * 2);
+  w.o = take(rows * m.qw * 2);
+  w.u = take(rows * m.uw * 2);
+  w.sstate = take((size_t)B * m.Di * 16 * 4);
+  w.cstate = take((size_t)B * m.Di * 3 * 4);
+  w.total = off;
+  return w;
+}
+
+struct DecodeWs {
+  size_t proj, part, o, xc, xbc, y, u, acc, total;
+  int n_splits;
+};
+DecodeWs decode_layout(const Dims& m, int B, int n_keys_max) {
+  DecodeWs w;
+  w.n_splits = cdiv(n_keys_max, DEC_KT);
+  size_t off = 256;
+  auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
+  w.proj = take((size_t)B * m.P * 2);
+  w.part = take((size_t)B * m.Hq * w.n_splits * 66 * 4);
+  w.o = take((size_t)B * m.qw * 2);
+  w.xc = take((size_t)B * m.Di * 2);
+  w.xbc = take((size_t)B * m.ld_xbc * 4);
+  w.y = take((size_t)B * m.Di * 2);
+  w.u = take((size_t)B * m.uw * 2);
+  w.acc = take((size_t)B * m.d * 4);
+  w.total = off;
+  return w;
+}
+
+// Decode keys: SWA reads at most M + W keys; a global layer up to max_tokens.
+int decode_max_keys(const hymba_layer_cfg* c, int max_tokens) {
+  return c->is_global ? max_tokens : c->n_meta + c->window;
+}
+
+int check_weights(const hymba_layer_weights* w, const Dims& m, bool need_meta) {
+  if (w == nullptr) return fail(HYMBA_ERR_INVALID_ARG, "weights is NULL");
+  const void* ptrs[] = {w->w_in, w->conv_w, w->conv_b, w->w_x, w->w_dt, w->dt_bias, w->A, w->g_attn, w->g_ssm, w->w_out};
+  for (const void* q : ptrs)
+    if (q == nullptr || !aligned16(q)) return fail(HYMBA_ERR_INVALID_ARG, "weight pointer NULL or not 16-byte aligned");
+  if (need_meta && m.M > 0 && (w->meta == nullptr || !aligned16(w->meta)))
+    return fail(HYMBA_ERR_INVALID_ARG, "meta tokens pointer");
+  if (w->w_dt_ld < m.R || w->w_dt_ld % 4) return fail(HYMBA_ERR_INVALID_ARG, "w_dt_ld %d", w->w_dt_ld);
+  return HYMBA_OK;
+}
+
+}  // namespace
+
+// ========================================================================================
+// C ABI
+// ========================================================================================
+extern "C" {
+
+int hymba_version(void) { return 10000; }
+
+const char* hymba_last_error(void) { return g_err.c_str(); }
+
+int hymba_set_wait_limit_ns(unsigned long long ns) {
+  HY_CUDA(cudaMemcpyToSymbol(g_wait_limit_ns, &ns, sizeof(ns)));
+  return HYMBA_OK;
+}
+
+int hymba_mixer_workspace_size(const hymba_layer_cfg* cfg, int batch, int n_tokens, int x_has_meta, int mode,
+                               size_t* bytes) {
+  HY_TRY(check_cfg(cfg));
+  if (bytes == nullptr || batch < 1) return fail(HYMBA_ERR_INVALID_ARG, "bytes NULL or batch < 1");
+  const Dims m = dims_of(cfg);
+  if (mode == HYMBA_MODE_PREFILL) {
+    if (n_tokens < 1) return fail(HYMBA_ERR_INVALID_ARG, "n_tokens < 1");
+    *bytes = prefill_layout(m, batch, n_tokens, x_has_meta).total;
+  } else if (mode == HYMBA_MODE_DECODE) {
+    // for a global layer n_tokens is the cache's max_tokens (keys read per step)
+    const int mk = cfg->is_global ? (n_tokens > 0 ? n_tokens : 1) : decode_max_keys(cfg, 0);
+    *bytes = decode_layout(m, batch, mk).total;
+  } else {
+    return fail(HYMBA_ERR_INVALID_ARG, "mode %d", mode);
+  }
+  return HYMBA_OK;
+}
+
+int hymba_mixer_stage_layout(const hymba_layer_cfg* cfg, int batch, int n_tokens, int x_has_meta,
+                             hymba_stage_layout* out) {
+  HY_TRY(check_cfg(cfg));
+  if (out == nullptr || batch < 1 || n_tokens < 1) return fail(HYMBA_ERR_INVALID_ARG, "stage layout args");
+  const Dims m = dims_of(cfg);
+  const PrefillWs w = prefill_layout(m, batch, n_tokens, x_has_meta);
+  out->q = w.q; out->xz = w.xz; out->xc = w.xc; out->xbc = w.xbc; out->delta = w.dT;
+  out->y = w.y; out->o = w.o; out->u = w.u;
+  out->ld_xbc = m.ld_xbc;
+  out->Tp = w.Tp;
+  return HYMBA_OK;
+}
+
+int hymba_workspace_init(void* ws, size_t ws_bytes, hymba_stream stream) {
+  if (ws == nullptr || ws_bytes < 256 || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(HYMBA_ERR_INVALID_ARG, "workspace NULL, < 256 bytes or not 256-byte aligned");
+  HY_CUDA(cudaMemsetAsync(ws, 0, 256, (cudaStream_t)stream));
+  return HYMBA_OK;
+}
+
+int hymba_status_read(void* ws, hymba_stream stream, int* status) {
+  if (ws == nullptr || status == nullptr) return fail(HYMBA_ERR_INVALID_ARG, "NULL argument");
+  DevStatus h;
+  HY_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
+  HY_CUDA(cudaMemcpy(&h, ws, sizeof(unsigned) * 2, cudaMemcpyDeviceToHost));
+  HY_CUDA(cudaMemset(ws, 0, 256));
+  *status = (h.flags & DEV_ERR_TIMEOUT) ? HYMBA_ERR_TIMEOUT : HYMBA_OK;
+  if (h.flags != 0) fail(*status, "device status flags 0x%x at site %u", h.flags, h.site);
+  return HYMBA_OK;
+}
+
+int hymba_kv_share_alloc(const hymba_layer_cfg* base, int n_layers, const uint8_t* is_global, int batch,
+                         int max_tokens, void* dev_buf, size_t buf_bytes, size_t* bytes_needed,
+                         int* layer_cache_id, int* layer_kv_role, hymba_kv_cache* caches, int max_caches,
+                         int* n_caches) {
+  if (base == nullptr || is_global == nullptr || layer_cache_id == nullptr || layer_kv_role == nullptr ||
+      bytes_needed == nullptr || n_caches == nullptr)
+    return fail(HYMBA_ERR_INVALID_ARG, "NULL argument");
+  if (n_layers < 1 || batch < 1 || max_tokens < 1) return fail(HYMBA_ERR_INVALID_ARG, "sizes");
+  if (base->head_dim < 1 || base->n_kv_heads < 1 || base->n_meta < 0 || base->window < 1)
+    return fail(HYMBA_ERR_INVALID_ARG, "cache sizes in base cfg");
+  // plan
+  int nc = 0;
+  int i = 0;
+  bool any_swa = false;
+  while (i < n_layers) {
+    if (is_global[i]) {
+      layer_cache_id[i] = nc++;
+      layer_kv_role[i] = HYMBA_KV_OWN;
+      i += 1;
+    } else if (i + 1 < n_layers && !is_global[i + 1]) {
+      layer_cache_id[i] = layer_cache_id[i + 1] = nc++;
+      layer_kv_role[i] = HYMBA_KV_PRODUCER;
+      layer_kv_role[i + 1] = HYMBA_KV_CONSUMER;
+      any_swa = true;
+      i += 2;
+    } else {
+      layer_cache_id[i] = nc++;
+      layer_kv_role[i] = HYMBA_KV_OWN;
+      any_swa = true;
+      i += 1;
+    }
+  }
+  *n_caches = nc;
+  const size_t row = (size_t)base->n_kv_heads * base->head_dim * 2;       // bytes per position
+  const size_t full = align256((size_t)batch * max_tokens * row);
+  const size_t meta = align256((size_t)batch * (base->n_meta > 0 ? base->n_meta : 1) * row);
+  const size_t ring = align256((size_t)batch * base->window * row);
+  size_t need = any_swa ? 2 * full : 0;     // shared prefill view
+  for (int l = 0; l < n_layers; ++l) {
+    const bool first = (l == 0) || layer_cache_id[l] != layer_cache_id[l - 1];
+    if (!first) continue;
+    need += is_global[l] ? 2 * full : 2 * (meta + ring);
+  }
+  *bytes_needed = need;
+  if (dev_buf == nullptr) return HYMBA_OK;
+  if (caches == nullptr || max_caches < nc) return fail(HYMBA_ERR_INVALID_ARG, "caches array too small (%d)", nc);
+  if (buf_bytes < need) return fail(HYMBA_ERR_WORKSPACE, "cache buffer %zu < %zu bytes", buf_bytes, need);
+  if (reinterpret_cast<uintptr_t>(dev_buf) & 255u) return fail(HYMBA_ERR_INVALID_ARG, "cache buffer not 256-byte aligned");
+  uint8_t* p = static_cast<uint8_t*>(dev_buf);
+  hymba_bf16 *view_k = nullptr, *view_v = nullptr;
+  if (any_swa) {
+    view_k = reinterpret_cast<hymba_bf16*>(p); p += full;
+    view_v = reinterpret_cast<hymba_bf16*>(p); p += full;
+  }
+  for (int l = 0; l < n_layers; ++l) {
+    const bool first = (l == 0) || layer_cache_id[l] != layer_cache_id[l - 1];
+    if (!first) continue;
+    hymba_kv_cache& c = caches[layer_cache_id[l]];
+    memset(&c, 0, sizeof(c));
+    c.batch = batch;
+    c.n_kv_heads = base->n_kv_heads;
+    c.head_dim = base->head_dim;
+    c.n_meta = base->n_meta;
+    c.window = base->window;
+    c.max_tokens = max_tokens;
+    if (is_global[l]) {
+      c.kind = HYMBA_CACHE_GLOBAL;
+      c.k = reinterpret_cast<hymba_bf16*>(p); p += full;
+      c.v = reinterpret_cast<hymba_bf16*>(p); p += full;
+    } else {
+      c.kind = HYMBA_CACHE_SWA;
+      c.meta_k = reinterpret_cast<hymba_bf16*>(p); p += meta;
+      c.meta_v = reinterpret_cast<hymba_bf16*>(p); p += meta;
+      c.ring_k = reinterpret_cast<hymba_bf16*>(p); p += ring;
+      c.ring_v = reinterpret_cast<hymba_bf16*>(p); p += ring;
+      c.k = view_k;
+      c.v = view_v;
+    }
+  }
+  return HYMBA_OK;
+}
+
+int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x,
+                        int x_has_meta, int B, int n_tokens, hymba_kv_cache* kv, float* ssm_state_out,
+                        float* conv_state_out, const hymba_bf16* residual, hymba_bf16* out, void* ws,
+                        size_t ws_bytes, hymba_stream stream) {
+  HY_TRY(check_cfg(cfg));
+  DeviceInfo* dev = nullptr;
+  HY_TRY(device_info(&dev));
+  const Dims m = dims_of(cfg);
+  if (B < 1 || n_tokens < 1) return fail(HYMBA_ERR_INVALID_ARG, "batch %d / n_tokens %d", B, n_tokens);
+  HY_TRY(check_weights(w, m, !x_has_meta));
+  if (x == nullptr || out == nullptr || kv == nullptr || !aligned16(x) || !aligned16(out))
+    return fail(HYMBA_ERR_INVALID_ARG, "x/out/kv pointer");
+  if (residual != nullptr && !aligned16(residual)) return fail(HYMBA_ERR_INVALID_ARG, "residual alignment");
+  const PrefillWs L = prefill_layout(m, B, n_tokens, x_has_meta);
+  const int T = L.T;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return fail(HYMBA_ERR_INVALID_ARG, "workspace");
+  if (ws_bytes < L.total) return fail(HYMBA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
+  if (kv->k == nullptr || kv->v == nullptr || kv->max_tokens < T || kv->batch < B || kv->n_kv_heads != m.Hkv ||
+      kv->head_dim != m.D)
+    return fail(HYMBA_ERR_INVALID_ARG, "kv cache view (k/v, max_tokens >= %d, batch, heads)", T);
+  const bool own_kv = cfg->kv_role != HYMBA_KV_CONSUMER;
+  if (own_kv && !cfg->is_global && kv->kind == HYMBA_CACHE_SWA &&
+      (kv->meta_k == nullptr && m.M > 0 || kv->ring_k == nullptr || kv->window != m.W || kv->n_meta != m.M))
+    return fail(HYMBA_ERR_INVALID_ARG, "SWA cache meta/ring buffers");
+  cudaStream_t st = (cudaStream_t)stream;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  DevStatus* status = reinterpret_cast<DevStatus*>(ws);
+  auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(wsb + off); };
+  auto f32 = [&](size_t off) { return reinterpret_cast<float*>(wsb + off); };
+  const size_t rows = (size_t)B * T;
+  const int Lmax = kv->max_tokens;
+
+  // 1. in_proj with RoPE on Q/K, scattering Q, K, V, x|z
+  {
+    GemmCall c;
+    if (!x_has_meta && m.M > 0) {
+      c.a0 = w->meta; c.rows0 = m.M; c.lda0 = m.d;
+      c.a1 = x; c.nb1 = B; c.rows1 = n_tokens; c.lda1 = m.d; c.a1_bstride = (long long)n_tokens * m.d;
+      c.p.row_off1 = m.M;
+    } else {
+      c.a1 = x; c.nb1 = B; c.rows1 = T; c.lda1 = m.d; c.a1_bstride = (long long)T * m.d;
+      c.p.row_off1 = 0;
+    }
+    c.b = w->w_in; c.N = m.P; c.ldb = m.d; c.K = m.d;
+    c.bn = 256;
+    c.p.mode = EPI_PROJ;
+    c.p.out_batches = B;
+    c.p.T_out = T;
+    c.p.status = status;
+    int ns = 0;
+    c.p.seg[ns++] = Segment{0, m.qw, bf(L.q), (long long)T * m.qw, m.qw, 1};
+    if (own_kv) {
+      c.p.seg[ns++] = Segment{m.qw, m.qw + m.kvw, kv->k, (long long)Lmax * m.kvw, m.kvw, 1};
+      c.p.seg[ns++] = Segment{m.qw + m.kvw, m.qw + 2 * m.kvw, kv->v, (long long)Lmax * m.kvw, m.kvw, 0};
+    }
+    c.p.seg[ns++] = Segment{m.xz_off, m.xz_off + 2 * m.Di, bf(L.xz), (long long)T * 2 * m.Di, 2 * m.Di, 0};
+    c.p.nseg = ns;
+    fill_rope_theta(c.p.rope_theta, cfg->rope_base);
+    HY_TRY(run_gemm(c, *dev, st));
+  }
+  // 2. conv1d + SiLU (writes xc, xcT and the conv state)
+  float* cstate = conv_state_out != nullptr ? conv_state_out : f32(L.cstate);
+  {
+    dim3 grid(cdiv(m.Di, CONV_CC), cdiv(T, CONV_TC), B);
+    conv1d_silu_kernel<<<grid, 256, 0, st>>>(bf(L.xz), 2 * m.Di, w->conv_w, w->conv_b, bf(L.xc), bf(L.xcT), cstate,
+                                              T, L.Tp, m.Di);
+    HY_CUDA(cudaGetLastError());
+  }
+  // 3. x_proj (split-K, fp32 atomics): [dt_low | B | C]
+  {
+    HY_CUDA(cudaMemsetAsync(f32(L.xbc), 0, rows * m.ld_xbc * 4, st));
+    GemmCall c;
+    c.a1 = bf(L.xc); c.nb1 = 1; c.rows1 = (int)rows; c.lda1 = m.Di; c.a1_bstride = (long long)rows * m.Di;
+    c.b = w->w_x; c.N = m.R + 2 * m.S; c.ldb = m.Di; c.K = m.Di;
+    c.bn = pick_bn_cover(c.N);
+    const int mt = cdiv(rows, GEMM_BM);
+    const int kb = cdiv(m.Di, 64);
+    int sk = cdiv(dev->sms, mt);
+    c.split_k = sk > kb ? kb : sk;
+    c.p.mode = EPI_ATOMIC_F32;
+    c.p.out = f32(L.xbc);
+    c.p.ld_out = m.ld_xbc;
+    c.p.n_valid = c.N;
+    c.p.status = status;
+    HY_TRY(run_gemm(c, *dev, st));
+  }
+  // 4. dt_proj (tf32) with softplus(+bias), stored time-major
+  {
+    GemmCall c;
+    c.tf32 = true;
+    c.a1 = f32(L.xbc); c.nb1 = B; c.rows1 = T; c.lda1 = m.ld_xbc; c.a1_bstride = (long long)T * m.ld_xbc;
+    c.b = w->w_dt; c.N = m.Di; c.ldb = w->w_dt_ld; c.K = m.R;
+    c.bn = pick_bn_wide(B * cdiv(T, GEMM_BM), m.Di, dev->sms);
+    c.p.mode = EPI_SOFTPLUS_T;
+    c.p.out = f32(L.dT);
+    c.p.T_out = L.Tp;
+    c.p.bias = w->dt_bias;
+    c.p.n_valid = m.Di;
+    c.p.status = status;
+    HY_TRY(run_gemm(c, *dev, st));
+  }
+  // 5. attention (block-skipped SWA + meta, or global causal)
+  {
+    CUtensorMap mq, mk, mv;
+    const uint32_t box[3] = {64, 128, 1};
+    {
+      const uint64_t dims[3] = {(uint64_t)m.qw, (uint64_t)T, (uint64_t)B};
+      const uint64_t str[2] = {(uint64_t)m.qw * 2, (uint64_t)T * m.qw * 2};
+      HY_TRY(make_map(&mq, bf(L.q), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dims, str, box));
+    }
+    {
+      const uint64_t dims[3] = {(uint64_t)m.kvw, (uint64_t)T, (uint64_t)B};
+      const uint64_t str[2] = {(uint64_t)m.kvw * 2, (uint64_t)Lmax * m.kvw * 2};
+      HY_TRY(make_map(&mk, kv->k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dims, str, box));
+      HY_TRY(make_map(&mv, kv->v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dims, str, box));
+    }
+    AttnParams ap;
+    ap.T = T; ap.Hq = m.Hq; ap.Hkv = m.Hkv; ap.n_meta = m.M; ap.window = m.W; ap.is_global = cfg->is_global;
+    ap.q_tiles = cdiv(T, 128);
+    ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)m.D));
+    ap.out = bf(L.o);
+    ap.ld_out = m.qw;
+    ap.status = status;
+    static bool attr[64] = {false};
+    int d = 0;
+    cudaGetDevice(&d);
+    if (!attr[d & 63]) {
+      HY_CUDA(cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ATT_SMEM));
+      attr[d & 63] = true;
+    }
+    dim3 grid(ap.q_tiles, m.Hq, B);
+    attn_fwd_kernel<<<grid, ATT_THREADS, ATT_SMEM, st>>>(mq, mk, mv, ap);
+    HY_CUDA(cudaGetLastError());
+  }
+  // 6. selective scan
+  float* sstate = ssm_state_out != nullptr ? ssm_state_out : f32(L.sstate);
+  {
+    dim3 grid(m.Di / SCAN_CH, B);
+    selective_scan_kernel<<<grid, SCAN_THREADS, 0, st>>>(bf(L.xcT), f32(L.dT), f32(L.xbc) + m.R, m.ld_xbc, w->A,
+                                                         bf(L.y), sstate, T, L.Tp, m.Di);
+    HY_CUDA(cudaGetLastError());
+  }
+  // 7. per-branch RMSNorm, gate, beta, average
+  {
+    branch_norm_avg_kernel<<<(unsigned)rows, 256, 0, st>>>(bf(L.o), m.qw, m.qw, bf(L.y), m.Di, bf(L.xz) + m.Di,
+                                                           2 * m.Di, m.Di, w->g_attn, w->g_ssm, cfg->norm_eps,
+                                                           bf(L.u), m.uw);
+    HY_CUDA(cudaGetLastError());
+  }
+  // 8. out_proj (+ residual)
+  {
+    GemmCall c;
+    c.a1 = bf(L.u); c.nb1 = 1; c.rows1 = (int)rows; c.lda1 = m.uw; c.a1_bstride = (long long)rows * m.uw;
+    c.b = w->w_out; c.N = m.d; c.ldb = m.uw; c.K = m.uw;
+    c.bn = pick_bn_wide(cdiv(rows, GEMM_BM), m.d, dev->sms);
+    c.p.mode = EPI_BF16;
+    c.p.out = out;
+    c.p.ld_out = m.d;
+    c.p.n_valid = m.d;
+    c.p.residual = reinterpret_cast<const __nv_bfloat16*>(residual);
+    c.p.ld_res = m.d;
+    c.p.status = status;
+    HY_TRY(run_gemm(c, *dev, st));
+  }
+  // 9. SWA decode cache: meta rows and the last W positions
+  if (own_kv && !cfg->is_global && kv->kind == HYMBA_CACHE_SWA) {
+    const int first_win = T - m.W > m.M ? T - m.W : m.M;
+    const int n_rows = m.M + (T - first_win);
+    const int n = n_rows * (m.kvw / 8);
+    dim3 grid(cdiv(n, 256), B);
+    swa_cache_finalize_kernel<<<grid, 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(kv->k), reinterpret_cast<const __nv_bfloat16*>(kv->v), Lmax, T, m.M,
+        m.W, m.kvw, reinterpret_cast<__nv_bfloat16*>(kv->meta_k), reinterpret_cast<__nv_bfloat16*>(kv->meta_v),
+        reinterpret_cast<__nv_bfloat16*>(kv->ring_k), reinterpret_cast<__nv_bfloat16*>(kv->ring_v));
+    HY_CUDA(cudaGetLastError());
+  }
+  return HYMBA_OK;
+}
+
+int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x, int B,
+                       int position, hymba_kv_cache* kv, float* ssm_state, float* conv_state,
+                       const hymba_bf16* residual, hymba_bf16* out, void* ws, size_t ws_bytes,
+                       hymba_stream stream) {
+  HY_TRY(check_cfg(cfg));
+  DeviceInfo* dev = nullptr;
+  HY_TRY(device_info(&dev));
+  const Dims m = dims_of(cfg);
+  if (B < 1) return fail(HYMBA_ERR_INVALID_ARG, "batch %d", B);
+  HY_TRY(check_weights(w, m, false));
+  if (x == nullptr || out == nullptr || kv == nullptr || ssm_state == nullptr || conv_state == nullptr ||
+      !aligned16(x) || !aligned16(out) || !aligned16(conv_state) || !aligned16(ssm_state))
+    return fail(HYMBA_ERR_INVALID_ARG, "x/out/kv/state pointer");
+  if (position < m.M) return fail(HYMBA_ERR_INVALID_ARG, "position %d < n_meta %d", position, m.M);
+  if (kv->batch < B || kv->n_kv_heads != m.Hkv || kv->head_dim != m.D)
+    return fail(HYMBA_ERR_INVALID_ARG, "kv cache shape");
+  const bool global = cfg->is_global != 0;
+  if (global) {
+    if (kv->kind != HYMBA_CACHE_GLOBAL || kv->k == nullptr || position >= kv->max_tokens)
+      return fail(HYMBA_ERR_INVALID_ARG, "global cache / position %d >= max_tokens", position);
+  } else {
+    if (kv->kind != HYMBA_CACHE_SWA || kv->ring_k == nullptr || (m.M > 0 && kv->meta_k == nullptr) ||
+        kv->window != m.W || kv->n_meta != m.M)
+      return fail(HYMBA_ERR_INVALID_ARG, "SWA cache");
+  }
+  const int max_keys = decode_max_keys(cfg, kv->max_tokens);
+  const DecodeWs L = decode_layout(m, B, max_keys);
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return fail(HYMBA_ERR_INVALID_ARG, "workspace");
+  if (ws_bytes < L.total) return fail(HYMBA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
+  cudaStream_t st = (cudaStream_t)stream;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  DevStatus* status = reinterpret_cast<DevStatus*>(ws);
+  auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(wsb + off); };
+  auto f32 = [&](size_t off) { return reinterpret_cast<float*>(wsb + off); };
+  const bool own_kv = cfg->kv_role != HYMBA_KV_CONSUMER;
+
+  // 1. in_proj, weights as the M operand (swap-AB), transposed store -> proj [B, P]
+  {
+    GemmCall c;
+    c.a1 = w->w_in; c.nb1 = 1; c.rows1 = m.P; c.lda1 = m.d; c.a1_bstride = (long long)m.P * m.d;
+    c.b = x; c.N = B; c.ldb = m.d; c.K = m.d;
+    c.bn = pick_bn_cover(B);
+    c.p.mode = EPI_BF16_T;
+    c.p.out = bf(L.proj);
+    c.p.ld_out = m.P;
+    c.p.m_valid = m.P;
+    c.p.n_valid = B;
+    c.p.status = status;
+    HY_TRY(run_gemm(c, *dev, st));
+  }
+  // 2. attention over meta + window (or the whole causal prefix), split-K, then combine
+  {
+    DecAttnParams ap;
+    ap.proj = bf(L.proj);
+    ap.ld_proj = m.P;
+    ap.Hq = m.Hq; ap.Hkv = m.Hkv; ap.M = m.M; ap.W = m.W; ap.is_global = global ? 1 : 0;
+    ap.write_kv = own_kv ? 1 : 0;
+    ap.p = position;
+    if (global) {
+      ap.n_keys = position + 1;
+    } else {
+      const int win0 = position - m.W + 1 > m.M ? position - m.W + 1 : m.M;
+      ap.n_keys = m.M + (position - win0 + 1);
+    }
+    ap.n_splits = cdiv(ap.n_keys, DEC_KT);
+    ap.meta_k = reinterpret_cast<__nv_bfloat16*>(kv->meta_k);
+    ap.meta_v = reinterpret_cast<__nv_bfloat16*>(kv->meta_v);
+    ap.ring_k = reinterpret_cast<__nv_bfloat16*>(kv->ring_k);
+    ap.ring_v = reinterpret_cast<__nv_bfloat16*>(kv->ring_v);
+    ap.full_k = reinterpret_cast<__nv_bfloat16*>(kv->k);
+    ap.full_v = reinterpret_cast<__nv_bfloat16*>(kv->v);
+    ap.Lmax = kv->max_tokens;
+    ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)m.D));
+    fill_rope_theta(ap.rope_theta, cfg->rope_base);
+    ap.part = f32(L.part);
+    if (ap.n_splits > L.n_splits) return fail(HYMBA_ERR_WORKSPACE, "decode workspace sized for fewer keys");
+    dim3 grid(ap.n_splits, m.Hkv, B);
+    decode_attn_kernel<<<grid, 128, 0, st>>>(ap);
+    HY_CUDA(cudaGetLastError());
+    decode_attn_combine_kernel<<<dim3(m.Hq, B), 64, 0, st>>>(f32(L.part), ap.n_splits, m.Hq, bf(L.o), m.qw);
+    HY_CUDA(cudaGetLastError());
+  }
+  // 3. conv step
+  {
+    const int n = B * m.Di;
+    decode_conv_kernel<<<cdiv(n, 256), 256, 0, st>>>(bf(L.proj), m.P, m.xz_off, m.Di, w->conv_w, w->conv_b,
+                                                      conv_state, bf(L.xc), B);
+    HY_CUDA(cudaGetLastError());
+  }
+  // 4. x_proj (swap-AB, split-K into fp32)
+  {
+    HY_CUDA(cudaMemsetAsync(f32(L.xbc), 0, (size_t)B * m.ld_xbc * 4, st));
+    GemmCall c;
+    c.a1 = w->w_x; c.nb1 = 1; c.rows1 = m.R + 2 * m.S; c.lda1 = m.Di; c.a1_bstride = (long long)c.rows1 * m.Di;
+    c.b = bf(L.xc); c.N = B; c.ldb = m.Di; c.K = m.Di;
+    c.bn = pick_bn_cover(B);
+    const int tiles = cdiv(c.rows1, GEMM_BM) * cdiv(B, c.bn);
+    c.split_k = cdiv(dev->sms, tiles);
+    c.p.mode = EPI_ATOMIC_F32_T;
+    c.p.out = f32(L.xbc);
+    c.p.ld_out = m.ld_xbc;
+    c.p.m_valid = c.rows1;
+    c.p.n_valid = B;
+    c.p.status = status;
+    HY_TRY(run_gemm(c, *dev, st));
+  }
+  // 5. dt_proj + softplus + state update + C.h + gate
+  {
+    dim3 grid(m.Di / 16, B);
+    decode_ssm_kernel<<<grid, 256, 0, st>>>(f32(L.xbc), m.ld_xbc, m.R, w->w_dt, w->w_dt_ld, w->dt_bias, w->A,
+                                            bf(L.xc), bf(L.proj), m.P, m.xz_off + m.Di, ssm_state, bf(L.y), m.Di);
+    HY_CUDA(cudaGetLastError());
+  }
+  // 6. norm + average (y already gated)
+  {
+    branch_norm_avg_kernel<<<B, 256, 0, st>>>(bf(L.o), m.qw, m.qw, bf(L.y), m.Di, nullptr, 0, m.Di, w->g_attn,
+                                              w->g_ssm, cfg->norm_eps, bf(L.u), m.uw);
+    HY_CUDA(cudaGetLastError());
+  }
+  // 7. out_proj (swap-AB, split-K) and the bf16 (+ residual) store
+  {
+    HY_CUDA(cudaMemsetAsync(f32(L.acc), 0, (size_t)B * m.d * 4, st));
+    GemmCall c;
+    c.a1 = w->w_out; c.nb1 = 1; c.rows1 = m.d; c.lda1 = m.uw; c.a1_bstride = (long long)m.d * m.uw;
+    c.b = bf(L.u); c.N = B; c.ldb = m.uw; c.K = m.uw;
+    c.bn = pick_bn_cover(B);
+    const int tiles = cdiv(m.d, GEMM_BM) * cdiv(B, c.bn);
+    c.split_k = cdiv(dev->sms, tiles);
+    c.p.mode = EPI_ATOMIC_F32_T;
+    c.p.out = f32(L.acc);
+    c.p.ld_out = m.d;
+    c.p.m_valid = m.d;
+    c.p.n_valid = B;
+    c.p.status = status;
+    HY_TRY(run_gemm(c, *dev, st));
+    const int n = B * m.d;
+    f32_to_bf16_residual_kernel<<<cdiv(n, 256), 256, 0, st>>>(
+        f32(L.acc), reinterpret_cast<const __nv_bfloat16*>(residual), reinterpret_cast<__nv_bfloat16*>(out), n);
+    HY_CUDA(cudaGetLastError());
+  }
+  return HYMBA_OK;
+}
+
+int hymba_gemm_bf16(const hymba_bf16* A, const hymba_bf16* Bm, const hymba_bf16* residual, hymba_bf16* C, int M,
+                    int N, int K, void* status_ws, hymba_stream stream) {
+  DeviceInfo* dev = nullptr;
+  HY_TRY(device_info(&dev));
+  if (A == nullptr || Bm == nullptr || C == nullptr || M < 1 || N < 8 || K < 8 || N % 8 || K % 8 || !aligned16(C))
+    return fail(HYMBA_ERR_INVALID_ARG, "gemm arguments");
+  GemmCall c;
+  c.a1 = A; c.nb1 = 1; c.rows1 = M; c.lda1 = K; c.a1_bstride = (long long)M * K;
+  c.b = Bm; c.N = N; c.ldb = K; c.K = K;
+  c.bn = pick_bn_wide(cdiv(M, GEMM_BM), N, dev->sms);
+  c.p.mode = EPI_BF16;
+  c.p.out = C;
+  c.p.ld_out = N;
+  c.p.n_valid = N;
+  c.p.residual = reinterpret_cast<const __nv_bfloat16*>(residual);
+  c.p.ld_res = N;
+  c.p.status = reinterpret_cast<DevStatus*>(status_ws);
+  return run_gemm(c, *dev, (cudaStream_t)stream);
+}
+
+int hymba_rmsnorm(const hymba_bf16* x, const float* gain, int rows, int d, float eps, hymba_bf16* out,
+                  hymba_stream stream) {
+  if (x == nullptr || gain == nullptr || out == nullptr || rows < 1 || d < 8 || d % 8 || !aligned16(x) ||
+      !aligned16(out))
+    return fail(HYMBA_ERR_INVALID_ARG, "rmsnorm arguments");
+  rmsnorm_kernel<<<rows, 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<const __nv_bfloat16*>(x), gain, d, eps,
+                                                          reinterpret_cast<__nv_bfloat16*>(out));
+  HY_CUDA(cudaGetLastError());
+  return HYMBA_OK;
+}
+
+int hymba_ffn_swiglu(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hymba_bf16* w_down, int rows, int d,
+                     int F, hymba_bf16* act, const hymba_bf16* residual, hymba_bf16* out, void* status_ws,
+                     hymba_stream stream) {
+  DeviceInfo* dev = nullptr;
+  HY_TRY(device_info(&dev));
+  if (h == nullptr || w_gate_up == nullptr || w_down == nullptr || act == nullptr || out == nullptr || rows < 1 ||
+      d < 8 || d % 8 || F < 64 || F % 64 || !aligned16(act) || !aligned16(out))
+    return fail(HYMBA_ERR_INVALID_ARG, "ffn arguments");
+  cudaStream_t st = (cudaStream_t)stream;
+  {
+    GemmCall c;
+    c.a1 = h; c.nb1 = 1; c.rows1 = rows; c.lda1 = d; c.a1_bstride = (long long)rows * d;
+    c.b = w_gate_up; c.N = 2 * F; c.ldb = d; c.K = d;
+    c.bn = pick_bn_wide(cdiv(rows, GEMM_BM), 2 * F, dev->sms);
+    c.p.mode = EPI_SWIGLU;
+    c.p.out = act;
+    c.p.ld_out = F;
+    c.p.n_valid = 2 * F;
+    c.p.status = reinterpret_cast<DevStatus*>(status_ws);
+    HY_TRY(run_gemm(c, *dev, st));
+  }
+  {
+    GemmCall c;
+    c.a1 = act; c.nb1 = 1; c.rows1 = rows; c.lda1 = F; c.a1_bstride = (long long)rows * F;
+    c.b = w_down; c.N = d; c.ldb = F; c.K = F;
+    c.bn = pick_bn_wide(cdiv(rows, GEMM_BM), d, dev->sms);
+    c.p.mode = EPI_BF16;
+    c.p.out = out;
+    c.p.ld_out = d;
+    c.p.n_valid = d;
+    c.p.residual = reinterpret_cast<const __nv_bfloat16*>(residual);
+    c.p.ld_res = d;
+    c.p.status = reinterpret_cast<DevStatus*>(status_ws);
+    HY_TRY(run_gemm(c, *dev, st));
+  }
+  return HYMBA_OK;
+}
+
+int hymba_selftest_wait_timeout(void* ws, size_t ws_bytes, hymba_stream stream) {
+  if (ws == nullptr || ws_bytes < 256 || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(HYMBA_ERR_INVALID_ARG, "workspace");
+  wait_timeout_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(reinterpret_cast<DevStatus*>(ws));
+  HY_CUDA(cudaGetLastError());
+  return HYMBA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,241 @@
+// SSM branch kernels (prefill): causal depthwise conv1d + SiLU, and the selective scan.
+#pragma once
+#include "common.cuh"
+
+namespace hymba {
+
+// ----------------------------------------------------------------------------------------
+// conv1d (kernel width 4) + SiLU over time, per channel.
+//   x      [B*T, ld_x] bf16, channel c at column c (the x part of the in_proj output)
+//   xc     [B*T, Di]   bf16 row-major (A operand of x_proj)
+//   xcT    [B, Di, Tp] bf16 time-major (input of the scan), row stride Tp (multiple of 8)
+//   state  [B, Di, 3]  fp32: the last 3 inputs x[T-3..T-1] (zero before the start)
+// CTA: 64 channels x 64 time steps, 256 threads.
+// ----------------------------------------------------------------------------------------
+constexpr int CONV_TC = 64, CONV_CC = 64, CONV_K = 4;
+
+__global__ void __launch_bounds__(256)
+    conv1d_silu_kernel(const __nv_bfloat16* __restrict__ x, int ld_x, const float* __restrict__ w,
+                       const float* __restrict__ bias, __nv_bfloat16* __restrict__ xc,
+                       __nv_bfloat16* __restrict__ xcT, float* __restrict__ state, int T, int Tp, int Di) {
+  __shared__ float xs[CONV_TC + CONV_K - 1][CONV_CC + 1];
+  __shared__ __nv_bfloat16 ot[CONV_CC][CONV_TC + 8];
+  const int c0 = blockIdx.x * CONV_CC;
+  const int t0 = blockIdx.y * CONV_TC;
+  const int b = blockIdx.z;
+  const int tid = threadIdx.x;
+  // load x[t0-3 .. t0+63][c0 .. c0+63] (zero outside [0, T))
+  for (int i = tid; i < (CONV_TC + CONV_K - 1) * (CONV_CC / 8); i += 256) {
+    const int rr = i / (CONV_CC / 8), cv = (i % (CONV_CC / 8)) * 8;
+    const int t = t0 - (CONV_K - 1) + rr;
+    float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (t >= 0 && t < T && c0 + cv < Di) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(x + ((size_t)b * T + t) * ld_x + c0 + cv);
+      const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = __bfloat162float(hv[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) xs[rr][cv + e] = v[e];
+  }
+  __syncthreads();
+  // compute: thread -> channel (tid % 64), time rows (tid / 64) + 4k
+  const int cl = tid & 63;
+  const int c = c0 + cl;
+  float wk[CONV_K], bc = 0.f;
+#pragma unroll
+  for (int k = 0; k < CONV_K; ++k) wk[k] = c < Di ? w[c * CONV_K + k] : 0.f;
+  if (c < Di) bc = bias[c];
+  for (int tl = tid >> 6; tl < CONV_TC; tl += 4) {
+    float acc = bc;
+#pragma unroll
+    for (int k = 0; k < CONV_K; ++k) acc += wk[k] * xs[tl + k][cl];
+    const float y = acc / (1.f + __expf(-acc));
+    const __nv_bfloat16 yb = __float2bfloat16_rn(y);
+    ot[cl][tl] = yb;
+    const int t = t0 + tl;
+    if (t < T && c < Di) xc[((size_t)b * T + t) * Di + c] = yb;
+  }
+  __syncthreads();
+  // time-major store: row = channel, 64 contiguous time steps (8 x 16 B)
+  for (int i = tid; i < CONV_CC * (CONV_TC / 8); i += 256) {
+    const int ch = i / (CONV_TC / 8), tv = (i % (CONV_TC / 8)) * 8;
+    const int cc = c0 + ch, t = t0 + tv;
+    if (cc >= Di || t >= T) continue;
+    __nv_bfloat16* dst = xcT + ((size_t)b * Di + cc) * Tp + t;
+    if (t + 8 <= T) {
+      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(&ot[ch][tv]);
+    } else {
+      for (int e = 0; e < 8 && t + e < T; ++e) dst[e] = ot[ch][tv + e];
+    }
+  }
+  // conv state: the last 3 inputs (zero when T < 3)
+  if (t0 <= T - 1 && T - 1 < t0 + CONV_TC && tid < CONV_CC && c0 + tid < Di) {
+    for (int k = 0; k < CONV_K - 1; ++k) {
+      const int t = T - (CONV_K - 1) + k;       // absolute time
+      const int rr = t - t0 + (CONV_K - 1);      // row in xs
+      state[((size_t)b * Di + c0 + tid) * (CONV_K - 1) + k] = (t >= 0) ? xs[rr][tid] : 0.f;
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------------------
+// Selective scan, time-sequential per (channel, state) thread.
+//   h_t = exp(delta_t * A[c,s]) h_{t-1} + delta_t * B_t[s] * x_t ;  y_t = sum_s C_t[s] h_t[s]
+// 16 lanes of a warp hold the 16 states of one channel; the sum over states is a
+// reduce-scatter through 8 shuffles per 8 time steps.  The fp32 state stays in registers
+// for the whole sequence.  Inputs are staged through shared memory in chunks of 64 steps
+// (cp.async for the time-major x and delta, register transpose for B/C), 3 stages deep.
+//   xcT [B, Di, Tp] bf16; dT [B, Di, Tp] fp32 (Tp: row stride, multiple of 8; steps at or
+//   beyond T read as zero, so delta = 0 leaves the state unchanged); bc [B*T, ld_bc] fp32 (B at col 0..15, C at
+//   16..31 of the pointer); A [Di, 16]; y [B*T, Di] bf16 (not gated); state [B, Di, 16].
+// ----------------------------------------------------------------------------------------
+constexpr int SCAN_CH = 8;            // channels per CTA
+constexpr int SCAN_TC = 64;           // time steps per chunk
+constexpr int SCAN_NST = 3;           // pipeline stages
+constexpr int SCAN_THREADS = SCAN_CH * 16;
+
+struct ScanStage {
+  __nv_bfloat16 x[SCAN_CH][SCAN_TC];  // 8 x 128 B
+  float d[SCAN_CH][SCAN_TC];          // 8 x 256 B
+  float bcT[32][SCAN_TC + 4];         // [state (B 0..15, C 16..31)][t]
+};
+
+__global__ void __launch_bounds__(SCAN_THREADS)
+    selective_scan_kernel(const __nv_bfloat16* __restrict__ xcT, const float* __restrict__ dT,
+                          const float* __restrict__ bc, int ld_bc, const float* __restrict__ A,
+                          __nv_bfloat16* __restrict__ y, float* __restrict__ state, int T, int Tp, int Di) {
+  __shared__ __align__(16) ScanStage st[SCAN_NST];
+  __shared__ __align__(16) __nv_bfloat16 ys[SCAN_TC][SCAN_CH];
+  const int tid = threadIdx.x;
+  const int cl = tid >> 4;         // channel within CTA
+  const int s = tid & 15;          // state
+  const int c0 = blockIdx.x * SCAN_CH;
+  const int b = blockIdx.y;
+  const int c = c0 + cl;
+  const int n_chunks = (T + SCAN_TC - 1) / SCAN_TC;
+  const float A2 = A[(size_t)c * 16 + s] * 1.4426950408889634f;   // exp(d*A) = 2^(d*A*log2 e)
+
+  // async loads of the time-major x / delta rows of chunk k into stage k % NST
+  auto load_xd = [&](int k) {
+    ScanStage& S = st[k % SCAN_NST];
+    const int t0 = k * SCAN_TC;
+    // x: 8 channels x 8 pieces of 16 B; delta: 8 channels x 16 pieces
+    for (int i = tid; i < SCAN_CH * 24; i += SCAN_THREADS) {
+      const int ch = i / 24, piece = i % 24;
+      if (piece < 8) {
+        const int t = t0 + piece * 8;
+        const int nbytes = t >= T ? 0 : min(16, (T - t) * 2);
+        const __nv_bfloat16* src = xcT + ((size_t)b * Di + c0 + ch) * Tp + (t >= T ? 0 : t);
+        cp_async16(&S.x[ch][piece * 8], src, nbytes);
+      } else {
+        const int t = t0 + (piece - 8) * 4;
+        const int nbytes = t >= T ? 0 : min(16, (T - t) * 4);
+        const float* src = dT + ((size_t)b * Di + c0 + ch) * Tp + (t >= T ? 0 : t);
+        cp_async16(&S.d[ch][(piece - 8) * 4], src, nbytes);
+      }
+    }
+  };
+  // B/C of chunk k: 64 rows x 32 floats, loaded into registers (16 per thread) ...
+  float bcr[16];
+  auto load_bc = [&](int k) {
+    const int t0 = k * SCAN_TC;
+    const int row = tid >> 1, half = (tid & 1) * 16;
+    const int t = t0 + row;
+#pragma unroll
+    for (int e = 0; e < 16; e += 4) {
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (t < T) v = *reinterpret_cast<const float4*>(bc + ((size_t)b * T + t) * ld_bc + half + e);
+      bcr[e] = v.x; bcr[e + 1] = v.y; bcr[e + 2] = v.z; bcr[e + 3] = v.w;
+    }
+  };
+  // ... and stored transposed ([state][t]) into the stage
+  auto store_bc = [&](int k) {
+    ScanStage& S = st[k % SCAN_NST];
+    const int row = tid >> 1, half = (tid & 1) * 16;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) S.bcT[half + e][row] = bcr[e];
+  };
+
+  // prologue: chunks 0 .. NST-2
+  for (int k = 0; k < SCAN_NST - 1; ++k) {
+    if (k < n_chunks) {
+      load_xd(k);
+      load_bc(k);
+      store_bc(k);
+    }
+    cp_async_commit();
+  }
+
+  float h = 0.f;
+  const int l = tid & 15;
+  const int my_step = ((l >> 3) & 1) * 4 + ((l >> 2) & 1) * 2 + ((l >> 1) & 1);
+  for (int k = 0; k < n_chunks; ++k) {
+    const int kn = k + SCAN_NST - 1;
+    cp_async_wait<SCAN_NST - 2>();
+    __syncthreads();                       // chunk k visible; stage of chunk k-1 free
+    if (kn < n_chunks) {
+      load_xd(kn);
+      load_bc(kn);
+    }
+    cp_async_commit();
+    const ScanStage& S = st[k % SCAN_NST];
+#pragma unroll 1
+    for (int tt = 0; tt < SCAN_TC; tt += 8) {
+      const uint4 xr = *reinterpret_cast<const uint4*>(&S.x[cl][tt]);
+      const __nv_bfloat16* xh = reinterpret_cast<const __nv_bfloat16*>(&xr);
+      const float4 d0 = *reinterpret_cast<const float4*>(&S.d[cl][tt]);
+      const float4 d1 = *reinterpret_cast<const float4*>(&S.d[cl][tt + 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&S.bcT[s][tt]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&S.bcT[s][tt + 4]);
+      const float4 e0 = *reinterpret_cast<const float4*>(&S.bcT[16 + s][tt]);
+      const float4 e1 = *reinterpret_cast<const float4*>(&S.bcT[16 + s][tt + 4]);
+      const float dv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      const float cv[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float a = ex2_approx(dv[u] * A2);
+        h = fmaf(a, h, dv[u] * __bfloat162float(xh[u]) * bv[u]);
+        v[u] = cv[u] * h;
+      }
+      // reduce-scatter of v[0..7] over the 16 state lanes: lane l ends with the full sum
+      // of step my_step (lanes l and l^1 hold the same step)
+      const bool q3 = l & 8, q2 = l & 4, q1 = l & 2;
+      float w4[4];
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const float send = q3 ? v[k4] : v[k4 + 4];
+        const float keep = q3 ? v[k4 + 4] : v[k4];
+        w4[k4] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+      }
+      float w2[2];
+#pragma unroll
+      for (int k2 = 0; k2 < 2; ++k2) {
+        const float send = q2 ? w4[k2] : w4[k2 + 2];
+        const float keep = q2 ? w4[k2 + 2] : w4[k2];
+        w2[k2] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+      }
+      float w1;
+      {
+        const float send = q1 ? w2[0] : w2[1];
+        const float keep = q1 ? w2[1] : w2[0];
+        w1 = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+      }
+      w1 += __shfl_xor_sync(0xffffffffu, w1, 1);
+      if ((l & 1) == 0) ys[tt + my_step][cl] = __float2bfloat16_rn(w1);
+    }
+    if (kn < n_chunks) store_bc(kn);
+    __syncthreads();
+    // flush y rows of this chunk: 64 rows x 16 B
+    if (tid < SCAN_TC) {
+      const int t = k * SCAN_TC + tid;
+      if (t < T)
+        *reinterpret_cast<uint4*>(y + ((size_t)b * T + t) * Di + c0) = *reinterpret_cast<const uint4*>(&ys[tid][0]);
+    }
+  }
+  state[((size_t)b * Di + c) * 16 + s] = h;
+}
+
+}  // namespace hymba

@@ -1,0 +1,269 @@
+"""ctypes binding of libhymba.so (argument marshalling only).
+
+Every computation happens in the library's CUDA kernels; this module only turns torch
+tensors (device memory allocated by PyTorch) into the pointers and structs of the C ABI
+declared in include/hymba.h.  It raises if the library is missing: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhymba.so")
+HEADER_PATH = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "hymba.h")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
+KV_OWN, KV_PRODUCER, KV_CONSUMER = 0, 1, 2
+CACHE_SWA, CACHE_GLOBAL = 0, 1
+MODE_PREFILL, MODE_DECODE = 0, 1
+
+_c_int, _c_size, _vp = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+
+
+class HymbaError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"hymba error {code}: {msg}")
+        self.code = code
+
+
+class LayerCfg(ctypes.Structure):
+    _fields_ = [(n, _c_int) for n in ("d_model", "n_q_heads", "n_kv_heads", "head_dim", "d_inner",
+                                       "d_state", "d_conv", "dt_rank", "window", "n_meta",
+                                       "is_global", "kv_role")] + \
+               [("rope_base", ctypes.c_float), ("norm_eps", ctypes.c_float)]
+
+
+class LayerWeights(ctypes.Structure):
+    _fields_ = [("meta", _vp), ("w_in", _vp), ("conv_w", _vp), ("conv_b", _vp), ("w_x", _vp),
+                ("w_dt", _vp), ("w_dt_ld", _c_int), ("dt_bias", _vp), ("A", _vp),
+                ("g_attn", _vp), ("g_ssm", _vp), ("w_out", _vp)]
+
+
+class KVCache(ctypes.Structure):
+    _fields_ = [(n, _c_int) for n in ("kind", "batch", "n_kv_heads", "head_dim", "n_meta",
+                                       "window", "max_tokens")] + \
+               [(n, _vp) for n in ("meta_k", "meta_v", "ring_k", "ring_v", "k", "v")]
+
+
+class StageLayout(ctypes.Structure):
+    _fields_ = [(n, _c_size) for n in ("q", "xz", "xc", "xbc", "delta", "y", "o", "u")] + \
+               [("ld_xbc", _c_int), ("Tp", _c_int)]
+
+
+_LIB = None
+
+
+def header_functions():
+    """Names of the functions include/hymba.h declares."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^(?:int|const char\*)\s+(hymba_\w+)\s*\(", text, flags=re.M)))
+
+
+def lib():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with __graft_entry__.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        sig = {
+            "hymba_version": ([], _c_int),
+            "hymba_last_error": ([], ctypes.c_char_p),
+            "hymba_mixer_workspace_size": ([ctypes.POINTER(LayerCfg), _c_int, _c_int, _c_int, _c_int,
+                                            ctypes.POINTER(_c_size)], _c_int),
+            "hymba_workspace_init": ([_vp, _c_size, _vp], _c_int),
+            "hymba_status_read": ([_vp, _vp, ctypes.POINTER(_c_int)], _c_int),
+            "hymba_kv_share_alloc": ([ctypes.POINTER(LayerCfg), _c_int, ctypes.POINTER(ctypes.c_uint8),
+                                      _c_int, _c_int, _vp, _c_size, ctypes.POINTER(_c_size),
+                                      ctypes.POINTER(_c_int), ctypes.POINTER(_c_int),
+                                      ctypes.POINTER(KVCache), _c_int, ctypes.POINTER(_c_int)], _c_int),
+            "hymba_mixer_prefill": ([ctypes.POINTER(LayerCfg), ctypes.POINTER(LayerWeights), _vp, _c_int,
+                                     _c_int, _c_int, ctypes.POINTER(KVCache), _vp, _vp, _vp, _vp, _vp,
+                                     _c_size, _vp], _c_int),
+            "hymba_mixer_decode": ([ctypes.POINTER(LayerCfg), ctypes.POINTER(LayerWeights), _vp, _c_int,
+                                    _c_int, ctypes.POINTER(KVCache), _vp, _vp, _vp, _vp, _vp, _c_size,
+                                    _vp], _c_int),
+            "hymba_mixer_stage_layout": ([ctypes.POINTER(LayerCfg), _c_int, _c_int, _c_int,
+                                          ctypes.POINTER(StageLayout)], _c_int),
+            "hymba_gemm_bf16": ([_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp], _c_int),
+            "hymba_rmsnorm": ([_vp, _vp, _c_int, _c_int, ctypes.c_float, _vp, _vp], _c_int),
+            "hymba_ffn_swiglu": ([_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp], _c_int),
+            "hymba_set_wait_limit_ns": ([ctypes.c_ulonglong], _c_int),
+            "hymba_selftest_wait_timeout": ([_vp, _c_size, _vp], _c_int),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _LIB = L
+    return _LIB
+
+
+def check(rc):
+    if rc != OK:
+        raise HymbaError(rc, lib().hymba_last_error().decode())
+    return rc
+
+
+def ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def stream_handle(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+# ---------------------------------------------------------------------------------------
+# configuration / weights / caches
+# ---------------------------------------------------------------------------------------
+def make_cfg(dims) -> LayerCfg:
+    return LayerCfg(dims.d_model, dims.n_q_heads, dims.n_kv_heads, dims.head_dim, dims.d_inner,
+                    dims.d_state, dims.d_conv, dims.dt_rank, dims.window, dims.n_meta,
+                    int(dims.is_global), int(dims.kv_role), float(dims.rope_base), float(dims.norm_eps))
+
+
+_BF16_W = ("meta", "w_in", "w_x", "w_out")
+_F32_W = ("conv_w", "conv_b", "dt_bias", "A", "g_attn", "g_ssm")
+
+
+class DeviceWeights:
+    """A layer's weights in device memory plus the C struct pointing at them."""
+
+    def __init__(self, w: dict, device="cuda"):
+        self.t = {}
+        for k in _BF16_W:
+            self.t[k] = torch.from_numpy(np.ascontiguousarray(w[k], dtype=np.float32)).to(device).to(torch.bfloat16)
+        for k in _F32_W:
+            self.t[k] = torch.from_numpy(np.ascontiguousarray(w[k], dtype=np.float32)).to(device)
+        wdt = np.ascontiguousarray(w["w_dt"], dtype=np.float32)
+        ld = (wdt.shape[1] + 3) // 4 * 4
+        pad = np.zeros((wdt.shape[0], ld), dtype=np.float32)
+        pad[:, :wdt.shape[1]] = wdt
+        self.t["w_dt"] = torch.from_numpy(pad).to(device)
+        self.c = LayerWeights(ptr(self.t["meta"]), ptr(self.t["w_in"]), ptr(self.t["conv_w"]),
+                              ptr(self.t["conv_b"]), ptr(self.t["w_x"]), ptr(self.t["w_dt"]), ld,
+                              ptr(self.t["dt_bias"]), ptr(self.t["A"]), ptr(self.t["g_attn"]),
+                              ptr(self.t["g_ssm"]), ptr(self.t["w_out"]))
+
+
+class Cache:
+    """A KV cache (SWA meta + ring + prefill view, or global) owned by torch tensors."""
+
+    def __init__(self, dims, batch, max_tokens, kind=None, device="cuda", view=None):
+        kind = (CACHE_GLOBAL if dims.is_global else CACHE_SWA) if kind is None else kind
+        Hkv, D = dims.n_kv_heads, dims.head_dim
+        z = lambda *s: torch.zeros(*s, Hkv, D, dtype=torch.bfloat16, device=device)
+        self.t = {}
+        if view is None:
+            self.t["k"], self.t["v"] = z(batch, max_tokens), z(batch, max_tokens)
+        else:
+            self.t["k"], self.t["v"] = view
+        if kind == CACHE_SWA:
+            self.t["meta_k"], self.t["meta_v"] = z(batch, max(dims.n_meta, 1)), z(batch, max(dims.n_meta, 1))
+            self.t["ring_k"], self.t["ring_v"] = z(batch, dims.window), z(batch, dims.window)
+        g = lambda n: ptr(self.t[n]) if n in self.t else None
+        self.c = KVCache(kind, batch, Hkv, D, dims.n_meta, dims.window, max_tokens,
+                         g("meta_k"), g("meta_v"), g("ring_k"), g("ring_v"), g("k"), g("v"))
+
+
+def workspace_size(dims, batch, n_tokens, x_has_meta=0, mode=MODE_PREFILL):
+    n = ctypes.c_size_t()
+    cfg = make_cfg(dims)
+    check(lib().hymba_mixer_workspace_size(ctypes.byref(cfg), batch, n_tokens, x_has_meta, mode, ctypes.byref(n)))
+    return n.value
+
+
+def alloc_workspace(nbytes, device="cuda", stream=None):
+    ws = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+    off = (-ws.data_ptr()) % 256
+    view = ws[off:off + nbytes]
+    check(lib().hymba_workspace_init(ptr(view), nbytes, stream_handle(stream)))
+    return view
+
+
+def stage_layout(dims, batch, n_tokens, x_has_meta=0) -> StageLayout:
+    out = StageLayout()
+    cfg = make_cfg(dims)
+    check(lib().hymba_mixer_stage_layout(ctypes.byref(cfg), batch, n_tokens, x_has_meta, ctypes.byref(out)))
+    return out
+
+
+def status_read(ws, stream=None) -> int:
+    s = ctypes.c_int()
+    check(lib().hymba_status_read(ptr(ws), stream_handle(stream), ctypes.byref(s)))
+    return s.value
+
+
+def kv_share_alloc(base_dims, is_global, batch, max_tokens, dev_buf=None):
+    """Returns (bytes_needed, cache_id list, role list, caches list)."""
+    n = len(is_global)
+    cfg = make_cfg(base_dims)
+    g = (ctypes.c_uint8 * n)(*[int(v) for v in is_global])
+    cid, role = (ctypes.c_int * n)(), (ctypes.c_int * n)()
+    need = ctypes.c_size_t()
+    caches = (KVCache * n)()
+    nc = ctypes.c_int()
+    buf_bytes = 0 if dev_buf is None else dev_buf.numel() * dev_buf.element_size()
+    check(lib().hymba_kv_share_alloc(ctypes.byref(cfg), n, g, batch, max_tokens, ptr(dev_buf), buf_bytes,
+                                     ctypes.byref(need), cid, role, caches, n, ctypes.byref(nc)))
+    return need.value, list(cid), list(role), [caches[i] for i in range(nc.value)]
+
+
+# ---------------------------------------------------------------------------------------
+# entry points
+# ---------------------------------------------------------------------------------------
+def mixer_prefill(dims, dw: DeviceWeights, x, kv: Cache, out, ws, x_has_meta=0, ssm_state=None,
+                  conv_state=None, residual=None, stream=None, cfg=None):
+    cfg = make_cfg(dims) if cfg is None else cfg
+    B, n_tokens = x.shape[0], x.shape[1]
+    check(lib().hymba_mixer_prefill(ctypes.byref(cfg), ctypes.byref(dw.c), ptr(x), x_has_meta, B, n_tokens,
+                                    ctypes.byref(kv.c), ptr(ssm_state), ptr(conv_state), ptr(residual), ptr(out),
+                                    ptr(ws), ws.numel(), stream_handle(stream)))
+
+
+def mixer_decode(dims, dw: DeviceWeights, x, position, kv: Cache, ssm_state, conv_state, out, ws, residual=None,
+                 stream=None, cfg=None):
+    cfg = make_cfg(dims) if cfg is None else cfg
+    check(lib().hymba_mixer_decode(ctypes.byref(cfg), ctypes.byref(dw.c), ptr(x), x.shape[0], position,
+                                   ctypes.byref(kv.c), ptr(ssm_state), ptr(conv_state), ptr(residual), ptr(out),
+                                   ptr(ws), ws.numel(), stream_handle(stream)))
+
+
+def gemm_bf16(A, B, C, status_ws, residual=None, stream=None):
+    M, K = A.shape
+    N = B.shape[0]
+    check(lib().hymba_gemm_bf16(ptr(A), ptr(B), ptr(residual), ptr(C), M, N, K, ptr(status_ws),
+                                stream_handle(stream)))
+
+
+def rmsnorm(x, gain, eps, out, stream=None):
+    rows, d = x.shape
+    check(lib().hymba_rmsnorm(ptr(x), ptr(gain), rows, d, eps, ptr(out), stream_handle(stream)))
+
+
+def ffn_swiglu(h, w_gate_up, w_down, act, out, status_ws, residual=None, stream=None):
+    rows, d = h.shape
+    F = w_down.shape[1]
+    check(lib().hymba_ffn_swiglu(ptr(h), ptr(w_gate_up), ptr(w_down), rows, d, F, ptr(act), ptr(residual),
+                                 ptr(out), ptr(status_ws), stream_handle(stream)))
+
+
+def interleave_gate_up(w_gate, w_up):
+    """Stack gate and up rows in blocks of 32, the layout hymba_ffn_swiglu reads."""
+    F, d = w_gate.shape
+    g = w_gate.reshape(F // 32, 32, d)
+    u = w_up.reshape(F // 32, 32, d)
+    return np.concatenate([g, u], axis=1).reshape(2 * F, d)
+
+
+def set_wait_limit_ns(ns):
+    check(lib().hymba_set_wait_limit_ns(int(ns)))
+
+
+def selftest_wait_timeout(ws, stream=None):
+    check(lib().hymba_selftest_wait_timeout(ptr(ws), ws.numel(), stream_handle(stream)))

@@ -1,0 +1,251 @@
+/*
+ * hymba.h - C ABI of libhymba.so, the B200 (sm_100a) implementation of the Hymba
+ * hybrid-head mixer forward pass (prefill and decode) and its cross-layer KV sharing.
+ *
+ * The method (cited by page title and section; [JJ] and [MC] below):
+ *   [JJ] juejin.cn post "NVIDIA提出Hymba网络，Mamba+Attenation解决transformer的长序列低效难题"
+ *     §数学表示 1   meta tokens R prepended: X~ = [R, X]
+ *     §数学表示 2   one input projection W_in = [W_Q, W_K, W_V, W_SSM, W_G]
+ *     §数学表示 3   attention heads, eq. (1): softmax(Q K^T) V
+ *     §数学表示 4   SSM heads, eq. (2): alpha_ij = C_i prod exp(A Delta_k) B_j Delta_j,
+ *                   gated by G
+ *     §数学表示 5   per-branch normalisation, beta1/beta2 rescale, average, W_out
+ *     §Hymba 的整体架构  global attention in the first/middle/last blocks, sliding-window
+ *                   attention elsewhere, adjacent SWA blocks share one KV cache
+ *   [MC] model card "Hymba-1.5B-Base" §模型架构: GQA, RoPE, 16 SSM states, meta tokens visible
+ *     to every later token even under sliding-window attention.
+ * Readings where the pages are silent (1/sqrt(D) scale and causal mask; window = the last
+ * `window` positions including the query; half-split RoPE; Euler discretisation
+ * exp(Delta A), Delta B; no D skip term; SiLU gate; RMSNorm; W_out over the concatenation
+ * of both normalised branches times 1/2) are the ones the fp64 oracle states.
+ *
+ * Conventions for every entry point
+ *   - Returns HYMBA_OK (0) or an HYMBA_ERR_* code; hymba_last_error() gives a message
+ *     (thread-local, valid until the next call from the same thread).
+ *   - The library never allocates device memory.  The caller passes device pointers it
+ *     owns (inputs, outputs, weights, caches, workspace); the library keeps no pointer after
+ *     a call returns.
+ *   - Work is enqueued on `stream` (a cudaStream_t) and is asynchronous; no entry point
+ *     synchronises except hymba_status_read.  Calls may be captured in a CUDA graph.
+ *   - bf16 tensors are raw bfloat16 bits (uint16_t), row-major, contiguous unless a
+ *     leading dimension is given.  fp32 tensors are float, row-major.
+ *   - Device pointers must be 16-byte aligned; the workspace must be 256-byte aligned.
+ *   - Errors found on the device (a bounded wait that timed out) are OR'ed into a status
+ *     word at the start of the workspace and read with hymba_status_read.
+ */
+#ifndef HYMBA_H
+#define HYMBA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  HYMBA_OK = 0,
+  HYMBA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer */
+  HYMBA_ERR_UNSUPPORTED = 2,  /* shape outside what the kernels implement, or not sm_100 */
+  HYMBA_ERR_WORKSPACE = 3,    /* workspace smaller than hymba_mixer_workspace_size */
+  HYMBA_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed (message has details) */
+  HYMBA_ERR_TIMEOUT = 5,      /* status word: a device-side bounded wait gave up */
+};
+
+enum { HYMBA_KV_OWN = 0, HYMBA_KV_PRODUCER = 1, HYMBA_KV_CONSUMER = 2 };
+enum { HYMBA_CACHE_SWA = 0, HYMBA_CACHE_GLOBAL = 1 };
+enum { HYMBA_MODE_PREFILL = 0, HYMBA_MODE_DECODE = 1 };
+
+typedef uint16_t hymba_bf16;
+typedef struct CUstream_st* hymba_stream; /* identical to cudaStream_t; NULL = legacy stream */
+
+/* One mixer layer's sizes ([MC] §模型架构, [JJ] §数学表示).
+ * Supported: head_dim 64, d_state 16, d_conv 4, d_model % 8 == 0, d_inner % 64 == 0,
+ * n_q_heads % n_kv_heads == 0 with at most 6 query heads per KV head, dt_rank % 4 == 0 and
+ * dt_rank + 2*d_state <= 256, window >= 1, n_meta >= 0. */
+typedef struct hymba_layer_cfg {
+  int d_model;     /* d */
+  int n_q_heads;   /* Hq */
+  int n_kv_heads;  /* Hkv (GQA: query head h reads KV head h*Hkv/Hq) */
+  int head_dim;    /* D */
+  int d_inner;     /* Di, SSM channels */
+  int d_state;     /* S */
+  int d_conv;      /* causal conv width */
+  int dt_rank;     /* R */
+  int window;      /* W: a query sees the last W positions (itself included) plus the meta tokens */
+  int n_meta;      /* M meta tokens */
+  int is_global;   /* 1: full causal attention; 0: sliding window + meta */
+  int kv_role;     /* HYMBA_KV_OWN / PRODUCER (writes the shared cache) / CONSUMER (reads it) */
+  float rope_base; /* RoPE base (theta_j = base^(-2j/D)) */
+  float norm_eps;  /* RMSNorm epsilon */
+} hymba_layer_cfg;
+
+/* One layer's weights, all device pointers.
+ *   meta    [M, d]            bf16  meta tokens R
+ *   w_in    [P, d]            bf16  rows [Q (Hq*D) | K (Hkv*D) | V (Hkv*D) | x (Di) | z (Di)];
+ *                                   a consumer layer has no K and V rows (P = Hq*D + 2*Di)
+ *   conv_w  [Di, 4]           fp32  causal conv taps, tap 3 multiplies the current input
+ *   conv_b  [Di]              fp32
+ *   w_x     [R + 2S, Di]      bf16  rows [dt_low (R) | B (S) | C (S)]
+ *   w_dt    [Di, w_dt_ld]     fp32  first R columns used; w_dt_ld >= R, w_dt_ld % 4 == 0
+ *   dt_bias [Di]              fp32  Delta = softplus(dt_low W_dt^T + dt_bias)
+ *   A       [Di, S]           fp32  (negative) state matrix
+ *   g_attn  [Hq*D]            fp32  beta1
+ *   g_ssm   [Di]              fp32  beta2
+ *   w_out   [d, Hq*D + Di]    bf16  output projection */
+typedef struct hymba_layer_weights {
+  const hymba_bf16* meta;
+  const hymba_bf16* w_in;
+  const float* conv_w;
+  const float* conv_b;
+  const hymba_bf16* w_x;
+  const float* w_dt;
+  int w_dt_ld;
+  const float* dt_bias;
+  const float* A;
+  const float* g_attn;
+  const float* g_ssm;
+  const hymba_bf16* w_out;
+} hymba_layer_weights;
+
+/* A KV cache, shared by a producer/consumer pair of adjacent SWA layers or owned by one
+ * layer ([JJ] §Hymba 的整体架构).  All device pointers, bf16, K stored after RoPE.
+ *   kind HYMBA_CACHE_SWA:
+ *     meta_k, meta_v  [B, M, Hkv, D]   keys/values of the meta tokens
+ *     ring_k, ring_v  [B, W, Hkv, D]   input position p (>= M) lives in slot (p - M) mod W
+ *     k, v            [B, max_tokens, Hkv, D]  prefill view: the producer's prefill writes
+ *                     every position here, the consumer's prefill reads it (may be shared
+ *                     between caches when layers run in order)
+ *   kind HYMBA_CACHE_GLOBAL:
+ *     k, v            [B, max_tokens, Hkv, D]  position p at row p (prefill and decode)
+ */
+typedef struct hymba_kv_cache {
+  int kind;
+  int batch;
+  int n_kv_heads;
+  int head_dim;
+  int n_meta;
+  int window;
+  int max_tokens;
+  hymba_bf16* meta_k;
+  hymba_bf16* meta_v;
+  hymba_bf16* ring_k;
+  hymba_bf16* ring_v;
+  hymba_bf16* k;
+  hymba_bf16* v;
+} hymba_kv_cache;
+
+/* Library version (major*10000 + minor*100 + patch). */
+int hymba_version(void);
+
+/* Message of the last error raised on this thread ("" if none). */
+const char* hymba_last_error(void);
+
+/* Bytes of workspace one prefill (mode HYMBA_MODE_PREFILL, n_tokens rows per sequence) or
+ * decode step (HYMBA_MODE_DECODE, n_tokens ignored) needs.  x_has_meta: see prefill. */
+int hymba_mixer_workspace_size(const hymba_layer_cfg* cfg, int batch, int n_tokens, int x_has_meta, int mode,
+                               size_t* bytes);
+
+/* Zero the status word of a workspace (call once after allocating it). */
+int hymba_workspace_init(void* workspace, size_t ws_bytes, hymba_stream stream);
+
+/* Synchronise `stream`, copy the workspace status word to *status (0, or HYMBA_ERR_TIMEOUT
+ * when a device-side wait gave up), and clear it. */
+int hymba_status_read(void* workspace, hymba_stream stream, int* status);
+
+/* Plan and carve the KV caches of an n_layers stack ([JJ] §Hymba 的整体架构: adjacent SWA
+ * blocks share one cache; global blocks keep their own).  Layers are walked in order; an
+ * SWA layer followed by an SWA layer opens a pair (producer, consumer); an SWA layer whose
+ * successor is global or absent keeps its own cache.
+ *   base        sizes (n_kv_heads, head_dim, n_meta, window) shared by all layers
+ *   is_global   [n_layers] host array, 1 = full attention
+ *   batch, max_tokens   sequences and maximum positions (meta included) per sequence
+ *   dev_buf     device buffer to carve, or NULL to only compute *bytes_needed and the plan
+ *   layer_cache_id, layer_kv_role   [n_layers] host outputs
+ *   caches      [max_caches] host outputs (filled when dev_buf != NULL), *n_caches = count
+ * All SWA caches share one prefill view (k, v).  No kernel runs; nothing is zeroed. */
+int hymba_kv_share_alloc(const hymba_layer_cfg* base, int n_layers, const uint8_t* is_global, int batch,
+                         int max_tokens, void* dev_buf, size_t buf_bytes, size_t* bytes_needed,
+                         int* layer_cache_id, int* layer_kv_role, hymba_kv_cache* caches, int max_caches,
+                         int* n_caches);
+
+/* Prefill of one mixer layer over `batch` sequences ([JJ] §数学表示 1-6).
+ *   x          x_has_meta == 0: [B, n_tokens, d] input tokens; the meta tokens are prepended
+ *              (T = M + n_tokens).  x_has_meta == 1: [B, n_tokens, d] rows that already
+ *              start with the meta positions (T = n_tokens), as inside a stack.
+ *   kv         own/producer: K (after RoPE) and V of every position are written to kv->k/v
+ *              (max_tokens >= T) and, for an SWA cache, the meta rows and the last W
+ *              positions to meta_k/v and ring_k/v.  consumer: reads kv->k/v.
+ *   ssm_state_out  [B, Di, S] fp32 final SSM state, or NULL
+ *   conv_state_out [B, Di, 3] fp32 last three conv inputs, or NULL
+ *   residual   [B, T, d] bf16 added to the output, or NULL
+ *   out        [B, T, d] bf16 (all rows, meta rows included)
+ * Errors: INVALID_ARG (null/misaligned pointer, batch or n_tokens < 1, max_tokens < T),
+ * UNSUPPORTED (shape, device), WORKSPACE (too small), CUDA. */
+int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x,
+                        int x_has_meta, int batch, int n_tokens, hymba_kv_cache* kv, float* ssm_state_out,
+                        float* conv_state_out, const hymba_bf16* residual, hymba_bf16* out, void* workspace,
+                        size_t ws_bytes, hymba_stream stream);
+
+/* One decode step for `batch` sequences that all sit at position `position` (= M + number
+ * of tokens already in the context; the pages' released model generates with equal-length
+ * sequences).  x [B, d] bf16.  own/producer: the new K (after RoPE) and V go to ring slot
+ * (position - M) mod W (SWA) or row `position` (global) before attending; consumer: the
+ * producer's step must already have run.  ssm_state [B, Di, S] and conv_state [B, Di, 3]
+ * fp32 are read and updated in place.  residual [B, d] or NULL; out [B, d] bf16.
+ * Errors as prefill; INVALID_ARG also when position < M or (global) position >= max_tokens. */
+int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x, int batch,
+                       int position, hymba_kv_cache* kv, float* ssm_state, float* conv_state,
+                       const hymba_bf16* residual, hymba_bf16* out, void* workspace, size_t ws_bytes,
+                       hymba_stream stream);
+
+/* Byte offsets, inside a prefill workspace, of the stage buffers of the last prefill (for
+ * stage-by-stage checks).  Layouts (rows r = b*T + t):
+ *   q      [B*T, Hq*D]  bf16  queries after RoPE
+ *   xz     [B*T, 2*Di]  bf16  in_proj x | z columns
+ *   xc     [B*T, Di]    bf16  SiLU(conv(x))
+ *   xbc    [B*T, ld_xbc] fp32 x_proj output: dt_low | B | C
+ *   delta  [B, Di, Tp]  fp32  Delta, time-major with row stride Tp
+ *   y      [B*T, Di]    bf16  scan output before the gate
+ *   o      [B*T, Hq*D]  bf16  attention output
+ *   u      [B*T, Hq*D+Di] bf16 normalised, rescaled, averaged branches (out_proj input) */
+typedef struct hymba_stage_layout {
+  size_t q, xz, xc, xbc, delta, y, o, u;
+  int ld_xbc;
+  int Tp;
+} hymba_stage_layout;
+int hymba_mixer_stage_layout(const hymba_layer_cfg* cfg, int batch, int n_tokens, int x_has_meta,
+                             hymba_stage_layout* out);
+
+/* C[M, N] = A[M, K] * B[N, K]^T (+ residual[M, N]) on the tcgen05 GEMM, bf16 in/out, fp32
+ * accumulation.  K % 8 == 0, N % 8 == 0.  status_ws: a workspace (>= 256 bytes) whose
+ * status word receives device-side errors. */
+int hymba_gemm_bf16(const hymba_bf16* A, const hymba_bf16* B, const hymba_bf16* residual, hymba_bf16* C, int M,
+                    int N, int K, void* status_ws, hymba_stream stream);
+
+/* Stack harness pieces (one Hymba block = x + mixer(norm(x)), then + FFN(norm(.))):
+ * out[r, :] = x[r, :] / sqrt(mean(x[r, :]^2) + eps) * gain, rows x d bf16. */
+int hymba_rmsnorm(const hymba_bf16* x, const float* gain, int rows, int d, float eps, hymba_bf16* out,
+                  hymba_stream stream);
+
+/* SwiGLU FFN with residual: out = residual + W_down (SiLU(W_gate h) * (W_up h)).
+ *   h [rows, d] bf16; w_gate_up [2F, d] bf16 with gate and up rows interleaved in blocks of
+ *   32 (rows 64i..64i+31 = gate rows 32i.., rows 64i+32..64i+63 = up rows 32i..);
+ *   w_down [d, F] bf16; act [rows, F] bf16 scratch; residual [rows, d] or NULL; F % 64 == 0. */
+int hymba_ffn_swiglu(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hymba_bf16* w_down, int rows, int d,
+                     int F, hymba_bf16* act, const hymba_bf16* residual, hymba_bf16* out, void* status_ws,
+                     hymba_stream stream);
+
+/* Upper bound, in nanoseconds, of every device-side wait on an mbarrier (default 2e9).
+ * A wait that runs out records HYMBA_ERR_TIMEOUT in the status word and the kernel returns. */
+int hymba_set_wait_limit_ns(unsigned long long ns);
+
+/* Launch a kernel whose only wait is on a barrier nothing ever arrives at, so that the
+ * bounded wait runs out; the status word of `workspace` then reads HYMBA_ERR_TIMEOUT.
+ * Exercises the timeout path without faulting or hanging the device. */
+int hymba_selftest_wait_timeout(void* workspace, size_t ws_bytes, hymba_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HYMBA_H */

@@ -1,0 +1,100 @@
+"""Shared test helpers: tolerance checks and running the CUDA path on seeded inputs."""
+import numpy as np
+import torch
+
+from hybrid_attention_ssm_b200 import hymba as H
+from hybrid_attention_ssm_b200 import synth
+
+BF16_TOL = 2e-2      # max|err| <= 2e-2 * RMS(ref) for bf16 paths
+SCAN_TOL = 1e-4      # ||err||_inf <= 1e-4 * ||ref||_inf for the fp32 scan state
+
+
+def assert_rms(got, ref, tol=BF16_TOL, name=""):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, f"{name}: shape {got.shape} vs {ref.shape}"
+    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    err = float(np.max(np.abs(got - ref)))
+    assert err <= tol * rms, f"{name}: max|err| {err:.4e} > {tol} * RMS {rms:.4e} (ratio {err / max(rms, 1e-300):.3e})"
+    return err / max(rms, 1e-300)
+
+
+def assert_rel_inf(got, ref, tol=SCAN_TOL, name=""):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    den = float(np.max(np.abs(ref)))
+    err = float(np.max(np.abs(got - ref)))
+    assert err <= tol * den, f"{name}: inf-norm err {err:.4e} > {tol} * {den:.4e}"
+    return err / max(den, 1e-300)
+
+
+def to_np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def bf16_dev(a, device="cuda"):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device).to(torch.bfloat16)
+
+
+def f32_dev(a, device="cuda"):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+
+
+def ws_view(ws, off, shape, dtype):
+    """A typed view into the byte workspace at byte offset `off`."""
+    n = int(np.prod(shape))
+    es = torch.tensor([], dtype=dtype).element_size()
+    return ws[off:off + n * es].view(dtype).view(*shape)
+
+
+class PrefillRun:
+    """Runs hymba_mixer_prefill once on seeded inputs and keeps every buffer."""
+
+    def __init__(self, dims, w, X, x_has_meta=0, cache=None, residual=None, max_tokens=None):
+        self.dims, self.w = dims, w
+        B, n = X.shape[0], X.shape[1]
+        T = n if x_has_meta else dims.n_meta + n
+        self.T = T
+        self.dw = H.DeviceWeights(w)
+        self.x = bf16_dev(X)
+        self.cache = cache if cache is not None else H.Cache(dims, B, max_tokens or T)
+        self.out = torch.zeros(B, T, dims.d_model, dtype=torch.bfloat16, device="cuda")
+        self.ssm = torch.zeros(B, dims.d_inner, dims.d_state, dtype=torch.float32, device="cuda")
+        self.conv = torch.zeros(B, dims.d_inner, dims.d_conv - 1, dtype=torch.float32, device="cuda")
+        self.res = None if residual is None else bf16_dev(residual)
+        nbytes = H.workspace_size(dims, B, n, x_has_meta)
+        self.ws = H.alloc_workspace(nbytes)
+        H.mixer_prefill(dims, self.dw, self.x, self.cache, self.out, self.ws, x_has_meta=x_has_meta,
+                        ssm_state=self.ssm, conv_state=self.conv, residual=self.res)
+        torch.cuda.synchronize()
+        assert H.status_read(self.ws) == 0
+        self.layout = H.stage_layout(dims, B, n, x_has_meta)
+        self.B = B
+
+    def stage(self, name):
+        d, L, B, T = self.dims, self.layout, self.B, self.T
+        rows = B * T
+        if name == "q":
+            return to_np(ws_view(self.ws, L.q, (B, T, d.n_q_heads, d.head_dim), torch.bfloat16))
+        if name == "xz":
+            return to_np(ws_view(self.ws, L.xz, (B, T, 2 * d.d_inner), torch.bfloat16))
+        if name == "xc":
+            return to_np(ws_view(self.ws, L.xc, (B, T, d.d_inner), torch.bfloat16))
+        if name == "xbc":
+            return to_np(ws_view(self.ws, L.xbc, (B, T, L.ld_xbc), torch.float32))
+        if name == "delta":
+            dT = to_np(ws_view(self.ws, L.delta, (B, d.d_inner, L.Tp), torch.float32))
+            return np.transpose(dT[:, :, :T], (0, 2, 1))
+        if name == "y":
+            return to_np(ws_view(self.ws, L.y, (B, T, d.d_inner), torch.bfloat16))
+        if name == "o":
+            return to_np(ws_view(self.ws, L.o, (B, T, d.n_q_heads * d.head_dim), torch.bfloat16))
+        if name == "u":
+            return to_np(ws_view(self.ws, L.u, (B, T, d.attn_width + d.d_inner), torch.bfloat16))
+        raise KeyError(name)
+
+    def kv(self):
+        T = self.T
+        return to_np(self.cache.t["k"][:, :T]), to_np(self.cache.t["v"][:, :T])

@@ -1,0 +1,76 @@
+"""The C ABI library on the host: it loads without a GPU, exports every function that
+include/hymba.h declares, and its host-only logic (workspace sizing, stage layout, KV
+sharing plan, argument validation) behaves as documented."""
+import ctypes
+
+import numpy as np
+import pytest
+
+from hybrid_attention_ssm_b200 import build as hbuild
+from hybrid_attention_ssm_b200 import hymba as H
+from hybrid_attention_ssm_b200 import synth
+from oracle import hymba_oracle as orc
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    hbuild.build()
+    H.lib()
+
+
+def test_exports_every_declared_function():
+    names = H.header_functions()
+    assert len(names) >= 14
+    L = ctypes.CDLL(H.LIB_PATH)
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/hymba.h but not exported"
+    assert H.lib().hymba_version() >= 10000
+
+
+def test_workspace_sizes_grow_with_tokens():
+    d = synth.workloads()["swa"].dims
+    a = H.workspace_size(d, 1, 2048)
+    b = H.workspace_size(d, 1, 4096)
+    assert 0 < a < b
+    lay = H.stage_layout(d, 1, 2048)
+    offs = [lay.q, lay.xz, lay.xc, lay.xbc, lay.delta, lay.y, lay.o, lay.u]
+    assert all(o % 256 == 0 for o in offs) and offs == sorted(offs) and offs[-1] < a
+    assert lay.Tp % 8 == 0 and lay.Tp >= 2176 and lay.ld_xbc >= 132
+    dec = H.workspace_size(d, 64, 0, 0, H.MODE_DECODE)
+    assert dec > 0
+
+
+@pytest.mark.parametrize("field,value,code", [("head_dim", 32, H.ERR_UNSUPPORTED),
+                                              ("d_state", 8, H.ERR_UNSUPPORTED),
+                                              ("d_inner", 100, H.ERR_UNSUPPORTED),
+                                              ("n_kv_heads", 3, H.ERR_UNSUPPORTED),
+                                              ("dt_rank", 6, H.ERR_UNSUPPORTED),
+                                              ("window", 0, H.ERR_INVALID_ARG),
+                                              ("kv_role", 7, H.ERR_INVALID_ARG)])
+def test_invalid_configs_are_rejected(field, value, code):
+    d = synth.workloads()["tiny"].dims.replace(**{field: value})
+    with pytest.raises(H.HymbaError) as e:
+        H.workspace_size(d, 1, 16)
+    assert e.value.code == code
+
+
+def test_kv_share_plan_matches_oracle_reading():
+    d = synth.workloads()["stack"].dims
+    is_global = [1 if i in (0, 15, 31) else 0 for i in range(32)]
+    need, cid, role, caches = H.kv_share_alloc(d, is_global, 8, 4224)
+    ocid, orole = orc.kv_share_plan(is_global)
+    assert cid == ocid and role == orole
+    assert len(caches) == 18
+    row = d.n_kv_heads * d.head_dim * 2
+    full = 8 * 4224 * row
+    swa = 2 * (8 * d.n_meta * row + 8 * d.window * row)
+    assert need == 2 * full + 3 * 2 * full + 15 * swa      # view + 3 global + 15 SWA caches
+
+
+def test_kv_share_odd_patterns():
+    d = synth.workloads()["tiny"].dims
+    for pattern in ([0], [1], [0, 0, 0], [0, 1, 0, 0, 1], [1, 1, 1]):
+        need, cid, role, _ = H.kv_share_alloc(d, pattern, 1, 64)
+        ocid, orole = orc.kv_share_plan(pattern)
+        assert (cid, role) == (ocid, orole), pattern
+        assert need > 0
