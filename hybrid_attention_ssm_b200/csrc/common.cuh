@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace hymba {
@@ -233,6 +234,21 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+// n (multiple of 8) floats -> fp16 at a 16-byte aligned destination
+__device__ __forceinline__ void store_f16_row(void* dst, const float* v, int n) {
+  __half* d = reinterpret_cast<__half*>(dst);
+#pragma unroll
+  for (int i = 0; i < 64; i += 8) {
+    if (i < n) {
+      st_global_v4(d + i, pack_f16x2(v[i], v[i + 1]), pack_f16x2(v[i + 2], v[i + 3]),
+                   pack_f16x2(v[i + 4], v[i + 5]), pack_f16x2(v[i + 6], v[i + 7]));
+    }
+  }
+}
 // hardware base-2 exponential (MUFU), relative error ~2^-22, denormals flushed
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;

@@ -1,5 +1,5 @@
 // tcgen05 GEMM for sm_100a: D[m, n] = sum_k A[m, k] * B[n, k] (both operands K-major),
-// bf16 (kind::f16) or fp32 (kind::tf32) inputs, fp32 accumulation in TMEM, TMA-fed.
+// bf16 or fp16 (kind::f16) or fp32 (kind::tf32) inputs, fp32 accumulation in TMEM, TMA-fed.
 //
 // Persistent warp-specialised kernel, 192 threads:
 //   warp 0      TMA producer (one elected lane), STAGES-deep smem ring
@@ -22,14 +22,16 @@ enum EpiMode : int {
   EPI_ATOMIC_F32_T = 5, // transposed fp32 atomic add
   EPI_SWIGLU = 6,       // columns interleaved [gate(32) | up(32)] -> bf16 SiLU(gate)*up
   EPI_SOFTPLUS_T = 7,   // fp32 softplus(acc + bias[col]) stored time-major: out[(b*N + col)*T_out + row]
+  EPI_F32_T = 8,        // transposed fp32 store: out[n][m]
 };
 
 struct Segment {
   int col_begin, col_end;   // columns of D this segment covers (multiples of 64)
-  void* ptr;                // bf16 destination
+  void* ptr;                // destination (bf16 or fp16)
   long long bstride;        // batch stride in elements
   int ld;                   // row stride in elements
   int rope;                 // apply RoPE (head dim 64) to this segment
+  int f16;                  // 1: store fp16, 0: store bf16
 };
 
 struct GemmParams {
@@ -82,14 +84,18 @@ __device__ __forceinline__ void rope_pair_rotate(float* v, int pos, const double
   }
 }
 
-template <int BN, int STAGES, bool TF32>
+// element types of both operands: bf16, fp16 (kind::f16) or fp32 read as tf32 (kind::tf32)
+enum : int { ET_BF16 = 0, ET_F16 = 1, ET_TF32 = 2 };
+
+template <int BN, int STAGES, int ET>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA0, const __grid_constant__ CUtensorMap mapA1,
                    const __grid_constant__ CUtensorMap mapB, const __grid_constant__ GemmParams p) {
   using L = GemmSmem<BN, STAGES>;
   constexpr int ACC_STRIDE = BN <= 128 ? 128 : 256;       // TMEM columns per accumulator
   constexpr uint32_t TMEM_COLS = 2 * ACC_STRIDE;
-  constexpr uint32_t IDESC = make_idesc(GEMM_BM, BN, TF32 ? 2u : 1u, false, false);
+  constexpr bool TF32 = ET == ET_TF32;
+  constexpr uint32_t IDESC = make_idesc(GEMM_BM, BN, ET == ET_TF32 ? 2u : (ET == ET_BF16 ? 1u : 0u), false, false);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -244,14 +250,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const int pos = src0 ? rr : p.row_off1 + rr;
           if (sg.rope) rope_pair_rotate(v, pos, p.rope_theta);
           __nv_bfloat16* base = reinterpret_cast<__nv_bfloat16*>(sg.ptr) + (gc - sg.col_begin);
-          if (src0) {
-            for (int b = 0; b < p.out_batches; ++b)
-              store_bf16_row(base + b * sg.bstride + (size_t)pos * sg.ld, v, 64);
-          } else {
-            store_bf16_row(base + b1 * sg.bstride + (size_t)pos * sg.ld, v, 64);
+          const int b_lo = src0 ? 0 : b1, b_hi = src0 ? p.out_batches : b1 + 1;
+          for (int b = b_lo; b < b_hi; ++b) {
+            __nv_bfloat16* dst = base + b * sg.bstride + (size_t)pos * sg.ld;
+            if (sg.f16) store_f16_row(dst, v, 64);
+            else store_bf16_row(dst, v, 64);
           }
         }
-      } else if (p.mode == EPI_BF16_T || p.mode == EPI_ATOMIC_F32_T) {
+      } else if (p.mode == EPI_BF16_T || p.mode == EPI_ATOMIC_F32_T || p.mode == EPI_F32_T) {
         // accumulator row = output column (weight row), accumulator column = output row
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 32) {
@@ -264,6 +270,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             if (orow < p.n_valid) {
               if (p.mode == EPI_BF16_T)
                 reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)orow * p.ld_out + rr] = __float2bfloat16_rn(v[e]);
+              else if (p.mode == EPI_F32_T)
+                reinterpret_cast<float*>(p.out)[(size_t)orow * p.ld_out + rr] = v[e];
               else
                 atomicAdd(reinterpret_cast<float*>(p.out) + (size_t)orow * p.ld_out + rr, v[e]);
             }

@@ -129,20 +129,20 @@ struct GemmCall {
   int N = 0;
   long long ldb = 0;
   int K = 0;
-  bool tf32 = false;
+  int etype = ET_BF16;
   int bn = 256;
   int split_k = 1;
   GemmParams p{};
 };
 
-template <int BN, int STAGES, bool TF32>
+template <int BN, int STAGES, int ET>
 int launch_gemm_inst(const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& mb, const GemmParams& p,
                      int grid, cudaStream_t st) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   constexpr int smem = GemmSmem<BN, STAGES>::TOTAL;
-  auto kern = gemm_tc_kernel<BN, STAGES, TF32>;
+  auto kern = gemm_tc_kernel<BN, STAGES, ET>;
   if (!attr_set[dev & 63]) {
     HY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
     attr_set[dev & 63] = true;
@@ -153,9 +153,12 @@ int launch_gemm_inst(const CUtensorMap& m0, const CUtensorMap& m1, const CUtenso
 }
 
 int run_gemm(GemmCall& c, const DeviceInfo& dev, cudaStream_t st) {
-  const CUtensorMapDataType dt = c.tf32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  const int esz = c.tf32 ? 4 : 2;
-  const uint32_t kbox = c.tf32 ? 32 : 64;
+  const bool tf32 = c.etype == ET_TF32;
+  const CUtensorMapDataType dt = tf32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                      : (c.etype == ET_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                           : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+  const int esz = tf32 ? 4 : 2;
+  const uint32_t kbox = tf32 ? 32 : 64;
   CUtensorMap m0, m1, mb;
   {
     const uint64_t dims[3] = {(uint64_t)c.K, (uint64_t)c.rows1, (uint64_t)c.nb1};
@@ -192,14 +195,18 @@ int run_gemm(GemmCall& c, const DeviceInfo& dev, cudaStream_t st) {
   p.total_tiles = p.m_tiles * p.n_tiles_n * p.split_k;
   if (p.total_tiles <= 0) return HYMBA_OK;
   const int grid = p.total_tiles < dev.sms ? p.total_tiles : dev.sms;
-  if (c.tf32) {
-    if (c.bn == 256) return launch_gemm_inst<256, 4, true>(m0, m1, mb, p, grid, st);
-    if (c.bn == 128) return launch_gemm_inst<128, 6, true>(m0, m1, mb, p, grid, st);
+  if (tf32) {
+    if (c.bn == 256) return launch_gemm_inst<256, 4, ET_TF32>(m0, m1, mb, p, grid, st);
+    if (c.bn == 128) return launch_gemm_inst<128, 6, ET_TF32>(m0, m1, mb, p, grid, st);
+  } else if (c.etype == ET_F16) {
+    if (c.bn == 256) return launch_gemm_inst<256, 4, ET_F16>(m0, m1, mb, p, grid, st);
+    if (c.bn == 128) return launch_gemm_inst<128, 6, ET_F16>(m0, m1, mb, p, grid, st);
+    if (c.bn == 64) return launch_gemm_inst<64, 8, ET_F16>(m0, m1, mb, p, grid, st);
   } else {
-    if (c.bn == 256) return launch_gemm_inst<256, 4, false>(m0, m1, mb, p, grid, st);
-    if (c.bn == 160) return launch_gemm_inst<160, 5, false>(m0, m1, mb, p, grid, st);
-    if (c.bn == 128) return launch_gemm_inst<128, 6, false>(m0, m1, mb, p, grid, st);
-    if (c.bn == 64) return launch_gemm_inst<64, 8, false>(m0, m1, mb, p, grid, st);
+    if (c.bn == 256) return launch_gemm_inst<256, 4, ET_BF16>(m0, m1, mb, p, grid, st);
+    if (c.bn == 160) return launch_gemm_inst<160, 5, ET_BF16>(m0, m1, mb, p, grid, st);
+    if (c.bn == 128) return launch_gemm_inst<128, 6, ET_BF16>(m0, m1, mb, p, grid, st);
+    if (c.bn == 64) return launch_gemm_inst<64, 8, ET_BF16>(m0, m1, mb, p, grid, st);
   }
   return fail(HYMBA_ERR_UNSUPPORTED, "no GEMM tile width %d", c.bn);
 }
@@ -280,7 +287,7 @@ PrefillWs prefill_layout(const Dims& m, int B, int n_tokens, int x_has_meta) {
   w.xbc = take(rows * m.ld_xbc * 4);
   w.dT = take((size_t)B * m.Di * w.Tp * 4);
   w.y = take(rows * m.Di * 2);
-  w.o = take(rows * m.qw * 2);
+  w.o = take(rows * m.qw * 4);
   w.u = take(rows * m.uw * 2);
   w.sstate = take((size_t)B * m.Di * 16 * 4);
   w.cstate = take((size_t)B * m.Di * 3 * 4);
@@ -297,12 +304,12 @@ DecodeWs decode_layout(const Dims& m, int B, int n_keys_max) {
   w.n_splits = cdiv(n_keys_max, DEC_KT);
   size_t off = 256;
   auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
-  w.proj = take((size_t)B * m.P * 2);
+  w.proj = take((size_t)B * m.P * 4);
   w.part = take((size_t)B * m.Hq * w.n_splits * 66 * 4);
-  w.o = take((size_t)B * m.qw * 2);
+  w.o = take((size_t)B * m.qw * 4);
   w.xc = take((size_t)B * m.Di * 2);
   w.xbc = take((size_t)B * m.ld_xbc * 4);
-  w.y = take((size_t)B * m.Di * 2);
+  w.y = take((size_t)B * m.Di * 4);
   w.u = take((size_t)B * m.uw * 2);
   w.acc = take((size_t)B * m.d * 4);
   w.total = off;
@@ -439,10 +446,10 @@ int hymba_kv_share_alloc(const hymba_layer_cfg* base, int n_layers, const uint8_
   if (buf_bytes < need) return fail(HYMBA_ERR_WORKSPACE, "cache buffer %zu < %zu bytes", buf_bytes, need);
   if (reinterpret_cast<uintptr_t>(dev_buf) & 255u) return fail(HYMBA_ERR_INVALID_ARG, "cache buffer not 256-byte aligned");
   uint8_t* p = static_cast<uint8_t*>(dev_buf);
-  hymba_bf16 *view_k = nullptr, *view_v = nullptr;
+  hymba_f16 *view_k = nullptr, *view_v = nullptr;
   if (any_swa) {
-    view_k = reinterpret_cast<hymba_bf16*>(p); p += full;
-    view_v = reinterpret_cast<hymba_bf16*>(p); p += full;
+    view_k = reinterpret_cast<hymba_f16*>(p); p += full;
+    view_v = reinterpret_cast<hymba_f16*>(p); p += full;
   }
   for (int l = 0; l < n_layers; ++l) {
     const bool first = (l == 0) || layer_cache_id[l] != layer_cache_id[l - 1];
@@ -457,14 +464,14 @@ int hymba_kv_share_alloc(const hymba_layer_cfg* base, int n_layers, const uint8_
     c.max_tokens = max_tokens;
     if (is_global[l]) {
       c.kind = HYMBA_CACHE_GLOBAL;
-      c.k = reinterpret_cast<hymba_bf16*>(p); p += full;
-      c.v = reinterpret_cast<hymba_bf16*>(p); p += full;
+      c.k = reinterpret_cast<hymba_f16*>(p); p += full;
+      c.v = reinterpret_cast<hymba_f16*>(p); p += full;
     } else {
       c.kind = HYMBA_CACHE_SWA;
-      c.meta_k = reinterpret_cast<hymba_bf16*>(p); p += meta;
-      c.meta_v = reinterpret_cast<hymba_bf16*>(p); p += meta;
-      c.ring_k = reinterpret_cast<hymba_bf16*>(p); p += ring;
-      c.ring_v = reinterpret_cast<hymba_bf16*>(p); p += ring;
+      c.meta_k = reinterpret_cast<hymba_f16*>(p); p += meta;
+      c.meta_v = reinterpret_cast<hymba_f16*>(p); p += meta;
+      c.ring_k = reinterpret_cast<hymba_f16*>(p); p += ring;
+      c.ring_v = reinterpret_cast<hymba_f16*>(p); p += ring;
       c.k = view_k;
       c.v = view_v;
     }
@@ -501,6 +508,7 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
   DevStatus* status = reinterpret_cast<DevStatus*>(ws);
   auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(wsb + off); };
   auto f32 = [&](size_t off) { return reinterpret_cast<float*>(wsb + off); };
+  auto h16 = [&](size_t off) { return reinterpret_cast<__half*>(wsb + off); };
   const size_t rows = (size_t)B * T;
   const int Lmax = kv->max_tokens;
 
@@ -522,12 +530,12 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     c.p.T_out = T;
     c.p.status = status;
     int ns = 0;
-    c.p.seg[ns++] = Segment{0, m.qw, bf(L.q), (long long)T * m.qw, m.qw, 1};
+    c.p.seg[ns++] = Segment{0, m.qw, bf(L.q), (long long)T * m.qw, m.qw, 1, 1};
     if (own_kv) {
-      c.p.seg[ns++] = Segment{m.qw, m.qw + m.kvw, kv->k, (long long)Lmax * m.kvw, m.kvw, 1};
-      c.p.seg[ns++] = Segment{m.qw + m.kvw, m.qw + 2 * m.kvw, kv->v, (long long)Lmax * m.kvw, m.kvw, 0};
+      c.p.seg[ns++] = Segment{m.qw, m.qw + m.kvw, kv->k, (long long)Lmax * m.kvw, m.kvw, 1, 1};
+      c.p.seg[ns++] = Segment{m.qw + m.kvw, m.qw + 2 * m.kvw, kv->v, (long long)Lmax * m.kvw, m.kvw, 0, 1};
     }
-    c.p.seg[ns++] = Segment{m.xz_off, m.xz_off + 2 * m.Di, bf(L.xz), (long long)T * 2 * m.Di, 2 * m.Di, 0};
+    c.p.seg[ns++] = Segment{m.xz_off, m.xz_off + 2 * m.Di, bf(L.xz), (long long)T * 2 * m.Di, 2 * m.Di, 0, 0};
     c.p.nseg = ns;
     fill_rope_theta(c.p.rope_theta, cfg->rope_base);
     HY_TRY(run_gemm(c, *dev, st));
@@ -561,7 +569,7 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
   // 4. dt_proj (tf32) with softplus(+bias), stored time-major
   {
     GemmCall c;
-    c.tf32 = true;
+    c.etype = ET_TF32;
     c.a1 = f32(L.xbc); c.nb1 = B; c.rows1 = T; c.lda1 = m.ld_xbc; c.a1_bstride = (long long)T * m.ld_xbc;
     c.b = w->w_dt; c.N = m.Di; c.ldb = w->w_dt_ld; c.K = m.R;
     c.bn = pick_bn_wide(B * cdiv(T, GEMM_BM), m.Di, dev->sms);
@@ -580,19 +588,19 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     {
       const uint64_t dims[3] = {(uint64_t)m.qw, (uint64_t)T, (uint64_t)B};
       const uint64_t str[2] = {(uint64_t)m.qw * 2, (uint64_t)T * m.qw * 2};
-      HY_TRY(make_map(&mq, bf(L.q), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dims, str, box));
+      HY_TRY(make_map(&mq, bf(L.q), CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, dims, str, box));
     }
     {
       const uint64_t dims[3] = {(uint64_t)m.kvw, (uint64_t)T, (uint64_t)B};
       const uint64_t str[2] = {(uint64_t)m.kvw * 2, (uint64_t)Lmax * m.kvw * 2};
-      HY_TRY(make_map(&mk, kv->k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dims, str, box));
-      HY_TRY(make_map(&mv, kv->v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dims, str, box));
+      HY_TRY(make_map(&mk, kv->k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, dims, str, box));
+      HY_TRY(make_map(&mv, kv->v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, dims, str, box));
     }
     AttnParams ap;
     ap.T = T; ap.Hq = m.Hq; ap.Hkv = m.Hkv; ap.n_meta = m.M; ap.window = m.W; ap.is_global = cfg->is_global;
     ap.q_tiles = cdiv(T, 128);
     ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)m.D));
-    ap.out = bf(L.o);
+    ap.out = f32(L.o);
     ap.ld_out = m.qw;
     ap.status = status;
     static bool attr[64] = {false};
@@ -616,16 +624,17 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
   }
   // 7. per-branch RMSNorm, gate, beta, average
   {
-    branch_norm_avg_kernel<<<(unsigned)rows, 256, 0, st>>>(bf(L.o), m.qw, m.qw, bf(L.y), m.Di, bf(L.xz) + m.Di,
-                                                           2 * m.Di, m.Di, w->g_attn, w->g_ssm, cfg->norm_eps,
-                                                           bf(L.u), m.uw);
+    branch_norm_avg_kernel<__nv_bfloat16><<<(unsigned)rows, 256, 0, st>>>(
+        f32(L.o), m.qw, m.qw, bf(L.y), m.Di, bf(L.xz) + m.Di, 2 * m.Di, m.Di, w->g_attn, w->g_ssm, cfg->norm_eps,
+        h16(L.u), m.uw);
     HY_CUDA(cudaGetLastError());
   }
   // 8. out_proj (+ residual)
   {
     GemmCall c;
-    c.a1 = bf(L.u); c.nb1 = 1; c.rows1 = (int)rows; c.lda1 = m.uw; c.a1_bstride = (long long)rows * m.uw;
+    c.a1 = h16(L.u); c.nb1 = 1; c.rows1 = (int)rows; c.lda1 = m.uw; c.a1_bstride = (long long)rows * m.uw;
     c.b = w->w_out; c.N = m.d; c.ldb = m.uw; c.K = m.uw;
+    c.etype = ET_F16;
     c.bn = pick_bn_wide(cdiv(rows, GEMM_BM), m.d, dev->sms);
     c.p.mode = EPI_BF16;
     c.p.out = out;
@@ -643,9 +652,9 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     const int n = n_rows * (m.kvw / 8);
     dim3 grid(cdiv(n, 256), B);
     swa_cache_finalize_kernel<<<grid, 256, 0, st>>>(
-        reinterpret_cast<const __nv_bfloat16*>(kv->k), reinterpret_cast<const __nv_bfloat16*>(kv->v), Lmax, T, m.M,
-        m.W, m.kvw, reinterpret_cast<__nv_bfloat16*>(kv->meta_k), reinterpret_cast<__nv_bfloat16*>(kv->meta_v),
-        reinterpret_cast<__nv_bfloat16*>(kv->ring_k), reinterpret_cast<__nv_bfloat16*>(kv->ring_v));
+        reinterpret_cast<const __half*>(kv->k), reinterpret_cast<const __half*>(kv->v), Lmax, T, m.M, m.W, m.kvw,
+        reinterpret_cast<__half*>(kv->meta_k), reinterpret_cast<__half*>(kv->meta_v),
+        reinterpret_cast<__half*>(kv->ring_k), reinterpret_cast<__half*>(kv->ring_v));
     HY_CUDA(cudaGetLastError());
   }
   return HYMBA_OK;
@@ -685,6 +694,7 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
   DevStatus* status = reinterpret_cast<DevStatus*>(ws);
   auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(wsb + off); };
   auto f32 = [&](size_t off) { return reinterpret_cast<float*>(wsb + off); };
+  auto h16 = [&](size_t off) { return reinterpret_cast<__half*>(wsb + off); };
   const bool own_kv = cfg->kv_role != HYMBA_KV_CONSUMER;
 
   // 1. in_proj, weights as the M operand (swap-AB), transposed store -> proj [B, P]
@@ -693,8 +703,8 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     c.a1 = w->w_in; c.nb1 = 1; c.rows1 = m.P; c.lda1 = m.d; c.a1_bstride = (long long)m.P * m.d;
     c.b = x; c.N = B; c.ldb = m.d; c.K = m.d;
     c.bn = pick_bn_cover(B);
-    c.p.mode = EPI_BF16_T;
-    c.p.out = bf(L.proj);
+    c.p.mode = EPI_F32_T;
+    c.p.out = f32(L.proj);
     c.p.ld_out = m.P;
     c.p.m_valid = m.P;
     c.p.n_valid = B;
@@ -704,7 +714,7 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
   // 2. attention over meta + window (or the whole causal prefix), split-K, then combine
   {
     DecAttnParams ap;
-    ap.proj = bf(L.proj);
+    ap.proj = f32(L.proj);
     ap.ld_proj = m.P;
     ap.Hq = m.Hq; ap.Hkv = m.Hkv; ap.M = m.M; ap.W = m.W; ap.is_global = global ? 1 : 0;
     ap.write_kv = own_kv ? 1 : 0;
@@ -716,12 +726,12 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
       ap.n_keys = m.M + (position - win0 + 1);
     }
     ap.n_splits = cdiv(ap.n_keys, DEC_KT);
-    ap.meta_k = reinterpret_cast<__nv_bfloat16*>(kv->meta_k);
-    ap.meta_v = reinterpret_cast<__nv_bfloat16*>(kv->meta_v);
-    ap.ring_k = reinterpret_cast<__nv_bfloat16*>(kv->ring_k);
-    ap.ring_v = reinterpret_cast<__nv_bfloat16*>(kv->ring_v);
-    ap.full_k = reinterpret_cast<__nv_bfloat16*>(kv->k);
-    ap.full_v = reinterpret_cast<__nv_bfloat16*>(kv->v);
+    ap.meta_k = reinterpret_cast<__half*>(kv->meta_k);
+    ap.meta_v = reinterpret_cast<__half*>(kv->meta_v);
+    ap.ring_k = reinterpret_cast<__half*>(kv->ring_k);
+    ap.ring_v = reinterpret_cast<__half*>(kv->ring_v);
+    ap.full_k = reinterpret_cast<__half*>(kv->k);
+    ap.full_v = reinterpret_cast<__half*>(kv->v);
     ap.Lmax = kv->max_tokens;
     ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)m.D));
     fill_rope_theta(ap.rope_theta, cfg->rope_base);
@@ -730,13 +740,13 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     dim3 grid(ap.n_splits, m.Hkv, B);
     decode_attn_kernel<<<grid, 128, 0, st>>>(ap);
     HY_CUDA(cudaGetLastError());
-    decode_attn_combine_kernel<<<dim3(m.Hq, B), 64, 0, st>>>(f32(L.part), ap.n_splits, m.Hq, bf(L.o), m.qw);
+    decode_attn_combine_kernel<<<dim3(m.Hq, B), 64, 0, st>>>(f32(L.part), ap.n_splits, m.Hq, f32(L.o), m.qw);
     HY_CUDA(cudaGetLastError());
   }
   // 3. conv step
   {
     const int n = B * m.Di;
-    decode_conv_kernel<<<cdiv(n, 256), 256, 0, st>>>(bf(L.proj), m.P, m.xz_off, m.Di, w->conv_w, w->conv_b,
+    decode_conv_kernel<<<cdiv(n, 256), 256, 0, st>>>(f32(L.proj), m.P, m.xz_off, m.Di, w->conv_w, w->conv_b,
                                                       conv_state, bf(L.xc), B);
     HY_CUDA(cudaGetLastError());
   }
@@ -761,13 +771,13 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
   {
     dim3 grid(m.Di / 16, B);
     decode_ssm_kernel<<<grid, 256, 0, st>>>(f32(L.xbc), m.ld_xbc, m.R, w->w_dt, w->w_dt_ld, w->dt_bias, w->A,
-                                            bf(L.xc), bf(L.proj), m.P, m.xz_off + m.Di, ssm_state, bf(L.y), m.Di);
+                                            bf(L.xc), f32(L.proj), m.P, m.xz_off + m.Di, ssm_state, f32(L.y), m.Di);
     HY_CUDA(cudaGetLastError());
   }
   // 6. norm + average (y already gated)
   {
-    branch_norm_avg_kernel<<<B, 256, 0, st>>>(bf(L.o), m.qw, m.qw, bf(L.y), m.Di, nullptr, 0, m.Di, w->g_attn,
-                                              w->g_ssm, cfg->norm_eps, bf(L.u), m.uw);
+    branch_norm_avg_kernel<float><<<B, 256, 0, st>>>(f32(L.o), m.qw, m.qw, f32(L.y), m.Di, nullptr, 0, m.Di,
+                                                     w->g_attn, w->g_ssm, cfg->norm_eps, h16(L.u), m.uw);
     HY_CUDA(cudaGetLastError());
   }
   // 7. out_proj (swap-AB, split-K) and the bf16 (+ residual) store
@@ -775,7 +785,8 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     HY_CUDA(cudaMemsetAsync(f32(L.acc), 0, (size_t)B * m.d * 4, st));
     GemmCall c;
     c.a1 = w->w_out; c.nb1 = 1; c.rows1 = m.d; c.lda1 = m.uw; c.a1_bstride = (long long)m.d * m.uw;
-    c.b = bf(L.u); c.N = B; c.ldb = m.uw; c.K = m.uw;
+    c.b = h16(L.u); c.N = B; c.ldb = m.uw; c.K = m.uw;
+    c.etype = ET_F16;
     c.bn = pick_bn_cover(B);
     const int tiles = cdiv(m.d, GEMM_BM) * cdiv(B, c.bn);
     c.split_k = cdiv(dev->sms, tiles);

@@ -29,34 +29,47 @@ __device__ __forceinline__ void unpack8(const uint4& r, float* f) {
 #pragma unroll
   for (int e = 0; e < 8; ++e) f[e] = __bfloat162float(h[e]);
 }
+__device__ __forceinline__ void unpack8h(const uint4& r, float* f) {
+  const __half* h = reinterpret_cast<const __half*>(&r);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) f[e] = __half2float(h[e]);
+}
 
 // ----------------------------------------------------------------------------------------
 // u = 1/2 [ g_attn * rms(O) ; g_ssm * rms(y * SiLU(z)) ], one row per CTA (256 threads);
-// z == nullptr means y is already gated.
-// O [rows, ld_o] (attn_w columns), y [rows, ld_y], z [rows, ld_z] (di columns) -> u [rows,
-// ld_u].  Widths are multiples of 8.
+// z == nullptr means y is already gated.  O fp32 [rows, ld_o] (attn_w columns); y [rows,
+// ld_y] bf16 or fp32; z bf16 [rows, ld_z] (di columns) -> u fp16 [rows, ld_u].  fp16 holds
+// the normalised values with 8x finer rounding than bf16 and cannot overflow: after the
+// RMSNorm |value| <= sqrt(width) * |gain| / 2.  Widths are multiples of 8.
 // ----------------------------------------------------------------------------------------
+__device__ __forceinline__ void load8(const float* p, float* f) {
+  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float* f) {
+  unpack8(*reinterpret_cast<const uint4*>(p), f);
+}
+template <typename YT>
 __global__ void __launch_bounds__(256)
-    branch_norm_avg_kernel(const __nv_bfloat16* __restrict__ O, int ld_o, int attn_w,
-                           const __nv_bfloat16* __restrict__ y, int ld_y, const __nv_bfloat16* __restrict__ z,
-                           int ld_z, int di, const float* __restrict__ g_attn, const float* __restrict__ g_ssm,
-                           float eps, __nv_bfloat16* __restrict__ u, int ld_u) {
+    branch_norm_avg_kernel(const float* __restrict__ O, int ld_o, int attn_w, const YT* __restrict__ y, int ld_y,
+                           const __nv_bfloat16* __restrict__ z, int ld_z, int di, const float* __restrict__ g_attn,
+                           const float* __restrict__ g_ssm, float eps, __half* __restrict__ u, int ld_u) {
   __shared__ float red[32];
   const size_t row = blockIdx.x;
-  const __nv_bfloat16* o_r = O + row * ld_o;
-  const __nv_bfloat16* y_r = y + row * ld_y;
+  const float* o_r = O + row * ld_o;
+  const YT* y_r = y + row * ld_y;
   const __nv_bfloat16* z_r = z != nullptr ? z + row * ld_z : nullptr;
-  __nv_bfloat16* u_r = u + row * ld_u;
+  __half* u_r = u + row * ld_u;
   float sa = 0.f, ss = 0.f;
   for (int c = threadIdx.x * 8; c < attn_w; c += 256 * 8) {
     float f[8];
-    unpack8(*reinterpret_cast<const uint4*>(o_r + c), f);
+    load8(o_r + c, f);
 #pragma unroll
     for (int e = 0; e < 8; ++e) sa += f[e] * f[e];
   }
   for (int c = threadIdx.x * 8; c < di; c += 256 * 8) {
     float fy[8], fz[8];
-    unpack8(*reinterpret_cast<const uint4*>(y_r + c), fy);
+    load8(y_r + c, fy);
     if (z != nullptr) {
       unpack8(*reinterpret_cast<const uint4*>(z_r + c), fz);
 #pragma unroll
@@ -71,16 +84,16 @@ __global__ void __launch_bounds__(256)
   const float rs = 0.5f / sqrtf(ss / (float)di + eps);
   for (int c = threadIdx.x * 8; c < attn_w; c += 256 * 8) {
     float f[8];
-    unpack8(*reinterpret_cast<const uint4*>(o_r + c), f);
+    load8(o_r + c, f);
     uint32_t pk[4];
 #pragma unroll
     for (int e = 0; e < 8; e += 2)
-      pk[e / 2] = pack_bf16x2(f[e] * ra * g_attn[c + e], f[e + 1] * ra * g_attn[c + e + 1]);
+      pk[e / 2] = pack_f16x2(f[e] * ra * g_attn[c + e], f[e + 1] * ra * g_attn[c + e + 1]);
     *reinterpret_cast<uint4*>(u_r + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
   }
   for (int c = threadIdx.x * 8; c < di; c += 256 * 8) {
     float fy[8], fz[8];
-    unpack8(*reinterpret_cast<const uint4*>(y_r + c), fy);
+    load8(y_r + c, fy);
     if (z != nullptr) {
       unpack8(*reinterpret_cast<const uint4*>(z_r + c), fz);
 #pragma unroll
@@ -88,7 +101,7 @@ __global__ void __launch_bounds__(256)
     }
     uint32_t pk[4];
 #pragma unroll
-    for (int e = 0; e < 8; e += 2) pk[e / 2] = pack_bf16x2(fy[e] * rs * g_ssm[c + e], fy[e + 1] * rs * g_ssm[c + e + 1]);
+    for (int e = 0; e < 8; e += 2) pk[e / 2] = pack_f16x2(fy[e] * rs * g_ssm[c + e], fy[e + 1] * rs * g_ssm[c + e + 1]);
     *reinterpret_cast<uint4*>(u_r + attn_w + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
   }
 }
@@ -97,10 +110,10 @@ __global__ void __launch_bounds__(256)
 // SWA cache after prefill: meta rows [0, M) -> meta_k/v; rows [max(M, T-W), T) -> ring slot
 // (pos - M) mod W.  view_k/v [B, Lmax, Hkv*D]; meta [B, M, Hkv*D]; ring [B, W, Hkv*D].
 // ----------------------------------------------------------------------------------------
-__global__ void swa_cache_finalize_kernel(const __nv_bfloat16* __restrict__ vk, const __nv_bfloat16* __restrict__ vv,
+__global__ void swa_cache_finalize_kernel(const __half* __restrict__ vk, const __half* __restrict__ vv,
                                           int Lmax, int T, int M, int W, int row_elems,
-                                          __nv_bfloat16* __restrict__ meta_k, __nv_bfloat16* __restrict__ meta_v,
-                                          __nv_bfloat16* __restrict__ ring_k, __nv_bfloat16* __restrict__ ring_v) {
+                                          __half* __restrict__ meta_k, __half* __restrict__ meta_v,
+                                          __half* __restrict__ ring_k, __half* __restrict__ ring_v) {
   const int b = blockIdx.y;
   const int first_win = max(M, T - W);
   const int n_rows = M + (T - first_win);
@@ -108,7 +121,7 @@ __global__ void swa_cache_finalize_kernel(const __nv_bfloat16* __restrict__ vk, 
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_rows * vec_per_row; i += gridDim.x * blockDim.x) {
     const int rr = i / vec_per_row, cv = (i % vec_per_row) * 8;
     int pos;
-    __nv_bfloat16 *dk, *dv;
+    __half *dk, *dv;
     if (rr < M) {
       pos = rr;
       dk = meta_k + ((size_t)b * M + pos) * row_elems;
@@ -137,11 +150,11 @@ __global__ void swa_cache_finalize_kernel(const __nv_bfloat16* __restrict__ vk, 
 // Partial results per (b, h, split): m (log2 domain), l, o[64] unnormalised.
 // ----------------------------------------------------------------------------------------
 struct DecAttnParams {
-  const __nv_bfloat16* proj;  // [B, ld_proj]: q at 0, k at q_w, v at q_w + kv_w (when present)
+  const float* proj;          // [B, ld_proj] fp32: q at 0, k at q_w, v at q_w + kv_w (when present)
   int ld_proj;
   int Hq, Hkv, M, W, is_global, write_kv, p, n_keys, n_splits;
-  __nv_bfloat16 *meta_k, *meta_v, *ring_k, *ring_v;  // SWA cache
-  __nv_bfloat16 *full_k, *full_v;                    // global cache [B, Lmax, Hkv*D]
+  __half *meta_k, *meta_v, *ring_k, *ring_v;  // SWA cache (fp16)
+  __half *full_k, *full_v;                    // global cache [B, Lmax, Hkv*D] (fp16)
   int Lmax;
   float scale_log2;
   double rope_theta[32];
@@ -164,13 +177,13 @@ __device__ __forceinline__ void rope64_smem(float* v, int pos, const double* the
 }
 
 __global__ void __launch_bounds__(128) decode_attn_kernel(const __grid_constant__ DecAttnParams p) {
-  __shared__ __align__(16) __nv_bfloat16 ks[DEC_KT][72];   // padded rows (144 B)
-  __shared__ __align__(16) __nv_bfloat16 vs[DEC_KT][64];
-  __shared__ float qs[DEC_MAXG][64];
-  __shared__ float knew[64], vnew[64];
-  __shared__ float ps[DEC_MAXG][DEC_KT];
+  __shared__ __align__(16) __half ks[DEC_KT][72];   // padded rows (144 B)
+  __shared__ __align__(16) __half vs[DEC_KT][64];
+  __shared__ __align__(16) float qs[DEC_MAXG][64];
+  __shared__ __align__(16) float knew[64], vnew[64];
+  __shared__ __align__(16) float ps[DEC_MAXG][DEC_KT];
   __shared__ float red[DEC_MAXG][4];
-  __shared__ float opart[4][DEC_MAXG][64];
+  __shared__ __align__(16) float opart[4][DEC_MAXG][64];
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = p.Hq / p.Hkv;
@@ -181,18 +194,18 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const __grid_constant_
   const int win0 = p.is_global ? 0 : max(p.M, p.p - p.W + 1);
 
   // key index -> (cache row pointer) ; position p is the last key
-  auto key_row = [&](int kidx, bool is_v) -> const __nv_bfloat16* {
+  auto key_row = [&](int kidx, bool is_v) -> const __half* {
     if (p.is_global) {
-      const __nv_bfloat16* base = is_v ? p.full_v : p.full_k;
+      const __half* base = is_v ? p.full_v : p.full_k;
       return base + ((size_t)b * p.Lmax + kidx) * kvw + g * 64;
     }
     if (kidx < n_meta_keys) {
-      const __nv_bfloat16* base = is_v ? p.meta_v : p.meta_k;
+      const __half* base = is_v ? p.meta_v : p.meta_k;
       return base + ((size_t)b * p.M + kidx) * kvw + g * 64;
     }
     const int pos = win0 + (kidx - n_meta_keys);
     const int slot = (pos - p.M) % p.W;
-    const __nv_bfloat16* base = is_v ? p.ring_v : p.ring_k;
+    const __half* base = is_v ? p.ring_v : p.ring_k;
     return base + ((size_t)b * p.W + slot) * kvw + g * 64;
   };
   const bool last_is_new = p.write_kv != 0;   // position p comes from registers
@@ -208,21 +221,21 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const __grid_constant_
   cp_async_commit();
 
   // queries of this group with RoPE at position p, pre-scaled
-  const __nv_bfloat16* pr = p.proj + (size_t)b * p.ld_proj;
+  const float* pr = p.proj + (size_t)b * p.ld_proj;
   for (int i = tid; i < G * 64; i += 128) {
     const int hh = i >> 6, d = i & 63;
-    qs[hh][d] = __bfloat162float(pr[(g * G + hh) * 64 + d]);
+    qs[hh][d] = pr[(g * G + hh) * 64 + d];
   }
   if (last_is_new && tid < 64) {
-    knew[tid] = __bfloat162float(pr[p.Hq * 64 + g * 64 + tid]);
-    vnew[tid] = __bfloat162float(pr[p.Hq * 64 + kvw + g * 64 + tid]);
+    knew[tid] = pr[p.Hq * 64 + g * 64 + tid];
+    vnew[tid] = pr[p.Hq * 64 + kvw + g * 64 + tid];
   }
   __syncthreads();
   for (int i = warp; i < G + (last_is_new ? 1 : 0); i += 4) rope64_smem(i < G ? qs[i] : knew, p.p, p.rope_theta);
   __syncthreads();
   for (int i = tid; i < G * 64; i += 128) qs[i >> 6][i & 63] *= p.scale_log2;
   if (last_is_new && split == 0 && tid < 64) {
-    __nv_bfloat16 *dk, *dv;
+    __half *dk, *dv;
     if (p.is_global) {
       dk = p.full_k + ((size_t)b * p.Lmax + p.p) * kvw + g * 64;
       dv = p.full_v + ((size_t)b * p.Lmax + p.p) * kvw + g * 64;
@@ -231,16 +244,16 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const __grid_constant_
       dk = p.ring_k + ((size_t)b * p.W + slot) * kvw + g * 64;
       dv = p.ring_v + ((size_t)b * p.W + slot) * kvw + g * 64;
     }
-    dk[tid] = __float2bfloat16_rn(knew[tid]);
-    dv[tid] = __float2bfloat16_rn(vnew[tid]);
+    dk[tid] = __float2half_rn(knew[tid]);
+    dv[tid] = __float2half_rn(vnew[tid]);
   }
   cp_async_wait<0>();
   __syncthreads();
-  // the new token's row (rounded to bf16 like the cached copy)
+  // the new token's row (rounded to fp16 like the cached copy)
   if (last_is_new && p.n_keys - 1 >= k_first && p.n_keys - 1 < k_first + nk && tid < 64) {
     const int kk = p.n_keys - 1 - k_first;
-    ks[kk][tid] = __float2bfloat16_rn(knew[tid]);
-    vs[kk][tid] = __float2bfloat16_rn(vnew[tid]);
+    ks[kk][tid] = __float2half_rn(knew[tid]);
+    vs[kk][tid] = __float2half_rn(vnew[tid]);
   }
   __syncthreads();
 
@@ -251,7 +264,7 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const __grid_constant_
     float kf[64];
     if (kk < nk) {
 #pragma unroll
-      for (int d = 0; d < 64; d += 8) unpack8(*reinterpret_cast<const uint4*>(&ks[kk][d]), kf + d);
+      for (int d = 0; d < 64; d += 8) unpack8h(*reinterpret_cast<const uint4*>(&ks[kk][d]), kf + d);
     }
 #pragma unroll
     for (int hh = 0; hh < DEC_MAXG; ++hh) {
@@ -290,7 +303,7 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const __grid_constant_
 #pragma unroll
     for (int hh = 0; hh < DEC_MAXG; ++hh) acc[hh][0] = acc[hh][1] = 0.f;
     for (int kk = kq * 32; kk < kq * 32 + 32; ++kk) {
-      const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162*>(&vs[kk][dp * 2]);
+      const __half2 v2 = *reinterpret_cast<const __half2*>(&vs[kk][dp * 2]);
       const float v0 = __low2float(v2), v1 = __high2float(v2);
 #pragma unroll
       for (int hh = 0; hh < DEC_MAXG; ++hh) {
@@ -334,7 +347,7 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const __grid_constant_
 
 // merge the split partials of one (b, h): O = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i
 __global__ void decode_attn_combine_kernel(const float* __restrict__ part, int n_splits, int Hq,
-                                           __nv_bfloat16* __restrict__ out, int ld_out) {
+                                           float* __restrict__ out, int ld_out) {
   const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;   // 64 threads
   const float* pp = part + ((size_t)b * Hq + h) * n_splits * 66;
   float M = -1e30f;
@@ -345,14 +358,14 @@ __global__ void decode_attn_combine_kernel(const float* __restrict__ part, int n
     L += w * pp[i * 66 + 1];
     O += w * pp[i * 66 + 2 + d];
   }
-  out[(size_t)b * ld_out + h * 64 + d] = __float2bfloat16_rn(O / L);
+  out[(size_t)b * ld_out + h * 64 + d] = O / L;
 }
 
 // ----------------------------------------------------------------------------------------
 // decode conv step: window [state(3), x_new] -> xc = SiLU(b + w . window); state shifts.
-// x from proj [B, ld_proj] at column off_x; xc [B, Di] bf16; state [B, Di, 3] fp32 in place.
+// x from proj [B, ld_proj] fp32 at column off_x; xc [B, Di] bf16; state [B, Di, 3] fp32 in place.
 // ----------------------------------------------------------------------------------------
-__global__ void decode_conv_kernel(const __nv_bfloat16* __restrict__ proj, int ld_proj, int off_x, int Di,
+__global__ void decode_conv_kernel(const float* __restrict__ proj, int ld_proj, int off_x, int Di,
                                    const float* __restrict__ w, const float* __restrict__ bias,
                                    float* __restrict__ state, __nv_bfloat16* __restrict__ xc, int B) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -360,7 +373,7 @@ __global__ void decode_conv_kernel(const __nv_bfloat16* __restrict__ proj, int l
   const int b = i / Di, c = i % Di;
   float* st = state + (size_t)i * 3;
   const float x0 = st[0], x1 = st[1], x2 = st[2];
-  const float xn = __bfloat162float(proj[(size_t)b * ld_proj + off_x + c]);
+  const float xn = proj[(size_t)b * ld_proj + off_x + c];
   const float4 wv = *reinterpret_cast<const float4*>(w + (size_t)c * 4);
   const float acc = bias[c] + wv.x * x0 + wv.y * x1 + wv.z * x2 + wv.w * xn;
   xc[i] = __float2bfloat16_rn(silu_f(acc));
@@ -373,13 +386,13 @@ __global__ void decode_conv_kernel(const __nv_bfloat16* __restrict__ proj, int l
 // decode SSM step: dt = softplus(dt_low . W_dt[c] + bias), h = exp(dt A) h + dt B x,
 // y = (C . h) * SiLU(z).  CTA = 16 channels x 16 states of one sequence.
 //   xbc [B, ld_xbc] fp32: dt_low at 0..R-1, B at R.., C at R+16..; W_dt [Di, ld_dt] fp32;
-//   xc [B, Di] bf16; z from proj at column off_z; state [B, Di, 16] in place; y [B, Di] bf16.
+//   xc [B, Di] bf16; z from proj at column off_z; state [B, Di, 16] in place; y [B, Di] fp32.
 // ----------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
     decode_ssm_kernel(const float* __restrict__ xbc, int ld_xbc, int R, const float* __restrict__ w_dt, int ld_dt,
                       const float* __restrict__ dt_bias, const float* __restrict__ A,
-                      const __nv_bfloat16* __restrict__ xc, const __nv_bfloat16* __restrict__ proj, int ld_proj,
-                      int off_z, float* __restrict__ state, __nv_bfloat16* __restrict__ y, int Di) {
+                      const __nv_bfloat16* __restrict__ xc, const float* __restrict__ proj, int ld_proj,
+                      int off_z, float* __restrict__ state, float* __restrict__ y, int Di) {
   __shared__ float dl[256];
   __shared__ float bcs[32];
   const int b = blockIdx.y;
@@ -405,8 +418,8 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
   for (int o = 8; o > 0; o >>= 1) yv += __shfl_xor_sync(0xffffffffu, yv, o);
   if (s == 0) {
-    const float zz = __bfloat162float(proj[(size_t)b * ld_proj + off_z + c]);
-    y[(size_t)b * Di + c] = __float2bfloat16_rn(yv * silu_f(zz));
+    const float zz = proj[(size_t)b * ld_proj + off_z + c];
+    y[(size_t)b * Di + c] = yv * silu_f(zz);
   }
 }
 

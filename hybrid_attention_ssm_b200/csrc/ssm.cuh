@@ -18,8 +18,8 @@ __global__ void __launch_bounds__(256)
     conv1d_silu_kernel(const __nv_bfloat16* __restrict__ x, int ld_x, const float* __restrict__ w,
                        const float* __restrict__ bias, __nv_bfloat16* __restrict__ xc,
                        __nv_bfloat16* __restrict__ xcT, float* __restrict__ state, int T, int Tp, int Di) {
-  __shared__ float xs[CONV_TC + CONV_K - 1][CONV_CC + 1];
-  __shared__ __nv_bfloat16 ot[CONV_CC][CONV_TC + 8];
+  __shared__ __align__(16) float xs[CONV_TC + CONV_K - 1][CONV_CC + 1];
+  __shared__ __align__(16) __nv_bfloat16 ot[CONV_CC][CONV_TC + 8];
   const int c0 = blockIdx.x * CONV_CC;
   const int t0 = blockIdx.y * CONV_TC;
   const int b = blockIdx.z;

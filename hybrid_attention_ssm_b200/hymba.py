@@ -127,7 +127,7 @@ def make_cfg(dims) -> LayerCfg:
                     int(dims.is_global), int(dims.kv_role), float(dims.rope_base), float(dims.norm_eps))
 
 
-_BF16_W = ("meta", "w_in", "w_x", "w_out")
+_BF16_W = ("meta", "w_in", "w_x")
 _F32_W = ("conv_w", "conv_b", "dt_bias", "A", "g_attn", "g_ssm")
 
 
@@ -138,6 +138,8 @@ class DeviceWeights:
         self.t = {}
         for k in _BF16_W:
             self.t[k] = torch.from_numpy(np.ascontiguousarray(w[k], dtype=np.float32)).to(device).to(torch.bfloat16)
+        self.t["w_out"] = torch.from_numpy(np.ascontiguousarray(w["w_out"], dtype=np.float32)).to(device).to(
+            torch.float16)
         for k in _F32_W:
             self.t[k] = torch.from_numpy(np.ascontiguousarray(w[k], dtype=np.float32)).to(device)
         wdt = np.ascontiguousarray(w["w_dt"], dtype=np.float32)
@@ -157,7 +159,7 @@ class Cache:
     def __init__(self, dims, batch, max_tokens, kind=None, device="cuda", view=None):
         kind = (CACHE_GLOBAL if dims.is_global else CACHE_SWA) if kind is None else kind
         Hkv, D = dims.n_kv_heads, dims.head_dim
-        z = lambda *s: torch.zeros(*s, Hkv, D, dtype=torch.bfloat16, device=device)
+        z = lambda *s: torch.zeros(*s, Hkv, D, dtype=torch.float16, device=device)
         self.t = {}
         if view is None:
             self.t["k"], self.t["v"] = z(batch, max_tokens), z(batch, max_tokens)

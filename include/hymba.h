@@ -57,6 +57,7 @@ enum { HYMBA_CACHE_SWA = 0, HYMBA_CACHE_GLOBAL = 1 };
 enum { HYMBA_MODE_PREFILL = 0, HYMBA_MODE_DECODE = 1 };
 
 typedef uint16_t hymba_bf16;
+typedef uint16_t hymba_f16;   /* IEEE half bits */
 typedef struct CUstream_st* hymba_stream; /* identical to cudaStream_t; NULL = legacy stream */
 
 /* One mixer layer's sizes ([MC] §模型架构, [JJ] §数学表示).
@@ -92,7 +93,12 @@ typedef struct hymba_layer_cfg {
  *   A       [Di, S]           fp32  (negative) state matrix
  *   g_attn  [Hq*D]            fp32  beta1
  *   g_ssm   [Di]              fp32  beta2
- *   w_out   [d, Hq*D + Di]    bf16  output projection */
+ *   w_out   [d, Hq*D + Di]    fp16  output projection.  It multiplies the normalised,
+ *                                   rescaled branch outputs, which the library keeps in fp16:
+ *                                   after RMSNorm every value is at most sqrt(width)*|beta|/2
+ *                                   in magnitude, so fp16 cannot overflow and rounds 8x finer
+ *                                   than bf16.  bf16 weights convert to fp16 exactly when
+ *                                   6.1e-5 <= |w| <= 65504. */
 typedef struct hymba_layer_weights {
   const hymba_bf16* meta;
   const hymba_bf16* w_in;
@@ -105,11 +111,13 @@ typedef struct hymba_layer_weights {
   const float* A;
   const float* g_attn;
   const float* g_ssm;
-  const hymba_bf16* w_out;
+  const hymba_f16* w_out;
 } hymba_layer_weights;
 
 /* A KV cache, shared by a producer/consumer pair of adjacent SWA layers or owned by one
- * layer ([JJ] §Hymba 的整体架构).  All device pointers, bf16, K stored after RoPE.
+ * layer ([JJ] §Hymba 的整体架构).  All device pointers, fp16, K stored after RoPE.  The
+ * attention operands are fp16: keys, values and probabilities of a normalised-input layer
+ * sit far inside fp16's range, where it rounds 8x finer than bf16.
  *   kind HYMBA_CACHE_SWA:
  *     meta_k, meta_v  [B, M, Hkv, D]   keys/values of the meta tokens
  *     ring_k, ring_v  [B, W, Hkv, D]   input position p (>= M) lives in slot (p - M) mod W
@@ -127,12 +135,12 @@ typedef struct hymba_kv_cache {
   int n_meta;
   int window;
   int max_tokens;
-  hymba_bf16* meta_k;
-  hymba_bf16* meta_v;
-  hymba_bf16* ring_k;
-  hymba_bf16* ring_v;
-  hymba_bf16* k;
-  hymba_bf16* v;
+  hymba_f16* meta_k;
+  hymba_f16* meta_v;
+  hymba_f16* ring_k;
+  hymba_f16* ring_v;
+  hymba_f16* k;
+  hymba_f16* v;
 } hymba_kv_cache;
 
 /* Library version (major*10000 + minor*100 + patch). */
@@ -201,14 +209,14 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
 
 /* Byte offsets, inside a prefill workspace, of the stage buffers of the last prefill (for
  * stage-by-stage checks).  Layouts (rows r = b*T + t):
- *   q      [B*T, Hq*D]  bf16  queries after RoPE
+ *   q      [B*T, Hq*D]  fp16  queries after RoPE
  *   xz     [B*T, 2*Di]  bf16  in_proj x | z columns
  *   xc     [B*T, Di]    bf16  SiLU(conv(x))
  *   xbc    [B*T, ld_xbc] fp32 x_proj output: dt_low | B | C
  *   delta  [B, Di, Tp]  fp32  Delta, time-major with row stride Tp
  *   y      [B*T, Di]    bf16  scan output before the gate
- *   o      [B*T, Hq*D]  bf16  attention output
- *   u      [B*T, Hq*D+Di] bf16 normalised, rescaled, averaged branches (out_proj input) */
+ *   o      [B*T, Hq*D]  fp32  attention output
+ *   u      [B*T, Hq*D+Di] fp16 normalised, rescaled, averaged branches (out_proj input) */
 typedef struct hymba_stage_layout {
   size_t q, xz, xc, xbc, delta, y, o, u;
   int ld_xbc;

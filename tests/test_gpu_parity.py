@@ -11,7 +11,8 @@ from hybrid_attention_ssm_b200 import hymba as H
 from hybrid_attention_ssm_b200 import synth
 from oracle import hymba_oracle as orc
 
-from tests.helpers import (PrefillRun, assert_rel_inf, assert_rms, bf16_dev, f32_dev, to_np)
+from tests.helpers import (PrefillRun, assert_elem, assert_rel_inf, assert_rms, bf16_dev, f32_dev,
+                           to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -46,55 +47,52 @@ def test_gemm_matches_fp32_reference(M, N, K):
     ref = A.float() @ B.float().T + R.float()
     torch.cuda.synchronize()
     assert H.status_read(ws) == 0
-    assert_rms(to_np(C), to_np(ref), tol=1e-2, name=f"gemm {M}x{N}x{K}")
+    assert_rms(to_np(C), to_np(ref), name=f"gemm {M}x{N}x{K}")
 
 
 # ---------------------------------------------------------------------------------------
 # prefill: end to end and stage by stage
 # ---------------------------------------------------------------------------------------
 def _check_stages(run, ref, dims, w):
-    """Each stage against the oracle fed the GPU's own stage inputs."""
+    """Each stage against the oracle fed the GPU's own stage inputs.  Stages stored in 16
+    bits are checked elementwise against their unit roundoff; attention (bf16 P inside the
+    PV product) against the bf16-path bound."""
     B, T = run.B, run.T
     Di, R, S = dims.d_inner, dims.dt_rank, dims.d_state
     pos = np.arange(T)
-    # in_proj + RoPE
-    assert_rms(run.stage("q"), ref["Q"], name="Q")
+    # in_proj + RoPE, from the exact inputs
+    assert_elem(run.stage("q"), ref["Q"], name="Q")
     xz = run.stage("xz")
-    assert_rms(xz[..., :Di], ref["x_ssm"], name="x_ssm")
-    assert_rms(xz[..., Di:], ref["z"], name="z")
+    assert_elem(xz[..., :Di], ref["x_ssm"], name="x_ssm")
+    assert_elem(xz[..., Di:], ref["z"], name="z")
+    k = v = None
     if dims.kv_role != synth.KV_CONSUMER:
         k, v = run.kv()
-        assert_rms(k, ref["K"], name="K")
-        assert_rms(v, ref["V"], name="V")
-    # conv on the GPU's x
-    xc = run.stage("xc")
-    xbc = run.stage("xbc")
-    delta = run.stage("delta")
-    y = run.stage("y")
-    o = run.stage("o")
-    u = run.stage("u")
-    q = run.stage("q")
-    k, v = run.kv() if dims.kv_role != synth.KV_CONSUMER else (None, None)
+        assert_elem(k, ref["K"], name="K")
+        assert_elem(v, ref["V"], name="V")
+    xc, xbc, delta = run.stage("xc"), run.stage("xbc"), run.stage("delta")
+    y, o, u, q = run.stage("y"), run.stage("o"), run.stage("u"), run.stage("q")
+    out = to_np(run.out)
     for b in range(B):
         xc_ref, cst = orc.causal_conv1d_silu(xz[b, :, :Di], w["conv_w"], w["conv_b"])
-        assert_rms(xc[b], xc_ref, tol=1e-2, name="conv")
+        assert_elem(xc[b], xc_ref, name="conv")
         assert_rel_inf(to_np(run.conv[b]), cst, tol=1e-6, name="conv state")
         proj = xc[b] @ w["w_x"].astype(np.float64).T
         assert_rms(xbc[b, :, :R + 2 * S], proj, tol=1e-3, name="x_proj")
         d_ref = orc.softplus(xbc[b, :, :R] @ w["w_dt"].astype(np.float64).T + w["dt_bias"])
         assert_rel_inf(delta[b], d_ref, tol=5e-3, name="delta")
         # scan fed the GPU's own xc, delta, B, C, z
+        zb = xz[b, :, Di:]
         y_ref, h_ref = orc.selective_scan(xc[b], delta[b], w["A"], xbc[b, :, R:R + S],
-                                          xbc[b, :, R + S:R + 2 * S], xz[b, :, Di:])
+                                          xbc[b, :, R + S:R + 2 * S], zb)
         assert_rel_inf(to_np(run.ssm[b]), h_ref, tol=1e-4, name="scan state")
-        assert_rms(y[b] * orc.silu(xz[b, :, Di:]), y_ref, tol=1e-2, name="scan y")
+        assert_elem(y[b] * orc.silu(zb), y_ref, name="scan y")
         if k is not None:
             o_ref = orc.attention(q[b], k[b], v[b], pos, pos, dims.n_meta, dims.window, dims.is_global)
-            assert_rms(o[b], o_ref.reshape(T, -1), tol=1e-2, name="attention")
-        _, u_ref = orc.fuse_and_project(o[b], y[b] * orc.silu(xz[b, :, Di:]), w, dims)
-        assert_rms(u[b], u_ref, tol=1e-2, name="norm/avg")
-        out_ref = u[b] @ w["w_out"].astype(np.float64).T
-        assert_rms(to_np(run.out[b]), out_ref, tol=1e-2, name="out_proj")
+            assert_rms(o[b], o_ref.reshape(T, -1), name="attention")
+        _, u_ref = orc.fuse_and_project(o[b], y[b] * orc.silu(zb), w, dims)
+        assert_elem(u[b], u_ref, rel=2e-3, abs_rms=1e-4, name="norm/avg")
+        assert_elem(out[b], u[b] @ w["w_out"].astype(np.float64).T, name="out_proj")
 
 
 @pytest.mark.parametrize("name", ["tiny", "tiny_full"])
@@ -175,7 +173,7 @@ def test_prefill_shared_kv_pair():
     k, v = rp.kv()
     pos = np.arange(rc.T)
     o_ref = orc.attention(rc.stage("q")[0], k[0], v[0], pos, pos, cons.n_meta, cons.window, 0)
-    assert_rms(rc.stage("o")[0], o_ref.reshape(rc.T, -1), tol=1e-2, name="consumer attention")
+    assert_rms(rc.stage("o")[0], o_ref.reshape(rc.T, -1), name="consumer attention")
 
 
 def test_prefill_swa_hymba_layer():
@@ -229,7 +227,7 @@ def test_decode_pair_hymba():
     p = wl.decode_position
     cache = H.Cache(prod, wl.batch, 1)
     for n in ("meta_k", "meta_v", "ring_k", "ring_v"):
-        cache.t[n].copy_(bf16_dev(st_p[n]))
+        cache.t[n].copy_(f32_dev(st_p[n]).to(torch.float16))
     ssm_p, conv_p = f32_dev(st_p["ssm_state"]), f32_dev(st_p["conv_state"])
     ssm_c, conv_c = f32_dev(st_c["ssm_state"]), f32_dev(st_c["conv_state"])
     out_p = _decode(prod, wp, cache, st_p["x_new"], p, ssm_p, conv_p)
