@@ -113,9 +113,33 @@ int make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int rank,
 }
 
 // ----------------------------------------------------------------------------------------
+// kernel-level profiling: a CUDA event pair around every launch while enabled
+// ----------------------------------------------------------------------------------------
+struct ProfState {
+  bool on = false;
+  int cap = 0, n = 0;
+  cudaEvent_t* ev = nullptr;   // 2 * cap events
+  char (*names)[24] = nullptr;
+};
+ProfState g_prof;
+
+inline void prof_begin(const char* name, cudaStream_t st) {
+  if (!g_prof.on || g_prof.n >= g_prof.cap) return;
+  strncpy(g_prof.names[g_prof.n], name, 23);
+  g_prof.names[g_prof.n][23] = 0;
+  cudaEventRecord(g_prof.ev[2 * g_prof.n], st);
+}
+inline void prof_end(cudaStream_t st) {
+  if (!g_prof.on || g_prof.n >= g_prof.cap) return;
+  cudaEventRecord(g_prof.ev[2 * g_prof.n + 1], st);
+  ++g_prof.n;
+}
+
+// ----------------------------------------------------------------------------------------
 // GEMM launcher
 // ----------------------------------------------------------------------------------------
 struct GemmCall {
+  const char* name = "gemm";
   // A source 0 (optional): [rows0, K] row stride lda0 elements
   const void* a0 = nullptr;
   int rows0 = 0;
@@ -137,7 +161,7 @@ struct GemmCall {
 
 template <int BN, int STAGES, int ET>
 int launch_gemm_inst(const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& mb, const GemmParams& p,
-                     int grid, cudaStream_t st) {
+                     int grid, cudaStream_t st, const char* name) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -147,7 +171,9 @@ int launch_gemm_inst(const CUtensorMap& m0, const CUtensorMap& m1, const CUtenso
     HY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
     attr_set[dev & 63] = true;
   }
+  prof_begin(name, st);
   kern<<<grid, GEMM_THREADS, smem, st>>>(m0, m1, mb, p);
+  prof_end(st);
   HY_CUDA(cudaGetLastError());
   return HYMBA_OK;
 }
@@ -196,17 +222,17 @@ int run_gemm(GemmCall& c, const DeviceInfo& dev, cudaStream_t st) {
   if (p.total_tiles <= 0) return HYMBA_OK;
   const int grid = p.total_tiles < dev.sms ? p.total_tiles : dev.sms;
   if (tf32) {
-    if (c.bn == 256) return launch_gemm_inst<256, 4, ET_TF32>(m0, m1, mb, p, grid, st);
-    if (c.bn == 128) return launch_gemm_inst<128, 6, ET_TF32>(m0, m1, mb, p, grid, st);
+    if (c.bn == 256) return launch_gemm_inst<256, 4, ET_TF32>(m0, m1, mb, p, grid, st, c.name);
+    if (c.bn == 128) return launch_gemm_inst<128, 6, ET_TF32>(m0, m1, mb, p, grid, st, c.name);
   } else if (c.etype == ET_F16) {
-    if (c.bn == 256) return launch_gemm_inst<256, 4, ET_F16>(m0, m1, mb, p, grid, st);
-    if (c.bn == 128) return launch_gemm_inst<128, 6, ET_F16>(m0, m1, mb, p, grid, st);
-    if (c.bn == 64) return launch_gemm_inst<64, 8, ET_F16>(m0, m1, mb, p, grid, st);
+    if (c.bn == 256) return launch_gemm_inst<256, 4, ET_F16>(m0, m1, mb, p, grid, st, c.name);
+    if (c.bn == 128) return launch_gemm_inst<128, 6, ET_F16>(m0, m1, mb, p, grid, st, c.name);
+    if (c.bn == 64) return launch_gemm_inst<64, 8, ET_F16>(m0, m1, mb, p, grid, st, c.name);
   } else {
-    if (c.bn == 256) return launch_gemm_inst<256, 4, ET_BF16>(m0, m1, mb, p, grid, st);
-    if (c.bn == 160) return launch_gemm_inst<160, 5, ET_BF16>(m0, m1, mb, p, grid, st);
-    if (c.bn == 128) return launch_gemm_inst<128, 6, ET_BF16>(m0, m1, mb, p, grid, st);
-    if (c.bn == 64) return launch_gemm_inst<64, 8, ET_BF16>(m0, m1, mb, p, grid, st);
+    if (c.bn == 256) return launch_gemm_inst<256, 4, ET_BF16>(m0, m1, mb, p, grid, st, c.name);
+    if (c.bn == 160) return launch_gemm_inst<160, 5, ET_BF16>(m0, m1, mb, p, grid, st, c.name);
+    if (c.bn == 128) return launch_gemm_inst<128, 6, ET_BF16>(m0, m1, mb, p, grid, st, c.name);
+    if (c.bn == 64) return launch_gemm_inst<64, 8, ET_BF16>(m0, m1, mb, p, grid, st, c.name);
   }
   return fail(HYMBA_ERR_UNSUPPORTED, "no GEMM tile width %d", c.bn);
 }
@@ -340,6 +366,38 @@ int check_weights(const hymba_layer_weights* w, const Dims& m, bool need_meta) {
 extern "C" {
 
 int hymba_version(void) { return 10000; }
+
+int hymba_profile_begin(int max_records) {
+  if (max_records < 1) return fail(HYMBA_ERR_INVALID_ARG, "max_records < 1");
+  if (g_prof.cap < max_records) {
+    for (int i = 0; i < 2 * g_prof.cap; ++i) cudaEventDestroy(g_prof.ev[i]);
+    delete[] g_prof.ev;
+    delete[] g_prof.names;
+    g_prof.ev = new cudaEvent_t[2 * max_records];
+    g_prof.names = new char[max_records][24];
+    for (int i = 0; i < 2 * max_records; ++i) HY_CUDA(cudaEventCreate(&g_prof.ev[i]));
+    g_prof.cap = max_records;
+  }
+  g_prof.n = 0;
+  g_prof.on = true;
+  return HYMBA_OK;
+}
+
+int hymba_profile_end(hymba_prof_record* out, int max_records, int* n_records) {
+  if (out == nullptr || n_records == nullptr) return fail(HYMBA_ERR_INVALID_ARG, "NULL argument");
+  g_prof.on = false;
+  const int n = g_prof.n < max_records ? g_prof.n : max_records;
+  for (int i = 0; i < n; ++i) {
+    HY_CUDA(cudaEventSynchronize(g_prof.ev[2 * i + 1]));
+    float ms = 0.f;
+    HY_CUDA(cudaEventElapsedTime(&ms, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]));
+    memcpy(out[i].name, g_prof.names[i], 24);
+    out[i].ms = ms;
+  }
+  *n_records = n;
+  g_prof.n = 0;
+  return HYMBA_OK;
+}
 
 const char* hymba_last_error(void) { return g_err.c_str(); }
 
@@ -525,6 +583,7 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     }
     c.b = w->w_in; c.N = m.P; c.ldb = m.d; c.K = m.d;
     c.bn = 256;
+    c.name = "in_proj";
     c.p.mode = EPI_PROJ;
     c.p.out_batches = B;
     c.p.T_out = T;
@@ -544,8 +603,10 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
   float* cstate = conv_state_out != nullptr ? conv_state_out : f32(L.cstate);
   {
     dim3 grid(cdiv(m.Di, CONV_CC), cdiv(T, CONV_TC), B);
+    prof_begin("conv1d_silu", st);
     conv1d_silu_kernel<<<grid, 256, 0, st>>>(bf(L.xz), 2 * m.Di, w->conv_w, w->conv_b, bf(L.xc), bf(L.xcT), cstate,
                                               T, L.Tp, m.Di);
+    prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
   // 3. x_proj (split-K, fp32 atomics): [dt_low | B | C]
@@ -559,6 +620,7 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     const int kb = cdiv(m.Di, 64);
     int sk = cdiv(dev->sms, mt);
     c.split_k = sk > kb ? kb : sk;
+    c.name = "x_proj";
     c.p.mode = EPI_ATOMIC_F32;
     c.p.out = f32(L.xbc);
     c.p.ld_out = m.ld_xbc;
@@ -573,6 +635,7 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     c.a1 = f32(L.xbc); c.nb1 = B; c.rows1 = T; c.lda1 = m.ld_xbc; c.a1_bstride = (long long)T * m.ld_xbc;
     c.b = w->w_dt; c.N = m.Di; c.ldb = w->w_dt_ld; c.K = m.R;
     c.bn = pick_bn_wide(B * cdiv(T, GEMM_BM), m.Di, dev->sms);
+    c.name = "dt_proj";
     c.p.mode = EPI_SOFTPLUS_T;
     c.p.out = f32(L.dT);
     c.p.T_out = L.Tp;
@@ -611,22 +674,28 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
       attr[d & 63] = true;
     }
     dim3 grid(ap.q_tiles, m.Hq, B);
+    prof_begin("attention", st);
     attn_fwd_kernel<<<grid, ATT_THREADS, ATT_SMEM, st>>>(mq, mk, mv, ap);
+    prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
   // 6. selective scan
   float* sstate = ssm_state_out != nullptr ? ssm_state_out : f32(L.sstate);
   {
     dim3 grid(m.Di / SCAN_CH, B);
+    prof_begin("selective_scan", st);
     selective_scan_kernel<<<grid, SCAN_THREADS, 0, st>>>(bf(L.xcT), f32(L.dT), f32(L.xbc) + m.R, m.ld_xbc, w->A,
                                                          bf(L.y), sstate, T, L.Tp, m.Di);
+    prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
   // 7. per-branch RMSNorm, gate, beta, average
   {
+    prof_begin("norm_avg", st);
     branch_norm_avg_kernel<__nv_bfloat16><<<(unsigned)rows, 256, 0, st>>>(
         f32(L.o), m.qw, m.qw, bf(L.y), m.Di, bf(L.xz) + m.Di, 2 * m.Di, m.Di, w->g_attn, w->g_ssm, cfg->norm_eps,
         h16(L.u), m.uw);
+    prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
   // 8. out_proj (+ residual)
@@ -635,6 +704,7 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     c.a1 = h16(L.u); c.nb1 = 1; c.rows1 = (int)rows; c.lda1 = m.uw; c.a1_bstride = (long long)rows * m.uw;
     c.b = w->w_out; c.N = m.d; c.ldb = m.uw; c.K = m.uw;
     c.etype = ET_F16;
+    c.name = "out_proj";
     c.bn = pick_bn_wide(cdiv(rows, GEMM_BM), m.d, dev->sms);
     c.p.mode = EPI_BF16;
     c.p.out = out;
@@ -651,10 +721,12 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     const int n_rows = m.M + (T - first_win);
     const int n = n_rows * (m.kvw / 8);
     dim3 grid(cdiv(n, 256), B);
+    prof_begin("swa_cache_finalize", st);
     swa_cache_finalize_kernel<<<grid, 256, 0, st>>>(
         reinterpret_cast<const __half*>(kv->k), reinterpret_cast<const __half*>(kv->v), Lmax, T, m.M, m.W, m.kvw,
         reinterpret_cast<__half*>(kv->meta_k), reinterpret_cast<__half*>(kv->meta_v),
         reinterpret_cast<__half*>(kv->ring_k), reinterpret_cast<__half*>(kv->ring_v));
+    prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
   return HYMBA_OK;
@@ -703,6 +775,7 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     c.a1 = w->w_in; c.nb1 = 1; c.rows1 = m.P; c.lda1 = m.d; c.a1_bstride = (long long)m.P * m.d;
     c.b = x; c.N = B; c.ldb = m.d; c.K = m.d;
     c.bn = pick_bn_cover(B);
+    c.name = "decode_in_proj";
     c.p.mode = EPI_F32_T;
     c.p.out = f32(L.proj);
     c.p.ld_out = m.P;
@@ -738,16 +811,22 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     ap.part = f32(L.part);
     if (ap.n_splits > L.n_splits) return fail(HYMBA_ERR_WORKSPACE, "decode workspace sized for fewer keys");
     dim3 grid(ap.n_splits, m.Hkv, B);
+    prof_begin("decode_attn", st);
     decode_attn_kernel<<<grid, 128, 0, st>>>(ap);
+    prof_end(st);
     HY_CUDA(cudaGetLastError());
+    prof_begin("decode_attn_combine", st);
     decode_attn_combine_kernel<<<dim3(m.Hq, B), 64, 0, st>>>(f32(L.part), ap.n_splits, m.Hq, f32(L.o), m.qw);
+    prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
   // 3. conv step
   {
     const int n = B * m.Di;
+    prof_begin("decode_conv", st);
     decode_conv_kernel<<<cdiv(n, 256), 256, 0, st>>>(f32(L.proj), m.P, m.xz_off, m.Di, w->conv_w, w->conv_b,
                                                       conv_state, bf(L.xc), B);
+    prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
   // 4. x_proj (swap-AB, split-K into fp32)
@@ -757,6 +836,7 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     c.a1 = w->w_x; c.nb1 = 1; c.rows1 = m.R + 2 * m.S; c.lda1 = m.Di; c.a1_bstride = (long long)c.rows1 * m.Di;
     c.b = bf(L.xc); c.N = B; c.ldb = m.Di; c.K = m.Di;
     c.bn = pick_bn_cover(B);
+    c.name = "decode_x_proj";
     const int tiles = cdiv(c.rows1, GEMM_BM) * cdiv(B, c.bn);
     c.split_k = cdiv(dev->sms, tiles);
     c.p.mode = EPI_ATOMIC_F32_T;
@@ -770,14 +850,18 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
   // 5. dt_proj + softplus + state update + C.h + gate
   {
     dim3 grid(m.Di / 16, B);
+    prof_begin("decode_ssm", st);
     decode_ssm_kernel<<<grid, 256, 0, st>>>(f32(L.xbc), m.ld_xbc, m.R, w->w_dt, w->w_dt_ld, w->dt_bias, w->A,
                                             bf(L.xc), f32(L.proj), m.P, m.xz_off + m.Di, ssm_state, f32(L.y), m.Di);
+    prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
   // 6. norm + average (y already gated)
   {
+    prof_begin("decode_norm_avg", st);
     branch_norm_avg_kernel<float><<<B, 256, 0, st>>>(f32(L.o), m.qw, m.qw, f32(L.y), m.Di, nullptr, 0, m.Di,
                                                      w->g_attn, w->g_ssm, cfg->norm_eps, h16(L.u), m.uw);
+    prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
   // 7. out_proj (swap-AB, split-K) and the bf16 (+ residual) store
@@ -788,6 +872,7 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     c.b = h16(L.u); c.N = B; c.ldb = m.uw; c.K = m.uw;
     c.etype = ET_F16;
     c.bn = pick_bn_cover(B);
+    c.name = "decode_out_proj";
     const int tiles = cdiv(m.d, GEMM_BM) * cdiv(B, c.bn);
     c.split_k = cdiv(dev->sms, tiles);
     c.p.mode = EPI_ATOMIC_F32_T;
@@ -798,8 +883,10 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     c.p.status = status;
     HY_TRY(run_gemm(c, *dev, st));
     const int n = B * m.d;
+    prof_begin("decode_out_store", st);
     f32_to_bf16_residual_kernel<<<cdiv(n, 256), 256, 0, st>>>(
         f32(L.acc), reinterpret_cast<const __nv_bfloat16*>(residual), reinterpret_cast<__nv_bfloat16*>(out), n);
+    prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
   return HYMBA_OK;
@@ -830,8 +917,10 @@ int hymba_rmsnorm(const hymba_bf16* x, const float* gain, int rows, int d, float
   if (x == nullptr || gain == nullptr || out == nullptr || rows < 1 || d < 8 || d % 8 || !aligned16(x) ||
       !aligned16(out))
     return fail(HYMBA_ERR_INVALID_ARG, "rmsnorm arguments");
-  rmsnorm_kernel<<<rows, 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<const __nv_bfloat16*>(x), gain, d, eps,
+  prof_begin("rmsnorm", (cudaStream_t)stream);
+    rmsnorm_kernel<<<rows, 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<const __nv_bfloat16*>(x), gain, d, eps,
                                                           reinterpret_cast<__nv_bfloat16*>(out));
+    prof_end((cudaStream_t)stream);
   HY_CUDA(cudaGetLastError());
   return HYMBA_OK;
 }
@@ -850,6 +939,7 @@ int hymba_ffn_swiglu(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hym
     c.a1 = h; c.nb1 = 1; c.rows1 = rows; c.lda1 = d; c.a1_bstride = (long long)rows * d;
     c.b = w_gate_up; c.N = 2 * F; c.ldb = d; c.K = d;
     c.bn = pick_bn_wide(cdiv(rows, GEMM_BM), 2 * F, dev->sms);
+    c.name = "ffn_gate_up";
     c.p.mode = EPI_SWIGLU;
     c.p.out = act;
     c.p.ld_out = F;
@@ -861,6 +951,7 @@ int hymba_ffn_swiglu(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hym
     GemmCall c;
     c.a1 = act; c.nb1 = 1; c.rows1 = rows; c.lda1 = F; c.a1_bstride = (long long)rows * F;
     c.b = w_down; c.N = d; c.ldb = F; c.K = F;
+    c.name = "ffn_down";
     c.bn = pick_bn_wide(cdiv(rows, GEMM_BM), d, dev->sms);
     c.p.mode = EPI_BF16;
     c.p.out = out;

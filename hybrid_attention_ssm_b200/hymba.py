@@ -49,6 +49,10 @@ class KVCache(ctypes.Structure):
                [(n, _vp) for n in ("meta_k", "meta_v", "ring_k", "ring_v", "k", "v")]
 
 
+class ProfRecord(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 24), ("ms", ctypes.c_float)]
+
+
 class StageLayout(ctypes.Structure):
     _fields_ = [(n, _c_size) for n in ("q", "xz", "xc", "xbc", "delta", "y", "o", "u")] + \
                [("ld_xbc", _c_int), ("Tp", _c_int)]
@@ -94,6 +98,8 @@ def lib():
             "hymba_ffn_swiglu": ([_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp], _c_int),
             "hymba_set_wait_limit_ns": ([ctypes.c_ulonglong], _c_int),
             "hymba_selftest_wait_timeout": ([_vp, _c_size, _vp], _c_int),
+            "hymba_profile_begin": ([_c_int], _c_int),
+            "hymba_profile_end": ([ctypes.POINTER(ProfRecord), _c_int, ctypes.POINTER(_c_int)], _c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -261,6 +267,18 @@ def interleave_gate_up(w_gate, w_up):
     g = w_gate.reshape(F // 32, 32, d)
     u = w_up.reshape(F // 32, 32, d)
     return np.concatenate([g, u], axis=1).reshape(2 * F, d)
+
+
+def profile_begin(max_records=8192):
+    check(lib().hymba_profile_begin(max_records))
+
+
+def profile_end(max_records=8192):
+    """[(kernel name, milliseconds)] of every launch since profile_begin, in launch order."""
+    recs = (ProfRecord * max_records)()
+    n = ctypes.c_int()
+    check(lib().hymba_profile_end(recs, max_records, ctypes.byref(n)))
+    return [(recs[i].name.decode(), float(recs[i].ms)) for i in range(n.value)]
 
 
 def set_wait_limit_ns(ns):

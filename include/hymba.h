@@ -253,6 +253,18 @@ int hymba_set_wait_limit_ns(unsigned long long ns);
  * Exercises the timeout path without faulting or hanging the device. */
 int hymba_selftest_wait_timeout(void* workspace, size_t ws_bytes, hymba_stream stream);
 
+/* Kernel-level timing: while enabled, every kernel the library launches is bracketed by a
+ * pair of CUDA events on its stream (the events are created on the host by the first
+ * hymba_profile_begin; no device memory is allocated).  hymba_profile_end synchronises on
+ * the recorded events and returns, in launch order, each kernel's name and elapsed time.
+ * At most max_records launches are recorded; not thread-safe. */
+typedef struct hymba_prof_record {
+  char name[24];
+  float ms;
+} hymba_prof_record;
+int hymba_profile_begin(int max_records);
+int hymba_profile_end(hymba_prof_record* out, int max_records, int* n_records);
+
 #ifdef __cplusplus
 }
 #endif
