@@ -974,3 +974,62 @@ int hymba_selftest_wait_timeout(void* ws, size_t ws_bytes, hymba_stream stream) 
 }
 
 }  // extern "C"
+
+// ========================================================================================
+// Decode step without a caller-provided workspace.
+//
+// Some callers cannot allocate device memory at the point where they run a decode step:
+// code inside a region that is being captured into a CUDA graph (cudaMalloc is not a
+// capturable stream operation), serving loops that must not hit cudaMalloc's implicit
+// device synchronisation between tokens, and plugins whose host runtime owns every device
+// allocation and hands them only inputs and outputs.  For them the scratch memory of the
+// decode step lives in this file-scope device array instead of a workspace argument.
+// ========================================================================================
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB, held by every GPU that loads the library
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+void* g_noalloc_ptr[64] = {nullptr};
+std::mutex g_noalloc_mu;
+
+// Device address of g_noalloc_scratch on the current device (host code only sees a host
+// stand-in for the symbol, which must never be handed to a kernel).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  HY_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(HYMBA_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(HYMBA_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return HYMBA_OK;
+}
+
+}  // namespace
+
+extern "C" int hymba_mixer_decode_noalloc(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
+                                          const hymba_bf16* x, int batch, int position, hymba_kv_cache* kv,
+                                          float* ssm_state, float* conv_state, const hymba_bf16* residual,
+                                          hymba_bf16* out, hymba_stream stream) {
+  if (kv == nullptr) return fail(HYMBA_ERR_INVALID_ARG, "kv cache is NULL");
+  size_t need = 0;
+  HY_TRY(hymba_mixer_workspace_size(cfg, batch, kv->max_tokens, 0, HYMBA_MODE_DECODE, &need));
+  if (need > kNoAllocScratchBytes)
+    return fail(HYMBA_ERR_WORKSPACE,
+                "decode step needs %zu bytes of scratch, more than the %zu-byte built-in scratch; "
+                "use hymba_mixer_decode with a workspace",
+                need, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  HY_TRY(noalloc_scratch(&scratch));
+  // The array keeps the previous call's contents: the status word must start at zero (the
+  // other buffers the step reads are either fully written first or cleared by the step).
+  HY_CUDA(cudaMemsetAsync(scratch, 0, 256, (cudaStream_t)stream));
+  return hymba_mixer_decode(cfg, w, x, batch, position, kv, ssm_state, conv_state, residual, out, scratch,
+                            kNoAllocScratchBytes, stream);
+}

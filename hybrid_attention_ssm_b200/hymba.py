@@ -98,6 +98,8 @@ def lib():
             "hymba_ffn_swiglu": ([_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp], _c_int),
             "hymba_set_wait_limit_ns": ([ctypes.c_ulonglong], _c_int),
             "hymba_selftest_wait_timeout": ([_vp, _c_size, _vp], _c_int),
+            "hymba_mixer_decode_noalloc": ([ctypes.POINTER(LayerCfg), ctypes.POINTER(LayerWeights), _vp, _c_int,
+                                            _c_int, ctypes.POINTER(KVCache), _vp, _vp, _vp, _vp, _vp], _c_int),
             "hymba_profile_begin": ([_c_int], _c_int),
             "hymba_profile_end": ([ctypes.POINTER(ProfRecord), _c_int, ctypes.POINTER(_c_int)], _c_int),
         }
@@ -240,6 +242,15 @@ def mixer_decode(dims, dw: DeviceWeights, x, position, kv: Cache, ssm_state, con
     check(lib().hymba_mixer_decode(ctypes.byref(cfg), ctypes.byref(dw.c), ptr(x), x.shape[0], position,
                                    ctypes.byref(kv.c), ptr(ssm_state), ptr(conv_state), ptr(residual), ptr(out),
                                    ptr(ws), ws.numel(), stream_handle(stream)))
+
+
+def mixer_decode_noalloc(dims, dw: DeviceWeights, x, position, kv: Cache, ssm_state, conv_state, out,
+                         residual=None, stream=None, cfg=None):
+    """hymba_mixer_decode with the library's built-in scratch instead of a workspace."""
+    cfg = make_cfg(dims) if cfg is None else cfg
+    check(lib().hymba_mixer_decode_noalloc(ctypes.byref(cfg), ctypes.byref(dw.c), ptr(x), x.shape[0], position,
+                                           ctypes.byref(kv.c), ptr(ssm_state), ptr(conv_state), ptr(residual),
+                                           ptr(out), stream_handle(stream)))
 
 
 def gemm_bf16(A, B, C, status_ws, residual=None, stream=None):

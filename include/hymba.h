@@ -253,6 +253,26 @@ int hymba_set_wait_limit_ns(unsigned long long ns);
  * Exercises the timeout path without faulting or hanging the device. */
 int hymba_selftest_wait_timeout(void* workspace, size_t ws_bytes, hymba_stream stream);
 
+/* hymba_mixer_decode without a workspace argument, for callers that cannot allocate device
+ * memory where they run a decode step (inside a CUDA graph capture, in a serving loop
+ * that must not take cudaMalloc's device synchronisation, or as a plugin whose host
+ * runtime owns all device memory).  The pages have no counterpart: this is a deployment
+ * convenience of this library.  Arguments and results are those of hymba_mixer_decode.
+ *   - Scratch: a built-in 16 MiB device array (every GPU that loads the library holds it
+ *     until exit).  A step that needs more (hymba_mixer_workspace_size, mode DECODE, with
+ *     n_tokens = kv->max_tokens) is rejected with HYMBA_ERR_WORKSPACE; Hymba-1.5B-sized SWA
+ *     layers fit up to batch 64.
+ *   - The first call on each device looks up the array's device address; make that first
+ *     call before any stream capture.
+ *   - Every call on a device uses the same array: calls that can overlap on the GPU (for
+ *     example on two streams of one device) race on it; the caller must serialise them.
+ *   - The status word at the start of the array is cleared at every call, so device-side
+ *     timeouts of this variant are not reported; use hymba_mixer_decode to read them.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine. */
+int hymba_mixer_decode_noalloc(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x,
+                               int batch, int position, hymba_kv_cache* kv, float* ssm_state, float* conv_state,
+                               const hymba_bf16* residual, hymba_bf16* out, hymba_stream stream);
+
 /* Kernel-level timing: while enabled, every kernel the library launches is bracketed by a
  * pair of CUDA events on its stream (the events are created on the host by the first
  * hymba_profile_begin; no device memory is allocated).  hymba_profile_end synchronises on
