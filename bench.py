@@ -247,6 +247,11 @@ def run_hymba(args, rank, world, device):
     launches_per_step = len(recs) / args.steps
 
     # ---------------- e2e: host buffers through the C ABI ----------------
+    if args.no_e2e:
+        decode = None if args.no_decode else run_decode(args, device, world)
+        return {"tokens_per_step": B * T, "ms_per_step": ms_per_step, "step_ms_p50": float(np.median(step_ms)),
+                "e2e_ms": float("nan"), "h2d": 0, "d2h": 0, "roofline": roof, "step_roofline": step_roof,
+                "kernels": kern, "clocks": clk.summary(), "launches_per_step": launches_per_step, "decode": decode}
     xh = torch.from_numpy(X).to(torch.bfloat16).pin_memory()
     oh = torch.empty(B, T, dims.d_model, dtype=torch.bfloat16).pin_memory()
     e2e_steps = max(3, min(args.steps, 50))
@@ -267,7 +272,7 @@ def run_hymba(args, rank, world, device):
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         e2e_ms = float(t.item())
 
-    decode = run_decode(args, device, world)
+    decode = None if args.no_decode else run_decode(args, device, world)
     res = {
         "tokens_per_step": B * T,
         "ms_per_step": ms_per_step,
@@ -431,6 +436,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="hymba", choices=["hymba", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement (profiling runs)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer measurement (profiling runs)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
