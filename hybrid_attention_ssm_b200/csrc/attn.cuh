@@ -1,18 +1,22 @@
-// Prefill attention on tcgen05 for sm_100a, head dim 64, GQA, RoPE already applied.
-// Q, K, V and the probabilities P are fp16 (P in [0, 1] and the normalised-input
-// activations sit well inside fp16's range, where it rounds 8x finer than bf16); scores and
-// the output accumulate in fp32.
+// Prefill attention on tcgen05 for sm_100a: head dim 64, GQA, RoPE already applied, fp16
+// Q/K/V/P (keys, values and probabilities sit far inside fp16's range, where it rounds 8x
+// finer than bf16), fp32 scores and accumulators.
 //
-// One CTA per (query tile of 128 rows, query head, sequence).  The key tiles a CTA visits
-// are the meta-token tiles plus the tiles that intersect the sliding window of its rows
-// (or every causal tile for a global layer): block skipping, no dense mask.  Only tiles
-// that straddle the causal diagonal or the window edge apply an element mask.
+// One CTA per (query tile of 128 rows, query head, sequence); two CTAs share an SM
+// (256 TMEM columns and ~100 KB of shared memory each), so one CTA's softmax overlaps the
+// other's MMAs.  The key tiles a CTA visits are the meta-token tiles plus the tiles that
+// intersect the sliding window of its rows (every causal tile for a global layer): block
+// skipping, no dense mask.  Only tiles that straddle the causal diagonal or the window
+// edge apply an element mask.
 //
-// 192 threads: warp 0 issues TMA loads (Q once, K/V tiles through a 2-stage ring),
-// warp 1 allocates TMEM and issues the MMAs (S = Q K^T into a double-buffered TMEM tile,
-// O_j = P_j V_j into a double-buffered TMEM tile), warps 2..5 run the online softmax with
-// one query row per thread, write P (fp16) into 128B-swizzled shared memory for the PV
-// MMA, and accumulate O in registers.
+// 192 threads:
+//   warp 0      TMA: Q once, K/V tiles through a 2-stage ring
+//   warp 1      TMEM allocation and MMA issue: S = Q K^T (M128 N128 K64) into TMEM, then
+//               O += P V with P read straight from TMEM (the "A in tensor memory" form)
+//   warps 2..5  softmax, one query row per thread: the whole S row comes into registers
+//               with one wait, P = 2^(s - m) is packed to fp16 and written back over the
+//               S columns; O stays in TMEM and is rescaled only when the running max grows
+//               by more than 2^8 (P <= 256 otherwise), then divided by the row sum at the end.
 #pragma once
 #include "common.cuh"
 
@@ -33,16 +37,18 @@ constexpr int ATT_THREADS = 192;
 constexpr int ATT_STAGES = 2;
 constexpr int ATT_Q_BYTES = 128 * 128;
 constexpr int ATT_KV_BYTES = 128 * 128;          // one K or V tile: 128 keys x 64 dims fp16
-constexpr int ATT_P_BYTES = 128 * 256;           // P tile: 128 rows x 128 keys fp16
 constexpr int ATT_OFF_Q = 0;
 constexpr int ATT_OFF_K = ATT_OFF_Q + ATT_Q_BYTES;
 constexpr int ATT_OFF_V = ATT_OFF_K + ATT_STAGES * ATT_KV_BYTES;
-constexpr int ATT_OFF_P = ATT_OFF_V + ATT_STAGES * ATT_KV_BYTES;
-constexpr int ATT_OFF_BAR = ATT_OFF_P + 2 * ATT_P_BYTES;
-constexpr int ATT_SMEM = ATT_OFF_BAR + 256 + 1024;
+constexpr int ATT_OFF_BAR = ATT_OFF_V + ATT_STAGES * ATT_KV_BYTES;
+// requested dynamic shared memory: the tiles need ~81 KB; asking for more keeps a third
+// CTA (which would wait for TMEM) off the SM.
+constexpr int ATT_SMEM = 100 * 1024;
+constexpr uint32_t ATT_TMEM_COLS = 256;          // S/P: cols 0..127, O: cols 128..191
+constexpr float ATT_RESCALE_LOG2 = 8.f;          // lazy rescale threshold (P <= 2^8)
 
 // Key tiles (128 keys each) visited by query tile qt, in order: meta tiles first, then the
-// window.  Returns the count; tile(i) gives the i-th key-tile index.
+// window.
 struct KeyTiles {
   int n_meta_tiles;   // leading meta tiles that precede the window range
   int lo, hi;         // window tile range [lo, hi]
@@ -67,19 +73,81 @@ __device__ __forceinline__ KeyTiles key_tiles(const AttnParams& p, int qt) {
   return kt;
 }
 
-__global__ void __launch_bounds__(ATT_THREADS, 1)
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, fp16 inputs, fp32 accumulate.
+__device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 32 lanes x 128 fp32 columns of TMEM into registers with a single completion wait.
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float* v) {
+  uint32_t r[128];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+        : "=r"(r[c * 32 + 0]), "=r"(r[c * 32 + 1]), "=r"(r[c * 32 + 2]), "=r"(r[c * 32 + 3]), "=r"(r[c * 32 + 4]),
+          "=r"(r[c * 32 + 5]), "=r"(r[c * 32 + 6]), "=r"(r[c * 32 + 7]), "=r"(r[c * 32 + 8]), "=r"(r[c * 32 + 9]),
+          "=r"(r[c * 32 + 10]), "=r"(r[c * 32 + 11]), "=r"(r[c * 32 + 12]), "=r"(r[c * 32 + 13]),
+          "=r"(r[c * 32 + 14]), "=r"(r[c * 32 + 15]), "=r"(r[c * 32 + 16]), "=r"(r[c * 32 + 17]),
+          "=r"(r[c * 32 + 18]), "=r"(r[c * 32 + 19]), "=r"(r[c * 32 + 20]), "=r"(r[c * 32 + 21]),
+          "=r"(r[c * 32 + 22]), "=r"(r[c * 32 + 23]), "=r"(r[c * 32 + 24]), "=r"(r[c * 32 + 25]),
+          "=r"(r[c * 32 + 26]), "=r"(r[c * 32 + 27]), "=r"(r[c * 32 + 28]), "=r"(r[c * 32 + 29]),
+          "=r"(r[c * 32 + 30]), "=r"(r[c * 32 + 31])
+        : "r"(taddr + c * 32)
+        : "memory");
+  }
+  // the wait takes every loaded register as an operand so no use can move above it
+#pragma unroll
+  for (int i = 0; i < 128; i += 32) {
+    asm volatile(
+        "tcgen05.wait::ld.sync.aligned;\n"
+        : "+r"(r[i + 0]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]), "+r"(r[i + 5]),
+          "+r"(r[i + 6]), "+r"(r[i + 7]), "+r"(r[i + 8]), "+r"(r[i + 9]), "+r"(r[i + 10]), "+r"(r[i + 11]),
+          "+r"(r[i + 12]), "+r"(r[i + 13]), "+r"(r[i + 14]), "+r"(r[i + 15]), "+r"(r[i + 16]), "+r"(r[i + 17]),
+          "+r"(r[i + 18]), "+r"(r[i + 19]), "+r"(r[i + 20]), "+r"(r[i + 21]), "+r"(r[i + 22]), "+r"(r[i + 23]),
+          "+r"(r[i + 24]), "+r"(r[i + 25]), "+r"(r[i + 26]), "+r"(r[i + 27]), "+r"(r[i + 28]), "+r"(r[i + 29]),
+          "+r"(r[i + 30]), "+r"(r[i + 31])
+        :
+        : "memory");
+  }
+#pragma unroll
+  for (int i = 0; i < 128; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 32 lanes x 32 columns of 32-bit values from registers into TMEM (completion is awaited
+// with tmem_wait_st before the data is handed to the tensor core).
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__global__ void __launch_bounds__(ATT_THREADS, 2)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                     const __grid_constant__ CUtensorMap mapV, const __grid_constant__ AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ATT_OFF_BAR);
-  uint64_t* q_full = bars;                 // 1
-  uint64_t* kv_full = bars + 1;            // ATT_STAGES
-  uint64_t* kv_empty = kv_full + ATT_STAGES;
-  uint64_t* s_full = kv_empty + ATT_STAGES;  // 2
-  uint64_t* p_full = s_full + 2;             // 2
-  uint64_t* o_full = p_full + 2;             // 2
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 2);
+  uint64_t* q_full = bars;                   // 1
+  uint64_t* kv_full = bars + 1;              // ATT_STAGES
+  uint64_t* kv_empty = kv_full + ATT_STAGES; // ATT_STAGES
+  uint64_t* s_full = kv_empty + ATT_STAGES;  // S of tile j in TMEM
+  uint64_t* p_full = s_full + 1;             // P of tile j in TMEM (S read, rescale done)
+  uint64_t* o_done = p_full + 1;             // PV of tile j complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -97,22 +165,21 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
-      mbar_init(&o_full[i], 1);
-    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(o_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
+    tmem_alloc(tmem_slot, ATT_TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;   // S0: +0, S1: +128, O0: +256, O1: +320
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t TM_S = tmem, TM_O = tmem + 128;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -139,41 +206,39 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t IDESC_S = make_idesc(128, 128, 0u, false, false);   // fp16 Q, K
-      constexpr uint32_t IDESC_O = make_idesc(128, 64, 0u, false, true);     // fp16 P, V (MN-major)
+      constexpr uint32_t IDESC_S = make_idesc(128, 128, 0u, false, false);   // fp16 Q, K (K-major)
+      constexpr uint32_t IDESC_O = make_idesc(128, 64, 0u, false, true);     // fp16 P (TMEM), V MN-major
       const uint32_t sq = smem_u32(smem + ATT_OFF_Q);
       bool ok = mbar_wait(q_full, 0, abort_flag, p.status, 204);
-      // PV of tile j: O[j%2] = P[j%2] * V[stage of j]
+      // O += P(j) V(j): P in TMEM over the S columns, 8 steps of 16 keys (8 columns each)
       auto issue_pv = [&](int j) -> bool {
-        const int pb = j & 1;
-        if (!mbar_wait(&p_full[pb], (j >> 1) & 1u, abort_flag, p.status, 205)) return false;
+        if (!mbar_wait(p_full, j & 1u, abort_flag, p.status, 205)) return false;
         tc_fence_after();
         const int s = j % ATT_STAGES;
-        const uint32_t sp = smem_u32(smem + ATT_OFF_P + pb * ATT_P_BYTES);
         const uint32_t sv = smem_u32(smem + ATT_OFF_V + s * ATT_KV_BYTES);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ad = make_sdesc_sw128(sp + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = make_sdesc_sw128(sv + kk * 2048, 8192, 1024);
-          umma_f16(tmem + 256 + pb * 64, ad, bd, IDESC_O, kk > 0 ? 1u : 0u);
+          umma_f16_tmem_a(TM_O, TM_S + kk * 8, bd, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&o_full[pb]);
+        umma_commit(o_done);
         umma_commit(&kv_empty[s]);
         return true;
       };
       for (int i = 0; ok && i < n_tiles; ++i) {
         const int s = i % ATT_STAGES;
         if (!mbar_wait(&kv_full[s], (i / ATT_STAGES) & 1u, abort_flag, p.status, 206)) { ok = false; break; }
+        // S(i) overwrites the columns P(i-1) lives in: issue PV(i-1) first (in-order pipe)
+        if (i >= 1 && !issue_pv(i - 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t sk = smem_u32(smem + ATT_OFF_K + s * ATT_KV_BYTES);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t ad = make_sdesc_sw128(sq + kk * 32, 16, 1024);
           const uint64_t bd = make_sdesc_sw128(sk + kk * 32, 16, 1024);
-          umma_f16(tmem + (i & 1) * 128, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+          umma_f16(TM_S, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&s_full[i & 1]);
-        if (i >= 1 && !issue_pv(i - 1)) { ok = false; break; }
+        umma_commit(s_full);
       }
       if (ok && n_tiles > 0) issue_pv(n_tiles - 1);
     }
@@ -182,35 +247,27 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const int t0 = qt * 128;
-    const int qi = t0 + r;                         // absolute query position
+    const int qi = t0 + r;                       // absolute query position
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    float m_run = -1e30f, l_run = 0.f, alpha_prev = 1.f;
-    float o_acc[64];
-#pragma unroll
-    for (int d = 0; d < 64; ++d) o_acc[d] = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;
+    int o_waited = -1;                           // last tile whose PV completion we observed
 
-    auto consume_o = [&](int j) -> bool {
+    auto wait_o = [&](int j) -> bool {           // PV(j) complete (warp-uniform)
+      if (j < 0 || o_waited >= j) return true;
       int ok = 1;
-      if (lane == 0) ok = mbar_wait(&o_full[j & 1], (j >> 1) & 1u, abort_flag, p.status, 207) ? 1 : 0;
+      if (lane == 0) ok = mbar_wait(o_done, j & 1u, abort_flag, p.status, 207) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) return false;
-      tc_fence_after();
-      float ot[32];
-      const uint32_t ob = tmem + lane_off + 256 + (j & 1) * 64;
-      tmem_ld32(ob, ot);
-#pragma unroll
-      for (int d = 0; d < 32; ++d) o_acc[d] = o_acc[d] * alpha_prev + ot[d];
-      tmem_ld32(ob + 32, ot);
-#pragma unroll
-      for (int d = 0; d < 32; ++d) o_acc[32 + d] = o_acc[32 + d] * alpha_prev + ot[d];
-      return true;
+      if (ok) {
+        o_waited = j;
+        tc_fence_after();
+      }
+      return ok != 0;
     };
 
     bool ok = true;
     for (int i = 0; i < n_tiles; ++i) {
-      const int sb = i & 1;
       int w_ok = 1;
-      if (lane == 0) w_ok = mbar_wait(&s_full[sb], (i >> 1) & 1u, abort_flag, p.status, 208) ? 1 : 0;
+      if (lane == 0) w_ok = mbar_wait(s_full, i & 1u, abort_flag, p.status, 208) ? 1 : 0;
       w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
       if (!w_ok) { ok = false; break; }
       tc_fence_after();
@@ -218,71 +275,76 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       const int j0 = kt * 128;
       const bool full = (j0 + 127 <= t0) &&
                         (p.is_global || j0 + 127 < p.n_meta || (t0 + 127) - j0 < p.window);
-      const uint32_t sbase = tmem + lane_off + sb * 128;
-      // pass 1: row max of the scaled, masked scores
-      float mx = -1e30f;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(sbase + c * 32, v);
+      float s[128];
+      tmem_ld128(TM_S + lane_off, s);
+      float mx = -INFINITY;
+      if (full) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          float sc = v[e] * p.scale_log2;
-          if (!full) {
-            const int j = j0 + c * 32 + e;
-            const bool vis = (j <= qi) && (p.is_global || j < p.n_meta || qi - j < p.window);
-            sc = vis ? sc : -1e30f;
-          }
-          mx = fmaxf(mx, sc);
+        for (int e = 0; e < 128; ++e) {
+          s[e] *= p.scale_log2;
+          mx = fmaxf(mx, s[e]);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 128; ++e) {
+          const int j = j0 + e;
+          const bool vis = (j <= qi) && (p.is_global || j < p.n_meta || qi - j < p.window);
+          s[e] = vis ? s[e] * p.scale_log2 : -INFINITY;
+          mx = fmaxf(mx, s[e]);
         }
       }
-      const float m_new = fmaxf(m_run, mx);
-      const float alpha = exp2f(m_run - m_new);
-      // pass 2: P = exp2(s - m_new) -> bf16 in 128B-swizzled smem, row sums
+      // running max: rescale O (in TMEM) only when the max grows by more than 2^8
+      float alpha = 1.f;
+      bool resc = false;
+      if (m_run == -INFINITY) {
+        m_run = mx;                               // nothing accumulated for this row yet
+      } else if (mx > m_run + ATT_RESCALE_LOG2) {
+        alpha = exp2f(m_run - mx);
+        m_run = mx;
+        resc = true;
+      }
+      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
       float rs = 0.f;
-      uint8_t* prow = smem + ATT_OFF_P + sb * ATT_P_BYTES + r * 128;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(sbase + c * 32, v);
-        uint32_t pk[16];
+      uint32_t pk[64];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float s0 = v[e] * p.scale_log2, s1 = v[e + 1] * p.scale_log2;
-          if (!full) {
-            const int j = j0 + c * 32 + e;
-            const bool v0 = (j <= qi) && (p.is_global || j < p.n_meta || qi - j < p.window);
-            const bool v1 = (j + 1 <= qi) && (p.is_global || j + 1 < p.n_meta || qi - j - 1 < p.window);
-            s0 = v0 ? s0 : -1e30f;
-            s1 = v1 ? s1 : -1e30f;
-          }
-          const float p0 = exp2f(s0 - m_new), p1 = exp2f(s1 - m_new);
-          rs += p0 + p1;
-          pk[e >> 1] = pack_f16x2(p0, p1);
-        }
-        uint8_t* sub = prow + (c >> 1) * 16384;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int chunk = ((c & 1) * 4 + q) ^ (r & 7);
-          *reinterpret_cast<uint4*>(sub + chunk * 16) =
-              make_uint4(pk[q * 4 + 0], pk[q * 4 + 1], pk[q * 4 + 2], pk[q * 4 + 3]);
-        }
+      for (int e = 0; e < 128; e += 2) {
+        const float p0 = ex2_approx(s[e] - m_use), p1 = ex2_approx(s[e + 1] - m_use);
+        rs += p0 + p1;
+        pk[e >> 1] = pack_f16x2(p0, p1);
       }
-      l_run = l_run * alpha + rs;
-      m_run = m_new;
-      tc_fence_before();
-      fence_proxy_async_smem();
-      mbar_arrive(&p_full[sb]);
-      if (i >= 1 && !consume_o(i - 1)) { ok = false; break; }
-      alpha_prev = alpha;
-    }
-    if (ok && n_tiles > 0 && consume_o(n_tiles - 1) && qi < p.T) {
-      const float inv = 1.f / l_run;
-      float* dst = p.out + ((size_t)b * p.T + qi) * p.ld_out + h * 64;
+      l_run += rs;
+      // rescale O only after P is packed, so the S row is no longer live
+      if (__any_sync(0xffffffffu, resc)) {
+        if (!wait_o(i - 1)) { ok = false; break; }
+        float o[32];
 #pragma unroll
-      for (int d = 0; d < 64; d += 4)
-        *reinterpret_cast<float4*>(dst + d) =
-            make_float4(o_acc[d] * inv, o_acc[d + 1] * inv, o_acc[d + 2] * inv, o_acc[d + 3] * inv);
+        for (int hcol = 0; hcol < 64; hcol += 32) {
+          tmem_ld32(TM_O + lane_off + hcol, o);
+#pragma unroll
+          for (int d = 0; d < 32; ++d) o[d] *= alpha;
+          tmem_st32(TM_O + lane_off + hcol, reinterpret_cast<const uint32_t*>(o));
+        }
+        tmem_wait_st();
+        l_run *= alpha;
+      }
+      // P over the S columns (the tensor core is done with S(i): s_full completed)
+      tmem_st32(TM_S + lane_off, pk);
+      tmem_st32(TM_S + lane_off + 32, pk + 32);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    if (ok && n_tiles > 0 && wait_o(n_tiles - 1)) {
+      float o[64];
+      tmem_ld32(TM_O + lane_off, o);
+      tmem_ld32(TM_O + lane_off + 32, o + 32);
+      if (qi < p.T) {
+        const float inv = 1.f / l_run;
+        float* dst = p.out + ((size_t)b * p.T + qi) * p.ld_out + h * 64;
+#pragma unroll
+        for (int d = 0; d < 64; d += 4)
+          *reinterpret_cast<float4*>(dst + d) = make_float4(o[d] * inv, o[d + 1] * inv, o[d + 2] * inv, o[d + 3] * inv);
+      }
     }
   }
 
@@ -290,7 +352,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, ATT_TMEM_COLS);
   }
 }
 

@@ -257,6 +257,22 @@ __device__ __forceinline__ float ex2_approx(float x) {
 }
 
 __device__ __forceinline__ float softplus_f(float x) { return x > 20.f ? x : log1pf(expf(x)); }
+
+// hardware base-2 logarithm (MUFU), absolute error ~2^-22
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// softplus(x) = log(1 + e^x) from the hardware ex2/lg2: x for x > 15 (the remainder is
+// below 3.1e-7); with u = e^x, log1p(u) = ln2 * log2(1 + u) for u >= 2^-7 (relative error
+// below 3e-5 there), and the series u - u^2/2 + u^3/3 below (error below u^4/4).
+__device__ __forceinline__ float softplus_fast(float x) {
+  if (x > 15.f) return x;
+  const float u = ex2_approx(x * 1.4426950408889634f);
+  if (u < 0.0078125f) return u * (1.f - u * (0.5f - u * 0.33333334f));
+  return lg2_approx(1.f + u) * 0.6931471805599453f;
+}
 __device__ __forceinline__ float silu_f(float x) { return x / (1.f + expf(-x)); }
 
 }  // namespace hymba

@@ -315,20 +315,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
               for (int e = 0; e < nv; ++e) dst[e] = __float2bfloat16_rn(v[e]);
             }
           } else if (p.mode == EPI_ATOMIC_F32) {
+            // vector fp32 reductions (ld_out and n_valid are multiples of 4)
             float* dst = reinterpret_cast<float*>(p.out) + orow * p.ld_out + gc;
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (gc + e < p.n_valid) atomicAdd(dst + e, v[e]);
+            for (int e = 0; e < 32; e += 4)
+              if (gc + e < p.n_valid)
+                atomicAdd(reinterpret_cast<float4*>(dst + e), make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]));
           } else if (p.mode == EPI_SOFTPLUS) {
             float* dst = reinterpret_cast<float*>(p.out) + orow * p.ld_out + gc;
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-              if (gc + e < p.n_valid) dst[e] = softplus_f(v[e] + p.bias[gc + e]);
+              if (gc + e < p.n_valid) dst[e] = softplus_fast(v[e] + p.bias[gc + e]);
           } else {  // EPI_SOFTPLUS_T: lanes hold consecutive rows -> coalesced along time
             float* dst = reinterpret_cast<float*>(p.out) + ((size_t)b1 * p.N + gc) * p.T_out + rr;
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-              if (gc + e < p.n_valid) dst[(size_t)e * p.T_out] = softplus_f(v[e] + p.bias[gc + e]);
+              if (gc + e < p.n_valid) dst[(size_t)e * p.T_out] = softplus_fast(v[e] + p.bias[gc + e]);
           }
         }
       }

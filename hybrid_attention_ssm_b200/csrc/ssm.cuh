@@ -180,8 +180,10 @@ __global__ void __launch_bounds__(SCAN_THREADS)
     }
     cp_async_commit();
     const ScanStage& S = st[k % SCAN_NST];
-#pragma unroll 1
-    for (int tt = 0; tt < SCAN_TC; tt += 8) {
+    // Software pipeline over the 8 blocks of 8 steps: block q's recurrence runs while the
+    // state-sum of block q-1 goes through its shuffles, so the two latency chains overlap.
+    float vprev[8];
+    auto block_inputs = [&](int tt, float* dv, float* xv, float* bv, float* cv) {
       const uint4 xr = *reinterpret_cast<const uint4*>(&S.x[cl][tt]);
       const __nv_bfloat16* xh = reinterpret_cast<const __nv_bfloat16*>(&xr);
       const float4 d0 = *reinterpret_cast<const float4*>(&S.d[cl][tt]);
@@ -190,18 +192,28 @@ __global__ void __launch_bounds__(SCAN_THREADS)
       const float4 b1 = *reinterpret_cast<const float4*>(&S.bcT[s][tt + 4]);
       const float4 e0 = *reinterpret_cast<const float4*>(&S.bcT[16 + s][tt]);
       const float4 e1 = *reinterpret_cast<const float4*>(&S.bcT[16 + s][tt + 4]);
-      const float dv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-      const float cv[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
-      float v[8];
+      dv[0] = d0.x; dv[1] = d0.y; dv[2] = d0.z; dv[3] = d0.w; dv[4] = d1.x; dv[5] = d1.y; dv[6] = d1.z; dv[7] = d1.w;
+      bv[0] = b0.x; bv[1] = b0.y; bv[2] = b0.z; bv[3] = b0.w; bv[4] = b1.x; bv[5] = b1.y; bv[6] = b1.z; bv[7] = b1.w;
+      cv[0] = e0.x; cv[1] = e0.y; cv[2] = e0.z; cv[3] = e0.w; cv[4] = e1.x; cv[5] = e1.y; cv[6] = e1.z; cv[7] = e1.w;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) xv[u] = __bfloat162float(xh[u]);
+    };
+    auto recur = [&](const float* dv, const float* xv, const float* bv, const float* cv, float* v) {
+      float a[8], q[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const float a = ex2_approx(dv[u] * A2);
-        h = fmaf(a, h, dv[u] * __bfloat162float(xh[u]) * bv[u]);
+        a[u] = ex2_approx(dv[u] * A2);
+        q[u] = dv[u] * xv[u] * bv[u];
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        h = fmaf(a[u], h, q[u]);
         v[u] = cv[u] * h;
       }
-      // reduce-scatter of v[0..7] over the 16 state lanes: lane l ends with the full sum
-      // of step my_step (lanes l and l^1 hold the same step)
+    };
+    // reduce-scatter of v[0..7] over the 16 state lanes: lane l ends with the full sum of
+    // step my_step (lanes l and l^1 hold the same step)
+    auto reduce_store = [&](const float* v, int tt) {
       const bool q3 = l & 8, q2 = l & 4, q1 = l & 2;
       float w4[4];
 #pragma unroll
@@ -225,7 +237,22 @@ __global__ void __launch_bounds__(SCAN_THREADS)
       }
       w1 += __shfl_xor_sync(0xffffffffu, w1, 1);
       if ((l & 1) == 0) ys[tt + my_step][cl] = __float2bfloat16_rn(w1);
+    };
+    {
+      float dv[8], xv[8], bv[8], cv[8];
+      block_inputs(0, dv, xv, bv, cv);
+      recur(dv, xv, bv, cv, vprev);
     }
+#pragma unroll 1
+    for (int tt = 8; tt < SCAN_TC; tt += 8) {
+      float dv[8], xv[8], bv[8], cv[8], v[8];
+      block_inputs(tt, dv, xv, bv, cv);
+      recur(dv, xv, bv, cv, v);
+      reduce_store(vprev, tt - 8);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) vprev[u] = v[u];
+    }
+    reduce_store(vprev, SCAN_TC - 8);
     if (kn < n_chunks) store_bc(kn);
     __syncthreads();
     // flush y rows of this chunk: 64 rows x 16 B
