@@ -54,7 +54,7 @@ struct GemmParams {
   const float* bias;
   int nseg;
   Segment seg[5];
-  double rope_theta[32];    // base^(-2j/64), j < 32
+  const float2* rope_tab;   // [positions][32] (cos, sin) of pos * base^(-2j/64)
   DevStatus* status;
 };
 
@@ -70,18 +70,50 @@ struct GemmSmem {
   static constexpr int TOTAL = BAR_OFFSET + 256 + 1024;   // + barriers + alignment slack
 };
 
-__device__ __forceinline__ void rope_pair_rotate(float* v, int pos, const double* theta) {
-  // v[0..31] are the first halves x_j, v[32..63] the second halves x_{j+32}.
+// Rotate the pairs (v[j], v[j+32]) of one 64-wide head by the angles of position pos.
+__device__ __forceinline__ void rope_pair_rotate(float* v, const float2* __restrict__ tab_row) {
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    double a = (double)pos * theta[j];
-    a -= 6.283185307179586 * rint(a * 0.15915494309189535);
-    float s, c;
-    sincosf((float)a, &s, &c);
-    const float x1 = v[j], x2 = v[j + 32];
-    v[j] = x1 * c - x2 * s;
-    v[j + 32] = x2 * c + x1 * s;
+  for (int j = 0; j < 32; j += 2) {
+    const float4 cs = *reinterpret_cast<const float4*>(tab_row + j);   // (c_j, s_j, c_j+1, s_j+1)
+    float x1 = v[j], x2 = v[j + 32];
+    v[j] = x1 * cs.x - x2 * cs.y;
+    v[j + 32] = x2 * cs.x + x1 * cs.y;
+    x1 = v[j + 1], x2 = v[j + 33];
+    v[j + 1] = x1 * cs.z - x2 * cs.w;
+    v[j + 33] = x2 * cs.z + x1 * cs.w;
   }
+}
+
+// tcgen05.ld of 32 columns without waiting, and the wait that orders later uses of the
+// registers after the load (every register is an operand of the wait).
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t* r) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]),
+        "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]),
+        "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
+        "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+}
+
+// Branch-free softplus for the vectorised epilogue (same formula as softplus_fast).
+__device__ __forceinline__ float softplus_sel(float x) {
+  const float u = ex2_approx(fminf(x, 15.f) * 1.4426950408889634f);
+  const float small = u * (1.f - u * (0.5f - u * 0.33333334f));
+  const float big = lg2_approx(1.f + u) * 0.6931471805599453f;
+  return x > 15.f ? x : (u < 0.0078125f ? small : big);
 }
 
 // element types of both operands: bf16, fp16 (kind::f16) or fp32 read as tf32 (kind::tf32)
@@ -235,20 +267,31 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const bool row_ok = src0 ? (rr < p.rows0) : (rr < p.rows1);
       const int col_base = n * BN;
 
-      if (p.mode == EPI_PROJ) {
+      if (p.mode == EPI_PROJ || p.mode == EPI_SWIGLU) {
+        // 64-column chunks: both 32-column halves are loaded before one wait
+        const size_t orow = (size_t)b1 * p.rows1 + rr;
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 64) {
-          float v[64];
-          tmem_ld32(tbase + c0, v);
-          tmem_ld32(tbase + c0 + 32, v + 32);
+          uint32_t r[64];
+          tmem_ld32_async(tbase + c0, r);
+          tmem_ld32_async(tbase + c0 + 32, r + 32);
+          tmem_wait_ld_regs(r);
+          tmem_wait_ld_regs(r + 32);
+          float* v = reinterpret_cast<float*>(r);
           const int gc = col_base + c0;
           if (!row_ok || gc >= p.N) continue;
+          if (p.mode == EPI_SWIGLU) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = silu_f(v[e]) * v[e + 32];
+            store_bf16_row(reinterpret_cast<__nv_bfloat16*>(p.out) + orow * p.ld_out + gc / 2, v, 32);
+            continue;
+          }
           int si = 0;
 #pragma unroll 1
           while (si < p.nseg - 1 && gc >= p.seg[si].col_end) ++si;
-          const Segment sg = p.seg[si];
+          const Segment& sg = p.seg[si];
           const int pos = src0 ? rr : p.row_off1 + rr;
-          if (sg.rope) rope_pair_rotate(v, pos, p.rope_theta);
+          if (sg.rope) rope_pair_rotate(v, p.rope_tab + (size_t)pos * 32);
           __nv_bfloat16* base = reinterpret_cast<__nv_bfloat16*>(sg.ptr) + (gc - sg.col_begin);
           const int b_lo = src0 ? 0 : b1, b_hi = src0 ? p.out_batches : b1 + 1;
           for (int b = b_lo; b < b_hi; ++b) {
@@ -257,63 +300,55 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             else store_bf16_row(dst, v, 64);
           }
         }
-      } else if (p.mode == EPI_BF16_T || p.mode == EPI_ATOMIC_F32_T || p.mode == EPI_F32_T) {
-        // accumulator row = output column (weight row), accumulator column = output row
-#pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 32) {
-          float v[32];
-          tmem_ld32(tbase + c0, v);
-          if (!row_ok || rr >= p.m_valid) continue;
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int orow = col_base + c0 + e;
-            if (orow < p.n_valid) {
-              if (p.mode == EPI_BF16_T)
-                reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)orow * p.ld_out + rr] = __float2bfloat16_rn(v[e]);
-              else if (p.mode == EPI_F32_T)
-                reinterpret_cast<float*>(p.out)[(size_t)orow * p.ld_out + rr] = v[e];
-              else
-                atomicAdd(reinterpret_cast<float*>(p.out) + (size_t)orow * p.ld_out + rr, v[e]);
-            }
-          }
-        }
-      } else if (p.mode == EPI_SWIGLU) {
-        // B rows interleave 32 gate rows and 32 up rows; each 64-column chunk gives 32
-        // outputs SiLU(gate) * up at output columns (col_base + c0) / 2.
-        const size_t orow = (size_t)b1 * p.rows1 + rr;
-#pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 64) {
-          float v[64];
-          tmem_ld32(tbase + c0, v);
-          tmem_ld32(tbase + c0 + 32, v + 32);
-          const int gc = col_base + c0;
-          if (!row_ok || gc >= p.N) continue;
-#pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = silu_f(v[e]) * v[e + 32];
-          store_bf16_row(reinterpret_cast<__nv_bfloat16*>(p.out) + orow * p.ld_out + gc / 2, v, 32);
-        }
       } else {
+        // 32-column chunks, the next chunk's TMEM load in flight while this one is stored
         const size_t orow = (size_t)b1 * p.rows1 + rr;
-#pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 32) {
-          float v[32];
-          tmem_ld32(tbase + c0, v);
+        auto process = [&](uint32_t* r, int c0) {
+          float* v = reinterpret_cast<float*>(r);
           const int gc = col_base + c0;
-          if (!row_ok || gc >= p.n_valid) continue;
+          if (p.mode == EPI_BF16_T || p.mode == EPI_ATOMIC_F32_T || p.mode == EPI_F32_T) {
+            // accumulator row = output column (weight row), accumulator column = output row
+            if (!row_ok || rr >= p.m_valid) return;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int orow_t = gc + e;
+              if (orow_t < p.n_valid) {
+                if (p.mode == EPI_BF16_T)
+                  reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)orow_t * p.ld_out + rr] = __float2bfloat16_rn(v[e]);
+                else if (p.mode == EPI_F32_T)
+                  reinterpret_cast<float*>(p.out)[(size_t)orow_t * p.ld_out + rr] = v[e];
+                else
+                  atomicAdd(reinterpret_cast<float*>(p.out) + (size_t)orow_t * p.ld_out + rr, v[e]);
+              }
+            }
+            return;
+          }
+          if (!row_ok || gc >= p.n_valid) return;
+          const bool whole = gc + 32 <= p.n_valid;
           if (p.mode == EPI_BF16) {
             if (p.residual != nullptr) {
               const __nv_bfloat16* res = p.residual + orow * p.ld_res + gc;
+              if (whole) {
 #pragma unroll
-              for (int e = 0; e < 32; ++e)
-                if (gc + e < p.n_valid) v[e] += __bfloat162float(res[e]);
+                for (int e = 0; e < 32; e += 8) {
+                  float f[8];
+                  const uint4 raw = *reinterpret_cast<const uint4*>(res + e);
+                  const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+                  for (int k = 0; k < 8; ++k) f[k] = __bfloat162float(hv[k]);
+#pragma unroll
+                  for (int k = 0; k < 8; ++k) v[e + k] += f[k];
+                }
+              } else {
+                for (int e = 0; e < 32; ++e)
+                  if (gc + e < p.n_valid) v[e] += __bfloat162float(res[e]);
+              }
             }
             __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + orow * p.ld_out + gc;
-            const int nv = min(32, p.n_valid - gc);
-            if (nv == 32) {
-              store_bf16_row(dst, v, 32);
-            } else {
-              for (int e = 0; e < nv; ++e) dst[e] = __float2bfloat16_rn(v[e]);
-            }
+            if (whole) store_bf16_row(dst, v, 32);
+            else
+              for (int e = 0; e < 32; ++e)
+                if (gc + e < p.n_valid) dst[e] = __float2bfloat16_rn(v[e]);
           } else if (p.mode == EPI_ATOMIC_F32) {
             // vector fp32 reductions (ld_out and n_valid are multiples of 4)
             float* dst = reinterpret_cast<float*>(p.out) + orow * p.ld_out + gc;
@@ -321,16 +356,56 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             for (int e = 0; e < 32; e += 4)
               if (gc + e < p.n_valid)
                 atomicAdd(reinterpret_cast<float4*>(dst + e), make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]));
-          } else if (p.mode == EPI_SOFTPLUS) {
-            float* dst = reinterpret_cast<float*>(p.out) + orow * p.ld_out + gc;
+          } else {
+            float bb[32];
+            if (whole) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (gc + e < p.n_valid) dst[e] = softplus_fast(v[e] + p.bias[gc + e]);
-          } else {  // EPI_SOFTPLUS_T: lanes hold consecutive rows -> coalesced along time
-            float* dst = reinterpret_cast<float*>(p.out) + ((size_t)b1 * p.N + gc) * p.T_out + rr;
+              for (int e = 0; e < 32; e += 4) {
+                const float4 t = *reinterpret_cast<const float4*>(p.bias + gc + e);
+                bb[e] = t.x; bb[e + 1] = t.y; bb[e + 2] = t.z; bb[e + 3] = t.w;
+              }
+            } else {
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (gc + e < p.n_valid) dst[(size_t)e * p.T_out] = softplus_fast(v[e] + p.bias[gc + e]);
+              for (int e = 0; e < 32; ++e) bb[e] = (gc + e < p.n_valid) ? p.bias[gc + e] : 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = softplus_sel(v[e] + bb[e]);
+            if (p.mode == EPI_SOFTPLUS) {
+              float* dst = reinterpret_cast<float*>(p.out) + orow * p.ld_out + gc;
+              if (whole) {
+#pragma unroll
+                for (int e = 0; e < 32; e += 4)
+                  *reinterpret_cast<float4*>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+              } else {
+                for (int e = 0; e < 32; ++e)
+                  if (gc + e < p.n_valid) dst[e] = v[e];
+              }
+            } else {  // EPI_SOFTPLUS_T: lanes hold consecutive rows -> coalesced along time
+              float* dst = reinterpret_cast<float*>(p.out) + ((size_t)b1 * p.N + gc) * p.T_out + rr;
+              if (whole) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) dst[(size_t)e * p.T_out] = v[e];
+              } else {
+                for (int e = 0; e < 32; ++e)
+                  if (gc + e < p.n_valid) dst[(size_t)e * p.T_out] = v[e];
+              }
+            }
+          }
+        };
+        uint32_t ra[32], rb[32];
+        tmem_ld32_async(tbase, ra);
+        tmem_wait_ld_regs(ra);
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 64) {
+          const bool has_b = c0 + 32 < BN;
+          if (has_b) tmem_ld32_async(tbase + c0 + 32, rb);
+          process(ra, c0);
+          if (has_b) {
+            tmem_wait_ld_regs(rb);
+            const bool has_a = c0 + 64 < BN;
+            if (has_a) tmem_ld32_async(tbase + c0 + 64, ra);
+            process(rb, c0 + 32);
+            if (has_a) tmem_wait_ld_regs(ra);
           }
         }
       }

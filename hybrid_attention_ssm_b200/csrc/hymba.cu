@@ -262,7 +262,10 @@ int check_cfg(const hymba_layer_cfg* c) {
   if (c->d_state != 16) return fail(HYMBA_ERR_UNSUPPORTED, "d_state %d (only 16)", c->d_state);
   if (c->d_conv != 4) return fail(HYMBA_ERR_UNSUPPORTED, "d_conv %d (only 4)", c->d_conv);
   if (c->d_model < 8 || c->d_model % 8) return fail(HYMBA_ERR_UNSUPPORTED, "d_model %d (multiple of 8)", c->d_model);
-  if (c->d_inner < 64 || c->d_inner % 64) return fail(HYMBA_ERR_UNSUPPORTED, "d_inner %d (multiple of 64)", c->d_inner);
+  if (c->d_inner < 64 || c->d_inner % 64 || c->d_inner > 8 * 128 * NORM_MAXY)
+    return fail(HYMBA_ERR_UNSUPPORTED, "d_inner %d (multiple of 64, at most %d)", c->d_inner, 8 * 128 * NORM_MAXY);
+  if (c->n_q_heads * c->head_dim > 8 * 128 * NORM_MAXO)
+    return fail(HYMBA_ERR_UNSUPPORTED, "n_q_heads * head_dim above %d", 8 * 128 * NORM_MAXO);
   if (c->n_q_heads < 1 || c->n_kv_heads < 1 || c->n_q_heads % c->n_kv_heads)
     return fail(HYMBA_ERR_UNSUPPORTED, "heads %d/%d", c->n_q_heads, c->n_kv_heads);
   if (c->n_q_heads / c->n_kv_heads > DEC_MAXG)
@@ -296,7 +299,7 @@ Dims dims_of(const hymba_layer_cfg* c) {
 }
 
 struct PrefillWs {
-  size_t q, xz, xc, xcT, xbc, dT, y, o, u, sstate, cstate, total;
+  size_t q, xz, xc, xcT, xbc, dT, y, o, u, sstate, cstate, rope, total;
   int T, Tp;
 };
 PrefillWs prefill_layout(const Dims& m, int B, int n_tokens, int x_has_meta) {
@@ -317,6 +320,7 @@ PrefillWs prefill_layout(const Dims& m, int B, int n_tokens, int x_has_meta) {
   w.u = take(rows * m.uw * 2);
   w.sstate = take((size_t)B * m.Di * 16 * 4);
   w.cstate = take((size_t)B * m.Di * 3 * 4);
+  w.rope = take((size_t)w.T * 32 * 8);
   w.total = off;
   return w;
 }
@@ -570,6 +574,16 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
   const size_t rows = (size_t)B * T;
   const int Lmax = kv->max_tokens;
 
+  // 0. RoPE angle table for the T positions
+  {
+    RopeThetas th;
+    fill_rope_theta(th.t, cfg->rope_base);
+    const int n = T * 32;
+    prof_begin("rope_table", st);
+    rope_table_kernel<<<cdiv(n, 256), 256, 0, st>>>(reinterpret_cast<float2*>(wsb + L.rope), T, th);
+    prof_end(st);
+    HY_CUDA(cudaGetLastError());
+  }
   // 1. in_proj with RoPE on Q/K, scattering Q, K, V, x|z
   {
     GemmCall c;
@@ -596,13 +610,14 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     }
     c.p.seg[ns++] = Segment{m.xz_off, m.xz_off + 2 * m.Di, bf(L.xz), (long long)T * 2 * m.Di, 2 * m.Di, 0, 0};
     c.p.nseg = ns;
-    fill_rope_theta(c.p.rope_theta, cfg->rope_base);
+    c.p.rope_tab = reinterpret_cast<const float2*>(wsb + L.rope);
     HY_TRY(run_gemm(c, *dev, st));
   }
   // 2. conv1d + SiLU (writes xc, xcT and the conv state)
   float* cstate = conv_state_out != nullptr ? conv_state_out : f32(L.cstate);
   {
-    dim3 grid(cdiv(m.Di, CONV_CC), cdiv(T, CONV_TC), B);
+    const int threads = (m.Di / 2) * cdiv(T, CONV_RUN);
+    dim3 grid(cdiv(threads, 256), B);
     prof_begin("conv1d_silu", st);
     conv1d_silu_kernel<<<grid, 256, 0, st>>>(bf(L.xz), 2 * m.Di, w->conv_w, w->conv_b, bf(L.xc), bf(L.xcT), cstate,
                                               T, L.Tp, m.Di);
@@ -692,9 +707,9 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
   // 7. per-branch RMSNorm, gate, beta, average
   {
     prof_begin("norm_avg", st);
-    branch_norm_avg_kernel<__nv_bfloat16><<<(unsigned)rows, 256, 0, st>>>(
+    branch_norm_avg_kernel<__nv_bfloat16><<<cdiv(rows, NORM_ROWS), 128 * NORM_ROWS, 0, st>>>(
         f32(L.o), m.qw, m.qw, bf(L.y), m.Di, bf(L.xz) + m.Di, 2 * m.Di, m.Di, w->g_attn, w->g_ssm, cfg->norm_eps,
-        h16(L.u), m.uw);
+        h16(L.u), m.uw, (int)rows);
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
@@ -859,8 +874,8 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
   // 6. norm + average (y already gated)
   {
     prof_begin("decode_norm_avg", st);
-    branch_norm_avg_kernel<float><<<B, 256, 0, st>>>(f32(L.o), m.qw, m.qw, f32(L.y), m.Di, nullptr, 0, m.Di,
-                                                     w->g_attn, w->g_ssm, cfg->norm_eps, h16(L.u), m.uw);
+    branch_norm_avg_kernel<float><<<cdiv(B, NORM_ROWS), 128 * NORM_ROWS, 0, st>>>(
+        f32(L.o), m.qw, m.qw, f32(L.y), m.Di, nullptr, 0, m.Di, w->g_attn, w->g_ssm, cfg->norm_eps, h16(L.u), m.uw, B);
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }

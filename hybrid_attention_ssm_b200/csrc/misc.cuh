@@ -49,60 +49,98 @@ __device__ __forceinline__ void load8(const float* p, float* f) {
 __device__ __forceinline__ void load8(const __nv_bfloat16* p, float* f) {
   unpack8(*reinterpret_cast<const uint4*>(p), f);
 }
+constexpr int NORM_ROWS = 2;          // rows per CTA, 128 threads each
+constexpr int NORM_MAXO = 2;          // 8-element chunks of O per thread (attn_w <= 2048)
+constexpr int NORM_MAXY = 4;          // 8-element chunks of y per thread (d_inner <= 4096)
+
 template <typename YT>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(128 * NORM_ROWS)
     branch_norm_avg_kernel(const float* __restrict__ O, int ld_o, int attn_w, const YT* __restrict__ y, int ld_y,
                            const __nv_bfloat16* __restrict__ z, int ld_z, int di, const float* __restrict__ g_attn,
-                           const float* __restrict__ g_ssm, float eps, __half* __restrict__ u, int ld_u) {
-  __shared__ float red[32];
-  const size_t row = blockIdx.x;
+                           const float* __restrict__ g_ssm, float eps, __half* __restrict__ u, int ld_u, int rows) {
+  __shared__ float red[NORM_ROWS][4][2];
+  const int sub = threadIdx.x >> 7;                 // row within the CTA
+  const int t = threadIdx.x & 127;
+  const int wr = t >> 5, ln = t & 31;
+  const size_t row = (size_t)blockIdx.x * NORM_ROWS + sub;
+  const bool live = row < (size_t)rows;
   const float* o_r = O + row * ld_o;
   const YT* y_r = y + row * ld_y;
   const __nv_bfloat16* z_r = z != nullptr ? z + row * ld_z : nullptr;
   __half* u_r = u + row * ld_u;
+  // the whole row in registers: every load is issued before the first use
+  float fo[NORM_MAXO][8], fy[NORM_MAXY][8];
   float sa = 0.f, ss = 0.f;
-  for (int c = threadIdx.x * 8; c < attn_w; c += 256 * 8) {
-    float f[8];
-    load8(o_r + c, f);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) sa += f[e] * f[e];
+  for (int k = 0; k < NORM_MAXO; ++k) {
+    const int c = (t + k * 128) * 8;
+    if (live && c < attn_w) load8(o_r + c, fo[k]);
   }
-  for (int c = threadIdx.x * 8; c < di; c += 256 * 8) {
-    float fy[8], fz[8];
-    load8(y_r + c, fy);
-    if (z != nullptr) {
-      unpack8(*reinterpret_cast<const uint4*>(z_r + c), fz);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) fy[e] *= silu_f(fz[e]);
+  for (int k = 0; k < NORM_MAXY; ++k) {
+    const int c = (t + k * 128) * 8;
+    if (live && c < di) {
+      load8(y_r + c, fy[k]);
+      if (z != nullptr) {
+        float fz[8];
+        unpack8(*reinterpret_cast<const uint4*>(z_r + c), fz);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) fy[k][e] *= silu_f(fz[e]);
+      }
     }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) ss += fy[e] * fy[e];
   }
-  sa = block_sum_256(sa, red);
-  ss = block_sum_256(ss, red);
+#pragma unroll
+  for (int k = 0; k < NORM_MAXO; ++k) {
+    const int c = (t + k * 128) * 8;
+    if (live && c < attn_w)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sa += fo[k][e] * fo[k][e];
+  }
+#pragma unroll
+  for (int k = 0; k < NORM_MAXY; ++k) {
+    const int c = (t + k * 128) * 8;
+    if (live && c < di)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss += fy[k][e] * fy[k][e];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sa += __shfl_xor_sync(0xffffffffu, sa, o);
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  }
+  if (ln == 0) {
+    red[sub][wr][0] = sa;
+    red[sub][wr][1] = ss;
+  }
+  __syncthreads();
+  sa = red[sub][0][0] + red[sub][1][0] + red[sub][2][0] + red[sub][3][0];
+  ss = red[sub][0][1] + red[sub][1][1] + red[sub][2][1] + red[sub][3][1];
+  if (!live) return;
   const float ra = 0.5f / sqrtf(sa / (float)attn_w + eps);
   const float rs = 0.5f / sqrtf(ss / (float)di + eps);
-  for (int c = threadIdx.x * 8; c < attn_w; c += 256 * 8) {
-    float f[8];
-    load8(o_r + c, f);
-    uint32_t pk[4];
 #pragma unroll
-    for (int e = 0; e < 8; e += 2)
-      pk[e / 2] = pack_f16x2(f[e] * ra * g_attn[c + e], f[e + 1] * ra * g_attn[c + e + 1]);
-    *reinterpret_cast<uint4*>(u_r + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-  }
-  for (int c = threadIdx.x * 8; c < di; c += 256 * 8) {
-    float fy[8], fz[8];
-    load8(y_r + c, fy);
-    if (z != nullptr) {
-      unpack8(*reinterpret_cast<const uint4*>(z_r + c), fz);
+  for (int k = 0; k < NORM_MAXO; ++k) {
+    const int c = (t + k * 128) * 8;
+    if (c < attn_w) {
+      float g[8];
+      load8(g_attn + c, g);
+      uint32_t pk[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) fy[e] *= silu_f(fz[e]);
+      for (int e = 0; e < 8; e += 2) pk[e / 2] = pack_f16x2(fo[k][e] * ra * g[e], fo[k][e + 1] * ra * g[e + 1]);
+      *reinterpret_cast<uint4*>(u_r + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
-    uint32_t pk[4];
+  }
 #pragma unroll
-    for (int e = 0; e < 8; e += 2) pk[e / 2] = pack_f16x2(fy[e] * rs * g_ssm[c + e], fy[e + 1] * rs * g_ssm[c + e + 1]);
-    *reinterpret_cast<uint4*>(u_r + attn_w + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  for (int k = 0; k < NORM_MAXY; ++k) {
+    const int c = (t + k * 128) * 8;
+    if (c < di) {
+      float g[8];
+      load8(g_ssm + c, g);
+      uint32_t pk[4];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) pk[e / 2] = pack_f16x2(fy[k][e] * rs * g[e], fy[k][e + 1] * rs * g[e + 1]);
+      *reinterpret_cast<uint4*>(u_r + attn_w + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
   }
 }
 
@@ -421,6 +459,22 @@ __global__ void __launch_bounds__(256)
     const float zz = proj[(size_t)b * ld_proj + off_z + c];
     y[(size_t)b * Di + c] = yv * silu_f(zz);
   }
+}
+
+// RoPE angles: tab[pos][j] = (cos, sin) of pos * base^(-2j/64), the angle reduced mod 2*pi
+// in double precision before the fp32 sincos.
+struct RopeThetas {
+  double t[32];
+};
+__global__ void rope_table_kernel(float2* __restrict__ tab, int n_pos, const __grid_constant__ RopeThetas th) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n_pos * 32) return;
+  const int pos = i >> 5, j = i & 31;
+  double a = (double)pos * th.t[j];
+  a -= 6.283185307179586 * rint(a * 0.15915494309189535);
+  float s, c;
+  sincosf((float)a, &s, &c);
+  tab[i] = make_float2(c, s);
 }
 
 // out[r, :] = x[r, :] / sqrt(mean(x[r, :]^2) + eps) * gain  (one row per CTA, 256 threads)

@@ -12,69 +12,81 @@ namespace hymba {
 //   state  [B, Di, 3]  fp32: the last 3 inputs x[T-3..T-1] (zero before the start)
 // CTA: 64 channels x 64 time steps, 256 threads.
 // ----------------------------------------------------------------------------------------
-constexpr int CONV_TC = 64, CONV_CC = 64, CONV_K = 4;
+constexpr int CONV_K = 4;
+constexpr int CONV_RUN = 8;      // time steps per thread
 
+// Thread = (channel pair, run of 8 time steps): the 3-step history stays in registers,
+// loads and row-major stores are 4 bytes per lane (128 B per warp), the time-major store
+// is 16 contiguous bytes per channel.
 __global__ void __launch_bounds__(256)
     conv1d_silu_kernel(const __nv_bfloat16* __restrict__ x, int ld_x, const float* __restrict__ w,
                        const float* __restrict__ bias, __nv_bfloat16* __restrict__ xc,
                        __nv_bfloat16* __restrict__ xcT, float* __restrict__ state, int T, int Tp, int Di) {
-  __shared__ __align__(16) float xs[CONV_TC + CONV_K - 1][CONV_CC + 1];
-  __shared__ __align__(16) __nv_bfloat16 ot[CONV_CC][CONV_TC + 8];
-  const int c0 = blockIdx.x * CONV_CC;
-  const int t0 = blockIdx.y * CONV_TC;
-  const int b = blockIdx.z;
-  const int tid = threadIdx.x;
-  // load x[t0-3 .. t0+63][c0 .. c0+63] (zero outside [0, T))
-  for (int i = tid; i < (CONV_TC + CONV_K - 1) * (CONV_CC / 8); i += 256) {
-    const int rr = i / (CONV_CC / 8), cv = (i % (CONV_CC / 8)) * 8;
-    const int t = t0 - (CONV_K - 1) + rr;
-    float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    if (t >= 0 && t < T && c0 + cv < Di) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(x + ((size_t)b * T + t) * ld_x + c0 + cv);
-      const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&raw);
+  const int pairs = Di >> 1;
+  const int gid = blockIdx.x * blockDim.x + threadIdx.x;
+  const int cp = gid % pairs;
+  const int run = gid / pairs;
+  const int b = blockIdx.y;
+  const int t0 = run * CONV_RUN;
+  if (t0 >= T) return;
+  const int c = cp * 2;
+  const float4 w0 = *reinterpret_cast<const float4*>(w + (size_t)c * 4);
+  const float4 w1 = *reinterpret_cast<const float4*>(w + (size_t)(c + 1) * 4);
+  const float b0 = bias[c], b1 = bias[c + 1];
+  const __nv_bfloat16* xb = x + (size_t)b * T * ld_x + c;
+  float h0[3], h1[3];          // x[t-3], x[t-2], x[t-1] of both channels
 #pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = __bfloat162float(hv[e]);
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) xs[rr][cv + e] = v[e];
+  for (int k = 0; k < 3; ++k) {
+    const int t = t0 - 3 + k;
+    float2 f = make_float2(0.f, 0.f);
+    if (t >= 0) f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(xb + (size_t)t * ld_x));
+    h0[k] = f.x;
+    h1[k] = f.y;
   }
-  __syncthreads();
-  // compute: thread -> channel (tid % 64), time rows (tid / 64) + 4k
-  const int cl = tid & 63;
-  const int c = c0 + cl;
-  float wk[CONV_K], bc = 0.f;
+  const int n = min(CONV_RUN, T - t0);
+  float2 xv[CONV_RUN];
 #pragma unroll
-  for (int k = 0; k < CONV_K; ++k) wk[k] = c < Di ? w[c * CONV_K + k] : 0.f;
-  if (c < Di) bc = bias[c];
-  for (int tl = tid >> 6; tl < CONV_TC; tl += 4) {
-    float acc = bc;
+  for (int i = 0; i < CONV_RUN; ++i)
+    if (i < n) xv[i] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(xb + (size_t)(t0 + i) * ld_x));
+  __align__(16) __nv_bfloat16 o0[CONV_RUN], o1[CONV_RUN];
 #pragma unroll
-    for (int k = 0; k < CONV_K; ++k) acc += wk[k] * xs[tl + k][cl];
-    const float y = acc / (1.f + __expf(-acc));
-    const __nv_bfloat16 yb = __float2bfloat16_rn(y);
-    ot[cl][tl] = yb;
-    const int t = t0 + tl;
-    if (t < T && c < Di) xc[((size_t)b * T + t) * Di + c] = yb;
-  }
-  __syncthreads();
-  // time-major store: row = channel, 64 contiguous time steps (8 x 16 B)
-  for (int i = tid; i < CONV_CC * (CONV_TC / 8); i += 256) {
-    const int ch = i / (CONV_TC / 8), tv = (i % (CONV_TC / 8)) * 8;
-    const int cc = c0 + ch, t = t0 + tv;
-    if (cc >= Di || t >= T) continue;
-    __nv_bfloat16* dst = xcT + ((size_t)b * Di + cc) * Tp + t;
-    if (t + 8 <= T) {
-      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(&ot[ch][tv]);
+  for (int i = 0; i < CONV_RUN; ++i) {
+    if (i < n) {
+      const float a0 = b0 + w0.x * h0[0] + w0.y * h0[1] + w0.z * h0[2] + w0.w * xv[i].x;
+      const float a1 = b1 + w1.x * h1[0] + w1.y * h1[1] + w1.z * h1[2] + w1.w * xv[i].y;
+      h0[0] = h0[1]; h0[1] = h0[2]; h0[2] = xv[i].x;
+      h1[0] = h1[1]; h1[1] = h1[2]; h1[2] = xv[i].y;
+      const __nv_bfloat162 y2 = __floats2bfloat162_rn(silu_f(a0), silu_f(a1));
+      *reinterpret_cast<__nv_bfloat162*>(xc + ((size_t)b * T + t0 + i) * Di + c) = y2;
+      o0[i] = y2.x;
+      o1[i] = y2.y;
     } else {
-      for (int e = 0; e < 8 && t + e < T; ++e) dst[e] = ot[ch][tv + e];
+      o0[i] = __float2bfloat16_rn(0.f);
+      o1[i] = __float2bfloat16_rn(0.f);
     }
   }
-  // conv state: the last 3 inputs (zero when T < 3)
-  if (t0 <= T - 1 && T - 1 < t0 + CONV_TC && tid < CONV_CC && c0 + tid < Di) {
-    for (int k = 0; k < CONV_K - 1; ++k) {
-      const int t = T - (CONV_K - 1) + k;       // absolute time
-      const int rr = t - t0 + (CONV_K - 1);      // row in xs
-      state[((size_t)b * Di + c0 + tid) * (CONV_K - 1) + k] = (t >= 0) ? xs[rr][tid] : 0.f;
+  __nv_bfloat16* d0 = xcT + ((size_t)b * Di + c) * Tp + t0;
+  __nv_bfloat16* d1 = d0 + Tp;
+  if (n == CONV_RUN) {
+#pragma unroll
+    for (int i = 0; i < CONV_RUN; i += 8) {
+      *reinterpret_cast<uint4*>(d0 + i) = *reinterpret_cast<const uint4*>(o0 + i);
+      *reinterpret_cast<uint4*>(d1 + i) = *reinterpret_cast<const uint4*>(o1 + i);
+    }
+  } else {
+    for (int i = 0; i < n; ++i) {
+      d0[i] = o0[i];
+      d1[i] = o1[i];
+    }
+  }
+  // conv state: the last 3 inputs x[T-3..T-1] (zero when T < 3), from the last run
+  if (t0 + n == T) {
+    float* s0 = state + ((size_t)b * Di + c) * 3;
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      const bool valid = T - 3 + k >= 0;
+      s0[k] = valid ? h0[k] : 0.f;
+      s0[3 + k] = valid ? h1[k] : 0.f;
     }
   }
 }
