@@ -10,13 +10,16 @@
 // edge apply an element mask.
 //
 // 192 threads:
-//   warp 0      TMA: Q once, K/V tiles through a 2-stage ring
-//   warp 1      TMEM allocation and MMA issue: S = Q K^T (M128 N128 K64) into TMEM, then
-//               O += P V with P read straight from TMEM (the "A in tensor memory" form)
+//   warp 0      TMA: Q once, K/V tiles through a 3-stage ring
+//   warp 1      TMEM allocation and MMA issue: S = Q K^T (M128 N128 K64) into TMEM, and
+//               O += P V with P read straight from TMEM (the "A in tensor memory" form).
+//               S(i+1) is issued as soon as the softmax has read S(i), so it runs on the
+//               tensor core while the softmax of tile i is still computing P(i).
 //   warps 2..5  softmax, one query row per thread: the whole S row comes into registers
-//               with one wait, P = 2^(s - m) is packed to fp16 and written back over the
-//               S columns; O stays in TMEM and is rescaled only when the running max grows
-//               by more than 2^8 (P <= 256 otherwise), then divided by the row sum at the end.
+//               with one wait, P = 2^(s - m) is packed to fp16 into its own TMEM columns;
+//               O stays in TMEM and is rescaled only when the running max grows by more
+//               than 2^8 (P <= 256 otherwise), then divided by the row sum at the end.
+// TMEM columns: S 0..127, P 128..191 (fp16 pairs), O 192..255.
 #pragma once
 #include "common.cuh"
 
@@ -34,17 +37,20 @@ struct AttnParams {
 };
 
 constexpr int ATT_THREADS = 192;
-constexpr int ATT_STAGES = 2;
+constexpr int ATT_STAGES = 3;
 constexpr int ATT_Q_BYTES = 128 * 128;
 constexpr int ATT_KV_BYTES = 128 * 128;          // one K or V tile: 128 keys x 64 dims fp16
 constexpr int ATT_OFF_Q = 0;
 constexpr int ATT_OFF_K = ATT_OFF_Q + ATT_Q_BYTES;
 constexpr int ATT_OFF_V = ATT_OFF_K + ATT_STAGES * ATT_KV_BYTES;
 constexpr int ATT_OFF_BAR = ATT_OFF_V + ATT_STAGES * ATT_KV_BYTES;
-// requested dynamic shared memory: the tiles need ~81 KB; asking for more keeps a third
-// CTA (which would wait for TMEM) off the SM.
-constexpr int ATT_SMEM = 100 * 1024;
-constexpr uint32_t ATT_TMEM_COLS = 256;          // S/P: cols 0..127, O: cols 128..191
+// requested dynamic shared memory: the tiles and barriers need 112.25 KB; 113 KB is the
+// most two CTAs can each take on one SM (228 KB, 1 KB reserved per CTA), and it keeps a
+// third CTA (which would wait for TMEM) off the SM.  The kernel checks that the dynamic
+// window is aligned well enough for the 1 KB-aligned tiles to fit.
+constexpr int ATT_SMEM = 113 * 1024;
+constexpr int ATT_USED = ATT_OFF_BAR + 128;
+constexpr uint32_t ATT_TMEM_COLS = 256;
 constexpr float ATT_RESCALE_LOG2 = 8.f;          // lazy rescale threshold (P <= 2^8)
 
 // Key tiles (128 keys each) visited by query tile qt, in order: meta tiles first, then the
@@ -140,13 +146,18 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
                     const __grid_constant__ CUtensorMap mapV, const __grid_constant__ AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if ((size_t)(smem - smem_raw) + ATT_USED > (size_t)ATT_SMEM) {   // cannot happen with a 1 KB-aligned window
+    if (threadIdx.x == 0) report_error(p.status, DEV_ERR_BOUNDS, 299);
+    return;
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ATT_OFF_BAR);
   uint64_t* q_full = bars;                   // 1
   uint64_t* kv_full = bars + 1;              // ATT_STAGES
   uint64_t* kv_empty = kv_full + ATT_STAGES; // ATT_STAGES
-  uint64_t* s_full = kv_empty + ATT_STAGES;  // S of tile j in TMEM
-  uint64_t* p_full = s_full + 1;             // P of tile j in TMEM (S read, rescale done)
-  uint64_t* o_done = p_full + 1;             // PV of tile j complete
+  uint64_t* s_full = kv_empty + ATT_STAGES;  // S(i) in TMEM
+  uint64_t* s_free = s_full + 1;             // softmax has read S(i)
+  uint64_t* p_full = s_free + 1;             // P(i) in TMEM (and O rescaled)
+  uint64_t* o_done = p_full + 1;             // PV(i) complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -166,6 +177,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       mbar_init(&kv_empty[s], 1);
     }
     mbar_init(s_full, 1);
+    mbar_init(s_free, 128);
     mbar_init(p_full, 128);
     mbar_init(o_done, 1);
     *abort_flag = 0;
@@ -179,7 +191,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t TM_S = tmem, TM_O = tmem + 128;
+  const uint32_t TM_S = tmem, TM_P = tmem + 128, TM_O = tmem + 192;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -210,7 +222,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       constexpr uint32_t IDESC_O = make_idesc(128, 64, 0u, false, true);     // fp16 P (TMEM), V MN-major
       const uint32_t sq = smem_u32(smem + ATT_OFF_Q);
       bool ok = mbar_wait(q_full, 0, abort_flag, p.status, 204);
-      // O += P(j) V(j): P in TMEM over the S columns, 8 steps of 16 keys (8 columns each)
+      // O += P(j) V(j): P in its TMEM columns, 8 steps of 16 keys (8 columns each)
       auto issue_pv = [&](int j) -> bool {
         if (!mbar_wait(p_full, j & 1u, abort_flag, p.status, 205)) return false;
         tc_fence_after();
@@ -219,7 +231,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t bd = make_sdesc_sw128(sv + kk * 2048, 8192, 1024);
-          umma_f16_tmem_a(TM_O, TM_S + kk * 8, bd, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_f16_tmem_a(TM_O, TM_P + kk * 8, bd, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(o_done);
         umma_commit(&kv_empty[s]);
@@ -228,8 +240,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       for (int i = 0; ok && i < n_tiles; ++i) {
         const int s = i % ATT_STAGES;
         if (!mbar_wait(&kv_full[s], (i / ATT_STAGES) & 1u, abort_flag, p.status, 206)) { ok = false; break; }
-        // S(i) overwrites the columns P(i-1) lives in: issue PV(i-1) first (in-order pipe)
-        if (i >= 1 && !issue_pv(i - 1)) { ok = false; break; }
+        if (i >= 1 && !mbar_wait(s_free, (i - 1) & 1u, abort_flag, p.status, 209)) { ok = false; break; }
         tc_fence_after();
         const uint32_t sk = smem_u32(smem + ATT_OFF_K + s * ATT_KV_BYTES);
 #pragma unroll
@@ -239,6 +250,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
           umma_f16(TM_S, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
         }
         umma_commit(s_full);
+        if (i >= 1 && !issue_pv(i - 1)) { ok = false; break; }
       }
       if (ok && n_tiles > 0) issue_pv(n_tiles - 1);
     }
@@ -250,33 +262,26 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
     const int qi = t0 + r;                       // absolute query position
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     float m_run = -INFINITY, l_run = 0.f;
-    int o_waited = -1;                           // last tile whose PV completion we observed
 
-    auto wait_o = [&](int j) -> bool {           // PV(j) complete (warp-uniform)
-      if (j < 0 || o_waited >= j) return true;
+    auto wait_bar = [&](uint64_t* bar, int j, unsigned site) -> bool {   // warp-uniform
       int ok = 1;
-      if (lane == 0) ok = mbar_wait(o_done, j & 1u, abort_flag, p.status, 207) ? 1 : 0;
+      if (lane == 0) ok = mbar_wait(bar, j & 1u, abort_flag, p.status, site) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (ok) {
-        o_waited = j;
-        tc_fence_after();
-      }
+      if (ok) tc_fence_after();
       return ok != 0;
     };
 
     bool ok = true;
     for (int i = 0; i < n_tiles; ++i) {
-      int w_ok = 1;
-      if (lane == 0) w_ok = mbar_wait(s_full, i & 1u, abort_flag, p.status, 208) ? 1 : 0;
-      w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
-      if (!w_ok) { ok = false; break; }
-      tc_fence_after();
+      if (!wait_bar(s_full, i, 208)) { ok = false; break; }
       const int kt = kts.tile(i);
       const int j0 = kt * 128;
       const bool full = (j0 + 127 <= t0) &&
                         (p.is_global || j0 + 127 < p.n_meta || (t0 + 127) - j0 < p.window);
       float s[128];
       tmem_ld128(TM_S + lane_off, s);
+      tc_fence_before();
+      mbar_arrive(s_free);                       // the tensor core may compute S(i+1) now
       float mx = -INFINITY;
       if (full) {
 #pragma unroll
@@ -285,10 +290,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
           mx = fmaxf(mx, s[e]);
         }
       } else {
+        const int lo = p.is_global ? -1 : qi - p.window + 1;   // window keys are >= lo
 #pragma unroll
         for (int e = 0; e < 128; ++e) {
           const int j = j0 + e;
-          const bool vis = (j <= qi) && (p.is_global || j < p.n_meta || qi - j < p.window);
+          const bool vis = (j <= qi) && (j >= lo || j < p.n_meta);
           s[e] = vis ? s[e] * p.scale_log2 : -INFINITY;
           mx = fmaxf(mx, s[e]);
         }
@@ -313,9 +319,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
         pk[e >> 1] = pack_f16x2(p0, p1);
       }
       l_run += rs;
-      // rescale O only after P is packed, so the S row is no longer live
+      // PV(i-1) must be done before P(i) replaces P(i-1) and before O is rescaled
+      if (i >= 1 && !wait_bar(o_done, i - 1, 207)) { ok = false; break; }
       if (__any_sync(0xffffffffu, resc)) {
-        if (!wait_o(i - 1)) { ok = false; break; }
         float o[32];
 #pragma unroll
         for (int hcol = 0; hcol < 64; hcol += 32) {
@@ -324,17 +330,15 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
           for (int d = 0; d < 32; ++d) o[d] *= alpha;
           tmem_st32(TM_O + lane_off + hcol, reinterpret_cast<const uint32_t*>(o));
         }
-        tmem_wait_st();
         l_run *= alpha;
       }
-      // P over the S columns (the tensor core is done with S(i): s_full completed)
-      tmem_st32(TM_S + lane_off, pk);
-      tmem_st32(TM_S + lane_off + 32, pk + 32);
+      tmem_st32(TM_P + lane_off, pk);
+      tmem_st32(TM_P + lane_off + 32, pk + 32);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full);
     }
-    if (ok && n_tiles > 0 && wait_o(n_tiles - 1)) {
+    if (ok && n_tiles > 0 && wait_bar(o_done, n_tiles - 1, 210)) {
       float o[64];
       tmem_ld32(TM_O + lane_off, o);
       tmem_ld32(TM_O + lane_off + 32, o + 32);

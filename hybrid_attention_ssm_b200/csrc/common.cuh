@@ -273,6 +273,16 @@ __device__ __forceinline__ float softplus_fast(float x) {
   if (u < 0.0078125f) return u * (1.f - u * (0.5f - u * 0.33333334f));
   return lg2_approx(1.f + u) * 0.6931471805599453f;
 }
-__device__ __forceinline__ float silu_f(float x) { return x / (1.f + expf(-x)); }
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// SiLU(x) = x * sigmoid(x) from the hardware ex2 and reciprocal (relative error ~1e-7,
+// far below the bf16/fp16 rounding of every result it feeds); large negative x gives
+// 2^(+big) = inf, rcp(inf) = 0 and the correct limit 0.
+__device__ __forceinline__ float silu_f(float x) {
+  return x * rcp_approx(1.f + ex2_approx(-1.4426950408889634f * x));
+}
 
 }  // namespace hymba

@@ -23,6 +23,8 @@ enum EpiMode : int {
   EPI_SWIGLU = 6,       // columns interleaved [gate(32) | up(32)] -> bf16 SiLU(gate)*up
   EPI_SOFTPLUS_T = 7,   // fp32 softplus(acc + bias[col]) stored time-major: out[(b*N + col)*T_out + row]
   EPI_F32_T = 8,        // transposed fp32 store: out[n][m]
+  EPI_F32_PART = 9,     // fp32 store of split ks's partial sum at out + ks*split_stride (row-major)
+  EPI_F32_T_PART = 10,  // the same, transposed
 };
 
 struct Segment {
@@ -46,6 +48,7 @@ struct GemmParams {
   int out_batches, T_out, row_off1;
   int mode;
   void* out;
+  long long split_stride;   // elements between the partial-sum slices of two splits
   int ld_out;
   int n_valid;              // columns (or, transposed, rows of out) that exist
   int m_valid;              // for transposed stores: valid M rows (output columns)
@@ -242,6 +245,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const int r = quad * 32 + lane;          // accumulator row of this thread
     int lt = 0;
     for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++lt) {
+      const int ks = tile % p.split_k;
       const int t2 = tile / p.split_k;
       const int m = t2 % p.m_tiles;
       const int n = t2 / p.m_tiles;
@@ -306,19 +310,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         auto process = [&](uint32_t* r, int c0) {
           float* v = reinterpret_cast<float*>(r);
           const int gc = col_base + c0;
-          if (p.mode == EPI_BF16_T || p.mode == EPI_ATOMIC_F32_T || p.mode == EPI_F32_T) {
+          if (p.mode == EPI_BF16_T || p.mode == EPI_ATOMIC_F32_T || p.mode == EPI_F32_T ||
+              p.mode == EPI_F32_T_PART) {
             // accumulator row = output column (weight row), accumulator column = output row
             if (!row_ok || rr >= p.m_valid) return;
+            float* outf = reinterpret_cast<float*>(p.out) + (p.mode == EPI_F32_T_PART ? ks * p.split_stride : 0);
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               const int orow_t = gc + e;
               if (orow_t < p.n_valid) {
                 if (p.mode == EPI_BF16_T)
                   reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)orow_t * p.ld_out + rr] = __float2bfloat16_rn(v[e]);
-                else if (p.mode == EPI_F32_T)
-                  reinterpret_cast<float*>(p.out)[(size_t)orow_t * p.ld_out + rr] = v[e];
+                else if (p.mode == EPI_ATOMIC_F32_T)
+                  atomicAdd(outf + (size_t)orow_t * p.ld_out + rr, v[e]);
                 else
-                  atomicAdd(reinterpret_cast<float*>(p.out) + (size_t)orow_t * p.ld_out + rr, v[e]);
+                  outf[(size_t)orow_t * p.ld_out + rr] = v[e];
               }
             }
             return;
@@ -349,13 +355,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             else
               for (int e = 0; e < 32; ++e)
                 if (gc + e < p.n_valid) dst[e] = __float2bfloat16_rn(v[e]);
-          } else if (p.mode == EPI_ATOMIC_F32) {
-            // vector fp32 reductions (ld_out and n_valid are multiples of 4)
-            float* dst = reinterpret_cast<float*>(p.out) + orow * p.ld_out + gc;
+          } else if (p.mode == EPI_ATOMIC_F32 || p.mode == EPI_F32_PART) {
+            // fp32 partial sums, 4-wide (ld_out and n_valid are multiples of 4)
+            float* dst = reinterpret_cast<float*>(p.out) + (p.mode == EPI_F32_PART ? ks * p.split_stride : 0) +
+                         orow * p.ld_out + gc;
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
-              if (gc + e < p.n_valid)
-                atomicAdd(reinterpret_cast<float4*>(dst + e), make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]));
+              if (gc + e < p.n_valid) {
+                const float4 q = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                if (p.mode == EPI_F32_PART) *reinterpret_cast<float4*>(dst + e) = q;
+                else atomicAdd(reinterpret_cast<float4*>(dst + e), q);
+              }
           } else {
             float bb[32];
             if (whole) {

@@ -298,9 +298,18 @@ Dims dims_of(const hymba_layer_cfg* c) {
   return x;
 }
 
+// Split-K factors depend only on the shapes (never on the device), so workspace sizes and
+// results are reproducible: enough splits to cover ~160 SMs, capped.
+int splits_for(int tiles, int k_blocks, int cap) {
+  int s = (160 + tiles - 1) / tiles;
+  if (s > cap) s = cap;
+  if (s > k_blocks) s = k_blocks;
+  return s < 1 ? 1 : s;
+}
+
 struct PrefillWs {
-  size_t q, xz, xc, xcT, xbc, dT, y, o, u, sstate, cstate, rope, total;
-  int T, Tp;
+  size_t q, xz, xc, xcT, xbc, xbc_part, dT, y, o, u, sstate, cstate, rope, total;
+  int T, Tp, xproj_split;
 };
 PrefillWs prefill_layout(const Dims& m, int B, int n_tokens, int x_has_meta) {
   PrefillWs w;
@@ -314,6 +323,8 @@ PrefillWs prefill_layout(const Dims& m, int B, int n_tokens, int x_has_meta) {
   w.xc = take(rows * m.Di * 2);
   w.xcT = take((size_t)B * m.Di * w.Tp * 2);
   w.xbc = take(rows * m.ld_xbc * 4);
+  w.xproj_split = splits_for(cdiv((long long)rows, GEMM_BM), cdiv(m.Di, 64), 16);
+  w.xbc_part = take((size_t)w.xproj_split * rows * m.ld_xbc * 4);
   w.dT = take((size_t)B * m.Di * w.Tp * 4);
   w.y = take(rows * m.Di * 2);
   w.o = take(rows * m.qw * 4);
@@ -326,8 +337,8 @@ PrefillWs prefill_layout(const Dims& m, int B, int n_tokens, int x_has_meta) {
 }
 
 struct DecodeWs {
-  size_t proj, part, o, xc, xbc, y, u, acc, total;
-  int n_splits;
+  size_t proj, part, o, xc, xbc, xbc_part, y, u, acc_part, total;
+  int n_splits, xproj_split, oproj_split;
 };
 DecodeWs decode_layout(const Dims& m, int B, int n_keys_max) {
   DecodeWs w;
@@ -339,9 +350,14 @@ DecodeWs decode_layout(const Dims& m, int B, int n_keys_max) {
   w.o = take((size_t)B * m.qw * 4);
   w.xc = take((size_t)B * m.Di * 2);
   w.xbc = take((size_t)B * m.ld_xbc * 4);
+  const int bn = B <= 64 ? 64 : (B <= 128 ? 128 : 256);
+  const int n_tiles = cdiv(B, bn);
+  w.xproj_split = splits_for(cdiv(m.R + 2 * m.S, GEMM_BM) * n_tiles, cdiv(m.Di, 64), 32);
+  w.xbc_part = take((size_t)w.xproj_split * B * m.ld_xbc * 4);
   w.y = take((size_t)B * m.Di * 4);
   w.u = take((size_t)B * m.uw * 2);
-  w.acc = take((size_t)B * m.d * 4);
+  w.oproj_split = splits_for(cdiv(m.d, GEMM_BM) * n_tiles, cdiv(m.uw, 64), 32);
+  w.acc_part = take((size_t)w.oproj_split * B * m.d * 4);
   w.total = off;
   return w;
 }
@@ -624,24 +640,27 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
-  // 3. x_proj (split-K, fp32 atomics): [dt_low | B | C]
+  // 3. x_proj (split-K into per-split slices, then a fixed-order sum): [dt_low | B | C]
   {
-    HY_CUDA(cudaMemsetAsync(f32(L.xbc), 0, rows * m.ld_xbc * 4, st));
     GemmCall c;
+    c.name = "x_proj";
     c.a1 = bf(L.xc); c.nb1 = 1; c.rows1 = (int)rows; c.lda1 = m.Di; c.a1_bstride = (long long)rows * m.Di;
     c.b = w->w_x; c.N = m.R + 2 * m.S; c.ldb = m.Di; c.K = m.Di;
     c.bn = pick_bn_cover(c.N);
-    const int mt = cdiv(rows, GEMM_BM);
-    const int kb = cdiv(m.Di, 64);
-    int sk = cdiv(dev->sms, mt);
-    c.split_k = sk > kb ? kb : sk;
-    c.name = "x_proj";
-    c.p.mode = EPI_ATOMIC_F32;
-    c.p.out = f32(L.xbc);
+    c.split_k = L.xproj_split;
+    c.p.mode = EPI_F32_PART;
+    c.p.out = f32(L.xbc_part);
+    c.p.split_stride = (long long)rows * m.ld_xbc;
     c.p.ld_out = m.ld_xbc;
     c.p.n_valid = c.N;
     c.p.status = status;
     HY_TRY(run_gemm(c, *dev, st));
+    const int n = (int)(rows * m.ld_xbc);
+    prof_begin("splitk_reduce", st);
+    splitk_reduce_kernel<<<cdiv(n / 4, 256), 256, 0, st>>>(f32(L.xbc_part), L.xproj_split, (long long)n, n,
+                                                            nullptr, f32(L.xbc), 0);
+    prof_end(st);
+    HY_CUDA(cudaGetLastError());
   }
   // 4. dt_proj (tf32) with softplus(+bias), stored time-major
   {
@@ -698,9 +717,18 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
   float* sstate = ssm_state_out != nullptr ? ssm_state_out : f32(L.sstate);
   {
     dim3 grid(m.Di / SCAN_CH, B);
+    static bool attr_scan[64] = {false};
+    int dcur = 0;
+    cudaGetDevice(&dcur);
+    if (!attr_scan[dcur & 63]) {
+      HY_CUDA(cudaFuncSetAttribute(selective_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)sizeof(ScanSmem)));
+      attr_scan[dcur & 63] = true;
+    }
     prof_begin("selective_scan", st);
-    selective_scan_kernel<<<grid, SCAN_THREADS, 0, st>>>(bf(L.xcT), f32(L.dT), f32(L.xbc) + m.R, m.ld_xbc, w->A,
-                                                         bf(L.y), sstate, T, L.Tp, m.Di);
+    selective_scan_kernel<<<grid, SCAN_THREADS, sizeof(ScanSmem), st>>>(bf(L.xcT), f32(L.dT), f32(L.xbc) + m.R,
+                                                                         m.ld_xbc, w->A, bf(L.y), sstate, T, L.Tp,
+                                                                         m.Di);
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
@@ -844,23 +872,28 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
-  // 4. x_proj (swap-AB, split-K into fp32)
+  // 4. x_proj (swap-AB, split-K into per-split slices, fixed-order sum)
   {
-    HY_CUDA(cudaMemsetAsync(f32(L.xbc), 0, (size_t)B * m.ld_xbc * 4, st));
     GemmCall c;
     c.a1 = w->w_x; c.nb1 = 1; c.rows1 = m.R + 2 * m.S; c.lda1 = m.Di; c.a1_bstride = (long long)c.rows1 * m.Di;
     c.b = bf(L.xc); c.N = B; c.ldb = m.Di; c.K = m.Di;
     c.bn = pick_bn_cover(B);
     c.name = "decode_x_proj";
-    const int tiles = cdiv(c.rows1, GEMM_BM) * cdiv(B, c.bn);
-    c.split_k = cdiv(dev->sms, tiles);
-    c.p.mode = EPI_ATOMIC_F32_T;
-    c.p.out = f32(L.xbc);
+    c.split_k = L.xproj_split;
+    c.p.mode = EPI_F32_T_PART;
+    c.p.out = f32(L.xbc_part);
+    c.p.split_stride = (long long)B * m.ld_xbc;
     c.p.ld_out = m.ld_xbc;
     c.p.m_valid = c.rows1;
     c.p.n_valid = B;
     c.p.status = status;
     HY_TRY(run_gemm(c, *dev, st));
+    const int n = B * m.ld_xbc;
+    prof_begin("decode_splitk_reduce", st);
+    splitk_reduce_kernel<<<cdiv(n / 4, 256), 256, 0, st>>>(f32(L.xbc_part), L.xproj_split, (long long)n, n, nullptr,
+                                                            f32(L.xbc), 0);
+    prof_end(st);
+    HY_CUDA(cudaGetLastError());
   }
   // 5. dt_proj + softplus + state update + C.h + gate
   {
@@ -879,19 +912,19 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
-  // 7. out_proj (swap-AB, split-K) and the bf16 (+ residual) store
+  // 7. out_proj (swap-AB, split-K into per-split slices), then the fixed-order sum with the
+  //    residual and the bf16 store
   {
-    HY_CUDA(cudaMemsetAsync(f32(L.acc), 0, (size_t)B * m.d * 4, st));
     GemmCall c;
     c.a1 = w->w_out; c.nb1 = 1; c.rows1 = m.d; c.lda1 = m.uw; c.a1_bstride = (long long)m.d * m.uw;
     c.b = h16(L.u); c.N = B; c.ldb = m.uw; c.K = m.uw;
     c.etype = ET_F16;
     c.bn = pick_bn_cover(B);
     c.name = "decode_out_proj";
-    const int tiles = cdiv(m.d, GEMM_BM) * cdiv(B, c.bn);
-    c.split_k = cdiv(dev->sms, tiles);
-    c.p.mode = EPI_ATOMIC_F32_T;
-    c.p.out = f32(L.acc);
+    c.split_k = L.oproj_split;
+    c.p.mode = EPI_F32_T_PART;
+    c.p.out = f32(L.acc_part);
+    c.p.split_stride = (long long)B * m.d;
     c.p.ld_out = m.d;
     c.p.m_valid = m.d;
     c.p.n_valid = B;
@@ -899,8 +932,8 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     HY_TRY(run_gemm(c, *dev, st));
     const int n = B * m.d;
     prof_begin("decode_out_store", st);
-    f32_to_bf16_residual_kernel<<<cdiv(n, 256), 256, 0, st>>>(
-        f32(L.acc), reinterpret_cast<const __nv_bfloat16*>(residual), reinterpret_cast<__nv_bfloat16*>(out), n);
+    splitk_reduce_kernel<<<cdiv(n / 4, 256), 256, 0, st>>>(f32(L.acc_part), L.oproj_split, (long long)n, n,
+                                                            reinterpret_cast<const __nv_bfloat16*>(residual), out, 1);
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }

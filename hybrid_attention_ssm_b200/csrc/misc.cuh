@@ -515,6 +515,32 @@ __global__ void wait_timeout_selftest_kernel(DevStatus* st) {
   if (threadIdx.x == 0) mbar_wait(&bar, 0, nullptr, st, 900);
 }
 
+// Fixed-order sum of split-K partial slices: out[i] = sum_s part[s*stride + i] (+ residual),
+// as fp32 or bf16; n is a multiple of 4.  The order never changes, so results are
+// identical from run to run.
+__global__ void splitk_reduce_kernel(const float* __restrict__ part, int n_split, long long stride, int n,
+                                     const __nv_bfloat16* __restrict__ residual, void* __restrict__ out,
+                                     int out_bf16) {
+  const int i = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (i >= n) return;
+  float4 acc = *reinterpret_cast<const float4*>(part + i);
+  for (int s = 1; s < n_split; ++s) {
+    const float4 q = *reinterpret_cast<const float4*>(part + (size_t)s * stride + i);
+    acc.x += q.x; acc.y += q.y; acc.z += q.z; acc.w += q.w;
+  }
+  if (residual != nullptr) {
+    const __nv_bfloat162 r0 = *reinterpret_cast<const __nv_bfloat162*>(residual + i);
+    const __nv_bfloat162 r1 = *reinterpret_cast<const __nv_bfloat162*>(residual + i + 2);
+    acc.x += __low2float(r0); acc.y += __high2float(r0); acc.z += __low2float(r1); acc.w += __high2float(r1);
+  }
+  if (out_bf16) {
+    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out) + i;
+    *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+  } else {
+    *reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + i) = acc;
+  }
+}
+
 // out[r, c] = bf16(acc[r, c] + residual[r, c])
 __global__ void f32_to_bf16_residual_kernel(const float* __restrict__ acc, const __nv_bfloat16* __restrict__ res,
                                             __nv_bfloat16* __restrict__ out, int n) {

@@ -94,13 +94,17 @@ __global__ void __launch_bounds__(256)
 // ----------------------------------------------------------------------------------------
 // Selective scan, time-sequential per (channel, state) thread.
 //   h_t = exp(delta_t * A[c,s]) h_{t-1} + delta_t * B_t[s] * x_t ;  y_t = sum_s C_t[s] h_t[s]
-// 16 lanes of a warp hold the 16 states of one channel; the sum over states is a
-// reduce-scatter through 8 shuffles per 8 time steps.  The fp32 state stays in registers
-// for the whole sequence.  Inputs are staged through shared memory in chunks of 64 steps
-// (cp.async for the time-major x and delta, register transpose for B/C), 3 stages deep.
+// CTA = 8 channels x 16 states.  The fp32 state stays in a register for the whole
+// sequence.  Inputs go through shared memory in chunks of 64 steps, 3 stages deep: delta,
+// delta*x (formed once per step and channel while staging) and B/C transposed to
+// [state][t] so each thread reads 4 steps per 128-bit load.  Each thread writes its
+// C_t[s] h_t[s] terms to a swizzled buffer; after the chunk, one thread per (4 steps,
+// channel) sums the 16 states (bank-conflict-free on both sides) and the y rows leave as
+// 16-byte stores.
 //   xcT [B, Di, Tp] bf16; dT [B, Di, Tp] fp32 (Tp: row stride, multiple of 8; steps at or
-//   beyond T read as zero, so delta = 0 leaves the state unchanged); bc [B*T, ld_bc] fp32 (B at col 0..15, C at
-//   16..31 of the pointer); A [Di, 16]; y [B*T, Di] bf16 (not gated); state [B, Di, 16].
+//   beyond T read as zero, so delta = 0 leaves the state unchanged); bc [B*T, ld_bc] fp32
+//   (B at col 0..15, C at 16..31 of the pointer); A [Di, 16]; y [B*T, Di] bf16 (not gated);
+//   state [B, Di, 16].
 // ----------------------------------------------------------------------------------------
 constexpr int SCAN_CH = 8;            // channels per CTA
 constexpr int SCAN_TC = 64;           // time steps per chunk
@@ -108,17 +112,22 @@ constexpr int SCAN_NST = 3;           // pipeline stages
 constexpr int SCAN_THREADS = SCAN_CH * 16;
 
 struct ScanStage {
-  __nv_bfloat16 x[SCAN_CH][SCAN_TC];  // 8 x 128 B
-  float d[SCAN_CH][SCAN_TC];          // 8 x 256 B
+  float d[SCAN_CH][SCAN_TC];          // delta
+  float dx[SCAN_CH][SCAN_TC];         // delta * x
   float bcT[32][SCAN_TC + 4];         // [state (B 0..15, C 16..31)][t]
+};
+struct ScanSmem {
+  ScanStage st[SCAN_NST];
+  float part[SCAN_TC / 4][16][SCAN_CH][4];   // C*h terms: [t/4][state][channel ^ (state&7)][t%4]
+  __nv_bfloat16 ys[SCAN_TC][SCAN_CH];
 };
 
 __global__ void __launch_bounds__(SCAN_THREADS)
     selective_scan_kernel(const __nv_bfloat16* __restrict__ xcT, const float* __restrict__ dT,
                           const float* __restrict__ bc, int ld_bc, const float* __restrict__ A,
                           __nv_bfloat16* __restrict__ y, float* __restrict__ state, int T, int Tp, int Di) {
-  __shared__ __align__(16) ScanStage st[SCAN_NST];
-  __shared__ __align__(16) __nv_bfloat16 ys[SCAN_TC][SCAN_CH];
+  extern __shared__ __align__(16) uint8_t scan_smem_raw[];
+  ScanSmem& sm = *reinterpret_cast<ScanSmem*>(scan_smem_raw);
   const int tid = threadIdx.x;
   const int cl = tid >> 4;         // channel within CTA
   const int s = tid & 15;          // state
@@ -128,150 +137,111 @@ __global__ void __launch_bounds__(SCAN_THREADS)
   const int n_chunks = (T + SCAN_TC - 1) / SCAN_TC;
   const float A2 = A[(size_t)c * 16 + s] * 1.4426950408889634f;   // exp(d*A) = 2^(d*A*log2 e)
 
-  // async loads of the time-major x / delta rows of chunk k into stage k % NST
-  auto load_xd = [&](int k) {
-    ScanStage& S = st[k % SCAN_NST];
-    const int t0 = k * SCAN_TC;
-    // x: 8 channels x 8 pieces of 16 B; delta: 8 channels x 16 pieces
-    for (int i = tid; i < SCAN_CH * 24; i += SCAN_THREADS) {
-      const int ch = i / 24, piece = i % 24;
-      if (piece < 8) {
-        const int t = t0 + piece * 8;
-        const int nbytes = t >= T ? 0 : min(16, (T - t) * 2);
-        const __nv_bfloat16* src = xcT + ((size_t)b * Di + c0 + ch) * Tp + (t >= T ? 0 : t);
-        cp_async16(&S.x[ch][piece * 8], src, nbytes);
-      } else {
-        const int t = t0 + (piece - 8) * 4;
-        const int nbytes = t >= T ? 0 : min(16, (T - t) * 4);
-        const float* src = dT + ((size_t)b * Di + c0 + ch) * Tp + (t >= T ? 0 : t);
-        cp_async16(&S.d[ch][(piece - 8) * 4], src, nbytes);
-      }
+  // staging of chunk k through registers: thread -> (channel lch, 4 steps lq*4..) for
+  // delta and x, and (row, 16 of B|C) for the B/C rows
+  const int lch = tid >> 4, lq = tid & 15;
+  float4 rd;
+  uint2 rx;
+  float rbc[16];
+  auto load_chunk = [&](int k) {
+    const int t = k * SCAN_TC + lq * 4;
+    const size_t row = ((size_t)b * Di + c0 + lch) * Tp;
+    rd = make_float4(0.f, 0.f, 0.f, 0.f);
+    rx = make_uint2(0u, 0u);
+    if (t + 4 <= T) {
+      rd = *reinterpret_cast<const float4*>(dT + row + t);
+      rx = *reinterpret_cast<const uint2*>(xcT + row + t);
+    } else {
+      float dd[4] = {0.f, 0.f, 0.f, 0.f};
+      __nv_bfloat16 xx[4] = {__float2bfloat16_rn(0.f), __float2bfloat16_rn(0.f), __float2bfloat16_rn(0.f),
+                             __float2bfloat16_rn(0.f)};
+      for (int e = 0; e < 4; ++e)
+        if (t + e < T) {
+          dd[e] = dT[row + t + e];
+          xx[e] = xcT[row + t + e];
+        }
+      rd = make_float4(dd[0], dd[1], dd[2], dd[3]);
+      rx = *reinterpret_cast<const uint2*>(xx);
     }
-  };
-  // B/C of chunk k: 64 rows x 32 floats, loaded into registers (16 per thread) ...
-  float bcr[16];
-  auto load_bc = [&](int k) {
-    const int t0 = k * SCAN_TC;
-    const int row = tid >> 1, half = (tid & 1) * 16;
-    const int t = t0 + row;
+    const int brow = tid >> 1, half = (tid & 1) * 16;
+    const int tb = k * SCAN_TC + brow;
 #pragma unroll
     for (int e = 0; e < 16; e += 4) {
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (t < T) v = *reinterpret_cast<const float4*>(bc + ((size_t)b * T + t) * ld_bc + half + e);
-      bcr[e] = v.x; bcr[e + 1] = v.y; bcr[e + 2] = v.z; bcr[e + 3] = v.w;
+      if (tb < T) v = *reinterpret_cast<const float4*>(bc + ((size_t)b * T + tb) * ld_bc + half + e);
+      rbc[e] = v.x; rbc[e + 1] = v.y; rbc[e + 2] = v.z; rbc[e + 3] = v.w;
     }
   };
-  // ... and stored transposed ([state][t]) into the stage
-  auto store_bc = [&](int k) {
-    ScanStage& S = st[k % SCAN_NST];
-    const int row = tid >> 1, half = (tid & 1) * 16;
+  auto store_chunk = [&](int k) {
+    ScanStage& S = sm.st[k % SCAN_NST];
+    const __nv_bfloat16* xh = reinterpret_cast<const __nv_bfloat16*>(&rx);
+    *reinterpret_cast<float4*>(&S.d[lch][lq * 4]) = rd;
+    *reinterpret_cast<float4*>(&S.dx[lch][lq * 4]) =
+        make_float4(rd.x * __bfloat162float(xh[0]), rd.y * __bfloat162float(xh[1]), rd.z * __bfloat162float(xh[2]),
+                    rd.w * __bfloat162float(xh[3]));
+    const int brow = tid >> 1, half = (tid & 1) * 16;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) S.bcT[half + e][row] = bcr[e];
+    for (int e = 0; e < 16; ++e) S.bcT[half + e][brow] = rbc[e];
   };
 
   // prologue: chunks 0 .. NST-2
-  for (int k = 0; k < SCAN_NST - 1; ++k) {
-    if (k < n_chunks) {
-      load_xd(k);
-      load_bc(k);
-      store_bc(k);
-    }
-    cp_async_commit();
+  for (int k = 0; k < SCAN_NST - 1 && k < n_chunks; ++k) {
+    load_chunk(k);
+    store_chunk(k);
   }
-
   float h = 0.f;
-  const int l = tid & 15;
-  const int my_step = ((l >> 3) & 1) * 4 + ((l >> 2) & 1) * 2 + ((l >> 1) & 1);
+  const int sw = s & 7;
   for (int k = 0; k < n_chunks; ++k) {
     const int kn = k + SCAN_NST - 1;
-    cp_async_wait<SCAN_NST - 2>();
-    __syncthreads();                       // chunk k visible; stage of chunk k-1 free
-    if (kn < n_chunks) {
-      load_xd(kn);
-      load_bc(kn);
-    }
-    cp_async_commit();
-    const ScanStage& S = st[k % SCAN_NST];
-    // Software pipeline over the 8 blocks of 8 steps: block q's recurrence runs while the
-    // state-sum of block q-1 goes through its shuffles, so the two latency chains overlap.
-    float vprev[8];
-    auto block_inputs = [&](int tt, float* dv, float* xv, float* bv, float* cv) {
-      const uint4 xr = *reinterpret_cast<const uint4*>(&S.x[cl][tt]);
-      const __nv_bfloat16* xh = reinterpret_cast<const __nv_bfloat16*>(&xr);
+    __syncthreads();                       // chunk k staged; its part/ys buffers free
+    if (kn < n_chunks) load_chunk(kn);     // in flight during the compute below
+    const ScanStage& S = sm.st[k % SCAN_NST];
+#pragma unroll 2
+    for (int tt = 0; tt < SCAN_TC; tt += 8) {
       const float4 d0 = *reinterpret_cast<const float4*>(&S.d[cl][tt]);
       const float4 d1 = *reinterpret_cast<const float4*>(&S.d[cl][tt + 4]);
+      const float4 q0 = *reinterpret_cast<const float4*>(&S.dx[cl][tt]);
+      const float4 q1 = *reinterpret_cast<const float4*>(&S.dx[cl][tt + 4]);
       const float4 b0 = *reinterpret_cast<const float4*>(&S.bcT[s][tt]);
       const float4 b1 = *reinterpret_cast<const float4*>(&S.bcT[s][tt + 4]);
       const float4 e0 = *reinterpret_cast<const float4*>(&S.bcT[16 + s][tt]);
       const float4 e1 = *reinterpret_cast<const float4*>(&S.bcT[16 + s][tt + 4]);
-      dv[0] = d0.x; dv[1] = d0.y; dv[2] = d0.z; dv[3] = d0.w; dv[4] = d1.x; dv[5] = d1.y; dv[6] = d1.z; dv[7] = d1.w;
-      bv[0] = b0.x; bv[1] = b0.y; bv[2] = b0.z; bv[3] = b0.w; bv[4] = b1.x; bv[5] = b1.y; bv[6] = b1.z; bv[7] = b1.w;
-      cv[0] = e0.x; cv[1] = e0.y; cv[2] = e0.z; cv[3] = e0.w; cv[4] = e1.x; cv[5] = e1.y; cv[6] = e1.z; cv[7] = e1.w;
+      const float dv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+      const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      const float cv[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+      float a[8], v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) xv[u] = __bfloat162float(xh[u]);
-    };
-    auto recur = [&](const float* dv, const float* xv, const float* bv, const float* cv, float* v) {
-      float a[8], q[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        a[u] = ex2_approx(dv[u] * A2);
-        q[u] = dv[u] * xv[u] * bv[u];
-      }
+      for (int u = 0; u < 8; ++u) a[u] = ex2_approx(dv[u] * A2);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        h = fmaf(a[u], h, q[u]);
+        h = fmaf(a[u], h, qv[u] * bv[u]);
         v[u] = cv[u] * h;
       }
-    };
-    // reduce-scatter of v[0..7] over the 16 state lanes: lane l ends with the full sum of
-    // step my_step (lanes l and l^1 hold the same step)
-    auto reduce_store = [&](const float* v, int tt) {
-      const bool q3 = l & 8, q2 = l & 4, q1 = l & 2;
-      float w4[4];
-#pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4) {
-        const float send = q3 ? v[k4] : v[k4 + 4];
-        const float keep = q3 ? v[k4 + 4] : v[k4];
-        w4[k4] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-      }
-      float w2[2];
-#pragma unroll
-      for (int k2 = 0; k2 < 2; ++k2) {
-        const float send = q2 ? w4[k2] : w4[k2 + 2];
-        const float keep = q2 ? w4[k2 + 2] : w4[k2];
-        w2[k2] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-      }
-      float w1;
-      {
-        const float send = q1 ? w2[0] : w2[1];
-        const float keep = q1 ? w2[1] : w2[0];
-        w1 = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-      }
-      w1 += __shfl_xor_sync(0xffffffffu, w1, 1);
-      if ((l & 1) == 0) ys[tt + my_step][cl] = __float2bfloat16_rn(w1);
-    };
-    {
-      float dv[8], xv[8], bv[8], cv[8];
-      block_inputs(0, dv, xv, bv, cv);
-      recur(dv, xv, bv, cv, vprev);
+      *reinterpret_cast<float4*>(&sm.part[tt >> 2][s][cl ^ sw][0]) = make_float4(v[0], v[1], v[2], v[3]);
+      *reinterpret_cast<float4*>(&sm.part[(tt >> 2) + 1][s][cl ^ sw][0]) = make_float4(v[4], v[5], v[6], v[7]);
     }
-#pragma unroll 1
-    for (int tt = 8; tt < SCAN_TC; tt += 8) {
-      float dv[8], xv[8], bv[8], cv[8], v[8];
-      block_inputs(tt, dv, xv, bv, cv);
-      recur(dv, xv, bv, cv, v);
-      reduce_store(vprev, tt - 8);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) vprev[u] = v[u];
-    }
-    reduce_store(vprev, SCAN_TC - 8);
-    if (kn < n_chunks) store_bc(kn);
+    if (kn < n_chunks) store_chunk(kn);
     __syncthreads();
-    // flush y rows of this chunk: 64 rows x 16 B
+    // sum over the 16 states: thread -> (4 steps tg, channel ch)
+    {
+      const int tg = tid >> 3, ch = tid & 7;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int st = 0; st < 16; ++st) {
+        const float4 q = *reinterpret_cast<const float4*>(&sm.part[tg][st][ch ^ (st & 7)][0]);
+        acc.x += q.x; acc.y += q.y; acc.z += q.z; acc.w += q.w;
+      }
+      sm.ys[tg * 4 + 0][ch] = __float2bfloat16_rn(acc.x);
+      sm.ys[tg * 4 + 1][ch] = __float2bfloat16_rn(acc.y);
+      sm.ys[tg * 4 + 2][ch] = __float2bfloat16_rn(acc.z);
+      sm.ys[tg * 4 + 3][ch] = __float2bfloat16_rn(acc.w);
+    }
+    __syncthreads();
     if (tid < SCAN_TC) {
       const int t = k * SCAN_TC + tid;
       if (t < T)
-        *reinterpret_cast<uint4*>(y + ((size_t)b * T + t) * Di + c0) = *reinterpret_cast<const uint4*>(&ys[tid][0]);
+        *reinterpret_cast<uint4*>(y + ((size_t)b * T + t) * Di + c0) = *reinterpret_cast<const uint4*>(&sm.ys[tid][0]);
     }
   }
   state[((size_t)b * Di + c) * 16 + s] = h;
