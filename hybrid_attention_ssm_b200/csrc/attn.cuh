@@ -2,9 +2,10 @@
 // Q/K/V/P (keys, values and probabilities sit far inside fp16's range, where it rounds 8x
 // finer than bf16), fp32 scores and accumulators.
 //
-// One CTA per (query tile of 128 rows, query head, sequence); two CTAs share an SM
-// (256 TMEM columns and ~100 KB of shared memory each), so one CTA's softmax overlaps the
-// other's MMAs.  The key tiles a CTA visits are the meta-token tiles plus the tiles that
+// Persistent: two CTAs per SM (256 TMEM columns and 113 KB of shared memory each) loop over
+// the (query tile of 128 rows, query head, sequence) work items, heaviest first, so one
+// CTA's softmax overlaps the other's MMAs and no wave is left half empty.  The TMA warp
+// prefetches the next item's Q and K/V while the current item finishes.  The key tiles a CTA visits are the meta-token tiles plus the tiles that
 // intersect the sliding window of its rows (every causal tile for a global layer): block
 // skipping, no dense mask.  Only tiles that straddle the causal diagonal or the window
 // edge apply an element mask.
@@ -30,6 +31,7 @@ struct AttnParams {
   int Hq, Hkv;
   int n_meta, window, is_global;
   int q_tiles;
+  int n_items;        // q_tiles * Hq * B work items
   float scale_log2;   // log2(e) / sqrt(head_dim)
   float* out;         // O [B*T, ld_out] fp32, head h at columns h*64
   int ld_out;
@@ -49,7 +51,7 @@ constexpr int ATT_OFF_BAR = ATT_OFF_V + ATT_STAGES * ATT_KV_BYTES;
 // third CTA (which would wait for TMEM) off the SM.  The kernel checks that the dynamic
 // window is aligned well enough for the 1 KB-aligned tiles to fit.
 constexpr int ATT_SMEM = 113 * 1024;
-constexpr int ATT_USED = ATT_OFF_BAR + 128;
+constexpr int ATT_USED = ATT_OFF_BAR + 160;
 constexpr uint32_t ATT_TMEM_COLS = 256;
 constexpr float ATT_RESCALE_LOG2 = 8.f;          // lazy rescale threshold (P <= 2^8)
 
@@ -141,9 +143,18 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// work item w -> (query tile, head, sequence); longest query tiles first
+__device__ __forceinline__ void attn_item(const AttnParams& p, int w, int B, int& qt, int& h, int& b) {
+  const int per_qt = p.Hq * B;
+  qt = p.q_tiles - 1 - w / per_qt;
+  const int r = w % per_qt;
+  h = r % p.Hq;
+  b = r / p.Hq;
+}
+
 __global__ void __launch_bounds__(ATT_THREADS, 2)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
-                    const __grid_constant__ CUtensorMap mapV, const __grid_constant__ AttnParams p) {
+                    const __grid_constant__ CUtensorMap mapV, const __grid_constant__ AttnParams p, int B) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   if ((size_t)(smem - smem_raw) + ATT_USED > (size_t)ATT_SMEM) {   // cannot happen with a 1 KB-aligned window
@@ -151,8 +162,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
     return;
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ATT_OFF_BAR);
-  uint64_t* q_full = bars;                   // 1
-  uint64_t* kv_full = bars + 1;              // ATT_STAGES
+  uint64_t* q_full = bars;                   // Q of the current item loaded
+  uint64_t* q_empty = bars + 1;              // every S of the current item issued and done
+  uint64_t* kv_full = bars + 2;              // ATT_STAGES
   uint64_t* kv_empty = kv_full + ATT_STAGES; // ATT_STAGES
   uint64_t* s_full = kv_empty + ATT_STAGES;  // S(i) in TMEM
   uint64_t* s_free = s_full + 1;             // softmax has read S(i)
@@ -163,15 +175,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int qt = p.q_tiles - 1 - blockIdx.x;     // longest rows first
-  const int h = blockIdx.y;
-  const int b = blockIdx.z;
-  const int g = (h * p.Hkv) / p.Hq;
-  const KeyTiles kts = key_tiles(p, qt);
-  const int n_tiles = kts.count();
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < ATT_STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
@@ -194,74 +201,90 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
   const uint32_t TM_S = tmem, TM_P = tmem + 128, TM_O = tmem + 192;
 
   if (warp == 0) {
+    // ------------------------------ TMA producer ------------------------------
     if (lane == 0) {
       tma_prefetch_desc(&mapQ);
       tma_prefetch_desc(&mapK);
       tma_prefetch_desc(&mapV);
-      mbar_arrive_expect_tx(q_full, ATT_Q_BYTES);
-      tma_load_3d(smem + ATT_OFF_Q, &mapQ, q_full, h * 64, qt * 128, b);
-      int issued = 0;
-      for (int i = 0; i < n_tiles; ++i) {
-        const int s = i % ATT_STAGES;
-        const uint32_t ph = (i / ATT_STAGES) & 1u;
-        if (!mbar_wait(&kv_empty[s], ph ^ 1u, abort_flag, p.status, 201)) break;
-        const int kt = kts.tile(i);
-        mbar_arrive_expect_tx(&kv_full[s], 2 * ATT_KV_BYTES);
-        tma_load_3d(smem + ATT_OFF_K + s * ATT_KV_BYTES, &mapK, &kv_full[s], g * 64, kt * 128, b);
-        tma_load_3d(smem + ATT_OFF_V + s * ATT_KV_BYTES, &mapV, &kv_full[s], g * 64, kt * 128, b);
-        issued = i + 1;
+      int gi = 0, it = 0;                    // tiles and items issued by this CTA
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x, ++it) {
+        int qt, h, b;
+        attn_item(p, w, B, qt, h, b);
+        const int g = (h * p.Hkv) / p.Hq;
+        const KeyTiles kts = key_tiles(p, qt);
+        if (it > 0 && !mbar_wait(q_empty, (it - 1) & 1u, abort_flag, p.status, 200)) { ok = false; break; }
+        mbar_arrive_expect_tx(q_full, ATT_Q_BYTES);
+        tma_load_3d(smem + ATT_OFF_Q, &mapQ, q_full, h * 64, qt * 128, b);
+        for (int i = 0; i < kts.count(); ++i, ++gi) {
+          const int s = gi % ATT_STAGES;
+          if (!mbar_wait(&kv_empty[s], ((gi / ATT_STAGES) & 1u) ^ 1u, abort_flag, p.status, 201)) {
+            ok = false;
+            break;
+          }
+          const int kt = kts.tile(i);
+          mbar_arrive_expect_tx(&kv_full[s], 2 * ATT_KV_BYTES);
+          tma_load_3d(smem + ATT_OFF_K + s * ATT_KV_BYTES, &mapK, &kv_full[s], g * 64, kt * 128, b);
+          tma_load_3d(smem + ATT_OFF_V + s * ATT_KV_BYTES, &mapV, &kv_full[s], g * 64, kt * 128, b);
+        }
       }
       // drain every load still in flight
-      mbar_wait(q_full, 0, nullptr, p.status, 202);
-      for (int j = max(0, issued - ATT_STAGES); j < issued; ++j)
+      if (it > 0) mbar_wait(q_full, (it - 1) & 1u, nullptr, p.status, 202);
+      for (int j = max(0, gi - ATT_STAGES); j < gi; ++j)
         mbar_wait(&kv_full[j % ATT_STAGES], (j / ATT_STAGES) & 1u, nullptr, p.status, 203);
     }
   } else if (warp == 1) {
+    // ------------------------------ MMA issuer ------------------------------
     if (lane == 0) {
       constexpr uint32_t IDESC_S = make_idesc(128, 128, 0u, false, false);   // fp16 Q, K (K-major)
       constexpr uint32_t IDESC_O = make_idesc(128, 64, 0u, false, true);     // fp16 P (TMEM), V MN-major
       const uint32_t sq = smem_u32(smem + ATT_OFF_Q);
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.status, 204);
-      // O += P(j) V(j): P in its TMEM columns, 8 steps of 16 keys (8 columns each)
-      auto issue_pv = [&](int j) -> bool {
-        if (!mbar_wait(p_full, j & 1u, abort_flag, p.status, 205)) return false;
+      // O (+)= P(gj) V(gj): P in its TMEM columns, 8 steps of 16 keys (8 columns each)
+      auto issue_pv = [&](int gj, bool first) -> bool {
+        if (!mbar_wait(p_full, gj & 1u, abort_flag, p.status, 205)) return false;
         tc_fence_after();
-        const int s = j % ATT_STAGES;
+        const int s = gj % ATT_STAGES;
         const uint32_t sv = smem_u32(smem + ATT_OFF_V + s * ATT_KV_BYTES);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t bd = make_sdesc_sw128(sv + kk * 2048, 8192, 1024);
-          umma_f16_tmem_a(TM_O, TM_P + kk * 8, bd, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_f16_tmem_a(TM_O, TM_P + kk * 8, bd, IDESC_O, (!first || kk > 0) ? 1u : 0u);
         }
         umma_commit(o_done);
         umma_commit(&kv_empty[s]);
         return true;
       };
-      for (int i = 0; ok && i < n_tiles; ++i) {
-        const int s = i % ATT_STAGES;
-        if (!mbar_wait(&kv_full[s], (i / ATT_STAGES) & 1u, abort_flag, p.status, 206)) { ok = false; break; }
-        if (i >= 1 && !mbar_wait(s_free, (i - 1) & 1u, abort_flag, p.status, 209)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t sk = smem_u32(smem + ATT_OFF_K + s * ATT_KV_BYTES);
+      int gi = 0, it = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x, ++it) {
+        int qt, h, b;
+        attn_item(p, w, B, qt, h, b);
+        const int n_tiles = key_tiles(p, qt).count();
+        if (!mbar_wait(q_full, it & 1u, abort_flag, p.status, 204)) { ok = false; break; }
+        for (int i = 0; i < n_tiles; ++i, ++gi) {
+          const int s = gi % ATT_STAGES;
+          if (!mbar_wait(&kv_full[s], (gi / ATT_STAGES) & 1u, abort_flag, p.status, 206)) { ok = false; break; }
+          if (gi >= 1 && !mbar_wait(s_free, (gi - 1) & 1u, abort_flag, p.status, 209)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sk = smem_u32(smem + ATT_OFF_K + s * ATT_KV_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = make_sdesc_sw128(sq + kk * 32, 16, 1024);
-          const uint64_t bd = make_sdesc_sw128(sk + kk * 32, 16, 1024);
-          umma_f16(TM_S, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = make_sdesc_sw128(sq + kk * 32, 16, 1024);
+            const uint64_t bd = make_sdesc_sw128(sk + kk * 32, 16, 1024);
+            umma_f16(TM_S, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(s_full);
+          if (i == n_tiles - 1) umma_commit(q_empty);          // Q no longer read
+          if (i >= 1 && !issue_pv(gi - 1, i == 1)) { ok = false; break; }
         }
-        umma_commit(s_full);
-        if (i >= 1 && !issue_pv(i - 1)) { ok = false; break; }
+        if (ok && n_tiles > 0 && !issue_pv(gi - 1, n_tiles == 1)) ok = false;
       }
-      if (ok && n_tiles > 0) issue_pv(n_tiles - 1);
     }
   } else {
     // ------------------------------ softmax warps ------------------------------
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
-    const int t0 = qt * 128;
-    const int qi = t0 + r;                       // absolute query position
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    float m_run = -INFINITY, l_run = 0.f;
 
     auto wait_bar = [&](uint64_t* bar, int j, unsigned site) -> bool {   // warp-uniform
       int ok = 1;
@@ -271,77 +294,106 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       return ok != 0;
     };
 
+    int gi = 0;
     bool ok = true;
-    for (int i = 0; i < n_tiles; ++i) {
-      if (!wait_bar(s_full, i, 208)) { ok = false; break; }
-      const int kt = kts.tile(i);
-      const int j0 = kt * 128;
-      const bool full = (j0 + 127 <= t0) &&
-                        (p.is_global || j0 + 127 < p.n_meta || (t0 + 127) - j0 < p.window);
-      float s[128];
-      tmem_ld128(TM_S + lane_off, s);
-      tc_fence_before();
-      mbar_arrive(s_free);                       // the tensor core may compute S(i+1) now
-      float mx = -INFINITY;
-      if (full) {
+    for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
+      int qt, h, b;
+      attn_item(p, w, B, qt, h, b);
+      const KeyTiles kts = key_tiles(p, qt);
+      const int n_tiles = kts.count();
+      const int t0 = qt * 128;
+      const int qi = t0 + r;                     // absolute query position
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int i = 0; i < n_tiles; ++i, ++gi) {
+        if (!wait_bar(s_full, gi, 208)) { ok = false; break; }
+        const int j0 = kts.tile(i) * 128;
+        const bool causal_full = j0 + 127 <= t0;
+        const bool window_full = p.is_global || j0 + 127 < p.n_meta || (t0 + 127) - j0 < p.window;
+        float s[128];
+        tmem_ld128(TM_S + lane_off, s);
+        tc_fence_before();
+        mbar_arrive(s_free);                     // the tensor core may compute S(i+1) now
+        // row max of the raw scores (the positive scale keeps the order), 8 independent
+        // partial maxima; invisible keys become -inf (tile kinds: full, diagonal only,
+        // window edge only, both)
+        float mxp[8];
 #pragma unroll
-        for (int e = 0; e < 128; ++e) {
-          s[e] *= p.scale_log2;
-          mx = fmaxf(mx, s[e]);
+        for (int k = 0; k < 8; ++k) mxp[k] = -INFINITY;
+        const int e_hi = qi - j0;                          // causal: e <= e_hi
+        const int e_lo = qi - p.window + 1 - j0;           // window: e >= e_lo
+        const int e_meta = p.n_meta - j0;                  // meta: e < e_meta
+        if (causal_full && window_full) {
+#pragma unroll
+          for (int e = 0; e < 128; ++e) mxp[e & 7] = fmaxf(mxp[e & 7], s[e]);
+        } else if (window_full) {
+#pragma unroll
+          for (int e = 0; e < 128; ++e) {
+            s[e] = e <= e_hi ? s[e] : -INFINITY;
+            mxp[e & 7] = fmaxf(mxp[e & 7], s[e]);
+          }
+        } else if (causal_full) {
+#pragma unroll
+          for (int e = 0; e < 128; ++e) {
+            s[e] = (e >= e_lo || e < e_meta) ? s[e] : -INFINITY;
+            mxp[e & 7] = fmaxf(mxp[e & 7], s[e]);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 128; ++e) {
+            s[e] = (e <= e_hi && (e >= e_lo || e < e_meta)) ? s[e] : -INFINITY;
+            mxp[e & 7] = fmaxf(mxp[e & 7], s[e]);
+          }
         }
-      } else {
-        const int lo = p.is_global ? -1 : qi - p.window + 1;   // window keys are >= lo
-#pragma unroll
-        for (int e = 0; e < 128; ++e) {
-          const int j = j0 + e;
-          const bool vis = (j <= qi) && (j >= lo || j < p.n_meta);
-          s[e] = vis ? s[e] * p.scale_log2 : -INFINITY;
-          mx = fmaxf(mx, s[e]);
+        const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                               fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]))) * p.scale_log2;
+        // running max (log2 units): rescale O (in TMEM) only when it grows by more than 2^8
+        float alpha = 1.f;
+        bool resc = false;
+        if (m_run == -INFINITY) {
+          m_run = mx;                             // nothing accumulated for this row yet
+        } else if (mx > m_run + ATT_RESCALE_LOG2) {
+          alpha = exp2f(m_run - mx);
+          m_run = mx;
+          resc = true;
         }
-      }
-      // running max: rescale O (in TMEM) only when the max grows by more than 2^8
-      float alpha = 1.f;
-      bool resc = false;
-      if (m_run == -INFINITY) {
-        m_run = mx;                               // nothing accumulated for this row yet
-      } else if (mx > m_run + ATT_RESCALE_LOG2) {
-        alpha = exp2f(m_run - mx);
-        m_run = mx;
-        resc = true;
-      }
-      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      float rs = 0.f;
-      uint32_t pk[64];
+        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+        float rsp[8];
 #pragma unroll
-      for (int e = 0; e < 128; e += 2) {
-        const float p0 = ex2_approx(s[e] - m_use), p1 = ex2_approx(s[e + 1] - m_use);
-        rs += p0 + p1;
-        pk[e >> 1] = pack_f16x2(p0, p1);
-      }
-      l_run += rs;
-      // PV(i-1) must be done before P(i) replaces P(i-1) and before O is rescaled
-      if (i >= 1 && !wait_bar(o_done, i - 1, 207)) { ok = false; break; }
-      if (__any_sync(0xffffffffu, resc)) {
-        float o[32];
+        for (int k = 0; k < 8; ++k) rsp[k] = 0.f;
+        uint32_t pk[64];
 #pragma unroll
-        for (int hcol = 0; hcol < 64; hcol += 32) {
-          tmem_ld32(TM_O + lane_off + hcol, o);
-#pragma unroll
-          for (int d = 0; d < 32; ++d) o[d] *= alpha;
-          tmem_st32(TM_O + lane_off + hcol, reinterpret_cast<const uint32_t*>(o));
+        for (int e = 0; e < 128; e += 2) {
+          const float p0 = ex2_approx(fmaf(s[e], p.scale_log2, -m_use));
+          const float p1 = ex2_approx(fmaf(s[e + 1], p.scale_log2, -m_use));
+          rsp[(e >> 1) & 7] += p0 + p1;
+          pk[e >> 1] = pack_f16x2(p0, p1);
         }
-        l_run *= alpha;
+        l_run += ((rsp[0] + rsp[1]) + (rsp[2] + rsp[3])) + ((rsp[4] + rsp[5]) + (rsp[6] + rsp[7]));
+        // PV of the previous tile must be done before P is replaced and O rescaled
+        if (i >= 1 && !wait_bar(o_done, gi - 1, 207)) { ok = false; break; }
+        if (__any_sync(0xffffffffu, resc)) {
+          float o[32];
+#pragma unroll
+          for (int hcol = 0; hcol < 64; hcol += 32) {
+            tmem_ld32(TM_O + lane_off + hcol, o);
+#pragma unroll
+            for (int d = 0; d < 32; ++d) o[d] *= alpha;
+            tmem_st32(TM_O + lane_off + hcol, reinterpret_cast<const uint32_t*>(o));
+          }
+          l_run *= alpha;
+        }
+        tmem_st32(TM_P + lane_off, pk);
+        tmem_st32(TM_P + lane_off + 32, pk + 32);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full);
       }
-      tmem_st32(TM_P + lane_off, pk);
-      tmem_st32(TM_P + lane_off + 32, pk + 32);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(p_full);
-    }
-    if (ok && n_tiles > 0 && wait_bar(o_done, n_tiles - 1, 210)) {
+      if (!ok || n_tiles == 0) break;
+      if (!wait_bar(o_done, gi - 1, 210)) { ok = false; break; }
       float o[64];
       tmem_ld32(TM_O + lane_off, o);
       tmem_ld32(TM_O + lane_off + 32, o + 32);
+      tc_fence_before();
       if (qi < p.T) {
         const float inv = 1.f / l_run;
         float* dst = p.out + ((size_t)b * p.T + qi) * p.ld_out + h * 64;

@@ -308,7 +308,7 @@ int splits_for(int tiles, int k_blocks, int cap) {
 }
 
 struct PrefillWs {
-  size_t q, xz, xc, xcT, xbc, xbc_part, dT, y, o, u, sstate, cstate, rope, total;
+  size_t q, xz, xc, xcT, xbc, xbc_part, bcT, dT, y, o, u, sstate, cstate, rope, total;
   int T, Tp, xproj_split;
 };
 PrefillWs prefill_layout(const Dims& m, int B, int n_tokens, int x_has_meta) {
@@ -325,6 +325,7 @@ PrefillWs prefill_layout(const Dims& m, int B, int n_tokens, int x_has_meta) {
   w.xbc = take(rows * m.ld_xbc * 4);
   w.xproj_split = splits_for(cdiv((long long)rows, GEMM_BM), cdiv(m.Di, 64), 16);
   w.xbc_part = take((size_t)w.xproj_split * rows * m.ld_xbc * 4);
+  w.bcT = take((size_t)B * 32 * w.Tp * 4);
   w.dT = take((size_t)B * m.Di * w.Tp * 4);
   w.y = take(rows * m.Di * 2);
   w.o = take(rows * m.qw * 4);
@@ -658,7 +659,8 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     const int n = (int)(rows * m.ld_xbc);
     prof_begin("splitk_reduce", st);
     splitk_reduce_kernel<<<cdiv(n / 4, 256), 256, 0, st>>>(f32(L.xbc_part), L.xproj_split, (long long)n, n,
-                                                            nullptr, f32(L.xbc), 0);
+                                                            nullptr, f32(L.xbc), 0, f32(L.bcT), m.ld_xbc, T, L.Tp,
+                                                            m.R);
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
@@ -696,6 +698,7 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     AttnParams ap;
     ap.T = T; ap.Hq = m.Hq; ap.Hkv = m.Hkv; ap.n_meta = m.M; ap.window = m.W; ap.is_global = cfg->is_global;
     ap.q_tiles = cdiv(T, 128);
+    ap.n_items = ap.q_tiles * m.Hq * B;
     ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)m.D));
     ap.out = f32(L.o);
     ap.ld_out = m.qw;
@@ -707,9 +710,9 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
       HY_CUDA(cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ATT_SMEM));
       attr[d & 63] = true;
     }
-    dim3 grid(ap.q_tiles, m.Hq, B);
+    const int grid = ap.n_items < 2 * dev->sms ? ap.n_items : 2 * dev->sms;   // two persistent CTAs per SM
     prof_begin("attention", st);
-    attn_fwd_kernel<<<grid, ATT_THREADS, ATT_SMEM, st>>>(mq, mk, mv, ap);
+    attn_fwd_kernel<<<grid, ATT_THREADS, ATT_SMEM, st>>>(mq, mk, mv, ap, B);
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
@@ -726,9 +729,8 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
       attr_scan[dcur & 63] = true;
     }
     prof_begin("selective_scan", st);
-    selective_scan_kernel<<<grid, SCAN_THREADS, sizeof(ScanSmem), st>>>(bf(L.xcT), f32(L.dT), f32(L.xbc) + m.R,
-                                                                         m.ld_xbc, w->A, bf(L.y), sstate, T, L.Tp,
-                                                                         m.Di);
+    selective_scan_kernel<<<grid, SCAN_THREADS, sizeof(ScanSmem), st>>>(bf(L.xcT), f32(L.dT), f32(L.bcT), w->A,
+                                                                         bf(L.y), sstate, T, L.Tp, m.Di);
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }

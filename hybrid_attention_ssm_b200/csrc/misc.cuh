@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(128 * NORM_ROWS)
   __half* u_r = u + row * ld_u;
   // the whole row in registers: every load is issued before the first use
   float fo[NORM_MAXO][8], fy[NORM_MAXY][8];
-  float sa = 0.f, ss = 0.f;
+  uint4 rz[NORM_MAXY];
 #pragma unroll
   for (int k = 0; k < NORM_MAXO; ++k) {
     const int c = (t + k * 128) * 8;
@@ -81,12 +81,18 @@ __global__ void __launch_bounds__(128 * NORM_ROWS)
     const int c = (t + k * 128) * 8;
     if (live && c < di) {
       load8(y_r + c, fy[k]);
-      if (z != nullptr) {
-        float fz[8];
-        unpack8(*reinterpret_cast<const uint4*>(z_r + c), fz);
+      if (z != nullptr) rz[k] = *reinterpret_cast<const uint4*>(z_r + c);
+    }
+  }
+  float sa = 0.f, ss = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) fy[k][e] *= silu_f(fz[e]);
-      }
+  for (int k = 0; k < NORM_MAXY; ++k) {
+    const int c = (t + k * 128) * 8;
+    if (live && c < di && z != nullptr) {
+      float fz[8];
+      unpack8(rz[k], fz);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) fy[k][e] *= silu_f(fz[e]);
     }
   }
 #pragma unroll
@@ -518,9 +524,12 @@ __global__ void wait_timeout_selftest_kernel(DevStatus* st) {
 // Fixed-order sum of split-K partial slices: out[i] = sum_s part[s*stride + i] (+ residual),
 // as fp32 or bf16; n is a multiple of 4.  The order never changes, so results are
 // identical from run to run.
+// When bcT is set, columns [tr_col0, tr_col0 + 32) of the [rows, ld] result (rows = b*T + t)
+// are also written time-major to bcT [B][32][Tp] (the scan's B/C input).
 __global__ void splitk_reduce_kernel(const float* __restrict__ part, int n_split, long long stride, int n,
                                      const __nv_bfloat16* __restrict__ residual, void* __restrict__ out,
-                                     int out_bf16) {
+                                     int out_bf16, float* __restrict__ bcT = nullptr, int ld = 0, int T = 0,
+                                     int Tp = 0, int tr_col0 = 0) {
   const int i = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
   if (i >= n) return;
   float4 acc = *reinterpret_cast<const float4*>(part + i);
@@ -538,6 +547,16 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, int n_split
     *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
   } else {
     *reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + i) = acc;
+  }
+  if (bcT != nullptr) {
+    const int row = i / ld, col = i % ld;       // 4 columns of one row (ld % 4 == 0)
+    const int b = row / T, t = row % T;
+    const float vals[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int cc = col + e - tr_col0;
+      if (cc >= 0 && cc < 32) bcT[((size_t)b * 32 + cc) * Tp + t] = vals[e];
+    }
   }
 }
 

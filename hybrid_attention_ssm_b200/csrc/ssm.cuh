@@ -94,38 +94,39 @@ __global__ void __launch_bounds__(256)
 // ----------------------------------------------------------------------------------------
 // Selective scan, time-sequential per (channel, state) thread.
 //   h_t = exp(delta_t * A[c,s]) h_{t-1} + delta_t * B_t[s] * x_t ;  y_t = sum_s C_t[s] h_t[s]
-// CTA = 8 channels x 16 states.  The fp32 state stays in a register for the whole
-// sequence.  Inputs go through shared memory in chunks of 64 steps, 3 stages deep: delta,
-// delta*x (formed once per step and channel while staging) and B/C transposed to
-// [state][t] so each thread reads 4 steps per 128-bit load.  Each thread writes its
-// C_t[s] h_t[s] terms to a swizzled buffer; after the chunk, one thread per (4 steps,
-// channel) sums the 16 states (bank-conflict-free on both sides) and the y rows leave as
-// 16-byte stores.
-//   xcT [B, Di, Tp] bf16; dT [B, Di, Tp] fp32 (Tp: row stride, multiple of 8; steps at or
-//   beyond T read as zero, so delta = 0 leaves the state unchanged); bc [B*T, ld_bc] fp32
-//   (B at col 0..15, C at 16..31 of the pointer); A [Di, 16]; y [B*T, Di] bf16 (not gated);
-//   state [B, Di, 16].
+// CTA = 8 channels x 16 states; the fp32 state stays in a register for the whole sequence.
+// All inputs are time-major, so every chunk of 64 steps arrives by cp.async (16-byte
+// pieces, zero-filled past T) into a 4-stage ring, three chunks ahead of the compute.  In
+// each half chunk the 32 exponentials (and input terms) are issued before the sequential
+// FMA chain.  Each thread writes its C_t[s] h_t[s] terms to a swizzled buffer; after the
+// half chunk, one thread per (4 steps, channel) sums the 16 states (bank-conflict-free on
+// both sides) and the y rows leave as 16-byte stores.
+//   xcT [B, Di, Tp] bf16; dT [B, Di, Tp] fp32; bcT [B, 32, Tp] fp32 (B rows 0..15, C rows
+//   16..31); Tp is a multiple of 8 and steps at or beyond T read as zero, so delta = 0
+//   leaves the state unchanged; A [Di, 16]; y [B*T, Di] bf16 (not gated); state [B, Di, 16].
 // ----------------------------------------------------------------------------------------
 constexpr int SCAN_CH = 8;            // channels per CTA
 constexpr int SCAN_TC = 64;           // time steps per chunk
-constexpr int SCAN_NST = 3;           // pipeline stages
+constexpr int SCAN_NST = 4;           // pipeline stages
+constexpr int SCAN_HALF = 32;         // steps per compute/reduce round
 constexpr int SCAN_THREADS = SCAN_CH * 16;
 
 struct ScanStage {
   float d[SCAN_CH][SCAN_TC];          // delta
-  float dx[SCAN_CH][SCAN_TC];         // delta * x
-  float bcT[32][SCAN_TC + 4];         // [state (B 0..15, C 16..31)][t]
+  __nv_bfloat16 x[SCAN_CH][SCAN_TC];  // x
+  float bc[32][SCAN_TC + 4];          // [state (B 0..15, C 16..31)][t]; rows padded to 272 B so the
+                                      // 16 state lanes reading one step hit distinct banks
 };
 struct ScanSmem {
   ScanStage st[SCAN_NST];
-  float part[SCAN_TC / 4][16][SCAN_CH][4];   // C*h terms: [t/4][state][channel ^ (state&7)][t%4]
-  __nv_bfloat16 ys[SCAN_TC][SCAN_CH];
+  float part[SCAN_HALF / 4][16][SCAN_CH][4];   // C*h terms: [t/4][state][channel ^ (state&7)][t%4]
+  __nv_bfloat16 ys[SCAN_HALF][SCAN_CH];
 };
 
 __global__ void __launch_bounds__(SCAN_THREADS)
     selective_scan_kernel(const __nv_bfloat16* __restrict__ xcT, const float* __restrict__ dT,
-                          const float* __restrict__ bc, int ld_bc, const float* __restrict__ A,
-                          __nv_bfloat16* __restrict__ y, float* __restrict__ state, int T, int Tp, int Di) {
+                          const float* __restrict__ bcT, const float* __restrict__ A, __nv_bfloat16* __restrict__ y,
+                          float* __restrict__ state, int T, int Tp, int Di) {
   extern __shared__ __align__(16) uint8_t scan_smem_raw[];
   ScanSmem& sm = *reinterpret_cast<ScanSmem*>(scan_smem_raw);
   const int tid = threadIdx.x;
@@ -137,111 +138,86 @@ __global__ void __launch_bounds__(SCAN_THREADS)
   const int n_chunks = (T + SCAN_TC - 1) / SCAN_TC;
   const float A2 = A[(size_t)c * 16 + s] * 1.4426950408889634f;   // exp(d*A) = 2^(d*A*log2 e)
 
-  // staging of chunk k through registers: thread -> (channel lch, 4 steps lq*4..) for
-  // delta and x, and (row, 16 of B|C) for the B/C rows
-  const int lch = tid >> 4, lq = tid & 15;
-  float4 rd;
-  uint2 rx;
-  float rbc[16];
+  // cp.async of chunk k: delta 8 rows x 16 pieces, x 8 rows x 8 pieces, B/C 32 rows x 16
+  // pieces = 704 pieces of 16 bytes, 5.5 per thread
   auto load_chunk = [&](int k) {
-    const int t = k * SCAN_TC + lq * 4;
-    const size_t row = ((size_t)b * Di + c0 + lch) * Tp;
-    rd = make_float4(0.f, 0.f, 0.f, 0.f);
-    rx = make_uint2(0u, 0u);
-    if (t + 4 <= T) {
-      rd = *reinterpret_cast<const float4*>(dT + row + t);
-      rx = *reinterpret_cast<const uint2*>(xcT + row + t);
-    } else {
-      float dd[4] = {0.f, 0.f, 0.f, 0.f};
-      __nv_bfloat16 xx[4] = {__float2bfloat16_rn(0.f), __float2bfloat16_rn(0.f), __float2bfloat16_rn(0.f),
-                             __float2bfloat16_rn(0.f)};
-      for (int e = 0; e < 4; ++e)
-        if (t + e < T) {
-          dd[e] = dT[row + t + e];
-          xx[e] = xcT[row + t + e];
-        }
-      rd = make_float4(dd[0], dd[1], dd[2], dd[3]);
-      rx = *reinterpret_cast<const uint2*>(xx);
-    }
-    const int brow = tid >> 1, half = (tid & 1) * 16;
-    const int tb = k * SCAN_TC + brow;
-#pragma unroll
-    for (int e = 0; e < 16; e += 4) {
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (tb < T) v = *reinterpret_cast<const float4*>(bc + ((size_t)b * T + tb) * ld_bc + half + e);
-      rbc[e] = v.x; rbc[e + 1] = v.y; rbc[e + 2] = v.z; rbc[e + 3] = v.w;
-    }
-  };
-  auto store_chunk = [&](int k) {
     ScanStage& S = sm.st[k % SCAN_NST];
-    const __nv_bfloat16* xh = reinterpret_cast<const __nv_bfloat16*>(&rx);
-    *reinterpret_cast<float4*>(&S.d[lch][lq * 4]) = rd;
-    *reinterpret_cast<float4*>(&S.dx[lch][lq * 4]) =
-        make_float4(rd.x * __bfloat162float(xh[0]), rd.y * __bfloat162float(xh[1]), rd.z * __bfloat162float(xh[2]),
-                    rd.w * __bfloat162float(xh[3]));
-    const int brow = tid >> 1, half = (tid & 1) * 16;
-#pragma unroll
-    for (int e = 0; e < 16; ++e) S.bcT[half + e][brow] = rbc[e];
+    const int t0 = k * SCAN_TC;
+    for (int i = tid; i < 704; i += SCAN_THREADS) {
+      if (i < 128) {
+        const int ch = i >> 4, pc = i & 15, t = t0 + pc * 4;
+        const int nb = t >= T ? 0 : min(16, (T - t) * 4);
+        cp_async16(&S.d[ch][pc * 4], dT + ((size_t)b * Di + c0 + ch) * Tp + (t >= T ? 0 : t), nb);
+      } else if (i < 192) {
+        const int j = i - 128, ch = j >> 3, pc = j & 7, t = t0 + pc * 8;
+        const int nb = t >= T ? 0 : min(16, (T - t) * 2);
+        cp_async16(&S.x[ch][pc * 8], xcT + ((size_t)b * Di + c0 + ch) * Tp + (t >= T ? 0 : t), nb);
+      } else {
+        const int j = i - 192, r = j >> 4, pc = j & 15, t = t0 + pc * 4;
+        const int nb = t >= T ? 0 : min(16, (T - t) * 4);
+        cp_async16(&S.bc[r][pc * 4], bcT + ((size_t)b * 32 + r) * Tp + (t >= T ? 0 : t), nb);
+      }
+    }
   };
 
-  // prologue: chunks 0 .. NST-2
-  for (int k = 0; k < SCAN_NST - 1 && k < n_chunks; ++k) {
-    load_chunk(k);
-    store_chunk(k);
+  for (int k = 0; k < SCAN_NST - 1; ++k) {
+    if (k < n_chunks) load_chunk(k);
+    cp_async_commit();
   }
   float h = 0.f;
   const int sw = s & 7;
   for (int k = 0; k < n_chunks; ++k) {
-    const int kn = k + SCAN_NST - 1;
-    __syncthreads();                       // chunk k staged; its part/ys buffers free
-    if (kn < n_chunks) load_chunk(kn);     // in flight during the compute below
+    cp_async_wait<SCAN_NST - 2>();
+    __syncthreads();                       // chunk k visible; the stage of chunk k-1 is free
+    if (k + SCAN_NST - 1 < n_chunks) load_chunk(k + SCAN_NST - 1);
+    cp_async_commit();
     const ScanStage& S = sm.st[k % SCAN_NST];
-#pragma unroll 2
-    for (int tt = 0; tt < SCAN_TC; tt += 8) {
-      const float4 d0 = *reinterpret_cast<const float4*>(&S.d[cl][tt]);
-      const float4 d1 = *reinterpret_cast<const float4*>(&S.d[cl][tt + 4]);
-      const float4 q0 = *reinterpret_cast<const float4*>(&S.dx[cl][tt]);
-      const float4 q1 = *reinterpret_cast<const float4*>(&S.dx[cl][tt + 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&S.bcT[s][tt]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&S.bcT[s][tt + 4]);
-      const float4 e0 = *reinterpret_cast<const float4*>(&S.bcT[16 + s][tt]);
-      const float4 e1 = *reinterpret_cast<const float4*>(&S.bcT[16 + s][tt + 4]);
-      const float dv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-      const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-      const float cv[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
-      float a[8], v[8];
+#pragma unroll 1
+    for (int hc = 0; hc < SCAN_TC; hc += SCAN_HALF) {
+      float a[SCAN_HALF], q[SCAN_HALF];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) a[u] = ex2_approx(dv[u] * A2);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        h = fmaf(a[u], h, qv[u] * bv[u]);
-        v[u] = cv[u] * h;
+      for (int u = 0; u < SCAN_HALF; u += 4) {
+        const float4 d4 = *reinterpret_cast<const float4*>(&S.d[cl][hc + u]);
+        const uint2 x2 = *reinterpret_cast<const uint2*>(&S.x[cl][hc + u]);
+        const float4 b4 = *reinterpret_cast<const float4*>(&S.bc[s][hc + u]);
+        const __nv_bfloat162 xa = *reinterpret_cast<const __nv_bfloat162*>(&x2.x);
+        const __nv_bfloat162 xb = *reinterpret_cast<const __nv_bfloat162*>(&x2.y);
+        a[u] = ex2_approx(d4.x * A2); a[u + 1] = ex2_approx(d4.y * A2);
+        a[u + 2] = ex2_approx(d4.z * A2); a[u + 3] = ex2_approx(d4.w * A2);
+        q[u] = d4.x * __low2float(xa) * b4.x; q[u + 1] = d4.y * __high2float(xa) * b4.y;
+        q[u + 2] = d4.z * __low2float(xb) * b4.z; q[u + 3] = d4.w * __high2float(xb) * b4.w;
       }
-      *reinterpret_cast<float4*>(&sm.part[tt >> 2][s][cl ^ sw][0]) = make_float4(v[0], v[1], v[2], v[3]);
-      *reinterpret_cast<float4*>(&sm.part[(tt >> 2) + 1][s][cl ^ sw][0]) = make_float4(v[4], v[5], v[6], v[7]);
-    }
-    if (kn < n_chunks) store_chunk(kn);
-    __syncthreads();
-    // sum over the 16 states: thread -> (4 steps tg, channel ch)
-    {
-      const int tg = tid >> 3, ch = tid & 7;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int st = 0; st < 16; ++st) {
-        const float4 q = *reinterpret_cast<const float4*>(&sm.part[tg][st][ch ^ (st & 7)][0]);
-        acc.x += q.x; acc.y += q.y; acc.z += q.z; acc.w += q.w;
+      for (int u = 0; u < SCAN_HALF; u += 4) {
+        const float4 c4 = *reinterpret_cast<const float4*>(&S.bc[16 + s][hc + u]);
+        float4 v;
+        h = fmaf(a[u], h, q[u]); v.x = c4.x * h;
+        h = fmaf(a[u + 1], h, q[u + 1]); v.y = c4.y * h;
+        h = fmaf(a[u + 2], h, q[u + 2]); v.z = c4.z * h;
+        h = fmaf(a[u + 3], h, q[u + 3]); v.w = c4.w * h;
+        *reinterpret_cast<float4*>(&sm.part[u >> 2][s][cl ^ sw][0]) = v;
       }
-      sm.ys[tg * 4 + 0][ch] = __float2bfloat16_rn(acc.x);
-      sm.ys[tg * 4 + 1][ch] = __float2bfloat16_rn(acc.y);
-      sm.ys[tg * 4 + 2][ch] = __float2bfloat16_rn(acc.z);
-      sm.ys[tg * 4 + 3][ch] = __float2bfloat16_rn(acc.w);
-    }
-    __syncthreads();
-    if (tid < SCAN_TC) {
-      const int t = k * SCAN_TC + tid;
-      if (t < T)
-        *reinterpret_cast<uint4*>(y + ((size_t)b * T + t) * Di + c0) = *reinterpret_cast<const uint4*>(&sm.ys[tid][0]);
+      __syncthreads();
+      // sum over the 16 states: thread -> (4 steps tg, channel ch), 8 x 8 = 64 threads
+      if (tid < 64) {
+        const int tg = tid >> 3, ch = tid & 7;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int st = 0; st < 16; ++st) {
+          const float4 q4 = *reinterpret_cast<const float4*>(&sm.part[tg][st][ch ^ (st & 7)][0]);
+          acc.x += q4.x; acc.y += q4.y; acc.z += q4.z; acc.w += q4.w;
+        }
+        sm.ys[tg * 4 + 0][ch] = __float2bfloat16_rn(acc.x);
+        sm.ys[tg * 4 + 1][ch] = __float2bfloat16_rn(acc.y);
+        sm.ys[tg * 4 + 2][ch] = __float2bfloat16_rn(acc.z);
+        sm.ys[tg * 4 + 3][ch] = __float2bfloat16_rn(acc.w);
+      }
+      __syncthreads();
+      if (tid < SCAN_HALF) {
+        const int t = k * SCAN_TC + hc + tid;
+        if (t < T)
+          *reinterpret_cast<uint4*>(y + ((size_t)b * T + t) * Di + c0) = *reinterpret_cast<const uint4*>(&sm.ys[tid][0]);
+      }
     }
   }
   state[((size_t)b * Di + c) * 16 + s] = h;
