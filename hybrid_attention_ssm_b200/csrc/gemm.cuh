@@ -20,7 +20,7 @@ enum EpiMode : int {
   EPI_SOFTPLUS = 3,     // fp32 store of softplus(acc + bias[col])
   EPI_BF16_T = 4,       // transposed bf16 store: out[n][m] (weights as the M operand)
   EPI_ATOMIC_F32_T = 5, // transposed fp32 atomic add
-  EPI_SWIGLU = 6,       // columns interleaved [gate(32) | up(32)] -> bf16 SiLU(gate)*up
+  EPI_SWIGLU = 6,       // columns interleaved [gate(32) | up(32)] -> fp16 SiLU(gate)*up
   EPI_SOFTPLUS_T = 7,   // fp32 softplus(acc + bias[col]) stored time-major: out[(b*N + col)*T_out + row]
   EPI_F32_T = 8,        // transposed fp32 store: out[n][m]
   EPI_F32_PART = 9,     // fp32 store of split ks's partial sum at out + ks*split_stride (row-major)
@@ -284,10 +284,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           float* v = reinterpret_cast<float*>(r);
           const int gc = col_base + c0;
           if (!row_ok || gc >= p.N) continue;
-          if (p.mode == EPI_SWIGLU) {
+          if (p.mode == EPI_SWIGLU) {   // fp16 activations (the down projection runs in fp16)
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = silu_f(v[e]) * v[e + 32];
-            store_bf16_row(reinterpret_cast<__nv_bfloat16*>(p.out) + orow * p.ld_out + gc / 2, v, 32);
+            store_f16_row(reinterpret_cast<__half*>(p.out) + orow * p.ld_out + gc / 2, v, 32);
             continue;
           }
           int si = 0;

@@ -975,8 +975,8 @@ int hymba_rmsnorm(const hymba_bf16* x, const float* gain, int rows, int d, float
   return HYMBA_OK;
 }
 
-int hymba_ffn_swiglu(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hymba_bf16* w_down, int rows, int d,
-                     int F, hymba_bf16* act, const hymba_bf16* residual, hymba_bf16* out, void* status_ws,
+int hymba_ffn_swiglu(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hymba_f16* w_down, int rows, int d,
+                     int F, hymba_f16* act, const hymba_bf16* residual, hymba_bf16* out, void* status_ws,
                      hymba_stream stream) {
   DeviceInfo* dev = nullptr;
   HY_TRY(device_info(&dev));
@@ -1001,6 +1001,7 @@ int hymba_ffn_swiglu(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hym
     GemmCall c;
     c.a1 = act; c.nb1 = 1; c.rows1 = rows; c.lda1 = F; c.a1_bstride = (long long)rows * F;
     c.b = w_down; c.N = d; c.ldb = F; c.K = F;
+    c.etype = ET_F16;
     c.name = "ffn_down";
     c.bn = pick_bn_wide(cdiv(rows, GEMM_BM), d, dev->sms);
     c.p.mode = EPI_BF16;
@@ -1012,6 +1013,24 @@ int hymba_ffn_swiglu(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hym
     c.p.status = reinterpret_cast<DevStatus*>(status_ws);
     HY_TRY(run_gemm(c, *dev, st));
   }
+  return HYMBA_OK;
+}
+
+int hymba_prepend_meta(const hymba_bf16* meta, const hymba_bf16* x, int batch, int n_meta, int n_tokens, int d,
+                       hymba_bf16* out, hymba_stream stream) {
+  if ((n_meta > 0 && meta == nullptr) || x == nullptr || out == nullptr || batch < 1 || n_meta < 0 ||
+      n_tokens < 0 || d < 8 || d % 8 || (meta != nullptr && !aligned16(meta)) || !aligned16(x) || !aligned16(out))
+    return fail(HYMBA_ERR_INVALID_ARG, "prepend_meta arguments");
+  const long long total = (long long)batch * (n_meta + n_tokens) * (d / 8);
+  if (total == 0) return HYMBA_OK;
+  const int grid = (int)((total + 255) / 256 < 4096 ? (total + 255) / 256 : 4096);
+  prof_begin("prepend_meta", (cudaStream_t)stream);
+  prepend_meta_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<const __nv_bfloat16*>(meta),
+                                                               reinterpret_cast<const __nv_bfloat16*>(x), batch,
+                                                               n_meta, n_tokens, d,
+                                                               reinterpret_cast<__nv_bfloat16*>(out));
+  prof_end((cudaStream_t)stream);
+  HY_CUDA(cudaGetLastError());
   return HYMBA_OK;
 }
 

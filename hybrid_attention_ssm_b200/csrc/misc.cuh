@@ -509,6 +509,22 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// out[b] = [meta; x[b]] : meta [M, d], x [B, N, d] -> out [B, M+N, d] (16-byte pieces)
+__global__ void prepend_meta_kernel(const __nv_bfloat16* __restrict__ meta, const __nv_bfloat16* __restrict__ x,
+                                    int B, int M, int N, int d, __nv_bfloat16* __restrict__ out) {
+  const int vec = d / 8;
+  const long long total = (long long)B * (M + N) * vec;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int v = (int)(i % vec);
+    const long long rowg = i / vec;
+    const int t = (int)(rowg % (M + N));
+    const int b = (int)(rowg / (M + N));
+    const __nv_bfloat16* src = t < M ? meta + (size_t)t * d : x + ((size_t)b * N + (t - M)) * d;
+    *reinterpret_cast<uint4*>(out + rowg * d + v * 8) = *reinterpret_cast<const uint4*>(src + v * 8);
+  }
+}
+
 // Waits on a barrier that nothing arrives at, through the same bounded wait the pipelined
 // kernels use; the wait runs out and records DEV_ERR_TIMEOUT.
 __global__ void wait_timeout_selftest_kernel(DevStatus* st) {

@@ -97,6 +97,7 @@ def lib():
             "hymba_rmsnorm": ([_vp, _vp, _c_int, _c_int, ctypes.c_float, _vp, _vp], _c_int),
             "hymba_ffn_swiglu": ([_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp], _c_int),
             "hymba_set_wait_limit_ns": ([ctypes.c_ulonglong], _c_int),
+            "hymba_prepend_meta": ([_vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp], _c_int),
             "hymba_selftest_wait_timeout": ([_vp, _c_size, _vp], _c_int),
             "hymba_mixer_decode_noalloc": ([ctypes.POINTER(LayerCfg), ctypes.POINTER(LayerWeights), _vp, _c_int,
                                             _c_int, ctypes.POINTER(KVCache), _vp, _vp, _vp, _vp, _vp], _c_int),
@@ -270,6 +271,13 @@ def ffn_swiglu(h, w_gate_up, w_down, act, out, status_ws, residual=None, stream=
     F = w_down.shape[1]
     check(lib().hymba_ffn_swiglu(ptr(h), ptr(w_gate_up), ptr(w_down), rows, d, F, ptr(act), ptr(residual),
                                  ptr(out), ptr(status_ws), stream_handle(stream)))
+
+
+def prepend_meta(meta, x, out, stream=None):
+    """out[b] = [meta; x[b]] (bf16, on the device)."""
+    B, N, d = x.shape
+    M = 0 if meta is None else meta.shape[0]
+    check(lib().hymba_prepend_meta(ptr(meta), ptr(x), B, M, N, d, ptr(out), stream_handle(stream)))
 
 
 def interleave_gate_up(w_gate, w_up):

@@ -1,0 +1,98 @@
+"""A stack of Hymba blocks on the C ABI (the 32-layer harness).
+
+Each block is norm -> hybrid-head mixer -> norm -> FFN with pre-norm residuals (juejin post
+"NVIDIA提出Hymba网络…", §Hymba 的整体架构).  The meta tokens are prepended once, to the
+residual stream, and every layer sees them as the first rows of its input; the first,
+middle and last layers attend globally, the others use a sliding window, and adjacent SWA
+layers share one KV cache (hymba_kv_share_alloc plans the pairs).  This module only
+allocates device memory and calls the library: every step runs in libhymba's kernels.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import hymba as H
+from . import synth
+
+
+class HymbaStack:
+    def __init__(self, wl: synth.Workload, seed: int = 0, device="cuda", keep_host_weights=False):
+        self.wl = wl
+        dims = wl.dims
+        self.B, self.N = wl.batch, wl.n_tokens
+        self.T = dims.n_meta + self.N
+        self.L = wl.n_layers
+        self.F = wl.ffn_dim
+        self.device = device
+        is_global = [1 if i in wl.global_layers else 0 for i in range(self.L)]
+        need, _, _, _ = H.kv_share_alloc(dims, is_global, self.B, self.T)
+        raw = torch.empty(need + 256, dtype=torch.uint8, device=device)
+        off = (-raw.data_ptr()) % 256
+        self._cache_raw = raw
+        self.cache_buf = raw[off:off + need]
+        _, self.cache_id, self.role, caches = H.kv_share_alloc(dims, is_global, self.B, self.T, self.cache_buf)
+        self.caches = []
+        for c in caches:
+            holder = H.Cache.__new__(H.Cache)
+            holder.t = {}
+            holder.c = c
+            self.caches.append(holder)
+        self.layers = []
+        self.host = [] if keep_host_weights else None
+        for l in range(self.L):
+            dl = dims.replace(is_global=is_global[l], kv_role=self.role[l])
+            w = synth.layer_weights(dl, seed=seed, layer=l, dt_bias_mean=wl.dt_bias_mean, dt_bias_std=wl.dt_bias_std)
+            bw = synth.block_weights(dl, self.F, seed=seed, layer=l)
+            dev = {
+                "g1": torch.from_numpy(bw["g_norm1"]).to(device),
+                "g2": torch.from_numpy(bw["g_norm2"]).to(device),
+                "w_gu": torch.from_numpy(H.interleave_gate_up(bw["w_gate"], bw["w_up"])).to(device).to(torch.bfloat16),
+                "w_down": torch.from_numpy(bw["w_down"]).to(device).to(torch.float16),
+            }
+            self.layers.append((dl, H.DeviceWeights(w), dev))
+            if keep_host_weights:
+                self.host.append((dl, w, bw))
+        # the stack's meta tokens R (those of layer 0's parameter set)
+        self.meta = torch.from_numpy(synth.layer_weights(dims, seed=seed, layer=0)["meta"]).to(device).to(torch.bfloat16)
+        rows = self.B * self.T
+        bf = dict(dtype=torch.bfloat16, device=device)
+        self.Hs = [torch.empty(self.B, self.T, dims.d_model, **bf) for _ in range(2)]
+        self.H1 = torch.empty(self.B, self.T, dims.d_model, **bf)
+        self.hn = torch.empty(self.B, self.T, dims.d_model, **bf)
+        self.act = torch.empty(rows, self.F, dtype=torch.float16, device=device)
+        ws_bytes = max(H.workspace_size(dl, self.B, self.T, 1) for dl, _, _ in self.layers)
+        self.ws = H.alloc_workspace(ws_bytes)
+
+    def cache_view(self, ptr_value, max_tokens, dl):
+        """fp16 view [B, max_tokens, Hkv, D] of a K or V buffer carved out of cache_buf."""
+        off = ptr_value - self.cache_buf.data_ptr()
+        n = self.B * max_tokens * dl.n_kv_heads * dl.head_dim * 2
+        return self.cache_buf[off:off + n].view(torch.float16).view(self.B, max_tokens, dl.n_kv_heads, dl.head_dim)
+
+    def forward(self, E, record=None):
+        """E [B, N, d] bf16 on the device -> residual stream after the last layer [B, T, d].
+        record: optional dict layer -> list, filled with (H_in, H_mid, H_out) copies of
+        sequence 0 and, for consumer layers, the producer K/V they read."""
+        d = self.wl.dims.d_model
+        cur = 0
+        H.prepend_meta(self.meta, E, self.Hs[cur])
+        for l, (dl, dw, dev) in enumerate(self.layers):
+            Hin = self.Hs[cur]
+            Hout = self.Hs[1 - cur]
+            kv = self.caches[self.cache_id[l]]
+            rows = self.B * self.T
+            if record is not None and l in record and dl.kv_role == H.KV_CONSUMER:
+                view_k = self.cache_view(kv.c.k, kv.c.max_tokens, dl)
+                view_v = self.cache_view(kv.c.v, kv.c.max_tokens, dl)
+                record[l].append(("kv", view_k[0, :self.T].float().cpu().numpy(),
+                                  view_v[0, :self.T].float().cpu().numpy()))
+            H.rmsnorm(Hin.view(rows, d), dev["g1"], dl.norm_eps, self.hn.view(rows, d))
+            H.mixer_prefill(dl, dw, self.hn, kv, self.H1, self.ws, x_has_meta=1, residual=Hin)
+            H.rmsnorm(self.H1.view(rows, d), dev["g2"], dl.norm_eps, self.hn.view(rows, d))
+            H.ffn_swiglu(self.hn.view(rows, d), dev["w_gu"], dev["w_down"], self.act, Hout.view(rows, d), self.ws,
+                         residual=self.H1.view(rows, d))
+            if record is not None and l in record:
+                record[l].append(("h", Hin[0].float().cpu().numpy(), self.H1[0].float().cpu().numpy(),
+                                  Hout[0].float().cpu().numpy()))
+            cur = 1 - cur
+        return self.Hs[cur]

@@ -239,10 +239,18 @@ int hymba_rmsnorm(const hymba_bf16* x, const float* gain, int rows, int d, float
 /* SwiGLU FFN with residual: out = residual + W_down (SiLU(W_gate h) * (W_up h)).
  *   h [rows, d] bf16; w_gate_up [2F, d] bf16 with gate and up rows interleaved in blocks of
  *   32 (rows 64i..64i+31 = gate rows 32i.., rows 64i+32..64i+63 = up rows 32i..);
- *   w_down [d, F] bf16; act [rows, F] bf16 scratch; residual [rows, d] or NULL; F % 64 == 0. */
-int hymba_ffn_swiglu(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hymba_bf16* w_down, int rows, int d,
-                     int F, hymba_bf16* act, const hymba_bf16* residual, hymba_bf16* out, void* status_ws,
+ *   w_down [d, F] fp16; act [rows, F] fp16 scratch (the activations feed the down
+ *   projection in fp16, 8x finer than bf16 for these O(1) values); residual [rows, d] bf16 or
+ *   NULL; out [rows, d] bf16; F % 64 == 0, d % 8 == 0. */
+int hymba_ffn_swiglu(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hymba_f16* w_down, int rows, int d,
+                     int F, hymba_f16* act, const hymba_bf16* residual, hymba_bf16* out, void* status_ws,
                      hymba_stream stream);
+
+/* Meta-token prefix of a stack's residual stream ([JJ] §数学表示 1: X~ = [R, X]):
+ * out[b] = [meta; x[b]], meta [n_meta, d], x [B, n_tokens, d], out [B, n_meta + n_tokens, d],
+ * all bf16, d % 8 == 0. */
+int hymba_prepend_meta(const hymba_bf16* meta, const hymba_bf16* x, int batch, int n_meta, int n_tokens, int d,
+                       hymba_bf16* out, hymba_stream stream);
 
 /* Upper bound, in nanoseconds, of every device-side wait on an mbarrier (default 2e9).
  * A wait that runs out records HYMBA_ERR_TIMEOUT in the status word and the kernel returns. */
