@@ -28,6 +28,38 @@ sys.path.insert(0, ROOT)
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 
 
+# ---------------------------------------------------------------------------------------
+# rank plumbing (replicas: no collective on the data path; these only synchronise and
+# reduce the timings)
+# ---------------------------------------------------------------------------------------
+def dist_env():
+    """(world, rank, local_rank) from the torchrun environment (1, 0, 0 when absent)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def barrier(world):
+    if world > 1:
+        import torch
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world, device):
+    """The largest value of x over all ranks (every rank gets it); x on one rank if world == 1."""
+    if world <= 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world, units_per_step_per_rank, ms_per_step):
+    """Units per second over all ranks: every rank processes its own units in the step time
+    (the max over ranks), weak scaling."""
+    return world * units_per_step_per_rank / (ms_per_step * 1e-3)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -149,6 +181,36 @@ class ClockSampler:
 # ---------------------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------------------
+def profile_kernels(step, n, flush, stream):
+    """Per-kernel device times of `step`: the step is captured once into a CUDA graph with
+    an event pair around every kernel the library launches, then replayed n times (L2
+    flushed before each replay); every replay re-records the events.  Returns [(name, ms)]
+    over all replays, free of host launch gaps."""
+    import torch
+    from hybrid_attention_ssm_b200 import hymba as H
+
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        step()
+        torch.cuda.synchronize()
+        H.profile_begin(4096)
+        with torch.cuda.graph(g, stream=side):
+            step()
+    torch.cuda.synchronize()
+    recs = []
+    for _ in range(n):
+        flush.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        recs += H.profile_read()
+    H.profile_end()
+    del g
+    torch.cuda.synchronize()
+    return recs
+
+
 def run_hymba(args, rank, world, device):
     import torch
     from hybrid_attention_ssm_b200 import build as hbuild
@@ -179,11 +241,9 @@ def run_hymba(args, rank, world, device):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
+    barrier(world)
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    H.profile_begin(64 * args.steps + 64)
     with ClockSampler(device.index if device.index is not None else 0) as clk:
         for i in range(args.steps):
             flush.zero_()                        # evict L2 between steps (not timed)
@@ -191,18 +251,14 @@ def run_hymba(args, rank, world, device):
             step()
             ev[i][1].record(stream)
         torch.cuda.synchronize()
-    recs = H.profile_end(64 * args.steps + 64)
-    if world > 1:
-        torch.distributed.barrier()
+        # per-kernel times: the same step as a graph with events around each kernel
+        recs = profile_kernels(step, args.steps, flush, stream)
+    barrier(world)
     torch.cuda.synchronize()
     assert H.status_read(ws) == 0, "device-side wait timed out"
     assert torch.isfinite(out.float()).all().item(), "non-finite output"
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = float(sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(sum(step_ms)), world, device)
     ms_per_step = total_ms / args.steps
 
     # per-kernel durations from the events around each launch in the timed region
@@ -244,7 +300,7 @@ def run_hymba(args, rank, world, device):
     step_roof = {"tensor_gflop_per_step": round(tensor_flops / 1e9, 2),
                  "achieved_tflops": round(tensor_flops / (ms_per_step * 1e-3) / 1e12, 1),
                  "frac_of_tensor_peak": round(tensor_flops / (ms_per_step * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
-    launches_per_step = len(recs) / args.steps
+    launches_per_step = len(recs) / args.steps   # kernels the library launched per step
 
     # ---------------- e2e: host buffers through the C ABI ----------------
     if args.no_e2e:
@@ -266,11 +322,7 @@ def run_hymba(args, rank, world, device):
         oh.copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, device)
 
     decode = None if args.no_decode else run_decode(args, device, world)
     res = {
@@ -320,17 +372,16 @@ def run_decode(args, device, world):
     torch.cuda.synchronize()
     n_steps = max(10, args.steps)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
-    # eager, profiled: per-kernel durations
+    # eager (host-launched) step time, for reference
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_steps)]
-    H.profile_begin(64 * n_steps + 64)
     for i in range(n_steps):
         flush.zero_()
         ev[i][0].record(stream)
         step()
         ev[i][1].record(stream)
     torch.cuda.synchronize()
-    recs = H.profile_end(64 * n_steps + 64)
     eager_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    recs = profile_kernels(step, n_steps, flush, stream)
     # CUDA graph of one step (the ABI calls are capturable: no sync, no allocation)
     g = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream()
@@ -348,11 +399,7 @@ def run_decode(args, device, world):
         g.replay()
         gev[i][1].record(stream)
     torch.cuda.synchronize()
-    graph_ms = float(np.mean([a.elapsed_time(b) for a, b in gev]))
-    if world > 1:
-        t = torch.tensor([graph_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        graph_ms = float(t.item())
+    graph_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in gev])), world, device)
     for L in layers:
         assert H.status_read(L["ws"]) == 0
     per = {}
@@ -378,15 +425,120 @@ def run_decode(args, device, world):
     roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
     roof["traffic"] = TRAFFIC.get(dom)
     return {
-        "metric": "decode steps/s (shared-KV SWA layer pair)", "value": round(1000.0 / graph_ms, 1),
+        "metric": "decode steps/s (shared-KV SWA layer pair)", "value": round(whole_job_rate(world, 1, graph_ms), 1),
         "unit": "steps/s", "ms_per_step": round(graph_ms, 5), "eager_ms_per_step": round(eager_ms, 5),
-        "tokens_per_s": round(B * 1000.0 / graph_ms, 1), "timing": "CUDA graph of the two C-ABI calls, L2 flushed",
+        "tokens_per_s": round(whole_job_rate(world, B, graph_ms), 1), "timing": "CUDA graph of the two C-ABI calls, L2 flushed",
         "config": {"workload": "decode_pair", "batch": B, "position": p, "window": prod.window,
                    "n_meta": prod.n_meta, "kv_heads": prod.n_kv_heads},
         "step_bytes": bytes_total, "step_hbm_gbs": round(bytes_total / (graph_ms * 1e-3) / 1e9, 1),
         "step_hbm_frac": round(bytes_total / (graph_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
         "roofline": roof, "kernels": kern, "launches_per_step": len(recs) / n_steps,
     }
+
+
+def run_global(args, device, world):
+    """One global-attention layer at batch 4, 128 + 8192 tokens (full causal attention)."""
+    import torch
+    from hybrid_attention_ssm_b200 import hymba as H
+    from hybrid_attention_ssm_b200 import synth
+
+    wl = synth.workloads()["global"]
+    dims = wl.dims
+    B, N = wl.batch, wl.n_tokens
+    T = dims.n_meta + N
+    w = synth.layer_weights(dims, seed=0, dt_bias_mean=wl.dt_bias_mean, dt_bias_std=wl.dt_bias_std)
+    dw = H.DeviceWeights(w)
+    g = torch.Generator(device=device)
+    g.manual_seed(7)
+    x = torch.randn(B, N, dims.d_model, generator=g, device=device).to(torch.bfloat16)
+    cache = H.Cache(dims, B, T)
+    out = torch.empty(B, T, dims.d_model, dtype=torch.bfloat16, device=device)
+    ws = H.alloc_workspace(H.workspace_size(dims, B, N))
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        H.mixer_prefill(dims, dw, x, cache, out, ws)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    n = max(3, min(args.steps, 10))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i in range(n):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in ev])), world, device)
+    recs = profile_kernels(step, 2, flush, stream)
+    assert H.status_read(ws) == 0
+    work, _ = prefill_work(dims, B, T)
+    per = {}
+    for name, t in recs:
+        per.setdefault(name, []).append(t)
+    kern = {k: {"avg_us": round(float(np.mean(v)) * 1e3, 1)} for k, v in per.items()}
+    for k, (bound, amount) in work.items():
+        if k in kern and bound == "tensor" and amount > 0:
+            kern[k]["tflops"] = round(amount / (kern[k]["avg_us"] * 1e-6) / 1e12, 1)
+    flops = sum(a for k, (b, a) in work.items() if b == "tensor")
+    peaks = load_peaks()
+    return {"workload": "global_layer_prefill", "batch": B, "seq_len": T, "ms_per_step": round(ms, 4),
+            "tokens_per_s": round(whole_job_rate(world, B * T, ms), 1),
+            "tensor_gflop_per_step": round(flops / 1e9, 1),
+            "frac_of_tensor_peak": round(flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+            "kernels": kern}
+
+
+def run_stack(args, device, world):
+    """The 32-layer stack (batch 8, 128 + 4096 tokens): mixer and FFN timed separately."""
+    import torch
+    from hybrid_attention_ssm_b200 import hymba as H
+    from hybrid_attention_ssm_b200 import synth
+    from hybrid_attention_ssm_b200.stack import HymbaStack
+
+    wl = synth.workloads()["stack"]
+    st = HymbaStack(wl, device=device, device_init=True)
+    g = torch.Generator(device=device)
+    g.manual_seed(11)
+    E = torch.randn(st.B, st.N, wl.dims.d_model, generator=g, device=device).to(torch.bfloat16)
+    stream = torch.cuda.current_stream()
+    st.forward(E)
+    torch.cuda.synchronize()
+    n = max(2, min(args.steps, 3))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i in range(n):
+        ev[i][0].record(stream)
+        st.forward(E)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in ev])), world, device)
+    H.profile_begin(4096)
+    st.forward(E)
+    torch.cuda.synchronize()
+    recs = H.profile_end(4096)
+    assert H.status_read(st.ws) == 0
+    cat = {"mixer": 0.0, "ffn": 0.0, "norm": 0.0}
+    for name, t in recs:
+        cat["ffn" if name.startswith("ffn") else ("norm" if name in ("rmsnorm", "prepend_meta") else "mixer")] += t
+    dims = wl.dims
+    T = st.T
+    mixer_flops = 0.0
+    for dl, _, _ in st.layers:
+        work, _ = prefill_work(dl, st.B, T)
+        mixer_flops += sum(a for k, (b, a) in work.items() if b == "tensor")
+    ffn_flops = st.L * 2.0 * st.B * T * dims.d_model * 3 * st.F
+    peaks = load_peaks()
+    return {"workload": "hymba_stack_32_layers", "batch": st.B, "seq_len": T, "layers": st.L, "ffn_dim": st.F,
+            "ms_per_forward": round(ms, 3), "tokens_per_s": round(whole_job_rate(world, st.B * T, ms), 1),
+            "mixer_ms": round(cat["mixer"], 3), "ffn_ms": round(cat["ffn"], 3), "norm_ms": round(cat["norm"], 3),
+            "mixer_tflops": round(mixer_flops / (cat["mixer"] * 1e-3) / 1e12, 1),
+            "ffn_tflops": round(ffn_flops / (cat["ffn"] * 1e-3) / 1e12, 1),
+            "mixer_frac_of_tensor_peak": round(mixer_flops / (cat["mixer"] * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+            "ffn_frac_of_tensor_peak": round(ffn_flops / (cat["ffn"] * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+            "timing": "CUDA events around whole forwards; mixer/FFN split from per-kernel events of one forward",
+            "weights": "random-init on the device (torch generator), distinct per layer"}
 
 
 # DRAM bytes per launch from ncu captures of the current kernels (None when not captured)
@@ -438,12 +590,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer measurement (profiling runs)")
+    ap.add_argument("--no-global", action="store_true", help="skip the global-layer measurement")
+    ap.add_argument("--no-stack", action="store_true", help="skip the 32-layer stack measurement")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = dist_env()
     metric = "hybrid-head layer prefill tokens/s + decode steps/s (1 B200), % roofline"
     cfg = {"workload": "swa_layer_prefill", "batch": 1, "n_meta": 128, "n_tokens": 2048, "seq_len": 2176,
            "d_model": 1600, "heads": "25q/5kv x 64", "window": 1024, "d_inner": 3200, "d_state": 16,
@@ -478,8 +630,8 @@ def main():
     device = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(device)
     r = run_hymba(args, rank, world, device)
-    tokens_per_s = world * r["tokens_per_step"] / (r["ms_per_step"] * 1e-3)
-    e2e = world * r["tokens_per_step"] / (r["e2e_ms"] * 1e-3)
+    tokens_per_s = whole_job_rate(world, r["tokens_per_step"], r["ms_per_step"])
+    e2e = whole_job_rate(world, r["tokens_per_step"], r["e2e_ms"])
     line = {"metric": metric, "value": round(tokens_per_s, 1), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(r["ms_per_step"], 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -491,6 +643,10 @@ def main():
             "gpu_launches": int(round(r["launches_per_step"] * args.steps)),
             "roofline": r["roofline"], "step_roofline": r["step_roofline"], "clocks": r["clocks"],
             "kernels": r["kernels"], "decode": r["decode"]}
+    if not args.no_global:
+        line["global_layer"] = run_global(args, device, world)
+    if not args.no_stack:
+        line["stack"] = run_stack(args, device, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, el, reps = time_oracle(2048, 10.0)
         line["cpu_baseline"] = {"value": round(rate, 2), "unit": "tokens/s", "cores": oracle_threads(),
@@ -498,7 +654,7 @@ def main():
                                 "sample": f"fp64 oracle prefill of the full SWA workload (128+2048 rows), "
                                           f"{reps} run(s) in {el:.1f} s"}
     if world > 1:
-        torch.distributed.barrier()
+        barrier(world)
         torch.distributed.destroy_process_group()
     if rank == 0:
         print(json.dumps(line))

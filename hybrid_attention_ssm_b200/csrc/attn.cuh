@@ -155,6 +155,8 @@ __device__ __forceinline__ void attn_item(const AttnParams& p, int w, int B, int
 __global__ void __launch_bounds__(ATT_THREADS, 2)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                     const __grid_constant__ CUtensorMap mapV, const __grid_constant__ AttnParams p, int B) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   if ((size_t)(smem - smem_raw) + ATT_USED > (size_t)ATT_SMEM) {   // cannot happen with a 1 KB-aligned window
@@ -324,7 +326,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
         const int e_meta = p.n_meta - j0;                  // meta: e < e_meta
         if (causal_full && window_full) {
 #pragma unroll
-          for (int e = 0; e < 128; ++e) mxp[e & 7] = fmaxf(mxp[e & 7], s[e]);
+          for (int e = 0; e < 128; e += 16)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mxp[k] = fmax3(mxp[k], s[e + k], s[e + 8 + k]);
         } else if (window_full) {
 #pragma unroll
           for (int e = 0; e < 128; ++e) {

@@ -1,30 +1,29 @@
 // tcgen05 GEMM for sm_100a: D[m, n] = sum_k A[m, k] * B[n, k] (both operands K-major),
 // bf16 or fp16 (kind::f16) or fp32 (kind::tf32) inputs, fp32 accumulation in TMEM, TMA-fed.
 //
-// Persistent warp-specialised kernel, 192 threads:
+// Persistent warp-specialised kernel, 320 threads:
 //   warp 0      TMA producer (one elected lane), STAGES-deep smem ring
 //   warp 1      TMEM allocator + MMA issuer (one elected lane)
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (thread = accumulator row),
-//               fused epilogue math, global stores
+//   warps 2..9  epilogue: tcgen05.ld of the accumulator (thread = accumulator row),
+//               fused epilogue math, global stores.  A warp may only read the TMEM lane
+//               quadrant warp%4, so two warps share each quadrant and split the tile's
+//               column chunks between them (two epilogue warps per SM sub-partition).
 // The accumulator is double-buffered in TMEM so the epilogue of tile i overlaps the
-// mainloop of tile i+1.  No TMA multicast, no clusters.
+// mainloop of tile i+1.  The epilogue is a template parameter, so each instance carries
+// only its own code.  No TMA multicast, no clusters.
 #pragma once
 #include "common.cuh"
 
 namespace hymba {
 
 enum EpiMode : int {
-  EPI_PROJ = 0,         // segmented bf16 stores with RoPE on marked segments (in_proj)
+  EPI_PROJ = 0,         // segmented bf16/fp16 stores with RoPE on marked segments (in_proj)
   EPI_BF16 = 1,         // bf16 store, optional bf16 residual add
-  EPI_ATOMIC_F32 = 2,   // fp32 atomic add (split-K partial sums)
-  EPI_SOFTPLUS = 3,     // fp32 store of softplus(acc + bias[col])
-  EPI_BF16_T = 4,       // transposed bf16 store: out[n][m] (weights as the M operand)
-  EPI_ATOMIC_F32_T = 5, // transposed fp32 atomic add
-  EPI_SWIGLU = 6,       // columns interleaved [gate(32) | up(32)] -> fp16 SiLU(gate)*up
-  EPI_SOFTPLUS_T = 7,   // fp32 softplus(acc + bias[col]) stored time-major: out[(b*N + col)*T_out + row]
-  EPI_F32_T = 8,        // transposed fp32 store: out[n][m]
-  EPI_F32_PART = 9,     // fp32 store of split ks's partial sum at out + ks*split_stride (row-major)
-  EPI_F32_T_PART = 10,  // the same, transposed
+  EPI_SWIGLU = 2,       // columns interleaved [gate(32) | up(32)] -> fp16 SiLU(gate)*up
+  EPI_SOFTPLUS_T = 3,   // fp32 softplus(acc + bias[col]) stored time-major: out[(b*N + col)*T_out + row]
+  EPI_F32_T = 4,        // transposed fp32 store: out[n][m] (weights as the M operand)
+  EPI_F32_PART = 5,     // fp32 store of split ks's partial sum at out + ks*split_stride (row-major)
+  EPI_F32_T_PART = 6,   // the same, transposed
 };
 
 struct Segment {
@@ -46,7 +45,6 @@ struct GemmParams {
   // output row mapping: a source-0 row r goes to rows {b*T_out + r}, b < out_batches;
   // a source-1 row (b, r) goes to b*T_out + row_off1 + r (position row_off1 + r)
   int out_batches, T_out, row_off1;
-  int mode;
   void* out;
   long long split_stride;   // elements between the partial-sum slices of two splits
   int ld_out;
@@ -61,7 +59,8 @@ struct GemmParams {
   DevStatus* status;
 };
 
-constexpr int GEMM_THREADS = 192;
+constexpr int GEMM_EPI_WARPS = 8;
+constexpr int GEMM_THREADS = 64 + 32 * GEMM_EPI_WARPS;
 constexpr int GEMM_BM = 128;
 
 template <int BN, int STAGES>
@@ -122,10 +121,12 @@ __device__ __forceinline__ float softplus_sel(float x) {
 // element types of both operands: bf16, fp16 (kind::f16) or fp32 read as tf32 (kind::tf32)
 enum : int { ET_BF16 = 0, ET_F16 = 1, ET_TF32 = 2 };
 
-template <int BN, int STAGES, int ET>
+template <int BN, int STAGES, int ET, int MODE>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA0, const __grid_constant__ CUtensorMap mapA1,
                    const __grid_constant__ CUtensorMap mapB, const __grid_constant__ GemmParams p) {
+  pdl_wait();
+  pdl_trigger();
   using L = GemmSmem<BN, STAGES>;
   constexpr int ACC_STRIDE = BN <= 128 ? 128 : 256;       // TMEM columns per accumulator
   constexpr uint32_t TMEM_COLS = 2 * ACC_STRIDE;
@@ -151,7 +152,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);
+      mbar_init(&acc_empty[b], GEMM_EPI_WARPS);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -242,6 +243,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   } else {
     // ------------------------------ epilogue ------------------------------
     const int quad = warp & 3;               // TMEM lanes this warp may access
+    const int half = (warp - 2) >> 2;        // which of the quadrant's two warps (column chunks)
     const int r = quad * 32 + lane;          // accumulator row of this thread
     int lt = 0;
     for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++lt) {
@@ -271,11 +273,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const bool row_ok = src0 ? (rr < p.rows0) : (rr < p.rows1);
       const int col_base = n * BN;
 
-      if (p.mode == EPI_PROJ || p.mode == EPI_SWIGLU) {
-        // 64-column chunks: both 32-column halves are loaded before one wait
+      if constexpr (MODE == EPI_PROJ || MODE == EPI_SWIGLU) {
+        // 64-column chunks (both 32-column halves loaded before one wait); the two warps
+        // of a quadrant take alternate chunks
+        static_assert(BN % 64 == 0, "64-column epilogue needs BN % 64 == 0");
         const size_t orow = (size_t)b1 * p.rows1 + rr;
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 64) {
+        for (int c0 = 64 * half; c0 < BN; c0 += 128) {
           uint32_t r[64];
           tmem_ld32_async(tbase + c0, r);
           tmem_ld32_async(tbase + c0 + 32, r + 32);
@@ -284,54 +288,49 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           float* v = reinterpret_cast<float*>(r);
           const int gc = col_base + c0;
           if (!row_ok || gc >= p.N) continue;
-          if (p.mode == EPI_SWIGLU) {   // fp16 activations (the down projection runs in fp16)
+          if constexpr (MODE == EPI_SWIGLU) {   // fp16 activations (the down projection runs in fp16)
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = silu_f(v[e]) * v[e + 32];
             store_f16_row(reinterpret_cast<__half*>(p.out) + orow * p.ld_out + gc / 2, v, 32);
-            continue;
-          }
-          int si = 0;
+          } else {
+            int si = 0;
 #pragma unroll 1
-          while (si < p.nseg - 1 && gc >= p.seg[si].col_end) ++si;
-          const Segment& sg = p.seg[si];
-          const int pos = src0 ? rr : p.row_off1 + rr;
-          if (sg.rope) rope_pair_rotate(v, p.rope_tab + (size_t)pos * 32);
-          __nv_bfloat16* base = reinterpret_cast<__nv_bfloat16*>(sg.ptr) + (gc - sg.col_begin);
-          const int b_lo = src0 ? 0 : b1, b_hi = src0 ? p.out_batches : b1 + 1;
-          for (int b = b_lo; b < b_hi; ++b) {
-            __nv_bfloat16* dst = base + b * sg.bstride + (size_t)pos * sg.ld;
-            if (sg.f16) store_f16_row(dst, v, 64);
-            else store_bf16_row(dst, v, 64);
+            while (si < p.nseg - 1 && gc >= p.seg[si].col_end) ++si;
+            const Segment& sg = p.seg[si];
+            const int pos = src0 ? rr : p.row_off1 + rr;
+            if (sg.rope) rope_pair_rotate(v, p.rope_tab + (size_t)pos * 32);
+            __nv_bfloat16* base = reinterpret_cast<__nv_bfloat16*>(sg.ptr) + (gc - sg.col_begin);
+            const int b_lo = src0 ? 0 : b1, b_hi = src0 ? p.out_batches : b1 + 1;
+            for (int b = b_lo; b < b_hi; ++b) {
+              __nv_bfloat16* dst = base + b * sg.bstride + (size_t)pos * sg.ld;
+              if (sg.f16) store_f16_row(dst, v, 64);
+              else store_bf16_row(dst, v, 64);
+            }
           }
         }
       } else {
-        // 32-column chunks, the next chunk's TMEM load in flight while this one is stored
+        // 32-column chunks j = half, half+2, ...; the next chunk's TMEM load is in flight
+        // while this one is processed
+        static_assert(BN % 32 == 0, "BN % 32 == 0");
+        constexpr int NCH = BN / 32;
         const size_t orow = (size_t)b1 * p.rows1 + rr;
         auto process = [&](uint32_t* r, int c0) {
           float* v = reinterpret_cast<float*>(r);
           const int gc = col_base + c0;
-          if (p.mode == EPI_BF16_T || p.mode == EPI_ATOMIC_F32_T || p.mode == EPI_F32_T ||
-              p.mode == EPI_F32_T_PART) {
+          if constexpr (MODE == EPI_F32_T || MODE == EPI_F32_T_PART) {
             // accumulator row = output column (weight row), accumulator column = output row
             if (!row_ok || rr >= p.m_valid) return;
-            float* outf = reinterpret_cast<float*>(p.out) + (p.mode == EPI_F32_T_PART ? ks * p.split_stride : 0);
+            float* outf = reinterpret_cast<float*>(p.out) + (MODE == EPI_F32_T_PART ? ks * p.split_stride : 0);
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               const int orow_t = gc + e;
-              if (orow_t < p.n_valid) {
-                if (p.mode == EPI_BF16_T)
-                  reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)orow_t * p.ld_out + rr] = __float2bfloat16_rn(v[e]);
-                else if (p.mode == EPI_ATOMIC_F32_T)
-                  atomicAdd(outf + (size_t)orow_t * p.ld_out + rr, v[e]);
-                else
-                  outf[(size_t)orow_t * p.ld_out + rr] = v[e];
-              }
+              if (orow_t < p.n_valid) outf[(size_t)orow_t * p.ld_out + rr] = v[e];
             }
             return;
           }
           if (!row_ok || gc >= p.n_valid) return;
           const bool whole = gc + 32 <= p.n_valid;
-          if (p.mode == EPI_BF16) {
+          if constexpr (MODE == EPI_BF16) {
             if (p.residual != nullptr) {
               const __nv_bfloat16* res = p.residual + orow * p.ld_res + gc;
               if (whole) {
@@ -355,18 +354,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             else
               for (int e = 0; e < 32; ++e)
                 if (gc + e < p.n_valid) dst[e] = __float2bfloat16_rn(v[e]);
-          } else if (p.mode == EPI_ATOMIC_F32 || p.mode == EPI_F32_PART) {
+          } else if constexpr (MODE == EPI_F32_PART) {
             // fp32 partial sums, 4-wide (ld_out and n_valid are multiples of 4)
-            float* dst = reinterpret_cast<float*>(p.out) + (p.mode == EPI_F32_PART ? ks * p.split_stride : 0) +
-                         orow * p.ld_out + gc;
+            float* dst = reinterpret_cast<float*>(p.out) + ks * p.split_stride + orow * p.ld_out + gc;
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
-              if (gc + e < p.n_valid) {
-                const float4 q = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-                if (p.mode == EPI_F32_PART) *reinterpret_cast<float4*>(dst + e) = q;
-                else atomicAdd(reinterpret_cast<float4*>(dst + e), q);
-              }
-          } else {
+              if (gc + e < p.n_valid)
+                *reinterpret_cast<float4*>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+          } else {  // EPI_SOFTPLUS_T: lanes hold consecutive rows -> coalesced along time
             float bb[32];
             if (whole) {
 #pragma unroll
@@ -380,41 +375,31 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             }
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = softplus_sel(v[e] + bb[e]);
-            if (p.mode == EPI_SOFTPLUS) {
-              float* dst = reinterpret_cast<float*>(p.out) + orow * p.ld_out + gc;
-              if (whole) {
+            float* dst = reinterpret_cast<float*>(p.out) + ((size_t)b1 * p.N + gc) * p.T_out + rr;
+            if (whole) {
 #pragma unroll
-                for (int e = 0; e < 32; e += 4)
-                  *reinterpret_cast<float4*>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-              } else {
-                for (int e = 0; e < 32; ++e)
-                  if (gc + e < p.n_valid) dst[e] = v[e];
-              }
-            } else {  // EPI_SOFTPLUS_T: lanes hold consecutive rows -> coalesced along time
-              float* dst = reinterpret_cast<float*>(p.out) + ((size_t)b1 * p.N + gc) * p.T_out + rr;
-              if (whole) {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) dst[(size_t)e * p.T_out] = v[e];
-              } else {
-                for (int e = 0; e < 32; ++e)
-                  if (gc + e < p.n_valid) dst[(size_t)e * p.T_out] = v[e];
-              }
+              for (int e = 0; e < 32; ++e) dst[(size_t)e * p.T_out] = v[e];
+            } else {
+              for (int e = 0; e < 32; ++e)
+                if (gc + e < p.n_valid) dst[(size_t)e * p.T_out] = v[e];
             }
           }
         };
         uint32_t ra[32], rb[32];
-        tmem_ld32_async(tbase, ra);
-        tmem_wait_ld_regs(ra);
+        if (half < NCH) {
+          tmem_ld32_async(tbase + 32 * half, ra);
+          tmem_wait_ld_regs(ra);
+        }
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 64) {
-          const bool has_b = c0 + 32 < BN;
-          if (has_b) tmem_ld32_async(tbase + c0 + 32, rb);
-          process(ra, c0);
+        for (int j = half; j < NCH; j += 4) {
+          const bool has_b = j + 2 < NCH;
+          if (has_b) tmem_ld32_async(tbase + 32 * (j + 2), rb);
+          process(ra, 32 * j);
           if (has_b) {
             tmem_wait_ld_regs(rb);
-            const bool has_a = c0 + 64 < BN;
-            if (has_a) tmem_ld32_async(tbase + c0 + 64, ra);
-            process(rb, c0 + 32);
+            const bool has_a = j + 4 < NCH;
+            if (has_a) tmem_ld32_async(tbase + 32 * (j + 4), ra);
+            process(rb, 32 * (j + 2));
             if (has_a) tmem_wait_ld_regs(ra);
           }
         }

@@ -9,6 +9,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "../../include/hymba.h"
 #include "attn.cuh"
@@ -45,6 +46,23 @@ int fail(int code, const char* fmt, ...) {
     int rc_ = (expr);           \
     if (rc_ != HYMBA_OK) return rc_; \
   } while (0)
+
+// Launches a kernel with programmatic stream serialisation: the grid may be launched while
+// the previous kernel on the stream drains; every kernel starts with pdl_wait().
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
@@ -93,7 +111,8 @@ int device_info(DeviceInfo** out) {
 // A 2-D or 3-D tiled map with 128-byte swizzle; dims/strides innermost first, strides in
 // bytes for dims 1.. ; box inner extent must be 128 bytes.
 int make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int rank, const uint64_t* dims,
-             const uint64_t* strides_bytes, const uint32_t* box) {
+             const uint64_t* strides_bytes, const uint32_t* box,
+             CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   if (!aligned16(base)) return fail(HYMBA_ERR_INVALID_ARG, "tensor base %p not 16-byte aligned", base);
   cuuint64_t d[3], s[2];
   cuuint32_t bx[3], es[3] = {1, 1, 1};
@@ -106,7 +125,7 @@ int make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int rank,
     if (s[i] % 16 != 0) return fail(HYMBA_ERR_INVALID_ARG, "tensor stride %llu not a multiple of 16", (unsigned long long)s[i]);
   }
   CUresult r = g_encode(m, dt, rank, const_cast<void*>(base), d, s, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(HYMBA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return HYMBA_OK;
@@ -123,15 +142,23 @@ struct ProfState {
 };
 ProfState g_prof;
 
+// Inside a stream capture the events become event-record nodes of the graph (the external
+// flag), so every replay re-records them.
+inline void prof_record(cudaEvent_t ev, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(st, &cs);
+  if (cs == cudaStreamCaptureStatusActive) cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal);
+  else cudaEventRecord(ev, st);
+}
 inline void prof_begin(const char* name, cudaStream_t st) {
   if (!g_prof.on || g_prof.n >= g_prof.cap) return;
   strncpy(g_prof.names[g_prof.n], name, 23);
   g_prof.names[g_prof.n][23] = 0;
-  cudaEventRecord(g_prof.ev[2 * g_prof.n], st);
+  prof_record(g_prof.ev[2 * g_prof.n], st);
 }
 inline void prof_end(cudaStream_t st) {
   if (!g_prof.on || g_prof.n >= g_prof.cap) return;
-  cudaEventRecord(g_prof.ev[2 * g_prof.n + 1], st);
+  prof_record(g_prof.ev[2 * g_prof.n + 1], st);
   ++g_prof.n;
 }
 
@@ -154,27 +181,107 @@ struct GemmCall {
   long long ldb = 0;
   int K = 0;
   int etype = ET_BF16;
+  int mode = EPI_BF16;
   int bn = 256;
   int split_k = 1;
   GemmParams p{};
 };
 
-template <int BN, int STAGES, int ET>
+template <int BN, int STAGES, int ET, int MODE>
 int launch_gemm_inst(const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& mb, const GemmParams& p,
                      int grid, cudaStream_t st, const char* name) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   constexpr int smem = GemmSmem<BN, STAGES>::TOTAL;
-  auto kern = gemm_tc_kernel<BN, STAGES, ET>;
+  auto kern = gemm_tc_kernel<BN, STAGES, ET, MODE>;
   if (!attr_set[dev & 63]) {
     HY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
     attr_set[dev & 63] = true;
   }
   prof_begin(name, st);
-  kern<<<grid, GEMM_THREADS, smem, st>>>(m0, m1, mb, p);
+  HY_CUDA(launch_pdl(kern, dim3(grid), dim3(GEMM_THREADS), smem, st, m0, m1, mb, p));
   prof_end(st);
-  HY_CUDA(cudaGetLastError());
+  return HYMBA_OK;
+}
+
+// Tile widths instantiated per (epilogue, operand type); anything else is rejected.
+template <int ET, int MODE>
+int launch_gemm_bn(int bn, const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& mb, const GemmParams& p,
+                   int grid, cudaStream_t st, const char* name) {
+  constexpr bool any_bn = MODE == EPI_F32_PART || MODE == EPI_F32_T || MODE == EPI_F32_T_PART;
+  if (bn == 256) return launch_gemm_inst<256, 4, ET, MODE>(m0, m1, mb, p, grid, st, name);
+  if constexpr (MODE != EPI_PROJ) {
+    if (bn == 128) return launch_gemm_inst<128, 6, ET, MODE>(m0, m1, mb, p, grid, st, name);
+  }
+  if constexpr (any_bn && ET != ET_TF32) {
+    if (bn == 160) return launch_gemm_inst<160, 5, ET, MODE>(m0, m1, mb, p, grid, st, name);
+    if (bn == 64) return launch_gemm_inst<64, 8, ET, MODE>(m0, m1, mb, p, grid, st, name);
+  }
+  return fail(HYMBA_ERR_UNSUPPORTED, "no GEMM instance for tile width %d, type %d, epilogue %d", bn, ET, MODE);
+}
+
+int launch_gemm_mode(const GemmCall& c, const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& mb,
+                     const GemmParams& p, int grid, cudaStream_t st) {
+  switch (c.mode) {
+    case EPI_PROJ:
+      if (c.etype == ET_BF16) return launch_gemm_bn<ET_BF16, EPI_PROJ>(c.bn, m0, m1, mb, p, grid, st, c.name);
+      break;
+    case EPI_BF16:
+      if (c.etype == ET_BF16) return launch_gemm_bn<ET_BF16, EPI_BF16>(c.bn, m0, m1, mb, p, grid, st, c.name);
+      if (c.etype == ET_F16) return launch_gemm_bn<ET_F16, EPI_BF16>(c.bn, m0, m1, mb, p, grid, st, c.name);
+      break;
+    case EPI_SWIGLU:
+      if (c.etype == ET_BF16) return launch_gemm_bn<ET_BF16, EPI_SWIGLU>(c.bn, m0, m1, mb, p, grid, st, c.name);
+      break;
+    case EPI_SOFTPLUS_T:
+      if (c.etype == ET_TF32) return launch_gemm_bn<ET_TF32, EPI_SOFTPLUS_T>(c.bn, m0, m1, mb, p, grid, st, c.name);
+      break;
+    case EPI_F32_T:
+      if (c.etype == ET_BF16) return launch_gemm_bn<ET_BF16, EPI_F32_T>(c.bn, m0, m1, mb, p, grid, st, c.name);
+      break;
+    case EPI_F32_PART:
+      if (c.etype == ET_BF16) return launch_gemm_bn<ET_BF16, EPI_F32_PART>(c.bn, m0, m1, mb, p, grid, st, c.name);
+      break;
+    case EPI_F32_T_PART:
+      if (c.etype == ET_BF16) return launch_gemm_bn<ET_BF16, EPI_F32_T_PART>(c.bn, m0, m1, mb, p, grid, st, c.name);
+      if (c.etype == ET_F16) return launch_gemm_bn<ET_F16, EPI_F32_T_PART>(c.bn, m0, m1, mb, p, grid, st, c.name);
+      break;
+    default:
+      break;
+  }
+  return fail(HYMBA_ERR_UNSUPPORTED, "no GEMM instance for epilogue %d with operand type %d", c.mode, c.etype);
+}
+
+// Branch norm + average: persistent CTAs, rows streamed through a bulk-copy ring.
+template <typename YT>
+int launch_branch_norm(const float* O, int ld_o, int attn_w, const YT* y, int ld_y, const __nv_bfloat16* z, int ld_z,
+                       int di, const float* g_attn, const float* g_ssm, float eps, __half* u, int ld_u, int rows,
+                       DevStatus* status, int sms, cudaStream_t st) {
+  if (rows <= 0) return HYMBA_OK;
+  if (attn_w % 4 || di % 8 || attn_w > 4 * NORM_THREADS * NORM_MAXO || di > 8 * NORM_THREADS * NORM_MAXY)
+    return fail(HYMBA_ERR_UNSUPPORTED, "branch norm widths %d/%d unsupported", attn_w, di);
+  const bool rows_ok = aligned16(O) && aligned16(y) && (z == nullptr || aligned16(z)) && aligned16(u) &&
+                       (ld_o * 4) % 16 == 0 && (ld_y * (int)sizeof(YT)) % 16 == 0 && (ld_z * 2) % 16 == 0 &&
+                       (ld_u * 2) % 16 == 0 && (attn_w * 2) % 16 == 0;
+  if (!rows_ok) return fail(HYMBA_ERR_INVALID_ARG, "branch norm rows must be 16-byte aligned");
+  const int stage = (norm_stage_bytes(attn_w, di, (int)sizeof(YT), z != nullptr) + 127) & ~127;
+  const int smem = NORM_STAGES * stage + 128;
+  static bool attr_set[2][64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  bool& set = attr_set[sizeof(YT) == 4][dev & 63];
+  if (!set) {
+    HY_CUDA(cudaFuncSetAttribute(branch_norm_avg_kernel<YT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 NORM_STAGES * ((norm_stage_bytes(2048, 4096, 4, true) + 127) & ~127) + 128));
+    set = true;
+  }
+  int per_sm = (200 * 1024) / smem;
+  if (per_sm < 1) per_sm = 1;
+  if (per_sm > 8) per_sm = 8;
+  const int grid = rows < sms * per_sm ? rows : sms * per_sm;
+  HY_CUDA(launch_pdl(branch_norm_avg_kernel<YT>, dim3(grid), dim3(NORM_THREADS), smem, st, O, ld_o, attn_w, y, ld_y,
+                     z, ld_z, di, g_attn, g_ssm, eps, u, ld_u, rows, status));
   return HYMBA_OK;
 }
 
@@ -221,20 +328,7 @@ int run_gemm(GemmCall& c, const DeviceInfo& dev, cudaStream_t st) {
   p.total_tiles = p.m_tiles * p.n_tiles_n * p.split_k;
   if (p.total_tiles <= 0) return HYMBA_OK;
   const int grid = p.total_tiles < dev.sms ? p.total_tiles : dev.sms;
-  if (tf32) {
-    if (c.bn == 256) return launch_gemm_inst<256, 4, ET_TF32>(m0, m1, mb, p, grid, st, c.name);
-    if (c.bn == 128) return launch_gemm_inst<128, 6, ET_TF32>(m0, m1, mb, p, grid, st, c.name);
-  } else if (c.etype == ET_F16) {
-    if (c.bn == 256) return launch_gemm_inst<256, 4, ET_F16>(m0, m1, mb, p, grid, st, c.name);
-    if (c.bn == 128) return launch_gemm_inst<128, 6, ET_F16>(m0, m1, mb, p, grid, st, c.name);
-    if (c.bn == 64) return launch_gemm_inst<64, 8, ET_F16>(m0, m1, mb, p, grid, st, c.name);
-  } else {
-    if (c.bn == 256) return launch_gemm_inst<256, 4, ET_BF16>(m0, m1, mb, p, grid, st, c.name);
-    if (c.bn == 160) return launch_gemm_inst<160, 5, ET_BF16>(m0, m1, mb, p, grid, st, c.name);
-    if (c.bn == 128) return launch_gemm_inst<128, 6, ET_BF16>(m0, m1, mb, p, grid, st, c.name);
-    if (c.bn == 64) return launch_gemm_inst<64, 8, ET_BF16>(m0, m1, mb, p, grid, st, c.name);
-  }
-  return fail(HYMBA_ERR_UNSUPPORTED, "no GEMM tile width %d", c.bn);
+  return launch_gemm_mode(c, m0, m1, mb, p, grid, st);
 }
 
 // smallest supported tile width covering n (for skinny N), else 256
@@ -338,15 +432,21 @@ PrefillWs prefill_layout(const Dims& m, int B, int n_tokens, int x_has_meta) {
 }
 
 struct DecodeWs {
-  size_t proj, part, o, xc, xbc, xbc_part, y, u, acc_part, total;
+  size_t proj, qrot, part, o, xc, xbc, xbc_part, y, u, acc_part, total;
   int n_splits, xproj_split, oproj_split;
 };
-DecodeWs decode_layout(const Dims& m, int B, int n_keys_max) {
+// Key tiles of one (sequence, kv head) in decode: SWA reads the meta tiles and the ring,
+// a global layer rows 0..p of its cache (p < n_keys_max).
+int decode_key_tiles(const Dims& m, bool global, int n_keys_max) {
+  return global ? cdiv(n_keys_max, DA_KT) : cdiv(m.M, DA_KT) + cdiv(m.W, DA_KT);
+}
+DecodeWs decode_layout(const Dims& m, int B, bool global, int n_keys_max) {
   DecodeWs w;
-  w.n_splits = cdiv(n_keys_max, DEC_KT);
+  w.n_splits = cdiv(decode_key_tiles(m, global, n_keys_max), DA_TPS);
   size_t off = 256;
   auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
   w.proj = take((size_t)B * m.P * 4);
+  w.qrot = take((size_t)B * m.Hq * 64 * 4);
   w.part = take((size_t)B * m.Hq * w.n_splits * 66 * 4);
   w.o = take((size_t)B * m.qw * 4);
   w.xc = take((size_t)B * m.Di * 2);
@@ -404,6 +504,21 @@ int hymba_profile_begin(int max_records) {
   return HYMBA_OK;
 }
 
+int hymba_profile_read(hymba_prof_record* out, int max_records, int* n_records) {
+  if (out == nullptr || n_records == nullptr) return fail(HYMBA_ERR_INVALID_ARG, "NULL argument");
+  g_prof.on = false;
+  const int n = g_prof.n < max_records ? g_prof.n : max_records;
+  for (int i = 0; i < n; ++i) {
+    HY_CUDA(cudaEventSynchronize(g_prof.ev[2 * i + 1]));
+    float ms = 0.f;
+    HY_CUDA(cudaEventElapsedTime(&ms, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]));
+    memcpy(out[i].name, g_prof.names[i], 24);
+    out[i].ms = ms;
+  }
+  *n_records = n;
+  return HYMBA_OK;
+}
+
 int hymba_profile_end(hymba_prof_record* out, int max_records, int* n_records) {
   if (out == nullptr || n_records == nullptr) return fail(HYMBA_ERR_INVALID_ARG, "NULL argument");
   g_prof.on = false;
@@ -438,7 +553,7 @@ int hymba_mixer_workspace_size(const hymba_layer_cfg* cfg, int batch, int n_toke
   } else if (mode == HYMBA_MODE_DECODE) {
     // for a global layer n_tokens is the cache's max_tokens (keys read per step)
     const int mk = cfg->is_global ? (n_tokens > 0 ? n_tokens : 1) : decode_max_keys(cfg, 0);
-    *bytes = decode_layout(m, batch, mk).total;
+    *bytes = decode_layout(m, batch, cfg->is_global != 0, mk).total;
   } else {
     return fail(HYMBA_ERR_INVALID_ARG, "mode %d", mode);
   }
@@ -597,7 +712,7 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     fill_rope_theta(th.t, cfg->rope_base);
     const int n = T * 32;
     prof_begin("rope_table", st);
-    rope_table_kernel<<<cdiv(n, 256), 256, 0, st>>>(reinterpret_cast<float2*>(wsb + L.rope), T, th);
+    HY_CUDA(launch_pdl(rope_table_kernel, dim3(cdiv(n, 256)), dim3(256), 0, st, reinterpret_cast<float2*>(wsb + L.rope), T, th));
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
@@ -615,7 +730,7 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     c.b = w->w_in; c.N = m.P; c.ldb = m.d; c.K = m.d;
     c.bn = 256;
     c.name = "in_proj";
-    c.p.mode = EPI_PROJ;
+    c.mode = EPI_PROJ;
     c.p.out_batches = B;
     c.p.T_out = T;
     c.p.status = status;
@@ -633,11 +748,10 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
   // 2. conv1d + SiLU (writes xc, xcT and the conv state)
   float* cstate = conv_state_out != nullptr ? conv_state_out : f32(L.cstate);
   {
-    const int threads = (m.Di / 2) * cdiv(T, CONV_RUN);
-    dim3 grid(cdiv(threads, 256), B);
+    dim3 grid(m.Di / CONV_TC, cdiv(T, CONV_TT), B);
     prof_begin("conv1d_silu", st);
-    conv1d_silu_kernel<<<grid, 256, 0, st>>>(bf(L.xz), 2 * m.Di, w->conv_w, w->conv_b, bf(L.xc), bf(L.xcT), cstate,
-                                              T, L.Tp, m.Di);
+    HY_CUDA(launch_pdl(conv1d_silu_kernel, grid, dim3(256), 0, st, bf(L.xz), 2 * m.Di, w->conv_w, w->conv_b, bf(L.xc),
+                       bf(L.xcT), cstate, T, L.Tp, m.Di));
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
@@ -649,7 +763,7 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     c.b = w->w_x; c.N = m.R + 2 * m.S; c.ldb = m.Di; c.K = m.Di;
     c.bn = pick_bn_cover(c.N);
     c.split_k = L.xproj_split;
-    c.p.mode = EPI_F32_PART;
+    c.mode = EPI_F32_PART;
     c.p.out = f32(L.xbc_part);
     c.p.split_stride = (long long)rows * m.ld_xbc;
     c.p.ld_out = m.ld_xbc;
@@ -658,9 +772,9 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     HY_TRY(run_gemm(c, *dev, st));
     const int n = (int)(rows * m.ld_xbc);
     prof_begin("splitk_reduce", st);
-    splitk_reduce_kernel<<<cdiv(n / 4, 256), 256, 0, st>>>(f32(L.xbc_part), L.xproj_split, (long long)n, n,
+    HY_CUDA(launch_pdl(splitk_reduce_kernel, dim3(cdiv(n / 4, 256)), dim3(256), 0, st, f32(L.xbc_part), L.xproj_split, (long long)n, n,
                                                             nullptr, f32(L.xbc), 0, f32(L.bcT), m.ld_xbc, T, L.Tp,
-                                                            m.R);
+                                                            m.R));
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
@@ -672,7 +786,7 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     c.b = w->w_dt; c.N = m.Di; c.ldb = w->w_dt_ld; c.K = m.R;
     c.bn = pick_bn_wide(B * cdiv(T, GEMM_BM), m.Di, dev->sms);
     c.name = "dt_proj";
-    c.p.mode = EPI_SOFTPLUS_T;
+    c.mode = EPI_SOFTPLUS_T;
     c.p.out = f32(L.dT);
     c.p.T_out = L.Tp;
     c.p.bias = w->dt_bias;
@@ -712,34 +826,52 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     }
     const int grid = ap.n_items < 2 * dev->sms ? ap.n_items : 2 * dev->sms;   // two persistent CTAs per SM
     prof_begin("attention", st);
-    attn_fwd_kernel<<<grid, ATT_THREADS, ATT_SMEM, st>>>(mq, mk, mv, ap, B);
+    HY_CUDA(launch_pdl(attn_fwd_kernel, dim3(grid), dim3(ATT_THREADS), ATT_SMEM, st, mq, mk, mv, ap, B));
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
   // 6. selective scan
   float* sstate = ssm_state_out != nullptr ? ssm_state_out : f32(L.sstate);
   {
+    // time-major inputs through tensor maps of extent T (zero fill past the last step)
+    CUtensorMap md, mx, mbc;
+    {
+      const uint64_t dims[2] = {(uint64_t)T, (uint64_t)B * m.Di};
+      const uint64_t str[1] = {(uint64_t)L.Tp * 4};
+      const uint32_t box[2] = {SCAN_TC, SCAN_CH};
+      HY_TRY(make_map(&md, f32(L.dT), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE));
+    }
+    {
+      const uint64_t dims[2] = {(uint64_t)T, (uint64_t)B * m.Di};
+      const uint64_t str[1] = {(uint64_t)L.Tp * 2};
+      const uint32_t box[2] = {SCAN_TC, SCAN_CH};
+      HY_TRY(make_map(&mx, bf(L.xcT), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE));
+    }
+    {
+      const uint64_t dims[2] = {(uint64_t)T, (uint64_t)B * 32};
+      const uint64_t str[1] = {(uint64_t)L.Tp * 4};
+      const uint32_t box[2] = {SCAN_BCW, 32};
+      HY_TRY(make_map(&mbc, f32(L.bcT), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE));
+    }
     dim3 grid(m.Di / SCAN_CH, B);
     static bool attr_scan[64] = {false};
     int dcur = 0;
     cudaGetDevice(&dcur);
     if (!attr_scan[dcur & 63]) {
-      HY_CUDA(cudaFuncSetAttribute(selective_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)sizeof(ScanSmem)));
+      HY_CUDA(cudaFuncSetAttribute(selective_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM));
       attr_scan[dcur & 63] = true;
     }
     prof_begin("selective_scan", st);
-    selective_scan_kernel<<<grid, SCAN_THREADS, sizeof(ScanSmem), st>>>(bf(L.xcT), f32(L.dT), f32(L.bcT), w->A,
-                                                                         bf(L.y), sstate, T, L.Tp, m.Di);
+    HY_CUDA(launch_pdl(selective_scan_kernel, grid, dim3(SCAN_THREADS), SCAN_SMEM, st, md, mx, mbc, w->A, bf(L.y),
+                       sstate, T, m.Di, status));
     prof_end(st);
-    HY_CUDA(cudaGetLastError());
   }
   // 7. per-branch RMSNorm, gate, beta, average
   {
     prof_begin("norm_avg", st);
-    branch_norm_avg_kernel<__nv_bfloat16><<<cdiv(rows, NORM_ROWS), 128 * NORM_ROWS, 0, st>>>(
-        f32(L.o), m.qw, m.qw, bf(L.y), m.Di, bf(L.xz) + m.Di, 2 * m.Di, m.Di, w->g_attn, w->g_ssm, cfg->norm_eps,
-        h16(L.u), m.uw, (int)rows);
+    HY_TRY(launch_branch_norm<__nv_bfloat16>(f32(L.o), m.qw, m.qw, bf(L.y), m.Di, bf(L.xz) + m.Di, 2 * m.Di, m.Di,
+                                             w->g_attn, w->g_ssm, cfg->norm_eps, h16(L.u), m.uw, (int)rows, status,
+                                             dev->sms, st));
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
@@ -751,7 +883,7 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     c.etype = ET_F16;
     c.name = "out_proj";
     c.bn = pick_bn_wide(cdiv(rows, GEMM_BM), m.d, dev->sms);
-    c.p.mode = EPI_BF16;
+    c.mode = EPI_BF16;
     c.p.out = out;
     c.p.ld_out = m.d;
     c.p.n_valid = m.d;
@@ -767,10 +899,10 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     const int n = n_rows * (m.kvw / 8);
     dim3 grid(cdiv(n, 256), B);
     prof_begin("swa_cache_finalize", st);
-    swa_cache_finalize_kernel<<<grid, 256, 0, st>>>(
+    HY_CUDA(launch_pdl(swa_cache_finalize_kernel, dim3(grid), dim3(256), 0, st,
         reinterpret_cast<const __half*>(kv->k), reinterpret_cast<const __half*>(kv->v), Lmax, T, m.M, m.W, m.kvw,
         reinterpret_cast<__half*>(kv->meta_k), reinterpret_cast<__half*>(kv->meta_v),
-        reinterpret_cast<__half*>(kv->ring_k), reinterpret_cast<__half*>(kv->ring_v));
+        reinterpret_cast<__half*>(kv->ring_k), reinterpret_cast<__half*>(kv->ring_v)));
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
@@ -803,7 +935,7 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
       return fail(HYMBA_ERR_INVALID_ARG, "SWA cache");
   }
   const int max_keys = decode_max_keys(cfg, kv->max_tokens);
-  const DecodeWs L = decode_layout(m, B, max_keys);
+  const DecodeWs L = decode_layout(m, B, global, max_keys);
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return fail(HYMBA_ERR_INVALID_ARG, "workspace");
   if (ws_bytes < L.total) return fail(HYMBA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
   cudaStream_t st = (cudaStream_t)stream;
@@ -821,7 +953,7 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     c.b = x; c.N = B; c.ldb = m.d; c.K = m.d;
     c.bn = pick_bn_cover(B);
     c.name = "decode_in_proj";
-    c.p.mode = EPI_F32_T;
+    c.mode = EPI_F32_T;
     c.p.out = f32(L.proj);
     c.p.ld_out = m.P;
     c.p.m_valid = m.P;
@@ -829,50 +961,90 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     c.p.status = status;
     HY_TRY(run_gemm(c, *dev, st));
   }
-  // 2. attention over meta + window (or the whole causal prefix), split-K, then combine
+  // 2. conv step, RoPE of q and the new k, the new k/v into the cache
+  {
+    DecPrepParams pp;
+    pp.proj = f32(L.proj);
+    pp.ld_proj = m.P;
+    pp.B = B;
+    pp.Di = m.Di;
+    pp.off_x = m.xz_off;
+    pp.conv_blocks = cdiv(B * m.Di, 256);
+    pp.conv_w = w->conv_w;
+    pp.conv_b = w->conv_b;
+    pp.conv_state = conv_state;
+    pp.xc = bf(L.xc);
+    pp.Hq = m.Hq; pp.Hkv = m.Hkv; pp.p = position; pp.write_kv = own_kv ? 1 : 0;
+    pp.is_global = global ? 1 : 0; pp.M = m.M; pp.W = m.W; pp.Lmax = kv->max_tokens;
+    pp.ring_k = reinterpret_cast<__half*>(kv->ring_k);
+    pp.ring_v = reinterpret_cast<__half*>(kv->ring_v);
+    pp.full_k = reinterpret_cast<__half*>(kv->k);
+    pp.full_v = reinterpret_cast<__half*>(kv->v);
+    pp.qrot = f32(L.qrot);
+    pp.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)m.D));
+    fill_rope_theta(pp.rope_theta, cfg->rope_base);
+    const int n_rope = B * (m.Hq + (own_kv ? m.Hkv : 0)) * 32;
+    prof_begin("decode_prep", st);
+    HY_CUDA(launch_pdl(decode_prep_kernel, dim3(pp.conv_blocks + cdiv(n_rope, 256)), dim3(256), 0, st, pp));
+    prof_end(st);
+  }
+  // 3. attention over meta + window (or rows 0..p), split over key tiles, then combine
   {
     DecAttnParams ap;
-    ap.proj = f32(L.proj);
-    ap.ld_proj = m.P;
-    ap.Hq = m.Hq; ap.Hkv = m.Hkv; ap.M = m.M; ap.W = m.W; ap.is_global = global ? 1 : 0;
-    ap.write_kv = own_kv ? 1 : 0;
-    ap.p = position;
+    ap.qrot = f32(L.qrot);
+    ap.Hq = m.Hq; ap.Hkv = m.Hkv; ap.M = m.M; ap.is_global = global ? 1 : 0;
+    const int kvw = m.Hkv * m.D;
+    CUtensorMap mmk, mmv, mk, mv;
+    auto map_rows = [&](CUtensorMap* mp, const void* base, long long rows) {
+      const uint64_t dims[2] = {(uint64_t)kvw, (uint64_t)rows};
+      const uint64_t str[1] = {(uint64_t)kvw * 2};
+      const uint32_t box[2] = {64, DA_KT};
+      return make_map(mp, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, dims, str, box);
+    };
     if (global) {
-      ap.n_keys = position + 1;
+      ap.n_meta_tiles = 0;
+      ap.n_main_valid = position + 1;
+      ap.rows_main = kv->max_tokens;
+      HY_TRY(map_rows(&mk, kv->k, (long long)B * kv->max_tokens));
+      HY_TRY(map_rows(&mv, kv->v, (long long)B * kv->max_tokens));
+      mmk = mk;
+      mmv = mv;
     } else {
-      const int win0 = position - m.W + 1 > m.M ? position - m.W + 1 : m.M;
-      ap.n_keys = m.M + (position - win0 + 1);
+      ap.n_meta_tiles = cdiv(m.M, DA_KT);
+      const int filled = position - m.M + 1;
+      ap.n_main_valid = filled < m.W ? filled : m.W;
+      ap.rows_main = m.W;
+      HY_TRY(map_rows(&mk, kv->ring_k, (long long)B * m.W));
+      HY_TRY(map_rows(&mv, kv->ring_v, (long long)B * m.W));
+      if (m.M > 0) {
+        HY_TRY(map_rows(&mmk, kv->meta_k, (long long)B * m.M));
+        HY_TRY(map_rows(&mmv, kv->meta_v, (long long)B * m.M));
+      } else {
+        mmk = mk;
+        mmv = mv;
+      }
     }
-    ap.n_splits = cdiv(ap.n_keys, DEC_KT);
-    ap.meta_k = reinterpret_cast<__half*>(kv->meta_k);
-    ap.meta_v = reinterpret_cast<__half*>(kv->meta_v);
-    ap.ring_k = reinterpret_cast<__half*>(kv->ring_k);
-    ap.ring_v = reinterpret_cast<__half*>(kv->ring_v);
-    ap.full_k = reinterpret_cast<__half*>(kv->k);
-    ap.full_v = reinterpret_cast<__half*>(kv->v);
-    ap.Lmax = kv->max_tokens;
-    ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)m.D));
-    fill_rope_theta(ap.rope_theta, cfg->rope_base);
-    ap.part = f32(L.part);
+    ap.n_tiles = ap.n_meta_tiles + cdiv(ap.n_main_valid, DA_KT);
+    ap.n_splits = cdiv(ap.n_tiles, DA_TPS);
     if (ap.n_splits > L.n_splits) return fail(HYMBA_ERR_WORKSPACE, "decode workspace sized for fewer keys");
-    dim3 grid(ap.n_splits, m.Hkv, B);
+    ap.n_items = B * m.Hkv * ap.n_splits;
+    ap.part = f32(L.part);
+    ap.status = status;
+    static bool attr_da[64] = {false};
+    int dcur = 0;
+    cudaGetDevice(&dcur);
+    if (!attr_da[dcur & 63]) {
+      HY_CUDA(cudaFuncSetAttribute(decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DA_SMEM));
+      attr_da[dcur & 63] = true;
+    }
+    const int grid = ap.n_items < 3 * dev->sms ? ap.n_items : 3 * dev->sms;
     prof_begin("decode_attn", st);
-    decode_attn_kernel<<<grid, 128, 0, st>>>(ap);
+    HY_CUDA(launch_pdl(decode_attn_kernel, dim3(grid), dim3(DA_THREADS), DA_SMEM, st, mmk, mmv, mk, mv, ap));
     prof_end(st);
-    HY_CUDA(cudaGetLastError());
     prof_begin("decode_attn_combine", st);
-    decode_attn_combine_kernel<<<dim3(m.Hq, B), 64, 0, st>>>(f32(L.part), ap.n_splits, m.Hq, f32(L.o), m.qw);
+    HY_CUDA(launch_pdl(decode_attn_combine_kernel, dim3(m.Hq, B), dim3(64), 0, st, f32(L.part), ap.n_splits, m.Hq,
+                       f32(L.o), m.qw));
     prof_end(st);
-    HY_CUDA(cudaGetLastError());
-  }
-  // 3. conv step
-  {
-    const int n = B * m.Di;
-    prof_begin("decode_conv", st);
-    decode_conv_kernel<<<cdiv(n, 256), 256, 0, st>>>(f32(L.proj), m.P, m.xz_off, m.Di, w->conv_w, w->conv_b,
-                                                      conv_state, bf(L.xc), B);
-    prof_end(st);
-    HY_CUDA(cudaGetLastError());
   }
   // 4. x_proj (swap-AB, split-K into per-split slices, fixed-order sum)
   {
@@ -882,7 +1054,7 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     c.bn = pick_bn_cover(B);
     c.name = "decode_x_proj";
     c.split_k = L.xproj_split;
-    c.p.mode = EPI_F32_T_PART;
+    c.mode = EPI_F32_T_PART;
     c.p.out = f32(L.xbc_part);
     c.p.split_stride = (long long)B * m.ld_xbc;
     c.p.ld_out = m.ld_xbc;
@@ -892,25 +1064,25 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     HY_TRY(run_gemm(c, *dev, st));
     const int n = B * m.ld_xbc;
     prof_begin("decode_splitk_reduce", st);
-    splitk_reduce_kernel<<<cdiv(n / 4, 256), 256, 0, st>>>(f32(L.xbc_part), L.xproj_split, (long long)n, n, nullptr,
-                                                            f32(L.xbc), 0);
+    HY_CUDA(launch_pdl(splitk_reduce_kernel, dim3(cdiv(n / 4, 256)), dim3(256), 0, st, f32(L.xbc_part), L.xproj_split, (long long)n, n, nullptr,
+                                                            f32(L.xbc), 0, (float*)nullptr, 0, 0, 0, 0));
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
   // 5. dt_proj + softplus + state update + C.h + gate
   {
-    dim3 grid(m.Di / 16, B);
+    dim3 grid(m.Di / 16, cdiv(B, DSSM_NB));
     prof_begin("decode_ssm", st);
-    decode_ssm_kernel<<<grid, 256, 0, st>>>(f32(L.xbc), m.ld_xbc, m.R, w->w_dt, w->w_dt_ld, w->dt_bias, w->A,
-                                            bf(L.xc), f32(L.proj), m.P, m.xz_off + m.Di, ssm_state, f32(L.y), m.Di);
+    HY_CUDA(launch_pdl(decode_ssm_kernel, grid, dim3(256), 0, st, f32(L.xbc), m.ld_xbc, m.R, w->w_dt, w->w_dt_ld,
+                       w->dt_bias, w->A, bf(L.xc), f32(L.proj), m.P, m.xz_off + m.Di, ssm_state, f32(L.y), m.Di, B));
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
   // 6. norm + average (y already gated)
   {
     prof_begin("decode_norm_avg", st);
-    branch_norm_avg_kernel<float><<<cdiv(B, NORM_ROWS), 128 * NORM_ROWS, 0, st>>>(
-        f32(L.o), m.qw, m.qw, f32(L.y), m.Di, nullptr, 0, m.Di, w->g_attn, w->g_ssm, cfg->norm_eps, h16(L.u), m.uw, B);
+    HY_TRY(launch_branch_norm<float>(f32(L.o), m.qw, m.qw, f32(L.y), m.Di, nullptr, 0, m.Di, w->g_attn, w->g_ssm,
+                                     cfg->norm_eps, h16(L.u), m.uw, B, status, dev->sms, st));
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
@@ -924,7 +1096,7 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     c.bn = pick_bn_cover(B);
     c.name = "decode_out_proj";
     c.split_k = L.oproj_split;
-    c.p.mode = EPI_F32_T_PART;
+    c.mode = EPI_F32_T_PART;
     c.p.out = f32(L.acc_part);
     c.p.split_stride = (long long)B * m.d;
     c.p.ld_out = m.d;
@@ -934,8 +1106,8 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     HY_TRY(run_gemm(c, *dev, st));
     const int n = B * m.d;
     prof_begin("decode_out_store", st);
-    splitk_reduce_kernel<<<cdiv(n / 4, 256), 256, 0, st>>>(f32(L.acc_part), L.oproj_split, (long long)n, n,
-                                                            reinterpret_cast<const __nv_bfloat16*>(residual), out, 1);
+    HY_CUDA(launch_pdl(splitk_reduce_kernel, dim3(cdiv(n / 4, 256)), dim3(256), 0, st, f32(L.acc_part), L.oproj_split, (long long)n, n,
+                                                            reinterpret_cast<const __nv_bfloat16*>(residual), out, 1, (float*)nullptr, 0, 0, 0, 0));
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
@@ -952,7 +1124,7 @@ int hymba_gemm_bf16(const hymba_bf16* A, const hymba_bf16* Bm, const hymba_bf16*
   c.a1 = A; c.nb1 = 1; c.rows1 = M; c.lda1 = K; c.a1_bstride = (long long)M * K;
   c.b = Bm; c.N = N; c.ldb = K; c.K = K;
   c.bn = pick_bn_wide(cdiv(M, GEMM_BM), N, dev->sms);
-  c.p.mode = EPI_BF16;
+  c.mode = EPI_BF16;
   c.p.out = C;
   c.p.ld_out = N;
   c.p.n_valid = N;
@@ -968,8 +1140,8 @@ int hymba_rmsnorm(const hymba_bf16* x, const float* gain, int rows, int d, float
       !aligned16(out))
     return fail(HYMBA_ERR_INVALID_ARG, "rmsnorm arguments");
   prof_begin("rmsnorm", (cudaStream_t)stream);
-    rmsnorm_kernel<<<rows, 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<const __nv_bfloat16*>(x), gain, d, eps,
-                                                          reinterpret_cast<__nv_bfloat16*>(out));
+    HY_CUDA(launch_pdl(rmsnorm_kernel, dim3(rows), dim3(256), 0, (cudaStream_t)stream, reinterpret_cast<const __nv_bfloat16*>(x), gain, d, eps,
+                                                          reinterpret_cast<__nv_bfloat16*>(out)));
     prof_end((cudaStream_t)stream);
   HY_CUDA(cudaGetLastError());
   return HYMBA_OK;
@@ -990,7 +1162,7 @@ int hymba_ffn_swiglu(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hym
     c.b = w_gate_up; c.N = 2 * F; c.ldb = d; c.K = d;
     c.bn = pick_bn_wide(cdiv(rows, GEMM_BM), 2 * F, dev->sms);
     c.name = "ffn_gate_up";
-    c.p.mode = EPI_SWIGLU;
+    c.mode = EPI_SWIGLU;
     c.p.out = act;
     c.p.ld_out = F;
     c.p.n_valid = 2 * F;
@@ -1004,7 +1176,7 @@ int hymba_ffn_swiglu(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hym
     c.etype = ET_F16;
     c.name = "ffn_down";
     c.bn = pick_bn_wide(cdiv(rows, GEMM_BM), d, dev->sms);
-    c.p.mode = EPI_BF16;
+    c.mode = EPI_BF16;
     c.p.out = out;
     c.p.ld_out = d;
     c.p.n_valid = d;
@@ -1025,10 +1197,10 @@ int hymba_prepend_meta(const hymba_bf16* meta, const hymba_bf16* x, int batch, i
   if (total == 0) return HYMBA_OK;
   const int grid = (int)((total + 255) / 256 < 4096 ? (total + 255) / 256 : 4096);
   prof_begin("prepend_meta", (cudaStream_t)stream);
-  prepend_meta_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<const __nv_bfloat16*>(meta),
+  HY_CUDA(launch_pdl(prepend_meta_kernel, dim3(grid), dim3(256), 0, (cudaStream_t)stream, reinterpret_cast<const __nv_bfloat16*>(meta),
                                                                reinterpret_cast<const __nv_bfloat16*>(x), batch,
                                                                n_meta, n_tokens, d,
-                                                               reinterpret_cast<__nv_bfloat16*>(out));
+                                                               reinterpret_cast<__nv_bfloat16*>(out)));
   prof_end((cudaStream_t)stream);
   HY_CUDA(cudaGetLastError());
   return HYMBA_OK;
@@ -1037,7 +1209,7 @@ int hymba_prepend_meta(const hymba_bf16* meta, const hymba_bf16* x, int batch, i
 int hymba_selftest_wait_timeout(void* ws, size_t ws_bytes, hymba_stream stream) {
   if (ws == nullptr || ws_bytes < 256 || (reinterpret_cast<uintptr_t>(ws) & 255u))
     return fail(HYMBA_ERR_INVALID_ARG, "workspace");
-  wait_timeout_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(reinterpret_cast<DevStatus*>(ws));
+  HY_CUDA(launch_pdl(wait_timeout_selftest_kernel, dim3(1), dim3(32), 0, (cudaStream_t)stream, reinterpret_cast<DevStatus*>(ws)));
   HY_CUDA(cudaGetLastError());
   return HYMBA_OK;
 }

@@ -10,215 +10,228 @@ namespace hymba {
 //   xc     [B*T, Di]   bf16 row-major (A operand of x_proj)
 //   xcT    [B, Di, Tp] bf16 time-major (input of the scan), row stride Tp (multiple of 8)
 //   state  [B, Di, 3]  fp32: the last 3 inputs x[T-3..T-1] (zero before the start)
-// CTA: 64 channels x 64 time steps, 256 threads.
 // ----------------------------------------------------------------------------------------
 constexpr int CONV_K = 4;
-constexpr int CONV_RUN = 8;      // time steps per thread
+constexpr int CONV_TT = 64;      // time steps per CTA
+constexpr int CONV_TC = 64;      // channels per CTA
+constexpr int CONV_P = CONV_TC + 8;   // smem row pitch (16-byte aligned rows)
 
-// Thread = (channel pair, run of 8 time steps): the 3-step history stays in registers,
-// loads and row-major stores are 4 bytes per lane (128 B per warp), the time-major store
-// is 16 contiguous bytes per channel.
+// CTA = 64 channels x 64 time steps, 256 threads.  The x tile (plus the 3 rows before it)
+// comes in as 128-byte row pieces; a thread walks 16 steps of one channel with the 3-step
+// history in registers and writes its outputs into a [t][c] and a [c][t] shared tile, from
+// which both layouts leave as 128-byte rows.
 __global__ void __launch_bounds__(256)
     conv1d_silu_kernel(const __nv_bfloat16* __restrict__ x, int ld_x, const float* __restrict__ w,
                        const float* __restrict__ bias, __nv_bfloat16* __restrict__ xc,
                        __nv_bfloat16* __restrict__ xcT, float* __restrict__ state, int T, int Tp, int Di) {
-  const int pairs = Di >> 1;
-  const int gid = blockIdx.x * blockDim.x + threadIdx.x;
-  const int cp = gid % pairs;
-  const int run = gid / pairs;
-  const int b = blockIdx.y;
-  const int t0 = run * CONV_RUN;
-  if (t0 >= T) return;
-  const int c = cp * 2;
-  const float4 w0 = *reinterpret_cast<const float4*>(w + (size_t)c * 4);
-  const float4 w1 = *reinterpret_cast<const float4*>(w + (size_t)(c + 1) * 4);
-  const float b0 = bias[c], b1 = bias[c + 1];
-  const __nv_bfloat16* xb = x + (size_t)b * T * ld_x + c;
-  float h0[3], h1[3];          // x[t-3], x[t-2], x[t-1] of both channels
-#pragma unroll
-  for (int k = 0; k < 3; ++k) {
-    const int t = t0 - 3 + k;
-    float2 f = make_float2(0.f, 0.f);
-    if (t >= 0) f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(xb + (size_t)t * ld_x));
-    h0[k] = f.x;
-    h1[k] = f.y;
+  pdl_wait();
+  pdl_trigger();
+  __shared__ __align__(16) __nv_bfloat16 xs[CONV_TT + CONV_K - 1][CONV_P];   // rows t0-3 .. t0+63
+  __shared__ __align__(16) __nv_bfloat16 orow[CONV_TT][CONV_P];               // [t][c]
+  __shared__ __align__(16) __nv_bfloat16 ocol[CONV_TC][CONV_P];               // [c][t]
+  const int c0 = blockIdx.x * CONV_TC, t0 = blockIdx.y * CONV_TT, b = blockIdx.z;
+  const int tid = threadIdx.x;
+  const __nv_bfloat16* xb = x + (size_t)b * T * ld_x + c0;
+  for (int i = tid; i < (CONV_TT + CONV_K - 1) * 8; i += 256) {
+    const int r = i >> 3, q = i & 7, t = t0 - (CONV_K - 1) + r;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (t >= 0 && t < T) v = *reinterpret_cast<const uint4*>(xb + (size_t)t * ld_x + q * 8);
+    *reinterpret_cast<uint4*>(&xs[r][q * 8]) = v;
   }
-  const int n = min(CONV_RUN, T - t0);
-  float2 xv[CONV_RUN];
+  __syncthreads();
+  {
+    const int cc = tid & 63, tq = (tid >> 6) * 16;   // channel, first of 16 steps
+    const float4 wv = *reinterpret_cast<const float4*>(w + (size_t)(c0 + cc) * 4);
+    const float bb = bias[c0 + cc];
+    float h0 = __bfloat162float(xs[tq][cc]), h1 = __bfloat162float(xs[tq + 1][cc]);
+    float h2 = __bfloat162float(xs[tq + 2][cc]);
 #pragma unroll
-  for (int i = 0; i < CONV_RUN; ++i)
-    if (i < n) xv[i] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(xb + (size_t)(t0 + i) * ld_x));
-  __align__(16) __nv_bfloat16 o0[CONV_RUN], o1[CONV_RUN];
-#pragma unroll
-  for (int i = 0; i < CONV_RUN; ++i) {
-    if (i < n) {
-      const float a0 = b0 + w0.x * h0[0] + w0.y * h0[1] + w0.z * h0[2] + w0.w * xv[i].x;
-      const float a1 = b1 + w1.x * h1[0] + w1.y * h1[1] + w1.z * h1[2] + w1.w * xv[i].y;
-      h0[0] = h0[1]; h0[1] = h0[2]; h0[2] = xv[i].x;
-      h1[0] = h1[1]; h1[1] = h1[2]; h1[2] = xv[i].y;
-      const __nv_bfloat162 y2 = __floats2bfloat162_rn(silu_f(a0), silu_f(a1));
-      *reinterpret_cast<__nv_bfloat162*>(xc + ((size_t)b * T + t0 + i) * Di + c) = y2;
-      o0[i] = y2.x;
-      o1[i] = y2.y;
-    } else {
-      o0[i] = __float2bfloat16_rn(0.f);
-      o1[i] = __float2bfloat16_rn(0.f);
+    for (int i = 0; i < 16; i += 2) {
+      const float xa = __bfloat162float(xs[tq + 3 + i][cc]);
+      const float ya = bb + wv.x * h0 + wv.y * h1 + wv.z * h2 + wv.w * xa;
+      const float xb2 = __bfloat162float(xs[tq + 4 + i][cc]);
+      const float yb = bb + wv.x * h1 + wv.y * h2 + wv.z * xa + wv.w * xb2;
+      h0 = h2; h1 = xa; h2 = xb2;
+      const __nv_bfloat162 o2 = __floats2bfloat162_rn(silu_f(ya), silu_f(yb));
+      orow[tq + i][cc] = o2.x;
+      orow[tq + i + 1][cc] = o2.y;
+      *reinterpret_cast<__nv_bfloat162*>(&ocol[cc][tq + i]) = o2;
     }
   }
-  __nv_bfloat16* d0 = xcT + ((size_t)b * Di + c) * Tp + t0;
-  __nv_bfloat16* d1 = d0 + Tp;
-  if (n == CONV_RUN) {
-#pragma unroll
-    for (int i = 0; i < CONV_RUN; i += 8) {
-      *reinterpret_cast<uint4*>(d0 + i) = *reinterpret_cast<const uint4*>(o0 + i);
-      *reinterpret_cast<uint4*>(d1 + i) = *reinterpret_cast<const uint4*>(o1 + i);
-    }
-  } else {
-    for (int i = 0; i < n; ++i) {
-      d0[i] = o0[i];
-      d1[i] = o1[i];
-    }
+  __syncthreads();
+  // row-major xc and time-major xcT, 128-byte rows (8 threads x 16 bytes)
+  for (int i = tid; i < CONV_TT * 8; i += 256) {
+    const int r = i >> 3, q = i & 7, t = t0 + r;
+    if (t < T)
+      *reinterpret_cast<uint4*>(xc + ((size_t)b * T + t) * Di + c0 + q * 8) =
+          *reinterpret_cast<const uint4*>(&orow[r][q * 8]);
   }
-  // conv state: the last 3 inputs x[T-3..T-1] (zero when T < 3), from the last run
-  if (t0 + n == T) {
-    float* s0 = state + ((size_t)b * Di + c) * 3;
+  for (int i = tid; i < CONV_TC * 8; i += 256) {
+    const int c = i >> 3, q = i & 7, t = t0 + q * 8;
+    if (t < T)   // pieces reaching past T only feed positions the scan reads as zero
+      *reinterpret_cast<uint4*>(xcT + ((size_t)b * Di + c0 + c) * Tp + t) = *reinterpret_cast<const uint4*>(&ocol[c][q * 8]);
+  }
+  // conv state: the last 3 inputs x[T-3..T-1] (zero before the start), from the last tile
+  if (t0 + CONV_TT >= T && tid < CONV_TC) {
+    float* s0 = state + ((size_t)b * Di + c0 + tid) * 3;
 #pragma unroll
     for (int k = 0; k < 3; ++k) {
-      const bool valid = T - 3 + k >= 0;
-      s0[k] = valid ? h0[k] : 0.f;
-      s0[3 + k] = valid ? h1[k] : 0.f;
+      const int t = T - 3 + k;
+      s0[k] = t >= 0 ? __bfloat162float(xs[t - t0 + CONV_K - 1][tid]) : 0.f;
     }
   }
 }
 
 // ----------------------------------------------------------------------------------------
-// Selective scan, time-sequential per (channel, state) thread.
-//   h_t = exp(delta_t * A[c,s]) h_{t-1} + delta_t * B_t[s] * x_t ;  y_t = sum_s C_t[s] h_t[s]
-// CTA = 8 channels x 16 states; the fp32 state stays in a register for the whole sequence.
-// All inputs are time-major, so every chunk of 64 steps arrives by cp.async (16-byte
-// pieces, zero-filled past T) into a 4-stage ring, three chunks ahead of the compute.  In
-// each half chunk the 32 exponentials (and input terms) are issued before the sequential
-// FMA chain.  Each thread writes its C_t[s] h_t[s] terms to a swizzled buffer; after the
-// half chunk, one thread per (4 steps, channel) sums the 16 states (bank-conflict-free on
-// both sides) and the y rows leave as 16-byte stores.
+// Selective scan + state carry ([JJ] §数学表示 4, eq. (2), Euler form):
+//   h_t[s] = exp(delta_t * A[s]) h_{t-1}[s] + delta_t B_t[s] x_t,   y_t = sum_s C_t[s] h_t[s]
+// One CTA = 8 channels x 16 states (128 threads); a warp owns two channels, a lane owns one
+// (channel, state) and keeps h in a register, walking T in order (no inter-chunk pass).
+// Each 64-step chunk arrives by three TMA loads (delta and x [8 channels x 64 steps],
+// B/C [32 rows x 68 steps: rows padded so that the 16 state lanes of one step hit distinct
+// banks]) into a 4-stage ring completed on mbarriers; loads past T are zero-filled, so
+// delta = 0 leaves the state unchanged.  Per chunk each warp first forms delta*x for its two
+// channels (once per step, not once per state), then runs the recurrence, writes its C*h
+// terms to a warp-private, XOR-swizzled buffer and sums the 16 states per (step, channel)
+// inside the warp: no CTA barrier until the end of the chunk, where the gathered 8-channel
+// y rows leave as 16-byte stores.
 //   xcT [B, Di, Tp] bf16; dT [B, Di, Tp] fp32; bcT [B, 32, Tp] fp32 (B rows 0..15, C rows
-//   16..31); Tp is a multiple of 8 and steps at or beyond T read as zero, so delta = 0
-//   leaves the state unchanged; A [Di, 16]; y [B*T, Di] bf16 (not gated); state [B, Di, 16].
+//   16..31), all read through tensor maps of extent T; A [Di, 16]; y [B*T, Di] bf16 (the
+//   SiLU(z) gate is applied by the branch norm); state [B, Di, 16] fp32.
 // ----------------------------------------------------------------------------------------
-constexpr int SCAN_CH = 8;            // channels per CTA
+constexpr int SCAN_CH = 8;            // channels per CTA (two per warp)
 constexpr int SCAN_TC = 64;           // time steps per chunk
-constexpr int SCAN_NST = 4;           // pipeline stages
-constexpr int SCAN_HALF = 32;         // steps per compute/reduce round
+constexpr int SCAN_NST = 4;           // TMA stages
+constexpr int SCAN_HALF = 32;         // steps per reduction round
+constexpr int SCAN_BCW = SCAN_TC + 4; // padded B/C row (the TMA box is this wide)
 constexpr int SCAN_THREADS = SCAN_CH * 16;
 
 struct ScanStage {
-  float d[SCAN_CH][SCAN_TC];          // delta
-  __nv_bfloat16 x[SCAN_CH][SCAN_TC];  // x
-  float bc[32][SCAN_TC + 4];          // [state (B 0..15, C 16..31)][t]; rows padded to 272 B so the
-                                      // 16 state lanes reading one step hit distinct banks
+  float d[SCAN_CH][SCAN_TC];          // delta      (box {64, 8} fp32, 2048 B)
+  __nv_bfloat16 x[SCAN_CH][SCAN_TC];  // x          (box {64, 8} bf16, 1024 B)
+  float bc[32][SCAN_BCW];             // B, C rows  (box {68, 32} fp32, 8704 B)
 };
+static_assert(sizeof(ScanStage) == 2048 + 1024 + 8704, "stage layout must match the TMA boxes");
+static_assert(sizeof(ScanStage) % 128 == 0, "stages stay 128-byte aligned");
+
 struct ScanSmem {
   ScanStage st[SCAN_NST];
-  float part[SCAN_HALF / 4][16][SCAN_CH][4];   // C*h terms: [t/4][state][channel ^ (state&7)][t%4]
-  __nv_bfloat16 ys[SCAN_HALF][SCAN_CH];
+  float part[4][SCAN_HALF * 2 * 16];           // per warp: [step/4 * 2 + channel][slot][4], slot = state ^ (row & 7)
+  float dx[4][2][SCAN_TC];                     // per warp: delta * x of its two channels
+  __nv_bfloat16 ys[2][SCAN_TC][SCAN_CH];       // y rows of a chunk, double-buffered
+  uint64_t full[SCAN_NST];
+  int abort;
 };
+constexpr int SCAN_SMEM = (int)sizeof(ScanSmem) + 128;   // + alignment slack
 
 __global__ void __launch_bounds__(SCAN_THREADS)
-    selective_scan_kernel(const __nv_bfloat16* __restrict__ xcT, const float* __restrict__ dT,
-                          const float* __restrict__ bcT, const float* __restrict__ A, __nv_bfloat16* __restrict__ y,
-                          float* __restrict__ state, int T, int Tp, int Di) {
-  extern __shared__ __align__(16) uint8_t scan_smem_raw[];
-  ScanSmem& sm = *reinterpret_cast<ScanSmem*>(scan_smem_raw);
+    selective_scan_kernel(const __grid_constant__ CUtensorMap mapD, const __grid_constant__ CUtensorMap mapX,
+                          const __grid_constant__ CUtensorMap mapBC, const float* __restrict__ A,
+                          __nv_bfloat16* __restrict__ y, float* __restrict__ state, int T, int Di, DevStatus* status) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ uint8_t scan_smem_raw[];
+  ScanSmem& sm = *reinterpret_cast<ScanSmem*>((reinterpret_cast<uintptr_t>(scan_smem_raw) + 127) & ~uintptr_t(127));
   const int tid = threadIdx.x;
-  const int cl = tid >> 4;         // channel within CTA
-  const int s = tid & 15;          // state
+  const int warp = tid >> 5, lane = tid & 31;
+  const int chl = lane >> 4;       // which of the warp's two channels
+  const int s = lane & 15;         // state
+  const int cw = warp * 2 + chl;   // channel within the CTA
   const int c0 = blockIdx.x * SCAN_CH;
   const int b = blockIdx.y;
-  const int c = c0 + cl;
+  const int c = c0 + cw;
   const int n_chunks = (T + SCAN_TC - 1) / SCAN_TC;
+  const int row_dx = b * Di + c0;  // first row of this CTA in the delta / x maps
   const float A2 = A[(size_t)c * 16 + s] * 1.4426950408889634f;   // exp(d*A) = 2^(d*A*log2 e)
 
-  // cp.async of chunk k: delta 8 rows x 16 pieces, x 8 rows x 8 pieces, B/C 32 rows x 16
-  // pieces = 704 pieces of 16 bytes, 5.5 per thread
-  auto load_chunk = [&](int k) {
-    ScanStage& S = sm.st[k % SCAN_NST];
-    const int t0 = k * SCAN_TC;
-    for (int i = tid; i < 704; i += SCAN_THREADS) {
-      if (i < 128) {
-        const int ch = i >> 4, pc = i & 15, t = t0 + pc * 4;
-        const int nb = t >= T ? 0 : min(16, (T - t) * 4);
-        cp_async16(&S.d[ch][pc * 4], dT + ((size_t)b * Di + c0 + ch) * Tp + (t >= T ? 0 : t), nb);
-      } else if (i < 192) {
-        const int j = i - 128, ch = j >> 3, pc = j & 7, t = t0 + pc * 8;
-        const int nb = t >= T ? 0 : min(16, (T - t) * 2);
-        cp_async16(&S.x[ch][pc * 8], xcT + ((size_t)b * Di + c0 + ch) * Tp + (t >= T ? 0 : t), nb);
-      } else {
-        const int j = i - 192, r = j >> 4, pc = j & 15, t = t0 + pc * 4;
-        const int nb = t >= T ? 0 : min(16, (T - t) * 4);
-        cp_async16(&S.bc[r][pc * 4], bcT + ((size_t)b * 32 + r) * Tp + (t >= T ? 0 : t), nb);
-      }
-    }
-  };
-
-  for (int k = 0; k < SCAN_NST - 1; ++k) {
-    if (k < n_chunks) load_chunk(k);
-    cp_async_commit();
+  if (tid == 0) {
+    for (int i = 0; i < SCAN_NST; ++i) mbar_init(&sm.full[i], 1);
+    sm.abort = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&mapD);
+    tma_prefetch_desc(&mapX);
+    tma_prefetch_desc(&mapBC);
   }
+  __syncthreads();
+  auto issue = [&](int k) {        // one thread: the three loads of chunk k
+    ScanStage& S = sm.st[k % SCAN_NST];
+    uint64_t* bar = &sm.full[k % SCAN_NST];
+    mbar_arrive_expect_tx(bar, (uint32_t)sizeof(ScanStage));
+    tma_load_2d(&S.d[0][0], &mapD, bar, k * SCAN_TC, row_dx);
+    tma_load_2d(&S.x[0][0], &mapX, bar, k * SCAN_TC, row_dx);
+    tma_load_2d(&S.bc[0][0], &mapBC, bar, k * SCAN_TC, b * 32);
+  };
+  int issued = 0;
+  if (tid == 0)
+    for (; issued < SCAN_NST - 1 && issued < n_chunks; ++issued) issue(issued);
+
   float h = 0.f;
-  const int sw = s & 7;
-  for (int k = 0; k < n_chunks; ++k) {
-    cp_async_wait<SCAN_NST - 2>();
-    __syncthreads();                       // chunk k visible; the stage of chunk k-1 is free
-    if (k + SCAN_NST - 1 < n_chunks) load_chunk(k + SCAN_NST - 1);
-    cp_async_commit();
+  float* part = sm.part[warp];
+  float* dxw = &sm.dx[warp][0][0];
+  int k = 0;
+  for (; k < n_chunks; ++k) {
+    // the stage of chunk k-1 is free (barrier at the end of the previous chunk)
+    if (tid == 0 && issued < n_chunks) issue(issued++);
+    const bool ok = mbar_wait(&sm.full[k % SCAN_NST], (uint32_t)(k / SCAN_NST) & 1u, &sm.abort, status, 301);
     const ScanStage& S = sm.st[k % SCAN_NST];
+    {  // delta * x of the warp's two channels: lane -> (channel lane/16, steps 4*(lane%16) ..)
+      const int ch = lane >> 4, t4 = (lane & 15) * 4;
+      const float4 d4 = *reinterpret_cast<const float4*>(&S.d[warp * 2 + ch][t4]);
+      const uint2 x2 = *reinterpret_cast<const uint2*>(&S.x[warp * 2 + ch][t4]);
+      const __nv_bfloat162 xa = *reinterpret_cast<const __nv_bfloat162*>(&x2.x);
+      const __nv_bfloat162 xb = *reinterpret_cast<const __nv_bfloat162*>(&x2.y);
+      *reinterpret_cast<float4*>(dxw + ch * SCAN_TC + t4) =
+          make_float4(d4.x * __low2float(xa), d4.y * __high2float(xa), d4.z * __low2float(xb), d4.w * __high2float(xb));
+    }
+    __syncwarp();
 #pragma unroll 1
     for (int hc = 0; hc < SCAN_TC; hc += SCAN_HALF) {
-      float a[SCAN_HALF], q[SCAN_HALF];
 #pragma unroll
       for (int u = 0; u < SCAN_HALF; u += 4) {
-        const float4 d4 = *reinterpret_cast<const float4*>(&S.d[cl][hc + u]);
-        const uint2 x2 = *reinterpret_cast<const uint2*>(&S.x[cl][hc + u]);
+        const float4 d4 = *reinterpret_cast<const float4*>(&S.d[cw][hc + u]);
+        const float4 q4 = *reinterpret_cast<const float4*>(dxw + chl * SCAN_TC + hc + u);
         const float4 b4 = *reinterpret_cast<const float4*>(&S.bc[s][hc + u]);
-        const __nv_bfloat162 xa = *reinterpret_cast<const __nv_bfloat162*>(&x2.x);
-        const __nv_bfloat162 xb = *reinterpret_cast<const __nv_bfloat162*>(&x2.y);
-        a[u] = ex2_approx(d4.x * A2); a[u + 1] = ex2_approx(d4.y * A2);
-        a[u + 2] = ex2_approx(d4.z * A2); a[u + 3] = ex2_approx(d4.w * A2);
-        q[u] = d4.x * __low2float(xa) * b4.x; q[u + 1] = d4.y * __high2float(xa) * b4.y;
-        q[u + 2] = d4.z * __low2float(xb) * b4.z; q[u + 3] = d4.w * __high2float(xb) * b4.w;
-      }
-#pragma unroll
-      for (int u = 0; u < SCAN_HALF; u += 4) {
         const float4 c4 = *reinterpret_cast<const float4*>(&S.bc[16 + s][hc + u]);
+        const float a0 = ex2_approx(d4.x * A2), a1 = ex2_approx(d4.y * A2);
+        const float a2 = ex2_approx(d4.z * A2), a3 = ex2_approx(d4.w * A2);
         float4 v;
-        h = fmaf(a[u], h, q[u]); v.x = c4.x * h;
-        h = fmaf(a[u + 1], h, q[u + 1]); v.y = c4.y * h;
-        h = fmaf(a[u + 2], h, q[u + 2]); v.z = c4.z * h;
-        h = fmaf(a[u + 3], h, q[u + 3]); v.w = c4.w * h;
-        *reinterpret_cast<float4*>(&sm.part[u >> 2][s][cl ^ sw][0]) = v;
+        h = fmaf(a0, h, q4.x * b4.x); v.x = c4.x * h;
+        h = fmaf(a1, h, q4.y * b4.y); v.y = c4.y * h;
+        h = fmaf(a2, h, q4.z * b4.z); v.z = c4.z * h;
+        h = fmaf(a3, h, q4.w * b4.w); v.w = c4.w * h;
+        const int row = (u >> 2) * 2 + chl;
+        *reinterpret_cast<float4*>(part + (row * 16 + (s ^ (row & 7))) * 4) = v;
       }
-      __syncthreads();
-      // sum over the 16 states: thread -> (4 steps tg, channel ch), 8 x 8 = 64 threads
-      if (tid < 64) {
-        const int tg = tid >> 3, ch = tid & 7;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      __syncwarp();
+      {  // lane -> (row = lane/2: step group and channel, pair = two of its four steps)
+        const int row = lane >> 1, pair = lane & 1;
+        float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
         for (int st = 0; st < 16; ++st) {
-          const float4 q4 = *reinterpret_cast<const float4*>(&sm.part[tg][st][ch ^ (st & 7)][0]);
-          acc.x += q4.x; acc.y += q4.y; acc.z += q4.z; acc.w += q4.w;
+          const float2 v2 = *reinterpret_cast<const float2*>(part + (row * 16 + (st ^ (row & 7))) * 4 + pair * 2);
+          acc.x += v2.x;
+          acc.y += v2.y;
         }
-        sm.ys[tg * 4 + 0][ch] = __float2bfloat16_rn(acc.x);
-        sm.ys[tg * 4 + 1][ch] = __float2bfloat16_rn(acc.y);
-        sm.ys[tg * 4 + 2][ch] = __float2bfloat16_rn(acc.z);
-        sm.ys[tg * 4 + 3][ch] = __float2bfloat16_rn(acc.w);
+        const int t = hc + (row >> 1) * 4 + pair * 2;
+        const int ch = warp * 2 + (row & 1);
+        sm.ys[k & 1][t][ch] = __float2bfloat16_rn(acc.x);
+        sm.ys[k & 1][t + 1][ch] = __float2bfloat16_rn(acc.y);
       }
-      __syncthreads();
-      if (tid < SCAN_HALF) {
-        const int t = k * SCAN_TC + hc + tid;
-        if (t < T)
-          *reinterpret_cast<uint4*>(y + ((size_t)b * T + t) * Di + c0) = *reinterpret_cast<const uint4*>(&sm.ys[tid][0]);
-      }
+      __syncwarp();
     }
+    if (__syncthreads_or(ok ? 0 : 1)) break;   // a wait gave up: every thread leaves together
+    if (tid < SCAN_TC) {
+      const int t = k * SCAN_TC + tid;
+      if (t < T)
+        *reinterpret_cast<uint4*>(y + ((size_t)b * T + t) * Di + c0) = *reinterpret_cast<const uint4*>(&sm.ys[k & 1][tid][0]);
+    }
+  }
+  if (k < n_chunks) {
+    // gave up: wait (bounded) for the loads still in flight before the CTA exits
+    if (tid == 0)
+      for (int j = k; j < issued; ++j)
+        mbar_wait(&sm.full[j % SCAN_NST], (uint32_t)(j / SCAN_NST) & 1u, nullptr, status, 302);
+    return;
   }
   state[((size_t)b * Di + c) * 16 + s] = h;
 }

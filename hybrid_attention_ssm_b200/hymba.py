@@ -102,6 +102,7 @@ def lib():
             "hymba_mixer_decode_noalloc": ([ctypes.POINTER(LayerCfg), ctypes.POINTER(LayerWeights), _vp, _c_int,
                                             _c_int, ctypes.POINTER(KVCache), _vp, _vp, _vp, _vp, _vp], _c_int),
             "hymba_profile_begin": ([_c_int], _c_int),
+            "hymba_profile_read": ([ctypes.POINTER(ProfRecord), _c_int, ctypes.POINTER(_c_int)], _c_int),
             "hymba_profile_end": ([ctypes.POINTER(ProfRecord), _c_int, ctypes.POINTER(_c_int)], _c_int),
         }
         for name, (args, res) in sig.items():
@@ -144,18 +145,23 @@ class DeviceWeights:
     """A layer's weights in device memory plus the C struct pointing at them."""
 
     def __init__(self, w: dict, device="cuda"):
+        """w: numpy arrays (as synth.layer_weights returns them) or float32 torch tensors."""
+        def dev(a, dtype):
+            if isinstance(a, torch.Tensor):
+                return a.to(device=device, dtype=torch.float32).contiguous().to(dtype)
+            return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device).to(dtype)
+
         self.t = {}
         for k in _BF16_W:
-            self.t[k] = torch.from_numpy(np.ascontiguousarray(w[k], dtype=np.float32)).to(device).to(torch.bfloat16)
-        self.t["w_out"] = torch.from_numpy(np.ascontiguousarray(w["w_out"], dtype=np.float32)).to(device).to(
-            torch.float16)
+            self.t[k] = dev(w[k], torch.bfloat16)
+        self.t["w_out"] = dev(w["w_out"], torch.float16)
         for k in _F32_W:
-            self.t[k] = torch.from_numpy(np.ascontiguousarray(w[k], dtype=np.float32)).to(device)
-        wdt = np.ascontiguousarray(w["w_dt"], dtype=np.float32)
+            self.t[k] = dev(w[k], torch.float32)
+        wdt = dev(w["w_dt"], torch.float32)
         ld = (wdt.shape[1] + 3) // 4 * 4
-        pad = np.zeros((wdt.shape[0], ld), dtype=np.float32)
+        pad = torch.zeros(wdt.shape[0], ld, dtype=torch.float32, device=device)
         pad[:, :wdt.shape[1]] = wdt
-        self.t["w_dt"] = torch.from_numpy(pad).to(device)
+        self.t["w_dt"] = pad
         self.c = LayerWeights(ptr(self.t["meta"]), ptr(self.t["w_in"]), ptr(self.t["conv_w"]),
                               ptr(self.t["conv_b"]), ptr(self.t["w_x"]), ptr(self.t["w_dt"]), ld,
                               ptr(self.t["dt_bias"]), ptr(self.t["A"]), ptr(self.t["g_attn"]),
@@ -290,6 +296,15 @@ def interleave_gate_up(w_gate, w_up):
 
 def profile_begin(max_records=8192):
     check(lib().hymba_profile_begin(max_records))
+
+
+def profile_read(max_records=8192):
+    """The records so far without clearing them (recording stops); after a captured CUDA
+    graph replays, these are that replay's kernel times."""
+    recs = (ProfRecord * max_records)()
+    n = ctypes.c_int()
+    check(lib().hymba_profile_read(recs, max_records, ctypes.byref(n)))
+    return [(recs[i].name.decode(), float(recs[i].ms)) for i in range(n.value)]
 
 
 def profile_end(max_records=8192):

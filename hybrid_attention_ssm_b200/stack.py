@@ -15,8 +15,30 @@ from . import hymba as H
 from . import synth
 
 
+def _device_weights(dl, F, seed, layer, dt_mean, dt_std, device):
+    """Random-init layer and block weights drawn on the device (same distributions as
+    synth.layer_weights / synth.block_weights, a torch generator instead of numpy's), for
+    timing runs where drawing 32 layers on the host would dominate."""
+    g = torch.Generator(device=device)
+    g.manual_seed(1000003 * (seed + 1) + layer)
+    d, Di, S, R = dl.d_model, dl.d_inner, dl.d_state, dl.dt_rank
+    n = lambda *shape, std=0.02, mean=0.0: torch.randn(*shape, generator=g, device=device) * std + mean
+    w = {
+        "meta": n(dl.n_meta, d), "w_in": n(dl.in_width, d), "conv_w": n(Di, dl.d_conv), "conv_b": n(Di),
+        "w_x": n(R + 2 * S, Di), "w_dt": n(Di, R), "dt_bias": n(Di, std=dt_std, mean=dt_mean),
+        "A": -torch.arange(1, S + 1, dtype=torch.float32, device=device).repeat(Di, 1),
+        "g_attn": n(dl.attn_width, mean=1.0), "g_ssm": n(Di, mean=1.0), "w_out": n(d, dl.out_in_width),
+    }
+    gate, up = n(F, d), n(F, d)
+    gu = torch.cat([gate.view(F // 32, 32, d), up.view(F // 32, 32, d)], dim=1).view(2 * F, d)
+    blk = {"g1": n(d, mean=1.0), "g2": n(d, mean=1.0), "w_gu": gu.to(torch.bfloat16),
+           "w_down": n(d, F).to(torch.float16)}
+    return w, blk
+
+
 class HymbaStack:
-    def __init__(self, wl: synth.Workload, seed: int = 0, device="cuda", keep_host_weights=False):
+    def __init__(self, wl: synth.Workload, seed: int = 0, device="cuda", keep_host_weights=False,
+                 device_init=False):
         self.wl = wl
         dims = wl.dims
         self.B, self.N = wl.batch, wl.n_tokens
@@ -41,6 +63,10 @@ class HymbaStack:
         self.host = [] if keep_host_weights else None
         for l in range(self.L):
             dl = dims.replace(is_global=is_global[l], kv_role=self.role[l])
+            if device_init:
+                w, dev = _device_weights(dl, self.F, seed, l, wl.dt_bias_mean, wl.dt_bias_std, device)
+                self.layers.append((dl, H.DeviceWeights(w, device), dev))
+                continue
             w = synth.layer_weights(dl, seed=seed, layer=l, dt_bias_mean=wl.dt_bias_mean, dt_bias_std=wl.dt_bias_std)
             bw = synth.block_weights(dl, self.F, seed=seed, layer=l)
             dev = {
@@ -53,7 +79,11 @@ class HymbaStack:
             if keep_host_weights:
                 self.host.append((dl, w, bw))
         # the stack's meta tokens R (those of layer 0's parameter set)
-        self.meta = torch.from_numpy(synth.layer_weights(dims, seed=seed, layer=0)["meta"]).to(device).to(torch.bfloat16)
+        if device_init:
+            self.meta = self.layers[0][1].t["meta"]
+        else:
+            self.meta = torch.from_numpy(synth.layer_weights(dims, seed=seed, layer=0)["meta"]).to(device).to(
+                torch.bfloat16)
         rows = self.B * self.T
         bf = dict(dtype=torch.bfloat16, device=device)
         self.Hs = [torch.empty(self.B, self.T, dims.d_model, **bf) for _ in range(2)]

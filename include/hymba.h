@@ -285,12 +285,17 @@ int hymba_mixer_decode_noalloc(const hymba_layer_cfg* cfg, const hymba_layer_wei
  * pair of CUDA events on its stream (the events are created on the host by the first
  * hymba_profile_begin; no device memory is allocated).  hymba_profile_end synchronises on
  * the recorded events and returns, in launch order, each kernel's name and elapsed time.
- * At most max_records launches are recorded; not thread-safe. */
+ * At most max_records launches are recorded; not thread-safe.
+ * hymba_profile_read stops recording and returns the same records without clearing them:
+ * after the launches were captured into a CUDA graph, every replay re-records the events,
+ * and a read after each replay gives that replay's kernel times without host launch gaps.
+ * hymba_profile_end then clears the records. */
 typedef struct hymba_prof_record {
   char name[24];
   float ms;
 } hymba_prof_record;
 int hymba_profile_begin(int max_records);
+int hymba_profile_read(hymba_prof_record* out, int max_records, int* n_records);
 int hymba_profile_end(hymba_prof_record* out, int max_records, int* n_records);
 
 #ifdef __cplusplus
