@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
   pdl_wait();
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem<1024>(smem_raw);
   if ((size_t)(smem - smem_raw) + ATT_USED > (size_t)ATT_SMEM) {   // cannot happen with a 1 KB-aligned window
     if (threadIdx.x == 0) report_error(p.status, DEV_ERR_BOUNDS, 299);
     return;

@@ -97,6 +97,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   return mbar_wait_slow(bar, parity, abort, st, site);
 }
 
+// Align a dynamic shared-memory base by pointer arithmetic on the shared array itself, so
+// the compiler keeps knowing the result is in shared memory and emits shared loads and
+// stores (an integer round trip would turn every access into a generic one).
+template <int ALIGN>
+__device__ __forceinline__ uint8_t* align_smem(uint8_t* raw) {
+  return raw + ((ALIGN - (smem_u32(raw) & (ALIGN - 1))) & (ALIGN - 1));
+}
+
 // ----------------------------------------------------------------------------------------
 // TMA (no multicast anywhere in this library)
 // ----------------------------------------------------------------------------------------

@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   constexpr uint32_t IDESC = make_idesc(GEMM_BM, BN, ET == ET_TF32 ? 2u : (ET == ET_BF16 ? 1u : 0u), false, false);
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem<1024>(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFFSET);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;

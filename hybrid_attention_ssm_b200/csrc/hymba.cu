@@ -7,6 +7,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
 #include <string>
 #include <utility>
@@ -214,6 +215,12 @@ int launch_gemm_bn(int bn, const CUtensorMap& m0, const CUtensorMap& m1, const C
   if constexpr (MODE != EPI_PROJ) {
     if (bn == 128) return launch_gemm_inst<128, 6, ET, MODE>(m0, m1, mb, p, grid, st, name);
   }
+  if constexpr ((MODE == EPI_PROJ || MODE == EPI_SWIGLU) && ET == ET_BF16) {
+    if (bn == 192) return launch_gemm_inst<192, 5, ET, MODE>(m0, m1, mb, p, grid, st, name);
+  }
+  if constexpr (MODE == EPI_BF16) {
+    if (bn == 224) return launch_gemm_inst<224, 5, ET, MODE>(m0, m1, mb, p, grid, st, name);
+  }
   if constexpr (any_bn && ET != ET_TF32) {
     if (bn == 160) return launch_gemm_inst<160, 5, ET, MODE>(m0, m1, mb, p, grid, st, name);
     if (bn == 64) return launch_gemm_inst<64, 8, ET, MODE>(m0, m1, mb, p, grid, st, name);
@@ -342,6 +349,23 @@ int pick_bn_cover(int n) {
 int pick_bn_wide(int m_tiles, int N, int sms) {
   return (long long)m_tiles * cdiv(N, 256) >= sms ? 256 : 128;
 }
+// Tile width among `cands` minimising (rounds of the persistent grid) x (operand bytes per
+// k-block): the mainloops run at the rate shared memory is fed, so a round of tiles costs
+// k_blocks times those bytes whether or not every SM has a tile.
+int pick_bn_rounds(int m_tiles, int N, int sms, std::initializer_list<int> cands) {
+  int best = *cands.begin();
+  double best_cost = 1e300;
+  for (int bn : cands) {
+    const long long tiles = (long long)m_tiles * cdiv(N, bn);
+    const long long rounds = (tiles + sms - 1) / sms;
+    const double cost = (double)rounds * (GEMM_BM + bn);
+    if (cost < best_cost * 0.999) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
+}
 
 void fill_rope_theta(double* theta, float base) {
   for (int j = 0; j < 32; ++j) theta[j] = std::pow((double)base, -2.0 * j / 64.0);
@@ -394,8 +418,10 @@ Dims dims_of(const hymba_layer_cfg* c) {
 
 // Split-K factors depend only on the shapes (never on the device), so workspace sizes and
 // results are reproducible: enough splits to cover ~160 SMs, capped.
+// split-K factor: as many splits as keep every tile's splits within one round of a B200's
+// 148 SMs (fixed here so that workspace sizes do not depend on the device)
 int splits_for(int tiles, int k_blocks, int cap) {
-  int s = (160 + tiles - 1) / tiles;
+  int s = 148 / tiles;
   if (s > cap) s = cap;
   if (s > k_blocks) s = k_blocks;
   return s < 1 ? 1 : s;
@@ -432,8 +458,8 @@ PrefillWs prefill_layout(const Dims& m, int B, int n_tokens, int x_has_meta) {
 }
 
 struct DecodeWs {
-  size_t proj, qrot, part, o, xc, xbc, xbc_part, y, u, acc_part, total;
-  int n_splits, xproj_split, oproj_split;
+  size_t proj, qrot, counters, part, o, xc, xbc, xbc_part, y, u, acc_part, total;
+  int n_splits, xproj_split, oproj_split, in_split;
 };
 // Key tiles of one (sequence, kv head) in decode: SWA reads the meta tiles and the ring,
 // a global layer rows 0..p of its cache (p < n_keys_max).
@@ -445,15 +471,23 @@ DecodeWs decode_layout(const Dims& m, int B, bool global, int n_keys_max) {
   w.n_splits = cdiv(decode_key_tiles(m, global, n_keys_max), DA_TPS);
   size_t off = 256;
   auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
-  w.proj = take((size_t)B * m.P * 4);
+  // in_proj split-K: enough weight tiles in flight for every SM of a B200 (148); the
+  // consumers add the slices
+  {
+    const int bn0 = B <= 64 ? 64 : (B <= 128 ? 128 : 256);
+    const int tiles = cdiv(m.P, GEMM_BM) * cdiv(B, bn0);
+    w.in_split = 148 / tiles < 1 ? 1 : (148 / tiles > DEC_MAX_IN_SPLIT ? DEC_MAX_IN_SPLIT : 148 / tiles);
+  }
+  w.proj = take((size_t)w.in_split * B * m.P * 4);
   w.qrot = take((size_t)B * m.Hq * 64 * 4);
+  w.counters = take((size_t)B * m.Hkv * 4);
   w.part = take((size_t)B * m.Hq * w.n_splits * 66 * 4);
   w.o = take((size_t)B * m.qw * 4);
   w.xc = take((size_t)B * m.Di * 2);
   w.xbc = take((size_t)B * m.ld_xbc * 4);
   const int bn = B <= 64 ? 64 : (B <= 128 ? 128 : 256);
   const int n_tiles = cdiv(B, bn);
-  w.xproj_split = splits_for(cdiv(m.R + 2 * m.S, GEMM_BM) * n_tiles, cdiv(m.Di, 64), 32);
+  w.xproj_split = splits_for(cdiv(m.R + 2 * m.S, GEMM_BM) * n_tiles, cdiv(m.Di, 64), DEC_MAX_XPROJ_SPLIT);
   w.xbc_part = take((size_t)w.xproj_split * B * m.ld_xbc * 4);
   w.y = take((size_t)B * m.Di * 4);
   w.u = take((size_t)B * m.uw * 2);
@@ -728,7 +762,10 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
       c.p.row_off1 = 0;
     }
     c.b = w->w_in; c.N = m.P; c.ldb = m.d; c.K = m.d;
-    c.bn = 256;
+    {
+      const int m_tiles = (c.a0 != nullptr ? cdiv(c.rows0, GEMM_BM) : 0) + c.nb1 * cdiv(c.rows1, GEMM_BM);
+      c.bn = pick_bn_rounds(m_tiles, m.P, dev->sms, {256, 192});
+    }
     c.name = "in_proj";
     c.mode = EPI_PROJ;
     c.p.out_batches = B;
@@ -882,7 +919,7 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     c.b = w->w_out; c.N = m.d; c.ldb = m.uw; c.K = m.uw;
     c.etype = ET_F16;
     c.name = "out_proj";
-    c.bn = pick_bn_wide(cdiv(rows, GEMM_BM), m.d, dev->sms);
+    c.bn = pick_bn_rounds(cdiv(rows, GEMM_BM), m.d, dev->sms, {256, 224, 128});
     c.mode = EPI_BF16;
     c.p.out = out;
     c.p.ld_out = m.d;
@@ -953,8 +990,10 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     c.b = x; c.N = B; c.ldb = m.d; c.K = m.d;
     c.bn = pick_bn_cover(B);
     c.name = "decode_in_proj";
-    c.mode = EPI_F32_T;
+    c.mode = EPI_F32_T_PART;
+    c.split_k = L.in_split;
     c.p.out = f32(L.proj);
+    c.p.split_stride = (long long)B * m.P;
     c.p.ld_out = m.P;
     c.p.m_valid = m.P;
     c.p.n_valid = B;
@@ -965,6 +1004,8 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
   {
     DecPrepParams pp;
     pp.proj = f32(L.proj);
+    pp.n_slices = L.in_split;
+    pp.proj_stride = (long long)B * m.P;
     pp.ld_proj = m.P;
     pp.B = B;
     pp.Di = m.Di;
@@ -983,6 +1024,8 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     pp.qrot = f32(L.qrot);
     pp.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)m.D));
     fill_rope_theta(pp.rope_theta, cfg->rope_base);
+    pp.counters = reinterpret_cast<unsigned*>(wsb + L.counters);
+    pp.n_counters = B * m.Hkv;
     const int n_rope = B * (m.Hq + (own_kv ? m.Hkv : 0)) * 32;
     prof_begin("decode_prep", st);
     HY_CUDA(launch_pdl(decode_prep_kernel, dim3(pp.conv_blocks + cdiv(n_rope, 256)), dim3(256), 0, st, pp));
@@ -1029,6 +1072,9 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     if (ap.n_splits > L.n_splits) return fail(HYMBA_ERR_WORKSPACE, "decode workspace sized for fewer keys");
     ap.n_items = B * m.Hkv * ap.n_splits;
     ap.part = f32(L.part);
+    ap.out = f32(L.o);
+    ap.ld_out = m.qw;
+    ap.counters = reinterpret_cast<unsigned*>(wsb + L.counters);
     ap.status = status;
     static bool attr_da[64] = {false};
     int dcur = 0;
@@ -1040,10 +1086,6 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     const int grid = ap.n_items < 3 * dev->sms ? ap.n_items : 3 * dev->sms;
     prof_begin("decode_attn", st);
     HY_CUDA(launch_pdl(decode_attn_kernel, dim3(grid), dim3(DA_THREADS), DA_SMEM, st, mmk, mmv, mk, mv, ap));
-    prof_end(st);
-    prof_begin("decode_attn_combine", st);
-    HY_CUDA(launch_pdl(decode_attn_combine_kernel, dim3(m.Hq, B), dim3(64), 0, st, f32(L.part), ap.n_splits, m.Hq,
-                       f32(L.o), m.qw));
     prof_end(st);
   }
   // 4. x_proj (swap-AB, split-K into per-split slices, fixed-order sum)
@@ -1061,20 +1103,16 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     c.p.m_valid = c.rows1;
     c.p.n_valid = B;
     c.p.status = status;
-    HY_TRY(run_gemm(c, *dev, st));
-    const int n = B * m.ld_xbc;
-    prof_begin("decode_splitk_reduce", st);
-    HY_CUDA(launch_pdl(splitk_reduce_kernel, dim3(cdiv(n / 4, 256)), dim3(256), 0, st, f32(L.xbc_part), L.xproj_split, (long long)n, n, nullptr,
-                                                            f32(L.xbc), 0, (float*)nullptr, 0, 0, 0, 0));
-    prof_end(st);
-    HY_CUDA(cudaGetLastError());
+    HY_TRY(run_gemm(c, *dev, st));   // the SSM step adds the slices (fixed order)
   }
   // 5. dt_proj + softplus + state update + C.h + gate
   {
-    dim3 grid(m.Di / 16, cdiv(B, DSSM_NB));
+    dim3 grid(m.Di / DSSM_NC, cdiv(B, DSSM_NB));
     prof_begin("decode_ssm", st);
-    HY_CUDA(launch_pdl(decode_ssm_kernel, grid, dim3(256), 0, st, f32(L.xbc), m.ld_xbc, m.R, w->w_dt, w->w_dt_ld,
-                       w->dt_bias, w->A, bf(L.xc), f32(L.proj), m.P, m.xz_off + m.Di, ssm_state, f32(L.y), m.Di, B));
+    HY_CUDA(launch_pdl(decode_ssm_kernel, grid, dim3(DSSM_NB * DSSM_NC), 0, st, f32(L.xbc_part),
+                       (long long)B * m.ld_xbc, L.xproj_split, m.ld_xbc, m.R, w->w_dt, w->w_dt_ld,
+                       w->dt_bias, w->A, bf(L.xc), f32(L.proj), m.P, (long long)B * m.P, L.in_split,
+                       m.xz_off + m.Di, ssm_state, f32(L.y), m.Di, B));
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
@@ -1123,7 +1161,7 @@ int hymba_gemm_bf16(const hymba_bf16* A, const hymba_bf16* Bm, const hymba_bf16*
   GemmCall c;
   c.a1 = A; c.nb1 = 1; c.rows1 = M; c.lda1 = K; c.a1_bstride = (long long)M * K;
   c.b = Bm; c.N = N; c.ldb = K; c.K = K;
-  c.bn = pick_bn_wide(cdiv(M, GEMM_BM), N, dev->sms);
+  c.bn = pick_bn_rounds(cdiv(M, GEMM_BM), N, dev->sms, {256, 224, 128});
   c.mode = EPI_BF16;
   c.p.out = C;
   c.p.ld_out = N;
@@ -1160,7 +1198,7 @@ int hymba_ffn_swiglu(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hym
     GemmCall c;
     c.a1 = h; c.nb1 = 1; c.rows1 = rows; c.lda1 = d; c.a1_bstride = (long long)rows * d;
     c.b = w_gate_up; c.N = 2 * F; c.ldb = d; c.K = d;
-    c.bn = pick_bn_wide(cdiv(rows, GEMM_BM), 2 * F, dev->sms);
+    c.bn = pick_bn_rounds(cdiv(rows, GEMM_BM), 2 * F, dev->sms, {256, 192, 128});
     c.name = "ffn_gate_up";
     c.mode = EPI_SWIGLU;
     c.p.out = act;
@@ -1175,7 +1213,7 @@ int hymba_ffn_swiglu(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hym
     c.b = w_down; c.N = d; c.ldb = F; c.K = F;
     c.etype = ET_F16;
     c.name = "ffn_down";
-    c.bn = pick_bn_wide(cdiv(rows, GEMM_BM), d, dev->sms);
+    c.bn = pick_bn_rounds(cdiv(rows, GEMM_BM), d, dev->sms, {256, 224, 128});
     c.mode = EPI_BF16;
     c.p.out = out;
     c.p.ld_out = d;
@@ -1228,7 +1266,7 @@ int hymba_selftest_wait_timeout(void* ws, size_t ws_bytes, hymba_stream stream) 
 // ========================================================================================
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB, held by every GPU that loads the library
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;   // 32 MiB, held by every GPU that loads the library
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 void* g_noalloc_ptr[64] = {nullptr};

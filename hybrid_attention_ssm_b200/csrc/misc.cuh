@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(NORM_THREADS)
   pdl_wait();
   pdl_trigger();
   extern __shared__ uint8_t norm_smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(norm_smem_raw) + 127) & ~uintptr_t(127));
+  uint8_t* base = align_smem<128>(norm_smem_raw);
   __shared__ uint64_t full[NORM_STAGES];
   __shared__ float red[2][4][2];   // double-buffered by row parity: one barrier per row
   __shared__ int abort_flag;
@@ -102,6 +102,21 @@ __global__ void __launch_bounds__(NORM_THREADS)
   if (t == 0)
     for (; issued < NORM_STAGES && issued < n_mine; ++issued) issue(issued);
   const float inv_a = 1.f / (float)attn_w, inv_s = 1.f / (float)di;
+  // this thread's columns are the same in every row: their gains stay in registers
+  float ga[NORM_MAXO][4], gs[NORM_MAXY][8];
+#pragma unroll
+  for (int k = 0; k < NORM_MAXO; ++k) {
+    const int c = (t + k * NORM_THREADS) * 4;
+    if (c < attn_w) {
+      const float4 g = *reinterpret_cast<const float4*>(g_attn + c);
+      ga[k][0] = g.x; ga[k][1] = g.y; ga[k][2] = g.z; ga[k][3] = g.w;
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < NORM_MAXY; ++k) {
+    const int c = (t + k * NORM_THREADS) * 8;
+    if (c < di) load8(g_ssm + c, gs[k]);
+  }
   int i = 0;
   for (; i < n_mine; ++i) {
     const size_t row = (size_t)blockIdx.x + (size_t)i * gridDim.x;
@@ -157,21 +172,19 @@ __global__ void __launch_bounds__(NORM_THREADS)
 #pragma unroll
     for (int k = 0; k < NORM_MAXO; ++k) {
       const int c = (t + k * NORM_THREADS) * 4;
-      if (c < attn_w) {
-        const float4 g = *reinterpret_cast<const float4*>(g_attn + c);
-        *reinterpret_cast<uint2*>(u_r + c) = make_uint2(pack_f16x2(fo[k][0] * ra * g.x, fo[k][1] * ra * g.y),
-                                                        pack_f16x2(fo[k][2] * ra * g.z, fo[k][3] * ra * g.w));
-      }
+      if (c < attn_w)
+        *reinterpret_cast<uint2*>(u_r + c) =
+            make_uint2(pack_f16x2(fo[k][0] * ra * ga[k][0], fo[k][1] * ra * ga[k][1]),
+                       pack_f16x2(fo[k][2] * ra * ga[k][2], fo[k][3] * ra * ga[k][3]));
     }
 #pragma unroll
     for (int k = 0; k < NORM_MAXY; ++k) {
       const int c = (t + k * NORM_THREADS) * 8;
       if (c < di) {
-        float g[8];
-        load8(g_ssm + c, g);
         uint32_t pk[4];
 #pragma unroll
-        for (int e = 0; e < 8; e += 2) pk[e / 2] = pack_f16x2(fy[k][e] * rs * g[e], fy[k][e + 1] * rs * g[e + 1]);
+        for (int e = 0; e < 8; e += 2)
+          pk[e / 2] = pack_f16x2(fy[k][e] * rs * gs[k][e], fy[k][e + 1] * rs * gs[k][e + 1]);
         *reinterpret_cast<uint4*>(u_r + attn_w + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
     }
@@ -224,8 +237,25 @@ __global__ void swa_cache_finalize_kernel(const __half* __restrict__ vk, const _
 // the cache.  Conv: window [state(3), x_new] -> xc = SiLU(b + w . window), the state shifts;
 // x from proj [B, ld_proj] fp32 at column off_x; xc [B, Di] bf16; state [B, Di, 3] fp32.
 // ----------------------------------------------------------------------------------------
+// Sum of the n <= NMAX split-K slices of an fp32 projection, in slice order (deterministic).
+// The bound is a compile-time constant so that every load is issued before the first add.
+template <int NMAX>
+__device__ __forceinline__ float sum_slices(const float* p, long long stride, int n) {
+  float v[NMAX];
+#pragma unroll
+  for (int i = 0; i < NMAX; ++i) v[i] = i < n ? p[i * stride] : 0.f;
+  float s = v[0];
+#pragma unroll
+  for (int i = 1; i < NMAX; ++i) s += v[i];
+  return s;
+}
+constexpr int DEC_MAX_IN_SPLIT = 4;     // in_proj split-K slices (the layout caps them)
+constexpr int DEC_MAX_XPROJ_SPLIT = 8;  // x_proj split-K slices (the layout caps them)
+
 struct DecPrepParams {
-  const float* proj;
+  const float* proj;          // in_proj output: n_slices split-K slices [B, ld_proj], slice stride proj_stride
+  int n_slices;
+  long long proj_stride;
   int ld_proj, B, Di, off_x, conv_blocks;
   const float* conv_w;
   const float* conv_b;
@@ -236,6 +266,8 @@ struct DecPrepParams {
   float* qrot;
   float scale_log2;
   double rope_theta[32];
+  unsigned* counters;         // [B * Hkv] split counters of the attention step, zeroed here
+  int n_counters;
 };
 
 __global__ void __launch_bounds__(256) decode_prep_kernel(const __grid_constant__ DecPrepParams p) {
@@ -247,7 +279,7 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(const __grid_constant_
     const int b = i / p.Di, c = i % p.Di;
     float* st = p.conv_state + (size_t)i * 3;
     const float x0 = st[0], x1 = st[1], x2 = st[2];
-    const float xn = p.proj[(size_t)b * p.ld_proj + p.off_x + c];
+    const float xn = sum_slices<DEC_MAX_IN_SPLIT>(p.proj + (size_t)b * p.ld_proj + p.off_x + c, p.proj_stride, p.n_slices);
     const float4 wv = *reinterpret_cast<const float4*>(p.conv_w + (size_t)c * 4);
     const float acc = p.conv_b[c] + wv.x * x0 + wv.y * x1 + wv.z * x2 + wv.w * xn;
     p.xc[i] = __float2bfloat16_rn(silu_f(acc));
@@ -258,6 +290,7 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(const __grid_constant_
   }
   const int n_heads = p.Hq + (p.write_kv ? p.Hkv : 0);
   const int i = (blockIdx.x - p.conv_blocks) * 256 + threadIdx.x;
+  if (i < p.n_counters) p.counters[i] = 0u;
   if (i >= p.B * n_heads * 32) return;
   const int j = i & 31, hh = (i >> 5) % n_heads, b = (i >> 5) / n_heads;
   // angle p * theta_j reduced mod 2 pi in double precision, then the fp32 sincos
@@ -266,8 +299,9 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(const __grid_constant_
   float sn, cs;
   sincosf((float)a, &sn, &cs);
   const float* pr = p.proj + (size_t)b * p.ld_proj;
+  auto P = [&](int col) { return sum_slices<DEC_MAX_IN_SPLIT>(pr + col, p.proj_stride, p.n_slices); };
   if (hh < p.Hq) {
-    const float x1 = pr[hh * 64 + j], x2 = pr[hh * 64 + j + 32];
+    const float x1 = P(hh * 64 + j), x2 = P(hh * 64 + j + 32);
     float* q = p.qrot + ((size_t)b * p.Hq + hh) * 64;
     q[j] = (x1 * cs - x2 * sn) * p.scale_log2;
     q[j + 32] = (x2 * cs + x1 * sn) * p.scale_log2;
@@ -275,9 +309,8 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(const __grid_constant_
   }
   const int g = hh - p.Hq;
   const int kvw = p.Hkv * 64;
-  const float* kp = pr + p.Hq * 64 + g * 64;
-  const float* vp = kp + kvw;
-  const float k1 = kp[j], k2 = kp[j + 32];
+  const int kc = p.Hq * 64 + g * 64, vc = kc + kvw;
+  const float k1 = P(kc + j), k2 = P(kc + j + 32);
   size_t row;
   __half *dk, *dv;
   if (p.is_global) {
@@ -291,8 +324,8 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(const __grid_constant_
   }
   dk[j] = __float2half_rn(k1 * cs - k2 * sn);
   dk[j + 32] = __float2half_rn(k2 * cs + k1 * sn);
-  dv[j] = __float2half_rn(vp[j]);
-  dv[j + 32] = __float2half_rn(vp[j + 32]);
+  dv[j] = __float2half_rn(P(vc + j));
+  dv[j + 32] = __float2half_rn(P(vc + j + 32));
 }
 
 // ----------------------------------------------------------------------------------------
@@ -303,17 +336,25 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(const __grid_constant_
 // are visited in slot order (the softmax does not depend on the order).  Work item =
 // (b, g, split of DA_TPS tiles of 64 keys); persistent CTAs walk their items while one
 // thread keeps DA_STAGES K/V tile pairs in flight by TMA (128-byte swizzled boxes of the
-// [rows, Hkv*64] caches), so loads of the next item overlap the current one.  The query
-// heads of group g share each K/V tile: scores (thread = key, 3 heads), an online softmax
-// per head across the item's tiles, PV (thread = dim pair x key quarter).  Partial (m, l,
-// o[64]) per (b, head, split) go to part [B, Hq, n_splits, 66]; the combine kernel merges.
+// [rows, Hkv*64] caches), so loads of the next item overlap the current one.
+// The G <= 6 query heads of group g form the rows of 16 x 16 fp16 tensor-core fragments
+// (mma.sync m16n8k16, fp32 accumulation; rows >= G are zero): a tcgen05 tile would need
+// at least 64 query rows, and this kernel is bound by the K/V bytes, not by the math.  Each
+// of the 4 warps takes 16 keys of every tile: S = Q K^T from ldmatrix fragments of the
+// swizzled K tile, an online softmax in registers, O += P V with P reused from the S
+// accumulators and V fragments from ldmatrix.trans.  At the end of an item the 4 warps'
+// (m, l, O) are merged; the partial (m, l, o[64]) per (b, head, split) goes to
+// part [B, Hq, n_splits, 66], and the CTA that finishes the last split of (b, g) (a counter
+// per (b, g), zeroed by the prep kernel) merges the splits in split order into out.  Each
+// item's queries arrive by bulk copy together with its first K/V tile.
 // ----------------------------------------------------------------------------------------
 constexpr int DA_KT = 64;               // keys per tile
-constexpr int DA_STAGES = 4;
-constexpr int DA_TPS = 2;               // tiles per split
+constexpr int DA_STAGES = 3;
+constexpr int DA_TPS = 3;               // tiles per split
 constexpr int DA_THREADS = 128;
 constexpr int DA_TILE_BYTES = DA_KT * 128;
 constexpr int DEC_MAXG = 6;             // max query heads per KV head
+constexpr int DA_Q_BYTES = DEC_MAXG * 64 * 4;   // an item's queries ride with its first tile
 constexpr int DA_SMEM = DA_STAGES * 2 * DA_TILE_BYTES + 1024;
 
 struct DecAttnParams {
@@ -325,12 +366,32 @@ struct DecAttnParams {
   int rows_main;           // rows per sequence in the main cache (W or Lmax)
   int n_splits, n_items;
   float* part;
+  float* out;              // [B, ld_out] fp32: head h at columns h*64 (merged result)
+  int ld_out;
+  unsigned* counters;      // [B * Hkv], zero on entry
   DevStatus* status;
 };
 
-// element (key r, dim d) of a 64 x 64 fp16 tile stored with the 128-byte swizzle
-__device__ __forceinline__ const __half* sw128_row_chunk(const uint8_t* tile, int r, int chunk) {
-  return reinterpret_cast<const __half*>(tile + r * 128 + ((chunk ^ (r & 7)) << 4));
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr) : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr) : "memory");
+}
+// d (16x8 fp32) += a (16x16 fp16, row-major) * b (16x8 fp16, column-major)
+__device__ __forceinline__ void mma_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                          uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+               "{%0, %1, %2, %3};"
+               : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// shared address of the 16-byte chunk `chunk` of row r in a 64 x 64 fp16 tile stored with
+// the 128-byte swizzle
+__device__ __forceinline__ uint32_t sw128_addr(uint32_t tile, int r, int chunk) {
+  return tile + r * 128 + ((chunk ^ (r & 7)) << 4);
 }
 
 __global__ void __launch_bounds__(DA_THREADS)
@@ -340,14 +401,14 @@ __global__ void __launch_bounds__(DA_THREADS)
   pdl_wait();
   pdl_trigger();
   extern __shared__ uint8_t da_smem_raw[];
-  uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(da_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* tiles = align_smem<1024>(da_smem_raw);
   __shared__ uint64_t full[DA_STAGES];
-  __shared__ __align__(16) float qs[DEC_MAXG][64];
-  __shared__ __align__(16) float ps[DEC_MAXG][DA_KT];
-  __shared__ float mrun[DEC_MAXG], lrun[DEC_MAXG], alph[DEC_MAXG];
-  __shared__ __align__(16) float opart[4][DEC_MAXG][64];
-  __shared__ int abort_flag;
+  __shared__ __align__(16) float qbuf[DA_STAGES][DEC_MAXG * 64];
+  __shared__ float cm[4][8], cl[4][8];
+  __shared__ __align__(16) float co[4][8][64];
+  __shared__ int abort_flag, last_split;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gq = lane >> 2, tq = lane & 3;   // fragment row (query head) and column pair
   const int G = p.Hq / p.Hkv;
   if (tid == 0) {
     for (int i = 0; i < DA_STAGES; ++i) mbar_init(&full[i], 1);
@@ -374,7 +435,9 @@ __global__ void __launch_bounds__(DA_THREADS)
     const int ti = split * DA_TPS + pt;
     const int stg = issued % DA_STAGES;
     uint8_t* kt = tiles + stg * 2 * DA_TILE_BYTES;
-    mbar_arrive_expect_tx(&full[stg], 2 * DA_TILE_BYTES);
+    const uint32_t q_bytes = pt == 0 ? (uint32_t)(G * 64 * 4) : 0u;
+    mbar_arrive_expect_tx(&full[stg], 2 * DA_TILE_BYTES + q_bytes);
+    if (pt == 0) bulk_load(&qbuf[stg][0], p.qrot + ((size_t)b * p.Hq + g * G) * 64, q_bytes, &full[stg]);
     if (ti < p.n_meta_tiles) {
       tma_load_2d(kt, &mapMK, &full[stg], g * 64, b * p.M + ti * DA_KT);
       tma_load_2d(kt + DA_TILE_BYTES, &mapMV, &full[stg], g * 64, b * p.M + ti * DA_KT);
@@ -389,216 +452,256 @@ __global__ void __launch_bounds__(DA_THREADS)
   if (tid == 0)
     for (int k = 0; k < DA_STAGES - 1; ++k) issue_next();
 
+  const uint32_t tiles_u32 = smem_u32(tiles);
+  // ldmatrix row of this lane: K fragments (keys x dims), V fragments (.trans)
+  const int k_row = warp * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
+  const int k_chk = (lane >> 3) & 1;
+  const int v_row = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+  const int v_chk = (lane >> 4) & 1;
   int ct = 0;   // tiles consumed
   bool ok = true;
   for (int w = blockIdx.x; w < p.n_items; w += gridDim.x) {
     const int split = w % p.n_splits, bg = w / p.n_splits;
     const int g = bg % p.Hkv, b = bg / p.Hkv;
     const int nt = item_tiles(w);
-    for (int i = tid; i < G * 64; i += DA_THREADS)
-      qs[i >> 6][i & 63] = p.qrot[((size_t)b * p.Hq + g * G + (i >> 6)) * 64 + (i & 63)];
-    if (tid < G) {
-      mrun[tid] = -INFINITY;
-      lrun[tid] = 0.f;
-    }
-    float acc[DEC_MAXG][2];
+    uint32_t qa[4][2];   // Q fragments (fp16): row gq = query head (zero beyond G), 4 x 16 dims
+    float m_run = -INFINITY, l_run = 0.f;
+    float o[8][4];
 #pragma unroll
-    for (int hh = 0; hh < DEC_MAXG; ++hh) acc[hh][0] = acc[hh][1] = 0.f;
-    __syncthreads();
+    for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
     for (int t = 0; t < nt; ++t, ++ct) {
       if (tid == 0) issue_next();   // the stage of tile ct-1 was released by the last barrier
       const int stg = ct % DA_STAGES;
       if (!mbar_wait(&full[stg], (uint32_t)(ct / DA_STAGES) & 1u, &abort_flag, p.status, 501)) ok = false;
-      const uint8_t* kt = tiles + stg * 2 * DA_TILE_BYTES;
-      const uint8_t* vt = kt + DA_TILE_BYTES;
+      if (t == 0) {   // the item's queries arrived with its first tile
+        const float* q = &qbuf[stg][gq * 64];
+#pragma unroll
+        for (int st = 0; st < 4; ++st) {
+          float2 lo = make_float2(0.f, 0.f), hi = make_float2(0.f, 0.f);
+          if (gq < G) {
+            lo = *reinterpret_cast<const float2*>(q + st * 16 + 2 * tq);
+            hi = *reinterpret_cast<const float2*>(q + st * 16 + 8 + 2 * tq);
+          }
+          qa[st][0] = pack_f16x2(lo.x, lo.y);
+          qa[st][1] = pack_f16x2(hi.x, hi.y);
+        }
+      }
+      const uint32_t kt = tiles_u32 + stg * 2 * DA_TILE_BYTES;
+      const uint32_t vt = kt + DA_TILE_BYTES;
       const int ti = split * DA_TPS + t;
       const bool meta = ti < p.n_meta_tiles;
       const int key0 = meta ? ti * DA_KT : (ti - p.n_meta_tiles) * DA_KT;
       const int lim = meta ? p.M : p.n_main_valid;
-      {  // scores: thread = (key kk, heads hg, hg+2, hg+4)
-        const int kk = tid & 63, hg = tid >> 6;
-        float kf[64];
+      // S = Q K^T for this warp's 16 keys (two n-tiles of 8)
+      float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < 8; ++c) unpack8h(*reinterpret_cast<const uint4*>(sw128_row_chunk(kt, kk, c)), kf + c * 8);
-        const bool vis = key0 + kk < lim;
-#pragma unroll
-        for (int j = 0; j < 3; ++j) {
-          const int hh = hg + 2 * j;
-          if (hh < G) {
-            float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-            for (int d = 0; d < 64; d += 8) {
-              const float4 q0 = *reinterpret_cast<const float4*>(&qs[hh][d]);
-              const float4 q1 = *reinterpret_cast<const float4*>(&qs[hh][d + 4]);
-              a0 = fmaf(q0.x, kf[d], a0); a1 = fmaf(q0.y, kf[d + 1], a1);
-              a0 = fmaf(q0.z, kf[d + 2], a0); a1 = fmaf(q0.w, kf[d + 3], a1);
-              a0 = fmaf(q1.x, kf[d + 4], a0); a1 = fmaf(q1.y, kf[d + 5], a1);
-              a0 = fmaf(q1.z, kf[d + 6], a0); a1 = fmaf(q1.w, kf[d + 7], a1);
-            }
-            ps[hh][kk] = vis ? a0 + a1 : -INFINITY;
-          }
-        }
+      for (int st = 0; st < 4; ++st) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(sw128_addr(kt, k_row, 2 * st + k_chk), b0, b1, b2, b3);
+        mma_16816(s0, qa[st][0], 0u, qa[st][1], 0u, b0, b1);
+        mma_16816(s1, qa[st][0], 0u, qa[st][1], 0u, b2, b3);
       }
-      __syncthreads();
-      // online softmax per head (warp per head)
-      for (int hh = warp; hh < G; hh += 4) {
-        const float v0 = ps[hh][lane], v1 = ps[hh][lane + 32];
-        float tm = fmaxf(v0, v1);
+      // keys of this lane: tile columns warp*16 + 2tq + {0,1} (s0) and + 8 (s1)
+      const int kb = key0 + warp * 16 + 2 * tq;
+      float v[4] = {kb < lim ? s0[0] : -INFINITY, kb + 1 < lim ? s0[1] : -INFINITY,
+                    kb + 8 < lim ? s1[0] : -INFINITY, kb + 9 < lim ? s1[1] : -INFINITY};
+      float tm = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
+      tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 1));
+      tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 2));
+      const float m_new = fmaxf(m_run, tm);
+      float al = 1.f, e[4] = {0.f, 0.f, 0.f, 0.f};
+      if (m_new != -INFINITY) {          // some key of this warp visible so far
+        al = ex2_approx(m_run - m_new);  // 0 while nothing was accumulated
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, o));
-        const float m_old = mrun[hh];
-        const float m_new = fmaxf(m_old, tm);        // finite: every tile holds a visible key
-        const float al = m_old == -INFINITY ? 0.f : ex2_approx(m_old - m_new);
-        const float e0 = ex2_approx(v0 - m_new), e1 = ex2_approx(v1 - m_new);
-        ps[hh][lane] = e0;
-        ps[hh][lane + 32] = e1;
-        float sm = e0 + e1;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
-        __syncwarp();
-        if (lane == 0) {
-          lrun[hh] = lrun[hh] * al + sm;
-          mrun[hh] = m_new;
-          alph[hh] = al;
-        }
+        for (int i = 0; i < 4; ++i) e[i] = ex2_approx(v[i] - m_new);
       }
-      __syncthreads();
-      {  // PV: thread = (dims 2*lane, 2*lane+1; keys 16*warp ..)
-        const int kq = warp;
+      float rs = (e[0] + e[1]) + (e[2] + e[3]);
+      rs += __shfl_xor_sync(0xffffffffu, rs, 1);
+      rs += __shfl_xor_sync(0xffffffffu, rs, 2);
+      l_run = l_run * al + rs;
+      m_run = m_new;
 #pragma unroll
-        for (int hh = 0; hh < DEC_MAXG; ++hh)
-          if (hh < G) {
-            const float al = alph[hh];
-            acc[hh][0] *= al;
-            acc[hh][1] *= al;
-          }
-#pragma unroll 4
-        for (int k = kq * 16; k < kq * 16 + 16; ++k) {
-          const __half2 v2 = *reinterpret_cast<const __half2*>(sw128_row_chunk(vt, k, lane >> 2) + (lane & 3) * 2);
-          const float v0 = __low2float(v2), v1 = __high2float(v2);
-#pragma unroll
-          for (int hh = 0; hh < DEC_MAXG; ++hh)
-            if (hh < G) {
-              const float pv = ps[hh][k];
-              acc[hh][0] = fmaf(pv, v0, acc[hh][0]);
-              acc[hh][1] = fmaf(pv, v1, acc[hh][1]);
-            }
-        }
+      for (int j = 0; j < 8; ++j) {
+        o[j][0] *= al;
+        o[j][1] *= al;
       }
-      if (__syncthreads_or(ok ? 0 : 1)) {   // a wait gave up: every thread leaves together
+      // O += P V: P is the A fragment of the warp's 16 keys (rows >= 8 zero)
+      const uint32_t pa0 = pack_f16x2(e[0], e[1]), pa2 = pack_f16x2(e[2], e[3]);
+#pragma unroll
+      for (int j = 0; j < 8; j += 2) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(sw128_addr(vt, v_row, j + v_chk), b0, b1, b2, b3);
+        mma_16816(o[j], pa0, 0u, pa2, 0u, b0, b1);
+        mma_16816(o[j + 1], pa0, 0u, pa2, 0u, b2, b3);
+      }
+      if (__syncthreads_or(ok ? 0 : 1)) {   // stage free; a wait gave up: every thread leaves
         ok = false;
         break;
       }
     }
     if (!ok) break;
-    // the item's partial: sum the four key quarters
-#pragma unroll
-    for (int hh = 0; hh < DEC_MAXG; ++hh)
-      if (hh < G) {
-        opart[warp][hh][2 * lane] = acc[hh][0];
-        opart[warp][hh][2 * lane + 1] = acc[hh][1];
+    // merge the 4 warps' states for rows (heads) < G
+    if (gq < 8) {
+      if (tq == 0) {
+        cm[warp][gq] = m_run;
+        cl[warp][gq] = l_run;
       }
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<float2*>(&co[warp][gq][8 * j + 2 * tq]) = make_float2(o[j][0], o[j][1]);
+    }
     __syncthreads();
     for (int i = tid; i < G * 64; i += DA_THREADS) {
       const int hh = i >> 6, d = i & 63;
+      float M = cm[0][hh];
+#pragma unroll
+      for (int k = 1; k < 4; ++k) M = fmaxf(M, cm[k][hh]);
+      float L = 0.f, O = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float wk = cm[k][hh] == -INFINITY ? 0.f : ex2_approx(cm[k][hh] - M);
+        L += wk * cl[k][hh];
+        O += wk * co[k][hh][d];
+      }
       float* dst = p.part + (((size_t)b * p.Hq + g * G + hh) * p.n_splits + split) * 66;
-      dst[2 + d] = opart[0][hh][d] + opart[1][hh][d] + opart[2][hh][d] + opart[3][hh][d];
+      dst[2 + d] = O;
       if (d == 0) {
-        dst[0] = mrun[hh];
-        dst[1] = lrun[hh];
+        dst[0] = M;
+        dst[1] = L;
       }
     }
-    __syncthreads();   // qs, mrun, opart are rewritten by the next item
+    // the CTA that completes the last split of (b, g) merges all splits, in split order
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) last_split = atomicAdd(&p.counters[b * p.Hkv + g], 1u) == (unsigned)(p.n_splits - 1);
+    __syncthreads();   // also: cm, cl, co are rewritten by the next item
+    if (last_split) {
+      __threadfence();
+      for (int i = tid; i < G * 64; i += DA_THREADS) {
+        const int hh = i >> 6, d = i & 63;
+        const float* pp = p.part + ((size_t)b * p.Hq + g * G + hh) * p.n_splits * 66;
+        float M = -INFINITY;
+        for (int k0 = 0; k0 < p.n_splits; k0 += 8) {   // 8 loads in flight at a time
+          float mv[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mv[k] = k0 + k < p.n_splits ? __ldcg(pp + (k0 + k) * 66) : -INFINITY;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) M = fmaxf(M, mv[k]);
+        }
+        float L = 0.f, O = 0.f;
+        for (int k0 = 0; k0 < p.n_splits; k0 += 8) {
+          float mv[8], lv[8], ov[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const bool in = k0 + k < p.n_splits;
+            mv[k] = in ? __ldcg(pp + (k0 + k) * 66) : -INFINITY;
+            lv[k] = in ? __ldcg(pp + (k0 + k) * 66 + 1) : 0.f;
+            ov[k] = in ? __ldcg(pp + (k0 + k) * 66 + 2 + d) : 0.f;
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float wk = ex2_approx(mv[k] - M);   // 0 for the padding (-inf)
+            L += wk * lv[k];
+            O += wk * ov[k];
+          }
+        }
+        p.out[(size_t)b * p.ld_out + (g * G + hh) * 64 + d] = O / L;
+      }
+    }
   }
   if (!ok && tid == 0)   // let the loads in flight land before the CTA exits
     for (int j = ct; j < issued; ++j)
       mbar_wait(&full[j % DA_STAGES], (uint32_t)(j / DA_STAGES) & 1u, nullptr, p.status, 502);
 }
 
-__global__ void decode_attn_combine_kernel(const float* __restrict__ part, int n_splits, int Hq,
-                                           float* __restrict__ out, int ld_out) {
-  pdl_wait();
-  pdl_trigger();
-  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;   // 64 threads
-  const float* pp = part + ((size_t)b * Hq + h) * n_splits * 66;
-  float M = -1e30f;
-  for (int i = 0; i < n_splits; ++i) M = fmaxf(M, pp[i * 66]);
-  float L = 0.f, O = 0.f;
-  for (int i = 0; i < n_splits; ++i) {
-    const float w = exp2f(pp[i * 66] - M);
-    L += w * pp[i * 66 + 1];
-    O += w * pp[i * 66 + 2 + d];
-  }
-  out[(size_t)b * ld_out + h * 64 + d] = O / L;
-}
-
 // ----------------------------------------------------------------------------------------
 // decode SSM step ([JJ] §数学表示 4, one step of eq. (2)): dt = softplus(dt_low . W_dt[c] +
-// bias), h = exp(dt A) h + dt B x, y = (C . h) * SiLU(z).  CTA = 16 channels x 16 states
-// and DSSM_NB sequences: each W_dt element is read once per CTA and used for all its
-// sequences, and every sequence's state is loaded before the dt dot products.
-//   xbc [B, ld_xbc] fp32: dt_low at 0..R-1, B at R.., C at R+16..; W_dt [Di, ld_dt] fp32;
-//   xc [B, Di] bf16; z from proj at column off_z; state [B, Di, 16] in place; y [B, Di] fp32.
-//   R + 32 <= 256.
+// bias), h = exp(dt A) h + dt B x, y = (C . h) * SiLU(z).  Thread = (sequence, channel)
+// with its 16 states in registers (64 contiguous bytes of the state, 16-byte loads and
+// stores); CTA = 32 channels x 8 sequences.  The CTA's W_dt rows (padded to an odd stride:
+// conflict-free) and the sequences' dt_low, B and C rows are staged in shared memory once.
+//   xbc: n_xbc split-K slices [B, ld_xbc] fp32 (stride xbc_stride) summed here in order:
+//   dt_low at 0..R-1, B at R.., C at R+16..; W_dt [Di, ld_dt] fp32;
+//   xc [B, Di] bf16; z from the in_proj slices (stride proj_stride) at column off_z; state
+//   [B, Di, 16] in place; y [B, Di] fp32.  R <= 224.
 // ----------------------------------------------------------------------------------------
-constexpr int DSSM_NB = 8;
+constexpr int DSSM_NB = 8;     // sequences per CTA
+constexpr int DSSM_NC = 32;    // channels per CTA
 
-__global__ void __launch_bounds__(256)
-    decode_ssm_kernel(const float* __restrict__ xbc, int ld_xbc, int R, const float* __restrict__ w_dt, int ld_dt,
+__global__ void __launch_bounds__(DSSM_NB * DSSM_NC)
+    decode_ssm_kernel(const float* __restrict__ xbc, long long xbc_stride, int n_xbc, int ld_xbc, int R,
+                      const float* __restrict__ w_dt, int ld_dt,
                       const float* __restrict__ dt_bias, const float* __restrict__ A,
                       const __nv_bfloat16* __restrict__ xc, const float* __restrict__ proj, int ld_proj,
-                      int off_z, float* __restrict__ state, float* __restrict__ y, int Di, int B) {
+                      long long proj_stride, int n_slices, int off_z, float* __restrict__ state,
+                      float* __restrict__ y, int Di, int B) {
   pdl_wait();
   pdl_trigger();
-  __shared__ float dl[DSSM_NB][224];
-  __shared__ float bcs[DSSM_NB][32];
+  __shared__ float wsh[DSSM_NC][225];          // W_dt rows, stride 225 (odd: conflict-free)
+  __shared__ __align__(16) float dl[DSSM_NB][256];   // dt_low | B | C of each sequence
   const int tid = threadIdx.x;
-  const int cl = tid >> 4, s = tid & 15;
-  const int c = blockIdx.x * 16 + cl;
-  const int b0 = blockIdx.y * DSSM_NB;
-  const int nb = min(DSSM_NB, B - b0);
-  // this lane's state of every sequence first (the loads overlap the dot products)
-  float h[DSSM_NB];
+  const int cl = tid & (DSSM_NC - 1), bl = tid / DSSM_NC;
+  const int c0 = blockIdx.x * DSSM_NC, b0 = blockIdx.y * DSSM_NB;
+  const int c = c0 + cl, b = b0 + bl;
+  const bool live = b < B;
+  // this thread's state first (the loads overlap the staging below)
+  float h[16];
+  float* hp = state + ((size_t)b * Di + c) * 16;
+  if (live) {
 #pragma unroll
-  for (int bi = 0; bi < DSSM_NB; ++bi)
-    h[bi] = bi < nb ? state[((size_t)(b0 + bi) * Di + c) * 16 + s] : 0.f;
-  for (int i = tid; i < DSSM_NB * R; i += 256) {
-    const int bi = i / R, r = i - bi * R;
-    dl[bi][r] = bi < nb ? xbc[(size_t)(b0 + bi) * ld_xbc + r] : 0.f;
+    for (int k = 0; k < 16; k += 4) {
+      const float4 v = *reinterpret_cast<const float4*>(hp + k);
+      h[k] = v.x; h[k + 1] = v.y; h[k + 2] = v.z; h[k + 3] = v.w;
+    }
   }
-  for (int i = tid; i < DSSM_NB * 32; i += 256) {
-    const int bi = i >> 5;
-    bcs[bi][i & 31] = bi < nb ? xbc[(size_t)(b0 + bi) * ld_xbc + R + (i & 31)] : 0.f;
+  {
+    const int r4 = R >> 2;   // R % 4 == 0
+    for (int i = tid; i < DSSM_NC * r4; i += DSSM_NB * DSSM_NC) {
+      const int cc = i / r4, q = i - cc * r4;
+      const float4 w4 = *reinterpret_cast<const float4*>(w_dt + (size_t)(c0 + cc) * ld_dt + q * 4);
+      wsh[cc][q * 4] = w4.x;
+      wsh[cc][q * 4 + 1] = w4.y;
+      wsh[cc][q * 4 + 2] = w4.z;
+      wsh[cc][q * 4 + 3] = w4.w;
+    }
   }
+  const int nrow = R + 32;    // <= 256 = threads: one element of every sequence per thread
+#pragma unroll
+  for (int bb = 0; bb < DSSM_NB; ++bb)
+    if (tid < nrow)
+      dl[bb][tid] = b0 + bb < B ? sum_slices<DEC_MAX_XPROJ_SPLIT>(xbc + (size_t)(b0 + bb) * ld_xbc + tid, xbc_stride, n_xbc)
+                                : 0.f;
   __syncthreads();
-  float acc[DSSM_NB];
-#pragma unroll
-  for (int bi = 0; bi < DSSM_NB; ++bi) acc[bi] = 0.f;
-  const float* wr = w_dt + (size_t)c * ld_dt;
-  for (int r = s; r < R; r += 16) {
-    const float wv = wr[r];
-#pragma unroll
-    for (int bi = 0; bi < DSSM_NB; ++bi) acc[bi] = fmaf(dl[bi][r], wv, acc[bi]);
+  if (!live) return;
+  float acc0 = 0.f, acc1 = 0.f;
+  int r = 0;
+  for (; r + 1 < R; r += 2) {
+    acc0 = fmaf(dl[bl][r], wsh[cl][r], acc0);
+    acc1 = fmaf(dl[bl][r + 1], wsh[cl][r + 1], acc1);
   }
+  if (r < R) acc0 = fmaf(dl[bl][r], wsh[cl][r], acc0);
+  const float dt = softplus_f(acc0 + acc1 + dt_bias[c]);
+  const float x = __bfloat162float(xc[(size_t)b * Di + c]);
+  const float dtx = dt * x;
+  const float* Bv = &dl[bl][R];
+  const float* Cv = &dl[bl][R + 16];
+  const float* Ar = A + (size_t)c * 16;
+  float yv0 = 0.f, yv1 = 0.f;
 #pragma unroll
-  for (int bi = 0; bi < DSSM_NB; ++bi)
+  for (int k = 0; k < 16; k += 4) {
+    const float4 a4 = *reinterpret_cast<const float4*>(Ar + k);
+    const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-    for (int o = 8; o > 0; o >>= 1) acc[bi] += __shfl_xor_sync(0xffffffffu, acc[bi], o);
-  const float bias = dt_bias[c];
-  const float Acs = A[(size_t)c * 16 + s];
-#pragma unroll
-  for (int bi = 0; bi < DSSM_NB; ++bi) {
-    if (bi >= nb) break;
-    const int b = b0 + bi;
-    const float dt = softplus_f(acc[bi] + bias);
-    const float x = __bfloat162float(xc[(size_t)b * Di + c]);
-    const float hn = fmaf(expf(dt * Acs), h[bi], dt * bcs[bi][s] * x);
-    state[((size_t)b * Di + c) * 16 + s] = hn;
-    float yv = bcs[bi][16 + s] * hn;
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) yv += __shfl_xor_sync(0xffffffffu, yv, o);
-    if (s == 0) y[(size_t)b * Di + c] = yv * silu_f(proj[(size_t)b * ld_proj + off_z + c]);
+    for (int e = 0; e < 4; ++e) {
+      const int sidx = k + e;
+      h[sidx] = fmaf(ex2_approx(dt * av[e] * 1.4426950408889634f), h[sidx], dtx * Bv[sidx]);
+      if (e & 1) yv1 = fmaf(Cv[sidx], h[sidx], yv1);
+      else yv0 = fmaf(Cv[sidx], h[sidx], yv0);
+    }
+    *reinterpret_cast<float4*>(hp + k) = make_float4(h[k], h[k + 1], h[k + 2], h[k + 3]);
   }
+  const float z = sum_slices<DEC_MAX_IN_SPLIT>(proj + (size_t)b * ld_proj + off_z + c, proj_stride, n_slices);
+  y[(size_t)b * Di + c] = (yv0 + yv1) * silu_f(z);
 }
 
 // RoPE angles: tab[pos][j] = (cos, sin) of pos * base^(-2j/64), the angle reduced mod 2*pi
@@ -692,10 +795,18 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, int n_split
   pdl_trigger();
   const int i = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
   if (i >= n) return;
-  float4 acc = *reinterpret_cast<const float4*>(part + i);
-  for (int s = 1; s < n_split; ++s) {
-    const float4 q = *reinterpret_cast<const float4*>(part + (size_t)s * stride + i);
-    acc.x += q.x; acc.y += q.y; acc.z += q.z; acc.w += q.w;
+  // slices in order, 8 loads in flight at a time (a runtime-bounded loop would wait for each)
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < n_split; s0 += 8) {
+    float4 q[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      q[k] = s0 + k < n_split ? *reinterpret_cast<const float4*>(part + (size_t)(s0 + k) * stride + i)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      acc.x += q[k].x; acc.y += q[k].y; acc.z += q[k].z; acc.w += q[k].w;
+    }
   }
   if (residual != nullptr) {
     const __nv_bfloat162 r0 = *reinterpret_cast<const __nv_bfloat162*>(residual + i);

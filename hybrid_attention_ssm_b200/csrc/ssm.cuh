@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(SCAN_THREADS)
   pdl_wait();
   pdl_trigger();
   extern __shared__ uint8_t scan_smem_raw[];
-  ScanSmem& sm = *reinterpret_cast<ScanSmem*>((reinterpret_cast<uintptr_t>(scan_smem_raw) + 127) & ~uintptr_t(127));
+  ScanSmem& sm = *reinterpret_cast<ScanSmem*>(align_smem<128>(scan_smem_raw));
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int chl = lane >> 4;       // which of the warp's two channels
@@ -186,19 +186,31 @@ __global__ void __launch_bounds__(SCAN_THREADS)
     __syncwarp();
 #pragma unroll 1
     for (int hc = 0; hc < SCAN_TC; hc += SCAN_HALF) {
+      // exponentials and input terms of the 32 steps first (independent: the MUFU and FMA
+      // pipes stay busy), then the sequential recurrence
+      float a[SCAN_HALF], bq[SCAN_HALF];
 #pragma unroll
       for (int u = 0; u < SCAN_HALF; u += 4) {
         const float4 d4 = *reinterpret_cast<const float4*>(&S.d[cw][hc + u]);
         const float4 q4 = *reinterpret_cast<const float4*>(dxw + chl * SCAN_TC + hc + u);
         const float4 b4 = *reinterpret_cast<const float4*>(&S.bc[s][hc + u]);
+        a[u] = ex2_approx(d4.x * A2);
+        a[u + 1] = ex2_approx(d4.y * A2);
+        a[u + 2] = ex2_approx(d4.z * A2);
+        a[u + 3] = ex2_approx(d4.w * A2);
+        bq[u] = q4.x * b4.x;
+        bq[u + 1] = q4.y * b4.y;
+        bq[u + 2] = q4.z * b4.z;
+        bq[u + 3] = q4.w * b4.w;
+      }
+#pragma unroll
+      for (int u = 0; u < SCAN_HALF; u += 4) {
         const float4 c4 = *reinterpret_cast<const float4*>(&S.bc[16 + s][hc + u]);
-        const float a0 = ex2_approx(d4.x * A2), a1 = ex2_approx(d4.y * A2);
-        const float a2 = ex2_approx(d4.z * A2), a3 = ex2_approx(d4.w * A2);
         float4 v;
-        h = fmaf(a0, h, q4.x * b4.x); v.x = c4.x * h;
-        h = fmaf(a1, h, q4.y * b4.y); v.y = c4.y * h;
-        h = fmaf(a2, h, q4.z * b4.z); v.z = c4.z * h;
-        h = fmaf(a3, h, q4.w * b4.w); v.w = c4.w * h;
+        h = fmaf(a[u], h, bq[u]); v.x = c4.x * h;
+        h = fmaf(a[u + 1], h, bq[u + 1]); v.y = c4.y * h;
+        h = fmaf(a[u + 2], h, bq[u + 2]); v.z = c4.z * h;
+        h = fmaf(a[u + 3], h, bq[u + 3]); v.w = c4.w * h;
         const int row = (u >> 2) * 2 + chl;
         *reinterpret_cast<float4*>(part + (row * 16 + (s ^ (row & 7))) * 4) = v;
       }

@@ -266,7 +266,7 @@ int hymba_selftest_wait_timeout(void* workspace, size_t ws_bytes, hymba_stream s
  * that must not take cudaMalloc's device synchronisation, or as a plugin whose host
  * runtime owns all device memory).  The pages have no counterpart: this is a deployment
  * convenience of this library.  Arguments and results are those of hymba_mixer_decode.
- *   - Scratch: a built-in 16 MiB device array (every GPU that loads the library holds it
+ *   - Scratch: a built-in 32 MiB device array (every GPU that loads the library holds it
  *     until exit).  A step that needs more (hymba_mixer_workspace_size, mode DECODE, with
  *     n_tokens = kv->max_tokens) is rejected with HYMBA_ERR_WORKSPACE; Hymba-1.5B-sized SWA
  *     layers fit up to batch 64.
