@@ -101,7 +101,6 @@ def prefill_work(dims, B, T):
         "conv1d_silu": ("hbm", rows * Di * 2.0 * 3),
         "selective_scan": ("hbm", rows * Di * (2 + 4 + 2) + rows * 32 * 4.0 + B * Di * S * 4.0),
         "norm_avg": ("hbm", rows * (dims.attn_width * 4.0 + Di * 2 * 2 + dims.out_in_width * 2)),
-        "swa_cache_finalize": ("hbm", 0.0),
     }
     # the scan's binding unit is the exponential: one per (row, channel, state)
     exps = rows * Di * S
@@ -541,8 +540,14 @@ def run_stack(args, device, world):
             "weights": "random-init on the device (torch generator), distinct per layer"}
 
 
-# DRAM bytes per launch from ncu captures of the current kernels (None when not captured)
-TRAFFIC = {}
+# DRAM bytes (read + write) per launch from one ncu capture of the current kernel on this
+# workload (profiles/ holds the summaries and commands); a kernel changed since its capture
+# has no entry.  ncu replays a kernel with cold caches: writes that stay in L2 do not show.
+TRAFFIC = {
+    "selective_scan": 42279680 + 16128,     # profiles/selective_scan_and_norm_swa.md
+    "norm_avg": 41827840 + 458496,          # profiles/selective_scan_and_norm_swa.md
+    "out_proj": 36292608 + 40704,           # profiles/gemm_out_proj_swa.md
+}
 
 
 # ---------------------------------------------------------------------------------------

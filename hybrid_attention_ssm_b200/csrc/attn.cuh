@@ -39,19 +39,26 @@ struct AttnParams {
 };
 
 constexpr int ATT_THREADS = 192;
-constexpr int ATT_STAGES = 3;
 constexpr int ATT_Q_BYTES = 128 * 128;
 constexpr int ATT_KV_BYTES = 128 * 128;          // one K or V tile: 128 keys x 64 dims fp16
-constexpr int ATT_OFF_Q = 0;
-constexpr int ATT_OFF_K = ATT_OFF_Q + ATT_Q_BYTES;
-constexpr int ATT_OFF_V = ATT_OFF_K + ATT_STAGES * ATT_KV_BYTES;
-constexpr int ATT_OFF_BAR = ATT_OFF_V + ATT_STAGES * ATT_KV_BYTES;
-// requested dynamic shared memory: the tiles and barriers need 112.25 KB; 113 KB is the
-// most two CTAs can each take on one SM (228 KB, 1 KB reserved per CTA), and it keeps a
-// third CTA (which would wait for TMEM) off the SM.  The kernel checks that the dynamic
-// window is aligned well enough for the 1 KB-aligned tiles to fit.
-constexpr int ATT_SMEM = 113 * 1024;
-constexpr int ATT_USED = ATT_OFF_BAR + 160;
+// Shared-memory layout for a K/V ring of STAGES tile pairs: Q, K ring, V ring, barriers.
+template <int STAGES>
+struct AttnLayout {
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + ATT_Q_BYTES;
+  static constexpr int OFF_V = OFF_K + STAGES * ATT_KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + STAGES * ATT_KV_BYTES;
+  static constexpr int USED = OFF_BAR + 160;
+  // requested dynamic shared memory: the tiles and barriers plus up to 1 KB to align the
+  // window.  3 stages: 113 KB, the most two CTAs can each take on one SM (228 KB, 1 KB
+  // reserved per CTA), which also keeps a third CTA (which would wait for TMEM) off the
+  // SM.  2 stages: 82 KB, for a prefill that runs this kernel beside the selective scan
+  // (one attention CTA and three scan CTAs per SM).
+  static constexpr int SMEM = STAGES == 3 ? 113 * 1024 : (USED + 1023 + 1023) / 1024 * 1024;
+};
+// (the kernel checks at run time that the aligned window holds the layout)
+static_assert(AttnLayout<3>::USED <= AttnLayout<3>::SMEM, "3-stage layout fits");
+static_assert(AttnLayout<2>::USED + 1023 <= AttnLayout<2>::SMEM, "2-stage layout fits");
 constexpr uint32_t ATT_TMEM_COLS = 256;
 constexpr float ATT_RESCALE_LOG2 = 8.f;          // lazy rescale threshold (P <= 2^8)
 
@@ -152,9 +159,13 @@ __device__ __forceinline__ void attn_item(const AttnParams& p, int w, int B, int
   b = r / p.Hq;
 }
 
+template <int ATT_STAGES>
 __global__ void __launch_bounds__(ATT_THREADS, 2)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                     const __grid_constant__ CUtensorMap mapV, const __grid_constant__ AttnParams p, int B) {
+  using AL = AttnLayout<ATT_STAGES>;
+  constexpr int ATT_OFF_Q = AL::OFF_Q, ATT_OFF_K = AL::OFF_K, ATT_OFF_V = AL::OFF_V, ATT_OFF_BAR = AL::OFF_BAR;
+  constexpr int ATT_USED = AL::USED, ATT_SMEM = AL::SMEM;
   pdl_wait();
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];

@@ -33,6 +33,12 @@ struct Segment {
   int ld;                   // row stride in elements
   int rope;                 // apply RoPE (head dim 64) to this segment
   int f16;                  // 1: store fp16, 0: store bf16
+  // optional second home of fp16 rows in an SWA decode cache ([B, M, ld] meta rows and a
+  // [B, W, ld] ring): position < M goes to meta[b][pos], position >= win0 to
+  // ring[b][(pos - M) mod W]
+  void* meta;
+  void* ring;
+  int M, W, win0;
 };
 
 struct GemmParams {
@@ -305,6 +311,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
               __nv_bfloat16* dst = base + b * sg.bstride + (size_t)pos * sg.ld;
               if (sg.f16) store_f16_row(dst, v, 64);
               else store_bf16_row(dst, v, 64);
+            }
+            if (sg.meta != nullptr && (pos < sg.M || pos >= sg.win0)) {
+              const int col = gc - sg.col_begin;
+              for (int b = b_lo; b < b_hi; ++b) {
+                __half* dst = pos < sg.M
+                                  ? reinterpret_cast<__half*>(sg.meta) + ((size_t)b * sg.M + pos) * sg.ld + col
+                                  : reinterpret_cast<__half*>(sg.ring) + ((size_t)b * sg.W + (pos - sg.M) % sg.W) * sg.ld + col;
+                store_f16_row(dst, v, 64);
+              }
             }
           }
         }

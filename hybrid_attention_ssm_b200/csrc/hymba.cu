@@ -143,6 +143,32 @@ struct ProfState {
 };
 ProfState g_prof;
 
+// ----------------------------------------------------------------------------------------
+// A library-owned side stream per (host thread, device) for the attention branch of a
+// prefill: it forks from the caller's stream after in_proj and joins before the branch norm
+// through two events, so the attention runs beside the conv -> x_proj -> dt_proj -> scan
+// chain (the scan alone leaves most of each SM idle at small batch).  Event fork/join is
+// also how stream capture follows work onto another stream, so a captured prefill becomes
+// a graph with two parallel branches.
+// ----------------------------------------------------------------------------------------
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+int side_stream(SideStream** out) {
+  thread_local SideStream per_dev[64];
+  int dev = 0;
+  HY_CUDA(cudaGetDevice(&dev));
+  SideStream& ss = per_dev[dev & 63];
+  if (ss.s == nullptr) {
+    HY_CUDA(cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking));
+    HY_CUDA(cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming));
+    HY_CUDA(cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming));
+  }
+  *out = &ss;
+  return HYMBA_OK;
+}
+
 // Inside a stream capture the events become event-record nodes of the graph (the external
 // flag), so every replay re-records them.
 inline void prof_record(cudaEvent_t ev, cudaStream_t st) {
@@ -289,6 +315,24 @@ int launch_branch_norm(const float* O, int ld_o, int attn_w, const YT* y, int ld
   const int grid = rows < sms * per_sm ? rows : sms * per_sm;
   HY_CUDA(launch_pdl(branch_norm_avg_kernel<YT>, dim3(grid), dim3(NORM_THREADS), smem, st, O, ld_o, attn_w, y, ld_y,
                      z, ld_z, di, g_attn, g_ssm, eps, u, ld_u, rows, status));
+  return HYMBA_OK;
+}
+
+template <int STAGES>
+int launch_attention(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnParams& ap,
+                     int B, int grid, cudaStream_t s) {
+  static bool attr[64] = {false};
+  int d = 0;
+  cudaGetDevice(&d);
+  auto kern = attn_fwd_kernel<STAGES>;
+  constexpr int smem = AttnLayout<STAGES>::SMEM;
+  if (!attr[d & 63]) {
+    HY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    attr[d & 63] = true;
+  }
+  prof_begin("attention", s);
+  HY_CUDA(launch_pdl(kern, dim3(grid), dim3(ATT_THREADS), smem, s, mq, mk, mv, ap, B));
+  prof_end(s);
   return HYMBA_OK;
 }
 
@@ -458,7 +502,7 @@ PrefillWs prefill_layout(const Dims& m, int B, int n_tokens, int x_has_meta) {
 }
 
 struct DecodeWs {
-  size_t proj, qrot, counters, part, o, xc, xbc, xbc_part, y, u, acc_part, total;
+  size_t proj, qrot, part, o, xc, xbc, xbc_part, y, u, acc_part, total;
   int n_splits, xproj_split, oproj_split, in_split;
 };
 // Key tiles of one (sequence, kv head) in decode: SWA reads the meta tiles and the ring,
@@ -480,7 +524,6 @@ DecodeWs decode_layout(const Dims& m, int B, bool global, int n_keys_max) {
   }
   w.proj = take((size_t)w.in_split * B * m.P * 4);
   w.qrot = take((size_t)B * m.Hq * 64 * 4);
-  w.counters = take((size_t)B * m.Hkv * 4);
   w.part = take((size_t)B * m.Hq * w.n_splits * 66 * 4);
   w.o = take((size_t)B * m.qw * 4);
   w.xc = take((size_t)B * m.Di * 2);
@@ -774,14 +817,26 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     int ns = 0;
     c.p.seg[ns++] = Segment{0, m.qw, bf(L.q), (long long)T * m.qw, m.qw, 1, 1};
     if (own_kv) {
-      c.p.seg[ns++] = Segment{m.qw, m.qw + m.kvw, kv->k, (long long)Lmax * m.kvw, m.kvw, 1, 1};
-      c.p.seg[ns++] = Segment{m.qw + m.kvw, m.qw + 2 * m.kvw, kv->v, (long long)Lmax * m.kvw, m.kvw, 0, 1};
+      Segment sk{m.qw, m.qw + m.kvw, kv->k, (long long)Lmax * m.kvw, m.kvw, 1, 1};
+      Segment sv{m.qw + m.kvw, m.qw + 2 * m.kvw, kv->v, (long long)Lmax * m.kvw, m.kvw, 0, 1};
+      if (!cfg->is_global && kv->kind == HYMBA_CACHE_SWA) {
+        // the decode cache of an SWA layer: meta rows and the last W positions, written by
+        // the epilogue next to the prefill view
+        const int win0 = T - m.W > m.M ? T - m.W : m.M;
+        sk.meta = kv->meta_k; sk.ring = kv->ring_k;
+        sv.meta = kv->meta_v; sv.ring = kv->ring_v;
+        sk.M = sv.M = m.M; sk.W = sv.W = m.W; sk.win0 = sv.win0 = win0;
+      }
+      c.p.seg[ns++] = sk;
+      c.p.seg[ns++] = sv;
     }
     c.p.seg[ns++] = Segment{m.xz_off, m.xz_off + 2 * m.Di, bf(L.xz), (long long)T * 2 * m.Di, 2 * m.Di, 0, 0};
     c.p.nseg = ns;
     c.p.rope_tab = reinterpret_cast<const float2*>(wsb + L.rope);
     HY_TRY(run_gemm(c, *dev, st));
   }
+  SideStream* side = nullptr;
+  HY_TRY(side_stream(&side));
   // 2. conv1d + SiLU (writes xc, xcT and the conv state)
   float* cstate = conv_state_out != nullptr ? conv_state_out : f32(L.cstate);
   {
@@ -810,7 +865,7 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     const int n = (int)(rows * m.ld_xbc);
     prof_begin("splitk_reduce", st);
     HY_CUDA(launch_pdl(splitk_reduce_kernel, dim3(cdiv(n / 4, 256)), dim3(256), 0, st, f32(L.xbc_part), L.xproj_split, (long long)n, n,
-                                                            nullptr, f32(L.xbc), 0, f32(L.bcT), m.ld_xbc, T, L.Tp,
+                                                            nullptr, f32(L.xbc), 0, h16(L.bcT), m.ld_xbc, T, L.Tp,
                                                             m.R));
     prof_end(st);
     HY_CUDA(cudaGetLastError());
@@ -831,7 +886,15 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     c.p.status = status;
     HY_TRY(run_gemm(c, *dev, st));
   }
-  // 5. attention (block-skipped SWA + meta, or global causal)
+  // 5. attention (block-skipped SWA + meta, or global causal).  When the scan alone cannot
+  //    fill the GPU (fewer than three of its CTAs per SM), the attention forks onto the side
+  //    stream after dt_proj and runs beside the scan: both are latency-bound and fit on one
+  //    SM together (one attention CTA, three scan CTAs).  Otherwise it runs in stream order.
+  const bool overlap = (long long)B * (m.Di / SCAN_CH) < 3LL * dev->sms;
+  if (overlap) {
+    HY_CUDA(cudaEventRecord(side->fork, st));
+    HY_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
+  }
   {
     CUtensorMap mq, mk, mv;
     const uint32_t box[3] = {64, 128, 1};
@@ -854,18 +917,12 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     ap.out = f32(L.o);
     ap.ld_out = m.qw;
     ap.status = status;
-    static bool attr[64] = {false};
-    int d = 0;
-    cudaGetDevice(&d);
-    if (!attr[d & 63]) {
-      HY_CUDA(cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ATT_SMEM));
-      attr[d & 63] = true;
+    if (overlap) {   // beside the scan: 2-stage ring, one CTA per SM, on the side stream
+      HY_TRY(launch_attention<2>(mq, mk, mv, ap, B, ap.n_items < dev->sms ? ap.n_items : dev->sms, side->s));
+    } else {         // alone: 3-stage ring, two CTAs per SM, in stream order
+      HY_TRY(launch_attention<3>(mq, mk, mv, ap, B, ap.n_items < 2 * dev->sms ? ap.n_items : 2 * dev->sms, st));
     }
-    const int grid = ap.n_items < 2 * dev->sms ? ap.n_items : 2 * dev->sms;   // two persistent CTAs per SM
-    prof_begin("attention", st);
-    HY_CUDA(launch_pdl(attn_fwd_kernel, dim3(grid), dim3(ATT_THREADS), ATT_SMEM, st, mq, mk, mv, ap, B));
-    prof_end(st);
-    HY_CUDA(cudaGetLastError());
+    if (overlap) HY_CUDA(cudaEventRecord(side->join, side->s));
   }
   // 6. selective scan
   float* sstate = ssm_state_out != nullptr ? ssm_state_out : f32(L.sstate);
@@ -884,11 +941,11 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
       const uint32_t box[2] = {SCAN_TC, SCAN_CH};
       HY_TRY(make_map(&mx, bf(L.xcT), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE));
     }
-    {
-      const uint64_t dims[2] = {(uint64_t)T, (uint64_t)B * 32};
+    {   // (B_s, C_s) fp16 pairs moved as 32-bit elements
+      const uint64_t dims[2] = {(uint64_t)T, (uint64_t)B * 16};
       const uint64_t str[1] = {(uint64_t)L.Tp * 4};
-      const uint32_t box[2] = {SCAN_BCW, 32};
-      HY_TRY(make_map(&mbc, f32(L.bcT), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE));
+      const uint32_t box[2] = {SCAN_BCW, 16};
+      HY_TRY(make_map(&mbc, f32(L.bcT), CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE));
     }
     dim3 grid(m.Di / SCAN_CH, B);
     static bool attr_scan[64] = {false};
@@ -903,7 +960,8 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
                        sstate, T, m.Di, status));
     prof_end(st);
   }
-  // 7. per-branch RMSNorm, gate, beta, average
+  // 7. per-branch RMSNorm, gate, beta, average (the attention branch joins here)
+  if (overlap) HY_CUDA(cudaStreamWaitEvent(st, side->join, 0));
   {
     prof_begin("norm_avg", st);
     HY_TRY(launch_branch_norm<__nv_bfloat16>(f32(L.o), m.qw, m.qw, bf(L.y), m.Di, bf(L.xz) + m.Di, 2 * m.Di, m.Di,
@@ -928,20 +986,6 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     c.p.ld_res = m.d;
     c.p.status = status;
     HY_TRY(run_gemm(c, *dev, st));
-  }
-  // 9. SWA decode cache: meta rows and the last W positions
-  if (own_kv && !cfg->is_global && kv->kind == HYMBA_CACHE_SWA) {
-    const int first_win = T - m.W > m.M ? T - m.W : m.M;
-    const int n_rows = m.M + (T - first_win);
-    const int n = n_rows * (m.kvw / 8);
-    dim3 grid(cdiv(n, 256), B);
-    prof_begin("swa_cache_finalize", st);
-    HY_CUDA(launch_pdl(swa_cache_finalize_kernel, dim3(grid), dim3(256), 0, st,
-        reinterpret_cast<const __half*>(kv->k), reinterpret_cast<const __half*>(kv->v), Lmax, T, m.M, m.W, m.kvw,
-        reinterpret_cast<__half*>(kv->meta_k), reinterpret_cast<__half*>(kv->meta_v),
-        reinterpret_cast<__half*>(kv->ring_k), reinterpret_cast<__half*>(kv->ring_v)));
-    prof_end(st);
-    HY_CUDA(cudaGetLastError());
   }
   return HYMBA_OK;
 }
@@ -1024,8 +1068,6 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     pp.qrot = f32(L.qrot);
     pp.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)m.D));
     fill_rope_theta(pp.rope_theta, cfg->rope_base);
-    pp.counters = reinterpret_cast<unsigned*>(wsb + L.counters);
-    pp.n_counters = B * m.Hkv;
     const int n_rope = B * (m.Hq + (own_kv ? m.Hkv : 0)) * 32;
     prof_begin("decode_prep", st);
     HY_CUDA(launch_pdl(decode_prep_kernel, dim3(pp.conv_blocks + cdiv(n_rope, 256)), dim3(256), 0, st, pp));
@@ -1072,9 +1114,6 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     if (ap.n_splits > L.n_splits) return fail(HYMBA_ERR_WORKSPACE, "decode workspace sized for fewer keys");
     ap.n_items = B * m.Hkv * ap.n_splits;
     ap.part = f32(L.part);
-    ap.out = f32(L.o);
-    ap.ld_out = m.qw;
-    ap.counters = reinterpret_cast<unsigned*>(wsb + L.counters);
     ap.status = status;
     static bool attr_da[64] = {false};
     int dcur = 0;
@@ -1086,6 +1125,10 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     const int grid = ap.n_items < 3 * dev->sms ? ap.n_items : 3 * dev->sms;
     prof_begin("decode_attn", st);
     HY_CUDA(launch_pdl(decode_attn_kernel, dim3(grid), dim3(DA_THREADS), DA_SMEM, st, mmk, mmv, mk, mv, ap));
+    prof_end(st);
+    prof_begin("decode_attn_combine", st);
+    HY_CUDA(launch_pdl(decode_attn_combine_kernel, dim3(m.Hq, B), dim3(64), 0, st, f32(L.part), ap.n_splits, m.Hq,
+                       f32(L.o), m.qw));
     prof_end(st);
   }
   // 4. x_proj (swap-AB, split-K into per-split slices, fixed-order sum)
@@ -1145,7 +1188,7 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     const int n = B * m.d;
     prof_begin("decode_out_store", st);
     HY_CUDA(launch_pdl(splitk_reduce_kernel, dim3(cdiv(n / 4, 256)), dim3(256), 0, st, f32(L.acc_part), L.oproj_split, (long long)n, n,
-                                                            reinterpret_cast<const __nv_bfloat16*>(residual), out, 1, (float*)nullptr, 0, 0, 0, 0));
+                                                            reinterpret_cast<const __nv_bfloat16*>(residual), out, 1, (__half*)nullptr, 0, 0, 0, 0));
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }

@@ -195,40 +195,6 @@ __global__ void __launch_bounds__(NORM_THREADS)
 }
 
 // ----------------------------------------------------------------------------------------
-// SWA cache after prefill: meta rows [0, M) -> meta_k/v; rows [max(M, T-W), T) -> ring slot
-// (pos - M) mod W.  view_k/v [B, Lmax, Hkv*D]; meta [B, M, Hkv*D]; ring [B, W, Hkv*D].
-// ----------------------------------------------------------------------------------------
-__global__ void swa_cache_finalize_kernel(const __half* __restrict__ vk, const __half* __restrict__ vv,
-                                          int Lmax, int T, int M, int W, int row_elems,
-                                          __half* __restrict__ meta_k, __half* __restrict__ meta_v,
-                                          __half* __restrict__ ring_k, __half* __restrict__ ring_v) {
-  pdl_wait();
-  pdl_trigger();
-  const int b = blockIdx.y;
-  const int first_win = max(M, T - W);
-  const int n_rows = M + (T - first_win);
-  const int vec_per_row = row_elems / 8;
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_rows * vec_per_row; i += gridDim.x * blockDim.x) {
-    const int rr = i / vec_per_row, cv = (i % vec_per_row) * 8;
-    int pos;
-    __half *dk, *dv;
-    if (rr < M) {
-      pos = rr;
-      dk = meta_k + ((size_t)b * M + pos) * row_elems;
-      dv = meta_v + ((size_t)b * M + pos) * row_elems;
-    } else {
-      pos = first_win + (rr - M);
-      const int slot = (pos - M) % W;
-      dk = ring_k + ((size_t)b * W + slot) * row_elems;
-      dv = ring_v + ((size_t)b * W + slot) * row_elems;
-    }
-    const size_t src = ((size_t)b * Lmax + pos) * row_elems + cv;
-    *reinterpret_cast<uint4*>(dk + cv) = *reinterpret_cast<const uint4*>(vk + src);
-    *reinterpret_cast<uint4*>(dv + cv) = *reinterpret_cast<const uint4*>(vv + src);
-  }
-}
-
-// ----------------------------------------------------------------------------------------
 // Decode step, before attention: the conv step of the SSM input (blocks [0, conv_blocks))
 // and RoPE of the new token's query heads and key heads at position p (the other blocks).
 // Rotated queries, pre-scaled by log2(e)/sqrt(D), go to qrot [B, Hq, 64]; an own/producer
@@ -266,8 +232,6 @@ struct DecPrepParams {
   float* qrot;
   float scale_log2;
   double rope_theta[32];
-  unsigned* counters;         // [B * Hkv] split counters of the attention step, zeroed here
-  int n_counters;
 };
 
 __global__ void __launch_bounds__(256) decode_prep_kernel(const __grid_constant__ DecPrepParams p) {
@@ -290,7 +254,6 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(const __grid_constant_
   }
   const int n_heads = p.Hq + (p.write_kv ? p.Hkv : 0);
   const int i = (blockIdx.x - p.conv_blocks) * 256 + threadIdx.x;
-  if (i < p.n_counters) p.counters[i] = 0u;
   if (i >= p.B * n_heads * 32) return;
   const int j = i & 31, hh = (i >> 5) % n_heads, b = (i >> 5) / n_heads;
   // angle p * theta_j reduced mod 2 pi in double precision, then the fp32 sincos
@@ -344,9 +307,8 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(const __grid_constant_
 // swizzled K tile, an online softmax in registers, O += P V with P reused from the S
 // accumulators and V fragments from ldmatrix.trans.  At the end of an item the 4 warps'
 // (m, l, O) are merged; the partial (m, l, o[64]) per (b, head, split) goes to
-// part [B, Hq, n_splits, 66], and the CTA that finishes the last split of (b, g) (a counter
-// per (b, g), zeroed by the prep kernel) merges the splits in split order into out.  Each
-// item's queries arrive by bulk copy together with its first K/V tile.
+// part [B, Hq, n_splits, 66] and decode_attn_combine_kernel merges the splits in split
+// order.  Each item's queries arrive by bulk copy together with its first K/V tile.
 // ----------------------------------------------------------------------------------------
 constexpr int DA_KT = 64;               // keys per tile
 constexpr int DA_STAGES = 3;
@@ -366,9 +328,6 @@ struct DecAttnParams {
   int rows_main;           // rows per sequence in the main cache (W or Lmax)
   int n_splits, n_items;
   float* part;
-  float* out;              // [B, ld_out] fp32: head h at columns h*64 (merged result)
-  int ld_out;
-  unsigned* counters;      // [B * Hkv], zero on entry
   DevStatus* status;
 };
 
@@ -406,7 +365,7 @@ __global__ void __launch_bounds__(DA_THREADS)
   __shared__ __align__(16) float qbuf[DA_STAGES][DEC_MAXG * 64];
   __shared__ float cm[4][8], cl[4][8];
   __shared__ __align__(16) float co[4][8][64];
-  __shared__ int abort_flag, last_split;
+  __shared__ int abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gq = lane >> 2, tq = lane & 3;   // fragment row (query head) and column pair
   const int G = p.Hq / p.Hkv;
@@ -570,48 +529,47 @@ __global__ void __launch_bounds__(DA_THREADS)
         dst[1] = L;
       }
     }
-    // the CTA that completes the last split of (b, g) merges all splits, in split order
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) last_split = atomicAdd(&p.counters[b * p.Hkv + g], 1u) == (unsigned)(p.n_splits - 1);
-    __syncthreads();   // also: cm, cl, co are rewritten by the next item
-    if (last_split) {
-      __threadfence();
-      for (int i = tid; i < G * 64; i += DA_THREADS) {
-        const int hh = i >> 6, d = i & 63;
-        const float* pp = p.part + ((size_t)b * p.Hq + g * G + hh) * p.n_splits * 66;
-        float M = -INFINITY;
-        for (int k0 = 0; k0 < p.n_splits; k0 += 8) {   // 8 loads in flight at a time
-          float mv[8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) mv[k] = k0 + k < p.n_splits ? __ldcg(pp + (k0 + k) * 66) : -INFINITY;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) M = fmaxf(M, mv[k]);
-        }
-        float L = 0.f, O = 0.f;
-        for (int k0 = 0; k0 < p.n_splits; k0 += 8) {
-          float mv[8], lv[8], ov[8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const bool in = k0 + k < p.n_splits;
-            mv[k] = in ? __ldcg(pp + (k0 + k) * 66) : -INFINITY;
-            lv[k] = in ? __ldcg(pp + (k0 + k) * 66 + 1) : 0.f;
-            ov[k] = in ? __ldcg(pp + (k0 + k) * 66 + 2 + d) : 0.f;
-          }
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const float wk = ex2_approx(mv[k] - M);   // 0 for the padding (-inf)
-            L += wk * lv[k];
-            O += wk * ov[k];
-          }
-        }
-        p.out[(size_t)b * p.ld_out + (g * G + hh) * 64 + d] = O / L;
-      }
-    }
+    __syncthreads();   // cm, cl, co are rewritten by the next item
   }
   if (!ok && tid == 0)   // let the loads in flight land before the CTA exits
     for (int j = ct; j < issued; ++j)
       mbar_wait(&full[j % DA_STAGES], (uint32_t)(j / DA_STAGES) & 1u, nullptr, p.status, 502);
+}
+
+// merge of the decode attention splits: out[b, h*64 + d] = sum_s w_s o_s / sum_s w_s l_s,
+// w_s = 2^(m_s - max m), in split order (64 threads per (head, sequence))
+__global__ void decode_attn_combine_kernel(const float* __restrict__ part, int n_splits, int Hq,
+                                           float* __restrict__ out, int ld_out) {
+  pdl_wait();
+  pdl_trigger();
+  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;   // 64 threads
+  const float* pp = part + ((size_t)b * Hq + h) * n_splits * 66;
+  float M = -1e30f;
+  for (int i0 = 0; i0 < n_splits; i0 += 8) {   // 8 splits' loads in flight at a time
+    float mv[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) mv[k] = i0 + k < n_splits ? pp[(i0 + k) * 66] : -1e30f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) M = fmaxf(M, mv[k]);
+  }
+  float L = 0.f, O = 0.f;
+  for (int i0 = 0; i0 < n_splits; i0 += 8) {
+    float mv[8], lv[8], ov[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const bool in = i0 + k < n_splits;
+      mv[k] = in ? pp[(i0 + k) * 66] : -INFINITY;
+      lv[k] = in ? pp[(i0 + k) * 66 + 1] : 0.f;
+      ov[k] = in ? pp[(i0 + k) * 66 + 2 + d] : 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float w = exp2f(mv[k] - M);   // 0 for the padding
+      L += w * lv[k];
+      O += w * ov[k];
+    }
+  }
+  out[(size_t)b * ld_out + h * 64 + d] = O / L;
 }
 
 // ----------------------------------------------------------------------------------------
@@ -647,12 +605,15 @@ __global__ void __launch_bounds__(DSSM_NB * DSSM_NC)
   // this thread's state first (the loads overlap the staging below)
   float h[16];
   float* hp = state + ((size_t)b * Di + c) * 16;
+  float x = 0.f, z = 0.f;
   if (live) {
 #pragma unroll
     for (int k = 0; k < 16; k += 4) {
       const float4 v = *reinterpret_cast<const float4*>(hp + k);
       h[k] = v.x; h[k + 1] = v.y; h[k + 2] = v.z; h[k + 3] = v.w;
     }
+    x = __bfloat162float(xc[(size_t)b * Di + c]);
+    z = sum_slices<DEC_MAX_IN_SPLIT>(proj + (size_t)b * ld_proj + off_z + c, proj_stride, n_slices);
   }
   {
     const int r4 = R >> 2;   // R % 4 == 0
@@ -681,7 +642,6 @@ __global__ void __launch_bounds__(DSSM_NB * DSSM_NC)
   }
   if (r < R) acc0 = fmaf(dl[bl][r], wsh[cl][r], acc0);
   const float dt = softplus_f(acc0 + acc1 + dt_bias[c]);
-  const float x = __bfloat162float(xc[(size_t)b * Di + c]);
   const float dtx = dt * x;
   const float* Bv = &dl[bl][R];
   const float* Cv = &dl[bl][R + 16];
@@ -700,7 +660,6 @@ __global__ void __launch_bounds__(DSSM_NB * DSSM_NC)
     }
     *reinterpret_cast<float4*>(hp + k) = make_float4(h[k], h[k + 1], h[k + 2], h[k + 3]);
   }
-  const float z = sum_slices<DEC_MAX_IN_SPLIT>(proj + (size_t)b * ld_proj + off_z + c, proj_stride, n_slices);
   y[(size_t)b * Di + c] = (yv0 + yv1) * silu_f(z);
 }
 
@@ -789,7 +748,7 @@ __global__ void wait_timeout_selftest_kernel(DevStatus* st) {
 // are also written time-major to bcT [B][32][Tp] (the scan's B/C input).
 __global__ void splitk_reduce_kernel(const float* __restrict__ part, int n_split, long long stride, int n,
                                      const __nv_bfloat16* __restrict__ residual, void* __restrict__ out,
-                                     int out_bf16, float* __restrict__ bcT = nullptr, int ld = 0, int T = 0,
+                                     int out_bf16, __half* __restrict__ bcp = nullptr, int ld = 0, int T = 0,
                                      int Tp = 0, int tr_col0 = 0) {
   pdl_wait();
   pdl_trigger();
@@ -819,14 +778,14 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, int n_split
   } else {
     *reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + i) = acc;
   }
-  if (bcT != nullptr) {
+  if (bcp != nullptr) {   // the scan's copy of B and C: fp16 pairs (B_s, C_s), state-major
     const int row = i / ld, col = i % ld;       // 4 columns of one row (ld % 4 == 0)
     const int b = row / T, t = row % T;
     const float vals[4] = {acc.x, acc.y, acc.z, acc.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const int cc = col + e - tr_col0;
-      if (cc >= 0 && cc < 32) bcT[((size_t)b * 32 + cc) * Tp + t] = vals[e];
+      const int cc = col + e - tr_col0;         // 0..15: B_s, 16..31: C_s
+      if (cc >= 0 && cc < 32) bcp[(((size_t)b * 16 + (cc & 15)) * Tp + t) * 2 + (cc >> 4)] = __float2half_rn(vals[e]);
     }
   }
 }

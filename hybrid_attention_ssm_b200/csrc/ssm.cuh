@@ -85,40 +85,45 @@ __global__ void __launch_bounds__(256)
 // ----------------------------------------------------------------------------------------
 // Selective scan + state carry ([JJ] §数学表示 4, eq. (2), Euler form):
 //   h_t[s] = exp(delta_t * A[s]) h_{t-1}[s] + delta_t B_t[s] x_t,   y_t = sum_s C_t[s] h_t[s]
-// One CTA = 8 channels x 16 states (128 threads); a warp owns two channels, a lane owns one
-// (channel, state) and keeps h in a register, walking T in order (no inter-chunk pass).
-// Each 64-step chunk arrives by three TMA loads (delta and x [8 channels x 64 steps],
-// B/C [32 rows x 68 steps: rows padded so that the 16 state lanes of one step hit distinct
-// banks]) into a 4-stage ring completed on mbarriers; loads past T are zero-filled, so
-// delta = 0 leaves the state unchanged.  Per chunk each warp first forms delta*x for its two
-// channels (once per step, not once per state), then runs the recurrence, writes its C*h
-// terms to a warp-private, XOR-swizzled buffer and sums the 16 states per (step, channel)
-// inside the warp: no CTA barrier until the end of the chunk, where the gathered 8-channel
-// y rows leave as 16-byte stores.
-//   xcT [B, Di, Tp] bf16; dT [B, Di, Tp] fp32; bcT [B, 32, Tp] fp32 (B rows 0..15, C rows
-//   16..31), all read through tensor maps of extent T; A [Di, 16]; y [B*T, Di] bf16 (the
-//   SiLU(z) gate is applied by the branch norm); state [B, Di, 16] fp32.
+// The recurrence is cheap; what bounds a scan over (channel, state) lanes is the operand
+// traffic from shared memory to registers (every update needs delta, delta*x, B and C).
+// A lane therefore owns two states (s, s+8) of one channel: delta and delta*x are read once
+// per two updates, B and C arrive as one fp16 pair per state and step, and the 16-state
+// sum of C*h halves before it leaves the lane.  CTA = 8 channels x 16 states = 64 lanes
+// (two warps of 4 channels x 8 lanes), h in registers, T walked in order.
+// Each 64-step chunk arrives by three TMA loads into a SCAN_NST-stage ring completed on
+// mbarriers: delta [8 channels x 64] fp32, x [8 x 64] bf16, and the (B, C) fp16 pairs
+// [16 states x 68 steps] (rows padded so that the 8 state rows of a lane group fall in
+// distinct banks).  Loads past T are zero-filled, so delta = 0 leaves the state unchanged.
+// A warp turns its 4 channels' delta and x into (delta, delta*x) pairs, runs the recurrence
+// for 32 steps, writes each lane's C.h partial sums to an XOR-swizzled warp buffer and sums
+// the 8 lanes of each channel; one CTA barrier per chunk, after which the 8-channel y rows
+// leave as 16-byte stores.
+//   xcT [B, Di, Tp] bf16; dT [B, Di, Tp] fp32; bcp [B, 16, Tp] of (B_s, C_s) fp16 pairs; all
+//   read through tensor maps of extent T; A [Di, 16]; y [B*T, Di] bf16 (the SiLU(z) gate is
+//   applied by the branch norm); state [B, Di, 16] fp32.
 // ----------------------------------------------------------------------------------------
-constexpr int SCAN_CH = 8;            // channels per CTA (two per warp)
+constexpr int SCAN_CH = 8;            // channels per CTA (four per warp)
 constexpr int SCAN_TC = 64;           // time steps per chunk
 constexpr int SCAN_NST = 4;           // TMA stages
 constexpr int SCAN_HALF = 32;         // steps per reduction round
-constexpr int SCAN_BCW = SCAN_TC + 4; // padded B/C row (the TMA box is this wide)
-constexpr int SCAN_THREADS = SCAN_CH * 16;
+constexpr int SCAN_BCW = SCAN_TC + 4; // padded (B, C) row (the TMA box is this wide)
+constexpr int SCAN_THREADS = SCAN_CH * 8;
+constexpr int SCAN_DDW = SCAN_TC + 2; // (delta, delta*x) row, padded
 
 struct ScanStage {
-  float d[SCAN_CH][SCAN_TC];          // delta      (box {64, 8} fp32, 2048 B)
-  __nv_bfloat16 x[SCAN_CH][SCAN_TC];  // x          (box {64, 8} bf16, 1024 B)
-  float bc[32][SCAN_BCW];             // B, C rows  (box {68, 32} fp32, 8704 B)
+  float d[SCAN_CH][SCAN_TC];          // delta          (box {64, 8} fp32, 2048 B)
+  __nv_bfloat16 x[SCAN_CH][SCAN_TC];  // x              (box {64, 8} bf16, 1024 B)
+  uint32_t bc[16][SCAN_BCW];          // (B_s, C_s) fp16 pairs (box {68, 16} 32-bit, 4352 B)
 };
-static_assert(sizeof(ScanStage) == 2048 + 1024 + 8704, "stage layout must match the TMA boxes");
+static_assert(sizeof(ScanStage) == 2048 + 1024 + 4352, "stage layout must match the TMA boxes");
 static_assert(sizeof(ScanStage) % 128 == 0, "stages stay 128-byte aligned");
 
 struct ScanSmem {
   ScanStage st[SCAN_NST];
-  float part[4][SCAN_HALF * 2 * 16];           // per warp: [step/4 * 2 + channel][slot][4], slot = state ^ (row & 7)
-  float dx[4][2][SCAN_TC];                     // per warp: delta * x of its two channels
-  __nv_bfloat16 ys[2][SCAN_TC][SCAN_CH];       // y rows of a chunk, double-buffered
+  float2 dd[SCAN_CH][SCAN_DDW];                 // (delta, delta*x) per channel and step
+  float part[2][SCAN_HALF * 4 * 8];             // per warp: [step/4][channel][lane slot][4]
+  __nv_bfloat16 ys[2][SCAN_TC][SCAN_CH];        // y rows of a chunk, double-buffered
   uint64_t full[SCAN_NST];
   int abort;
 };
@@ -134,15 +139,16 @@ __global__ void __launch_bounds__(SCAN_THREADS)
   ScanSmem& sm = *reinterpret_cast<ScanSmem*>(align_smem<128>(scan_smem_raw));
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int chl = lane >> 4;       // which of the warp's two channels
-  const int s = lane & 15;         // state
-  const int cw = warp * 2 + chl;   // channel within the CTA
+  const int cl4 = lane >> 3;         // channel of the warp (0..3)
+  const int l8 = lane & 7;           // states l8 and l8 + 8
+  const int cw = warp * 4 + cl4;     // channel within the CTA
   const int c0 = blockIdx.x * SCAN_CH;
   const int b = blockIdx.y;
   const int c = c0 + cw;
   const int n_chunks = (T + SCAN_TC - 1) / SCAN_TC;
-  const int row_dx = b * Di + c0;  // first row of this CTA in the delta / x maps
-  const float A2 = A[(size_t)c * 16 + s] * 1.4426950408889634f;   // exp(d*A) = 2^(d*A*log2 e)
+  const int row_dx = b * Di + c0;    // first row of this CTA in the delta / x maps
+  const float A0 = A[(size_t)c * 16 + l8] * 1.4426950408889634f;       // exp(d*A) = 2^(d*A*log2 e)
+  const float A1 = A[(size_t)c * 16 + l8 + 8] * 1.4426950408889634f;
 
   if (tid == 0) {
     for (int i = 0; i < SCAN_NST; ++i) mbar_init(&sm.full[i], 1);
@@ -159,81 +165,100 @@ __global__ void __launch_bounds__(SCAN_THREADS)
     mbar_arrive_expect_tx(bar, (uint32_t)sizeof(ScanStage));
     tma_load_2d(&S.d[0][0], &mapD, bar, k * SCAN_TC, row_dx);
     tma_load_2d(&S.x[0][0], &mapX, bar, k * SCAN_TC, row_dx);
-    tma_load_2d(&S.bc[0][0], &mapBC, bar, k * SCAN_TC, b * 32);
+    tma_load_2d(&S.bc[0][0], &mapBC, bar, k * SCAN_TC, b * 16);
   };
   int issued = 0;
   if (tid == 0)
     for (; issued < SCAN_NST - 1 && issued < n_chunks; ++issued) issue(issued);
 
-  float h = 0.f;
+  float h0 = 0.f, h1 = 0.f;
   float* part = sm.part[warp];
-  float* dxw = &sm.dx[warp][0][0];
   int k = 0;
   for (; k < n_chunks; ++k) {
     // the stage of chunk k-1 is free (barrier at the end of the previous chunk)
     if (tid == 0 && issued < n_chunks) issue(issued++);
     const bool ok = mbar_wait(&sm.full[k % SCAN_NST], (uint32_t)(k / SCAN_NST) & 1u, &sm.abort, status, 301);
     const ScanStage& S = sm.st[k % SCAN_NST];
-    {  // delta * x of the warp's two channels: lane -> (channel lane/16, steps 4*(lane%16) ..)
-      const int ch = lane >> 4, t4 = (lane & 15) * 4;
-      const float4 d4 = *reinterpret_cast<const float4*>(&S.d[warp * 2 + ch][t4]);
-      const uint2 x2 = *reinterpret_cast<const uint2*>(&S.x[warp * 2 + ch][t4]);
-      const __nv_bfloat162 xa = *reinterpret_cast<const __nv_bfloat162*>(&x2.x);
-      const __nv_bfloat162 xb = *reinterpret_cast<const __nv_bfloat162*>(&x2.y);
-      *reinterpret_cast<float4*>(dxw + ch * SCAN_TC + t4) =
-          make_float4(d4.x * __low2float(xa), d4.y * __high2float(xa), d4.z * __low2float(xb), d4.w * __high2float(xb));
+    {  // (delta, delta*x) of the warp's 4 channels: lane -> channel lane/8, steps 8*(lane%8) ..
+      const int ch = warp * 4 + (lane >> 3), t8 = (lane & 7) * 8;
+      const float4 da = *reinterpret_cast<const float4*>(&S.d[ch][t8]);
+      const float4 db = *reinterpret_cast<const float4*>(&S.d[ch][t8 + 4]);
+      const uint4 xr = *reinterpret_cast<const uint4*>(&S.x[ch][t8]);
+      float xf[8];
+      unpack8(xr, xf);
+      const float dv[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+#pragma unroll
+      for (int e = 0; e < 8; e += 2)
+        *reinterpret_cast<float4*>(&sm.dd[ch][t8 + e]) = make_float4(dv[e], dv[e] * xf[e], dv[e + 1], dv[e + 1] * xf[e + 1]);
     }
     __syncwarp();
 #pragma unroll 1
     for (int hc = 0; hc < SCAN_TC; hc += SCAN_HALF) {
-      // exponentials and input terms of the 32 steps first (independent: the MUFU and FMA
-      // pipes stay busy), then the sequential recurrence
-      float a[SCAN_HALF], bq[SCAN_HALF];
 #pragma unroll
-      for (int u = 0; u < SCAN_HALF; u += 4) {
-        const float4 d4 = *reinterpret_cast<const float4*>(&S.d[cw][hc + u]);
-        const float4 q4 = *reinterpret_cast<const float4*>(dxw + chl * SCAN_TC + hc + u);
-        const float4 b4 = *reinterpret_cast<const float4*>(&S.bc[s][hc + u]);
-        a[u] = ex2_approx(d4.x * A2);
-        a[u + 1] = ex2_approx(d4.y * A2);
-        a[u + 2] = ex2_approx(d4.z * A2);
-        a[u + 3] = ex2_approx(d4.w * A2);
-        bq[u] = q4.x * b4.x;
-        bq[u + 1] = q4.y * b4.y;
-        bq[u + 2] = q4.z * b4.z;
-        bq[u + 3] = q4.w * b4.w;
-      }
+      for (int u8 = 0; u8 < SCAN_HALF; u8 += 8) {
+        // 8 steps: operands and the 16 exponentials first (independent of the state), then
+        // the two recurrences; keeps enough independent work in flight per warp
+        float ea0[8], ea1[8], eb0[8], eb1[8], ec0[8], ec1[8];
 #pragma unroll
-      for (int u = 0; u < SCAN_HALF; u += 4) {
-        const float4 c4 = *reinterpret_cast<const float4*>(&S.bc[16 + s][hc + u]);
-        float4 v;
-        h = fmaf(a[u], h, bq[u]); v.x = c4.x * h;
-        h = fmaf(a[u + 1], h, bq[u + 1]); v.y = c4.y * h;
-        h = fmaf(a[u + 2], h, bq[u + 2]); v.z = c4.z * h;
-        h = fmaf(a[u + 3], h, bq[u + 3]); v.w = c4.w * h;
-        const int row = (u >> 2) * 2 + chl;
-        *reinterpret_cast<float4*>(part + (row * 16 + (s ^ (row & 7))) * 4) = v;
+        for (int u = 0; u < 8; u += 4) {
+          const float4 p01 = *reinterpret_cast<const float4*>(&sm.dd[cw][hc + u8 + u]);       // steps u, u+1
+          const float4 p23 = *reinterpret_cast<const float4*>(&sm.dd[cw][hc + u8 + u + 2]);   // steps u+2, u+3
+          const uint4 q0 = *reinterpret_cast<const uint4*>(&S.bc[l8][hc + u8 + u]);
+          const uint4 q1 = *reinterpret_cast<const uint4*>(&S.bc[l8 + 8][hc + u8 + u]);
+          const float dl[4] = {p01.x, p01.z, p23.x, p23.z};
+          const float dxl[4] = {p01.y, p01.w, p23.y, p23.w};
+          const uint32_t w0[4] = {q0.x, q0.y, q0.z, q0.w};
+          const uint32_t w1[4] = {q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 bc0 = __half22float2(*reinterpret_cast<const __half2*>(&w0[e]));   // (B, C) of state l8
+            const float2 bc1 = __half22float2(*reinterpret_cast<const __half2*>(&w1[e]));   // (B, C) of state l8+8
+            ea0[u + e] = ex2_approx(dl[e] * A0);
+            ea1[u + e] = ex2_approx(dl[e] * A1);
+            eb0[u + e] = dxl[e] * bc0.x;
+            eb1[u + e] = dxl[e] * bc1.x;
+            ec0[u + e] = bc0.y;
+            ec1[u + e] = bc1.y;
+          }
+        }
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          h0 = fmaf(ea0[e], h0, eb0[e]);
+          h1 = fmaf(ea1[e], h1, eb1[e]);
+          v[e] = fmaf(ec1[e], h1, ec0[e] * h0);
+        }
+        // slot l8 ^ f(step group, channel): conflict-free on both the write and the read side
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int g = (u8 >> 2) + q;
+          const int slot = l8 ^ ((g * 4 + cl4) & 7);
+          *reinterpret_cast<float4*>(part + ((g * 4 + cl4) * 8 + slot) * 4) =
+              make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
       }
       __syncwarp();
-      {  // lane -> (row = lane/2: step group and channel, pair = two of its four steps)
-        const int row = lane >> 1, pair = lane & 1;
-        float2 acc = make_float2(0.f, 0.f);
+      {  // lane -> (step group g = lane/4, channel ch = lane%4): sum of the 8 lanes, 4 steps
+        const int g = lane >> 2, ch = lane & 3;
+        const int f = (g * 4 + ch) & 7;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int st = 0; st < 16; ++st) {
-          const float2 v2 = *reinterpret_cast<const float2*>(part + (row * 16 + (st ^ (row & 7))) * 4 + pair * 2);
-          acc.x += v2.x;
-          acc.y += v2.y;
+        for (int l = 0; l < 8; ++l) {
+          const float4 q = *reinterpret_cast<const float4*>(part + ((g * 4 + ch) * 8 + (l ^ f)) * 4);
+          acc.x += q.x; acc.y += q.y; acc.z += q.z; acc.w += q.w;
         }
-        const int t = hc + (row >> 1) * 4 + pair * 2;
-        const int ch = warp * 2 + (row & 1);
-        sm.ys[k & 1][t][ch] = __float2bfloat16_rn(acc.x);
-        sm.ys[k & 1][t + 1][ch] = __float2bfloat16_rn(acc.y);
+        const int t = hc + g * 4;
+        const int cc = warp * 4 + ch;
+        sm.ys[k & 1][t][cc] = __float2bfloat16_rn(acc.x);
+        sm.ys[k & 1][t + 1][cc] = __float2bfloat16_rn(acc.y);
+        sm.ys[k & 1][t + 2][cc] = __float2bfloat16_rn(acc.z);
+        sm.ys[k & 1][t + 3][cc] = __float2bfloat16_rn(acc.w);
       }
       __syncwarp();
     }
     if (__syncthreads_or(ok ? 0 : 1)) break;   // a wait gave up: every thread leaves together
-    if (tid < SCAN_TC) {
-      const int t = k * SCAN_TC + tid;
+    {
+      const int t = k * SCAN_TC + tid;        // 64 threads: one y row each
       if (t < T)
         *reinterpret_cast<uint4*>(y + ((size_t)b * T + t) * Di + c0) = *reinterpret_cast<const uint4*>(&sm.ys[k & 1][tid][0]);
     }
@@ -245,7 +270,8 @@ __global__ void __launch_bounds__(SCAN_THREADS)
         mbar_wait(&sm.full[j % SCAN_NST], (uint32_t)(j / SCAN_NST) & 1u, nullptr, status, 302);
     return;
   }
-  state[((size_t)b * Di + c) * 16 + s] = h;
+  state[((size_t)b * Di + c) * 16 + l8] = h0;
+  state[((size_t)b * Di + c) * 16 + l8 + 8] = h1;
 }
 
 }  // namespace hymba

@@ -81,10 +81,11 @@ def _check_stages(run, ref, dims, w):
         assert_rms(xbc[b, :, :R + 2 * S], proj, tol=1e-3, name="x_proj")
         d_ref = orc.softplus(xbc[b, :, :R] @ w["w_dt"].astype(np.float64).T + w["dt_bias"])
         assert_rel_inf(delta[b], d_ref, tol=5e-3, name="delta")
-        # scan fed the GPU's own xc, delta, B, C, z
+        # scan fed the GPU's own xc, delta, B, C, z (the scan reads B and C as fp16)
         zb = xz[b, :, Di:]
-        y_ref, h_ref = orc.selective_scan(xc[b], delta[b], w["A"], xbc[b, :, R:R + S],
-                                          xbc[b, :, R + S:R + 2 * S], zb)
+        bm16 = xbc[b, :, R:R + S].astype(np.float16).astype(np.float64)
+        cm16 = xbc[b, :, R + S:R + 2 * S].astype(np.float16).astype(np.float64)
+        y_ref, h_ref = orc.selective_scan(xc[b], delta[b], w["A"], bm16, cm16, zb)
         assert_rel_inf(to_np(run.ssm[b]), h_ref, tol=1e-4, name="scan state")
         assert_elem(y[b] * orc.silu(zb), y_ref, name="scan y")
         if k is not None:
