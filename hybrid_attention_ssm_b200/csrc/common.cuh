@@ -74,15 +74,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Bounded wait on phase `parity` of `bar`.  Returns false (and records the site in the
 // status word) when the wait exceeds g_wait_limit_ns, or when another warp of the CTA has
 // already given up (`*abort` set), so that no wait in these kernels can spin forever.
+// The clock is read only once a wait has polled 256 times: most waits in a pipeline end
+// within a few polls, and reading the global timer on every wait cost about a microsecond
+// per hand-off.  The limit is measured from that first reading.
 static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
                                                    DevStatus* st, unsigned site) {
-  const uint64_t t0 = globaltimer_ns();
-  const uint64_t limit = g_wait_limit_ns;
+  uint64_t t0 = 0;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 31u) == 0u) {
+    if ((it & 255u) == 0u) {
       if (abort != nullptr && *abort) return false;
-      if (globaltimer_ns() - t0 > limit) {
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > g_wait_limit_ns) {
         if (abort != nullptr) *abort = 1;
         report_error(st, DEV_ERR_TIMEOUT, site);
         return false;
