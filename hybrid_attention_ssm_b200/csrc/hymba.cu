@@ -1073,8 +1073,14 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     HY_CUDA(launch_pdl(decode_prep_kernel, dim3(pp.conv_blocks + cdiv(n_rope, 256)), dim3(256), 0, st, pp));
     prof_end(st);
   }
-  // 3. attention over meta + window (or rows 0..p), split over key tiles, then combine
+  // 3. attention over meta + window (or rows 0..p), split over key tiles, then combine.
+  //    The two branches are independent from here to the norm: the attention runs on the
+  //    side stream beside x_proj and the SSM step (both chains are latency-bound kernels
+  //    that leave most of the GPU idle), joined before the norm.
+  SideStream* side = nullptr;
+  HY_TRY(side_stream(&side));
   {
+    const cudaStream_t ast = side->s;
     DecAttnParams ap;
     ap.qrot = f32(L.qrot);
     ap.Hq = m.Hq; ap.Hkv = m.Hkv; ap.M = m.M; ap.is_global = global ? 1 : 0;
@@ -1123,13 +1129,16 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
       attr_da[dcur & 63] = true;
     }
     const int grid = ap.n_items < 3 * dev->sms ? ap.n_items : 3 * dev->sms;
-    prof_begin("decode_attn", st);
-    HY_CUDA(launch_pdl(decode_attn_kernel, dim3(grid), dim3(DA_THREADS), DA_SMEM, st, mmk, mmv, mk, mv, ap));
-    prof_end(st);
-    prof_begin("decode_attn_combine", st);
-    HY_CUDA(launch_pdl(decode_attn_combine_kernel, dim3(m.Hq, B), dim3(64), 0, st, f32(L.part), ap.n_splits, m.Hq,
+    HY_CUDA(cudaEventRecord(side->fork, st));   // every host-side check has passed
+    HY_CUDA(cudaStreamWaitEvent(ast, side->fork, 0));
+    prof_begin("decode_attn", ast);
+    HY_CUDA(launch_pdl(decode_attn_kernel, dim3(grid), dim3(DA_THREADS), DA_SMEM, ast, mmk, mmv, mk, mv, ap));
+    prof_end(ast);
+    prof_begin("decode_attn_combine", ast);
+    HY_CUDA(launch_pdl(decode_attn_combine_kernel, dim3(m.Hq, B), dim3(64), 0, ast, f32(L.part), ap.n_splits, m.Hq,
                        f32(L.o), m.qw));
-    prof_end(st);
+    prof_end(ast);
+    HY_CUDA(cudaEventRecord(side->join, ast));
   }
   // 4. x_proj (swap-AB, split-K into per-split slices, fixed-order sum)
   {
@@ -1152,14 +1161,15 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
   {
     dim3 grid(m.Di / DSSM_NC, cdiv(B, DSSM_NB));
     prof_begin("decode_ssm", st);
-    HY_CUDA(launch_pdl(decode_ssm_kernel, grid, dim3(DSSM_NB * DSSM_NC), 0, st, f32(L.xbc_part),
+    HY_CUDA(launch_pdl(decode_ssm_kernel, grid, dim3(DSSM_THREADS), dssm_smem_bytes(m.R), st, f32(L.xbc_part),
                        (long long)B * m.ld_xbc, L.xproj_split, m.ld_xbc, m.R, w->w_dt, w->w_dt_ld,
                        w->dt_bias, w->A, bf(L.xc), f32(L.proj), m.P, (long long)B * m.P, L.in_split,
                        m.xz_off + m.Di, ssm_state, f32(L.y), m.Di, B));
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
-  // 6. norm + average (y already gated)
+  // 6. norm + average (y already gated); the attention branch joins here
+  HY_CUDA(cudaStreamWaitEvent(st, side->join, 0));
   {
     prof_begin("decode_norm_avg", st);
     HY_TRY(launch_branch_norm<float>(f32(L.o), m.qw, m.qw, f32(L.y), m.Di, nullptr, 0, m.Di, w->g_attn, w->g_ssm,

@@ -574,19 +574,27 @@ __global__ void decode_attn_combine_kernel(const float* __restrict__ part, int n
 
 // ----------------------------------------------------------------------------------------
 // decode SSM step ([JJ] §数学表示 4, one step of eq. (2)): dt = softplus(dt_low . W_dt[c] +
-// bias), h = exp(dt A) h + dt B x, y = (C . h) * SiLU(z).  Thread = (sequence, channel)
-// with its 16 states in registers (64 contiguous bytes of the state, 16-byte loads and
-// stores); CTA = 32 channels x 8 sequences.  The CTA's W_dt rows (padded to an odd stride:
-// conflict-free) and the sequences' dt_low, B and C rows are staged in shared memory once.
+// bias), h = exp(dt A) h + dt B x, y = (C . h) * SiLU(z).  Thread = one channel x four
+// sequences, their 4 x 16 states in registers (64 contiguous bytes per sequence, 16-byte
+// loads issued before anything else); CTA = 32 channels x 16 sequences.  The CTA's W_dt
+// rows and the sequences' dt_low, B and C rows are staged transposed in shared memory once,
+// so that one W_dt value and one 16-byte broadcast of four sequences' dt_low feed four FMAs.
 //   xbc: n_xbc split-K slices [B, ld_xbc] fp32 (stride xbc_stride) summed here in order:
 //   dt_low at 0..R-1, B at R.., C at R+16..; W_dt [Di, ld_dt] fp32;
 //   xc [B, Di] bf16; z from the in_proj slices (stride proj_stride) at column off_z; state
 //   [B, Di, 16] in place; y [B, Di] fp32.  R <= 224.
 // ----------------------------------------------------------------------------------------
-constexpr int DSSM_NB = 8;     // sequences per CTA
-constexpr int DSSM_NC = 32;    // channels per CTA
+constexpr int DSSM_NC = 32;    // channels per CTA: one per lane
+constexpr int DSSM_NB = 16;    // sequences per CTA
+constexpr int DSSM_BPT = 4;    // sequences per thread; the lanes of a warp share them
+constexpr int DSSM_THREADS = DSSM_NC * DSSM_NB / DSSM_BPT;   // 128
+// dynamic shared memory: W_dt rows of the CTA's channels [R][32] and the summed x_proj
+// outputs of its sequences [R + 32][16] (dt_low | B | C), both transposed
+__host__ __device__ constexpr size_t dssm_smem_bytes(int R) {
+  return ((size_t)R * DSSM_NC + (size_t)(R + 32) * DSSM_NB) * sizeof(float);
+}
 
-__global__ void __launch_bounds__(DSSM_NB * DSSM_NC)
+__global__ void __launch_bounds__(DSSM_THREADS, 3)
     decode_ssm_kernel(const float* __restrict__ xbc, long long xbc_stride, int n_xbc, int ld_xbc, int R,
                       const float* __restrict__ w_dt, int ld_dt,
                       const float* __restrict__ dt_bias, const float* __restrict__ A,
@@ -595,72 +603,131 @@ __global__ void __launch_bounds__(DSSM_NB * DSSM_NC)
                       float* __restrict__ y, int Di, int B) {
   pdl_wait();
   pdl_trigger();
-  __shared__ float wsh[DSSM_NC][225];          // W_dt rows, stride 225 (odd: conflict-free)
-  __shared__ __align__(16) float dl[DSSM_NB][256];   // dt_low | B | C of each sequence
+  extern __shared__ __align__(16) float dssm_sh[];
+  float* wsh = dssm_sh;                    // W_dt[c0 + cl][r] at r * 32 + cl
+  float* dlT = dssm_sh + R * DSSM_NC;      // x_proj output [b0 + bl][col] at col * 16 + bl
   const int tid = threadIdx.x;
-  const int cl = tid & (DSSM_NC - 1), bl = tid / DSSM_NC;
+  const int cl = tid & (DSSM_NC - 1), bq = tid / DSSM_NC;
   const int c0 = blockIdx.x * DSSM_NC, b0 = blockIdx.y * DSSM_NB;
-  const int c = c0 + cl, b = b0 + bl;
-  const bool live = b < B;
-  // this thread's state first (the loads overlap the staging below)
-  float h[16];
-  float* hp = state + ((size_t)b * Di + c) * 16;
-  float x = 0.f, z = 0.f;
-  if (live) {
+  const int c = c0 + cl;
+  // this thread's states (four sequences x 16) first: their loads overlap the staging
+  float h[DSSM_BPT][16];
+  float xv[DSSM_BPT], zv[DSSM_BPT];
 #pragma unroll
-    for (int k = 0; k < 16; k += 4) {
-      const float4 v = *reinterpret_cast<const float4*>(hp + k);
-      h[k] = v.x; h[k + 1] = v.y; h[k + 2] = v.z; h[k + 3] = v.w;
+  for (int j = 0; j < DSSM_BPT; ++j) {
+    const int b = b0 + bq * DSSM_BPT + j;
+    if (b < B) {
+      const float* hp = state + ((size_t)b * Di + c) * 16;
+#pragma unroll
+      for (int k = 0; k < 16; k += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(hp + k);
+        h[j][k] = v.x; h[j][k + 1] = v.y; h[j][k + 2] = v.z; h[j][k + 3] = v.w;
+      }
+      xv[j] = __bfloat162float(xc[(size_t)b * Di + c]);
+      zv[j] = sum_slices<DEC_MAX_IN_SPLIT>(proj + (size_t)b * ld_proj + off_z + c, proj_stride, n_slices);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 16; ++k) h[j][k] = 0.f;
+      xv[j] = 0.f;
+      zv[j] = 0.f;
     }
-    x = __bfloat162float(xc[(size_t)b * Di + c]);
-    z = sum_slices<DEC_MAX_IN_SPLIT>(proj + (size_t)b * ld_proj + off_z + c, proj_stride, n_slices);
   }
+  // W_dt rows, transposed (R % 4 == 0); four loads in flight per thread
   {
-    const int r4 = R >> 2;   // R % 4 == 0
-    for (int i = tid; i < DSSM_NC * r4; i += DSSM_NB * DSSM_NC) {
-      const int cc = i / r4, q = i - cc * r4;
-      const float4 w4 = *reinterpret_cast<const float4*>(w_dt + (size_t)(c0 + cc) * ld_dt + q * 4);
-      wsh[cc][q * 4] = w4.x;
-      wsh[cc][q * 4 + 1] = w4.y;
-      wsh[cc][q * 4 + 2] = w4.z;
-      wsh[cc][q * 4 + 3] = w4.w;
+    const int n_items = DSSM_NC * (R >> 2);
+    for (int i0 = tid; i0 < n_items; i0 += 4 * DSSM_THREADS) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * DSSM_THREADS;
+        if (i < n_items)
+          v[u] = *reinterpret_cast<const float4*>(w_dt + (size_t)(c0 + (i & (DSSM_NC - 1))) * ld_dt + (i / DSSM_NC) * 4);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * DSSM_THREADS;
+        if (i < n_items) {
+          float* w = wsh + (i / DSSM_NC) * 4 * DSSM_NC + (i & (DSSM_NC - 1));
+          w[0] = v[u].x; w[DSSM_NC] = v[u].y; w[2 * DSSM_NC] = v[u].z; w[3 * DSSM_NC] = v[u].w;
+        }
+      }
     }
   }
-  const int nrow = R + 32;    // <= 256 = threads: one element of every sequence per thread
+  // x_proj outputs of the CTA's sequences, their split-K slices summed in a fixed order;
+  // item i = (column quad i / 16, sequence i % 16): lanes l and l + 16 read one 32-byte sector
+  {
+    const int n_items = DSSM_NB * ((R + 32) >> 2);
+    for (int i = tid; i < n_items; i += DSSM_THREADS) {
+      const int bl = i & (DSSM_NB - 1), q = i / DSSM_NB;
+      const bool ok = b0 + bl < B;
+      const float* src = xbc + (size_t)(b0 + bl) * ld_xbc + q * 4;
+      float4 v[DEC_MAX_XPROJ_SPLIT];
 #pragma unroll
-  for (int bb = 0; bb < DSSM_NB; ++bb)
-    if (tid < nrow)
-      dl[bb][tid] = b0 + bb < B ? sum_slices<DEC_MAX_XPROJ_SPLIT>(xbc + (size_t)(b0 + bb) * ld_xbc + tid, xbc_stride, n_xbc)
-                                : 0.f;
-  __syncthreads();
-  if (!live) return;
-  float acc0 = 0.f, acc1 = 0.f;
-  int r = 0;
-  for (; r + 1 < R; r += 2) {
-    acc0 = fmaf(dl[bl][r], wsh[cl][r], acc0);
-    acc1 = fmaf(dl[bl][r + 1], wsh[cl][r + 1], acc1);
+      for (int k = 0; k < DEC_MAX_XPROJ_SPLIT; ++k)
+        v[k] = (ok && k < n_xbc) ? *reinterpret_cast<const float4*>(src + k * xbc_stride) : make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 acc = v[0];
+#pragma unroll
+      for (int k = 1; k < DEC_MAX_XPROJ_SPLIT; ++k) {
+        acc.x += v[k].x; acc.y += v[k].y; acc.z += v[k].z; acc.w += v[k].w;
+      }
+      float* d = dlT + q * 4 * DSSM_NB + bl;
+      d[0] = acc.x; d[DSSM_NB] = acc.y; d[2 * DSSM_NB] = acc.z; d[3 * DSSM_NB] = acc.w;
+    }
   }
-  if (r < R) acc0 = fmaf(dl[bl][r], wsh[cl][r], acc0);
-  const float dt = softplus_f(acc0 + acc1 + dt_bias[c]);
-  const float dtx = dt * x;
-  const float* Bv = &dl[bl][R];
-  const float* Cv = &dl[bl][R + 16];
+  __syncthreads();
+  // dt_low . W_dt[c] for the four sequences (two partial sums each)
+  float acc[2][DSSM_BPT];
+#pragma unroll
+  for (int j = 0; j < DSSM_BPT; ++j) acc[0][j] = acc[1][j] = 0.f;
+  const float* dq = dlT + bq * DSSM_BPT;
+#pragma unroll 2
+  for (int r = 0; r < R; r += 2) {     // R even
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float w = wsh[(r + e) * DSSM_NC + cl];
+      const float4 d = *reinterpret_cast<const float4*>(dq + (r + e) * DSSM_NB);
+      acc[e][0] = fmaf(d.x, w, acc[e][0]);
+      acc[e][1] = fmaf(d.y, w, acc[e][1]);
+      acc[e][2] = fmaf(d.z, w, acc[e][2]);
+      acc[e][3] = fmaf(d.w, w, acc[e][3]);
+    }
+  }
+  const float bias = dt_bias[c];
+  float dt[DSSM_BPT], dtx[DSSM_BPT], yv[2][DSSM_BPT];
+#pragma unroll
+  for (int j = 0; j < DSSM_BPT; ++j) {
+    dt[j] = softplus_f(acc[0][j] + acc[1][j] + bias);
+    dtx[j] = dt[j] * xv[j];
+    yv[0][j] = yv[1][j] = 0.f;
+  }
   const float* Ar = A + (size_t)c * 16;
-  float yv0 = 0.f, yv1 = 0.f;
 #pragma unroll
   for (int k = 0; k < 16; k += 4) {
     const float4 a4 = *reinterpret_cast<const float4*>(Ar + k);
-    const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+    const float a2[4] = {a4.x * 1.4426950408889634f, a4.y * 1.4426950408889634f, a4.z * 1.4426950408889634f,
+                         a4.w * 1.4426950408889634f};   // exp(dt*A) = 2^(dt*A*log2 e)
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const int sidx = k + e;
-      h[sidx] = fmaf(ex2_approx(dt * av[e] * 1.4426950408889634f), h[sidx], dtx * Bv[sidx]);
-      if (e & 1) yv1 = fmaf(Cv[sidx], h[sidx], yv1);
-      else yv0 = fmaf(Cv[sidx], h[sidx], yv0);
+      const int s = k + e;
+      const float4 b4 = *reinterpret_cast<const float4*>(dq + (R + s) * DSSM_NB);
+      const float4 c4 = *reinterpret_cast<const float4*>(dq + (R + 16 + s) * DSSM_NB);
+      const float bv[4] = {b4.x, b4.y, b4.z, b4.w}, cv[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+      for (int j = 0; j < DSSM_BPT; ++j) {
+        h[j][s] = fmaf(ex2_approx(dt[j] * a2[e]), h[j][s], dtx[j] * bv[j]);
+        yv[s & 1][j] = fmaf(cv[j], h[j][s], yv[s & 1][j]);
+      }
     }
-    *reinterpret_cast<float4*>(hp + k) = make_float4(h[k], h[k + 1], h[k + 2], h[k + 3]);
   }
-  y[(size_t)b * Di + c] = (yv0 + yv1) * silu_f(z);
+#pragma unroll
+  for (int j = 0; j < DSSM_BPT; ++j) {
+    const int b = b0 + bq * DSSM_BPT + j;
+    if (b >= B) continue;
+    float* hp = state + ((size_t)b * Di + c) * 16;
+#pragma unroll
+    for (int k = 0; k < 16; k += 4) *reinterpret_cast<float4*>(hp + k) = make_float4(h[j][k], h[j][k + 1], h[j][k + 2], h[j][k + 3]);
+    y[(size_t)b * Di + c] = (yv[0][j] + yv[1][j]) * silu_f(zv[j]);
+  }
 }
 
 // RoPE angles: tab[pos][j] = (cos, sin) of pos * base^(-2j/64), the angle reduced mod 2*pi

@@ -171,7 +171,8 @@ __global__ void __launch_bounds__(SCAN_THREADS)
   if (tid == 0)
     for (; issued < SCAN_NST - 1 && issued < n_chunks; ++issued) issue(issued);
 
-  float h0 = 0.f, h1 = 0.f;
+  uint64_t h01 = 0;                  // (h of state l8, h of state l8 + 8)
+  const uint64_t A01 = f2_pack(A0, A1);
   float* part = sm.part[warp];
   int k = 0;
   for (; k < n_chunks; ++k) {
@@ -196,9 +197,10 @@ __global__ void __launch_bounds__(SCAN_THREADS)
     for (int hc = 0; hc < SCAN_TC; hc += SCAN_HALF) {
 #pragma unroll
       for (int u8 = 0; u8 < SCAN_HALF; u8 += 8) {
-        // 8 steps: operands and the 16 exponentials first (independent of the state), then
-        // the two recurrences; keeps enough independent work in flight per warp
-        float ea0[8], ea1[8], eb0[8], eb1[8], ec0[8], ec1[8];
+        // 8 steps; the lane's two states travel as (state l8, state l8 + 8) pairs through
+        // the paired fp32 instructions.  Operands and exponentials first (independent of
+        // the state), then the recurrence.
+        uint64_t ea[8], eb[8], ec[8];
 #pragma unroll
         for (int u = 0; u < 8; u += 4) {
           const float4 p01 = *reinterpret_cast<const float4*>(&sm.dd[cw][hc + u8 + u]);       // steps u, u+1
@@ -213,20 +215,18 @@ __global__ void __launch_bounds__(SCAN_THREADS)
           for (int e = 0; e < 4; ++e) {
             const float2 bc0 = __half22float2(*reinterpret_cast<const __half2*>(&w0[e]));   // (B, C) of state l8
             const float2 bc1 = __half22float2(*reinterpret_cast<const __half2*>(&w1[e]));   // (B, C) of state l8+8
-            ea0[u + e] = ex2_approx(dl[e] * A0);
-            ea1[u + e] = ex2_approx(dl[e] * A1);
-            eb0[u + e] = dxl[e] * bc0.x;
-            eb1[u + e] = dxl[e] * bc1.x;
-            ec0[u + e] = bc0.y;
-            ec1[u + e] = bc1.y;
+            const uint64_t arg = f2_mul(f2_pack(dl[e], dl[e]), A01);
+            ea[u + e] = f2_pack(ex2_approx(f2_lo(arg)), ex2_approx(f2_hi(arg)));
+            eb[u + e] = f2_mul(f2_pack(dxl[e], dxl[e]), f2_pack(bc0.x, bc1.x));
+            ec[u + e] = f2_pack(bc0.y, bc1.y);
           }
         }
         float v[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          h0 = fmaf(ea0[e], h0, eb0[e]);
-          h1 = fmaf(ea1[e], h1, eb1[e]);
-          v[e] = fmaf(ec1[e], h1, ec0[e] * h0);
+          h01 = f2_fma(ea[e], h01, eb[e]);
+          const uint64_t ch = f2_mul(ec[e], h01);
+          v[e] = f2_lo(ch) + f2_hi(ch);
         }
         // slot l8 ^ f(step group, channel): conflict-free on both the write and the read side
 #pragma unroll
@@ -270,8 +270,8 @@ __global__ void __launch_bounds__(SCAN_THREADS)
         mbar_wait(&sm.full[j % SCAN_NST], (uint32_t)(j / SCAN_NST) & 1u, nullptr, status, 302);
     return;
   }
-  state[((size_t)b * Di + c) * 16 + l8] = h0;
-  state[((size_t)b * Di + c) * 16 + l8 + 8] = h1;
+  state[((size_t)b * Di + c) * 16 + l8] = f2_lo(h01);
+  state[((size_t)b * Di + c) * 16 + l8 + 8] = f2_hi(h01);
 }
 
 }  // namespace hymba
