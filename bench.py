@@ -417,7 +417,10 @@ def run_decode(args, device, world):
         if name in wk and wk[name] > 0:
             e["gbs"] = round(wk[name] / (avg * 1e-3) / 1e9, 1)
         kern[name] = e
-    dom = max(per, key=lambda n: float(np.sum(per[n])))
+    # the dominant decode kernel is the one that moves the most bytes (the attention over the
+    # K/V cache); event times of the two concurrent branches overlap, so time shares would
+    # rank a kernel that waits for SMs above one that works
+    dom = max(per, key=lambda n: wk.get(n, 0.0))
     dom_avg = float(np.mean(per[dom])) * 1e-3
     roof = {"bound": "hbm", "kernel": dom, "achieved": round(wk.get(dom, 0.0) / dom_avg / 1e9, 1),
             "peak": peaks["hbm_gbs"], "unit": "GB/s"}
@@ -544,7 +547,6 @@ def run_stack(args, device, world):
 # workload (profiles/ holds the summaries and commands); a kernel changed since its capture
 # has no entry.  ncu replays a kernel with cold caches: writes that stay in L2 do not show.
 TRAFFIC = {
-    "selective_scan": 42279680 + 16128,     # profiles/selective_scan_and_norm_swa.md
     "norm_avg": 41827840 + 458496,          # profiles/selective_scan_and_norm_swa.md
     "out_proj": 36292608 + 40704,           # profiles/gemm_out_proj_swa.md
 }

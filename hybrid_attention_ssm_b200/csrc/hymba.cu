@@ -389,9 +389,13 @@ int pick_bn_cover(int n) {
   if (n <= 160) return 160;
   return 256;
 }
-// tile width for a wide N: 256 unless that leaves most SMs idle
-int pick_bn_wide(int m_tiles, int N, int sms) {
-  return (long long)m_tiles * cdiv(N, 256) >= sms ? 256 : 128;
+// Tile width for an epilogue-bound GEMM (a short K and a heavy epilogue): the one that
+// gives the busiest SM the fewest accumulator columns, (rounds of the persistent grid) x
+// width; the narrower wins a tie (its next tile's MMAs overlap the epilogue sooner).
+int pick_bn_epilogue(int m_tiles, int N, int sms) {
+  const long long r128 = ((long long)m_tiles * cdiv(N, 128) + sms - 1) / sms;
+  const long long r256 = ((long long)m_tiles * cdiv(N, 256) + sms - 1) / sms;
+  return r256 * 256 < r128 * 128 ? 256 : 128;
 }
 // Tile width among `cands` minimising (rounds of the persistent grid) x (operand bytes per
 // k-block): the mainloops run at the rate shared memory is fed, so a round of tiles costs
@@ -876,7 +880,7 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     c.etype = ET_TF32;
     c.a1 = f32(L.xbc); c.nb1 = B; c.rows1 = T; c.lda1 = m.ld_xbc; c.a1_bstride = (long long)T * m.ld_xbc;
     c.b = w->w_dt; c.N = m.Di; c.ldb = w->w_dt_ld; c.K = m.R;
-    c.bn = pick_bn_wide(B * cdiv(T, GEMM_BM), m.Di, dev->sms);
+    c.bn = pick_bn_epilogue(B * cdiv(T, GEMM_BM), m.Di, dev->sms);
     c.name = "dt_proj";
     c.mode = EPI_SOFTPLUS_T;
     c.p.out = f32(L.dT);
@@ -1128,6 +1132,7 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
       HY_CUDA(cudaFuncSetAttribute(decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DA_SMEM));
       attr_da[dcur & 63] = true;
     }
+    // three CTAs per SM (four would fit) leave room for the SSM step running beside it
     const int grid = ap.n_items < 3 * dev->sms ? ap.n_items : 3 * dev->sms;
     HY_CUDA(cudaEventRecord(side->fork, st));   // every host-side check has passed
     HY_CUDA(cudaStreamWaitEvent(ast, side->fork, 0));

@@ -353,7 +353,7 @@ __device__ __forceinline__ uint32_t sw128_addr(uint32_t tile, int r, int chunk) 
   return tile + r * 128 + ((chunk ^ (r & 7)) << 4);
 }
 
-__global__ void __launch_bounds__(DA_THREADS)
+__global__ void __launch_bounds__(DA_THREADS, 4)
     decode_attn_kernel(const __grid_constant__ CUtensorMap mapMK, const __grid_constant__ CUtensorMap mapMV,
                        const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                        const __grid_constant__ DecAttnParams p) {
@@ -364,7 +364,6 @@ __global__ void __launch_bounds__(DA_THREADS)
   __shared__ uint64_t full[DA_STAGES];
   __shared__ __align__(16) float qbuf[DA_STAGES][DEC_MAXG * 64];
   __shared__ float cm[4][8], cl[4][8];
-  __shared__ __align__(16) float co[4][8][64];
   __shared__ int abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gq = lane >> 2, tq = lane & 3;   // fragment row (query head) and column pair
@@ -499,7 +498,10 @@ __global__ void __launch_bounds__(DA_THREADS)
       }
     }
     if (!ok) break;
-    // merge the 4 warps' states for rows (heads) < G
+    // merge the 4 warps' states for rows (heads) < G.  The warps' O rows go to the stage of
+    // the item's last tile: the barrier above released it, and the producer refills it only
+    // at the top of the next item, after the barrier that ends this merge.
+    float (*co)[8][64] = reinterpret_cast<float (*)[8][64]>(tiles + ((ct - 1) % DA_STAGES) * 2 * DA_TILE_BYTES);
     if (gq < 8) {
       if (tq == 0) {
         cm[warp][gq] = m_run;
@@ -529,6 +531,7 @@ __global__ void __launch_bounds__(DA_THREADS)
         dst[1] = L;
       }
     }
+    fence_proxy_async_smem();   // the O rows were written through the generic proxy; TMA refills the stage
     __syncthreads();   // cm, cl, co are rewritten by the next item
   }
   if (!ok && tid == 0)   // let the loads in flight land before the CTA exits
@@ -588,10 +591,12 @@ constexpr int DSSM_NC = 32;    // channels per CTA: one per lane
 constexpr int DSSM_NB = 16;    // sequences per CTA
 constexpr int DSSM_BPT = 4;    // sequences per thread; the lanes of a warp share them
 constexpr int DSSM_THREADS = DSSM_NC * DSSM_NB / DSSM_BPT;   // 128
+constexpr int DSSM_A_LD = 20;  // A rows in shared memory (16 + 4: conflict-free 16-byte reads)
 // dynamic shared memory: W_dt rows of the CTA's channels [R][32] and the summed x_proj
-// outputs of its sequences [R + 32][16] (dt_low | B | C), both transposed
+// outputs of its sequences [R + 32][16] (dt_low | B | C), both transposed, then the
+// channels' A * log2(e) rows [32][20] and dt biases [32]
 __host__ __device__ constexpr size_t dssm_smem_bytes(int R) {
-  return ((size_t)R * DSSM_NC + (size_t)(R + 32) * DSSM_NB) * sizeof(float);
+  return ((size_t)R * DSSM_NC + (size_t)(R + 32) * DSSM_NB + DSSM_NC * DSSM_A_LD + DSSM_NC) * sizeof(float);
 }
 
 __global__ void __launch_bounds__(DSSM_THREADS, 3)
@@ -606,6 +611,8 @@ __global__ void __launch_bounds__(DSSM_THREADS, 3)
   extern __shared__ __align__(16) float dssm_sh[];
   float* wsh = dssm_sh;                    // W_dt[c0 + cl][r] at r * 32 + cl
   float* dlT = dssm_sh + R * DSSM_NC;      // x_proj output [b0 + bl][col] at col * 16 + bl
+  float* ash = dlT + (R + 32) * DSSM_NB;   // A[c0 + cl][s] * log2(e) at cl * 20 + s
+  float* bsh = ash + DSSM_NC * DSSM_A_LD;  // dt_bias[c0 + cl]
   const int tid = threadIdx.x;
   const int cl = tid & (DSSM_NC - 1), bq = tid / DSSM_NC;
   const int c0 = blockIdx.x * DSSM_NC, b0 = blockIdx.y * DSSM_NB;
@@ -632,6 +639,10 @@ __global__ void __launch_bounds__(DSSM_THREADS, 3)
       zv[j] = 0.f;
     }
   }
+  // the channels' A rows and dt biases ride with the W_dt loads (one 16-byte piece of A per thread)
+  static_assert(DSSM_THREADS == DSSM_NC * 4, "one quarter of an A row per thread");
+  const float4 a_in = *reinterpret_cast<const float4*>(A + (size_t)(c0 + (tid >> 2)) * 16 + (tid & 3) * 4);
+  const float bias_in = tid < DSSM_NC ? dt_bias[c0 + tid] : 0.f;
   // W_dt rows, transposed (R % 4 == 0); four loads in flight per thread
   {
     const int n_items = DSSM_NC * (R >> 2);
@@ -653,6 +664,10 @@ __global__ void __launch_bounds__(DSSM_THREADS, 3)
       }
     }
   }
+  *reinterpret_cast<float4*>(ash + (tid >> 2) * DSSM_A_LD + (tid & 3) * 4) =
+      make_float4(a_in.x * 1.4426950408889634f, a_in.y * 1.4426950408889634f, a_in.z * 1.4426950408889634f,
+                  a_in.w * 1.4426950408889634f);   // exp(dt*A) = 2^(dt*A*log2 e)
+  if (tid < DSSM_NC) bsh[tid] = bias_in;
   // x_proj outputs of the CTA's sequences, their split-K slices summed in a fixed order;
   // item i = (column quad i / 16, sequence i % 16): lanes l and l + 16 read one 32-byte sector
   {
@@ -692,7 +707,7 @@ __global__ void __launch_bounds__(DSSM_THREADS, 3)
       acc[e][3] = fmaf(d.w, w, acc[e][3]);
     }
   }
-  const float bias = dt_bias[c];
+  const float bias = bsh[cl];
   float dt[DSSM_BPT], dtx[DSSM_BPT], yv[2][DSSM_BPT];
 #pragma unroll
   for (int j = 0; j < DSSM_BPT; ++j) {
@@ -700,12 +715,10 @@ __global__ void __launch_bounds__(DSSM_THREADS, 3)
     dtx[j] = dt[j] * xv[j];
     yv[0][j] = yv[1][j] = 0.f;
   }
-  const float* Ar = A + (size_t)c * 16;
 #pragma unroll
   for (int k = 0; k < 16; k += 4) {
-    const float4 a4 = *reinterpret_cast<const float4*>(Ar + k);
-    const float a2[4] = {a4.x * 1.4426950408889634f, a4.y * 1.4426950408889634f, a4.z * 1.4426950408889634f,
-                         a4.w * 1.4426950408889634f};   // exp(dt*A) = 2^(dt*A*log2 e)
+    const float4 a4 = *reinterpret_cast<const float4*>(ash + cl * DSSM_A_LD + k);
+    const float a2[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int s = k + e;
