@@ -547,8 +547,17 @@ def run_stack(args, device, world):
 # workload (profiles/ holds the summaries and commands); a kernel changed since its capture
 # has no entry.  ncu replays a kernel with cold caches: writes that stay in L2 do not show.
 TRAFFIC = {
-    "norm_avg": 41827840 + 458496,          # profiles/selective_scan_and_norm_swa.md
-    "out_proj": 36292608 + 40704,           # profiles/gemm_out_proj_swa.md
+    "selective_scan": 42143488 + 5376,
+    "norm_avg": 41828352 + 261632,
+    "in_proj": 35336704 + 976384,
+    "x_proj": 14797824 + 256,
+    "dt_proj": 2486784 + 0,
+    "out_proj": 36292608 + 15104,
+    "attention": 9816320 + 768,
+    "conv1d_silu": 13999616 + 768,
+    "decode_attn": 94810880 + 4270592,
+    "decode_prep": 5318912 + 0,
+    "decode_ssm": 16947200 + 0,
 }
 
 
