@@ -236,35 +236,12 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// sm_100 paired fp32 arithmetic and the three-input max (one instruction for two lanes'
-// worth of values, or for two comparisons).
+// three-input max (one instruction for two comparisons)
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-// (d0, d1) = (a0, a1) * (b, b) + (c, c)
-__device__ __forceinline__ void ffma2_bc(float& d0, float& d1, float a0, float a1, float b, float c) {
-  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\t"
-      "mov.b64 rb, {%4, %4};\n\t"
-      "mov.b64 rc, {%5, %5};\n\t"
-      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
-      "mov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b), "f"(c));
-}
-// (d0, d1) += (a0, a1)
-__device__ __forceinline__ void fadd2_acc(float& d0, float& d1, float a0, float a1) {
-  asm("{\n\t.reg .b64 ra, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\t"
-      "mov.b64 rd, {%0, %1};\n\t"
-      "add.rn.f32x2 rd, rd, ra;\n\t"
-      "mov.b64 {%0, %1}, rd;\n\t}"
-      : "+f"(d0), "+f"(d1)
-      : "f"(a0), "f"(a1));
-}
-
 // Paired fp32 arithmetic on (x, y) pairs kept in 64-bit registers (sm_100 f32x2 forms).
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
@@ -302,14 +279,6 @@ __device__ __forceinline__ void store_bf16_row(__nv_bfloat16* dst, const float* 
   }
 }
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -339,15 +308,6 @@ __device__ __forceinline__ float lg2_approx(float x) {
   float y;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-// softplus(x) = log(1 + e^x) from the hardware ex2/lg2: x for x > 15 (the remainder is
-// below 3.1e-7); with u = e^x, log1p(u) = ln2 * log2(1 + u) for u >= 2^-7 (relative error
-// below 3e-5 there), and the series u - u^2/2 + u^3/3 below (error below u^4/4).
-__device__ __forceinline__ float softplus_fast(float x) {
-  if (x > 15.f) return x;
-  const float u = ex2_approx(x * 1.4426950408889634f);
-  if (u < 0.0078125f) return u * (1.f - u * (0.5f - u * 0.33333334f));
-  return lg2_approx(1.f + u) * 0.6931471805599453f;
 }
 __device__ __forceinline__ float rcp_approx(float x) {
   float y;

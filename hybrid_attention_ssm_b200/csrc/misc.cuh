@@ -1,6 +1,6 @@
-// Memory-bound kernels: per-branch RMSNorm + beta + average, SWA cache finalisation,
-// decode-step attention (RoPE, ring write, split-K over keys), conv/SSM decode step,
-// split-K finalisation.
+// Memory-bound kernels: per-branch RMSNorm + beta + average, the decode step (conv step and
+// RoPE with the cache write, attention split over key tiles and its merge, the SSM step),
+// split-K finalisation, RoPE tables, the stack's RMSNorm and the meta prepend.
 #pragma once
 #include "common.cuh"
 
@@ -28,11 +28,6 @@ __device__ __forceinline__ void unpack8(const uint4& r, float* f) {
   const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&r);
 #pragma unroll
   for (int e = 0; e < 8; ++e) f[e] = __bfloat162float(h[e]);
-}
-__device__ __forceinline__ void unpack8h(const uint4& r, float* f) {
-  const __half* h = reinterpret_cast<const __half*>(&r);
-#pragma unroll
-  for (int e = 0; e < 8; ++e) f[e] = __half2float(h[e]);
 }
 
 // ----------------------------------------------------------------------------------------
@@ -868,18 +863,6 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, int n_split
       if (cc >= 0 && cc < 32) bcp[(((size_t)b * 16 + (cc & 15)) * Tp + t) * 2 + (cc >> 4)] = __float2half_rn(vals[e]);
     }
   }
-}
-
-// out[r, c] = bf16(acc[r, c] + residual[r, c])
-__global__ void f32_to_bf16_residual_kernel(const float* __restrict__ acc, const __nv_bfloat16* __restrict__ res,
-                                            __nv_bfloat16* __restrict__ out, int n) {
-  pdl_wait();
-  pdl_trigger();
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  float v = acc[i];
-  if (res != nullptr) v += __bfloat162float(res[i]);
-  out[i] = __float2bfloat16_rn(v);
 }
 
 }  // namespace hymba
