@@ -169,6 +169,23 @@ int side_stream(SideStream** out) {
   return HYMBA_OK;
 }
 
+// Between a fork and its join, an error return would leave work on the side stream outside
+// the caller's stream (and a stream capture with an unjoined branch).  The guard joins the
+// side stream back into the caller's stream when it goes out of scope still open.
+struct ForkGuard {
+  SideStream* side;
+  cudaStream_t st;
+  bool open = false;
+  ForkGuard(SideStream* s, cudaStream_t stream) : side(s), st(stream) {}
+  ForkGuard(const ForkGuard&) = delete;
+  ForkGuard& operator=(const ForkGuard&) = delete;
+  ~ForkGuard() {
+    if (!open) return;
+    cudaEventRecord(side->join, side->s);   // best effort: the call is already failing
+    cudaStreamWaitEvent(st, side->join, 0);
+  }
+};
+
 // Inside a stream capture the events become event-record nodes of the graph (the external
 // flag), so every replay re-records them.
 inline void prof_record(cudaEvent_t ev, cudaStream_t st) {
@@ -895,9 +912,11 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
   //    stream after dt_proj and runs beside the scan: both are latency-bound and fit on one
   //    SM together (one attention CTA, three scan CTAs).  Otherwise it runs in stream order.
   const bool overlap = (long long)B * (m.Di / SCAN_CH) < 3LL * dev->sms;
+  ForkGuard fork_guard(side, st);
   if (overlap) {
     HY_CUDA(cudaEventRecord(side->fork, st));
     HY_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
+    fork_guard.open = true;
   }
   {
     CUtensorMap mq, mk, mv;
@@ -965,7 +984,10 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     prof_end(st);
   }
   // 7. per-branch RMSNorm, gate, beta, average (the attention branch joins here)
-  if (overlap) HY_CUDA(cudaStreamWaitEvent(st, side->join, 0));
+  if (overlap) {
+    HY_CUDA(cudaStreamWaitEvent(st, side->join, 0));
+    fork_guard.open = false;
+  }
   {
     prof_begin("norm_avg", st);
     HY_TRY(launch_branch_norm<__nv_bfloat16>(f32(L.o), m.qw, m.qw, bf(L.y), m.Di, bf(L.xz) + m.Di, 2 * m.Di, m.Di,
@@ -1083,6 +1105,7 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
   //    that leave most of the GPU idle), joined before the norm.
   SideStream* side = nullptr;
   HY_TRY(side_stream(&side));
+  ForkGuard fork_guard(side, st);
   {
     const cudaStream_t ast = side->s;
     DecAttnParams ap;
@@ -1136,6 +1159,7 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     const int grid = ap.n_items < 3 * dev->sms ? ap.n_items : 3 * dev->sms;
     HY_CUDA(cudaEventRecord(side->fork, st));   // every host-side check has passed
     HY_CUDA(cudaStreamWaitEvent(ast, side->fork, 0));
+    fork_guard.open = true;
     prof_begin("decode_attn", ast);
     HY_CUDA(launch_pdl(decode_attn_kernel, dim3(grid), dim3(DA_THREADS), DA_SMEM, ast, mmk, mmv, mk, mv, ap));
     prof_end(ast);
@@ -1175,6 +1199,7 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
   }
   // 6. norm + average (y already gated); the attention branch joins here
   HY_CUDA(cudaStreamWaitEvent(st, side->join, 0));
+  fork_guard.open = false;
   {
     prof_begin("decode_norm_avg", st);
     HY_TRY(launch_branch_norm<float>(f32(L.o), m.qw, m.qw, f32(L.y), m.Di, nullptr, 0, m.Di, w->g_attn, w->g_ssm,
