@@ -130,6 +130,22 @@ def test_conv_state_carry():
     np.testing.assert_allclose(last_full, x[-3:].T)
 
 
+def test_x_proj_column_layout():
+    """The boundary fixes the rows of W_x as [dt_low (R) | B (S) | C (S)].  With W_x a row
+    selection the projection hands out xc's own columns, so each output must be the
+    corresponding slice of xc; with W_dt = 0, Delta is softplus(bias) in every row."""
+    rng = np.random.default_rng(13)
+    L, Di, R, S = 5, 12, 3, 4
+    xc = rng.normal(size=(L, Di))
+    w_x = np.eye(R + 2 * S, Di)
+    bias = rng.normal(size=Di)
+    delta, Bm, Cm, dt_low = orc.ssm_params(xc, w_x, np.zeros((Di, R)), bias, R, S)
+    np.testing.assert_array_equal(dt_low, xc[:, :R])
+    np.testing.assert_array_equal(Bm, xc[:, R:R + S])
+    np.testing.assert_array_equal(Cm, xc[:, R + S:R + 2 * S])
+    np.testing.assert_allclose(delta, np.log1p(np.exp(bias))[None, :].repeat(L, axis=0), rtol=1e-15)
+
+
 def test_elementwise_closed_forms():
     assert orc.softplus(0.0) == pytest.approx(math.log(2.0), rel=1e-15)
     assert orc.softplus(50.0) == pytest.approx(50.0, rel=1e-15)
