@@ -219,6 +219,25 @@ def test_prefill_then_decode_matches_longer_prefill(is_global):
     assert_rel_inf(to_np(run.ssm), ref["ssm_state"], tol=2e-2, name="state after decode")
 
 
+def test_prefill_and_decode_at_the_size_limits():
+    """Every width at the largest value the library accepts: d_inner 4096 and Hq*D 2048 (the
+    norm's per-thread chunks full), dt_rank 224 (dt_low | B | C = 256 columns: the widest
+    x_proj tile and the largest decode SSM staging), 4 query heads per KV head."""
+    dims = WL["tiny"].dims.replace(d_model=1024, n_q_heads=32, n_kv_heads=8, d_inner=4096, dt_rank=224,
+                                   n_meta=8, window=48)
+    w = _w(dims, seed=21)
+    N = 60
+    X = synth.bf16_round(np.random.default_rng(22).normal(size=(2, N + 1, dims.d_model)).astype(np.float32))
+    T = dims.n_meta + N
+    run = PrefillRun(dims, w, X[:, :N], max_tokens=T + 1)
+    ref_n = orc.mixer_prefill(dims, w, X[:, :N])
+    assert_rms(to_np(run.out), ref_n["out"], name="prefill out at the limits")
+    assert_rel_inf(to_np(run.ssm), ref_n["ssm_state"], tol=2e-2, name="ssm state at the limits")
+    out = _decode(dims, w, run.cache, X[:, N], T, run.ssm, run.conv)
+    ref = orc.mixer_prefill(dims, w, X)
+    assert_rms(to_np(out), ref["out"][:, -1], name="decode at the limits vs oracle prefill(T+1)")
+
+
 def test_decode_pair_hymba():
     wl = WL["decode_pair"]
     prod = wl.dims
