@@ -656,6 +656,7 @@ def main():
             "e2e": {"value": round(e2e, 1), "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"],
                     "d2h_bytes_per_step": r["d2h"],
                     "how": "pinned host X -> device, C-ABI prefill, device -> pinned host out; CUDA events"},
+            "input_tokens_per_s": round(tokens_per_s * cfg["n_tokens"] / cfg["seq_len"], 1),   # B*N / time
             "gpu_launches": int(round(r["launches_per_step"] * args.steps)),
             "roofline": r["roofline"], "step_roofline": r["step_roofline"], "clocks": r["clocks"],
             "kernels": r["kernels"], "decode": r["decode"]}
