@@ -134,8 +134,6 @@ template <int BN, int STAGES, int ET, int MODE>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA0, const __grid_constant__ CUtensorMap mapA1,
                    const __grid_constant__ CUtensorMap mapB, const __grid_constant__ GemmParams p) {
-  pdl_wait();
-  pdl_trigger();
   using L = GemmSmem<BN, STAGES>;
   constexpr int ACC_STRIDE = BN <= 128 ? 128 : 256;       // TMEM columns per accumulator
   constexpr uint32_t TMEM_COLS = 2 * ACC_STRIDE;
@@ -179,6 +177,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // The set-up above touches only this CTA's shared memory, its TMEM and the kernel
+  // parameters, so it overlaps the previous kernel's tail.  Every access to global memory
+  // comes after the wait.  A CTA launched early can only meet TMEM held by CTAs of the
+  // previous kernel, which are all running by then and free it when they finish.
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
