@@ -549,10 +549,10 @@ def run_stack(args, device, world):
 TRAFFIC = {
     "selective_scan": 42143488 + 5376,
     "norm_avg": 41828352 + 261632,
-    "in_proj": 35336704 + 976384,
+    "in_proj": 35357184 + 1401856,
     "x_proj": 14797824 + 256,
-    "dt_proj": 2486784 + 0,
-    "out_proj": 36292608 + 15104,
+    "dt_proj": 2488320 + 0,
+    "out_proj": 36292864 + 22784,
     "attention": 9816320 + 768,
     "conv1d_silu": 13999616 + 768,
     "decode_attn": 94810880 + 4270592,
