@@ -308,7 +308,8 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(const __grid_constant_
 constexpr int DA_KT = 64;               // keys per tile
 constexpr int DA_STAGES = 3;
 constexpr int DA_TPS = 3;               // tiles per split
-constexpr int DA_THREADS = 128;
+constexpr int DA_CONSUMERS = 128;      // 4 consumer warps
+constexpr int DA_THREADS = DA_CONSUMERS + 32;   // + the producer warp
 constexpr int DA_TILE_BYTES = DA_KT * 128;
 constexpr int DEC_MAXG = 6;             // max query heads per KV head
 constexpr int DA_Q_BYTES = DEC_MAXG * 64 * 4;   // an item's queries ride with its first tile
@@ -348,7 +349,11 @@ __device__ __forceinline__ uint32_t sw128_addr(uint32_t tile, int r, int chunk) 
   return tile + r * 128 + ((chunk ^ (r & 7)) << 4);
 }
 
-__global__ void __launch_bounds__(DA_THREADS, 4)
+__device__ __forceinline__ void da_consumer_sync() {   // the four consumer warps only
+  asm volatile("bar.sync 1, %0;" ::"n"(DA_CONSUMERS) : "memory");
+}
+
+__global__ void __launch_bounds__(DA_THREADS, 3)
     decode_attn_kernel(const __grid_constant__ CUtensorMap mapMK, const __grid_constant__ CUtensorMap mapMV,
                        const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                        const __grid_constant__ DecAttnParams p) {
@@ -356,15 +361,18 @@ __global__ void __launch_bounds__(DA_THREADS, 4)
   pdl_trigger();
   extern __shared__ uint8_t da_smem_raw[];
   uint8_t* tiles = align_smem<1024>(da_smem_raw);
-  __shared__ uint64_t full[DA_STAGES];
+  __shared__ uint64_t full[DA_STAGES], empty[DA_STAGES];
   __shared__ __align__(16) float qbuf[DA_STAGES][DEC_MAXG * 64];
   __shared__ float cm[4][8], cl[4][8];
+  __shared__ __align__(16) float co[4][8][64];
   __shared__ int abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int gq = lane >> 2, tq = lane & 3;   // fragment row (query head) and column pair
   const int G = p.Hq / p.Hkv;
   if (tid == 0) {
-    for (int i = 0; i < DA_STAGES; ++i) mbar_init(&full[i], 1);
+    for (int i = 0; i < DA_STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], DA_CONSUMERS / 32);
+    }
     abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&mapMK);
@@ -373,38 +381,51 @@ __global__ void __launch_bounds__(DA_THREADS, 4)
     tma_prefetch_desc(&mapV);
   }
   __syncthreads();
-
   auto item_tiles = [&](int w) { return min(DA_TPS, p.n_tiles - (w % p.n_splits) * DA_TPS); };
-  // producer state (thread 0): the next (item, tile) of this CTA's sequence
-  int pw = blockIdx.x, pt = 0, issued = 0;
-  auto issue_next = [&]() {
-    while (pw < p.n_items && pt >= item_tiles(pw)) {
-      pw += gridDim.x;
-      pt = 0;
-    }
-    if (pw >= p.n_items) return;
-    const int split = pw % p.n_splits, bg = pw / p.n_splits;
-    const int g = bg % p.Hkv, b = bg / p.Hkv;
-    const int ti = split * DA_TPS + pt;
-    const int stg = issued % DA_STAGES;
-    uint8_t* kt = tiles + stg * 2 * DA_TILE_BYTES;
-    const uint32_t q_bytes = pt == 0 ? (uint32_t)(G * 64 * 4) : 0u;
-    mbar_arrive_expect_tx(&full[stg], 2 * DA_TILE_BYTES + q_bytes);
-    if (pt == 0) bulk_load(&qbuf[stg][0], p.qrot + ((size_t)b * p.Hq + g * G) * 64, q_bytes, &full[stg]);
-    if (ti < p.n_meta_tiles) {
-      tma_load_2d(kt, &mapMK, &full[stg], g * 64, b * p.M + ti * DA_KT);
-      tma_load_2d(kt + DA_TILE_BYTES, &mapMV, &full[stg], g * 64, b * p.M + ti * DA_KT);
-    } else {
-      const int r0 = b * p.rows_main + (ti - p.n_meta_tiles) * DA_KT;
-      tma_load_2d(kt, &mapK, &full[stg], g * 64, r0);
-      tma_load_2d(kt + DA_TILE_BYTES, &mapV, &full[stg], g * 64, r0);
-    }
-    ++pt;
-    ++issued;
-  };
-  if (tid == 0)
-    for (int k = 0; k < DA_STAGES - 1; ++k) issue_next();
 
+  if (warp == DA_CONSUMERS / 32) {
+    // ------------------------------ producer warp ------------------------------
+    // Streams this CTA's (item, tile) sequence through the ring; a stage is refilled once
+    // the four consumer warps have released it.
+    if (lane == 0) {
+      int issued = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
+        const int split = w % p.n_splits, bg = w / p.n_splits;
+        const int g = bg % p.Hkv, b = bg / p.Hkv;
+        const int nt = item_tiles(w);
+        for (int t = 0; t < nt; ++t, ++issued) {
+          const int stg = issued % DA_STAGES;
+          if (issued >= DA_STAGES &&
+              !mbar_wait(&empty[stg], (uint32_t)(issued / DA_STAGES - 1) & 1u, &abort_flag, p.status, 503)) {
+            ok = false;
+            break;
+          }
+          const int ti = split * DA_TPS + t;
+          uint8_t* kt = tiles + stg * 2 * DA_TILE_BYTES;
+          const uint32_t q_bytes = t == 0 ? (uint32_t)(G * 64 * 4) : 0u;
+          mbar_arrive_expect_tx(&full[stg], 2 * DA_TILE_BYTES + q_bytes);
+          if (t == 0) bulk_load(&qbuf[stg][0], p.qrot + ((size_t)b * p.Hq + g * G) * 64, q_bytes, &full[stg]);
+          if (ti < p.n_meta_tiles) {
+            tma_load_2d(kt, &mapMK, &full[stg], g * 64, b * p.M + ti * DA_KT);
+            tma_load_2d(kt + DA_TILE_BYTES, &mapMV, &full[stg], g * 64, b * p.M + ti * DA_KT);
+          } else {
+            const int r0 = b * p.rows_main + (ti - p.n_meta_tiles) * DA_KT;
+            tma_load_2d(kt, &mapK, &full[stg], g * 64, r0);
+            tma_load_2d(kt + DA_TILE_BYTES, &mapV, &full[stg], g * 64, r0);
+          }
+        }
+      }
+      // the last fills may still be in flight (all of them, if the consumers gave up): let
+      // them land before the CTA can exit
+      for (int j = issued > DA_STAGES ? issued - DA_STAGES : 0; j < issued; ++j)
+        mbar_wait(&full[j % DA_STAGES], (uint32_t)(j / DA_STAGES) & 1u, nullptr, p.status, 504);
+    }
+    return;
+  }
+
+  // ------------------------------ consumer warps ------------------------------
+  const int gq = lane >> 2, tq = lane & 3;   // fragment row (query head) and column pair
   const uint32_t tiles_u32 = smem_u32(tiles);
   // ldmatrix row of this lane: K fragments (keys x dims), V fragments (.trans)
   const int k_row = warp * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
@@ -423,9 +444,12 @@ __global__ void __launch_bounds__(DA_THREADS, 4)
 #pragma unroll
     for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
     for (int t = 0; t < nt; ++t, ++ct) {
-      if (tid == 0) issue_next();   // the stage of tile ct-1 was released by the last barrier
       const int stg = ct % DA_STAGES;
-      if (!mbar_wait(&full[stg], (uint32_t)(ct / DA_STAGES) & 1u, &abort_flag, p.status, 501)) ok = false;
+      // after a wait has given up, the warps keep walking the items (so that every one of
+      // them reaches the same merge barriers) without waiting or releasing stages
+      if (ok) ok = mbar_wait(&full[stg], (uint32_t)(ct / DA_STAGES) & 1u, &abort_flag, p.status, 501);
+      ok = __all_sync(0xffffffffu, ok);   // one verdict per warp: the shuffles below need all lanes
+      if (!ok) continue;
       if (t == 0) {   // the item's queries arrived with its first tile
         const float* q = &qbuf[stg][gq * 64];
 #pragma unroll
@@ -487,16 +511,10 @@ __global__ void __launch_bounds__(DA_THREADS, 4)
         mma_16816(o[j], pa0, 0u, pa2, 0u, b0, b1);
         mma_16816(o[j + 1], pa0, 0u, pa2, 0u, b2, b3);
       }
-      if (__syncthreads_or(ok ? 0 : 1)) {   // stage free; a wait gave up: every thread leaves
-        ok = false;
-        break;
-      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stg]);   // this warp is done with the stage
     }
-    if (!ok) break;
-    // merge the 4 warps' states for rows (heads) < G.  The warps' O rows go to the stage of
-    // the item's last tile: the barrier above released it, and the producer refills it only
-    // at the top of the next item, after the barrier that ends this merge.
-    float (*co)[8][64] = reinterpret_cast<float (*)[8][64]>(tiles + ((ct - 1) % DA_STAGES) * 2 * DA_TILE_BYTES);
+    // merge the 4 warps' states for rows (heads) < G
     if (gq < 8) {
       if (tq == 0) {
         cm[warp][gq] = m_run;
@@ -506,32 +524,30 @@ __global__ void __launch_bounds__(DA_THREADS, 4)
       for (int j = 0; j < 8; ++j)
         *reinterpret_cast<float2*>(&co[warp][gq][8 * j + 2 * tq]) = make_float2(o[j][0], o[j][1]);
     }
-    __syncthreads();
-    for (int i = tid; i < G * 64; i += DA_THREADS) {
-      const int hh = i >> 6, d = i & 63;
-      float M = cm[0][hh];
+    da_consumer_sync();
+    if (ok) {
+      for (int i = tid; i < G * 64; i += DA_CONSUMERS) {
+        const int hh = i >> 6, d = i & 63;
+        float M = cm[0][hh];
 #pragma unroll
-      for (int k = 1; k < 4; ++k) M = fmaxf(M, cm[k][hh]);
-      float L = 0.f, O = 0.f;
+        for (int k = 1; k < 4; ++k) M = fmaxf(M, cm[k][hh]);
+        float L = 0.f, O = 0.f;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float wk = cm[k][hh] == -INFINITY ? 0.f : ex2_approx(cm[k][hh] - M);
-        L += wk * cl[k][hh];
-        O += wk * co[k][hh][d];
-      }
-      float* dst = p.part + (((size_t)b * p.Hq + g * G + hh) * p.n_splits + split) * 66;
-      dst[2 + d] = O;
-      if (d == 0) {
-        dst[0] = M;
-        dst[1] = L;
+        for (int k = 0; k < 4; ++k) {
+          const float wk = cm[k][hh] == -INFINITY ? 0.f : ex2_approx(cm[k][hh] - M);
+          L += wk * cl[k][hh];
+          O += wk * co[k][hh][d];
+        }
+        float* dst = p.part + (((size_t)b * p.Hq + g * G + hh) * p.n_splits + split) * 66;
+        dst[2 + d] = O;
+        if (d == 0) {
+          dst[0] = M;
+          dst[1] = L;
+        }
       }
     }
-    fence_proxy_async_smem();   // the O rows were written through the generic proxy; TMA refills the stage
-    __syncthreads();   // cm, cl, co are rewritten by the next item
+    da_consumer_sync();   // cm, cl, co are rewritten by the next item
   }
-  if (!ok && tid == 0)   // let the loads in flight land before the CTA exits
-    for (int j = ct; j < issued; ++j)
-      mbar_wait(&full[j % DA_STAGES], (uint32_t)(j / DA_STAGES) & 1u, nullptr, p.status, 502);
 }
 
 // merge of the decode attention splits: out[b, h*64 + d] = sum_s w_s o_s / sum_s w_s l_s,
