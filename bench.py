@@ -555,6 +555,7 @@ TRAFFIC = {
     "out_proj": 36292864 + 22784,
     "attention": 9816320 + 768,
     "conv1d_silu": 13999616 + 768,
+    "decode_attn": 94806016 + 2965760,
     "decode_prep": 5318912 + 0,
     "decode_ssm": 16947200 + 0,
 }
