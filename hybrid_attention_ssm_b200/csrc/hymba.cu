@@ -445,10 +445,12 @@ int check_cfg(const hymba_layer_cfg* c) {
   if (c->d_state != 16) return fail(HYMBA_ERR_UNSUPPORTED, "d_state %d (only 16)", c->d_state);
   if (c->d_conv != 4) return fail(HYMBA_ERR_UNSUPPORTED, "d_conv %d (only 4)", c->d_conv);
   if (c->d_model < 8 || c->d_model % 8) return fail(HYMBA_ERR_UNSUPPORTED, "d_model %d (multiple of 8)", c->d_model);
-  if (c->d_inner < 64 || c->d_inner % 64 || c->d_inner > 8 * 128 * NORM_MAXY)
-    return fail(HYMBA_ERR_UNSUPPORTED, "d_inner %d (multiple of 64, at most %d)", c->d_inner, 8 * 128 * NORM_MAXY);
-  if (c->n_q_heads * c->head_dim > 8 * 128 * NORM_MAXO)
-    return fail(HYMBA_ERR_UNSUPPORTED, "n_q_heads * head_dim above %d", 8 * 128 * NORM_MAXO);
+  // the branch norm holds a row in registers: 8-element chunks of y, 4-element chunks of O
+  if (c->d_inner < 64 || c->d_inner % 64 || c->d_inner > 8 * NORM_THREADS * NORM_MAXY)
+    return fail(HYMBA_ERR_UNSUPPORTED, "d_inner %d (multiple of 64, at most %d)", c->d_inner,
+                8 * NORM_THREADS * NORM_MAXY);
+  if (c->n_q_heads * c->head_dim > 4 * NORM_THREADS * NORM_MAXO)
+    return fail(HYMBA_ERR_UNSUPPORTED, "n_q_heads * head_dim above %d", 4 * NORM_THREADS * NORM_MAXO);
   if (c->n_q_heads < 1 || c->n_kv_heads < 1 || c->n_q_heads % c->n_kv_heads)
     return fail(HYMBA_ERR_UNSUPPORTED, "heads %d/%d", c->n_q_heads, c->n_kv_heads);
   if (c->n_q_heads / c->n_kv_heads > DEC_MAXG)

@@ -61,9 +61,11 @@ typedef uint16_t hymba_f16;   /* IEEE half bits */
 typedef struct CUstream_st* hymba_stream; /* identical to cudaStream_t; NULL = legacy stream */
 
 /* One mixer layer's sizes ([MC] §模型架构, [JJ] §数学表示).
- * Supported: head_dim 64, d_state 16, d_conv 4, d_model % 8 == 0, d_inner % 64 == 0,
- * n_q_heads % n_kv_heads == 0 with at most 6 query heads per KV head, dt_rank % 4 == 0 and
- * dt_rank + 2*d_state <= 256, window >= 1, n_meta >= 0. */
+ * Supported: head_dim 64, d_state 16, d_conv 4, d_model % 8 == 0, d_inner % 64 == 0 and
+ * d_inner <= 4096, n_q_heads * head_dim <= 2048, n_q_heads % n_kv_heads == 0 with at most 6
+ * query heads per KV head, dt_rank % 4 == 0 and dt_rank + 2*d_state <= 256, window >= 1,
+ * n_meta >= 0.  Anything else is refused with HYMBA_ERR_UNSUPPORTED / HYMBA_ERR_INVALID_ARG
+ * before a kernel is launched. */
 typedef struct hymba_layer_cfg {
   int d_model;     /* d */
   int n_q_heads;   /* Hq */

@@ -54,6 +54,20 @@ def test_invalid_configs_are_rejected(field, value, code):
     assert e.value.code == code
 
 
+def test_size_limits_are_accepted_and_one_step_beyond_rejected():
+    """The widest configuration the kernels take (the GPU parity suite runs it) passes the
+    host checks; one step past any of its limits is refused before anything launches."""
+    lim = synth.workloads()["tiny"].dims.replace(d_model=1024, n_q_heads=32, n_kv_heads=8, d_inner=4096,
+                                                 dt_rank=224, n_meta=8, window=48)
+    assert H.workspace_size(lim, 2, 60) > 0
+    assert H.workspace_size(lim, 2, 69, 0, H.MODE_DECODE) > 0
+    for kw in (dict(d_inner=4096 + 64), dict(n_q_heads=33, n_kv_heads=11), dict(dt_rank=228),
+               dict(n_q_heads=28, n_kv_heads=4)):
+        with pytest.raises(H.HymbaError) as e:
+            H.workspace_size(lim.replace(**kw), 2, 60)
+        assert e.value.code == H.ERR_UNSUPPORTED, kw
+
+
 def test_kv_share_plan_matches_oracle_reading():
     d = synth.workloads()["stack"].dims
     is_global = [1 if i in (0, 15, 31) else 0 for i in range(32)]
