@@ -111,7 +111,7 @@ __device__ __forceinline__ uint8_t* align_smem(uint8_t* raw) {
 }
 
 // ----------------------------------------------------------------------------------------
-// TMA (no multicast anywhere in this library)
+// TMA: every load lands in the issuing CTA's own shared memory
 // ----------------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
   asm volatile(
@@ -126,7 +126,7 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
-// Untiled bulk copy global -> shared (no multicast): both addresses 16-byte aligned, bytes a
+// Untiled bulk copy global -> this CTA's shared memory: both addresses 16-byte aligned, bytes a
 // multiple of 16; completion counted on `bar` as transaction bytes.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"

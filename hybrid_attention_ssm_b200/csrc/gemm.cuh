@@ -10,7 +10,7 @@
 //               column chunks between them (two epilogue warps per SM sub-partition).
 // The accumulator is double-buffered in TMEM so the epilogue of tile i overlaps the
 // mainloop of tile i+1.  The epilogue is a template parameter, so each instance carries
-// only its own code.  No TMA multicast, no clusters.
+// only its own code.  Each CTA loads its own tiles; no thread-block clusters.
 #pragma once
 #include "common.cuh"
 
