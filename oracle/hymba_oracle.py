@@ -20,9 +20,10 @@ All arithmetic is float64 on the given (bf16-rounded) inputs.  Matrix products u
 matmul as a library primitive; nothing is blocked, fused or reordered beyond the
 definitions.
 
-Parity pins: every function here is pinned by tests/test_oracle_pins.py except the RoPE
-pairing convention, the 1/2 of the average, the eps of the RMSNorm and the omitted D skip
-term, which are readings of silent passages (parity unpinned for those choices only).
+Parity pins: every function here, the SwiGLU FFN and the block composition included, is
+pinned by tests/test_oracle_pins.py except the RoPE pairing convention, the 1/2 of the
+average, the eps of the RMSNorm and the omitted D skip term, which are readings of silent
+passages (parity unpinned for those choices only).
 """
 from __future__ import annotations
 

@@ -21,7 +21,7 @@ from tests import test_oracle_pins as pins
 
 ORIG = {name: getattr(orc, name) for name in
         ("selective_scan", "causal_conv1d_silu", "visibility_mask", "attention", "softplus", "ssm_params",
-         "split_in_proj", "rmsnorm", "silu", "rope")}
+         "split_in_proj", "rmsnorm", "silu", "rope", "ffn_swiglu", "hymba_block")}
 
 
 def _pin_calls(golden_dir):
@@ -45,6 +45,9 @@ def _pin_calls(golden_dir):
         ("consumer decode ring", pins.test_consumer_decode_reads_producer_ring, {}),
         ("kv share plan", pins.test_kv_share_plan_hymba_layout, {}),
         ("block residual", pins.test_block_residual_identity, {}),
+        ("ffn hand-derived", pins.test_ffn_swiglu_hand_derived, {"golden_dir": golden_dir}),
+        ("block = its sublayers in order", pins.test_block_is_its_two_sublayers_in_order, {}),
+        ("block pre-norm", pins.test_block_sublayers_read_normalised_stream, {}),
     ]
     for args in [(1, 0, 3), (0, 4, 3), (0, 1, 2), (0, 7, 0)]:
         calls.append((f"attention vs SDPA {args}", pins.test_attention_matches_torch_sdpa,
@@ -118,6 +121,29 @@ def _swap_kv(proj, dims):
     return Q, V, K, xs, z
 
 
+def _ffn_variant(v, bw, swap=False, silu_on_up=False, add=False):
+    v = np.asarray(v, dtype=np.float64)
+    g = v @ np.asarray(bw["w_gate"], dtype=np.float64).T
+    u = v @ np.asarray(bw["w_up"], dtype=np.float64).T
+    if swap:
+        g, u = u, g
+    if silu_on_up:
+        act = g * ORIG["silu"](u)
+    elif add:
+        act = ORIG["silu"](g) + u
+    else:
+        act = ORIG["silu"](g) * u
+    return act @ np.asarray(bw["w_down"], dtype=np.float64).T
+
+
+def _block_variant(dims, w, bw, H, kv_in=None, norm2_on_input=False, no_ffn_residual=False, no_norm1=False):
+    h_in = H if no_norm1 else orc.rmsnorm(H, bw["g_norm1"], dims.norm_eps)
+    r = orc.mixer_prefill(dims, w, h_in, x_has_meta=True, kv_in=kv_in, residual=H)
+    H1 = r["out"]
+    f = orc.ffn_swiglu(orc.rmsnorm(H if norm2_on_input else H1, bw["g_norm2"], dims.norm_eps), bw)
+    return (f if no_ffn_residual else H1 + f), r
+
+
 MISTAKES = {
     "scan: exponent sign flipped": ("selective_scan",
                                     lambda xc, d, A, Bm, Cm, z, h0=None: ORIG["selective_scan"](xc, d, -np.asarray(A), Bm, Cm, z, h0)),
@@ -147,6 +173,14 @@ MISTAKES = {
                                                     * np.asarray(gain, dtype=np.float64)),
     "RMSNorm: gain dropped": ("rmsnorm", lambda v, gain, eps: ORIG["rmsnorm"](v, np.ones_like(np.asarray(gain, dtype=np.float64)), eps)),
     "SiLU replaced by sigmoid": ("silu", lambda x: 1.0 / (1.0 + np.exp(-np.asarray(x, dtype=np.float64)))),
+    "FFN: gate and up swapped": ("ffn_swiglu", lambda v, bw: _ffn_variant(v, bw, swap=True)),
+    "FFN: SiLU applied to the up branch": ("ffn_swiglu", lambda v, bw: _ffn_variant(v, bw, silu_on_up=True)),
+    "FFN: product replaced by a sum": ("ffn_swiglu", lambda v, bw: _ffn_variant(v, bw, add=True)),
+    "block: second norm applied to the block input": (
+        "hymba_block", lambda *a, **k: _block_variant(*a, norm2_on_input=True, **k)),
+    "block: FFN residual dropped": ("hymba_block", lambda *a, **k: _block_variant(*a, no_ffn_residual=True, **k)),
+    "block: mixer reads the un-normalised stream": (
+        "hymba_block", lambda *a, **k: _block_variant(*a, no_norm1=True, **k)),
     "RoPE: angle sign flipped for every other position": (
         "rope", lambda x, positions, base: ORIG["rope"](x, np.asarray(positions) * np.where(np.arange(len(positions)) % 2, -1, 1), base)),
 }

@@ -379,6 +379,54 @@ def test_block_residual_identity():
     np.testing.assert_array_equal(out, H)
 
 
+def test_ffn_swiglu_hand_derived(golden_dir):
+    """SwiGLU on a d = 2, F = 2 case whose SiLU values have closed forms (ln 3 inputs):
+    the gate branch goes through SiLU, the up branch does not, the two multiply, and
+    W_down maps the product back (an asymmetric W_down, so a transposed one fails)."""
+    with open(os.path.join(golden_dir, "ffn_swiglu_closed_form.json")) as f:
+        c = json.load(f)
+    bw = {k: np.array(c[k]) for k in ("w_gate", "w_up", "w_down")}
+    np.testing.assert_allclose(orc.ffn_swiglu(np.array(c["v"]), bw), np.array(c["out"]), rtol=1e-13, atol=1e-15)
+
+
+def _block_case(eps=1e-6):
+    dims = _small_dims(norm_eps=eps)
+    w = _weights(dims)
+    bw = {k: v.astype(np.float64) for k, v in synth.block_weights(dims, 24, seed=3).items()}
+    # FFN weights large enough that its update is far above rounding
+    for k in ("w_gate", "w_up", "w_down"):
+        bw[k] = bw[k] * 25.0
+    return dims, w, bw, _x(1, 8, dims.d_model, seed=4)
+
+
+def test_block_is_its_two_sublayers_in_order():
+    """[JJ] §Hymba 的整体架构: norm -> mixer -> norm -> FFN, each sublayer adding to the
+    residual stream.  The whole block must equal its mixer sublayer alone (FFN output
+    zeroed) followed by its FFN sublayer alone (mixer output zeroed): the FFN reads the
+    stream after the mixer's update, not the block's input."""
+    dims, w, bw, H = _block_case()
+    full, _ = orc.hymba_block(dims, w, bw, H)
+    bw_no_ffn = dict(bw); bw_no_ffn["w_down"] = np.zeros_like(bw["w_down"])
+    w_no_mix = dict(w); w_no_mix["w_out"] = np.zeros_like(w["w_out"])
+    H1, _ = orc.hymba_block(dims, w, bw_no_ffn, H)
+    two_step, _ = orc.hymba_block(dims, w_no_mix, bw, H1)
+    assert np.max(np.abs(H1 - H)) > 1e-3 and np.max(np.abs(two_step - H1)) > 1e-3   # both sublayers act
+    np.testing.assert_allclose(full, two_step, rtol=1e-12, atol=1e-13)
+
+
+def test_block_sublayers_read_normalised_stream():
+    """Pre-norm: each sublayer reads RMSNorm of the stream, so with eps = 0 its update does
+    not change when the stream is scaled by c > 0 (the residual itself scales)."""
+    dims, w, bw, H = _block_case(eps=0.0)
+    bw_no_ffn = dict(bw); bw_no_ffn["w_down"] = np.zeros_like(bw["w_down"])
+    w_no_mix = dict(w); w_no_mix["w_out"] = np.zeros_like(w["w_out"])
+    for ww, bb in ((w, bw_no_ffn), (w_no_mix, bw)):
+        upd1 = orc.hymba_block(dims, ww, bb, H)[0] - H
+        upd7 = orc.hymba_block(dims, ww, bb, 7.5 * H)[0] - 7.5 * H
+        assert np.max(np.abs(upd1)) > 1e-3
+        np.testing.assert_allclose(upd7, upd1, rtol=1e-9, atol=1e-11)
+
+
 def test_tiny_workload_runs_and_is_finite():
     w = synth.layer_weights(TINY.dims, seed=0)
     X = synth.prefill_input(TINY, seed=0)
