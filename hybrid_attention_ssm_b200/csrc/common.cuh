@@ -13,8 +13,9 @@ namespace hymba {
 // device status word (first 256 bytes of every workspace)
 // ----------------------------------------------------------------------------------------
 enum : unsigned {
-  DEV_ERR_TIMEOUT = 1u,   // a bounded wait gave up
-  DEV_ERR_BOUNDS = 2u,    // an index check failed and the access was skipped
+  DEV_ERR_TIMEOUT = 1u,     // a bounded wait gave up
+  DEV_ERR_BOUNDS = 2u,      // an index check failed and the access was skipped
+  DEV_ERR_FP16_RANGE = 4u,  // a value stored as fp16 had |v| >= 65520 and became +-inf
 };
 
 struct DevStatus {
@@ -31,6 +32,16 @@ __device__ __forceinline__ void report_error(DevStatus* st, unsigned flag, unsig
     atomicOr(&st->flags, flag);
     atomicExch(&st->site, site);
   }
+}
+
+// Values that fp16 cannot hold: |v| >= 65520 rounds to +-inf (the largest finite fp16 is
+// 65504).  Checked before a store to fp16, recorded in the status word; the store proceeds.
+template <int N>
+__device__ __forceinline__ void f16_range_guard(const float* v, DevStatus* st, unsigned site) {
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < N; ++i) m = fmaxf(m, fabsf(v[i]));
+  if (m >= 65520.f) report_error(st, DEV_ERR_FP16_RANGE, site);
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

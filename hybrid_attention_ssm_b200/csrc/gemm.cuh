@@ -20,7 +20,7 @@ enum EpiMode : int {
   EPI_PROJ = 0,         // segmented bf16/fp16 stores with RoPE on marked segments (in_proj)
   EPI_BF16 = 1,         // bf16 store, optional bf16 residual add
   EPI_SWIGLU = 2,       // columns interleaved [gate(32) | up(32)] -> fp16 SiLU(gate)*up
-  EPI_SOFTPLUS_T = 3,   // fp32 softplus(acc + bias[col]) stored time-major: out[(b*N + col)*T_out + row]
+  EPI_SOFTPLUS = 3,     // fp32 softplus(acc + bias[col]), row-major: out[row * ld_out + col]
   EPI_F32_T = 4,        // transposed fp32 store: out[n][m] (weights as the M operand)
   EPI_F32_PART = 5,     // fp32 store of split ks's partial sum at out + ks*split_stride (row-major)
   EPI_F32_T_PART = 6,   // the same, transposed
@@ -69,13 +69,20 @@ constexpr int GEMM_EPI_WARPS = 8;
 constexpr int GEMM_THREADS = 64 + 32 * GEMM_EPI_WARPS;
 constexpr int GEMM_BM = 128;
 
-template <int BN, int STAGES>
+// Shared memory an epilogue stages its output through: EPI_SOFTPLUS transposes each warp's
+// 32 x 32 fp32 block (rows padded to 33 words) so that every store writes one whole row.
+__host__ __device__ constexpr int gemm_epi_bytes(int mode) {
+  return mode == 3 /* EPI_SOFTPLUS */ ? GEMM_EPI_WARPS * 32 * 33 * 4 : 0;
+}
+
+template <int BN, int STAGES, int EPI_BYTES = 0>
 struct GemmSmem {
   static constexpr int A_BYTES = GEMM_BM * 128;
   static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
-  static constexpr int TOTAL = BAR_OFFSET + 256 + 1024;   // + barriers + alignment slack
+  static constexpr int EPI_OFFSET = BAR_OFFSET + 256;
+  static constexpr int TOTAL = EPI_OFFSET + EPI_BYTES + 1024;   // + barriers, staging, alignment slack
 };
 
 // Rotate the pairs (v[j], v[j+32]) of one 64-wide head by the angles of position pos.
@@ -134,7 +141,8 @@ template <int BN, int STAGES, int ET, int MODE>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA0, const __grid_constant__ CUtensorMap mapA1,
                    const __grid_constant__ CUtensorMap mapB, const __grid_constant__ GemmParams p) {
-  using L = GemmSmem<BN, STAGES>;
+  using L = GemmSmem<BN, STAGES, gemm_epi_bytes(MODE)>;
+  static_assert(L::TOTAL <= 232448, "shared memory of one CTA");
   constexpr int ACC_STRIDE = BN <= 128 ? 128 : 256;       // TMEM columns per accumulator
   constexpr uint32_t TMEM_COLS = 2 * ACC_STRIDE;
   constexpr bool TF32 = ET == ET_TF32;
@@ -304,6 +312,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           if constexpr (MODE == EPI_SWIGLU) {   // fp16 activations (the down projection runs in fp16)
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = silu_f(v[e]) * v[e + 32];
+            f16_range_guard<32>(v, p.status, 121);
             store_f16_row(reinterpret_cast<__half*>(p.out) + orow * p.ld_out + gc / 2, v, 32);
           } else {
             int si = 0;
@@ -312,6 +321,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             const Segment& sg = p.seg[si];
             const int pos = src0 ? rr : p.row_off1 + rr;
             if (sg.rope) rope_pair_rotate(v, p.rope_tab + (size_t)pos * 32);
+            if (sg.f16) f16_range_guard<64>(v, p.status, 120);
             __nv_bfloat16* base = reinterpret_cast<__nv_bfloat16*>(sg.ptr) + (gc - sg.col_begin);
             const int b_lo = src0 ? 0 : b1, b_hi = src0 ? p.out_batches : b1 + 1;
             for (int b = b_lo; b < b_hi; ++b) {
@@ -350,6 +360,24 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             }
             return;
           }
+          if constexpr (MODE == EPI_SOFTPLUS) {
+            // softplus(acc + bias) of the warp's 32 rows x 32 columns, transposed through this
+            // warp's shared tile: lane j then stores column gc + j of row r, 128-byte rows
+            if (gc >= p.n_valid) return;          // the same for the whole warp
+            float* tile = reinterpret_cast<float*>(smem + L::EPI_OFFSET) + (warp - 2) * (32 * 33);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) tile[lane * 33 + e] = softplus_sel(v[e] + p.bias[min(gc + e, p.n_valid - 1)]);
+            __syncwarp();
+            const int rows_valid = src0 ? p.rows0 : p.rows1;
+            const int rr0 = rr - lane;            // accumulator row of lane 0
+            const bool col_ok = gc + lane < p.n_valid;
+            float* dst = reinterpret_cast<float*>(p.out) + ((size_t)b1 * p.rows1 + rr0) * p.ld_out + gc + lane;
+#pragma unroll 4
+            for (int q = 0; q < 32; ++q)
+              if (rr0 + q < rows_valid && col_ok) dst[(size_t)q * p.ld_out] = tile[q * 33 + lane];
+            __syncwarp();
+            return;
+          }
           if (!row_ok || gc >= p.n_valid) return;
           const bool whole = gc + 32 <= p.n_valid;
           if constexpr (MODE == EPI_BF16) {
@@ -383,28 +411,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             for (int e = 0; e < 32; e += 4)
               if (gc + e < p.n_valid)
                 *reinterpret_cast<float4*>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-          } else {  // EPI_SOFTPLUS_T: lanes hold consecutive rows -> coalesced along time
-            float bb[32];
-            if (whole) {
-#pragma unroll
-              for (int e = 0; e < 32; e += 4) {
-                const float4 t = *reinterpret_cast<const float4*>(p.bias + gc + e);
-                bb[e] = t.x; bb[e + 1] = t.y; bb[e + 2] = t.z; bb[e + 3] = t.w;
-              }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 32; ++e) bb[e] = (gc + e < p.n_valid) ? p.bias[gc + e] : 0.f;
-            }
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = softplus_sel(v[e] + bb[e]);
-            float* dst = reinterpret_cast<float*>(p.out) + ((size_t)b1 * p.N + gc) * p.T_out + rr;
-            if (whole) {
-#pragma unroll
-              for (int e = 0; e < 32; ++e) dst[(size_t)e * p.T_out] = v[e];
-            } else {
-              for (int e = 0; e < 32; ++e)
-                if (gc + e < p.n_valid) dst[(size_t)e * p.T_out] = v[e];
-            }
           }
         };
         uint32_t ra[32], rb[32];

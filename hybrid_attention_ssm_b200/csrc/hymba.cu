@@ -237,7 +237,7 @@ int launch_gemm_inst(const CUtensorMap& m0, const CUtensorMap& m1, const CUtenso
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
-  constexpr int smem = GemmSmem<BN, STAGES>::TOTAL;
+  constexpr int smem = GemmSmem<BN, STAGES, gemm_epi_bytes(MODE)>::TOTAL;
   auto kern = gemm_tc_kernel<BN, STAGES, ET, MODE>;
   if (!attr_set[dev & 63]) {
     HY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
@@ -254,6 +254,10 @@ template <int ET, int MODE>
 int launch_gemm_bn(int bn, const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& mb, const GemmParams& p,
                    int grid, cudaStream_t st, const char* name) {
   constexpr bool any_bn = MODE == EPI_F32_PART || MODE == EPI_F32_T || MODE == EPI_F32_T_PART;
+  if constexpr (MODE == EPI_SOFTPLUS) {   // short K (dt_rank): 4 stages, room for the staging tiles
+    if (bn == 128) return launch_gemm_inst<128, 4, ET, MODE>(m0, m1, mb, p, grid, st, name);
+    return fail(HYMBA_ERR_UNSUPPORTED, "no GEMM instance for tile width %d with the softplus epilogue", bn);
+  }
   if (bn == 256) return launch_gemm_inst<256, 4, ET, MODE>(m0, m1, mb, p, grid, st, name);
   if constexpr (MODE != EPI_PROJ) {
     if (bn == 128) return launch_gemm_inst<128, 6, ET, MODE>(m0, m1, mb, p, grid, st, name);
@@ -284,8 +288,8 @@ int launch_gemm_mode(const GemmCall& c, const CUtensorMap& m0, const CUtensorMap
     case EPI_SWIGLU:
       if (c.etype == ET_BF16) return launch_gemm_bn<ET_BF16, EPI_SWIGLU>(c.bn, m0, m1, mb, p, grid, st, c.name);
       break;
-    case EPI_SOFTPLUS_T:
-      if (c.etype == ET_TF32) return launch_gemm_bn<ET_TF32, EPI_SOFTPLUS_T>(c.bn, m0, m1, mb, p, grid, st, c.name);
+    case EPI_SOFTPLUS:
+      if (c.etype == ET_TF32) return launch_gemm_bn<ET_TF32, EPI_SOFTPLUS>(c.bn, m0, m1, mb, p, grid, st, c.name);
       break;
     case EPI_F32_T:
       if (c.etype == ET_BF16) return launch_gemm_bn<ET_BF16, EPI_F32_T>(c.bn, m0, m1, mb, p, grid, st, c.name);
@@ -406,14 +410,6 @@ int pick_bn_cover(int n) {
   if (n <= 160) return 160;
   return 256;
 }
-// Tile width for an epilogue-bound GEMM (a short K and a heavy epilogue): the one that
-// gives the busiest SM the fewest accumulator columns, (rounds of the persistent grid) x
-// width; the narrower wins a tie (its next tile's MMAs overlap the epilogue sooner).
-int pick_bn_epilogue(int m_tiles, int N, int sms) {
-  const long long r128 = ((long long)m_tiles * cdiv(N, 128) + sms - 1) / sms;
-  const long long r256 = ((long long)m_tiles * cdiv(N, 256) + sms - 1) / sms;
-  return r256 * 256 < r128 * 128 ? 256 : 128;
-}
 // Tile width among `cands` minimising (rounds of the persistent grid) x (operand bytes per
 // k-block): the mainloops run at the rate shared memory is fed, so a round of tiles costs
 // k_blocks times those bytes whether or not every SM has a tile.
@@ -495,25 +491,43 @@ int splits_for(int tiles, int k_blocks, int cap) {
 }
 
 struct PrefillWs {
-  size_t q, xz, xc, xcT, xbc, xbc_part, bcT, dT, y, o, u, sstate, cstate, rope, total;
-  int T, Tp, xproj_split;
+  size_t q, xz, xc, xbc, xbc_part, delta, carry, sumd, y, o, u, sstate, cstate, rope, total;
+  int T, xproj_split, scan_L, scan_chunks;
 };
+// Time chunks of the selective scan.  Every chunk of a pass runs at once: the CTAs of the
+// output pass, (Di / 64) x n_chunks x B, must fit in one wave of a B200's 148 SMs, else a
+// second wave doubles the time of the serial walk over a chunk.  An SM holds 10 scan CTAs
+// (registers), 8 beside the attention CTA when the two branches overlap (small batch, as
+// the prefill decides).  Within that, as many chunks as fit: shorter chunks, shorter walk.
+// Fixed to 148 SMs so that workspace sizes do not depend on the device; the chunk length
+// is a multiple of the scan's TMA stage.
+void scan_chunking(int B, int Di, int T, int* L, int* n_chunks) {
+  const long long per_sm = (long long)B * Di < 24LL * 148 ? 8 : 10;
+  const long long groups = (long long)B * (Di / SC_CH);
+  long long c = 148LL * per_sm / groups;
+  const long long cmax = (T + SC_SUB - 1) / SC_SUB;
+  if (c > cmax) c = cmax;
+  if (c < 1) c = 1;
+  const int len = SC_SUB * cdiv(cdiv(T, c), SC_SUB);
+  *L = len;
+  *n_chunks = cdiv(T, len);
+}
 PrefillWs prefill_layout(const Dims& m, int B, int n_tokens, int x_has_meta) {
   PrefillWs w;
   w.T = x_has_meta ? n_tokens : m.M + n_tokens;
-  w.Tp = (w.T + 7) & ~7;
+  scan_chunking(B, m.Di, w.T, &w.scan_L, &w.scan_chunks);
   const size_t rows = (size_t)B * w.T;
   size_t off = 256;
   auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
   w.q = take(rows * m.qw * 2);
   w.xz = take(rows * 2 * m.Di * 2);
   w.xc = take(rows * m.Di * 2);
-  w.xcT = take((size_t)B * m.Di * w.Tp * 2);
   w.xbc = take(rows * m.ld_xbc * 4);
   w.xproj_split = splits_for(cdiv((long long)rows, GEMM_BM), cdiv(m.Di, 64), 16);
   w.xbc_part = take((size_t)w.xproj_split * rows * m.ld_xbc * 4);
-  w.bcT = take((size_t)B * 32 * w.Tp * 4);
-  w.dT = take((size_t)B * m.Di * w.Tp * 4);
+  w.delta = take(rows * m.Di * 4);
+  w.carry = take((size_t)B * (w.scan_chunks - 1) * m.Di * 16 * 4);
+  w.sumd = take((size_t)B * (w.scan_chunks - 1) * m.Di * 4);
   w.y = take(rows * m.Di * 2);
   w.o = take(rows * m.qw * 4);
   w.u = take(rows * m.uw * 2);
@@ -522,6 +536,20 @@ PrefillWs prefill_layout(const Dims& m, int B, int n_tokens, int x_has_meta) {
   w.rope = take((size_t)w.T * 32 * 8);
   w.total = off;
   return w;
+}
+
+// Device copies of a host prefill's input and output, after the prefill's own workspace.
+struct HostStaging {
+  size_t x, out, x_bytes, out_bytes, total;
+};
+HostStaging host_staging(const PrefillWs& L, const Dims& m, int B, int n_tokens) {
+  HostStaging h;
+  h.x_bytes = (size_t)B * n_tokens * m.d * 2;
+  h.out_bytes = (size_t)B * L.T * m.d * 2;
+  h.x = align256(L.total);
+  h.out = align256(h.x + h.x_bytes);
+  h.total = align256(h.out + h.out_bytes);
+  return h;
 }
 
 struct DecodeWs {
@@ -647,9 +675,10 @@ int hymba_mixer_workspace_size(const hymba_layer_cfg* cfg, int batch, int n_toke
   HY_TRY(check_cfg(cfg));
   if (bytes == nullptr || batch < 1) return fail(HYMBA_ERR_INVALID_ARG, "bytes NULL or batch < 1");
   const Dims m = dims_of(cfg);
-  if (mode == HYMBA_MODE_PREFILL) {
+  if (mode == HYMBA_MODE_PREFILL || mode == HYMBA_MODE_PREFILL_HOST) {
     if (n_tokens < 1) return fail(HYMBA_ERR_INVALID_ARG, "n_tokens < 1");
-    *bytes = prefill_layout(m, batch, n_tokens, x_has_meta).total;
+    const PrefillWs L = prefill_layout(m, batch, n_tokens, x_has_meta);
+    *bytes = mode == HYMBA_MODE_PREFILL ? L.total : host_staging(L, m, batch, n_tokens).total;
   } else if (mode == HYMBA_MODE_DECODE) {
     // for a global layer n_tokens is the cache's max_tokens (keys read per step)
     const int mk = cfg->is_global ? (n_tokens > 0 ? n_tokens : 1) : decode_max_keys(cfg, 0);
@@ -666,10 +695,27 @@ int hymba_mixer_stage_layout(const hymba_layer_cfg* cfg, int batch, int n_tokens
   if (out == nullptr || batch < 1 || n_tokens < 1) return fail(HYMBA_ERR_INVALID_ARG, "stage layout args");
   const Dims m = dims_of(cfg);
   const PrefillWs w = prefill_layout(m, batch, n_tokens, x_has_meta);
-  out->q = w.q; out->xz = w.xz; out->xc = w.xc; out->xbc = w.xbc; out->delta = w.dT;
+  out->q = w.q; out->xz = w.xz; out->xc = w.xc; out->xbc = w.xbc; out->delta = w.delta;
   out->y = w.y; out->o = w.o; out->u = w.u;
   out->ld_xbc = m.ld_xbc;
-  out->Tp = w.Tp;
+  out->scan_chunks = w.scan_chunks;
+  out->scan_chunk_len = w.scan_L;
+  return HYMBA_OK;
+}
+
+int hymba_decode_stage_layout(const hymba_layer_cfg* cfg, int batch, int max_tokens, hymba_decode_stages* out) {
+  HY_TRY(check_cfg(cfg));
+  if (out == nullptr || batch < 1) return fail(HYMBA_ERR_INVALID_ARG, "decode stage layout args");
+  const Dims m = dims_of(cfg);
+  const int mk = cfg->is_global ? (max_tokens > 0 ? max_tokens : 1) : decode_max_keys(cfg, 0);
+  const DecodeWs w = decode_layout(m, batch, cfg->is_global != 0, mk);
+  out->proj = w.proj; out->xc = w.xc; out->xbc_part = w.xbc_part; out->y = w.y;
+  out->proj_slice_stride = (long long)batch * m.P;
+  out->xbc_slice_stride = (long long)batch * m.ld_xbc;
+  out->in_split = w.in_split;
+  out->xproj_split = w.xproj_split;
+  out->ld_proj = m.P;
+  out->ld_xbc = m.ld_xbc;
   return HYMBA_OK;
 }
 
@@ -686,7 +732,10 @@ int hymba_status_read(void* ws, hymba_stream stream, int* status) {
   HY_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
   HY_CUDA(cudaMemcpy(&h, ws, sizeof(unsigned) * 2, cudaMemcpyDeviceToHost));
   HY_CUDA(cudaMemset(ws, 0, 256));
-  *status = (h.flags & DEV_ERR_TIMEOUT) ? HYMBA_ERR_TIMEOUT : HYMBA_OK;
+  *status = (h.flags & DEV_ERR_TIMEOUT)      ? HYMBA_ERR_TIMEOUT
+            : (h.flags & DEV_ERR_FP16_RANGE) ? HYMBA_ERR_FP16_RANGE
+            : (h.flags & DEV_ERR_BOUNDS)     ? HYMBA_ERR_INVALID_ARG
+                                             : HYMBA_OK;
   if (h.flags != 0) fail(*status, "device status flags 0x%x at site %u", h.flags, h.site);
   return HYMBA_OK;
 }
@@ -866,7 +915,7 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     dim3 grid(m.Di / CONV_TC, cdiv(T, CONV_TT), B);
     prof_begin("conv1d_silu", st);
     HY_CUDA(launch_pdl(conv1d_silu_kernel, grid, dim3(256), 0, st, bf(L.xz), 2 * m.Di, w->conv_w, w->conv_b, bf(L.xc),
-                       bf(L.xcT), cstate, T, L.Tp, m.Di));
+                       cstate, T, m.Di));
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
@@ -887,33 +936,33 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     HY_TRY(run_gemm(c, *dev, st));
     const int n = (int)(rows * m.ld_xbc);
     prof_begin("splitk_reduce", st);
-    HY_CUDA(launch_pdl(splitk_reduce_kernel, dim3(cdiv(n / 4, 256)), dim3(256), 0, st, f32(L.xbc_part), L.xproj_split, (long long)n, n,
-                                                            nullptr, f32(L.xbc), 0, h16(L.bcT), m.ld_xbc, T, L.Tp,
-                                                            m.R));
+    HY_CUDA(launch_pdl(splitk_reduce_kernel, dim3(cdiv(n / 4, 256)), dim3(256), 0, st, f32(L.xbc_part),
+                       L.xproj_split, (long long)n, n, nullptr, f32(L.xbc), 0));
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
-  // 4. dt_proj (tf32) with softplus(+bias), stored time-major
+  // 4. dt_proj (tf32) with softplus(+bias): delta [B*T, Di] fp32
   {
     GemmCall c;
     c.etype = ET_TF32;
     c.a1 = f32(L.xbc); c.nb1 = B; c.rows1 = T; c.lda1 = m.ld_xbc; c.a1_bstride = (long long)T * m.ld_xbc;
     c.b = w->w_dt; c.N = m.Di; c.ldb = w->w_dt_ld; c.K = m.R;
-    c.bn = pick_bn_epilogue(B * cdiv(T, GEMM_BM), m.Di, dev->sms);
+    c.bn = 128;
     c.name = "dt_proj";
-    c.mode = EPI_SOFTPLUS_T;
-    c.p.out = f32(L.dT);
-    c.p.T_out = L.Tp;
+    c.mode = EPI_SOFTPLUS;
+    c.p.out = f32(L.delta);
+    c.p.ld_out = m.Di;
     c.p.bias = w->dt_bias;
     c.p.n_valid = m.Di;
     c.p.status = status;
     HY_TRY(run_gemm(c, *dev, st));
   }
-  // 5. attention (block-skipped SWA + meta, or global causal).  When the scan alone cannot
-  //    fill the GPU (fewer than three of its CTAs per SM), the attention forks onto the side
-  //    stream after dt_proj and runs beside the scan: both are latency-bound and fit on one
-  //    SM together (one attention CTA, three scan CTAs).  Otherwise it runs in stream order.
-  const bool overlap = (long long)B * (m.Di / SCAN_CH) < 3LL * dev->sms;
+  // 5. attention (block-skipped SWA + meta, or global causal).  At small batch (fewer than
+  //    24 channels x sequences per SM) the attention forks onto the side stream after dt_proj
+  //    and runs beside the scan: both leave most of an SM's issue slots idle at that size and
+  //    fit on one SM together (one 2-stage attention CTA beside the scan's small CTAs).
+  //    Otherwise it runs in stream order.
+  const bool overlap = (long long)B * m.Di < 24LL * dev->sms;
   ForkGuard fork_guard(side, st);
   if (overlap) {
     HY_CUDA(cudaEventRecord(side->fork, st));
@@ -949,40 +998,59 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     }
     if (overlap) HY_CUDA(cudaEventRecord(side->join, side->s));
   }
-  // 6. selective scan
+  // 6. selective scan in time chunks: chunk end states, carry, outputs
   float* sstate = ssm_state_out != nullptr ? ssm_state_out : f32(L.sstate);
   {
-    // time-major inputs through tensor maps of extent T (zero fill past the last step)
+    // row-major inputs through tensor maps of B*T rows (zero fill past the last row)
     CUtensorMap md, mx, mbc;
     {
-      const uint64_t dims[2] = {(uint64_t)T, (uint64_t)B * m.Di};
-      const uint64_t str[1] = {(uint64_t)L.Tp * 4};
-      const uint32_t box[2] = {SCAN_TC, SCAN_CH};
-      HY_TRY(make_map(&md, f32(L.dT), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE));
+      const uint64_t dims[2] = {(uint64_t)m.Di, (uint64_t)rows};
+      const uint64_t str[1] = {(uint64_t)m.Di * 4};
+      const uint32_t box[2] = {SC_CH, SC_SUB};
+      HY_TRY(make_map(&md, f32(L.delta), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE));
     }
     {
-      const uint64_t dims[2] = {(uint64_t)T, (uint64_t)B * m.Di};
-      const uint64_t str[1] = {(uint64_t)L.Tp * 2};
-      const uint32_t box[2] = {SCAN_TC, SCAN_CH};
-      HY_TRY(make_map(&mx, bf(L.xcT), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE));
+      const uint64_t dims[2] = {(uint64_t)m.Di, (uint64_t)rows};
+      const uint64_t str[1] = {(uint64_t)m.Di * 2};
+      const uint32_t box[2] = {SC_CH, SC_SUB};
+      HY_TRY(make_map(&mx, bf(L.xc), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE));
     }
-    {   // (B_s, C_s) fp16 pairs moved as 32-bit elements
-      const uint64_t dims[2] = {(uint64_t)T, (uint64_t)B * 16};
-      const uint64_t str[1] = {(uint64_t)L.Tp * 4};
-      const uint32_t box[2] = {SCAN_BCW, 16};
-      HY_TRY(make_map(&mbc, f32(L.bcT), CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE));
+    {   // the B | C columns of the x_proj output (column offset dt_rank, a multiple of 4)
+      const uint64_t dims[2] = {32, (uint64_t)rows};
+      const uint64_t str[1] = {(uint64_t)m.ld_xbc * 4};
+      const uint32_t box[2] = {32, SC_SUB};
+      HY_TRY(make_map(&mbc, f32(L.xbc) + m.R, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, dims, str, box,
+                      CU_TENSOR_MAP_SWIZZLE_NONE));
     }
-    dim3 grid(m.Di / SCAN_CH, B);
+    ScanParams sp;
+    sp.T = T; sp.Di = m.Di; sp.L = L.scan_L; sp.n_chunks = L.scan_chunks;
+    sp.A = w->A;
+    sp.carry = f32(L.carry);
+    sp.sumd = f32(L.sumd);
+    sp.y = bf(L.y);
+    sp.state = sstate;
+    sp.status = status;
     static bool attr_scan[64] = {false};
     int dcur = 0;
     cudaGetDevice(&dcur);
     if (!attr_scan[dcur & 63]) {
-      HY_CUDA(cudaFuncSetAttribute(selective_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM));
+      HY_CUDA(cudaFuncSetAttribute(scan_chunk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SC_SMEM));
+      HY_CUDA(cudaFuncSetAttribute(scan_chunk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SC_SMEM));
       attr_scan[dcur & 63] = true;
     }
+    if (L.scan_chunks > 1) {
+      prof_begin("scan_chunk_end", st);
+      HY_CUDA(launch_pdl(scan_chunk_kernel<false>, dim3(m.Di / SC_CH, L.scan_chunks - 1, B), dim3(SC_THREADS), SC_SMEM,
+                         st, md, mx, mbc, sp));
+      prof_end(st);
+      const long long n = (long long)B * m.Di * 16;
+      prof_begin("scan_carry", st);
+      HY_CUDA(launch_pdl(scan_carry_kernel, dim3(cdiv(n, 256)), dim3(256), 0, st, sp, B));
+      prof_end(st);
+    }
     prof_begin("selective_scan", st);
-    HY_CUDA(launch_pdl(selective_scan_kernel, grid, dim3(SCAN_THREADS), SCAN_SMEM, st, md, mx, mbc, w->A, bf(L.y),
-                       sstate, T, m.Di, status));
+    HY_CUDA(launch_pdl(scan_chunk_kernel<true>, dim3(m.Di / SC_CH, L.scan_chunks, B), dim3(SC_THREADS), SC_SMEM, st,
+                       md, mx, mbc, sp));
     prof_end(st);
   }
   // 7. per-branch RMSNorm, gate, beta, average (the attention branch joins here)
@@ -1018,9 +1086,33 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
   return HYMBA_OK;
 }
 
-int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x, int B,
-                       int position, hymba_kv_cache* kv, float* ssm_state, float* conv_state,
-                       const hymba_bf16* residual, hymba_bf16* out, void* ws, size_t ws_bytes,
+int hymba_mixer_prefill_host(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x_host,
+                             int x_has_meta, int B, int n_tokens, hymba_kv_cache* kv, float* ssm_state_out,
+                             float* conv_state_out, hymba_bf16* out_host, void* ws, size_t ws_bytes,
+                             hymba_stream stream) {
+  HY_TRY(check_cfg(cfg));
+  if (x_host == nullptr || out_host == nullptr || B < 1 || n_tokens < 1)
+    return fail(HYMBA_ERR_INVALID_ARG, "x_host/out_host NULL, batch or n_tokens < 1");
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return fail(HYMBA_ERR_INVALID_ARG, "workspace");
+  const Dims m = dims_of(cfg);
+  const PrefillWs L = prefill_layout(m, B, n_tokens, x_has_meta);
+  const HostStaging h = host_staging(L, m, B, n_tokens);
+  if (ws_bytes < h.total) return fail(HYMBA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, h.total);
+  const cudaStream_t st = (cudaStream_t)stream;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  HY_CUDA(cudaMemcpyAsync(wsb + h.x, x_host, h.x_bytes, cudaMemcpyHostToDevice, st));
+  HY_TRY(hymba_mixer_prefill(cfg, w, reinterpret_cast<const hymba_bf16*>(wsb + h.x), x_has_meta, B, n_tokens, kv,
+                             ssm_state_out, conv_state_out, nullptr, reinterpret_cast<hymba_bf16*>(wsb + h.out), ws,
+                             L.total, stream));
+  HY_CUDA(cudaMemcpyAsync(out_host, wsb + h.out, h.out_bytes, cudaMemcpyDeviceToHost, st));
+  return HYMBA_OK;
+}
+
+// The decode step; positions == NULL: every sequence at `position`; otherwise sequence b at
+// positions[b] (device memory), each <= `position`, which sizes the attention's key splits.
+static int decode_impl(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x, int B,
+                       int position, const int* positions, hymba_kv_cache* kv, float* ssm_state,
+                       float* conv_state, const hymba_bf16* residual, hymba_bf16* out, void* ws, size_t ws_bytes,
                        hymba_stream stream) {
   HY_TRY(check_cfg(cfg));
   DeviceInfo* dev = nullptr;
@@ -1088,12 +1180,15 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     pp.conv_state = conv_state;
     pp.xc = bf(L.xc);
     pp.Hq = m.Hq; pp.Hkv = m.Hkv; pp.p = position; pp.write_kv = own_kv ? 1 : 0;
+    pp.positions = positions;
+    pp.max_position = position;
     pp.is_global = global ? 1 : 0; pp.M = m.M; pp.W = m.W; pp.Lmax = kv->max_tokens;
     pp.ring_k = reinterpret_cast<__half*>(kv->ring_k);
     pp.ring_v = reinterpret_cast<__half*>(kv->ring_v);
     pp.full_k = reinterpret_cast<__half*>(kv->k);
     pp.full_v = reinterpret_cast<__half*>(kv->v);
     pp.qrot = f32(L.qrot);
+    pp.status = status;
     pp.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)m.D));
     fill_rope_theta(pp.rope_theta, cfg->rope_base);
     const int n_rope = B * (m.Hq + (own_kv ? m.Hkv : 0)) * 32;
@@ -1144,6 +1239,9 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
         mmv = mv;
       }
     }
+    ap.positions = positions;
+    ap.W = m.W;
+    ap.max_position = position;
     ap.n_tiles = ap.n_meta_tiles + cdiv(ap.n_main_valid, DA_KT);
     ap.n_splits = cdiv(ap.n_tiles, DA_TPS);
     if (ap.n_splits > L.n_splits) return fail(HYMBA_ERR_WORKSPACE, "decode workspace sized for fewer keys");
@@ -1230,11 +1328,29 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     const int n = B * m.d;
     prof_begin("decode_out_store", st);
     HY_CUDA(launch_pdl(splitk_reduce_kernel, dim3(cdiv(n / 4, 256)), dim3(256), 0, st, f32(L.acc_part), L.oproj_split, (long long)n, n,
-                                                            reinterpret_cast<const __nv_bfloat16*>(residual), out, 1, (__half*)nullptr, 0, 0, 0, 0));
+                                                            reinterpret_cast<const __nv_bfloat16*>(residual), out, 1));
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
   return HYMBA_OK;
+}
+
+int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x, int B,
+                       int position, hymba_kv_cache* kv, float* ssm_state, float* conv_state,
+                       const hymba_bf16* residual, hymba_bf16* out, void* ws, size_t ws_bytes,
+                       hymba_stream stream) {
+  return decode_impl(cfg, w, x, B, position, nullptr, kv, ssm_state, conv_state, residual, out, ws, ws_bytes,
+                     stream);
+}
+
+int hymba_mixer_decode_ragged(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x, int B,
+                              const int* positions, int max_position, hymba_kv_cache* kv, float* ssm_state,
+                              float* conv_state, const hymba_bf16* residual, hymba_bf16* out, void* ws,
+                              size_t ws_bytes, hymba_stream stream) {
+  if (positions == nullptr || (reinterpret_cast<uintptr_t>(positions) & 3u))
+    return fail(HYMBA_ERR_INVALID_ARG, "positions pointer NULL or not 4-byte aligned");
+  return decode_impl(cfg, w, x, B, max_position, positions, kv, ssm_state, conv_state, residual, out, ws,
+                     ws_bytes, stream);
 }
 
 int hymba_gemm_bf16(const hymba_bf16* A, const hymba_bf16* Bm, const hymba_bf16* residual, hymba_bf16* C, int M,
@@ -1343,10 +1459,9 @@ int hymba_selftest_wait_timeout(void* ws, size_t ws_bytes, hymba_stream stream) 
 // Decode step without a caller-provided workspace.
 //
 // Some callers cannot allocate device memory at the point where they run a decode step:
-// code inside a region that is being captured into a CUDA graph (cudaMalloc is not a
-// capturable stream operation), serving loops that must not hit cudaMalloc's implicit
-// device synchronisation between tokens, and plugins whose host runtime owns every device
-// allocation and hands them only inputs and outputs.  For them the scratch memory of the
+// serving loops that must not hit cudaMalloc's implicit device synchronisation between
+// tokens, and plugins whose host runtime owns every device allocation and hands them only
+// inputs and outputs.  For them the scratch memory of the
 // decode step lives in this file-scope device array instead of a workspace argument.
 // ========================================================================================
 namespace {

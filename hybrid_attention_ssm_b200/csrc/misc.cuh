@@ -223,9 +223,12 @@ struct DecPrepParams {
   float* conv_state;
   __nv_bfloat16* xc;
   int Hq, Hkv, p, write_kv, is_global, M, W, Lmax;
+  const int* positions;       // per-sequence positions [B] (device), or NULL: every sequence at p
+  int max_position;           // with positions: the caller's bound on them
   __half *ring_k, *ring_v, *full_k, *full_v;
   float* qrot;
   float scale_log2;
+  DevStatus* status;
   double rope_theta[32];
 };
 
@@ -251,8 +254,17 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(const __grid_constant_
   const int i = (blockIdx.x - p.conv_blocks) * 256 + threadIdx.x;
   if (i >= p.B * n_heads * 32) return;
   const int j = i & 31, hh = (i >> 5) % n_heads, b = (i >> 5) / n_heads;
-  // angle p * theta_j reduced mod 2 pi in double precision, then the fp32 sincos
-  double a = (double)p.p * p.rope_theta[j];
+  int pos = p.p;
+  if (p.positions != nullptr) {
+    pos = p.positions[b];
+    // a position the cache cannot hold: record it and leave this sequence's cache alone
+    if (pos < p.M || pos > p.max_position || (p.is_global && pos >= p.Lmax)) {
+      if (j == 0) report_error(p.status, DEV_ERR_BOUNDS, 232);
+      return;
+    }
+  }
+  // angle pos * theta_j reduced mod 2 pi in double precision, then the fp32 sincos
+  double a = (double)pos * p.rope_theta[j];
   a -= 6.283185307179586 * rint(a * 0.15915494309189535);
   float sn, cs;
   sincosf((float)a, &sn, &cs);
@@ -261,8 +273,10 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(const __grid_constant_
   if (hh < p.Hq) {
     const float x1 = P(hh * 64 + j), x2 = P(hh * 64 + j + 32);
     float* q = p.qrot + ((size_t)b * p.Hq + hh) * 64;
-    q[j] = (x1 * cs - x2 * sn) * p.scale_log2;
-    q[j + 32] = (x2 * cs + x1 * sn) * p.scale_log2;
+    const float qv[2] = {(x1 * cs - x2 * sn) * p.scale_log2, (x2 * cs + x1 * sn) * p.scale_log2};
+    f16_range_guard<2>(qv, p.status, 230);   // the attention reads q as fp16
+    q[j] = qv[0];
+    q[j + 32] = qv[1];
     return;
   }
   const int g = hh - p.Hq;
@@ -272,18 +286,20 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(const __grid_constant_
   size_t row;
   __half *dk, *dv;
   if (p.is_global) {
-    row = ((size_t)b * p.Lmax + p.p) * kvw + g * 64;
+    row = ((size_t)b * p.Lmax + pos) * kvw + g * 64;
     dk = p.full_k + row;
     dv = p.full_v + row;
   } else {
-    row = ((size_t)b * p.W + (p.p - p.M) % p.W) * kvw + g * 64;
+    row = ((size_t)b * p.W + (pos - p.M) % p.W) * kvw + g * 64;
     dk = p.ring_k + row;
     dv = p.ring_v + row;
   }
-  dk[j] = __float2half_rn(k1 * cs - k2 * sn);
-  dk[j + 32] = __float2half_rn(k2 * cs + k1 * sn);
-  dv[j] = __float2half_rn(P(vc + j));
-  dv[j + 32] = __float2half_rn(P(vc + j + 32));
+  const float kv[4] = {k1 * cs - k2 * sn, k2 * cs + k1 * sn, P(vc + j), P(vc + j + 32)};
+  f16_range_guard<4>(kv, p.status, 231);
+  dk[j] = __float2half_rn(kv[0]);
+  dk[j + 32] = __float2half_rn(kv[1]);
+  dv[j] = __float2half_rn(kv[2]);
+  dv[j + 32] = __float2half_rn(kv[3]);
 }
 
 // ----------------------------------------------------------------------------------------
@@ -319,13 +335,24 @@ struct DecAttnParams {
   const float* qrot;       // [B, Hq, 64] rotated, pre-scaled queries
   int Hq, Hkv, M, is_global;
   int n_meta_tiles;        // SWA: cdiv(M, 64); global: 0
-  int n_tiles;             // tiles per (b, g)
+  int n_tiles;             // tiles per (b, g) (with positions: the most any sequence has)
   int n_main_valid;        // SWA: filled ring slots; global: p + 1
   int rows_main;           // rows per sequence in the main cache (W or Lmax)
   int n_splits, n_items;
+  const int* positions;    // per-sequence positions [B] (device), or NULL: n_main_valid for all
+  int W, max_position;
   float* part;
   DevStatus* status;
 };
+
+// Keys of sequence b in the main cache (ring slots filled, or global rows 0..pos); 0 for a
+// position the cache cannot hold (the prep kernel reports it).
+__device__ __forceinline__ int da_main_valid(const DecAttnParams& p, int b) {
+  if (p.positions == nullptr) return p.n_main_valid;
+  const int pos = p.positions[b];
+  if (pos < p.M || pos > p.max_position || (p.is_global && pos >= p.rows_main)) return 0;
+  return p.is_global ? pos + 1 : min(pos - p.M + 1, p.W);
+}
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -381,7 +408,12 @@ __global__ void __launch_bounds__(DA_THREADS, 3)
     tma_prefetch_desc(&mapV);
   }
   __syncthreads();
-  auto item_tiles = [&](int w) { return min(DA_TPS, p.n_tiles - (w % p.n_splits) * DA_TPS); };
+  // tiles of item w: its split's share of the (b, g) tiles (none when the split lies past
+  // them, as it can for a sequence shorter than the batch's longest)
+  auto item_tiles = [&](int w, int main_valid) {
+    const int nt = p.n_meta_tiles + (main_valid + DA_KT - 1) / DA_KT;
+    return max(0, min(DA_TPS, nt - (w % p.n_splits) * DA_TPS));
+  };
 
   if (warp == DA_CONSUMERS / 32) {
     // ------------------------------ producer warp ------------------------------
@@ -393,7 +425,7 @@ __global__ void __launch_bounds__(DA_THREADS, 3)
       for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
         const int split = w % p.n_splits, bg = w / p.n_splits;
         const int g = bg % p.Hkv, b = bg / p.Hkv;
-        const int nt = item_tiles(w);
+        const int nt = item_tiles(w, da_main_valid(p, b));
         for (int t = 0; t < nt; ++t, ++issued) {
           const int stg = issued % DA_STAGES;
           if (issued >= DA_STAGES &&
@@ -437,7 +469,8 @@ __global__ void __launch_bounds__(DA_THREADS, 3)
   for (int w = blockIdx.x; w < p.n_items; w += gridDim.x) {
     const int split = w % p.n_splits, bg = w / p.n_splits;
     const int g = bg % p.Hkv, b = bg / p.Hkv;
-    const int nt = item_tiles(w);
+    const int main_valid = da_main_valid(p, b);
+    const int nt = item_tiles(w, main_valid);
     uint32_t qa[4][2];   // Q fragments (fp16): row gq = query head (zero beyond G), 4 x 16 dims
     float m_run = -INFINITY, l_run = 0.f;
     float o[8][4];
@@ -468,7 +501,7 @@ __global__ void __launch_bounds__(DA_THREADS, 3)
       const int ti = split * DA_TPS + t;
       const bool meta = ti < p.n_meta_tiles;
       const int key0 = meta ? ti * DA_KT : (ti - p.n_meta_tiles) * DA_KT;
-      const int lim = meta ? p.M : p.n_main_valid;
+      const int lim = meta ? p.M : main_valid;
       // S = Q K^T for this warp's 16 keys (two n-tiles of 8)
       float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -835,12 +868,9 @@ __global__ void wait_timeout_selftest_kernel(DevStatus* st) {
 // Fixed-order sum of split-K partial slices: out[i] = sum_s part[s*stride + i] (+ residual),
 // as fp32 or bf16; n is a multiple of 4.  The order never changes, so results are
 // identical from run to run.
-// When bcT is set, columns [tr_col0, tr_col0 + 32) of the [rows, ld] result (rows = b*T + t)
-// are also written time-major to bcT [B][32][Tp] (the scan's B/C input).
 __global__ void splitk_reduce_kernel(const float* __restrict__ part, int n_split, long long stride, int n,
                                      const __nv_bfloat16* __restrict__ residual, void* __restrict__ out,
-                                     int out_bf16, __half* __restrict__ bcp = nullptr, int ld = 0, int T = 0,
-                                     int Tp = 0, int tr_col0 = 0) {
+                                     int out_bf16) {
   pdl_wait();
   pdl_trigger();
   const int i = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
@@ -868,16 +898,6 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, int n_split
     *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
   } else {
     *reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + i) = acc;
-  }
-  if (bcp != nullptr) {   // the scan's copy of B and C: fp16 pairs (B_s, C_s), state-major
-    const int row = i / ld, col = i % ld;       // 4 columns of one row (ld % 4 == 0)
-    const int b = row / T, t = row % T;
-    const float vals[4] = {acc.x, acc.y, acc.z, acc.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int cc = col + e - tr_col0;         // 0..15: B_s, 16..31: C_s
-      if (cc >= 0 && cc < 32) bcp[(((size_t)b * 16 + (cc & 15)) * Tp + t) * 2 + (cc >> 4)] = __float2half_rn(vals[e]);
-    }
   }
 }
 

@@ -16,10 +16,10 @@ import torch
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhymba.so")
 HEADER_PATH = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "hymba.h")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_FP16_RANGE = range(7)
 KV_OWN, KV_PRODUCER, KV_CONSUMER = 0, 1, 2
 CACHE_SWA, CACHE_GLOBAL = 0, 1
-MODE_PREFILL, MODE_DECODE = 0, 1
+MODE_PREFILL, MODE_DECODE, MODE_PREFILL_HOST = 0, 1, 2
 
 _c_int, _c_size, _vp = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
 
@@ -55,7 +55,13 @@ class ProfRecord(ctypes.Structure):
 
 class StageLayout(ctypes.Structure):
     _fields_ = [(n, _c_size) for n in ("q", "xz", "xc", "xbc", "delta", "y", "o", "u")] + \
-               [("ld_xbc", _c_int), ("Tp", _c_int)]
+               [("ld_xbc", _c_int), ("scan_chunks", _c_int), ("scan_chunk_len", _c_int)]
+
+
+class DecodeStageLayout(ctypes.Structure):
+    _fields_ = [(n, _c_size) for n in ("proj", "xc", "xbc_part", "y")] + \
+               [("proj_slice_stride", ctypes.c_longlong), ("xbc_slice_stride", ctypes.c_longlong)] + \
+               [(n, _c_int) for n in ("in_split", "xproj_split", "ld_proj", "ld_xbc")]
 
 
 _LIB = None
@@ -91,8 +97,16 @@ def lib():
             "hymba_mixer_decode": ([ctypes.POINTER(LayerCfg), ctypes.POINTER(LayerWeights), _vp, _c_int,
                                     _c_int, ctypes.POINTER(KVCache), _vp, _vp, _vp, _vp, _vp, _c_size,
                                     _vp], _c_int),
+            "hymba_mixer_prefill_host": ([ctypes.POINTER(LayerCfg), ctypes.POINTER(LayerWeights), _vp, _c_int,
+                                          _c_int, _c_int, ctypes.POINTER(KVCache), _vp, _vp, _vp, _vp, _c_size,
+                                          _vp], _c_int),
+            "hymba_mixer_decode_ragged": ([ctypes.POINTER(LayerCfg), ctypes.POINTER(LayerWeights), _vp, _c_int,
+                                           _vp, _c_int, ctypes.POINTER(KVCache), _vp, _vp, _vp, _vp, _vp, _c_size,
+                                           _vp], _c_int),
             "hymba_mixer_stage_layout": ([ctypes.POINTER(LayerCfg), _c_int, _c_int, _c_int,
                                           ctypes.POINTER(StageLayout)], _c_int),
+            "hymba_decode_stage_layout": ([ctypes.POINTER(LayerCfg), _c_int, _c_int,
+                                           ctypes.POINTER(DecodeStageLayout)], _c_int),
             "hymba_gemm_bf16": ([_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp], _c_int),
             "hymba_rmsnorm": ([_vp, _vp, _c_int, _c_int, ctypes.c_float, _vp, _vp], _c_int),
             "hymba_ffn_swiglu": ([_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp], _c_int),
@@ -210,6 +224,13 @@ def stage_layout(dims, batch, n_tokens, x_has_meta=0) -> StageLayout:
     return out
 
 
+def decode_stage_layout(dims, batch, max_tokens) -> DecodeStageLayout:
+    out = DecodeStageLayout()
+    cfg = make_cfg(dims)
+    check(lib().hymba_decode_stage_layout(ctypes.byref(cfg), batch, max_tokens, ctypes.byref(out)))
+    return out
+
+
 def status_read(ws, stream=None) -> int:
     s = ctypes.c_int()
     check(lib().hymba_status_read(ptr(ws), stream_handle(stream), ctypes.byref(s)))
@@ -243,12 +264,34 @@ def mixer_prefill(dims, dw: DeviceWeights, x, kv: Cache, out, ws, x_has_meta=0, 
                                     ptr(ws), ws.numel(), stream_handle(stream)))
 
 
+def mixer_prefill_host(dims, dw: DeviceWeights, x_host, kv: Cache, out_host, ws, x_has_meta=0, ssm_state=None,
+                       conv_state=None, stream=None, cfg=None):
+    """hymba_mixer_prefill from host buffers: x_host [B, n, d] and out_host [B, T, d] are CPU
+    bf16 tensors (pinned for asynchronous copies); ws sized with MODE_PREFILL_HOST."""
+    assert not x_host.is_cuda and not out_host.is_cuda
+    cfg = make_cfg(dims) if cfg is None else cfg
+    B, n_tokens = x_host.shape[0], x_host.shape[1]
+    check(lib().hymba_mixer_prefill_host(ctypes.byref(cfg), ctypes.byref(dw.c), ptr(x_host), x_has_meta, B, n_tokens,
+                                         ctypes.byref(kv.c), ptr(ssm_state), ptr(conv_state), ptr(out_host), ptr(ws),
+                                         ws.numel(), stream_handle(stream)))
+
+
 def mixer_decode(dims, dw: DeviceWeights, x, position, kv: Cache, ssm_state, conv_state, out, ws, residual=None,
                  stream=None, cfg=None):
     cfg = make_cfg(dims) if cfg is None else cfg
     check(lib().hymba_mixer_decode(ctypes.byref(cfg), ctypes.byref(dw.c), ptr(x), x.shape[0], position,
                                    ctypes.byref(kv.c), ptr(ssm_state), ptr(conv_state), ptr(residual), ptr(out),
                                    ptr(ws), ws.numel(), stream_handle(stream)))
+
+
+def mixer_decode_ragged(dims, dw: DeviceWeights, x, positions, max_position, kv: Cache, ssm_state, conv_state, out,
+                        ws, residual=None, stream=None, cfg=None):
+    """hymba_mixer_decode with a position per sequence: positions is an int32 device tensor [B]."""
+    assert positions.dtype == torch.int32 and positions.is_cuda and positions.numel() == x.shape[0]
+    cfg = make_cfg(dims) if cfg is None else cfg
+    check(lib().hymba_mixer_decode_ragged(ctypes.byref(cfg), ctypes.byref(dw.c), ptr(x), x.shape[0], ptr(positions),
+                                          max_position, ctypes.byref(kv.c), ptr(ssm_state), ptr(conv_state),
+                                          ptr(residual), ptr(out), ptr(ws), ws.numel(), stream_handle(stream)))
 
 
 def mixer_decode_noalloc(dims, dw: DeviceWeights, x, position, kv: Cache, ssm_state, conv_state, out,

@@ -50,11 +50,13 @@ enum {
   HYMBA_ERR_WORKSPACE = 3,    /* workspace smaller than hymba_mixer_workspace_size */
   HYMBA_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed (message has details) */
   HYMBA_ERR_TIMEOUT = 5,      /* status word: a device-side bounded wait gave up */
+  HYMBA_ERR_FP16_RANGE = 6,   /* status word: a value stored in fp16 (queries, keys, values, the
+                                 KV cache, FFN activations) had |v| >= 65520 and became +-inf */
 };
 
 enum { HYMBA_KV_OWN = 0, HYMBA_KV_PRODUCER = 1, HYMBA_KV_CONSUMER = 2 };
 enum { HYMBA_CACHE_SWA = 0, HYMBA_CACHE_GLOBAL = 1 };
-enum { HYMBA_MODE_PREFILL = 0, HYMBA_MODE_DECODE = 1 };
+enum { HYMBA_MODE_PREFILL = 0, HYMBA_MODE_DECODE = 1, HYMBA_MODE_PREFILL_HOST = 2 };
 
 typedef uint16_t hymba_bf16;
 typedef uint16_t hymba_f16;   /* IEEE half bits */
@@ -151,16 +153,22 @@ int hymba_version(void);
 /* Message of the last error raised on this thread ("" if none). */
 const char* hymba_last_error(void);
 
-/* Bytes of workspace one prefill (mode HYMBA_MODE_PREFILL, n_tokens rows per sequence) or
- * decode step (HYMBA_MODE_DECODE, n_tokens ignored) needs.  x_has_meta: see prefill. */
+/* Bytes of workspace one prefill (mode HYMBA_MODE_PREFILL, n_tokens rows per sequence), one
+ * prefill from host buffers (HYMBA_MODE_PREFILL_HOST: the prefill's workspace plus device
+ * copies of the input and the output) or one decode step (HYMBA_MODE_DECODE; for a global
+ * layer n_tokens is the cache's max_tokens, otherwise ignored) needs.  x_has_meta: see
+ * prefill. */
 int hymba_mixer_workspace_size(const hymba_layer_cfg* cfg, int batch, int n_tokens, int x_has_meta, int mode,
                                size_t* bytes);
 
 /* Zero the status word of a workspace (call once after allocating it). */
 int hymba_workspace_init(void* workspace, size_t ws_bytes, hymba_stream stream);
 
-/* Synchronise `stream`, copy the workspace status word to *status (0, or HYMBA_ERR_TIMEOUT
- * when a device-side wait gave up), and clear it. */
+/* Synchronise `stream`, copy the workspace status word to *status and clear it.  *status is
+ * 0, or HYMBA_ERR_TIMEOUT when a device-side wait gave up, else HYMBA_ERR_FP16_RANGE when a
+ * value outside fp16's range was stored (the outputs of that call are then not finite; the
+ * layer's inputs must be normalised, as the block's RMSNorm does), else HYMBA_ERR_INVALID_ARG
+ * when a device-side index check skipped an access. */
 int hymba_status_read(void* workspace, hymba_stream stream, int* status);
 
 /* Plan and carve the KV caches of an n_layers stack ([JJ] §Hymba 的整体架构: adjacent SWA
@@ -197,6 +205,18 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
                         float* conv_state_out, const hymba_bf16* residual, hymba_bf16* out, void* workspace,
                         size_t ws_bytes, hymba_stream stream);
 
+/* hymba_mixer_prefill with the input and the output in HOST memory: x_host [B, n_tokens, d]
+ * and out_host [B, T, d] bf16 (page-locked memory lets the copies run asynchronously and
+ * overlap other streams' work; pageable memory works but the copies then block the host).
+ * Enqueued on `stream`: the copy of x_host into the workspace, the prefill, the copy of the
+ * output to out_host.  The workspace (mode HYMBA_MODE_PREFILL_HOST) holds the device copies.
+ * Weights, the KV cache and the states stay in device memory.  No residual.  Errors as
+ * hymba_mixer_prefill. */
+int hymba_mixer_prefill_host(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x_host,
+                             int x_has_meta, int batch, int n_tokens, hymba_kv_cache* kv, float* ssm_state_out,
+                             float* conv_state_out, hymba_bf16* out_host, void* workspace, size_t ws_bytes,
+                             hymba_stream stream);
+
 /* One decode step for `batch` sequences that all sit at position `position` (= M + number
  * of tokens already in the context; the pages' released model generates with equal-length
  * sequences).  x [B, d] bf16.  own/producer: the new K (after RoPE) and V go to ring slot
@@ -209,23 +229,56 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
                        const hymba_bf16* residual, hymba_bf16* out, void* workspace, size_t ws_bytes,
                        hymba_stream stream);
 
+/* The decode step for a batch whose sequences sit at different positions: sequence b's new
+ * token is at positions[b] (device memory, int32 [batch]), with n_meta <= positions[b] <=
+ * max_position (and, for a global layer, < kv->max_tokens).  Everything else as
+ * hymba_mixer_decode: each sequence's RoPE angle, ring slot (positions[b] - M) mod W (or
+ * global row positions[b]) and attended keys (the meta tokens plus its own filled window,
+ * or its rows 0..positions[b]) are its own.  This goes beyond the released model, which the
+ * jxzklqfsx.com news article (§4) notes cannot generate for padded batches with meta tokens
+ * and SWA.  max_position (host) sizes the attention's key splits.  A position outside those
+ * bounds is recorded in the status word (HYMBA_ERR_INVALID_ARG from hymba_status_read) and
+ * that sequence's cache is left unwritten; its outputs are then undefined. */
+int hymba_mixer_decode_ragged(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x,
+                              int batch, const int* positions, int max_position, hymba_kv_cache* kv,
+                              float* ssm_state, float* conv_state, const hymba_bf16* residual, hymba_bf16* out,
+                              void* workspace, size_t ws_bytes, hymba_stream stream);
+
 /* Byte offsets, inside a prefill workspace, of the stage buffers of the last prefill (for
  * stage-by-stage checks).  Layouts (rows r = b*T + t):
  *   q      [B*T, Hq*D]  fp16  queries after RoPE
  *   xz     [B*T, 2*Di]  bf16  in_proj x | z columns
  *   xc     [B*T, Di]    bf16  SiLU(conv(x))
  *   xbc    [B*T, ld_xbc] fp32 x_proj output: dt_low | B | C
- *   delta  [B, Di, Tp]  fp32  Delta, time-major with row stride Tp
+ *   delta  [B*T, Di]    fp32  Delta = softplus(dt_low W_dt^T + dt_bias)
  *   y      [B*T, Di]    bf16  scan output before the gate
  *   o      [B*T, Hq*D]  fp32  attention output
- *   u      [B*T, Hq*D+Di] fp16 normalised, rescaled, averaged branches (out_proj input) */
+ *   u      [B*T, Hq*D+Di] fp16 normalised, rescaled, averaged branches (out_proj input)
+ * scan_chunks / scan_chunk_len: the time chunks the selective scan is cut into (the last
+ * chunk may be shorter). */
 typedef struct hymba_stage_layout {
   size_t q, xz, xc, xbc, delta, y, o, u;
   int ld_xbc;
-  int Tp;
+  int scan_chunks, scan_chunk_len;
 } hymba_stage_layout;
 int hymba_mixer_stage_layout(const hymba_layer_cfg* cfg, int batch, int n_tokens, int x_has_meta,
                              hymba_stage_layout* out);
+
+/* Byte offsets, inside a decode workspace, of the stage buffers of the last decode step (for
+ * stage-by-stage checks).  max_tokens: the cache's max_tokens (it sizes a global layer's
+ * attention splits).  Layouts (B sequences, P = in_proj width):
+ *   proj      in_split slices of [B, P] fp32, slice stride proj_slice_stride elements: the
+ *             in_proj output [q | k | v | x | z] is the sum of the slices in slice order
+ *   xc        [B, Di]  bf16  SiLU(conv) of the new token
+ *   xbc_part  xproj_split slices of [B, ld_xbc] fp32, slice stride xbc_slice_stride
+ *             elements: x_proj's [dt_low | B | C] is the sum of the slices in slice order
+ *   y         [B, Di]  fp32  gated SSM output */
+typedef struct hymba_decode_stages {
+  size_t proj, xc, xbc_part, y;
+  long long proj_slice_stride, xbc_slice_stride;
+  int in_split, xproj_split, ld_proj, ld_xbc;
+} hymba_decode_stages;
+int hymba_decode_stage_layout(const hymba_layer_cfg* cfg, int batch, int max_tokens, hymba_decode_stages* out);
 
 /* C[M, N] = A[M, K] * B[N, K]^T (+ residual[M, N]) on the tcgen05 GEMM, bf16 in/out, fp32
  * accumulation.  K % 8 == 0, N % 8 == 0.  status_ws: a workspace (>= 256 bytes) whose
@@ -264,9 +317,9 @@ int hymba_set_wait_limit_ns(unsigned long long ns);
 int hymba_selftest_wait_timeout(void* workspace, size_t ws_bytes, hymba_stream stream);
 
 /* hymba_mixer_decode without a workspace argument, for callers that cannot allocate device
- * memory where they run a decode step (inside a CUDA graph capture, in a serving loop
- * that must not take cudaMalloc's device synchronisation, or as a plugin whose host
- * runtime owns all device memory).  The pages have no counterpart: this is a deployment
+ * memory where they run a decode step (a serving loop that must not take cudaMalloc's
+ * device synchronisation between tokens, or a plugin whose host runtime owns all device
+ * memory and hands it only inputs and outputs).  The pages have no counterpart: this is a deployment
  * convenience of this library.  Arguments and results are those of hymba_mixer_decode.
  *   - Scratch: a built-in 32 MiB device array (every GPU that loads the library holds it
  *     until exit).  A step that needs more (hymba_mixer_workspace_size, mode DECODE, with
@@ -276,8 +329,11 @@ int hymba_selftest_wait_timeout(void* workspace, size_t ws_bytes, hymba_stream s
  *     call before any stream capture.
  *   - Every call on a device uses the same array: calls that can overlap on the GPU (for
  *     example on two streams of one device) race on it; the caller must serialise them.
- *   - The status word at the start of the array is cleared at every call, so device-side
- *     timeouts of this variant are not reported; use hymba_mixer_decode to read them.
+ *   - The status word at the start of the array is cleared at every call and cannot be
+ *     read, so device-side errors of this variant (a bounded wait that runs out, an fp16
+ *     overflow) are not reported.  After such an error the step's outputs, states and new
+ *     cache slot are undefined, with no sign of it; a caller that must detect errors uses
+ *     hymba_mixer_decode and reads its workspace's status word.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine. */
 int hymba_mixer_decode_noalloc(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x,
                                int batch, int position, hymba_kv_cache* kv, float* ssm_state, float* conv_state,

@@ -89,27 +89,22 @@ class PrefillRun:
         self.layout = H.stage_layout(dims, B, n, x_has_meta)
         self.B = B
 
-    def stage(self, name):
+    def stage(self, name, b=None):
+        """A stage buffer as float64 [B, T, ...], or only sequence b's [T, ...] when b is given."""
         d, L, B, T = self.dims, self.layout, self.B, self.T
-        rows = B * T
-        if name == "q":
-            return to_np(ws_view(self.ws, L.q, (B, T, d.n_q_heads, d.head_dim), torch.float16))
-        if name == "xz":
-            return to_np(ws_view(self.ws, L.xz, (B, T, 2 * d.d_inner), torch.bfloat16))
-        if name == "xc":
-            return to_np(ws_view(self.ws, L.xc, (B, T, d.d_inner), torch.bfloat16))
-        if name == "xbc":
-            return to_np(ws_view(self.ws, L.xbc, (B, T, L.ld_xbc), torch.float32))
-        if name == "delta":
-            dT = to_np(ws_view(self.ws, L.delta, (B, d.d_inner, L.Tp), torch.float32))
-            return np.transpose(dT[:, :, :T], (0, 2, 1))
-        if name == "y":
-            return to_np(ws_view(self.ws, L.y, (B, T, d.d_inner), torch.bfloat16))
-        if name == "o":
-            return to_np(ws_view(self.ws, L.o, (B, T, d.n_q_heads * d.head_dim), torch.float32))
-        if name == "u":
-            return to_np(ws_view(self.ws, L.u, (B, T, d.attn_width + d.d_inner), torch.float16))
-        raise KeyError(name)
+        shapes = {
+            "q": (L.q, (B, T, d.n_q_heads, d.head_dim), torch.float16),
+            "xz": (L.xz, (B, T, 2 * d.d_inner), torch.bfloat16),
+            "xc": (L.xc, (B, T, d.d_inner), torch.bfloat16),
+            "xbc": (L.xbc, (B, T, L.ld_xbc), torch.float32),
+            "delta": (L.delta, (B, T, d.d_inner), torch.float32),
+            "y": (L.y, (B, T, d.d_inner), torch.bfloat16),
+            "o": (L.o, (B, T, d.n_q_heads * d.head_dim), torch.float32),
+            "u": (L.u, (B, T, d.attn_width + d.d_inner), torch.float16),
+        }
+        off, shape, dt = shapes[name]
+        v = ws_view(self.ws, off, shape, dt)
+        return to_np(v if b is None else v[b])
 
     def kv(self):
         T = self.T

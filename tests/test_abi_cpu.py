@@ -35,7 +35,21 @@ def test_workspace_sizes_grow_with_tokens():
     lay = H.stage_layout(d, 1, 2048)
     offs = [lay.q, lay.xz, lay.xc, lay.xbc, lay.delta, lay.y, lay.o, lay.u]
     assert all(o % 256 == 0 for o in offs) and offs == sorted(offs) and offs[-1] < a
-    assert lay.Tp % 8 == 0 and lay.Tp >= 2176 and lay.ld_xbc >= 132
+    assert lay.ld_xbc >= 132
+    assert lay.scan_chunks >= 1 and lay.scan_chunk_len % 8 == 0
+    assert lay.scan_chunks * lay.scan_chunk_len >= 2176 > (lay.scan_chunks - 1) * lay.scan_chunk_len
+
+
+@pytest.mark.parametrize("B,N,Di", [(1, 2048, 3200), (4, 8192, 3200), (8, 4096, 3200), (1, 120, 512),
+                                    (3, 1, 512), (64, 100, 3200), (2, 37, 64)])
+def test_scan_chunking_matches_bench_accounting(B, N, Di):
+    """bench.py counts the scan's bytes per chunk the way the library cuts T into chunks."""
+    import bench
+    d = synth.workloads()["tiny"].dims.replace(d_inner=Di, n_meta=8)
+    lay = H.stage_layout(d, B, N)
+    T = 8 + N
+    assert bench.scan_chunks(B, Di, T) == (lay.scan_chunk_len, lay.scan_chunks)
+    assert (lay.scan_chunks - 1) * lay.scan_chunk_len < T <= lay.scan_chunks * lay.scan_chunk_len
     dec = H.workspace_size(d, 64, 0, 0, H.MODE_DECODE)
     assert dec > 0
 

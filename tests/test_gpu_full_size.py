@@ -66,6 +66,12 @@ def test_global_layer_full_size_sampled_rows():
         ref, h = _oracle_rows(dims, w, Xt_b, rows)
         assert_rms(out[b, rows], ref, name=f"global layer rows (b={b})")
         assert_rel_inf(to_np(run.ssm[b]), h, tol=2e-2, name=f"global layer ssm state (b={b})")
+        # the scan over all 8320 steps, fed the GPU's own xc, delta, B, C: fp32 state at 1e-4
+        xc, delta, xbc = run.stage("xc", b), run.stage("delta", b), run.stage("xbc", b)
+        R_, S = dims.dt_rank, dims.d_state
+        _, h_own = orc.selective_scan(xc, delta, w["A"], xbc[:, R_:R_ + S], xbc[:, R_ + S:R_ + 2 * S],
+                                      np.zeros_like(xc))
+        assert_rel_inf(to_np(run.ssm[b]), h_own, tol=1e-4, name=f"global layer scan state, own inputs (b={b})")
 
 
 def _bf16_ulp(x):
@@ -126,3 +132,71 @@ def test_stack_32_layers_teacher_forced():
         # residual adds of the stack, within one bf16 step of the stored stream
         assert np.all(np.abs(h_mid - (h_in + mix_np)) <= _bf16_ulp(h_mid) + _bf16_ulp(mix_np)), f"{tag}: mixer residual"
         assert np.all(np.abs(h_out - (h_mid + ffn_np)) <= _bf16_ulp(h_out) + _bf16_ulp(ffn_np)), f"{tag}: FFN residual"
+
+
+def test_stack_32_layers_decode_step():
+    """The 32-layer decode step (first, middle and last layers global with full-length
+    caches; SWA pairs sharing one ring; each layer's FFN): prefill of the first N-1 tokens,
+    then one decode step for token N at position M + N - 1 for all 8 sequences.
+    - Every checked layer's mixer and FFN, rerun on copies of the inputs, caches and states
+      that layer saw inside the step, against the oracle's decode (bf16 bound), and the
+      stack's residual adds within one bf16 step.
+    - End to end, the decoded stream equals the last row of the 32-layer prefill of all N
+      tokens (different kernels and summation orders on the two paths; a wrong cache slot,
+      state or pairing would be an O(1) error): max|err| <= 1e-1 RMS."""
+    wl = WL["stack"]
+    st = HymbaStack(wl, seed=0, keep_host_weights=True, decode_room=1)
+    E = torch.from_numpy(synth.stack_embeddings(wl)).cuda().to(torch.bfloat16)
+    N, d = wl.n_tokens, wl.dims.d_model
+    check_layers = [0, 1, 2, 15, 16, 30, 31]
+    frec = {l: [] for l in check_layers}
+    full_last = to_np(st.forward(E, record=frec)[:, -1])
+    st.forward(E[:, :N - 1].contiguous())
+    rec = {l: {} for l in check_layers}
+    p = wl.dims.n_meta + N - 1
+    h = to_np(st.decode_step(E[:, N - 1].contiguous(), p, record=rec))
+    torch.cuda.synchronize()
+    assert H.status_read(st.dws) == 0 and H.status_read(st.ws) == 0
+    # drift of the decode path from the prefill path, layer by layer (sequence 0): it starts
+    # at zero (same embedding) and grows by the two paths' independent bf16 roundings
+    for l in check_layers:
+        h_pre = [it for it in frec[l] if it[0] == "h"][-1][1][-1]
+        assert_rms(rec[l]["h_in"][0], h_pre, tol=5e-2 if l <= 2 else 1.5e-1,
+                           name=f"decode vs prefill stream entering layer {l}")
+    assert_rms(h, full_last, tol=1.5e-1, name="32-layer decode step vs last row of the 32-layer prefill")
+    B = wl.batch
+    for l in check_layers:
+        dl, w, bw = st.host[l]
+        _, dw, dev = st.layers[l]
+        r = rec[l]
+        tag = f"decode layer {l} (kv role {dl.kv_role}, global {dl.is_global})"
+        # the mixer, rerun without the residual on copies of what the layer saw
+        cache = H.Cache(dl, B, st.max_tokens)
+        for n, arr in r["cache"].items():
+            cache.t[n].copy_(torch.from_numpy(arr.astype(np.float32)).cuda().to(torch.float16))
+        ssm = torch.from_numpy(r["ssm"]).cuda()
+        conv = torch.from_numpy(r["conv"]).cuda()
+        ws = H.alloc_workspace(H.workspace_size(dl, B, st.max_tokens, 0, H.MODE_DECODE))
+        mix = torch.empty(B, d, dtype=torch.bfloat16, device="cuda")
+        H.mixer_decode(dl, dw, torch.from_numpy(r["hn"].astype(np.float32)).cuda().to(torch.bfloat16), p, cache,
+                       ssm, conv, mix, ws)
+        act = torch.empty(B, st.F, dtype=torch.float16, device="cuda")
+        ffn = torch.empty(B, d, dtype=torch.bfloat16, device="cuda")
+        H.ffn_swiglu(torch.from_numpy(r["hn2"].astype(np.float32)).cuda().to(torch.bfloat16), dev["w_gu"],
+                     dev["w_down"], act, ffn, ws)
+        torch.cuda.synchronize()
+        assert H.status_read(ws) == 0
+        ocache = r["cache"] if dl.is_global else {n: r["cache"][n] for n in ("meta_k", "meta_v", "ring_k", "ring_v")}
+        ref = orc.mixer_decode(dl, w, r["hn"], p, ocache, r["ssm"], r["conv"])
+        mix_np, ffn_np = to_np(mix), to_np(ffn)
+        assert_rms(mix_np, ref["out"], name=f"{tag} mixer")
+        assert_rms(ffn_np, orc.ffn_swiglu(r["hn2"], bw), name=f"{tag} FFN")
+        assert_elem(r["hn"], orc.rmsnorm(r["h_in"], bw["g_norm1"], dl.norm_eps), name=f"{tag} norm 1")
+        assert_elem(r["hn2"], orc.rmsnorm(r["h_mid"], bw["g_norm2"], dl.norm_eps), name=f"{tag} norm 2")
+        assert np.all(np.abs(r["h_mid"] - (r["h_in"] + mix_np)) <= _bf16_ulp(r["h_mid"]) + _bf16_ulp(mix_np)), \
+            f"{tag}: mixer residual"
+        assert np.all(np.abs(r["h_out"] - (r["h_mid"] + ffn_np)) <= _bf16_ulp(r["h_out"]) + _bf16_ulp(ffn_np)), \
+            f"{tag}: FFN residual"
+        # the layer's states after the step agree with the oracle's
+        # (through the bf16 conv output of the new token, as every end-to-end state check)
+        assert_rel_inf(st.ssm[l].cpu().numpy(), ref["ssm_state"], tol=2e-2, name=f"{tag} ssm state")

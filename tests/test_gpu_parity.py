@@ -81,11 +81,9 @@ def _check_stages(run, ref, dims, w):
         assert_rms(xbc[b, :, :R + 2 * S], proj, tol=1e-3, name="x_proj")
         d_ref = orc.softplus(xbc[b, :, :R] @ w["w_dt"].astype(np.float64).T + w["dt_bias"])
         assert_rel_inf(delta[b], d_ref, tol=5e-3, name="delta")
-        # scan fed the GPU's own xc, delta, B, C, z (the scan reads B and C as fp16)
+        # scan fed the GPU's own xc, delta, B, C, z
         zb = xz[b, :, Di:]
-        bm16 = xbc[b, :, R:R + S].astype(np.float16).astype(np.float64)
-        cm16 = xbc[b, :, R + S:R + 2 * S].astype(np.float16).astype(np.float64)
-        y_ref, h_ref = orc.selective_scan(xc[b], delta[b], w["A"], bm16, cm16, zb)
+        y_ref, h_ref = orc.selective_scan(xc[b], delta[b], w["A"], xbc[b, :, R:R + S], xbc[b, :, R + S:R + 2 * S], zb)
         assert_rel_inf(to_np(run.ssm[b]), h_ref, tol=1e-4, name="scan state")
         assert_elem(y[b] * orc.silu(zb), y_ref, name="scan y")
         if k is not None:
@@ -158,6 +156,24 @@ def test_prefill_with_meta_in_input_and_residual():
     assert_rms(to_np(run.out), ref["out"], name="out")
 
 
+def test_prefill_from_host_buffers_equals_device_path():
+    """hymba_mixer_prefill_host (input and output in pinned host memory, copies enqueued by
+    the library) gives the device-buffer prefill's output bit for bit, on its own stream."""
+    wl = WL["tiny"]
+    dims = wl.dims
+    w = _w(dims, seed=51)
+    X = synth.bf16_round(np.random.default_rng(52).normal(size=(2, 77, dims.d_model)).astype(np.float32))
+    run = PrefillRun(dims, w, X)
+    xh = torch.from_numpy(X).to(torch.bfloat16).pin_memory()
+    oh = torch.zeros(2, run.T, dims.d_model, dtype=torch.bfloat16).pin_memory()
+    ws = H.alloc_workspace(H.workspace_size(dims, 2, 77, 0, H.MODE_PREFILL_HOST))
+    s = torch.cuda.Stream()
+    H.mixer_prefill_host(dims, run.dw, xh, H.Cache(dims, 2, run.T), oh, ws, stream=s)
+    s.synchronize()
+    assert H.status_read(ws, s) == 0
+    assert torch.equal(oh, run.out.cpu())
+
+
 def test_prefill_shared_kv_pair():
     wl = WL["tiny"]
     prod = wl.dims.replace(kv_role=synth.KV_PRODUCER)
@@ -177,6 +193,24 @@ def test_prefill_shared_kv_pair():
     assert_rms(rc.stage("o")[0], o_ref.reshape(rc.T, -1), name="consumer attention")
 
 
+@pytest.mark.parametrize("B,N", [(1, 120), (3, 700)])
+def test_prefill_scan_general_decays(B, N):
+    """A rows that are not the progression A[s] = (s+1) A[0] take the scan's general path
+    (one exponential per state); here half of the channels (whole warps) have such rows, the
+    rest the progression, so both paths run in one launch and against the oracle."""
+    dims = WL["tiny"].dims
+    w = _w(dims, seed=11)
+    rng = np.random.default_rng(12)
+    A = w["A"].copy()
+    A[dims.d_inner // 2:] = -rng.uniform(0.3, 6.0, size=(dims.d_inner // 2, dims.d_state)).astype(np.float32)
+    w["A"] = A
+    X = synth.bf16_round(rng.normal(size=(B, N, dims.d_model)).astype(np.float32))
+    run = PrefillRun(dims, w, X)
+    ref = orc.mixer_prefill(dims, w, X)
+    assert_rms(to_np(run.out), ref["out"], name="out")
+    _check_stages(run, ref, dims, w)
+
+
 def test_prefill_swa_hymba_layer():
     wl = WL["swa"]
     w = _w(wl.dims, wl=wl)
@@ -190,7 +224,7 @@ def test_prefill_swa_hymba_layer():
 # ---------------------------------------------------------------------------------------
 # decode
 # ---------------------------------------------------------------------------------------
-def _decode(dims, w, cache, x, position, ssm, conv, residual=None):
+def _decode(dims, w, cache, x, position, ssm, conv, residual=None, keep_ws=False):
     B = x.shape[0]
     dw = H.DeviceWeights(w)
     out = torch.zeros(B, dims.d_model, dtype=torch.bfloat16, device="cuda")
@@ -200,7 +234,29 @@ def _decode(dims, w, cache, x, position, ssm, conv, residual=None):
                    residual=None if residual is None else bf16_dev(residual))
     torch.cuda.synchronize()
     assert H.status_read(ws) == 0
-    return out
+    return (out, ws) if keep_ws else out
+
+
+def _check_decode_ssm_step(dims, w, ws, B, max_tokens, h0, h_gpu):
+    """The decode SSM step against the oracle fed the step's own inputs from the workspace
+    (xc, x_proj's dt_low | B | C summed over its split-K slices in order, z from in_proj):
+    the fp32 state within 1e-4 (inf-norm relative), the gated output y likewise."""
+    from tests.helpers import ws_view
+    L = H.decode_stage_layout(dims, B, max_tokens)
+    Di, R, S = dims.d_inner, dims.dt_rank, dims.d_state
+    proj = sum(to_np(ws_view(ws, L.proj + 4 * i * L.proj_slice_stride, (B, L.ld_proj), torch.float32))
+               for i in range(L.in_split))
+    xbc = sum(to_np(ws_view(ws, L.xbc_part + 4 * i * L.xbc_slice_stride, (B, L.ld_xbc), torch.float32))
+              for i in range(L.xproj_split))
+    xc = to_np(ws_view(ws, L.xc, (B, Di), torch.bfloat16))
+    y_gpu = to_np(ws_view(ws, L.y, (B, Di), torch.float32))
+    z = proj[:, L.ld_proj - Di:]
+    for b in range(B):
+        delta = orc.softplus(xbc[b:b + 1, :R] @ w["w_dt"].astype(np.float64).T + w["dt_bias"])
+        y_ref, h_ref = orc.selective_scan(xc[b:b + 1], delta, w["A"], xbc[b:b + 1, R:R + S],
+                                          xbc[b:b + 1, R + S:R + 2 * S], z[b:b + 1], h0=h0[b])
+        assert_rel_inf(h_gpu[b], h_ref, tol=1e-4, name=f"decode ssm state, own inputs (b={b})")
+        assert_rel_inf(y_gpu[b], y_ref[0], tol=1e-4, name=f"decode ssm y, own inputs (b={b})")
 
 
 @pytest.mark.parametrize("is_global", [0, 1])
@@ -250,8 +306,10 @@ def test_decode_pair_hymba():
         cache.t[n].copy_(f32_dev(st_p[n]).to(torch.float16))
     ssm_p, conv_p = f32_dev(st_p["ssm_state"]), f32_dev(st_p["conv_state"])
     ssm_c, conv_c = f32_dev(st_c["ssm_state"]), f32_dev(st_c["conv_state"])
-    out_p = _decode(prod, wp, cache, st_p["x_new"], p, ssm_p, conv_p)
+    out_p, ws_p = _decode(prod, wp, cache, st_p["x_new"], p, ssm_p, conv_p, keep_ws=True)
     out_c = _decode(cons, wc, cache, st_c["x_new"], p, ssm_c, conv_c)
+    _check_decode_ssm_step(prod, wp, ws_p, wl.batch, cache.c.max_tokens,
+                           st_p["ssm_state"].astype(np.float64), to_np(ssm_p))
     ocache = {n: st_p[n] for n in ("meta_k", "meta_v", "ring_k", "ring_v")}
     rp = orc.mixer_decode(prod, wp, st_p["x_new"], p, ocache, st_p["ssm_state"], st_p["conv_state"])
     rc = orc.mixer_decode(cons, wc, st_c["x_new"], p, rp["cache"], st_c["ssm_state"], st_c["conv_state"])
@@ -262,6 +320,173 @@ def test_decode_pair_hymba():
     slot = orc.ring_slot(p, prod.n_meta, prod.window)
     assert_rms(to_np(cache.t["ring_k"][:, slot]), rp["cache"]["ring_k"][:, slot], name="new ring k")
     assert_rms(to_np(cache.t["ring_v"][:, slot]), rp["cache"]["ring_v"][:, slot], name="new ring v")
+
+
+def test_decode_global_layer_hymba_width():
+    """A global (full-attention) layer's decode step at Hymba width: 25/5 heads, d_inner 3200,
+    batch 8, new token at position 128 + 4096 over a full-length cache of N(0,1) keys and
+    values, against the oracle's decode over the same cache; the new K/V row and the SSM
+    step (own inputs, 1e-4) too."""
+    import dataclasses
+    wl = dataclasses.replace(WL["decode_pair"], batch=8)
+    dims = wl.dims.replace(is_global=1, kv_role=synth.KV_OWN)
+    B, p = wl.batch, 128 + 4096
+    Lmax = p + 1
+    w = _w(dims, layer=2, wl=wl)
+    st = synth.decode_state(wl, layer=2)
+    kv = synth.global_cache(wl, Lmax, layer=2)
+    cache = H.Cache(dims, B, Lmax, kind=H.CACHE_GLOBAL)
+    cache.t["k"].copy_(f32_dev(kv["k"]).to(torch.float16))
+    cache.t["v"].copy_(f32_dev(kv["v"]).to(torch.float16))
+    ssm, conv = f32_dev(st["ssm_state"]), f32_dev(st["conv_state"])
+    out, ws = _decode(dims, w, cache, st["x_new"], p, ssm, conv, keep_ws=True)
+    ref = orc.mixer_decode(dims, w, st["x_new"], p, {"k": kv["k"], "v": kv["v"]}, st["ssm_state"],
+                           st["conv_state"])
+    assert_rms(to_np(out), ref["out"], name="global decode out")
+    assert_rms(to_np(cache.t["k"][:, p]), ref["cache"]["k"][:, p], name="new k row")
+    assert_rms(to_np(cache.t["v"][:, p]), ref["cache"]["v"][:, p], name="new v row")
+    assert_rel_inf(to_np(conv), ref["conv_state"], tol=1e-2, name="conv state")
+    _check_decode_ssm_step(dims, w, ws, B, Lmax, st["ssm_state"].astype(np.float64), to_np(ssm))
+
+
+# ---------------------------------------------------------------------------------------
+# decode with a position per sequence
+# ---------------------------------------------------------------------------------------
+def _ragged_case(dims, B, positions, seed, Lmax=None):
+    rng = np.random.default_rng(seed)
+    Hkv, D, M, W = dims.n_kv_heads, dims.head_dim, dims.n_meta, dims.window
+    r = lambda *shape: synth.bf16_round(rng.normal(size=shape).astype(np.float32))
+    st = {"x_new": r(B, dims.d_model), "ssm_state": rng.normal(size=(B, dims.d_inner, dims.d_state)).astype(np.float32),
+          "conv_state": rng.normal(size=(B, dims.d_inner, dims.d_conv - 1)).astype(np.float32)}
+    if dims.is_global:
+        cache = {"k": r(B, Lmax, Hkv, D), "v": r(B, Lmax, Hkv, D)}
+    else:
+        cache = {"meta_k": r(B, M, Hkv, D), "meta_v": r(B, M, Hkv, D), "ring_k": r(B, W, Hkv, D),
+                 "ring_v": r(B, W, Hkv, D)}
+    return st, cache
+
+
+def _ragged_run(dims, w, st, cache, positions, Lmax, dev_cache=None):
+    B = len(positions)
+    if dev_cache is None:
+        dev_cache = H.Cache(dims, B, Lmax)
+        for n, a in cache.items():
+            dev_cache.t[n].copy_(f32_dev(a).to(torch.float16))
+    ssm, conv = f32_dev(st["ssm_state"]), f32_dev(st["conv_state"])
+    out = torch.zeros(B, dims.d_model, dtype=torch.bfloat16, device="cuda")
+    ws = H.alloc_workspace(H.workspace_size(dims, B, Lmax, 0, H.MODE_DECODE))
+    pos = torch.tensor(positions, dtype=torch.int32, device="cuda")
+    H.mixer_decode_ragged(dims, H.DeviceWeights(w), bf16_dev(st["x_new"]), pos, max(positions), dev_cache, ssm,
+                          conv, out, ws)
+    torch.cuda.synchronize()
+    assert H.status_read(ws) == 0
+    return out, ssm, conv, dev_cache
+
+
+def _ragged_oracle(dims, w, st, cache, positions):
+    outs, states, caches = [], [], []
+    for b, p in enumerate(positions):
+        cb = {n: a[b:b + 1] for n, a in cache.items()}
+        r = orc.mixer_decode(dims, w, st["x_new"][b:b + 1], p, cb, st["ssm_state"][b:b + 1], st["conv_state"][b:b + 1])
+        outs.append(r["out"][0]); states.append(r["ssm_state"][0]); caches.append(r["cache"])
+    return np.stack(outs), np.stack(states), {n: np.concatenate([c[n] for c in caches]) for n in cache}
+
+
+@pytest.mark.parametrize("is_global", [0, 1])
+def test_decode_ragged_positions(is_global):
+    """Sequences at different positions in one decode call: the first input token (one
+    filled ring slot), a partly filled ring, a ring exactly full, a wrapped ring, and for a
+    global layer caches filled to different lengths; each sequence against the oracle's
+    decode at its own position, then a consumer layer reading the producer's ring."""
+    dims = WL["tiny"].dims.replace(window=32, is_global=is_global,
+                                   kv_role=synth.KV_OWN if is_global else synth.KV_PRODUCER)
+    M, W = dims.n_meta, dims.window
+    positions = [M, M + 5, M + W - 1, M + W, M + 3 * W + 7, M + 1]
+    Lmax = max(positions) + 1 if is_global else 1
+    w = _w(dims, seed=41)
+    st, cache = _ragged_case(dims, len(positions), positions, seed=42, Lmax=Lmax)
+    out, ssm, conv, dcache = _ragged_run(dims, w, st, cache, positions, Lmax)
+    ref_out, ref_state, ref_cache = _ragged_oracle(dims, w, st, cache, positions)
+    assert_rms(to_np(out), ref_out, name="ragged decode out")
+    assert_rel_inf(to_np(ssm), ref_state, tol=1e-3, name="ragged decode ssm state")
+    for b, p in enumerate(positions):   # the one cache row each sequence wrote
+        if is_global:
+            assert_rms(to_np(dcache.t["k"][b, p]), ref_cache["k"][b, p], name=f"k row (b={b})")
+        else:
+            slot = orc.ring_slot(p, M, W)
+            assert_rms(to_np(dcache.t["ring_k"][b, slot]), ref_cache["ring_k"][b, slot], name=f"ring k (b={b})")
+            assert_rms(to_np(dcache.t["ring_v"][b, slot]), ref_cache["ring_v"][b, slot], name=f"ring v (b={b})")
+    if not is_global:   # the consumer of the pair reads the producer's updated ring
+        cons = dims.replace(kv_role=synth.KV_CONSUMER)
+        wc = _w(cons, seed=43)
+        stc, _ = _ragged_case(cons, len(positions), positions, seed=44)
+        outc, _, _, _ = _ragged_run(cons, wc, stc, None, positions, Lmax, dev_cache=dcache)
+        refc, _, _ = _ragged_oracle(cons, wc, stc, ref_cache, positions)
+        assert_rms(to_np(outc), refc, name="ragged decode consumer out")
+
+
+def test_decode_ragged_equal_positions_is_the_uniform_step():
+    """With every sequence at the same position the per-sequence step is the uniform step,
+    bit for bit (Hymba-width SWA producer, batch 16)."""
+    wl = WL["decode_pair"]
+    dims = wl.dims
+    B, p = 16, wl.decode_position
+    w = _w(dims, wl=wl)
+    st, cache = _ragged_case(dims, B, [p] * B, seed=45)
+    out_r, ssm_r, _, cache_r = _ragged_run(dims, w, st, cache, [p] * B, 1)
+    c2 = H.Cache(dims, B, 1)
+    for n, a in cache.items():
+        c2.t[n].copy_(f32_dev(a).to(torch.float16))
+    ssm, conv = f32_dev(st["ssm_state"]), f32_dev(st["conv_state"])
+    out = _decode(dims, w, c2, st["x_new"], p, ssm, conv)
+    assert torch.equal(out, out_r) and torch.equal(ssm, ssm_r)
+    assert torch.equal(c2.t["ring_k"], cache_r.t["ring_k"])
+
+
+def test_decode_ragged_hymba_width():
+    """Hymba-width SWA layer, batch 12, positions spread from the first input token to far
+    past the window."""
+    wl = WL["decode_pair"]
+    dims = wl.dims
+    rng = np.random.default_rng(46)
+    positions = sorted(int(v) for v in rng.integers(dims.n_meta, dims.n_meta + 4000, size=10)) + [dims.n_meta, 1151]
+    w = _w(dims, wl=wl, layer=3)
+    st, cache = _ragged_case(dims, len(positions), positions, seed=47)
+    out, ssm, _, _ = _ragged_run(dims, w, st, cache, positions, 1)
+    ref_out, ref_state, _ = _ragged_oracle(dims, w, st, cache, positions)
+    assert_rms(to_np(out), ref_out, name="ragged decode out (Hymba width)")
+    assert_rel_inf(to_np(ssm), ref_state, tol=1e-3, name="ragged decode ssm state (Hymba width)")
+
+
+# ---------------------------------------------------------------------------------------
+# fp16 range: a layer input far outside the normalised range is reported, not hidden
+# ---------------------------------------------------------------------------------------
+def test_fp16_overflow_is_reported():
+    """Queries, keys and values are stored in fp16.  With inputs scaled by 1e6 the
+    projections exceed fp16's range (|v| >= 65520 rounds to inf); prefill and decode must
+    then report HYMBA_ERR_FP16_RANGE in the status word, and a normal call must not."""
+    dims = WL["tiny"].dims.replace(window=16)
+    w = _w(dims, seed=31)
+    rng = np.random.default_rng(32)
+    X = synth.bf16_round(rng.normal(size=(1, 40, dims.d_model)).astype(np.float32))
+    dw = H.DeviceWeights(w)
+    for scale, want in ((1.0, H.OK), (1e6, H.ERR_FP16_RANGE)):
+        x = bf16_dev(X * scale)
+        T = dims.n_meta + 40
+        cache = H.Cache(dims, 1, T + 1)
+        out = torch.zeros(1, T, dims.d_model, dtype=torch.bfloat16, device="cuda")
+        ws = H.alloc_workspace(H.workspace_size(dims, 1, 40))
+        ssm = torch.zeros(1, dims.d_inner, dims.d_state, device="cuda")
+        conv = torch.zeros(1, dims.d_inner, dims.d_conv - 1, device="cuda")
+        H.mixer_prefill(dims, dw, x, cache, out, ws, ssm_state=ssm, conv_state=conv)
+        assert H.status_read(ws) == want, f"prefill, input scale {scale}"
+        if scale == 1.0:   # decode from the finite state, with a new token scaled up
+            dws = H.alloc_workspace(H.workspace_size(dims, 1, T + 1, 0, H.MODE_DECODE))
+            o1 = torch.zeros(1, dims.d_model, dtype=torch.bfloat16, device="cuda")
+            xn = bf16_dev(synth.bf16_round(rng.normal(size=(1, dims.d_model)).astype(np.float32)) * 1e6)
+            H.mixer_decode(dims, dw, xn, T, cache, ssm, conv, o1, dws)
+            assert H.status_read(dws) == H.ERR_FP16_RANGE, "decode, input scale 1e6"
+    assert H.status_read(ws) == 0   # read-and-clear
 
 
 # ---------------------------------------------------------------------------------------

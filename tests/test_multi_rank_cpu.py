@@ -82,3 +82,11 @@ def test_time_oracle_small_sample():
     """The cpu_baseline leg times the oracle on a bounded sample of the SWA workload."""
     rate, el, reps = bench.time_oracle(16, 0.0)
     assert rate > 0 and reps >= 1 and el > 0
+
+
+def test_reference_arm_runs_exactly_the_reported_steps():
+    """The reference arm times exactly `steps` oracle steps after `warmup` untimed ones, each a
+    bounded sample of the workload (here the smallest, 64 input tokens)."""
+    rate, ms, n, el = bench.reference_steps(2, 1, total_budget_s=0.0)
+    assert n == 64 and rate > 0
+    assert ms == pytest.approx(1000.0 * el / 2)

@@ -1,6 +1,6 @@
 """hymba_mixer_decode_noalloc: the decode step for callers that cannot allocate device
-memory (inside a CUDA graph capture, in a serving loop that must not take cudaMalloc's
-device synchronisation, or as a plugin whose host runtime owns all device memory).  It
+memory (a serving loop that must not take cudaMalloc's device synchronisation between
+tokens, or a plugin whose host runtime owns all device memory).  It
 keeps its scratch in a built-in device array instead of a caller workspace, so it must give
 the same results as hymba_mixer_decode with a workspace, call after call, although the
 array keeps the previous call's contents.
