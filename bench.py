@@ -89,9 +89,8 @@ def visible_pairs(T, M, W, is_global):
 def scan_chunks(B, Di, T):
     """Time chunks of the selective scan as the library cuts them (chunk length, count): as
     many as keep the output pass's (Di/64) x chunks x B CTAs within one wave of 148 SMs at
-    10 CTAs per SM (8 when the attention runs beside the scan, B*Di < 24*148), length a
-    multiple of 8."""
-    per_sm = 8 if B * Di < 24 * 148 else 10
+    10 CTAs per SM, length a multiple of 8."""
+    per_sm = 10
     c = max(1, min(148 * per_sm // (B * (Di // 64)), -(-T // 8)))
     L = 8 * -(-(-(-T // c)) // 8)
     return L, -(-T // L)
@@ -332,12 +331,14 @@ def run_hymba(args, rank, world, device):
                  "exp2_unit": "T/s", "chunks": scan_chunks(B, dims.d_inner, T)[1]}
     launches_per_step = len(recs) / args.steps   # kernels the library launched per step
 
+    prefix = None if args.no_prefix else run_prefix(args, dims, dw, x, flush, stream, ms_per_step, world)
+
     # ---------------- e2e: host buffers through the C ABI ----------------
     if args.no_e2e:
         decode = None if args.no_decode else run_decode(args, device, world)
         return {"tokens_per_step": B * T, "ms_per_step": ms_per_step, "step_ms_p50": float(np.median(step_ms)),
                 "e2e_ms": float("nan"), "h2d": 0, "d2h": 0, "roofline": roof, "step_roofline": step_roof,
-                "scan_roofline": scan_roof,
+                "scan_roofline": scan_roof, "meta_prefix": prefix,
                 "kernels": kern, "clocks": clk.summary(), "launches_per_step": launches_per_step, "decode": decode}
     # every step copies its input from pinned host memory and its output back inside one C-ABI
     # call (hymba_mixer_prefill_host); two streams alternate steps, as a serving loop with two
@@ -380,11 +381,50 @@ def run_hymba(args, rank, world, device):
         "step_ms_p50": float(np.median(step_ms)),
         "e2e_ms": e2e_ms,
         "h2d": int(xh.numel() * 2), "d2h": int(ohs[0].numel() * 2),
-        "roofline": roof, "step_roofline": step_roof, "scan_roofline": scan_roof, "kernels": kern,
+        "roofline": roof, "step_roofline": step_roof, "scan_roofline": scan_roof, "meta_prefix": prefix,
+        "kernels": kern,
         "clocks": clk.summary(),
         "launches_per_step": launches_per_step, "decode": decode, "dims": dims, "wl": wl,
     }
     return res
+
+
+def run_prefix(args, dims, dw, x, flush, stream, full_ms, world):
+    """The same layer from its precomputed meta-token prefix: the prefix is built once, then
+    each step prefills only the input rows (hymba_mixer_prefill_prefix), L2 flushed between
+    steps.  Reported beside the full step."""
+    import torch
+    from hybrid_attention_ssm_b200 import hymba as H
+
+    B, N = x.shape[0], x.shape[1]
+    M = dims.n_meta
+    meta_out = torch.empty(M, dims.d_model, dtype=torch.bfloat16, device=x.device)
+    bws = H.alloc_workspace(H.workspace_size(dims, 1, M, 1))
+    pre = H.Prefix(dims, dw, dw.t["meta"], meta_out, bws)
+    cache = H.Cache(dims, B, M + N)
+    out = torch.empty(B, N, dims.d_model, dtype=torch.bfloat16, device=x.device)
+    ws = H.alloc_workspace(H.workspace_size(dims, B, N))
+
+    def step():
+        H.mixer_prefill_prefix(dims, dw, x, pre, cache, out, ws)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    n = max(5, min(args.steps, 50))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    assert H.status_read(ws) == 0 and H.status_read(bws) == 0
+    ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in ev])), world, x.device)
+    return {"ms_per_step": round(ms, 5), "input_tokens_per_s": round(whole_job_rate(world, B * N, ms), 1),
+            "full_step_ms": round(full_ms, 5), "saved_frac": round(1.0 - ms / full_ms, 4),
+            "how": "meta-token prefix built once (hymba_meta_prefix_build); each step prefills the "
+                   f"{N} input rows only (hymba_mixer_prefill_prefix)"}
 
 
 def run_decode(args, device, world):
@@ -542,6 +582,30 @@ def run_global(args, device, world):
             "tensor_gflop_per_step": round(flops / 1e9, 1),
             "frac_of_tensor_peak": round(flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
             "kernels": kern}
+
+
+def profile_global(n, device):
+    """n prefills of the global layer and nothing else, for a profiler's launch list."""
+    import torch
+    from hybrid_attention_ssm_b200 import hymba as H
+    from hybrid_attention_ssm_b200 import synth
+
+    wl = synth.workloads()["global"]
+    dims = wl.dims
+    B, N = wl.batch, wl.n_tokens
+    T = dims.n_meta + N
+    w = synth.layer_weights(dims, seed=0, dt_bias_mean=wl.dt_bias_mean, dt_bias_std=wl.dt_bias_std)
+    dw = H.DeviceWeights(w)
+    g = torch.Generator(device=device)
+    g.manual_seed(7)
+    x = torch.randn(B, N, dims.d_model, generator=g, device=device).to(torch.bfloat16)
+    cache = H.Cache(dims, B, T)
+    out = torch.empty(B, T, dims.d_model, dtype=torch.bfloat16, device=device)
+    ws = H.alloc_workspace(H.workspace_size(dims, B, N))
+    for _ in range(n):
+        H.mixer_prefill(dims, dw, x, cache, out, ws)
+    torch.cuda.synchronize()
+    assert H.status_read(ws) == 0
 
 
 def run_stack(args, device, world):
@@ -738,6 +802,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer measurement (profiling runs)")
     ap.add_argument("--no-global", action="store_true", help="skip the global-layer measurement")
     ap.add_argument("--no-stack", action="store_true", help="skip the 32-layer stack measurement")
+    ap.add_argument("--no-prefix", action="store_true", help="skip the precomputed meta-prefix measurement")
+    ap.add_argument("--profile-global", type=int, default=0, metavar="N",
+                    help="profiling runs: only N prefills of the global layer (batch 4, 128 + 8192 "
+                         "tokens), no timing and no JSON line")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -772,6 +840,9 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     device = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(device)
+    if args.profile_global > 0:
+        profile_global(args.profile_global, device)
+        return
     r = run_hymba(args, rank, world, device)
     tokens_per_s = whole_job_rate(world, r["tokens_per_step"], r["ms_per_step"])
     e2e = whole_job_rate(world, r["tokens_per_step"], r["e2e_ms"])
@@ -789,7 +860,7 @@ def main():
             "gpu_launches": int(round(r["launches_per_step"] * args.steps)),
             "step_roofline": r["step_roofline"], "roofline": r["roofline"], "scan_roofline": r["scan_roofline"],
             "clocks": r["clocks"],
-            "kernels": r["kernels"], "decode": r["decode"]}
+            "kernels": r["kernels"], "meta_prefix": r["meta_prefix"], "decode": r["decode"]}
     if not args.no_global:
         line["global_layer"] = run_global(args, device, world)
     if not args.no_stack:

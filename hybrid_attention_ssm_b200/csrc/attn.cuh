@@ -28,9 +28,10 @@ namespace hymba {
 
 struct AttnParams {
   int T;              // rows per sequence (meta included)
+  int q_off;          // first query row (M when the meta rows come from a precomputed prefix)
   int Hq, Hkv;
   int n_meta, window, is_global;
-  int q_tiles;
+  int q_tiles;        // tiles of 128 query rows over rows q_off .. T-1
   int n_items;        // q_tiles * Hq * B work items
   float scale_log2;   // log2(e) / sqrt(head_dim)
   float* out;         // O [B*T, ld_out] fp32, head h at columns h*64
@@ -73,7 +74,7 @@ struct KeyTiles {
 
 __device__ __forceinline__ KeyTiles key_tiles(const AttnParams& p, int qt) {
   KeyTiles kt;
-  const int t0 = qt * 128;
+  const int t0 = p.q_off + qt * 128;
   const int t1 = min(t0 + 127, p.T - 1);
   kt.hi = t1 >> 7;
   if (p.is_global) {
@@ -228,7 +229,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
         const KeyTiles kts = key_tiles(p, qt);
         if (it > 0 && !mbar_wait(q_empty, (it - 1) & 1u, abort_flag, p.status, 200)) { ok = false; break; }
         mbar_arrive_expect_tx(q_full, ATT_Q_BYTES);
-        tma_load_3d(smem + ATT_OFF_Q, &mapQ, q_full, h * 64, qt * 128, b);
+        tma_load_3d(smem + ATT_OFF_Q, &mapQ, q_full, h * 64, p.q_off + qt * 128, b);
         for (int i = 0; i < kts.count(); ++i, ++gi) {
           const int s = gi % ATT_STAGES;
           if (!mbar_wait(&kv_empty[s], ((gi / ATT_STAGES) & 1u) ^ 1u, abort_flag, p.status, 201)) {
@@ -314,7 +315,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       attn_item(p, w, B, qt, h, b);
       const KeyTiles kts = key_tiles(p, qt);
       const int n_tiles = kts.count();
-      const int t0 = qt * 128;
+      const int t0 = p.q_off + qt * 128;
       const int qi = t0 + r;                     // absolute query position
       float m_run = -INFINITY, l_run = 0.f;
       for (int i = 0; i < n_tiles; ++i, ++gi) {

@@ -82,27 +82,42 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same test, but a thread whose phase is not complete is suspended (it issues nothing)
+// until the phase completes or about `hint_ns` have passed, whichever comes first.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait on phase `parity` of `bar`.  Returns false (and records the site in the
 // status word) when the wait exceeds g_wait_limit_ns, or when another warp of the CTA has
 // already given up (`*abort` set), so that no wait in these kernels can spin forever.
-// The clock is read only once a wait has polled 256 times: most waits in a pipeline end
-// within a few polls, and reading the global timer on every wait cost about a microsecond
-// per hand-off.  The limit is measured from that first reading.
+// A few quick polls first (most waits in a pipeline end within them); then each poll
+// suspends the waiting thread for up to 20 us or until the phase completes, so a waiting
+// warp takes no issue slots from the warps that are working.  The clock is read once per
+// suspended poll; the limit is measured from the first reading.
 static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
                                                    DevStatus* st, unsigned site) {
-  uint64_t t0 = 0;
-  for (uint32_t it = 1;; ++it) {
+  for (int it = 0; it < 16; ++it)
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0u) {
-      if (abort != nullptr && *abort) return false;
-      const uint64_t now = globaltimer_ns();
-      if (t0 == 0) {
-        t0 = now;
-      } else if (now - t0 > g_wait_limit_ns) {
-        if (abort != nullptr) *abort = 1;
-        report_error(st, DEV_ERR_TIMEOUT, site);
-        return false;
-      }
+  uint64_t t0 = 0;
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if (abort != nullptr && *abort) return false;
+    const uint64_t now = globaltimer_ns();
+    if (t0 == 0) {
+      t0 = now;
+    } else if (now - t0 > g_wait_limit_ns) {
+      if (abort != nullptr) *abort = 1;
+      report_error(st, DEV_ERR_TIMEOUT, site);
+      return false;
     }
   }
 }
@@ -264,6 +279,11 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
@@ -312,7 +332,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-__device__ __forceinline__ float softplus_f(float x) { return x > 20.f ? x : log1pf(expf(x)); }
 
 // hardware base-2 logarithm (MUFU), absolute error ~2^-22
 __device__ __forceinline__ float lg2_approx(float x) {
@@ -320,6 +339,21 @@ __device__ __forceinline__ float lg2_approx(float x) {
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+
+// softplus(x) = log(1 + e^x) with CUDA's expf/log1pf (the decode step's form)
+__device__ __forceinline__ float softplus_f(float x) { return x > 20.f ? x : log1pf(expf(x)); }
+
+// softplus(x) = log(1 + e^x) from the hardware ex2/lg2, branch-free for the epilogue: x for
+// x > 15 (the remainder is below 3.1e-7); with u = e^x, log1p(u) = ln2 * log2(1 + u) for
+// u >= 2^-7 (relative error below 3e-5 there), and the series u - u^2/2 + u^3/3 below
+// (error below u^4/4).
+__device__ __forceinline__ float softplus_sel(float x) {
+  const float u = ex2_approx(fminf(x, 15.f) * 1.4426950408889634f);
+  const float small = u * (1.f - u * (0.5f - u * 0.33333334f));
+  const float big = lg2_approx(1.f + u) * 0.6931471805599453f;
+  return x > 15.f ? x : (u < 0.0078125f ? small : big);
+}
+
 __device__ __forceinline__ float rcp_approx(float x) {
   float y;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

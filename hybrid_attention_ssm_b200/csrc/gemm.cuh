@@ -20,7 +20,7 @@ enum EpiMode : int {
   EPI_PROJ = 0,         // segmented bf16/fp16 stores with RoPE on marked segments (in_proj)
   EPI_BF16 = 1,         // bf16 store, optional bf16 residual add
   EPI_SWIGLU = 2,       // columns interleaved [gate(32) | up(32)] -> fp16 SiLU(gate)*up
-  EPI_SOFTPLUS = 3,     // fp32 softplus(acc + bias[col]), row-major: out[row * ld_out + col]
+  EPI_F32_ROWS = 3,     // fp32 row-major store out[row * ld_out + col], 128-byte rows per store
   EPI_F32_T = 4,        // transposed fp32 store: out[n][m] (weights as the M operand)
   EPI_F32_PART = 5,     // fp32 store of split ks's partial sum at out + ks*split_stride (row-major)
   EPI_F32_T_PART = 6,   // the same, transposed
@@ -51,6 +51,10 @@ struct GemmParams {
   // output row mapping: a source-0 row r goes to rows {b*T_out + r}, b < out_batches;
   // a source-1 row (b, r) goes to b*T_out + row_off1 + r (position row_off1 + r)
   int out_batches, T_out, row_off1;
+  // 1: only the epilogue warps wait for the previous kernel on the stream.  For a GEMM whose
+  // operands no kernel of the same call writes (the caller's input and the weights), so the
+  // mainloop overlaps a previous kernel that only prepares what the epilogue reads.
+  int wait_late;
   void* out;
   long long split_stride;   // elements between the partial-sum slices of two splits
   int ld_out;
@@ -69,10 +73,10 @@ constexpr int GEMM_EPI_WARPS = 8;
 constexpr int GEMM_THREADS = 64 + 32 * GEMM_EPI_WARPS;
 constexpr int GEMM_BM = 128;
 
-// Shared memory an epilogue stages its output through: EPI_SOFTPLUS transposes each warp's
+// Shared memory an epilogue stages its output through: EPI_F32_ROWS transposes each warp's
 // 32 x 32 fp32 block (rows padded to 33 words) so that every store writes one whole row.
 __host__ __device__ constexpr int gemm_epi_bytes(int mode) {
-  return mode == 3 /* EPI_SOFTPLUS */ ? GEMM_EPI_WARPS * 32 * 33 * 4 : 0;
+  return mode == 3 /* EPI_F32_ROWS */ ? GEMM_EPI_WARPS * 32 * 33 * 4 : 0;
 }
 
 template <int BN, int STAGES, int EPI_BYTES = 0>
@@ -121,17 +125,6 @@ __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t* r) {
         "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
       :
       : "memory");
-}
-
-// softplus(x) = log(1 + e^x) from the hardware ex2/lg2, branch-free for the epilogue: x for
-// x > 15 (the remainder is below 3.1e-7); with u = e^x, log1p(u) = ln2 * log2(1 + u) for
-// u >= 2^-7 (relative error below 3e-5 there), and the series u - u^2/2 + u^3/3 below
-// (error below u^4/4).
-__device__ __forceinline__ float softplus_sel(float x) {
-  const float u = ex2_approx(fminf(x, 15.f) * 1.4426950408889634f);
-  const float small = u * (1.f - u * (0.5f - u * 0.33333334f));
-  const float big = lg2_approx(1.f + u) * 0.6931471805599453f;
-  return x > 15.f ? x : (u < 0.0078125f ? small : big);
 }
 
 // element types of both operands: bf16, fp16 (kind::f16) or fp32 read as tf32 (kind::tf32)
@@ -189,7 +182,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   // parameters, so it overlaps the previous kernel's tail.  Every access to global memory
   // comes after the wait.  A CTA launched early can only meet TMEM held by CTAs of the
   // previous kernel, which are all running by then and free it when they finish.
-  pdl_wait();
+  if (!p.wait_late || warp >= 2) pdl_wait();
   pdl_trigger();
 
   if (warp == 0) {
@@ -360,13 +353,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             }
             return;
           }
-          if constexpr (MODE == EPI_SOFTPLUS) {
-            // softplus(acc + bias) of the warp's 32 rows x 32 columns, transposed through this
-            // warp's shared tile: lane j then stores column gc + j of row r, 128-byte rows
+          if constexpr (MODE == EPI_F32_ROWS) {
+            // the warp's 32 rows x 32 columns, transposed through this warp's shared tile:
+            // lane j then stores column gc + j of row r, 128-byte rows
             if (gc >= p.n_valid) return;          // the same for the whole warp
             float* tile = reinterpret_cast<float*>(smem + L::EPI_OFFSET) + (warp - 2) * (32 * 33);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) tile[lane * 33 + e] = softplus_sel(v[e] + p.bias[min(gc + e, p.n_valid - 1)]);
+            for (int e = 0; e < 32; ++e) tile[lane * 33 + e] = v[e];
             __syncwarp();
             const int rows_valid = src0 ? p.rows0 : p.rows1;
             const int rr0 = rr - lane;            // accumulator row of lane 0

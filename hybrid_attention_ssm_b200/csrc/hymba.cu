@@ -145,11 +145,10 @@ ProfState g_prof;
 
 // ----------------------------------------------------------------------------------------
 // A library-owned side stream per (host thread, device) for the attention branch of a
-// prefill: it forks from the caller's stream after in_proj and joins before the branch norm
-// through two events, so the attention runs beside the conv -> x_proj -> dt_proj -> scan
-// chain (the scan alone leaves most of each SM idle at small batch).  Event fork/join is
-// also how stream capture follows work onto another stream, so a captured prefill becomes
-// a graph with two parallel branches.
+// decode step: it forks from the caller's stream after the decode prep kernel and joins
+// before the branch norm through two events, so the attention runs beside x_proj and the
+// SSM step.  Event fork/join is also how stream capture follows work onto another stream,
+// so a captured decode step becomes a graph with two parallel branches.
 // ----------------------------------------------------------------------------------------
 struct SideStream {
   cudaStream_t s = nullptr;
@@ -254,9 +253,9 @@ template <int ET, int MODE>
 int launch_gemm_bn(int bn, const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& mb, const GemmParams& p,
                    int grid, cudaStream_t st, const char* name) {
   constexpr bool any_bn = MODE == EPI_F32_PART || MODE == EPI_F32_T || MODE == EPI_F32_T_PART;
-  if constexpr (MODE == EPI_SOFTPLUS) {   // short K (dt_rank): 4 stages, room for the staging tiles
+  if constexpr (MODE == EPI_F32_ROWS) {   // short K (dt_rank): 4 stages, room for the staging tiles
     if (bn == 128) return launch_gemm_inst<128, 4, ET, MODE>(m0, m1, mb, p, grid, st, name);
-    return fail(HYMBA_ERR_UNSUPPORTED, "no GEMM instance for tile width %d with the softplus epilogue", bn);
+    return fail(HYMBA_ERR_UNSUPPORTED, "no GEMM instance for tile width %d with the row-store epilogue", bn);
   }
   if (bn == 256) return launch_gemm_inst<256, 4, ET, MODE>(m0, m1, mb, p, grid, st, name);
   if constexpr (MODE != EPI_PROJ) {
@@ -288,8 +287,8 @@ int launch_gemm_mode(const GemmCall& c, const CUtensorMap& m0, const CUtensorMap
     case EPI_SWIGLU:
       if (c.etype == ET_BF16) return launch_gemm_bn<ET_BF16, EPI_SWIGLU>(c.bn, m0, m1, mb, p, grid, st, c.name);
       break;
-    case EPI_SOFTPLUS:
-      if (c.etype == ET_TF32) return launch_gemm_bn<ET_TF32, EPI_SOFTPLUS>(c.bn, m0, m1, mb, p, grid, st, c.name);
+    case EPI_F32_ROWS:
+      if (c.etype == ET_TF32) return launch_gemm_bn<ET_TF32, EPI_F32_ROWS>(c.bn, m0, m1, mb, p, grid, st, c.name);
       break;
     case EPI_F32_T:
       if (c.etype == ET_BF16) return launch_gemm_bn<ET_BF16, EPI_F32_T>(c.bn, m0, m1, mb, p, grid, st, c.name);
@@ -491,18 +490,18 @@ int splits_for(int tiles, int k_blocks, int cap) {
 }
 
 struct PrefillWs {
-  size_t q, xz, xc, xbc, xbc_part, delta, carry, sumd, y, o, u, sstate, cstate, rope, total;
+  size_t q, xz, xc, xbc, xbc_part, dt_pre, carry, sumd, y, o, u, sstate, cstate, rope, total;
   int T, xproj_split, scan_L, scan_chunks;
 };
 // Time chunks of the selective scan.  Every chunk of a pass runs at once: the CTAs of the
 // output pass, (Di / 64) x n_chunks x B, must fit in one wave of a B200's 148 SMs, else a
-// second wave doubles the time of the serial walk over a chunk.  An SM holds 10 scan CTAs
-// (registers), 8 beside the attention CTA when the two branches overlap (small batch, as
-// the prefill decides).  Within that, as many chunks as fit: shorter chunks, shorter walk.
+// second wave doubles the time of the serial walk over a chunk.  An SM holds SC_PER_SM scan
+// CTAs (registers).  Within that, as many chunks as fit: shorter chunks, shorter walk.
 // Fixed to 148 SMs so that workspace sizes do not depend on the device; the chunk length
 // is a multiple of the scan's TMA stage.
-void scan_chunking(int B, int Di, int T, int* L, int* n_chunks) {
-  const long long per_sm = (long long)B * Di < 24LL * 148 ? 8 : 10;
+// *cap is the most chunks any row count up to T gets (the chunk buffers are sized for it).
+void scan_chunking(int B, int Di, int T, int* L, int* n_chunks, int* cap = nullptr) {
+  const long long per_sm = SC_PER_SM;
   const long long groups = (long long)B * (Di / SC_CH);
   long long c = 148LL * per_sm / groups;
   const long long cmax = (T + SC_SUB - 1) / SC_SUB;
@@ -511,11 +510,16 @@ void scan_chunking(int B, int Di, int T, int* L, int* n_chunks) {
   const int len = SC_SUB * cdiv(cdiv(T, c), SC_SUB);
   *L = len;
   *n_chunks = cdiv(T, len);
+  if (cap != nullptr) *cap = (int)c;
 }
-PrefillWs prefill_layout(const Dims& m, int B, int n_tokens, int x_has_meta) {
+// scan_from: the first row the scan walks (M when the meta rows come from a precomputed
+// prefix); the chunk buffers come last, so the other offsets do not depend on it.
+PrefillWs prefill_layout(const Dims& m, int B, int n_tokens, int x_has_meta, int scan_from = 0) {
   PrefillWs w;
   w.T = x_has_meta ? n_tokens : m.M + n_tokens;
-  scan_chunking(B, m.Di, w.T, &w.scan_L, &w.scan_chunks);
+  int cap = 1;
+  scan_chunking(B, m.Di, w.T, &w.scan_L, &w.scan_chunks, &cap);   // cap: for any rows <= T
+  if (scan_from > 0) scan_chunking(B, m.Di, w.T - scan_from, &w.scan_L, &w.scan_chunks);
   const size_t rows = (size_t)B * w.T;
   size_t off = 256;
   auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
@@ -525,15 +529,15 @@ PrefillWs prefill_layout(const Dims& m, int B, int n_tokens, int x_has_meta) {
   w.xbc = take(rows * m.ld_xbc * 4);
   w.xproj_split = splits_for(cdiv((long long)rows, GEMM_BM), cdiv(m.Di, 64), 16);
   w.xbc_part = take((size_t)w.xproj_split * rows * m.ld_xbc * 4);
-  w.delta = take(rows * m.Di * 4);
-  w.carry = take((size_t)B * (w.scan_chunks - 1) * m.Di * 16 * 4);
-  w.sumd = take((size_t)B * (w.scan_chunks - 1) * m.Di * 4);
+  w.dt_pre = take(rows * m.Di * 4);
   w.y = take(rows * m.Di * 2);
   w.o = take(rows * m.qw * 4);
   w.u = take(rows * m.uw * 2);
   w.sstate = take((size_t)B * m.Di * 16 * 4);
   w.cstate = take((size_t)B * m.Di * 3 * 4);
   w.rope = take((size_t)w.T * 32 * 8);
+  w.carry = take((size_t)B * (cap - 1) * m.Di * 16 * 4);
+  w.sumd = take((size_t)B * (cap - 1) * m.Di * 4);
   w.total = off;
   return w;
 }
@@ -695,7 +699,7 @@ int hymba_mixer_stage_layout(const hymba_layer_cfg* cfg, int batch, int n_tokens
   if (out == nullptr || batch < 1 || n_tokens < 1) return fail(HYMBA_ERR_INVALID_ARG, "stage layout args");
   const Dims m = dims_of(cfg);
   const PrefillWs w = prefill_layout(m, batch, n_tokens, x_has_meta);
-  out->q = w.q; out->xz = w.xz; out->xc = w.xc; out->xbc = w.xbc; out->delta = w.delta;
+  out->q = w.q; out->xz = w.xz; out->xc = w.xc; out->xbc = w.xbc; out->dt_pre = w.dt_pre;
   out->y = w.y; out->o = w.o; out->u = w.u;
   out->ld_xbc = m.ld_xbc;
   out->scan_chunks = w.scan_chunks;
@@ -822,20 +826,31 @@ int hymba_kv_share_alloc(const hymba_layer_cfg* base, int n_layers, const uint8_
   return HYMBA_OK;
 }
 
-int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x,
-                        int x_has_meta, int B, int n_tokens, hymba_kv_cache* kv, float* ssm_state_out,
-                        float* conv_state_out, const hymba_bf16* residual, hymba_bf16* out, void* ws,
-                        size_t ws_bytes, hymba_stream stream) {
+// The prefill.  prefix == NULL: every row, meta rows included.  Otherwise the meta rows come
+// from `prefix` (x holds only the input rows, x_has_meta == 0): their K/V are copied into the
+// cache, the conv and the scan start from the prefix states, and only rows M..T-1 are
+// computed; out and residual then hold those rows only, [B, n_tokens, d].
+static int prefill_impl(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x,
+                        int x_has_meta, int B, int n_tokens, const hymba_meta_prefix* prefix, hymba_kv_cache* kv,
+                        float* ssm_state_out, float* conv_state_out, const hymba_bf16* residual, hymba_bf16* out,
+                        void* ws, size_t ws_bytes, hymba_stream stream) {
   HY_TRY(check_cfg(cfg));
   DeviceInfo* dev = nullptr;
   HY_TRY(device_info(&dev));
   const Dims m = dims_of(cfg);
   if (B < 1 || n_tokens < 1) return fail(HYMBA_ERR_INVALID_ARG, "batch %d / n_tokens %d", B, n_tokens);
-  HY_TRY(check_weights(w, m, !x_has_meta));
+  HY_TRY(check_weights(w, m, !x_has_meta && prefix == nullptr));
   if (x == nullptr || out == nullptr || kv == nullptr || !aligned16(x) || !aligned16(out))
     return fail(HYMBA_ERR_INVALID_ARG, "x/out/kv pointer");
   if (residual != nullptr && !aligned16(residual)) return fail(HYMBA_ERR_INVALID_ARG, "residual alignment");
-  const PrefillWs L = prefill_layout(m, B, n_tokens, x_has_meta);
+  const int P0 = prefix != nullptr ? m.M : 0;   // first row computed
+  if (prefix != nullptr) {
+    if (x_has_meta) return fail(HYMBA_ERR_INVALID_ARG, "a precomputed prefix needs x without the meta rows");
+    if (prefix->ssm_state == nullptr || prefix->conv_state == nullptr || !aligned16(prefix->ssm_state) ||
+        (m.M > 0 && (prefix->k == nullptr || prefix->v == nullptr || !aligned16(prefix->k) || !aligned16(prefix->v))))
+      return fail(HYMBA_ERR_INVALID_ARG, "meta prefix pointers");
+  }
+  const PrefillWs L = prefill_layout(m, B, n_tokens, x_has_meta, P0);
   const int T = L.T;
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return fail(HYMBA_ERR_INVALID_ARG, "workspace");
   if (ws_bytes < L.total) return fail(HYMBA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
@@ -865,10 +880,26 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
+  // the meta rows' K/V from the prefix: into the prefill view and, for an SWA cache, its meta rows
+  if (prefix != nullptr && own_kv && m.M > 0) {
+    const bool swa = !cfg->is_global && kv->kind == HYMBA_CACHE_SWA;
+    const int row_vec = m.kvw / 8;   // 16-byte pieces per position
+    const long long n = (long long)B * m.M * row_vec;
+    prof_begin("prefix_kv", st);
+    HY_CUDA(launch_pdl(prefix_kv_kernel, dim3(cdiv(n, 256)), dim3(256), 0, st,
+                       reinterpret_cast<const __half*>(prefix->k), reinterpret_cast<const __half*>(prefix->v), B, m.M,
+                       row_vec, reinterpret_cast<__half*>(kv->k), reinterpret_cast<__half*>(kv->v), Lmax,
+                       swa ? reinterpret_cast<__half*>(kv->meta_k) : (__half*)nullptr,
+                       swa ? reinterpret_cast<__half*>(kv->meta_v) : (__half*)nullptr));
+    prof_end(st);
+  }
   // 1. in_proj with RoPE on Q/K, scattering Q, K, V, x|z
   {
     GemmCall c;
-    if (!x_has_meta && m.M > 0) {
+    if (prefix != nullptr) {   // the input rows only, at positions M..T-1
+      c.a1 = x; c.nb1 = B; c.rows1 = n_tokens; c.lda1 = m.d; c.a1_bstride = (long long)n_tokens * m.d;
+      c.p.row_off1 = m.M;
+    } else if (!x_has_meta && m.M > 0) {
       c.a0 = w->meta; c.rows0 = m.M; c.lda0 = m.d;
       c.a1 = x; c.nb1 = B; c.rows1 = n_tokens; c.lda1 = m.d; c.a1_bstride = (long long)n_tokens * m.d;
       c.p.row_off1 = m.M;
@@ -905,17 +936,19 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     c.p.seg[ns++] = Segment{m.xz_off, m.xz_off + 2 * m.Di, bf(L.xz), (long long)T * 2 * m.Di, 2 * m.Di, 0, 0};
     c.p.nseg = ns;
     c.p.rope_tab = reinterpret_cast<const float2*>(wsb + L.rope);
+    // x and W_in are inputs of the call: the mainloop may start while the RoPE table (read
+    // only by the epilogue) is still being written.  A kernel before the table kernel has
+    // completed by then: the table kernel waits for it before it lets this one launch.
+    c.p.wait_late = 1;
     HY_TRY(run_gemm(c, *dev, st));
   }
-  SideStream* side = nullptr;
-  HY_TRY(side_stream(&side));
-  // 2. conv1d + SiLU (writes xc, xcT and the conv state)
+  // 2. conv1d + SiLU (writes xc and the conv state)
   float* cstate = conv_state_out != nullptr ? conv_state_out : f32(L.cstate);
   {
-    dim3 grid(m.Di / CONV_TC, cdiv(T, CONV_TT), B);
+    dim3 grid(m.Di / CONV_TC, cdiv(T - P0, CONV_TT), B);
     prof_begin("conv1d_silu", st);
     HY_CUDA(launch_pdl(conv1d_silu_kernel, grid, dim3(256), 0, st, bf(L.xz), 2 * m.Di, w->conv_w, w->conv_b, bf(L.xc),
-                       cstate, T, m.Di));
+                       cstate, T, m.Di, P0, prefix != nullptr ? prefix->conv_state : (const float*)nullptr));
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
@@ -941,7 +974,8 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
-  // 4. dt_proj (tf32) with softplus(+bias): delta [B*T, Di] fp32
+  // 4. dt_proj (tf32): dt_pre = dt_low W_dt^T [B*T, Di] fp32 (the scan adds dt_bias and
+  //    applies the softplus as it reads it)
   {
     GemmCall c;
     c.etype = ET_TF32;
@@ -949,26 +983,16 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     c.b = w->w_dt; c.N = m.Di; c.ldb = w->w_dt_ld; c.K = m.R;
     c.bn = 128;
     c.name = "dt_proj";
-    c.mode = EPI_SOFTPLUS;
-    c.p.out = f32(L.delta);
+    c.mode = EPI_F32_ROWS;
+    c.p.out = f32(L.dt_pre);
     c.p.ld_out = m.Di;
-    c.p.bias = w->dt_bias;
     c.p.n_valid = m.Di;
     c.p.status = status;
     HY_TRY(run_gemm(c, *dev, st));
   }
-  // 5. attention (block-skipped SWA + meta, or global causal).  At small batch (fewer than
-  //    24 channels x sequences per SM) the attention forks onto the side stream after dt_proj
-  //    and runs beside the scan: both leave most of an SM's issue slots idle at that size and
-  //    fit on one SM together (one 2-stage attention CTA beside the scan's small CTAs).
-  //    Otherwise it runs in stream order.
-  const bool overlap = (long long)B * m.Di < 24LL * dev->sms;
-  ForkGuard fork_guard(side, st);
-  if (overlap) {
-    HY_CUDA(cudaEventRecord(side->fork, st));
-    HY_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
-    fork_guard.open = true;
-  }
+  // 5. attention (block-skipped SWA + meta, or global causal), 3-stage ring, two CTAs per
+  //    SM.  (Run beside the scan on a second stream instead, it gained nothing: the two
+  //    compete for the same registers, and the scan then needed two waves.)
   {
     CUtensorMap mq, mk, mv;
     const uint32_t box[3] = {64, 128, 1};
@@ -985,18 +1009,14 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     }
     AttnParams ap;
     ap.T = T; ap.Hq = m.Hq; ap.Hkv = m.Hkv; ap.n_meta = m.M; ap.window = m.W; ap.is_global = cfg->is_global;
-    ap.q_tiles = cdiv(T, 128);
+    ap.q_off = P0;
+    ap.q_tiles = cdiv(T - P0, 128);
     ap.n_items = ap.q_tiles * m.Hq * B;
     ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)m.D));
     ap.out = f32(L.o);
     ap.ld_out = m.qw;
     ap.status = status;
-    if (overlap) {   // beside the scan: 2-stage ring, one CTA per SM, on the side stream
-      HY_TRY(launch_attention<2>(mq, mk, mv, ap, B, ap.n_items < dev->sms ? ap.n_items : dev->sms, side->s));
-    } else {         // alone: 3-stage ring, two CTAs per SM, in stream order
-      HY_TRY(launch_attention<3>(mq, mk, mv, ap, B, ap.n_items < 2 * dev->sms ? ap.n_items : 2 * dev->sms, st));
-    }
-    if (overlap) HY_CUDA(cudaEventRecord(side->join, side->s));
+    HY_TRY(launch_attention<3>(mq, mk, mv, ap, B, ap.n_items < 2 * dev->sms ? ap.n_items : 2 * dev->sms, st));
   }
   // 6. selective scan in time chunks: chunk end states, carry, outputs
   float* sstate = ssm_state_out != nullptr ? ssm_state_out : f32(L.sstate);
@@ -1007,7 +1027,7 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
       const uint64_t dims[2] = {(uint64_t)m.Di, (uint64_t)rows};
       const uint64_t str[1] = {(uint64_t)m.Di * 4};
       const uint32_t box[2] = {SC_CH, SC_SUB};
-      HY_TRY(make_map(&md, f32(L.delta), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE));
+      HY_TRY(make_map(&md, f32(L.dt_pre), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE));
     }
     {
       const uint64_t dims[2] = {(uint64_t)m.Di, (uint64_t)rows};
@@ -1024,7 +1044,10 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     }
     ScanParams sp;
     sp.T = T; sp.Di = m.Di; sp.L = L.scan_L; sp.n_chunks = L.scan_chunks;
+    sp.t_begin = P0;
+    sp.h0 = prefix != nullptr ? prefix->ssm_state : nullptr;
     sp.A = w->A;
+    sp.dt_bias = w->dt_bias;
     sp.carry = f32(L.carry);
     sp.sumd = f32(L.sumd);
     sp.y = bf(L.y);
@@ -1053,11 +1076,7 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
                        md, mx, mbc, sp));
     prof_end(st);
   }
-  // 7. per-branch RMSNorm, gate, beta, average (the attention branch joins here)
-  if (overlap) {
-    HY_CUDA(cudaStreamWaitEvent(st, side->join, 0));
-    fork_guard.open = false;
-  }
+  // 7. per-branch RMSNorm, gate, beta, average
   {
     prof_begin("norm_avg", st);
     HY_TRY(launch_branch_norm<__nv_bfloat16>(f32(L.o), m.qw, m.qw, bf(L.y), m.Di, bf(L.xz) + m.Di, 2 * m.Di, m.Di,
@@ -1066,14 +1085,19 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
-  // 8. out_proj (+ residual)
+  // 8. out_proj (+ residual); with a prefix, rows M..T-1 of each sequence into out [B, N, d]
   {
     GemmCall c;
-    c.a1 = h16(L.u); c.nb1 = 1; c.rows1 = (int)rows; c.lda1 = m.uw; c.a1_bstride = (long long)rows * m.uw;
+    if (prefix != nullptr) {
+      c.a1 = h16(L.u) + (size_t)P0 * m.uw; c.nb1 = B; c.rows1 = n_tokens; c.lda1 = m.uw;
+      c.a1_bstride = (long long)T * m.uw;
+    } else {
+      c.a1 = h16(L.u); c.nb1 = 1; c.rows1 = (int)rows; c.lda1 = m.uw; c.a1_bstride = (long long)rows * m.uw;
+    }
     c.b = w->w_out; c.N = m.d; c.ldb = m.uw; c.K = m.uw;
     c.etype = ET_F16;
     c.name = "out_proj";
-    c.bn = pick_bn_rounds(cdiv(rows, GEMM_BM), m.d, dev->sms, {256, 224, 128});
+    c.bn = pick_bn_rounds(c.nb1 * cdiv(c.rows1, GEMM_BM), m.d, dev->sms, {256, 224, 128});
     c.mode = EPI_BF16;
     c.p.out = out;
     c.p.ld_out = m.d;
@@ -1084,6 +1108,76 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     HY_TRY(run_gemm(c, *dev, st));
   }
   return HYMBA_OK;
+}
+
+int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x,
+                        int x_has_meta, int B, int n_tokens, hymba_kv_cache* kv, float* ssm_state_out,
+                        float* conv_state_out, const hymba_bf16* residual, hymba_bf16* out, void* ws,
+                        size_t ws_bytes, hymba_stream stream) {
+  return prefill_impl(cfg, w, x, x_has_meta, B, n_tokens, nullptr, kv, ssm_state_out, conv_state_out, residual, out,
+                      ws, ws_bytes, stream);
+}
+
+int hymba_mixer_prefill_prefix(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x, int B,
+                               int n_tokens, const hymba_meta_prefix* prefix, hymba_kv_cache* kv,
+                               float* ssm_state_out, float* conv_state_out, const hymba_bf16* residual,
+                               hymba_bf16* out, void* ws, size_t ws_bytes, hymba_stream stream) {
+  if (prefix == nullptr) return fail(HYMBA_ERR_INVALID_ARG, "prefix is NULL");
+  return prefill_impl(cfg, w, x, 0, B, n_tokens, prefix, kv, ssm_state_out, conv_state_out, residual, out, ws,
+                      ws_bytes, stream);
+}
+
+int hymba_meta_prefix_size(const hymba_layer_cfg* cfg, size_t* bytes) {
+  HY_TRY(check_cfg(cfg));
+  if (bytes == nullptr) return fail(HYMBA_ERR_INVALID_ARG, "bytes is NULL");
+  const Dims m = dims_of(cfg);
+  const size_t kv = align256((size_t)(m.M > 0 ? m.M : 1) * m.kvw * 2);
+  *bytes = 2 * kv + align256((size_t)m.Di * 16 * 4) + align256((size_t)m.Di * 3 * 4);
+  return HYMBA_OK;
+}
+
+int hymba_meta_prefix_build(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* meta_rows,
+                            void* buf, size_t buf_bytes, const hymba_meta_prefix* producer,
+                            hymba_meta_prefix* prefix, hymba_bf16* meta_out, void* ws, size_t ws_bytes,
+                            hymba_stream stream) {
+  HY_TRY(check_cfg(cfg));
+  const Dims m = dims_of(cfg);
+  if (m.M < 1) return fail(HYMBA_ERR_INVALID_ARG, "n_meta is 0: there is no prefix");
+  if (meta_rows == nullptr || buf == nullptr || prefix == nullptr || meta_out == nullptr ||
+      (reinterpret_cast<uintptr_t>(buf) & 255u))
+    return fail(HYMBA_ERR_INVALID_ARG, "meta_rows/buf/prefix/meta_out NULL or buf not 256-byte aligned");
+  size_t need = 0;
+  HY_TRY(hymba_meta_prefix_size(cfg, &need));
+  if (buf_bytes < need) return fail(HYMBA_ERR_WORKSPACE, "prefix buffer %zu < %zu bytes", buf_bytes, need);
+  const bool consumer = cfg->kv_role == HYMBA_KV_CONSUMER;
+  if (consumer && (producer == nullptr || producer->k == nullptr || producer->v == nullptr))
+    return fail(HYMBA_ERR_INVALID_ARG, "a consumer layer's prefix needs its producer's prefix K/V");
+  uint8_t* p = static_cast<uint8_t*>(buf);
+  const size_t kvb = align256((size_t)m.M * m.kvw * 2);
+  prefix->k = reinterpret_cast<hymba_f16*>(p);
+  prefix->v = reinterpret_cast<hymba_f16*>(p + kvb);
+  prefix->ssm_state = reinterpret_cast<float*>(p + 2 * kvb);
+  prefix->conv_state = reinterpret_cast<float*>(p + 2 * kvb + align256((size_t)m.Di * 16 * 4));
+  // the M meta rows alone, as one sequence: their K/V go straight into the prefix (a
+  // one-sequence cache of M positions; a consumer reads its producer's), the states after
+  // them into the prefix, their outputs to meta_out
+  hymba_kv_cache c;
+  memset(&c, 0, sizeof(c));
+  c.kind = HYMBA_CACHE_GLOBAL;
+  c.batch = 1;
+  c.n_kv_heads = m.Hkv;
+  c.head_dim = m.D;
+  c.n_meta = m.M;
+  c.window = m.W;
+  c.max_tokens = m.M;
+  c.k = consumer ? const_cast<hymba_f16*>(producer->k) : prefix->k;
+  c.v = consumer ? const_cast<hymba_f16*>(producer->v) : prefix->v;
+  if (consumer) {
+    prefix->k = producer->k;
+    prefix->v = producer->v;
+  }
+  return prefill_impl(cfg, w, meta_rows, 1, 1, m.M, nullptr, &c, prefix->ssm_state, prefix->conv_state, nullptr,
+                      meta_out, ws, ws_bytes, stream);
 }
 
 int hymba_mixer_prefill_host(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x_host,
@@ -1255,7 +1349,9 @@ static int decode_impl(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
       HY_CUDA(cudaFuncSetAttribute(decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DA_SMEM));
       attr_da[dcur & 63] = true;
     }
-    // three CTAs per SM (four would fit) leave room for the SSM step running beside it
+    // three CTAs per SM (four would fit).  (Measured: this order, with x_proj and the SSM
+    // step queued behind the attention on the caller's stream, beat both x_proj first with
+    // two attention CTAs per SM and a single stream.)
     const int grid = ap.n_items < 3 * dev->sms ? ap.n_items : 3 * dev->sms;
     HY_CUDA(cudaEventRecord(side->fork, st));   // every host-side check has passed
     HY_CUDA(cudaStreamWaitEvent(ast, side->fork, 0));

@@ -865,6 +865,35 @@ __global__ void wait_timeout_selftest_kernel(DevStatus* st) {
   if (threadIdx.x == 0) mbar_wait(&bar, 0, nullptr, st, 900);
 }
 
+// The meta positions' K/V of a precomputed prefix ([M, Hkv*64] fp16 each, the same for every
+// sequence) copied into rows 0..M-1 of each sequence's prefill view [B, Lmax, Hkv*64] and,
+// when meta_k is set, into an SWA cache's meta rows [B, M, Hkv*64].  One 16-byte piece per
+// thread; row_vec pieces per position.
+__global__ void __launch_bounds__(256)
+    prefix_kv_kernel(const __half* __restrict__ pk, const __half* __restrict__ pv, int B, int M, int row_vec,
+                     __half* __restrict__ vk, __half* __restrict__ vv, int Lmax, __half* __restrict__ mk,
+                     __half* __restrict__ mv) {
+  pdl_wait();
+  pdl_trigger();
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)B * M * row_vec) return;
+  const int q = (int)(i % row_vec);
+  const long long br = i / row_vec;
+  const int r = (int)(br % M);
+  const int b = (int)(br / M);
+  const size_t src = ((size_t)r * row_vec + q) * 8;
+  const uint4 kq = *reinterpret_cast<const uint4*>(pk + src);
+  const uint4 vq = *reinterpret_cast<const uint4*>(pv + src);
+  const size_t dv = (((size_t)b * Lmax + r) * row_vec + q) * 8;
+  *reinterpret_cast<uint4*>(vk + dv) = kq;
+  *reinterpret_cast<uint4*>(vv + dv) = vq;
+  if (mk != nullptr) {
+    const size_t dm = (((size_t)b * M + r) * row_vec + q) * 8;
+    *reinterpret_cast<uint4*>(mk + dm) = kq;
+    *reinterpret_cast<uint4*>(mv + dm) = vq;
+  }
+}
+
 // Fixed-order sum of split-K partial slices: out[i] = sum_s part[s*stride + i] (+ residual),
 // as fp32 or bf16; n is a multiple of 4.  The order never changes, so results are
 // identical from run to run.

@@ -9,6 +9,9 @@ namespace hymba {
 //   x      [B*T, ld_x] bf16, channel c at column c (the x part of the in_proj output)
 //   xc     [B*T, Di]   bf16 row-major (A operand of x_proj and input of the scan)
 //   state  [B, Di, 3]  fp32: the last 3 inputs x[T-3..T-1] (zero before the start)
+// Rows t_begin .. T-1 are computed; inputs before t_begin come from hist [Di, 3] (the
+// inputs t_begin-3 .. t_begin-1, the same for every sequence), or are zero when hist is
+// NULL.
 // ----------------------------------------------------------------------------------------
 constexpr int CONV_K = 4;
 constexpr int CONV_TT = 64;      // time steps per CTA
@@ -22,18 +25,25 @@ constexpr int CONV_P = CONV_TC + 8;   // smem row pitch (16-byte aligned rows)
 __global__ void __launch_bounds__(256)
     conv1d_silu_kernel(const __nv_bfloat16* __restrict__ x, int ld_x, const float* __restrict__ w,
                        const float* __restrict__ bias, __nv_bfloat16* __restrict__ xc,
-                       float* __restrict__ state, int T, int Di) {
+                       float* __restrict__ state, int T, int Di, int t_begin, const float* __restrict__ hist) {
   pdl_wait();
   pdl_trigger();
   __shared__ __align__(16) __nv_bfloat16 xs[CONV_TT + CONV_K - 1][CONV_P];   // rows t0-3 .. t0+63
   __shared__ __align__(16) __nv_bfloat16 orow[CONV_TT][CONV_P];               // [t][c]
-  const int c0 = blockIdx.x * CONV_TC, t0 = blockIdx.y * CONV_TT, b = blockIdx.z;
+  const int c0 = blockIdx.x * CONV_TC, t0 = t_begin + blockIdx.y * CONV_TT, b = blockIdx.z;
   const int tid = threadIdx.x;
   const __nv_bfloat16* xb = x + (size_t)b * T * ld_x + c0;
   for (int i = tid; i < (CONV_TT + CONV_K - 1) * 8; i += 256) {
     const int r = i >> 3, q = i & 7, t = t0 - (CONV_K - 1) + r;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (t >= 0 && t < T) v = *reinterpret_cast<const uint4*>(xb + (size_t)t * ld_x + q * 8);
+    if (t >= t_begin && t < T) {
+      v = *reinterpret_cast<const uint4*>(xb + (size_t)t * ld_x + q * 8);
+    } else if (t < t_begin && t >= t_begin - 3 && hist != nullptr) {
+      __nv_bfloat16 hv[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) hv[e] = __float2bfloat16_rn(hist[(size_t)(c0 + q * 8 + e) * 3 + (t - t_begin + 3)]);
+      v = *reinterpret_cast<const uint4*>(hv);
+    }
     *reinterpret_cast<uint4*>(&xs[r][q * 8]) = v;
   }
   __syncthreads();
@@ -64,6 +74,7 @@ __global__ void __launch_bounds__(256)
           *reinterpret_cast<const uint4*>(&orow[r][q * 8]);
   }
   // conv state: the last 3 inputs x[T-3..T-1] (zero before the start), from the last tile
+  // (the rows before it are in xs too, history included)
   if (t0 + CONV_TT >= T && tid < CONV_TC) {
     float* s0 = state + ((size_t)b * Di + c0 + tid) * 3;
 #pragma unroll
@@ -90,9 +101,11 @@ __global__ void __launch_bounds__(256)
 //           last chunk, the final state.
 // A lane owns one (sequence, channel, chunk) and the channel's 16 states in registers, so
 // y_t = C_t . h_t is a sum inside the lane and B_t, C_t are the same for every lane of the
-// CTA (shared-memory broadcasts).  CTA = 64 channels (two warps) of one chunk; delta
-// [rows, Di] fp32, x [rows, Di] bf16 and (B | C) [rows, 32] fp32 stream in by TMA, 8 steps
-// per stage, all in their row-major producer layouts.
+// CTA (shared-memory broadcasts).  CTA = 64 channels (two warps) of one chunk; dt_pre
+// [rows, Di] fp32 (dt_low W_dt^T), x [rows, Di] bf16 and (B | C) [rows, 32] fp32 stream in by
+// TMA, 8 steps per stage, all in their row-major producer layouts.  dt_proj's bias and
+// softplus are applied here, as each step is read: delta = softplus(dt_pre + dt_bias), in
+// both passes, instead of a pass of their own over [rows, Di].
 // The 16 decays exp(delta A[s]) take 16 MUFU ex2 per step.  When a warp's A rows are the
 // progression A[s] = (s + 1) A[0] (the S4D-real initialisation -[1..16] of the workloads),
 // exp(delta A[s]) = exp(delta A[0])^(s+1): one ex2 and a multiplication tree give all 16.
@@ -103,9 +116,10 @@ constexpr int SC_CH = 64;      // channels per CTA, one lane each
 constexpr int SC_SUB = 8;      // steps per TMA stage
 constexpr int SC_NST = 4;      // ring stages
 constexpr int SC_THREADS = SC_CH;
+constexpr int SC_PER_SM = 10;  // CTAs resident per SM (the register budget of __launch_bounds__)
 
 struct ScStage {
-  float d[SC_SUB][SC_CH];            // delta rows    (box {64, 8} fp32, 2048 B)
+  float d[SC_SUB][SC_CH];            // dt_pre rows   (box {64, 8} fp32, 2048 B)
   __nv_bfloat16 x[SC_SUB][SC_CH];    // x rows        (box {64, 8} bf16, 1024 B)
   float bc[SC_SUB][32];              // B | C rows    (box {32, 8} fp32, 1024 B)
 };
@@ -120,7 +134,10 @@ constexpr int SC_SMEM = (int)sizeof(ScSmem) + 128;   // + alignment slack
 
 struct ScanParams {
   int T, Di, L, n_chunks;
+  int t_begin;           // first row scanned (the chunks cover rows t_begin .. T-1)
+  const float* h0;       // [Di, 16] state before row t_begin, the same for every sequence, or NULL (zero)
   const float* A;        // [Di, 16]
+  const float* dt_bias;  // [Di]
   float* carry;          // [B][n_chunks-1][Di][16]
   float* sumd;           // [B][n_chunks-1][Di]
   __nv_bfloat16* y;      // [B*T, Di]
@@ -155,7 +172,7 @@ __device__ __forceinline__ void scan_decays_pow(float d, float A20, uint64_t* a)
 }
 
 template <bool OUT>
-__global__ void __launch_bounds__(SC_THREADS, 10)
+__global__ void __launch_bounds__(SC_THREADS, SC_PER_SM)
     scan_chunk_kernel(const __grid_constant__ CUtensorMap mapD, const __grid_constant__ CUtensorMap mapX,
                       const __grid_constant__ CUtensorMap mapBC, const __grid_constant__ ScanParams p) {
   pdl_wait();
@@ -165,7 +182,7 @@ __global__ void __launch_bounds__(SC_THREADS, 10)
   const int tid = threadIdx.x;
   const int g = blockIdx.x, k = blockIdx.y, b = blockIdx.z;
   const int c = g * SC_CH + tid;
-  const int t0 = k * p.L;
+  const int t0 = p.t_begin + k * p.L;
   const int t1 = min(t0 + p.L, p.T);
   const int n_sub = (t1 - t0 + SC_SUB - 1) / SC_SUB;
   const int row0 = b * p.T + t0;
@@ -210,10 +227,19 @@ __global__ void __launch_bounds__(SC_THREADS, 10)
   }
   const bool pow_path = __all_sync(0xffffffffu, prog);
   const float A20 = f2_lo(A2[0]);
+  const float bias = p.dt_bias[c];
 
   uint64_t h[8];
   if (OUT && k > 0) {
     const float4* hs = reinterpret_cast<const float4*>(p.carry + (((size_t)b * (p.n_chunks - 1) + k - 1) * p.Di + c) * 16);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 v = hs[q];
+      h[2 * q] = f2_pack(v.x, v.y);
+      h[2 * q + 1] = f2_pack(v.z, v.w);
+    }
+  } else if (OUT && p.h0 != nullptr) {   // chunk 0 of the output pass from the given state
+    const float4* hs = reinterpret_cast<const float4*>(p.h0 + (size_t)c * 16);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const float4 v = hs[q];
@@ -227,6 +253,38 @@ __global__ void __launch_bounds__(SC_THREADS, 10)
   float sumd = 0.f;
   __nv_bfloat16* yrow = p.y + (size_t)row0 * p.Di + c;
 
+  // one step: decays, h = a h + dx B, and (output pass) y = C . h with two independent
+  // accumulators; B and C are read as (state 2q, state 2q+1) pairs straight into 64-bit
+  // registers
+  auto step = [&](const ScStage& S, int i, __nv_bfloat16* yp) {
+    const float d = softplus_sel(S.d[i][tid] + bias);   // delta of this step and channel
+    const float dx = d * __bfloat162float(S.x[i][tid]);
+    uint64_t a[8];
+    if (pow_path) scan_decays_pow(d, A20, a);
+    else scan_decays_general(d, A2, a);
+    const uint64_t dxp = f2_pack(dx, dx);
+    const ulonglong2* bc = reinterpret_cast<const ulonglong2*>(&S.bc[i][0]);   // the same address in every lane
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const ulonglong2 bv = bc[q];   // (B[4q], B[4q+1]), (B[4q+2], B[4q+3])
+      h[2 * q] = f2_fma(a[2 * q], h[2 * q], f2_mul(dxp, bv.x));
+      h[2 * q + 1] = f2_fma(a[2 * q + 1], h[2 * q + 1], f2_mul(dxp, bv.y));
+    }
+    if constexpr (OUT) {
+      uint64_t acc0 = 0ull, acc1 = 0ull;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const ulonglong2 cv = bc[4 + q];   // C[4q .. 4q+3]
+        acc0 = f2_fma(cv.x, h[2 * q], acc0);
+        acc1 = f2_fma(cv.y, h[2 * q + 1], acc1);
+      }
+      const uint64_t acc = f2_add(acc0, acc1);
+      *yp = __float2bfloat16_rn(f2_lo(acc) + f2_hi(acc));
+    } else {
+      sumd += d;
+    }
+  };
+
   int j = 0;
   for (; j < n_sub; ++j) {
     // the stage of sub-chunk j-1 is free (barrier at the end of the previous iteration)
@@ -234,34 +292,13 @@ __global__ void __launch_bounds__(SC_THREADS, 10)
     const bool ok = mbar_wait(&sm.full[j % SC_NST], (uint32_t)(j / SC_NST) & 1u, &sm.abort, p.status, 311);
     if (ok) {
       const ScStage& S = sm.st[j % SC_NST];
-      const int n_steps = min(SC_SUB, t1 - t0 - j * SC_SUB);
-#pragma unroll 2
-      for (int i = 0; i < n_steps; ++i) {
-        const float d = S.d[i][tid];
-        const float dx = d * __bfloat162float(S.x[i][tid]);
-        uint64_t a[8];
-        if (pow_path) scan_decays_pow(d, A20, a);
-        else scan_decays_general(d, A2, a);
-        const uint64_t dxp = f2_pack(dx, dx);
-        const float4* bc = reinterpret_cast<const float4*>(&S.bc[i][0]);
+      __nv_bfloat16* yj = yrow + (size_t)(j * SC_SUB) * p.Di;
+      const int n_steps = t1 - t0 - j * SC_SUB;
+      if (n_steps >= SC_SUB) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 bv = bc[q];   // B[4q .. 4q+3], the same address in every lane
-          h[2 * q] = f2_fma(a[2 * q], h[2 * q], f2_mul(dxp, f2_pack(bv.x, bv.y)));
-          h[2 * q + 1] = f2_fma(a[2 * q + 1], h[2 * q + 1], f2_mul(dxp, f2_pack(bv.z, bv.w)));
-        }
-        if constexpr (OUT) {
-          uint64_t acc = 0ull;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float4 cv = bc[4 + q];   // C[4q .. 4q+3]
-            acc = f2_fma(f2_pack(cv.x, cv.y), h[2 * q], acc);
-            acc = f2_fma(f2_pack(cv.z, cv.w), h[2 * q + 1], acc);
-          }
-          yrow[(size_t)(j * SC_SUB + i) * p.Di] = __float2bfloat16_rn(f2_lo(acc) + f2_hi(acc));
-        } else {
-          sumd += d;
-        }
+        for (int i = 0; i < SC_SUB; ++i) step(S, i, yj + (size_t)i * p.Di);
+      } else {
+        for (int i = 0; i < n_steps; ++i) step(S, i, yj + (size_t)i * p.Di);
       }
     }
     if (__syncthreads_or(ok ? 0 : 1)) break;   // a wait gave up: every thread leaves together
@@ -306,7 +343,7 @@ __global__ void __launch_bounds__(256)
   float* e = p.carry + ((size_t)b * nk * p.Di + c) * 16 + s;
   const float* sd = p.sumd + (size_t)b * nk * p.Di + c;
   const size_t es = (size_t)p.Di * 16;
-  float h = 0.f;
+  float h = p.h0 != nullptr ? p.h0[(size_t)c * 16 + s] : 0.f;
   for (int k0 = 0; k0 < nk; k0 += 8) {
     float ev[8], dv[8];
 #pragma unroll

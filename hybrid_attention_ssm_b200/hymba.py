@@ -54,8 +54,12 @@ class ProfRecord(ctypes.Structure):
 
 
 class StageLayout(ctypes.Structure):
-    _fields_ = [(n, _c_size) for n in ("q", "xz", "xc", "xbc", "delta", "y", "o", "u")] + \
+    _fields_ = [(n, _c_size) for n in ("q", "xz", "xc", "xbc", "dt_pre", "y", "o", "u")] + \
                [("ld_xbc", _c_int), ("scan_chunks", _c_int), ("scan_chunk_len", _c_int)]
+
+
+class MetaPrefix(ctypes.Structure):
+    _fields_ = [("k", _vp), ("v", _vp), ("ssm_state", _vp), ("conv_state", _vp)]
 
 
 class DecodeStageLayout(ctypes.Structure):
@@ -100,6 +104,13 @@ def lib():
             "hymba_mixer_prefill_host": ([ctypes.POINTER(LayerCfg), ctypes.POINTER(LayerWeights), _vp, _c_int,
                                           _c_int, _c_int, ctypes.POINTER(KVCache), _vp, _vp, _vp, _vp, _c_size,
                                           _vp], _c_int),
+            "hymba_meta_prefix_size": ([ctypes.POINTER(LayerCfg), ctypes.POINTER(_c_size)], _c_int),
+            "hymba_meta_prefix_build": ([ctypes.POINTER(LayerCfg), ctypes.POINTER(LayerWeights), _vp, _vp, _c_size,
+                                         ctypes.POINTER(MetaPrefix), ctypes.POINTER(MetaPrefix), _vp, _vp, _c_size,
+                                         _vp], _c_int),
+            "hymba_mixer_prefill_prefix": ([ctypes.POINTER(LayerCfg), ctypes.POINTER(LayerWeights), _vp, _c_int,
+                                            _c_int, ctypes.POINTER(MetaPrefix), ctypes.POINTER(KVCache), _vp, _vp,
+                                            _vp, _vp, _vp, _c_size, _vp], _c_int),
             "hymba_mixer_decode_ragged": ([ctypes.POINTER(LayerCfg), ctypes.POINTER(LayerWeights), _vp, _c_int,
                                            _vp, _c_int, ctypes.POINTER(KVCache), _vp, _vp, _vp, _vp, _vp, _c_size,
                                            _vp], _c_int),
@@ -274,6 +285,51 @@ def mixer_prefill_host(dims, dw: DeviceWeights, x_host, kv: Cache, out_host, ws,
     check(lib().hymba_mixer_prefill_host(ctypes.byref(cfg), ctypes.byref(dw.c), ptr(x_host), x_has_meta, B, n_tokens,
                                          ctypes.byref(kv.c), ptr(ssm_state), ptr(conv_state), ptr(out_host), ptr(ws),
                                          ws.numel(), stream_handle(stream)))
+
+
+class Prefix:
+    """A layer's precomputed meta-token prefix (hymba_meta_prefix_build), owned by a torch buffer."""
+
+    def __init__(self, dims, dw: DeviceWeights, meta_rows, meta_out, ws, producer=None, stream=None, device="cuda"):
+        cfg = make_cfg(dims)
+        n = ctypes.c_size_t()
+        check(lib().hymba_meta_prefix_size(ctypes.byref(cfg), ctypes.byref(n)))
+        raw = torch.empty(n.value + 256, dtype=torch.uint8, device=device)
+        off = (-raw.data_ptr()) % 256
+        self._raw = raw
+        self.buf = raw[off:off + n.value]
+        self.c = MetaPrefix()
+        self.producer = producer
+        check(lib().hymba_meta_prefix_build(ctypes.byref(cfg), ctypes.byref(dw.c), ptr(meta_rows), ptr(self.buf),
+                                            n.value, None if producer is None else ctypes.byref(producer.c),
+                                            ctypes.byref(self.c), ptr(meta_out), ptr(ws), ws.numel(),
+                                            stream_handle(stream)))
+        self.dims = dims
+
+    def tensor(self, name):
+        """Device view of the prefix's k / v [M, Hkv, D] fp16, ssm_state [Di, S] or conv_state
+        [Di, 3] fp32 (a consumer's k / v live in its producer's buffer)."""
+        d = self.dims
+        shapes = {"k": ((d.n_meta, d.n_kv_heads, d.head_dim), torch.float16),
+                  "v": ((d.n_meta, d.n_kv_heads, d.head_dim), torch.float16),
+                  "ssm_state": ((d.d_inner, d.d_state), torch.float32),
+                  "conv_state": ((d.d_inner, d.d_conv - 1), torch.float32)}
+        shape, dt = shapes[name]
+        owner = self.producer if name in ("k", "v") and self.producer is not None else self
+        off = getattr(self.c, name) - owner.buf.data_ptr()
+        n = int(np.prod(shape)) * torch.tensor([], dtype=dt).element_size()
+        return owner.buf[off:off + n].view(dt).view(*shape)
+
+
+def mixer_prefill_prefix(dims, dw: DeviceWeights, x, prefix: Prefix, kv: Cache, out, ws, ssm_state=None,
+                         conv_state=None, residual=None, stream=None, cfg=None):
+    """hymba_mixer_prefill of the input rows only, from a precomputed meta-token prefix."""
+    cfg = make_cfg(dims) if cfg is None else cfg
+    B, n_tokens = x.shape[0], x.shape[1]
+    check(lib().hymba_mixer_prefill_prefix(ctypes.byref(cfg), ctypes.byref(dw.c), ptr(x), B, n_tokens,
+                                           ctypes.byref(prefix.c), ctypes.byref(kv.c), ptr(ssm_state),
+                                           ptr(conv_state), ptr(residual), ptr(out), ptr(ws), ws.numel(),
+                                           stream_handle(stream)))
 
 
 def mixer_decode(dims, dw: DeviceWeights, x, position, kv: Cache, ssm_state, conv_state, out, ws, residual=None,

@@ -205,6 +205,48 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
                         float* conv_state_out, const hymba_bf16* residual, hymba_bf16* out, void* workspace,
                         size_t ws_bytes, hymba_stream stream);
 
+/* A layer's meta-token prefix, computed once ([JJ] §深入理解元 Tokens: the meta tokens are
+ * fixed at inference, so what they produce can be computed offline).  The meta rows never
+ * see the input rows (they come first and attention is causal), so these are the same for
+ * every input: the keys (after RoPE) and values of the M meta positions, and the SSM and
+ * conv states after the M meta rows.  A consumer layer's k/v are its producer's. */
+typedef struct hymba_meta_prefix {
+  hymba_f16* k;        /* [M, Hkv, D] fp16 */
+  hymba_f16* v;        /* [M, Hkv, D] fp16 */
+  float* ssm_state;    /* [Di, S] fp32 */
+  float* conv_state;   /* [Di, 3] fp32: the last three conv inputs of the meta rows */
+} hymba_meta_prefix;
+
+/* Bytes of device memory one layer's prefix occupies (k, v, ssm_state, conv_state). */
+int hymba_meta_prefix_size(const hymba_layer_cfg* cfg, size_t* bytes);
+
+/* Compute a layer's prefix: one prefill of its M meta rows alone.
+ *   meta_rows  [M, d] bf16: the meta rows of this layer's input (the meta tokens R for a
+ *              single layer; the residual stream's meta rows, normalised, inside a stack)
+ *   buf        device buffer of hymba_meta_prefix_size bytes, 256-byte aligned; *prefix
+ *              receives pointers into it
+ *   producer   for a consumer layer (kv_role 2), its producer's prefix: the meta keys and
+ *              values it reads (and that *prefix then points to); NULL otherwise
+ *   meta_out   [M, d] bf16: the layer's output rows for the meta positions
+ *   workspace  as hymba_mixer_prefill for batch 1, n_tokens = M, x_has_meta = 1.
+ * Errors as hymba_mixer_prefill; INVALID_ARG when n_meta == 0. */
+int hymba_meta_prefix_build(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* meta_rows,
+                            void* buf, size_t buf_bytes, const hymba_meta_prefix* producer,
+                            hymba_meta_prefix* prefix, hymba_bf16* meta_out, void* workspace, size_t ws_bytes,
+                            hymba_stream stream);
+
+/* hymba_mixer_prefill from a precomputed prefix: x [B, n_tokens, d] holds only the input
+ * rows (positions M .. M + n_tokens - 1), and only those rows are computed.  The prefix's
+ * meta K/V are copied into the cache (the prefill view's rows 0..M-1 and, for an SWA cache,
+ * its meta rows; a consumer reads its producer's), the conv and the scan start from the
+ * prefix's states.  residual and out are [B, n_tokens, d].  ssm_state_out / conv_state_out
+ * as hymba_mixer_prefill.  Workspace: hymba_mixer_workspace_size (mode PREFILL, the same
+ * n_tokens, x_has_meta 0) suffices.  Errors as hymba_mixer_prefill. */
+int hymba_mixer_prefill_prefix(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x,
+                               int batch, int n_tokens, const hymba_meta_prefix* prefix, hymba_kv_cache* kv,
+                               float* ssm_state_out, float* conv_state_out, const hymba_bf16* residual,
+                               hymba_bf16* out, void* workspace, size_t ws_bytes, hymba_stream stream);
+
 /* hymba_mixer_prefill with the input and the output in HOST memory: x_host [B, n_tokens, d]
  * and out_host [B, T, d] bf16 (page-locked memory lets the copies run asynchronously and
  * overlap other streams' work; pageable memory works but the copies then block the host).
@@ -250,14 +292,14 @@ int hymba_mixer_decode_ragged(const hymba_layer_cfg* cfg, const hymba_layer_weig
  *   xz     [B*T, 2*Di]  bf16  in_proj x | z columns
  *   xc     [B*T, Di]    bf16  SiLU(conv(x))
  *   xbc    [B*T, ld_xbc] fp32 x_proj output: dt_low | B | C
- *   delta  [B*T, Di]    fp32  Delta = softplus(dt_low W_dt^T + dt_bias)
+ *   dt_pre [B*T, Di]    fp32  dt_low W_dt^T (the scan applies softplus(. + dt_bias))
  *   y      [B*T, Di]    bf16  scan output before the gate
  *   o      [B*T, Hq*D]  fp32  attention output
  *   u      [B*T, Hq*D+Di] fp16 normalised, rescaled, averaged branches (out_proj input)
  * scan_chunks / scan_chunk_len: the time chunks the selective scan is cut into (the last
  * chunk may be shorter). */
 typedef struct hymba_stage_layout {
-  size_t q, xz, xc, xbc, delta, y, o, u;
+  size_t q, xz, xc, xbc, dt_pre, y, o, u;
   int ld_xbc;
   int scan_chunks, scan_chunk_len;
 } hymba_stage_layout;

@@ -33,7 +33,7 @@ def test_workspace_sizes_grow_with_tokens():
     b = H.workspace_size(d, 1, 4096)
     assert 0 < a < b
     lay = H.stage_layout(d, 1, 2048)
-    offs = [lay.q, lay.xz, lay.xc, lay.xbc, lay.delta, lay.y, lay.o, lay.u]
+    offs = [lay.q, lay.xz, lay.xc, lay.xbc, lay.dt_pre, lay.y, lay.o, lay.u]
     assert all(o % 256 == 0 for o in offs) and offs == sorted(offs) and offs[-1] < a
     assert lay.ld_xbc >= 132
     assert lay.scan_chunks >= 1 and lay.scan_chunk_len % 8 == 0

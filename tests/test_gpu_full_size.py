@@ -66,9 +66,10 @@ def test_global_layer_full_size_sampled_rows():
         ref, h = _oracle_rows(dims, w, Xt_b, rows)
         assert_rms(out[b, rows], ref, name=f"global layer rows (b={b})")
         assert_rel_inf(to_np(run.ssm[b]), h, tol=2e-2, name=f"global layer ssm state (b={b})")
-        # the scan over all 8320 steps, fed the GPU's own xc, delta, B, C: fp32 state at 1e-4
-        xc, delta, xbc = run.stage("xc", b), run.stage("delta", b), run.stage("xbc", b)
+        # the scan over all 8320 steps, fed its own inputs (dt_pre, xc, B, C): fp32 state at 1e-4
+        xc, dt_pre, xbc = run.stage("xc", b), run.stage("dt_pre", b), run.stage("xbc", b)
         R_, S = dims.dt_rank, dims.d_state
+        delta = orc.softplus(dt_pre + w["dt_bias"])
         _, h_own = orc.selective_scan(xc, delta, w["A"], xbc[:, R_:R_ + S], xbc[:, R_ + S:R_ + 2 * S],
                                       np.zeros_like(xc))
         assert_rel_inf(to_np(run.ssm[b]), h_own, tol=1e-4, name=f"global layer scan state, own inputs (b={b})")

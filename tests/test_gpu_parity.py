@@ -70,7 +70,7 @@ def _check_stages(run, ref, dims, w):
         k, v = run.kv()
         assert_elem(k, ref["K"], name="K")
         assert_elem(v, ref["V"], name="V")
-    xc, xbc, delta = run.stage("xc"), run.stage("xbc"), run.stage("delta")
+    xc, xbc, dt_pre = run.stage("xc"), run.stage("xbc"), run.stage("dt_pre")
     y, o, u, q = run.stage("y"), run.stage("o"), run.stage("u"), run.stage("q")
     out = to_np(run.out)
     for b in range(B):
@@ -79,11 +79,12 @@ def _check_stages(run, ref, dims, w):
         assert_rel_inf(to_np(run.conv[b]), cst, tol=1e-6, name="conv state")
         proj = xc[b] @ w["w_x"].astype(np.float64).T
         assert_rms(xbc[b, :, :R + 2 * S], proj, tol=1e-3, name="x_proj")
-        d_ref = orc.softplus(xbc[b, :, :R] @ w["w_dt"].astype(np.float64).T + w["dt_bias"])
-        assert_rel_inf(delta[b], d_ref, tol=5e-3, name="delta")
-        # scan fed the GPU's own xc, delta, B, C, z
+        # dt_proj (tf32): dt_low W_dt^T, before the bias and softplus that the scan applies
+        assert_rel_inf(dt_pre[b], xbc[b, :, :R] @ w["w_dt"].astype(np.float64).T, tol=5e-3, name="dt_proj")
+        # the scan fed its own inputs (dt_pre, xc, B, C, z): delta = softplus(dt_pre + bias) in fp64
+        delta = orc.softplus(dt_pre[b] + w["dt_bias"])
         zb = xz[b, :, Di:]
-        y_ref, h_ref = orc.selective_scan(xc[b], delta[b], w["A"], xbc[b, :, R:R + S], xbc[b, :, R + S:R + 2 * S], zb)
+        y_ref, h_ref = orc.selective_scan(xc[b], delta, w["A"], xbc[b, :, R:R + S], xbc[b, :, R + S:R + 2 * S], zb)
         assert_rel_inf(to_np(run.ssm[b]), h_ref, tol=1e-4, name="scan state")
         assert_elem(y[b] * orc.silu(zb), y_ref, name="scan y")
         if k is not None:
@@ -172,6 +173,93 @@ def test_prefill_from_host_buffers_equals_device_path():
     s.synchronize()
     assert H.status_read(ws, s) == 0
     assert torch.equal(oh, run.out.cpu())
+
+
+# ---------------------------------------------------------------------------------------
+# meta-token prefix computed once, then prefills of the input rows only
+# ---------------------------------------------------------------------------------------
+def _prefix_run(dims, w, X, producer_prefix=None, cache=None, max_tokens=None):
+    """Build the layer's prefix from its meta tokens, then prefill X's rows from it."""
+    B, N = X.shape[0], X.shape[1]
+    M, T = dims.n_meta, dims.n_meta + X.shape[1]
+    dw = H.DeviceWeights(w)
+    meta_out = torch.zeros(M, dims.d_model, dtype=torch.bfloat16, device="cuda")
+    bws = H.alloc_workspace(H.workspace_size(dims, 1, M, 1))
+    pre = H.Prefix(dims, dw, dw.t["meta"], meta_out, bws, producer=producer_prefix)
+    cache = cache if cache is not None else H.Cache(dims, B, max_tokens or T)
+    out = torch.zeros(B, N, dims.d_model, dtype=torch.bfloat16, device="cuda")
+    ssm = torch.zeros(B, dims.d_inner, dims.d_state, device="cuda")
+    conv = torch.zeros(B, dims.d_inner, dims.d_conv - 1, device="cuda")
+    ws = H.alloc_workspace(H.workspace_size(dims, B, N))
+    H.mixer_prefill_prefix(dims, dw, bf16_dev(X), pre, cache, out, ws, ssm_state=ssm, conv_state=conv)
+    torch.cuda.synchronize()
+    assert H.status_read(bws) == 0 and H.status_read(ws) == 0
+    return dict(prefix=pre, meta_out=meta_out, cache=cache, out=out, ssm=ssm, conv=conv, ws=ws)
+
+
+@pytest.mark.parametrize("kw", [dict(B=1, N=120), dict(B=2, N=77, M=130, W=100), dict(B=3, N=1),
+                                dict(B=2, N=200, is_global=1), dict(B=1, N=300, W=1)])
+def test_prefill_from_meta_prefix(kw):
+    """[JJ] §深入理解元 Tokens: the meta tokens' work is done once.  A prefill of the input
+    rows from the layer's prefix equals rows M..T-1 of the full prefill: against the oracle
+    (bf16 bound) and against the full GPU prefill (the rows, the final states, the cache);
+    the prefix itself (meta output rows, meta K/V, states after the meta rows) equals the
+    full prefill's meta rows."""
+    dims = WL["tiny"].dims.replace(n_meta=kw.get("M", 8), window=kw.get("W", 32), is_global=kw.get("is_global", 0))
+    w = _w(dims, seed=61)
+    X = synth.bf16_round(np.random.default_rng(62).normal(size=(kw["B"], kw["N"], dims.d_model)).astype(np.float32))
+    M = dims.n_meta
+    full = PrefillRun(dims, w, X)
+    r = _prefix_run(dims, w, X)
+    ref = orc.mixer_prefill(dims, w, X)
+    assert_rms(to_np(r["out"]), ref["out"][:, M:], name="prefix prefill vs oracle rows M..T-1")
+    assert_rms(to_np(r["out"]), to_np(full.out[:, M:]), tol=5e-3, name="prefix prefill vs full prefill")
+    assert torch.equal(r["meta_out"], full.out[0, :M]), "meta rows of the output"
+    assert_rel_inf(to_np(r["ssm"]), to_np(full.ssm), tol=1e-4, name="final ssm state")
+    assert torch.equal(r["conv"], full.conv), "final conv state"
+    for n in (("k", "v") if dims.is_global else ("k", "v", "meta_k", "meta_v", "ring_k", "ring_v")):
+        a, b = r["cache"].t[n], full.cache.t[n]
+        if n in ("k", "v"):
+            a, b = a[:, :full.T], b[:, :full.T]
+        assert torch.equal(a, b), f"cache {n}"
+    # the prefix against the oracle's meta rows alone (meta rows never see X: P6)
+    om = orc.mixer_prefill(dims, w, w["meta"][None], x_has_meta=True)
+    pre = r["prefix"]
+    assert_rms(to_np(r["meta_out"]), om["out"][0], name="meta rows vs oracle")
+    assert_rms(to_np(pre.tensor("k")), om["K"][0], name="prefix K vs oracle")
+    assert_rms(to_np(pre.tensor("v")), om["V"][0], name="prefix V vs oracle")
+    assert_rel_inf(to_np(pre.tensor("ssm_state")), om["ssm_state"][0], tol=2e-2, name="prefix ssm state vs oracle")
+    assert_rel_inf(to_np(pre.tensor("conv_state")), om["conv_state"][0], tol=1e-2, name="prefix conv state vs oracle")
+
+
+def test_prefill_from_meta_prefix_shared_kv_pair():
+    """A consumer layer's prefix reads its producer's meta K/V; prefills of both layers from
+    their prefixes equal the full prefills of the pair."""
+    wl = WL["tiny"]
+    prod = wl.dims.replace(kv_role=synth.KV_PRODUCER)
+    cons = wl.dims.replace(kv_role=synth.KV_CONSUMER)
+    wp, wc = _w(prod, seed=63), _w(cons, seed=64)
+    X = synth.prefill_input(wl)
+    M = prod.n_meta
+    fp = PrefillRun(prod, wp, X)
+    fc = PrefillRun(cons, wc, X, cache=fp.cache)
+    rp = _prefix_run(prod, wp, X)
+    rc = _prefix_run(cons, wc, X, producer_prefix=rp["prefix"], cache=rp["cache"])
+    assert_rms(to_np(rp["out"]), to_np(fp.out[:, M:]), tol=5e-3, name="producer")
+    assert_rms(to_np(rc["out"]), to_np(fc.out[:, M:]), tol=5e-3, name="consumer")
+    assert torch.equal(rc["meta_out"], fc.out[0, :M]), "consumer meta rows"
+
+
+def test_prefill_from_meta_prefix_hymba_layer():
+    """The Hymba-shaped SWA layer (128 meta + 2048 tokens) from its prefix."""
+    wl = WL["swa"]
+    w = _w(wl.dims, wl=wl)
+    X = synth.prefill_input(wl)
+    M = wl.dims.n_meta
+    full = PrefillRun(wl.dims, w, X)
+    r = _prefix_run(wl.dims, w, X)
+    assert_rms(to_np(r["out"]), to_np(full.out[:, M:]), tol=5e-3, name="prefix prefill vs full prefill (swa)")
+    assert_rel_inf(to_np(r["ssm"]), to_np(full.ssm), tol=1e-4, name="final ssm state (swa)")
 
 
 def test_prefill_shared_kv_pair():
