@@ -713,16 +713,16 @@ def run_stack_decode(args, st, E, world):
 # workload (profiles/ holds the summaries and commands); a kernel changed since its capture
 # has no entry.  ncu replays a kernel with cold caches: writes that stay in L2 do not show.
 TRAFFIC = {
-    "selective_scan": 42143488 + 5376,
-    "norm_avg": 41828352 + 261632,
-    "in_proj": 35357184 + 1401856,
-    "x_proj": 14797824 + 256,
-    "dt_proj": 2488320 + 0,
-    "out_proj": 36292864 + 22784,
-    "attention": 9816320 + 768,
-    "conv1d_silu": 13999616 + 768,
-    "decode_attn": 94806016 + 2965760,
-    "decode_prep": 5318912 + 0,
+    "in_proj": 35320064 + 787968,
+    "conv1d_silu": 13999616 + 0,
+    "x_proj": 14799360 + 768,
+    "dt_proj": 2442496 + 0,
+    "attention": 9817344 + 0,
+    "scan_chunk_end": 42369280 + 16128,
+    "scan_carry": 6089472 + 0,
+    "selective_scan": 48214272 + 553472,
+    "norm_avg": 41828864 + 295680,
+    "out_proj": 36293632 + 17664,
     "decode_ssm": 16947200 + 0,
 }
 
