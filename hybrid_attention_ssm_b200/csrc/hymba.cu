@@ -1523,6 +1523,104 @@ int hymba_ffn_swiglu(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hym
   return HYMBA_OK;
 }
 
+// Decode-shaped FFN: the weights as the M operand (swap-AB) so that their rows, not the few
+// token rows, spread the work over the SMs, split over K into fp32 slices summed in a fixed
+// order.
+namespace {
+struct FfnDecWs {
+  size_t part1, act, part2, total;
+  int s1, s2;
+};
+FfnDecWs ffn_dec_layout(int rows, int d, int F) {
+  FfnDecWs w;
+  const int bn = rows <= 64 ? 64 : (rows <= 128 ? 128 : 256);
+  const int nt = cdiv(rows, bn);
+  w.s1 = splits_for(cdiv(2 * F, GEMM_BM) * nt, cdiv(d, 64), 8);
+  w.s2 = splits_for(cdiv(d, GEMM_BM) * nt, cdiv(F, 64), 16);
+  size_t off = 256;
+  auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
+  w.part1 = take((size_t)w.s1 * rows * 2 * F * 4);
+  w.act = take((size_t)rows * F * 2);
+  w.part2 = take((size_t)w.s2 * rows * d * 4);
+  w.total = off;
+  return w;
+}
+}  // namespace
+
+int hymba_ffn_workspace_size(int rows, int d, int F, size_t* bytes) {
+  if (bytes == nullptr || rows < 1 || rows > 256 || d < 8 || d % 8 || F < 64 || F % 64)
+    return fail(HYMBA_ERR_INVALID_ARG, "ffn workspace arguments (rows 1..256, d % 8, F % 64)");
+  *bytes = ffn_dec_layout(rows, d, F).total;
+  return HYMBA_OK;
+}
+
+int hymba_ffn_swiglu_decode(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hymba_f16* w_down, int rows,
+                            int d, int F, const hymba_bf16* residual, hymba_bf16* out, void* ws, size_t ws_bytes,
+                            hymba_stream stream) {
+  DeviceInfo* dev = nullptr;
+  HY_TRY(device_info(&dev));
+  size_t need = 0;
+  HY_TRY(hymba_ffn_workspace_size(rows, d, F, &need));
+  if (h == nullptr || w_gate_up == nullptr || w_down == nullptr || out == nullptr || !aligned16(h) ||
+      !aligned16(out) || (residual != nullptr && !aligned16(residual)))
+    return fail(HYMBA_ERR_INVALID_ARG, "ffn decode pointers");
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return fail(HYMBA_ERR_INVALID_ARG, "workspace");
+  if (ws_bytes < need) return fail(HYMBA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
+  const FfnDecWs L = ffn_dec_layout(rows, d, F);
+  cudaStream_t st = (cudaStream_t)stream;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  DevStatus* status = reinterpret_cast<DevStatus*>(ws);
+  float* part1 = reinterpret_cast<float*>(wsb + L.part1);
+  float* part2 = reinterpret_cast<float*>(wsb + L.part2);
+  __half* act = reinterpret_cast<__half*>(wsb + L.act);
+  {  // [gate | up] slices, transposed: part1[s][r][2F]
+    GemmCall c;
+    c.a1 = w_gate_up; c.nb1 = 1; c.rows1 = 2 * F; c.lda1 = d; c.a1_bstride = (long long)2 * F * d;
+    c.b = h; c.N = rows; c.ldb = d; c.K = d;
+    c.bn = pick_bn_cover(rows);
+    c.name = "ffn_dec_gate_up";
+    c.split_k = L.s1;
+    c.mode = EPI_F32_T_PART;
+    c.p.out = part1;
+    c.p.split_stride = (long long)rows * 2 * F;
+    c.p.ld_out = 2 * F;
+    c.p.m_valid = 2 * F;
+    c.p.n_valid = rows;
+    c.p.status = status;
+    HY_TRY(run_gemm(c, *dev, st));
+  }
+  {
+    const long long n = (long long)rows * F;
+    prof_begin("ffn_dec_swiglu", st);
+    HY_CUDA(launch_pdl(swiglu_slices_kernel, dim3(cdiv(n, 256)), dim3(256), 0, st, (const float*)part1, L.s1,
+                       (long long)rows * 2 * F, rows, F, act, status));
+    prof_end(st);
+  }
+  {  // down projection slices part2[s][r][d], then their sum with the residual
+    GemmCall c;
+    c.a1 = w_down; c.nb1 = 1; c.rows1 = d; c.lda1 = F; c.a1_bstride = (long long)d * F;
+    c.b = act; c.N = rows; c.ldb = F; c.K = F;
+    c.etype = ET_F16;
+    c.bn = pick_bn_cover(rows);
+    c.name = "ffn_dec_down";
+    c.split_k = L.s2;
+    c.mode = EPI_F32_T_PART;
+    c.p.out = part2;
+    c.p.split_stride = (long long)rows * d;
+    c.p.ld_out = d;
+    c.p.m_valid = d;
+    c.p.n_valid = rows;
+    c.p.status = status;
+    HY_TRY(run_gemm(c, *dev, st));
+    const int n = rows * d;
+    prof_begin("ffn_dec_out", st);
+    HY_CUDA(launch_pdl(splitk_reduce_kernel, dim3(cdiv(n / 4, 256)), dim3(256), 0, st, (const float*)part2, L.s2,
+                       (long long)n, n, reinterpret_cast<const __nv_bfloat16*>(residual), out, 1));
+    prof_end(st);
+  }
+  return HYMBA_OK;
+}
+
 int hymba_prepend_meta(const hymba_bf16* meta, const hymba_bf16* x, int batch, int n_meta, int n_tokens, int d,
                        hymba_bf16* out, hymba_stream stream) {
   if ((n_meta > 0 && meta == nullptr) || x == nullptr || out == nullptr || batch < 1 || n_meta < 0 ||

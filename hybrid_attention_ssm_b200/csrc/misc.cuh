@@ -894,6 +894,28 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// SwiGLU of a decode FFN's gate/up projection: act[r, f] = SiLU(g) * u, with g and u the
+// sums, in slice order, of n_split fp32 slices [rows, 2F] whose columns interleave gate and
+// up in blocks of 32 (gate f at column 64 (f / 32) + f % 32, up 32 columns later); fp16 out.
+__global__ void __launch_bounds__(256)
+    swiglu_slices_kernel(const float* __restrict__ part, int n_split, long long stride, int rows, int F,
+                         __half* __restrict__ act, DevStatus* status) {
+  pdl_wait();
+  pdl_trigger();
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)rows * F) return;
+  const int r = (int)(i / F), f = (int)(i % F);
+  const size_t gc = (size_t)r * 2 * F + (size_t)(f >> 5) * 64 + (f & 31);
+  float g = 0.f, u = 0.f;
+  for (int s = 0; s < n_split; ++s) {
+    g += part[(size_t)s * stride + gc];
+    u += part[(size_t)s * stride + gc + 32];
+  }
+  const float a[1] = {silu_f(g) * u};
+  f16_range_guard<1>(a, status, 240);
+  act[i] = __float2half_rn(a[0]);
+}
+
 // Fixed-order sum of split-K partial slices: out[i] = sum_s part[s*stride + i] (+ residual),
 // as fp32 or bf16; n is a multiple of 4.  The order never changes, so results are
 // identical from run to run.

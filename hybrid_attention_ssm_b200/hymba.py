@@ -121,6 +121,8 @@ def lib():
             "hymba_gemm_bf16": ([_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp], _c_int),
             "hymba_rmsnorm": ([_vp, _vp, _c_int, _c_int, ctypes.c_float, _vp, _vp], _c_int),
             "hymba_ffn_swiglu": ([_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp], _c_int),
+            "hymba_ffn_workspace_size": ([_c_int, _c_int, _c_int, ctypes.POINTER(_c_size)], _c_int),
+            "hymba_ffn_swiglu_decode": ([_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _c_size, _vp], _c_int),
             "hymba_set_wait_limit_ns": ([ctypes.c_ulonglong], _c_int),
             "hymba_prepend_meta": ([_vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp], _c_int),
             "hymba_selftest_wait_timeout": ([_vp, _c_size, _vp], _c_int),
@@ -391,6 +393,20 @@ def interleave_gate_up(w_gate, w_up):
     g = w_gate.reshape(F // 32, 32, d)
     u = w_up.reshape(F // 32, 32, d)
     return np.concatenate([g, u], axis=1).reshape(2 * F, d)
+
+
+def ffn_workspace_size(rows, d, F) -> int:
+    n = ctypes.c_size_t()
+    check(lib().hymba_ffn_workspace_size(rows, d, F, ctypes.byref(n)))
+    return n.value
+
+
+def ffn_swiglu_decode(h, w_gate_up, w_down, out, ws, residual=None, stream=None):
+    """hymba_ffn_swiglu_decode: the SwiGLU FFN of a few rows (decode), ws sized by ffn_workspace_size."""
+    rows, d = h.shape
+    F = w_down.shape[1]
+    check(lib().hymba_ffn_swiglu_decode(ptr(h), ptr(w_gate_up), ptr(w_down), rows, d, F, ptr(residual), ptr(out),
+                                        ptr(ws), ws.numel(), stream_handle(stream)))
 
 
 def profile_begin(max_records=8192):

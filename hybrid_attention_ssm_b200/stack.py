@@ -110,7 +110,7 @@ class HymbaStack:
             self.dh = [torch.empty(self.B, dims.d_model, **bf) for _ in range(2)]
             self.dh1 = torch.empty(self.B, dims.d_model, **bf)
             self.dhn = torch.empty(self.B, dims.d_model, **bf)
-            self.dact = torch.empty(self.B, self.F, dtype=torch.float16, device=device)
+            self.fws = H.alloc_workspace(H.ffn_workspace_size(self.B, dims.d_model, self.F))
 
     def cache_view(self, ptr_value, max_tokens, dl):
         """fp16 view [B, max_tokens, Hkv, D] of a K or V buffer carved out of cache_buf."""
@@ -193,7 +193,7 @@ class HymbaStack:
             H.mixer_decode(dl, dw, self.dhn, position, kv, self.ssm[l], self.conv[l], self.dh1, self.dws,
                            residual=hin)
             H.rmsnorm(self.dh1, dev["g2"], dl.norm_eps, self.dhn)
-            H.ffn_swiglu(self.dhn, dev["w_gu"], dev["w_down"], self.dact, hout, self.dws, residual=self.dh1)
+            H.ffn_swiglu_decode(self.dhn, dev["w_gu"], dev["w_down"], hout, self.fws, residual=self.dh1)
             if record is not None and l in record:
                 record[l].update(h_mid=self.dh1.float().cpu().numpy(), hn2=self.dhn.float().cpu().numpy(),
                                  h_out=hout.float().cpu().numpy())

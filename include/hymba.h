@@ -343,6 +343,16 @@ int hymba_ffn_swiglu(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hym
                      int F, hymba_f16* act, const hymba_bf16* residual, hymba_bf16* out, void* status_ws,
                      hymba_stream stream);
 
+/* The same FFN for a few rows (a decode step: rows = sequences, 1..256): the weights are the M
+ * operand of the tensor-core GEMMs, so that their rows spread the weight streaming over the
+ * SMs, and K is split into fp32 slices summed in a fixed order.  The same function as
+ * hymba_ffn_swiglu; gate and up are kept in fp32 until the activation (fp16).  The workspace
+ * (hymba_ffn_workspace_size) holds the slices, the activations and the status word. */
+int hymba_ffn_workspace_size(int rows, int d, int F, size_t* bytes);
+int hymba_ffn_swiglu_decode(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hymba_f16* w_down, int rows,
+                            int d, int F, const hymba_bf16* residual, hymba_bf16* out, void* workspace,
+                            size_t ws_bytes, hymba_stream stream);
+
 /* Meta-token prefix of a stack's residual stream ([JJ] §数学表示 1: X~ = [R, X]):
  * out[b] = [meta; x[b]], meta [n_meta, d], x [B, n_tokens, d], out [B, n_meta + n_tokens, d],
  * all bf16, d % 8 == 0. */

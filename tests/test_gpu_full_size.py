@@ -157,7 +157,7 @@ def test_stack_32_layers_decode_step():
     p = wl.dims.n_meta + N - 1
     h = to_np(st.decode_step(E[:, N - 1].contiguous(), p, record=rec))
     torch.cuda.synchronize()
-    assert H.status_read(st.dws) == 0 and H.status_read(st.ws) == 0
+    assert H.status_read(st.dws) == 0 and H.status_read(st.ws) == 0 and H.status_read(st.fws) == 0
     # drift of the decode path from the prefill path, layer by layer (sequence 0): it starts
     # at zero (same embedding) and grows by the two paths' independent bf16 roundings
     for l in check_layers:
@@ -181,12 +181,12 @@ def test_stack_32_layers_decode_step():
         mix = torch.empty(B, d, dtype=torch.bfloat16, device="cuda")
         H.mixer_decode(dl, dw, torch.from_numpy(r["hn"].astype(np.float32)).cuda().to(torch.bfloat16), p, cache,
                        ssm, conv, mix, ws)
-        act = torch.empty(B, st.F, dtype=torch.float16, device="cuda")
         ffn = torch.empty(B, d, dtype=torch.bfloat16, device="cuda")
-        H.ffn_swiglu(torch.from_numpy(r["hn2"].astype(np.float32)).cuda().to(torch.bfloat16), dev["w_gu"],
-                     dev["w_down"], act, ffn, ws)
+        fws = H.alloc_workspace(H.ffn_workspace_size(B, d, st.F))
+        H.ffn_swiglu_decode(torch.from_numpy(r["hn2"].astype(np.float32)).cuda().to(torch.bfloat16), dev["w_gu"],
+                            dev["w_down"], ffn, fws)
         torch.cuda.synchronize()
-        assert H.status_read(ws) == 0
+        assert H.status_read(ws) == 0 and H.status_read(fws) == 0
         ocache = r["cache"] if dl.is_global else {n: r["cache"][n] for n in ("meta_k", "meta_v", "ring_k", "ring_v")}
         ref = orc.mixer_decode(dl, w, r["hn"], p, ocache, r["ssm"], r["conv"])
         mix_np, ffn_np = to_np(mix), to_np(ffn)

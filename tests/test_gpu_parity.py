@@ -438,6 +438,38 @@ def test_decode_global_layer_hymba_width():
 
 
 # ---------------------------------------------------------------------------------------
+# the SwiGLU FFN of the stack harness, for a few rows (decode) and many (prefill)
+# ---------------------------------------------------------------------------------------
+@pytest.mark.parametrize("rows", [1, 8, 64, 200])
+def test_ffn_swiglu_decode(rows):
+    """The decode-shaped FFN (weights as the M operand, split-K) against the oracle's SwiGLU
+    and against the prefill-shaped FFN, at the stack's sizes (d 1600, F 5504), with a
+    residual."""
+    d, F = 1600, 5504
+    dims = WL["stack"].dims
+    bw = synth.block_weights(dims, F, seed=5, layer=3)
+    rng = np.random.default_rng(70 + rows)
+    hx = synth.bf16_round(rng.normal(size=(rows, d)).astype(np.float32))
+    res = synth.bf16_round(rng.normal(size=(rows, d)).astype(np.float32))
+    w_gu = torch.from_numpy(H.interleave_gate_up(bw["w_gate"], bw["w_up"])).cuda().to(torch.bfloat16)
+    w_dn = torch.from_numpy(bw["w_down"]).cuda().to(torch.float16)
+    h, r = bf16_dev(hx), bf16_dev(res)
+    out = torch.empty(rows, d, dtype=torch.bfloat16, device="cuda")
+    ws = H.alloc_workspace(H.ffn_workspace_size(rows, d, F))
+    H.ffn_swiglu_decode(h, w_gu, w_dn, out, ws, residual=r)
+    out2 = torch.empty_like(out)
+    act = torch.empty(rows, F, dtype=torch.float16, device="cuda")
+    ws2 = H.alloc_workspace(256)
+    H.ffn_swiglu(h, w_gu, w_dn, act, out2, ws2, residual=r)
+    torch.cuda.synchronize()
+    assert H.status_read(ws) == 0 and H.status_read(ws2) == 0
+    # the output is bf16(residual + FFN): compare the sum, whose rounding is what is stored
+    ref = orc.ffn_swiglu(hx, bw) + res
+    assert_rms(to_np(out), ref, name=f"decode FFN ({rows} rows) vs oracle")
+    assert_rms(to_np(out), to_np(out2), name=f"decode FFN vs prefill FFN ({rows} rows)")
+
+
+# ---------------------------------------------------------------------------------------
 # decode with a position per sequence
 # ---------------------------------------------------------------------------------------
 def _ragged_case(dims, B, positions, seed, Lmax=None):
