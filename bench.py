@@ -427,8 +427,9 @@ def run_prefix(args, dims, dw, x, flush, stream, full_ms, world):
                    f"{N} input rows only (hymba_mixer_prefill_prefix)"}
 
 
-def run_decode(args, device, world):
-    """Decode step of the shared-KV SWA pair: producer then consumer, batch 64, position 4128."""
+def decode_pair_setup(device):
+    """The shared-KV SWA pair at batch 64, position 4128: its layers, cache, and one step
+    (producer then consumer) as a function."""
     import torch
     from hybrid_attention_ssm_b200 import hymba as H
     from hybrid_attention_ssm_b200 import synth
@@ -451,12 +452,37 @@ def run_decode(args, device, world):
             ssm=torch.from_numpy(st["ssm_state"]).to(device), conv=torch.from_numpy(st["conv_state"]).to(device),
             out=torch.empty(B, dims.d_model, dtype=torch.bfloat16, device=device),
             ws=H.alloc_workspace(H.workspace_size(dims, B, 1, 0, H.MODE_DECODE))))
-    stream = torch.cuda.current_stream()
 
     def step():
         for L in layers:
             H.mixer_decode(L["dims"], L["dw"], L["x"], p, cache, L["ssm"], L["conv"], L["out"], L["ws"])
 
+    return wl, layers, cache, step
+
+
+def profile_decode(n, device):
+    """n eager decode steps of the shared-KV SWA pair and nothing else, for a profiler's
+    launch list."""
+    import torch
+    from hybrid_attention_ssm_b200 import hymba as H
+
+    _, layers, _, step = decode_pair_setup(device)
+    for _ in range(n):
+        step()
+    torch.cuda.synchronize()
+    for L in layers:
+        assert H.status_read(L["ws"]) == 0
+
+
+def run_decode(args, device, world):
+    """Decode step of the shared-KV SWA pair: producer then consumer, batch 64, position 4128."""
+    import torch
+    from hybrid_attention_ssm_b200 import hymba as H
+
+    wl, layers, cache, step = decode_pair_setup(device)
+    prod = wl.dims
+    B, p = wl.batch, wl.decode_position
+    stream = torch.cuda.current_stream()
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize()
@@ -606,6 +632,27 @@ def profile_global(n, device):
         H.mixer_prefill(dims, dw, x, cache, out, ws)
     torch.cuda.synchronize()
     assert H.status_read(ws) == 0
+
+
+def profile_stack_decode(n, device):
+    """The stack's prefill once, then n eager decode steps and nothing else, for a profiler's
+    launch list."""
+    import torch
+    from hybrid_attention_ssm_b200 import hymba as H
+    from hybrid_attention_ssm_b200 import synth
+    from hybrid_attention_ssm_b200.stack import HymbaStack
+
+    wl = synth.workloads()["stack"]
+    st = HymbaStack(wl, device=device, device_init=True, decode_room=1)
+    g = torch.Generator(device=device)
+    g.manual_seed(11)
+    E = torch.randn(st.B, st.N, wl.dims.d_model, generator=g, device=device).to(torch.bfloat16)
+    st.forward(E)
+    x = E[:, -1].contiguous()
+    for _ in range(n):
+        st.decode_step(x, st.T)
+    torch.cuda.synchronize()
+    assert H.status_read(st.ws) == 0 and H.status_read(st.dws) == 0 and H.status_read(st.fws) == 0
 
 
 def run_stack(args, device, world):
@@ -806,6 +853,12 @@ def main():
     ap.add_argument("--profile-global", type=int, default=0, metavar="N",
                     help="profiling runs: only N prefills of the global layer (batch 4, 128 + 8192 "
                          "tokens), no timing and no JSON line")
+    ap.add_argument("--profile-decode", type=int, default=0, metavar="N",
+                    help="profiling runs: N eager decode steps of the shared-KV SWA pair, no timing "
+                         "and no JSON line")
+    ap.add_argument("--profile-stack-decode", type=int, default=0, metavar="N",
+                    help="profiling runs: the 32-layer stack's prefill, then N decode steps, no timing "
+                         "and no JSON line")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -842,6 +895,12 @@ def main():
     torch.cuda.set_device(device)
     if args.profile_global > 0:
         profile_global(args.profile_global, device)
+        return
+    if args.profile_decode > 0:
+        profile_decode(args.profile_decode, device)
+        return
+    if args.profile_stack_decode > 0:
+        profile_stack_decode(args.profile_stack_decode, device)
         return
     r = run_hymba(args, rank, world, device)
     tokens_per_s = whole_job_rate(world, r["tokens_per_step"], r["ms_per_step"])

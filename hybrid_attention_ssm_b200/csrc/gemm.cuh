@@ -55,6 +55,15 @@ struct GemmParams {
   // operands no kernel of the same call writes (the caller's input and the weights), so the
   // mainloop overlaps a previous kernel that only prepares what the epilogue reads.
   int wait_late;
+  // 1: the A operand (weights) is read-only for the whole stream: the producer issues the A
+  // tiles of its first tile's first STAGES k-blocks before it waits for the previous kernel,
+  // so the weight stream starts while that kernel runs (decode GEMMs, weights as M operand).
+  int prefetch_a;
+  // with prefetch_a, 1: the producer also lets the next kernel launch before its own wait,
+  // so that kernel's CTAs are resident (and waiting) before this one starts its mainloop;
+  // for a next kernel whose launch latency is on the critical path and no other stream's
+  // kernel needs the SM room meanwhile.  0: only the warps that have waited trigger it.
+  int trigger_early;
   void* out;
   long long split_stride;   // elements between the partial-sum slices of two splits
   int ld_out;
@@ -182,14 +191,48 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   // parameters, so it overlaps the previous kernel's tail.  Every access to global memory
   // comes after the wait.  A CTA launched early can only meet TMEM held by CTAs of the
   // previous kernel, which are all running by then and free it when they finish.
-  if (!p.wait_late || warp >= 2) pdl_wait();
-  pdl_trigger();
+  // With prefetch_a the producer warp waits in its own branch, after its early A loads, and
+  // (unless trigger_early) leaves the launch of the next kernel to the warps that have
+  // waited: a dependent launched before this kernel's own predecessor has finished holds SM
+  // room that a kernel on another stream (the decode attention) may need.
+  const bool early_a = p.prefetch_a && warp == 0;
+  if ((!p.wait_late && !early_a) || warp >= 2) pdl_wait();
+  if (!early_a || p.trigger_early) pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
     if (lane == 0) {
+      auto load_a = [&](uint8_t* sa, uint64_t* bar, int m, int kc) {
+        if (m < p.tiles0) {
+          tma_load_2d(sa, &mapA0, bar, kc, m * GEMM_BM);
+        } else {
+          const int idx = m - p.tiles0;
+          tma_load_3d(sa, &mapA1, bar, kc, (idx % p.tiles1) * GEMM_BM, idx / p.tiles1);
+        }
+      };
+      // k-blocks (counted from the CTA's first) whose A tile is already in flight: stages
+      // 0..pre-1 of the first tile, loaded before the wait with the stage's full byte count
+      // expected, so their B loads below complete them
+      uint32_t pre = 0;
+      if (p.prefetch_a) {
+        if ((int)blockIdx.x < p.total_tiles) {
+          const int tile = blockIdx.x;
+          const int ks = tile % p.split_k;
+          const int m = (tile / p.split_k) % p.m_tiles;
+          const int kb0 = (int)((long long)ks * p.k_blocks / p.split_k);
+          const int kb1 = (int)((long long)(ks + 1) * p.k_blocks / p.split_k);
+          pre = (uint32_t)min(kb1 - kb0, STAGES);
+          for (uint32_t j = 0; j < pre; ++j) {
+            mbar_arrive_expect_tx(&full[j], L::STAGE_BYTES);
+            load_a(smem + j * L::STAGE_BYTES, &full[j], m, (kb0 + (int)j) * (TF32 ? 32 : 64));
+          }
+        }
+        pdl_wait();
+      }
       uint32_t it = 0;
-      for (int tile = blockIdx.x; tile < p.total_tiles && !*abort_flag; tile += gridDim.x) {
+      // the first tile is always entered when it has A tiles in flight: their stages get
+      // their B loads before any wait, so the drain below finds every issued stage complete
+      for (int tile = blockIdx.x; tile < p.total_tiles && (it < pre || !*abort_flag); tile += gridDim.x) {
         const int ks = tile % p.split_k;
         const int t2 = tile / p.split_k;
         const int m = t2 % p.m_tiles;
@@ -199,16 +242,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
-          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status, 101)) break;
           uint8_t* sa = smem + s * L::STAGE_BYTES;
           uint8_t* sb = sa + L::A_BYTES;
-          mbar_arrive_expect_tx(&full[s], L::STAGE_BYTES);
           const int kc = kb * (TF32 ? 32 : 64);
-          if (m < p.tiles0) {
-            tma_load_2d(sa, &mapA0, &full[s], kc, m * GEMM_BM);
-          } else {
-            const int idx = m - p.tiles0;
-            tma_load_3d(sa, &mapA1, &full[s], kc, (idx % p.tiles1) * GEMM_BM, idx / p.tiles1);
+          if (it >= pre) {
+            if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status, 101)) break;
+            mbar_arrive_expect_tx(&full[s], L::STAGE_BYTES);
+            load_a(sa, &full[s], m, kc);
           }
           tma_load_2d(sb, &mapB, &full[s], kc, n * BN);
         }

@@ -488,6 +488,23 @@ int splits_for(int tiles, int k_blocks, int cap) {
   if (s > k_blocks) s = k_blocks;
   return s < 1 ? 1 : s;
 }
+// Split-K for the decode GEMMs (a few activation rows, the weights streamed as the M
+// operand): the split that gives the busiest of 148 persistent CTAs the fewest k-blocks,
+// ceil(tiles * s / 148) tiles of ceil(k_blocks / s) each; on a tie the smaller split (fewer
+// slices to add).  E.g. 86 weight tiles of 25 k-blocks: s = 1 streams on 86 SMs only (25
+// k-blocks each), s = 5 on all of them (3 tiles of 5).
+int splits_balanced(int tiles, int k_blocks, int cap) {
+  int best = 1;
+  long long best_cost = -1;
+  for (int s = 1; s <= cap && s <= k_blocks; ++s) {
+    const long long cost = (long long)cdiv((long long)tiles * s, 148) * cdiv(k_blocks, s);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
+}
 
 struct PrefillWs {
   size_t q, xz, xc, xbc, xbc_part, dt_pre, carry, sumd, y, o, u, sstate, cstate, rope, total;
@@ -574,8 +591,7 @@ DecodeWs decode_layout(const Dims& m, int B, bool global, int n_keys_max) {
   // consumers add the slices
   {
     const int bn0 = B <= 64 ? 64 : (B <= 128 ? 128 : 256);
-    const int tiles = cdiv(m.P, GEMM_BM) * cdiv(B, bn0);
-    w.in_split = 148 / tiles < 1 ? 1 : (148 / tiles > DEC_MAX_IN_SPLIT ? DEC_MAX_IN_SPLIT : 148 / tiles);
+    w.in_split = splits_balanced(cdiv(m.P, GEMM_BM) * cdiv(B, bn0), cdiv(m.d, 64), DEC_MAX_IN_SPLIT);
   }
   w.proj = take((size_t)w.in_split * B * m.P * 4);
   w.qrot = take((size_t)B * m.Hq * 64 * 4);
@@ -585,11 +601,11 @@ DecodeWs decode_layout(const Dims& m, int B, bool global, int n_keys_max) {
   w.xbc = take((size_t)B * m.ld_xbc * 4);
   const int bn = B <= 64 ? 64 : (B <= 128 ? 128 : 256);
   const int n_tiles = cdiv(B, bn);
-  w.xproj_split = splits_for(cdiv(m.R + 2 * m.S, GEMM_BM) * n_tiles, cdiv(m.Di, 64), DEC_MAX_XPROJ_SPLIT);
+  w.xproj_split = splits_balanced(cdiv(m.R + 2 * m.S, GEMM_BM) * n_tiles, cdiv(m.Di, 64), DEC_MAX_XPROJ_SPLIT);
   w.xbc_part = take((size_t)w.xproj_split * B * m.ld_xbc * 4);
   w.y = take((size_t)B * m.Di * 4);
   w.u = take((size_t)B * m.uw * 2);
-  w.oproj_split = splits_for(cdiv(m.d, GEMM_BM) * n_tiles, cdiv(m.uw, 64), 32);
+  w.oproj_split = splits_balanced(cdiv(m.d, GEMM_BM) * n_tiles, cdiv(m.uw, 64), 32);
   w.acc_part = take((size_t)w.oproj_split * B * m.d * 4);
   w.total = off;
   return w;
@@ -1245,6 +1261,7 @@ static int decode_impl(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
   {
     GemmCall c;
     c.a1 = w->w_in; c.nb1 = 1; c.rows1 = m.P; c.lda1 = m.d; c.a1_bstride = (long long)m.P * m.d;
+    c.p.prefetch_a = 1;   // weights: their first stages load before the wait
     c.b = x; c.N = B; c.ldb = m.d; c.K = m.d;
     c.bn = pick_bn_cover(B);
     c.name = "decode_in_proj";
@@ -1297,6 +1314,7 @@ static int decode_impl(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
   SideStream* side = nullptr;
   HY_TRY(side_stream(&side));
   ForkGuard fork_guard(side, st);
+  int attn_items = 0;   // the attention's work items (its grid is min(items, 3 per SM))
   {
     const cudaStream_t ast = side->s;
     DecAttnParams ap;
@@ -1352,6 +1370,7 @@ static int decode_impl(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     // three CTAs per SM (four would fit).  (Measured: this order, with x_proj and the SSM
     // step queued behind the attention on the caller's stream, beat both x_proj first with
     // two attention CTAs per SM and a single stream.)
+    attn_items = ap.n_items;
     const int grid = ap.n_items < 3 * dev->sms ? ap.n_items : 3 * dev->sms;
     HY_CUDA(cudaEventRecord(side->fork, st));   // every host-side check has passed
     HY_CUDA(cudaStreamWaitEvent(ast, side->fork, 0));
@@ -1369,6 +1388,10 @@ static int decode_impl(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
   {
     GemmCall c;
     c.a1 = w->w_x; c.nb1 = 1; c.rows1 = m.R + 2 * m.S; c.lda1 = m.Di; c.a1_bstride = (long long)c.rows1 * m.Di;
+    c.p.prefetch_a = 1;   // weights: their first stages load before the wait
+    // when the attention grid leaves SM room (fewer items than its CTA slots), the SSM step's
+    // CTAs may take it early: their launch latency is then on the step's critical path
+    c.p.trigger_early = attn_items < 3 * dev->sms ? 1 : 0;
     c.b = bf(L.xc); c.N = B; c.ldb = m.Di; c.K = m.Di;
     c.bn = pick_bn_cover(B);
     c.name = "decode_x_proj";
@@ -1408,6 +1431,7 @@ static int decode_impl(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
   {
     GemmCall c;
     c.a1 = w->w_out; c.nb1 = 1; c.rows1 = m.d; c.lda1 = m.uw; c.a1_bstride = (long long)m.d * m.uw;
+    c.p.prefetch_a = 1;   // weights: their first stages load before the wait
     c.b = h16(L.u); c.N = B; c.ldb = m.uw; c.K = m.uw;
     c.etype = ET_F16;
     c.bn = pick_bn_cover(B);
@@ -1535,8 +1559,8 @@ FfnDecWs ffn_dec_layout(int rows, int d, int F) {
   FfnDecWs w;
   const int bn = rows <= 64 ? 64 : (rows <= 128 ? 128 : 256);
   const int nt = cdiv(rows, bn);
-  w.s1 = splits_for(cdiv(2 * F, GEMM_BM) * nt, cdiv(d, 64), 8);
-  w.s2 = splits_for(cdiv(d, GEMM_BM) * nt, cdiv(F, 64), 16);
+  w.s1 = splits_balanced(cdiv(2 * F, GEMM_BM) * nt, cdiv(d, 64), 8);
+  w.s2 = splits_balanced(cdiv(d, GEMM_BM) * nt, cdiv(F, 64), 16);
   size_t off = 256;
   auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
   w.part1 = take((size_t)w.s1 * rows * 2 * F * 4);
@@ -1549,8 +1573,29 @@ FfnDecWs ffn_dec_layout(int rows, int d, int F) {
 
 int hymba_ffn_workspace_size(int rows, int d, int F, size_t* bytes) {
   if (bytes == nullptr || rows < 1 || rows > 256 || d < 8 || d % 8 || F < 64 || F % 64)
-    return fail(HYMBA_ERR_INVALID_ARG, "ffn workspace arguments (rows 1..256, d % 8, F % 64)");
+    return fail(HYMBA_ERR_INVALID_ARG, "ffn workspace arguments (rows 1..256, d a multiple of 8, F of 64)");
   *bytes = ffn_dec_layout(rows, d, F).total;
+  return HYMBA_OK;
+}
+
+int hymba_l2_prefetch(const void* const* ranges, const size_t* bytes, int n_ranges, hymba_stream stream) {
+  if (ranges == nullptr || bytes == nullptr || n_ranges < 1 || n_ranges > L2PF_MAX_RANGES)
+    return fail(HYMBA_ERR_INVALID_ARG, "l2_prefetch: 1..8 ranges");
+  L2Ranges r{};
+  long long chunks = 0;
+  for (int i = 0; i < n_ranges; ++i) {
+    if (ranges[i] == nullptr || !aligned16(ranges[i])) return fail(HYMBA_ERR_INVALID_ARG, "l2_prefetch: range pointer");
+    r.ptr[i] = static_cast<const char*>(ranges[i]);
+    r.bytes[i] = bytes[i];
+    chunks += (long long)((bytes[i] + L2PF_CHUNK - 1) / L2PF_CHUNK);
+  }
+  r.n = n_ranges;
+  if (chunks == 0) return HYMBA_OK;
+  const int grid = (int)std::min<long long>(cdiv(chunks, (long long)L2PF_THREADS), 148);
+  prof_begin("l2_prefetch", (cudaStream_t)stream);
+  l2_prefetch_kernel<<<grid, L2PF_THREADS, 0, (cudaStream_t)stream>>>(r);
+  prof_end((cudaStream_t)stream);
+  HY_CUDA(cudaGetLastError());
   return HYMBA_OK;
 }
 
@@ -1576,6 +1621,7 @@ int hymba_ffn_swiglu_decode(const hymba_bf16* h, const hymba_bf16* w_gate_up, co
   {  // [gate | up] slices, transposed: part1[s][r][2F]
     GemmCall c;
     c.a1 = w_gate_up; c.nb1 = 1; c.rows1 = 2 * F; c.lda1 = d; c.a1_bstride = (long long)2 * F * d;
+    c.p.prefetch_a = 1;   // weights: their first stages load before the wait
     c.b = h; c.N = rows; c.ldb = d; c.K = d;
     c.bn = pick_bn_cover(rows);
     c.name = "ffn_dec_gate_up";
@@ -1599,6 +1645,7 @@ int hymba_ffn_swiglu_decode(const hymba_bf16* h, const hymba_bf16* w_gate_up, co
   {  // down projection slices part2[s][r][d], then their sum with the residual
     GemmCall c;
     c.a1 = w_down; c.nb1 = 1; c.rows1 = d; c.lda1 = F; c.a1_bstride = (long long)d * F;
+    c.p.prefetch_a = 1;   // weights: their first stages load before the wait
     c.b = act; c.N = rows; c.ldb = F; c.K = F;
     c.etype = ET_F16;
     c.bn = pick_bn_cover(rows);

@@ -952,4 +952,36 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, int n_split
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// L2 prefetch of read-only ranges (weights a later kernel of the same step streams).  One
+// thread per 32 KB chunk issues a bulk prefetch and exits: the copy engine brings the chunk
+// into L2 while the latency-bound kernels before its consumer run.  A hint only: nothing
+// waits for it, and a range's last partial 16 bytes are not prefetched.
+// ---------------------------------------------------------------------------------------
+constexpr int L2PF_MAX_RANGES = 8;
+constexpr unsigned L2PF_CHUNK = 32768;
+constexpr int L2PF_THREADS = 128;
+struct L2Ranges {
+  const char* ptr[L2PF_MAX_RANGES];
+  unsigned long long bytes[L2PF_MAX_RANGES];
+  int n;
+};
+
+__global__ void __launch_bounds__(L2PF_THREADS) l2_prefetch_kernel(L2Ranges r) {
+  long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  long long first = 0;   // chunk index of range k's first chunk
+  for (int k = 0; k < r.n; ++k) {
+    const long long nch = (long long)((r.bytes[k] + L2PF_CHUNK - 1) / L2PF_CHUNK);
+    for (; g < first + nch; g += stride) {
+      const unsigned long long off = (unsigned long long)(g - first) * L2PF_CHUNK;
+      const unsigned long long left = r.bytes[k] - off;
+      const unsigned size = (unsigned)(left < L2PF_CHUNK ? left : L2PF_CHUNK) & ~15u;
+      if (size > 0)
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(r.ptr[k] + off), "r"(size) : "memory");
+    }
+    first += nch;
+  }
+}
+
 }  // namespace hymba

@@ -123,6 +123,7 @@ def lib():
             "hymba_ffn_swiglu": ([_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp], _c_int),
             "hymba_ffn_workspace_size": ([_c_int, _c_int, _c_int, ctypes.POINTER(_c_size)], _c_int),
             "hymba_ffn_swiglu_decode": ([_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _c_size, _vp], _c_int),
+            "hymba_l2_prefetch": ([ctypes.POINTER(_vp), ctypes.POINTER(_c_size), _c_int, _vp], _c_int),
             "hymba_set_wait_limit_ns": ([ctypes.c_ulonglong], _c_int),
             "hymba_prepend_meta": ([_vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp], _c_int),
             "hymba_selftest_wait_timeout": ([_vp, _c_size, _vp], _c_int),
@@ -407,6 +408,14 @@ def ffn_swiglu_decode(h, w_gate_up, w_down, out, ws, residual=None, stream=None)
     F = w_down.shape[1]
     check(lib().hymba_ffn_swiglu_decode(ptr(h), ptr(w_gate_up), ptr(w_down), rows, d, F, ptr(residual), ptr(out),
                                         ptr(ws), ws.numel(), stream_handle(stream)))
+
+
+def l2_prefetch(tensors, stream=None):
+    """hymba_l2_prefetch: an L2 prefetch hint for up to 8 device tensors (read-only ranges)."""
+    n = len(tensors)
+    ptrs = (_vp * n)(*[t.data_ptr() for t in tensors])
+    sizes = (_c_size * n)(*[t.numel() * t.element_size() for t in tensors])
+    check(lib().hymba_l2_prefetch(ptrs, sizes, n, stream_handle(stream)))
 
 
 def profile_begin(max_records=8192):

@@ -353,6 +353,15 @@ int hymba_ffn_swiglu_decode(const hymba_bf16* h, const hymba_bf16* w_gate_up, co
                             int d, int F, const hymba_bf16* residual, hymba_bf16* out, void* workspace,
                             size_t ws_bytes, hymba_stream stream);
 
+/* L2 prefetch hint for read-only device ranges that a later kernel on another stream (or
+ * later on this one) will stream, e.g. the weights of a decode step's projections while the
+ * latency-bound attention and scan kernels before them run.  ranges[i] / bytes[i]: up to 8
+ * device pointers (16-byte aligned) and sizes, both arrays on the host; the call only enqueues
+ * one kernel that issues bulk L2 prefetches of 32 KB pieces and returns without waiting for
+ * them.  No result is defined and no memory is written: a hint the hardware may drop.
+ * Errors: HYMBA_ERR_INVALID_ARG for n_ranges outside 1..8, a null or misaligned pointer. */
+int hymba_l2_prefetch(const void* const* ranges, const size_t* bytes, int n_ranges, hymba_stream stream);
+
 /* Meta-token prefix of a stack's residual stream ([JJ] §数学表示 1: X~ = [R, X]):
  * out[b] = [meta; x[b]], meta [n_meta, d], x [B, n_tokens, d], out [B, n_meta + n_tokens, d],
  * all bf16, d % 8 == 0. */
