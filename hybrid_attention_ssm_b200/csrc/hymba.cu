@@ -1407,12 +1407,25 @@ static int decode_impl(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
   }
   // 5. dt_proj + softplus + state update + C.h + gate
   {
-    dim3 grid(m.Di / DSSM_NC, cdiv(B, DSSM_NB));
+    // four sequences per thread from 64 sequences on (each W_dt row read feeds four dot
+    // products); below that one, so that a small batch still spreads over the SMs
+    static size_t attr_ssm[64][2] = {};   // dynamic shared memory allowed so far
+    int dcur = 0;
+    HY_CUDA(cudaGetDevice(&dcur));
+    const int wide = B >= 64 ? 1 : 0;
+    auto kern = wide ? decode_ssm_kernel<4> : decode_ssm_kernel<1>;
+    const int nb = wide ? 16 : 4;
+    const size_t smem = dssm_smem_bytes(nb / 4, L.xproj_split, m.ld_xbc, m.R);
+    if (smem > attr_ssm[dcur & 63][wide]) {
+      HY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+      attr_ssm[dcur & 63][wide] = smem;
+    }
+    dim3 grid(m.Di / DSSM_NC, cdiv(B, nb));
     prof_begin("decode_ssm", st);
-    HY_CUDA(launch_pdl(decode_ssm_kernel, grid, dim3(DSSM_THREADS), dssm_smem_bytes(m.R), st, f32(L.xbc_part),
-                       (long long)B * m.ld_xbc, L.xproj_split, m.ld_xbc, m.R, w->w_dt, w->w_dt_ld,
+    HY_CUDA(launch_pdl(kern, grid, dim3(DSSM_THREADS), smem, st,
+                       f32(L.xbc_part), (long long)B * m.ld_xbc, L.xproj_split, m.ld_xbc, m.R, w->w_dt, w->w_dt_ld,
                        w->dt_bias, w->A, bf(L.xc), f32(L.proj), m.P, (long long)B * m.P, L.in_split,
-                       m.xz_off + m.Di, ssm_state, f32(L.y), m.Di, B));
+                       m.xz_off + m.Di, ssm_state, f32(L.y), m.Di, B, status));
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }

@@ -621,52 +621,62 @@ __global__ void decode_attn_combine_kernel(const float* __restrict__ part, int n
 
 // ----------------------------------------------------------------------------------------
 // decode SSM step ([JJ] §数学表示 4, one step of eq. (2)): dt = softplus(dt_low . W_dt[c] +
-// bias), h = exp(dt A) h + dt B x, y = (C . h) * SiLU(z).  Thread = one channel x four
-// sequences, their 4 x 16 states in registers (64 contiguous bytes per sequence, 16-byte
-// loads issued before anything else); CTA = 32 channels x 16 sequences.  The CTA's W_dt
-// rows and the sequences' dt_low, B and C rows are staged transposed in shared memory once,
-// so that one W_dt value and one 16-byte broadcast of four sequences' dt_low feed four FMAs.
-//   xbc: n_xbc split-K slices [B, ld_xbc] fp32 (stride xbc_stride) summed here in order:
-//   dt_low at 0..R-1, B at R.., C at R+16..; W_dt [Di, ld_dt] fp32;
-//   xc [B, Di] bf16; z from the in_proj slices (stride proj_stride) at column off_z; state
-//   [B, Di, 16] in place; y [B, Di] fp32.  R <= 224.
+// bias), h = exp(dt A) h + dt B x, y = (C . h) * SiLU(z).
+// CTA = 64 channels x NB sequences, 256 threads; thread = one channel x BPT sequences
+// (NB = 4 BPT), their BPT x 16 states in registers.  Everything the CTA reads arrives in one
+// round: bulk copies bring the x_proj slices of its sequences and the W_dt rows of its
+// channels into shared memory while every thread loads its states, x, z and A row; the
+// slices are then added in slice order in shared memory.
+//   xbc: n_xbc split-K slices [B, ld_xbc] fp32 (stride xbc_stride): dt_low at 0..R-1, B at
+//   R.., C at R+16..; W_dt [Di, ld_dt] fp32; xc [B, Di] bf16; z from the in_proj slices
+//   (stride proj_stride) at column off_z; state [B, Di, 16] in place; y [B, Di] fp32.
+//   R % 4 == 0, ld_xbc % 4 == 0, Di % 64 == 0; 16-byte aligned rows.
 // ----------------------------------------------------------------------------------------
-constexpr int DSSM_NC = 32;    // channels per CTA: one per lane
-constexpr int DSSM_NB = 16;    // sequences per CTA
-constexpr int DSSM_BPT = 4;    // sequences per thread; the lanes of a warp share them
-constexpr int DSSM_THREADS = DSSM_NC * DSSM_NB / DSSM_BPT;   // 128
-constexpr int DSSM_A_LD = 20;  // A rows in shared memory (16 + 4: conflict-free 16-byte reads)
-// dynamic shared memory: W_dt rows of the CTA's channels [R][32] and the summed x_proj
-// outputs of its sequences [R + 32][16] (dt_low | B | C), both transposed, then the
-// channels' A * log2(e) rows [32][20] and dt biases [32]
-__host__ __device__ constexpr size_t dssm_smem_bytes(int R) {
-  return ((size_t)R * DSSM_NC + (size_t)(R + 32) * DSSM_NB + DSSM_NC * DSSM_A_LD + DSSM_NC) * sizeof(float);
+constexpr int DSSM_NC = 64;        // channels per CTA
+constexpr int DSSM_THREADS = 256;
+// dynamic shared memory: the x_proj slices [n_xbc][NB][ld_xbc], W_dt rows [64][R], mbarrier
+__host__ __device__ constexpr size_t dssm_smem_bytes(int bpt, int n_xbc, int ld_xbc, int R) {
+  return ((size_t)n_xbc * 4 * bpt * ld_xbc + (size_t)DSSM_NC * R) * sizeof(float) + 16;
 }
 
-__global__ void __launch_bounds__(DSSM_THREADS, 3)
+template <int BPT>
+__global__ void __launch_bounds__(DSSM_THREADS, BPT == 1 ? 3 : 2)
     decode_ssm_kernel(const float* __restrict__ xbc, long long xbc_stride, int n_xbc, int ld_xbc, int R,
                       const float* __restrict__ w_dt, int ld_dt,
                       const float* __restrict__ dt_bias, const float* __restrict__ A,
                       const __nv_bfloat16* __restrict__ xc, const float* __restrict__ proj, int ld_proj,
                       long long proj_stride, int n_slices, int off_z, float* __restrict__ state,
-                      float* __restrict__ y, int Di, int B) {
-  pdl_wait();
-  pdl_trigger();
-  extern __shared__ __align__(16) float dssm_sh[];
-  float* wsh = dssm_sh;                    // W_dt[c0 + cl][r] at r * 32 + cl
-  float* dlT = dssm_sh + R * DSSM_NC;      // x_proj output [b0 + bl][col] at col * 16 + bl
-  float* ash = dlT + (R + 32) * DSSM_NB;   // A[c0 + cl][s] * log2(e) at cl * 20 + s
-  float* bsh = ash + DSSM_NC * DSSM_A_LD;  // dt_bias[c0 + cl]
+                      float* __restrict__ y, int Di, int B, DevStatus* status) {
+  constexpr int NB = 4 * BPT;   // sequences per CTA
+  // Unlike the other kernels, this one reads part of its input before pdl_wait(): the
+  // states (written only by this kernel, in an earlier step), A, dt_bias and W_dt.  Its
+  // launch implies that the kernel two places before it on the stream has completed (each
+  // kernel lets the next one launch only after its own wait, or, the x_proj GEMM before
+  // this one, after its launch), so every earlier writer of the states is done; the reads
+  // overlap the x_proj GEMM.  What that GEMM and the prep kernel write (the x_proj slices,
+  // x and z) is read after the wait.
+  extern __shared__ __align__(128) float dssm_sh[];
+  float* xs = dssm_sh;                                  // slice k, sequence bl: xs[(k * NB + bl) * ld_xbc]
+  float* wsh = xs + (size_t)n_xbc * NB * ld_xbc;        // W_dt row cl: wsh[cl * R]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(wsh + DSSM_NC * R);
+  __shared__ int ok_sh;
   const int tid = threadIdx.x;
   const int cl = tid & (DSSM_NC - 1), bq = tid / DSSM_NC;
-  const int c0 = blockIdx.x * DSSM_NC, b0 = blockIdx.y * DSSM_NB;
+  const int c0 = blockIdx.x * DSSM_NC, b0 = blockIdx.y * NB;
   const int c = c0 + cl;
-  // this thread's states (four sequences x 16) first: their loads overlap the staging
-  float h[DSSM_BPT][16];
-  float xv[DSSM_BPT], zv[DSSM_BPT];
+  const int nb = min(NB, B - b0);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(bar, (uint32_t)(((size_t)n_xbc * nb * ld_xbc + (size_t)DSSM_NC * R) * sizeof(float)));
+  }
+  __syncthreads();   // the expected byte count is set before any copy can complete
+  if (tid < DSSM_NC)
+    bulk_load(wsh + tid * R, w_dt + (size_t)(c0 + tid) * ld_dt, (uint32_t)(R * sizeof(float)), bar);
+  float h[BPT][16];
 #pragma unroll
-  for (int j = 0; j < DSSM_BPT; ++j) {
-    const int b = b0 + bq * DSSM_BPT + j;
+  for (int j = 0; j < BPT; ++j) {
+    const int b = b0 + bq * BPT + j;
     if (b < B) {
       const float* hp = state + ((size_t)b * Di + c) * 16;
 #pragma unroll
@@ -674,111 +684,96 @@ __global__ void __launch_bounds__(DSSM_THREADS, 3)
         const float4 v = *reinterpret_cast<const float4*>(hp + k);
         h[j][k] = v.x; h[j][k + 1] = v.y; h[j][k + 2] = v.z; h[j][k + 3] = v.w;
       }
-      xv[j] = __bfloat162float(xc[(size_t)b * Di + c]);
-      zv[j] = sum_slices<DEC_MAX_IN_SPLIT>(proj + (size_t)b * ld_proj + off_z + c, proj_stride, n_slices);
     } else {
 #pragma unroll
       for (int k = 0; k < 16; ++k) h[j][k] = 0.f;
-      xv[j] = 0.f;
-      zv[j] = 0.f;
     }
   }
-  // the channels' A rows and dt biases ride with the W_dt loads (one 16-byte piece of A per thread)
-  static_assert(DSSM_THREADS == DSSM_NC * 4, "one quarter of an A row per thread");
-  const float4 a_in = *reinterpret_cast<const float4*>(A + (size_t)(c0 + (tid >> 2)) * 16 + (tid & 3) * 4);
-  const float bias_in = tid < DSSM_NC ? dt_bias[c0 + tid] : 0.f;
-  // W_dt rows, transposed (R % 4 == 0); four loads in flight per thread
-  {
-    const int n_items = DSSM_NC * (R >> 2);
-    for (int i0 = tid; i0 < n_items; i0 += 4 * DSSM_THREADS) {
-      float4 v[4];
+  float a2[16];   // A[c] * log2(e): exp(dt A) = 2^(dt A log2 e)
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = i0 + u * DSSM_THREADS;
-        if (i < n_items)
-          v[u] = *reinterpret_cast<const float4*>(w_dt + (size_t)(c0 + (i & (DSSM_NC - 1))) * ld_dt + (i / DSSM_NC) * 4);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = i0 + u * DSSM_THREADS;
-        if (i < n_items) {
-          float* w = wsh + (i / DSSM_NC) * 4 * DSSM_NC + (i & (DSSM_NC - 1));
-          w[0] = v[u].x; w[DSSM_NC] = v[u].y; w[2 * DSSM_NC] = v[u].z; w[3 * DSSM_NC] = v[u].w;
-        }
-      }
-    }
+  for (int k = 0; k < 16; k += 4) {
+    const float4 v = *reinterpret_cast<const float4*>(A + (size_t)c * 16 + k);
+    a2[k] = v.x * 1.4426950408889634f; a2[k + 1] = v.y * 1.4426950408889634f;
+    a2[k + 2] = v.z * 1.4426950408889634f; a2[k + 3] = v.w * 1.4426950408889634f;
   }
-  *reinterpret_cast<float4*>(ash + (tid >> 2) * DSSM_A_LD + (tid & 3) * 4) =
-      make_float4(a_in.x * 1.4426950408889634f, a_in.y * 1.4426950408889634f, a_in.z * 1.4426950408889634f,
-                  a_in.w * 1.4426950408889634f);   // exp(dt*A) = 2^(dt*A*log2 e)
-  if (tid < DSSM_NC) bsh[tid] = bias_in;
-  // x_proj outputs of the CTA's sequences, their split-K slices summed in a fixed order;
-  // item i = (column quad i / 16, sequence i % 16): lanes l and l + 16 read one 32-byte sector
+  const float bias = dt_bias[c];
+  pdl_wait();
+  pdl_trigger();
+  if (tid >= DSSM_NC && tid < DSSM_NC + n_xbc) {
+    const int k = tid - DSSM_NC;
+    bulk_load(xs + (size_t)k * NB * ld_xbc, xbc + k * xbc_stride + (size_t)b0 * ld_xbc,
+              (uint32_t)((size_t)nb * ld_xbc * sizeof(float)), bar);
+  }
+  float xv[BPT], zv[BPT];
+#pragma unroll
+  for (int j = 0; j < BPT; ++j) {
+    const int b = b0 + bq * BPT + j;
+    xv[j] = b < B ? __bfloat162float(xc[(size_t)b * Di + c]) : 0.f;
+    zv[j] = b < B ? sum_slices<DEC_MAX_IN_SPLIT>(proj + (size_t)b * ld_proj + off_z + c, proj_stride, n_slices) : 0.f;
+  }
+  if (tid == 0) ok_sh = mbar_wait(bar, 0, nullptr, status, 250) ? 1 : 0;
+  __syncthreads();
+  if (!ok_sh) return;
+  // add the slices in slice order into slice 0 (16-byte pieces of the [nb][ld_xbc] block)
   {
-    const int n_items = DSSM_NB * ((R + 32) >> 2);
-    for (int i = tid; i < n_items; i += DSSM_THREADS) {
-      const int bl = i & (DSSM_NB - 1), q = i / DSSM_NB;
-      const bool ok = b0 + bl < B;
-      const float* src = xbc + (size_t)(b0 + bl) * ld_xbc + q * 4;
-      float4 v[DEC_MAX_XPROJ_SPLIT];
-#pragma unroll
-      for (int k = 0; k < DEC_MAX_XPROJ_SPLIT; ++k)
-        v[k] = (ok && k < n_xbc) ? *reinterpret_cast<const float4*>(src + k * xbc_stride) : make_float4(0.f, 0.f, 0.f, 0.f);
-      float4 acc = v[0];
-#pragma unroll
-      for (int k = 1; k < DEC_MAX_XPROJ_SPLIT; ++k) {
-        acc.x += v[k].x; acc.y += v[k].y; acc.z += v[k].z; acc.w += v[k].w;
+    const int n4 = nb * ld_xbc / 4;
+    const size_t sstride = (size_t)NB * ld_xbc;
+    for (int i = tid; i < n4; i += DSSM_THREADS) {
+      float4 acc = reinterpret_cast<const float4*>(xs)[i];
+      for (int k = 1; k < n_xbc; ++k) {
+        const float4 v = reinterpret_cast<const float4*>(xs + k * sstride)[i];
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
       }
-      float* d = dlT + q * 4 * DSSM_NB + bl;
-      d[0] = acc.x; d[DSSM_NB] = acc.y; d[2 * DSSM_NB] = acc.z; d[3 * DSSM_NB] = acc.w;
+      reinterpret_cast<float4*>(xs)[i] = acc;
     }
   }
   __syncthreads();
-  // dt_low . W_dt[c] for the four sequences (two partial sums each)
-  float acc[2][DSSM_BPT];
+  // dt_low . W_dt[c] for the thread's sequences (the warp's lanes share the sequences, so
+  // the dt_low reads are broadcasts)
+  float dt[BPT], dtx[BPT], yv[2][BPT];
+  {
+    float acc[BPT][2];
 #pragma unroll
-  for (int j = 0; j < DSSM_BPT; ++j) acc[0][j] = acc[1][j] = 0.f;
-  const float* dq = dlT + bq * DSSM_BPT;
+    for (int j = 0; j < BPT; ++j) acc[j][0] = acc[j][1] = 0.f;
+    const float* wr = wsh + cl * R;
 #pragma unroll 2
-  for (int r = 0; r < R; r += 2) {     // R even
+    for (int r = 0; r < R; r += 4) {
+      const float4 w = *reinterpret_cast<const float4*>(wr + r);
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const float w = wsh[(r + e) * DSSM_NC + cl];
-      const float4 d = *reinterpret_cast<const float4*>(dq + (r + e) * DSSM_NB);
-      acc[e][0] = fmaf(d.x, w, acc[e][0]);
-      acc[e][1] = fmaf(d.y, w, acc[e][1]);
-      acc[e][2] = fmaf(d.z, w, acc[e][2]);
-      acc[e][3] = fmaf(d.w, w, acc[e][3]);
+      for (int j = 0; j < BPT; ++j) {
+        const float4 d = *reinterpret_cast<const float4*>(xs + (bq * BPT + j) * ld_xbc + r);
+        acc[j][0] = fmaf(d.x, w.x, acc[j][0]);
+        acc[j][1] = fmaf(d.y, w.y, acc[j][1]);
+        acc[j][0] = fmaf(d.z, w.z, acc[j][0]);
+        acc[j][1] = fmaf(d.w, w.w, acc[j][1]);
+      }
     }
-  }
-  const float bias = bsh[cl];
-  float dt[DSSM_BPT], dtx[DSSM_BPT], yv[2][DSSM_BPT];
 #pragma unroll
-  for (int j = 0; j < DSSM_BPT; ++j) {
-    dt[j] = softplus_f(acc[0][j] + acc[1][j] + bias);
-    dtx[j] = dt[j] * xv[j];
-    yv[0][j] = yv[1][j] = 0.f;
+    for (int j = 0; j < BPT; ++j) {
+      dt[j] = softplus_f(acc[j][0] + acc[j][1] + bias);
+      dtx[j] = dt[j] * xv[j];
+      yv[0][j] = yv[1][j] = 0.f;
+    }
   }
 #pragma unroll
   for (int k = 0; k < 16; k += 4) {
-    const float4 a4 = *reinterpret_cast<const float4*>(ash + cl * DSSM_A_LD + k);
-    const float a2[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int s = k + e;
-      const float4 b4 = *reinterpret_cast<const float4*>(dq + (R + s) * DSSM_NB);
-      const float4 c4 = *reinterpret_cast<const float4*>(dq + (R + 16 + s) * DSSM_NB);
+    for (int j = 0; j < BPT; ++j) {
+      const float* row = xs + (bq * BPT + j) * ld_xbc + R;
+      const float4 b4 = *reinterpret_cast<const float4*>(row + k);
+      const float4 c4 = *reinterpret_cast<const float4*>(row + 16 + k);
       const float bv[4] = {b4.x, b4.y, b4.z, b4.w}, cv[4] = {c4.x, c4.y, c4.z, c4.w};
 #pragma unroll
-      for (int j = 0; j < DSSM_BPT; ++j) {
-        h[j][s] = fmaf(ex2_approx(dt[j] * a2[e]), h[j][s], dtx[j] * bv[j]);
-        yv[s & 1][j] = fmaf(cv[j], h[j][s], yv[s & 1][j]);
+      for (int e = 0; e < 4; ++e) {
+        const int s = k + e;
+        h[j][s] = fmaf(ex2_approx(dt[j] * a2[s]), h[j][s], dtx[j] * bv[e]);
+        yv[s & 1][j] = fmaf(cv[e], h[j][s], yv[s & 1][j]);
       }
     }
   }
 #pragma unroll
-  for (int j = 0; j < DSSM_BPT; ++j) {
-    const int b = b0 + bq * DSSM_BPT + j;
+  for (int j = 0; j < BPT; ++j) {
+    const int b = b0 + bq * BPT + j;
     if (b >= B) continue;
     float* hp = state + ((size_t)b * Di + c) * 16;
 #pragma unroll
