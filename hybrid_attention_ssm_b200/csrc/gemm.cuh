@@ -10,7 +10,15 @@
 //               column chunks between them (two epilogue warps per SM sub-partition).
 // The accumulator is double-buffered in TMEM so the epilogue of tile i overlaps the
 // mainloop of tile i+1.  The epilogue is a template parameter, so each instance carries
-// only its own code.  Each CTA loads its own tiles; no thread-block clusters.
+// only its own code.
+//
+// PAIR: the CTAs run as clusters of two on two SMs, and one tcgen05.mma.cta_group::2 of
+// M = 256 covers both CTAs' 128-row A tiles against a BN-wide B tile of which each CTA holds
+// one half: per k-block an SM then moves 16 KB of A and BN/2 x 128 B of B into shared memory
+// instead of 16 KB + BN x 128 B, for the same MMA work.  Each CTA loads its own tiles (no
+// multicast loads); the loads of both complete on the even CTA's barrier, whose single MMA
+// thread issues the pair's MMAs and commits them to both CTAs' barriers.  Each CTA's
+// epilogue reads its own TMEM rows, as in the single-CTA form.
 #pragma once
 #include "common.cuh"
 
@@ -51,6 +59,7 @@ struct GemmParams {
   // output row mapping: a source-0 row r goes to rows {b*T_out + r}, b < out_batches;
   // a source-1 row (b, r) goes to b*T_out + row_off1 + r (position row_off1 + r)
   int out_batches, T_out, row_off1;
+  int m_pairs;              // PAIR: cdiv(m_tiles, 2); total_tiles counts pair tiles
   // 1: only the epilogue warps wait for the previous kernel on the stream.  For a GEMM whose
   // operands no kernel of the same call writes (the caller's input and the weights), so the
   // mainloop overlaps a previous kernel that only prepares what the epilogue reads.
@@ -88,10 +97,10 @@ __host__ __device__ constexpr int gemm_epi_bytes(int mode) {
   return mode == 3 /* EPI_F32_ROWS */ ? GEMM_EPI_WARPS * 32 * 33 * 4 : 0;
 }
 
-template <int BN, int STAGES, int EPI_BYTES = 0>
+template <int BN, int STAGES, int EPI_BYTES = 0, bool PAIR = false>
 struct GemmSmem {
   static constexpr int A_BYTES = GEMM_BM * 128;
-  static constexpr int B_BYTES = BN * 128;
+  static constexpr int B_BYTES = (PAIR ? BN / 2 : BN) * 128;   // PAIR: this CTA's half of the B tile
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
   static constexpr int EPI_OFFSET = BAR_OFFSET + 256;
@@ -139,16 +148,19 @@ __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t* r) {
 // element types of both operands: bf16, fp16 (kind::f16) or fp32 read as tf32 (kind::tf32)
 enum : int { ET_BF16 = 0, ET_F16 = 1, ET_TF32 = 2 };
 
-template <int BN, int STAGES, int ET, int MODE>
+template <int BN, int STAGES, int ET, int MODE, bool PAIR = false>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA0, const __grid_constant__ CUtensorMap mapA1,
                    const __grid_constant__ CUtensorMap mapB, const __grid_constant__ GemmParams p) {
-  using L = GemmSmem<BN, STAGES, gemm_epi_bytes(MODE)>;
+  using L = GemmSmem<BN, STAGES, gemm_epi_bytes(MODE), PAIR>;
   static_assert(L::TOTAL <= 232448, "shared memory of one CTA");
+  static_assert(!PAIR || (ET != ET_TF32 && BN % 32 == 0), "pair tiles: 16-bit operands, BN / 2 a multiple of 16");
+  static_assert(L::STAGE_BYTES % 1024 == 0, "stage buffers keep the 1024-byte swizzle alignment");
   constexpr int ACC_STRIDE = BN <= 128 ? 128 : 256;       // TMEM columns per accumulator
   constexpr uint32_t TMEM_COLS = 2 * ACC_STRIDE;
   constexpr bool TF32 = ET == ET_TF32;
-  constexpr uint32_t IDESC = make_idesc(GEMM_BM, BN, ET == ET_TF32 ? 2u : (ET == ET_BF16 ? 1u : 0u), false, false);
+  constexpr uint32_t IDESC =
+      make_idesc(PAIR ? 2 * GEMM_BM : GEMM_BM, BN, ET == ET_TF32 ? 2u : (ET == ET_BF16 ? 1u : 0u), false, false);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem<1024>(smem_raw);
@@ -161,6 +173,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // PAIR: rank in the pair (its M tile is 2 * pair + rank) and the pair's tile stream
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int tile0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int tile_step = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  const int m_count = PAIR ? p.m_pairs : p.m_tiles;
+  auto tile_m = [&](int t2) { return PAIR ? 2 * (t2 % m_count) + (int)rank : t2 % m_count; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -169,7 +187,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], GEMM_EPI_WARPS);
+      mbar_init(&acc_empty[b], PAIR ? 2 * GEMM_EPI_WARPS : GEMM_EPI_WARPS);   // PAIR: both CTAs' epilogues
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -180,11 +198,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     tma_prefetch_desc(&mapB);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();   // both CTAs' barriers and TMEM exist before either signals the other
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // The set-up above touches only this CTA's shared memory, its TMEM and the kernel
@@ -214,7 +238,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       // 0..pre-1 of the first tile, loaded before the wait with the stage's full byte count
       // expected, so their B loads below complete them
       uint32_t pre = 0;
-      if (p.prefetch_a) {
+      if (!PAIR && p.prefetch_a) {
         if ((int)blockIdx.x < p.total_tiles) {
           const int tile = blockIdx.x;
           const int ks = tile % p.split_k;
@@ -232,11 +256,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       uint32_t it = 0;
       // the first tile is always entered when it has A tiles in flight: their stages get
       // their B loads before any wait, so the drain below finds every issued stage complete
-      for (int tile = blockIdx.x; tile < p.total_tiles && (it < pre || !*abort_flag); tile += gridDim.x) {
+      for (int tile = tile0; tile < p.total_tiles && (it < pre || !*abort_flag); tile += tile_step) {
         const int ks = tile % p.split_k;
         const int t2 = tile / p.split_k;
-        const int m = t2 % p.m_tiles;
-        const int n = t2 / p.m_tiles;
+        const int m = tile_m(t2);
+        const int n = t2 / m_count;
         const int kb0 = (int)((long long)ks * p.k_blocks / p.split_k);
         const int kb1 = (int)((long long)(ks + 1) * p.k_blocks / p.split_k);
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
@@ -245,25 +269,46 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           uint8_t* sa = smem + s * L::STAGE_BYTES;
           uint8_t* sb = sa + L::A_BYTES;
           const int kc = kb * (TF32 ? 32 : 64);
-          if (it >= pre) {
+          if constexpr (PAIR) {
+            // both CTAs' A tiles and B halves complete on the even CTA's full[s]; that CTA
+            // expects the bytes of both
             if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status, 101)) break;
-            mbar_arrive_expect_tx(&full[s], L::STAGE_BYTES);
-            load_a(sa, &full[s], m, kc);
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * L::STAGE_BYTES);
+            const uint32_t bar = smem_cluster_addr(&full[s], 0);
+            if (m < p.tiles0) {
+              tma_load_2d_pair(sa, &mapA0, bar, kc, m * GEMM_BM);
+            } else {
+              const int idx = m - p.tiles0;   // past the last tile (odd count): a zero-filled tile
+              tma_load_3d_pair(sa, &mapA1, bar, kc, (idx % p.tiles1) * GEMM_BM, idx / p.tiles1);
+            }
+            tma_load_2d_pair(sb, &mapB, bar, kc, n * BN + (int)rank * (BN / 2));
+          } else {
+            if (it >= pre) {
+              if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status, 101)) break;
+              mbar_arrive_expect_tx(&full[s], L::STAGE_BYTES);
+              load_a(sa, &full[s], m, kc);
+            }
+            tma_load_2d(sb, &mapB, &full[s], kc, n * BN);
           }
-          tma_load_2d(sb, &mapB, &full[s], kc, n * BN);
         }
       }
       // Drain: wait until every load issued has landed (their consumer may have given up).
-      for (uint32_t j = (it > (uint32_t)STAGES ? it - STAGES : 0u); j < it; ++j) {
-        mbar_wait(&full[j % STAGES], (j / STAGES) & 1u, nullptr, p.status, 102);
+      // PAIR: the loads complete on the even CTA's barriers, which that CTA drains; the odd
+      // CTA's last loads have landed once the even CTA's MMAs have consumed them, before the
+      // closing cluster barrier.
+      if (!PAIR || rank == 0) {
+        for (uint32_t j = (it > (uint32_t)STAGES ? it - STAGES : 0u); j < it; ++j) {
+          mbar_wait(&full[j % STAGES], (j / STAGES) & 1u, nullptr, p.status, 102);
+        }
       }
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer ------------------------------
-    if (lane == 0) {
+    // PAIR: the even CTA's thread issues the pair's MMAs; the odd CTA's warp 1 only holds TMEM
+    if (lane == 0 && (!PAIR || rank == 0)) {
       uint32_t it = 0;
       int lt = 0;
-      for (int tile = blockIdx.x; tile < p.total_tiles && !*abort_flag; tile += gridDim.x, ++lt) {
+      for (int tile = tile0; tile < p.total_tiles && !*abort_flag; tile += tile_step, ++lt) {
         const int ks = tile % p.split_k;
         const int kb0 = (int)((long long)ks * p.k_blocks / p.split_k);
         const int kb1 = (int)((long long)(ks + 1) * p.k_blocks / p.split_k);
@@ -285,13 +330,24 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             const uint64_t ad = make_sdesc_sw128(sa + kk * 32, 16, 1024);
             const uint64_t bd = make_sdesc_sw128(sb + kk * 32, 16, 1024);
             const uint32_t acc = (kb > kb0 || kk > 0) ? 1u : 0u;
-            if (TF32) umma_tf32(d_tmem, ad, bd, IDESC, acc);
+            if constexpr (PAIR) umma_f16_pair(d_tmem, ad, bd, IDESC, acc);
+            else if (TF32) umma_tf32(d_tmem, ad, bd, IDESC, acc);
             else umma_f16(d_tmem, ad, bd, IDESC, acc);
           }
-          umma_commit(&empty[s]);
+          if constexpr (PAIR) {   // both CTAs' stage s is free
+            umma_commit_pair(smem_cluster_addr(&empty[s], 0));
+            umma_commit_pair(smem_cluster_addr(&empty[s], 1));
+          } else {
+            umma_commit(&empty[s]);
+          }
         }
         if (!ok) break;
-        umma_commit(&acc_full[ab]);
+        if constexpr (PAIR) {
+          umma_commit_pair(smem_cluster_addr(&acc_full[ab], 0));
+          umma_commit_pair(smem_cluster_addr(&acc_full[ab], 1));
+        } else {
+          umma_commit(&acc_full[ab]);
+        }
       }
     }
   } else {
@@ -300,11 +356,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const int half = (warp - 2) >> 2;        // which of the quadrant's two warps (column chunks)
     const int r = quad * 32 + lane;          // accumulator row of this thread
     int lt = 0;
-    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++lt) {
+    for (int tile = tile0; tile < p.total_tiles; tile += tile_step, ++lt) {
       const int ks = tile % p.split_k;
       const int t2 = tile / p.split_k;
-      const int m = t2 % p.m_tiles;
-      const int n = t2 / p.m_tiles;
+      const int m = tile_m(t2);
+      const int n = t2 / m_count;
       const int ab = lt & 1;
       const uint32_t aph = (lt >> 1) & 1u;
       int ok = 1;
@@ -324,7 +380,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         b1 = idx / p.tiles1;
         rr = (idx % p.tiles1) * GEMM_BM + r;
       }
-      const bool row_ok = src0 ? (rr < p.rows0) : (rr < p.rows1);
+      const bool row_ok = m < p.m_tiles && (src0 ? (rr < p.rows0) : (rr < p.rows1));
       const int col_base = n * BN;
 
       if constexpr (MODE == EPI_PROJ || MODE == EPI_SWIGLU) {
@@ -467,15 +523,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      if (lane == 0) {
+        if constexpr (PAIR) mbar_arrive_cluster(smem_cluster_addr(&acc_empty[ab], 0));
+        else mbar_arrive(&acc_empty[ab]);
+      }
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();   // no CTA leaves while the other may still signal or read it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 

@@ -227,25 +227,73 @@ struct GemmCall {
   int mode = EPI_BF16;
   int bn = 256;
   int split_k = 1;
+  // CTA pairs (cta_group::2, clusters of two): 256-row pair tiles, each CTA loading half of
+  // the B tile.  Instantiated for the large prefill GEMMs only.
+  bool pair = false;
   GemmParams p{};
 };
 
-template <int BN, int STAGES, int ET, int MODE>
+template <int BN, int STAGES, int ET, int MODE, bool PAIR = false>
 int launch_gemm_inst(const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& mb, const GemmParams& p,
                      int grid, cudaStream_t st, const char* name) {
   static bool attr_set[64] = {false};
+  static int max_pairs[64] = {0};   // PAIR: clusters of two that fit on the device at once
   int dev = 0;
   cudaGetDevice(&dev);
-  constexpr int smem = GemmSmem<BN, STAGES, gemm_epi_bytes(MODE)>::TOTAL;
-  auto kern = gemm_tc_kernel<BN, STAGES, ET, MODE>;
+  constexpr int smem = GemmSmem<BN, STAGES, gemm_epi_bytes(MODE), PAIR>::TOTAL;
+  auto kern = gemm_tc_kernel<BN, STAGES, ET, MODE, PAIR>;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   if (!attr_set[dev & 63]) {
     HY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    if constexpr (PAIR) {
+      // A persistent grid of pairs must be resident at once: a GPC with an odd number of free
+      // SMs leaves one out, so ask the occupancy calculator rather than halving the SM count.
+      cudaLaunchConfig_t q{};
+      q.gridDim = dim3(2);
+      q.blockDim = dim3(GEMM_THREADS);
+      q.dynamicSmemBytes = smem;
+      q.attrs = attr + 1;
+      q.numAttrs = 1;
+      int n = 0;
+      HY_CUDA(cudaOccupancyMaxActiveClusters(&n, kern, &q));
+      if (n < 1) return fail(HYMBA_ERR_UNSUPPORTED, "no SM pair can hold a %d-byte GEMM CTA", smem);
+      max_pairs[dev & 63] = n;
+    }
     attr_set[dev & 63] = true;
   }
   prof_begin(name, st);
-  HY_CUDA(launch_pdl(kern, dim3(grid), dim3(GEMM_THREADS), smem, st, m0, m1, mb, p));
+  if constexpr (PAIR) {
+    const int pairs = p.total_tiles < max_pairs[dev & 63] ? p.total_tiles : max_pairs[dev & 63];
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(GEMM_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    HY_CUDA(cudaLaunchKernelEx(&cfg, kern, m0, m1, mb, p));
+  } else {
+    (void)attr;
+    HY_CUDA(launch_pdl(kern, dim3(grid), dim3(GEMM_THREADS), smem, st, m0, m1, mb, p));
+  }
   prof_end(st);
   return HYMBA_OK;
+}
+
+// Pair tiles are 256 x 256: a CTA's stage holds its 16 KB A tile and 128 rows of B, six
+// stages.  (Measured on the Hymba layer shapes: 6 stages beat 7, and narrower pair tiles lose
+// to the single-CTA tiles of the same width.)
+template <int ET, int MODE>
+int launch_gemm_bn_pair(int bn, const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& mb,
+                        const GemmParams& p, cudaStream_t st, const char* name) {
+  if (bn == 256) return launch_gemm_inst<256, 6, ET, MODE, true>(m0, m1, mb, p, 0, st, name);
+  return fail(HYMBA_ERR_UNSUPPORTED, "no pair GEMM instance for tile width %d, type %d, epilogue %d", bn, ET, MODE);
 }
 
 // Tile widths instantiated per (epilogue, operand type); anything else is rejected.
@@ -276,6 +324,12 @@ int launch_gemm_bn(int bn, const CUtensorMap& m0, const CUtensorMap& m1, const C
 
 int launch_gemm_mode(const GemmCall& c, const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& mb,
                      const GemmParams& p, int grid, cudaStream_t st) {
+  if (c.pair) {
+    if (c.mode == EPI_PROJ && c.etype == ET_BF16) return launch_gemm_bn_pair<ET_BF16, EPI_PROJ>(c.bn, m0, m1, mb, p, st, c.name);
+    if (c.mode == EPI_BF16 && c.etype == ET_F16) return launch_gemm_bn_pair<ET_F16, EPI_BF16>(c.bn, m0, m1, mb, p, st, c.name);
+    if (c.mode == EPI_SWIGLU && c.etype == ET_BF16) return launch_gemm_bn_pair<ET_BF16, EPI_SWIGLU>(c.bn, m0, m1, mb, p, st, c.name);
+    return fail(HYMBA_ERR_UNSUPPORTED, "no pair GEMM for epilogue %d with operand type %d", c.mode, c.etype);
+  }
   switch (c.mode) {
     case EPI_PROJ:
       if (c.etype == ET_BF16) return launch_gemm_bn<ET_BF16, EPI_PROJ>(c.bn, m0, m1, mb, p, grid, st, c.name);
@@ -381,7 +435,7 @@ int run_gemm(GemmCall& c, const DeviceInfo& dev, cudaStream_t st) {
   {
     const uint64_t dims[2] = {(uint64_t)c.K, (uint64_t)c.N};
     const uint64_t str[1] = {(uint64_t)c.ldb * esz};
-    const uint32_t box[2] = {kbox, (uint32_t)c.bn};
+    const uint32_t box[2] = {kbox, (uint32_t)(c.pair ? c.bn / 2 : c.bn)};   // a pair CTA loads half the B tile
     HY_TRY(make_map(&mb, c.b, dt, 2, dims, str, box));
   }
   GemmParams& p = c.p;
@@ -396,7 +450,8 @@ int run_gemm(GemmCall& c, const DeviceInfo& dev, cudaStream_t st) {
   p.k_blocks = cdiv(c.K, kbox);
   p.split_k = c.split_k < 1 ? 1 : (c.split_k > p.k_blocks ? p.k_blocks : c.split_k);
   p.m_tiles = p.tiles0 + c.nb1 * p.tiles1;
-  p.total_tiles = p.m_tiles * p.n_tiles_n * p.split_k;
+  p.m_pairs = (p.m_tiles + 1) / 2;
+  p.total_tiles = (c.pair ? p.m_pairs : p.m_tiles) * p.n_tiles_n * p.split_k;
   if (p.total_tiles <= 0) return HYMBA_OK;
   const int grid = p.total_tiles < dev.sms ? p.total_tiles : dev.sms;
   return launch_gemm_mode(c, m0, m1, mb, p, grid, st);
@@ -425,6 +480,17 @@ int pick_bn_rounds(int m_tiles, int N, int sms, std::initializer_list<int> cands
     }
   }
   return best;
+}
+// Single-CTA tiles of width bn_single, or 256 x 256 pair tiles (cta_group::2)?  A round of
+// pair tiles (sms / 2 pairs) took 0.9 of the time of a round of 128 x 256 tiles on the
+// Hymba layer shapes (half the B tile per SM; the mainloop is bound by the operand feed from
+// L2, not by the MMAs); a round of narrower single tiles costs in proportion to its operand
+// bytes.  So pairs win at large M, and lose where they add a round (e.g. 17 row tiles x 34
+// column tiles: 4 single rounds, 5 pair rounds).
+bool pair_tiles_pay(int m_tiles, int N, int sms, int bn_single) {
+  const long long rounds_s = cdiv((long long)m_tiles * cdiv(N, bn_single), sms);
+  const long long rounds_p = cdiv((long long)cdiv(m_tiles, 2) * cdiv(N, 256), sms / 2);
+  return 0.9 * (double)rounds_p < (double)rounds_s * (GEMM_BM + bn_single) / (GEMM_BM + 256);
 }
 
 void fill_rope_theta(double* theta, float base) {
@@ -927,6 +993,8 @@ static int prefill_impl(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     {
       const int m_tiles = (c.a0 != nullptr ? cdiv(c.rows0, GEMM_BM) : 0) + c.nb1 * cdiv(c.rows1, GEMM_BM);
       c.bn = pick_bn_rounds(m_tiles, m.P, dev->sms, {256, 192});
+      c.pair = pair_tiles_pay(m_tiles, m.P, dev->sms, c.bn);
+      if (c.pair) c.bn = 256;
     }
     c.name = "in_proj";
     c.mode = EPI_PROJ;
@@ -1114,6 +1182,8 @@ static int prefill_impl(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     c.etype = ET_F16;
     c.name = "out_proj";
     c.bn = pick_bn_rounds(c.nb1 * cdiv(c.rows1, GEMM_BM), m.d, dev->sms, {256, 224, 128});
+    c.pair = pair_tiles_pay(c.nb1 * cdiv(c.rows1, GEMM_BM), m.d, dev->sms, c.bn);
+    if (c.pair) c.bn = 256;
     c.mode = EPI_BF16;
     c.p.out = out;
     c.p.ld_out = m.d;
@@ -1533,6 +1603,8 @@ int hymba_ffn_swiglu(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hym
     c.a1 = h; c.nb1 = 1; c.rows1 = rows; c.lda1 = d; c.a1_bstride = (long long)rows * d;
     c.b = w_gate_up; c.N = 2 * F; c.ldb = d; c.K = d;
     c.bn = pick_bn_rounds(cdiv(rows, GEMM_BM), 2 * F, dev->sms, {256, 192, 128});
+    c.pair = pair_tiles_pay(cdiv(rows, GEMM_BM), 2 * F, dev->sms, c.bn);
+    if (c.pair) c.bn = 256;
     c.name = "ffn_gate_up";
     c.mode = EPI_SWIGLU;
     c.p.out = act;
@@ -1548,6 +1620,8 @@ int hymba_ffn_swiglu(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hym
     c.etype = ET_F16;
     c.name = "ffn_down";
     c.bn = pick_bn_rounds(cdiv(rows, GEMM_BM), d, dev->sms, {256, 224, 128});
+    c.pair = pair_tiles_pay(cdiv(rows, GEMM_BM), d, dev->sms, c.bn);
+    if (c.pair) c.bn = 256;
     c.mode = EPI_BF16;
     c.p.out = out;
     c.p.ld_out = d;
