@@ -92,9 +92,15 @@ constexpr int GEMM_THREADS = 64 + 32 * GEMM_EPI_WARPS;
 constexpr int GEMM_BM = 128;
 
 // Shared memory an epilogue stages its output through: EPI_F32_ROWS transposes each warp's
-// 32 x 32 fp32 block (rows padded to 33 words) so that every store writes one whole row.
+// 32 x 32 fp32 block (rows padded to 33 words) so that every store writes one whole row;
+// EPI_BF16 exchanges each warp's 32 x 32 bf16 block (rows of 64 bytes padded to 80) so that
+// four lanes load or store one row's 64 bytes (two whole 32-byte sectors) instead of each lane
+// touching 16 bytes of its own row.
+constexpr int GEMM_BF16_TILE_WORDS = 20;   // words per staged row
 __host__ __device__ constexpr int gemm_epi_bytes(int mode) {
-  return mode == 3 /* EPI_F32_ROWS */ ? GEMM_EPI_WARPS * 32 * 33 * 4 : 0;
+  return mode == 3 /* EPI_F32_ROWS */ ? GEMM_EPI_WARPS * 32 * 33 * 4
+         : mode == 1 /* EPI_BF16 */   ? GEMM_EPI_WARPS * 32 * GEMM_BF16_TILE_WORDS * 4
+                                      : 0;
 }
 
 template <int BN, int STAGES, int EPI_BYTES = 0, bool PAIR = false>
@@ -466,6 +472,55 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
               if (rr0 + q < rows_valid && col_ok) dst[(size_t)q * p.ld_out] = tile[q * 33 + lane];
             __syncwarp();
             return;
+          }
+          if constexpr (MODE == EPI_BF16) {
+            // whole 32-column chunks: the residual comes in and the result goes out through
+            // this warp's staging block, rows read and written by four lanes each (all lanes
+            // take part; rows past the tile's valid rows are neither read nor written)
+            if (gc >= p.n_valid) return;          // the same for the whole warp
+            if (gc + 32 <= p.n_valid) {
+              uint32_t* tile = reinterpret_cast<uint32_t*>(smem + L::EPI_OFFSET) + (warp - 2) * (32 * GEMM_BF16_TILE_WORDS);
+              const int rows_valid = src0 ? p.rows0 : p.rows1;
+              const int rr0 = rr - lane;            // accumulator row of lane 0
+              const size_t orow0 = (size_t)b1 * p.rows1 + rr0;
+              const int pr = lane >> 2, pc = lane & 3;   // row in a group of 8, 16-byte piece
+              const bool tile_ok = m < p.m_tiles;
+              if (p.residual != nullptr) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const int j = pr + 8 * i;
+                  if (tile_ok && rr0 + j < rows_valid)
+                    *reinterpret_cast<uint4*>(tile + j * GEMM_BF16_TILE_WORDS + pc * 4) =
+                        *reinterpret_cast<const uint4*>(p.residual + (orow0 + j) * p.ld_res + gc + pc * 8);
+                }
+                __syncwarp();
+#pragma unroll
+                for (int e = 0; e < 32; e += 8) {
+                  const uint4 raw = *reinterpret_cast<const uint4*>(tile + lane * GEMM_BF16_TILE_WORDS + e / 2);
+                  const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+                  for (int k = 0; k < 8; ++k) v[e + k] += __bfloat162float(hv[k]);
+                }
+                __syncwarp();
+              }
+#pragma unroll
+              for (int e = 0; e < 32; e += 8)
+                *reinterpret_cast<uint4*>(tile + lane * GEMM_BF16_TILE_WORDS + e / 2) =
+                    make_uint4(pack_bf16x2(v[e], v[e + 1]), pack_bf16x2(v[e + 2], v[e + 3]),
+                               pack_bf16x2(v[e + 4], v[e + 5]), pack_bf16x2(v[e + 6], v[e + 7]));
+              __syncwarp();
+              __nv_bfloat16* outb = reinterpret_cast<__nv_bfloat16*>(p.out);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int j = pr + 8 * i;
+                if (tile_ok && rr0 + j < rows_valid) {
+                  const uint4 w = *reinterpret_cast<const uint4*>(tile + j * GEMM_BF16_TILE_WORDS + pc * 4);
+                  st_global_v4(outb + (orow0 + j) * p.ld_out + gc + pc * 8, w.x, w.y, w.z, w.w);
+                }
+              }
+              __syncwarp();
+              return;
+            }
           }
           if (!row_ok || gc >= p.n_valid) return;
           const bool whole = gc + 32 <= p.n_valid;

@@ -313,7 +313,7 @@ int launch_gemm_bn(int bn, const CUtensorMap& m0, const CUtensorMap& m1, const C
     if (bn == 192) return launch_gemm_inst<192, 5, ET, MODE>(m0, m1, mb, p, grid, st, name);
   }
   if constexpr (MODE == EPI_BF16) {
-    if (bn == 224) return launch_gemm_inst<224, 5, ET, MODE>(m0, m1, mb, p, grid, st, name);
+    if (bn == 224) return launch_gemm_inst<224, 4, ET, MODE>(m0, m1, mb, p, grid, st, name);
   }
   if constexpr (any_bn && ET != ET_TF32) {
     if (bn == 160) return launch_gemm_inst<160, 5, ET, MODE>(m0, m1, mb, p, grid, st, name);
