@@ -910,11 +910,12 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) inputs, N(0,0.02) weights, dt logits N(-4,1))",
             "config": cfg,
-            "e2e": {"value": round(e2e, 1), "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"],
-                    "d2h_bytes_per_step": r["d2h"],
-                    "how": "hymba_mixer_prefill_host per step (pinned host X -> device, prefill, device -> "
-                           "pinned host out, one C-ABI call); two streams alternate steps so copies overlap compute; "
-                           "CUDA events"},
+            "e2e": None if args.no_e2e else {
+                "value": round(e2e, 1), "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"],
+                "d2h_bytes_per_step": r["d2h"],
+                "how": "hymba_mixer_prefill_host per step (pinned host X -> device, prefill, device -> "
+                       "pinned host out, one C-ABI call); two streams alternate steps so copies overlap compute; "
+                       "CUDA events"},
             "input_tokens_per_s": round(tokens_per_s * cfg["n_tokens"] / cfg["seq_len"], 1),   # B*N / time
             "gpu_launches": int(round(r["launches_per_step"] * args.steps)),
             "step_roofline": r["step_roofline"], "roofline": r["roofline"], "scan_roofline": r["scan_roofline"],

@@ -60,6 +60,11 @@ struct GemmParams {
   // a source-1 row (b, r) goes to b*T_out + row_off1 + r (position row_off1 + r)
   int out_batches, T_out, row_off1;
   int m_pairs;              // PAIR: cdiv(m_tiles, 2); total_tiles counts pair tiles
+  // 1: the column tiles of one row tile (or pair) are consecutive in the tile order, so the
+  // CTAs at work at any moment share a few A row tiles and sweep the whole B operand (the
+  // weights, 15-35 MB, which stay in L2); for an A operand too large to stay in L2 next to
+  // them.  0: row tiles inner (each B column tile is shared by the CTAs at work).
+  int n_inner;
   // 1: only the epilogue warps wait for the previous kernel on the stream.  For a GEMM whose
   // operands no kernel of the same call writes (the caller's input and the weights), so the
   // mainloop overlaps a previous kernel that only prepares what the epilogue reads.
@@ -183,8 +188,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
   const int tile0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int tile_step = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
-  const int m_count = PAIR ? p.m_pairs : p.m_tiles;
-  auto tile_m = [&](int t2) { return PAIR ? 2 * (t2 % m_count) + (int)rank : t2 % m_count; };
+  const int m_count = PAIR ? p.m_pairs : p.m_tiles;   // row tiles, or pairs of them
+  // Tile order (GemmParams::n_inner): row tiles (or pairs) inner, or column tiles inner.
+  auto tile_m = [&](int t2) {
+    const int mi = p.n_inner ? t2 / p.n_tiles_n : t2 % m_count;
+    return PAIR ? 2 * mi + (int)rank : mi;
+  };
+  auto tile_n = [&](int t2) { return p.n_inner ? t2 % p.n_tiles_n : t2 / m_count; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -248,7 +258,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if ((int)blockIdx.x < p.total_tiles) {
           const int tile = blockIdx.x;
           const int ks = tile % p.split_k;
-          const int m = (tile / p.split_k) % p.m_tiles;
+          const int m = tile_m(tile / p.split_k);
           const int kb0 = (int)((long long)ks * p.k_blocks / p.split_k);
           const int kb1 = (int)((long long)(ks + 1) * p.k_blocks / p.split_k);
           pre = (uint32_t)min(kb1 - kb0, STAGES);
@@ -266,7 +276,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         const int ks = tile % p.split_k;
         const int t2 = tile / p.split_k;
         const int m = tile_m(t2);
-        const int n = t2 / m_count;
+        const int n = tile_n(t2);
         const int kb0 = (int)((long long)ks * p.k_blocks / p.split_k);
         const int kb1 = (int)((long long)(ks + 1) * p.k_blocks / p.split_k);
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
@@ -366,7 +376,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const int ks = tile % p.split_k;
       const int t2 = tile / p.split_k;
       const int m = tile_m(t2);
-      const int n = t2 / m_count;
+      const int n = tile_n(t2);
       const int ab = lt & 1;
       const uint32_t aph = (lt >> 1) & 1u;
       int ok = 1;
