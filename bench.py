@@ -760,17 +760,17 @@ def run_stack_decode(args, st, E, world):
 # workload (profiles/ holds the summaries and commands); a kernel changed since its capture
 # has no entry.  ncu replays a kernel with cold caches: writes that stay in L2 do not show.
 TRAFFIC = {
-    "in_proj": 35320064 + 787968,
+    "in_proj": 35381760 + 1385216,
     "conv1d_silu": 13999616 + 0,
-    "x_proj": 14799360 + 768,
-    "dt_proj": 2442496 + 0,
+    "x_proj": 14809344 + 768,
+    "dt_proj": 2453504 + 0,
     "attention": 9817344 + 0,
     "scan_chunk_end": 42369280 + 16128,
     "scan_carry": 6089472 + 0,
     "selective_scan": 48214272 + 553472,
     "norm_avg": 41828864 + 295680,
-    "out_proj": 36293632 + 17664,
-    "decode_ssm": 16947200 + 0,
+    "out_proj": 36304640 + 74496,
+    "decode_ssm": 16950784 + 0,
 }
 
 
