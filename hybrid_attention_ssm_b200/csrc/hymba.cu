@@ -304,22 +304,23 @@ int launch_gemm_bn(int bn, const CUtensorMap& m0, const CUtensorMap& m1, const C
   if constexpr (MODE == EPI_F32_ROWS) {   // short K (dt_rank): 4 stages, room for the staging tiles
     if (bn == 128) return launch_gemm_inst<128, 4, ET, MODE>(m0, m1, mb, p, grid, st, name);
     return fail(HYMBA_ERR_UNSUPPORTED, "no GEMM instance for tile width %d with the row-store epilogue", bn);
+  } else {
+    if (bn == 256) return launch_gemm_inst<256, 4, ET, MODE>(m0, m1, mb, p, grid, st, name);
+    if constexpr (MODE != EPI_PROJ) {
+      if (bn == 128) return launch_gemm_inst<128, 6, ET, MODE>(m0, m1, mb, p, grid, st, name);
+    }
+    if constexpr ((MODE == EPI_PROJ || MODE == EPI_SWIGLU) && ET == ET_BF16) {
+      if (bn == 192) return launch_gemm_inst<192, 5, ET, MODE>(m0, m1, mb, p, grid, st, name);
+    }
+    if constexpr (MODE == EPI_BF16) {
+      if (bn == 224) return launch_gemm_inst<224, 4, ET, MODE>(m0, m1, mb, p, grid, st, name);
+    }
+    if constexpr (any_bn && ET != ET_TF32) {
+      if (bn == 160) return launch_gemm_inst<160, 5, ET, MODE>(m0, m1, mb, p, grid, st, name);
+      if (bn == 64) return launch_gemm_inst<64, 8, ET, MODE>(m0, m1, mb, p, grid, st, name);
+    }
+    return fail(HYMBA_ERR_UNSUPPORTED, "no GEMM instance for tile width %d, type %d, epilogue %d", bn, ET, MODE);
   }
-  if (bn == 256) return launch_gemm_inst<256, 4, ET, MODE>(m0, m1, mb, p, grid, st, name);
-  if constexpr (MODE != EPI_PROJ) {
-    if (bn == 128) return launch_gemm_inst<128, 6, ET, MODE>(m0, m1, mb, p, grid, st, name);
-  }
-  if constexpr ((MODE == EPI_PROJ || MODE == EPI_SWIGLU) && ET == ET_BF16) {
-    if (bn == 192) return launch_gemm_inst<192, 5, ET, MODE>(m0, m1, mb, p, grid, st, name);
-  }
-  if constexpr (MODE == EPI_BF16) {
-    if (bn == 224) return launch_gemm_inst<224, 4, ET, MODE>(m0, m1, mb, p, grid, st, name);
-  }
-  if constexpr (any_bn && ET != ET_TF32) {
-    if (bn == 160) return launch_gemm_inst<160, 5, ET, MODE>(m0, m1, mb, p, grid, st, name);
-    if (bn == 64) return launch_gemm_inst<64, 8, ET, MODE>(m0, m1, mb, p, grid, st, name);
-  }
-  return fail(HYMBA_ERR_UNSUPPORTED, "no GEMM instance for tile width %d, type %d, epilogue %d", bn, ET, MODE);
 }
 
 int launch_gemm_mode(const GemmCall& c, const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& mb,
