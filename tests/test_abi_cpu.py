@@ -102,3 +102,31 @@ def test_kv_share_odd_patterns():
         ocid, orole = orc.kv_share_plan(pattern)
         assert (cid, role) == (ocid, orole), pattern
         assert need > 0
+
+
+def test_l2_prefetch_arguments_are_checked_on_the_host():
+    """hymba_l2_prefetch refuses 0 or more than 8 ranges and null or misaligned pointers
+    before it launches anything."""
+    L = H.lib()
+    ptrs = (ctypes.c_void_p * 9)(*([256] * 9))
+    sizes = (ctypes.c_size_t * 9)(*([4096] * 9))
+    for n in (0, 9):
+        assert L.hymba_l2_prefetch(ptrs, sizes, n, None) == H.ERR_INVALID_ARG
+    bad = (ctypes.c_void_p * 1)(None)
+    assert L.hymba_l2_prefetch(bad, sizes, 1, None) == H.ERR_INVALID_ARG
+    odd = (ctypes.c_void_p * 1)(264)
+    assert L.hymba_l2_prefetch(odd, sizes, 1, None) == H.ERR_INVALID_ARG
+
+
+def test_ffn_decode_workspace_sizes():
+    """The decode FFN's workspace holds its split-K slices and activations: it grows with the
+    rows, and shapes outside the kernels' limits are refused."""
+    a = H.ffn_workspace_size(1, 1600, 5504)
+    b = H.ffn_workspace_size(8, 1600, 5504)
+    c = H.ffn_workspace_size(64, 1600, 5504)
+    assert 0 < a < b < c
+    assert c >= 64 * 5504 * 2 + 64 * 1600 * 4   # fp16 activations and at least one fp32 slice
+    for rows, d, F in ((0, 1600, 5504), (257, 1600, 5504), (8, 1602, 5504), (8, 1600, 5500)):
+        with pytest.raises(H.HymbaError) as e:
+            H.ffn_workspace_size(rows, d, F)
+        assert e.value.code == H.ERR_INVALID_ARG

@@ -469,6 +469,22 @@ def test_ffn_swiglu_decode(rows):
     assert_rms(to_np(out), to_np(out2), name=f"decode FFN vs prefill FFN ({rows} rows)")
 
 
+def test_l2_prefetch_hint_runs_and_writes_nothing():
+    """hymba_l2_prefetch enqueues its bulk L2 prefetches for up to 8 ranges (odd sizes
+    included) on a stream and leaves every byte as it was."""
+    g = torch.Generator(device="cuda")
+    g.manual_seed(3)
+    ts = [torch.randn(n, generator=g, device="cuda") for n in (1, 1000, 8192 + 3, 1 << 20, 5 << 20)]
+    before = [t.clone() for t in ts]
+    s = torch.cuda.Stream()
+    H.l2_prefetch(ts, stream=s)
+    H.l2_prefetch(ts[:1])
+    s.synchronize()
+    torch.cuda.synchronize()
+    for a, b in zip(ts, before):
+        assert torch.equal(a, b)
+
+
 # ---------------------------------------------------------------------------------------
 # decode with a position per sequence
 # ---------------------------------------------------------------------------------------
