@@ -481,7 +481,7 @@ __global__ void __launch_bounds__(DA_THREADS, 3)
       // after a wait has given up, the warps keep walking the items (so that every one of
       // them reaches the same merge barriers) without waiting or releasing stages
       if (ok) ok = mbar_wait(&full[stg], (uint32_t)(ct / DA_STAGES) & 1u, &abort_flag, p.status, 501);
-      ok = __all_sync(0xffffffffu, ok);   // one verdict per warp: the shuffles below need all lanes
+      ok = __all_sync(0xffffffffu, ok);   // one decision per warp: the shuffles below need all lanes
       if (!ok) continue;
       if (t == 0) {   // the item's queries arrived with its first tile
         const float* q = &qbuf[stg][gq * 64];
