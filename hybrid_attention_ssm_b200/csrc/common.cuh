@@ -228,9 +228,10 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 // ----------------------------------------------------------------------------------------
 // CTA pairs (a cluster of two CTAs on two SMs, cta_group::2): one MMA of M = 256 reads the
 // A rows and the halves of B that each CTA holds at the same shared-memory offset, and writes
-// each CTA's 128 accumulator rows into that CTA's TMEM.  No load here is multicast: each CTA
-// fetches its own operands; only the completion of a load, an MMA commit or an arrival is
-// signalled on the other CTA's barrier, through its shared::cluster address.
+// each CTA's 128 accumulator rows into that CTA's TMEM.  Every load fills only the issuing
+// CTA's shared memory with that CTA's own operands; only the completion of a load, an MMA
+// commit or an arrival is signalled on the other CTA's barrier, through its shared::cluster
+// address.
 // ----------------------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;

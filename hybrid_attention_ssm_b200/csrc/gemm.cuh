@@ -15,8 +15,8 @@
 // PAIR: the CTAs run as clusters of two on two SMs, and one tcgen05.mma.cta_group::2 of
 // M = 256 covers both CTAs' 128-row A tiles against a BN-wide B tile of which each CTA holds
 // one half: per k-block an SM then moves 16 KB of A and BN/2 x 128 B of B into shared memory
-// instead of 16 KB + BN x 128 B, for the same MMA work.  Each CTA loads its own tiles (no
-// multicast loads); the loads of both complete on the even CTA's barrier, whose single MMA
+// instead of 16 KB + BN x 128 B, for the same MMA work.  Each CTA loads its own tiles into
+// its own shared memory; the loads of both complete on the even CTA's barrier, whose single MMA
 // thread issues the pair's MMAs and commits them to both CTAs' barriers.  Each CTA's
 // epilogue reads its own TMEM rows, as in the single-CTA form.
 #pragma once
