@@ -66,6 +66,8 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 }
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+// threads of splitk_sum_rmsnorm_kernel for rows of d: one 16-byte piece each, whole warps
+inline int snorm_threads(int d) { return ((d / 4 + 31) / 32) * 32; }
 inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -1296,10 +1298,12 @@ int hymba_mixer_prefill_host(const hymba_layer_cfg* cfg, const hymba_layer_weigh
 
 // The decode step; positions == NULL: every sequence at `position`; otherwise sequence b at
 // positions[b] (device memory), each <= `position`, which sizes the attention's key splits.
+// norm_out != NULL: the final split-K sum also writes norm_out = RMSNorm(out) * norm_gain.
 static int decode_impl(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x, int B,
                        int position, const int* positions, hymba_kv_cache* kv, float* ssm_state,
                        float* conv_state, const hymba_bf16* residual, hymba_bf16* out, void* ws, size_t ws_bytes,
-                       hymba_stream stream) {
+                       hymba_stream stream, const float* norm_gain = nullptr, float norm_eps = 0.f,
+                       hymba_bf16* norm_out = nullptr) {
   HY_TRY(check_cfg(cfg));
   DeviceInfo* dev = nullptr;
   HY_TRY(device_info(&dev));
@@ -1536,8 +1540,15 @@ static int decode_impl(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     HY_TRY(run_gemm(c, *dev, st));
     const int n = B * m.d;
     prof_begin("decode_out_store", st);
-    HY_CUDA(launch_pdl(splitk_reduce_kernel, dim3(cdiv(n / 4, 256)), dim3(256), 0, st, f32(L.acc_part), L.oproj_split, (long long)n, n,
-                                                            reinterpret_cast<const __nv_bfloat16*>(residual), out, 1));
+    if (norm_out != nullptr) {
+      HY_CUDA(launch_pdl(splitk_sum_rmsnorm_kernel, dim3(B), dim3(snorm_threads(m.d)), 0, st, (const float*)f32(L.acc_part),
+                         L.oproj_split, (long long)n, m.d, reinterpret_cast<const __nv_bfloat16*>(residual),
+                         reinterpret_cast<__nv_bfloat16*>(out), norm_gain, norm_eps,
+                         reinterpret_cast<__nv_bfloat16*>(norm_out)));
+    } else {
+      HY_CUDA(launch_pdl(splitk_reduce_kernel, dim3(cdiv(n / 4, 256)), dim3(256), 0, st, f32(L.acc_part), L.oproj_split, (long long)n, n,
+                                                              reinterpret_cast<const __nv_bfloat16*>(residual), out, 1));
+    }
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
@@ -1550,6 +1561,19 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
                        hymba_stream stream) {
   return decode_impl(cfg, w, x, B, position, nullptr, kv, ssm_state, conv_state, residual, out, ws, ws_bytes,
                      stream);
+}
+
+int hymba_mixer_decode_norm(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x, int B,
+                            int position, hymba_kv_cache* kv, float* ssm_state, float* conv_state,
+                            const hymba_bf16* residual, hymba_bf16* out, const float* norm_gain, float norm_eps,
+                            hymba_bf16* norm_out, void* ws, size_t ws_bytes, hymba_stream stream) {
+  if (norm_gain == nullptr || norm_out == nullptr || !aligned16(norm_gain) || !aligned16(norm_out) || norm_out == out ||
+      norm_out == x)
+    return fail(HYMBA_ERR_INVALID_ARG, "norm gain / output NULL, misaligned, or aliasing out or x");
+  if (cfg != nullptr && cfg->d_model > SNORM_MAX_D)
+    return fail(HYMBA_ERR_UNSUPPORTED, "d_model %d above %d for the fused norm", cfg->d_model, SNORM_MAX_D);
+  return decode_impl(cfg, w, x, B, position, nullptr, kv, ssm_state, conv_state, residual, out, ws, ws_bytes, stream,
+                     norm_gain, norm_eps, norm_out);
 }
 
 int hymba_mixer_decode_ragged(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const hymba_bf16* x, int B,
@@ -1692,9 +1716,11 @@ int hymba_l2_prefetch(const void* const* ranges, const size_t* bytes, int n_rang
   return HYMBA_OK;
 }
 
-int hymba_ffn_swiglu_decode(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hymba_f16* w_down, int rows,
-                            int d, int F, const hymba_bf16* residual, hymba_bf16* out, void* ws, size_t ws_bytes,
-                            hymba_stream stream) {
+namespace {
+// norm_out != NULL: the final split-K sum also writes norm_out = RMSNorm(out) * norm_gain.
+int ffn_decode_impl(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hymba_f16* w_down, int rows, int d, int F,
+                    const hymba_bf16* residual, hymba_bf16* out, const float* norm_gain, float norm_eps,
+                    hymba_bf16* norm_out, void* ws, size_t ws_bytes, hymba_stream stream) {
   DeviceInfo* dev = nullptr;
   HY_TRY(device_info(&dev));
   size_t need = 0;
@@ -1754,11 +1780,36 @@ int hymba_ffn_swiglu_decode(const hymba_bf16* h, const hymba_bf16* w_gate_up, co
     HY_TRY(run_gemm(c, *dev, st));
     const int n = rows * d;
     prof_begin("ffn_dec_out", st);
-    HY_CUDA(launch_pdl(splitk_reduce_kernel, dim3(cdiv(n / 4, 256)), dim3(256), 0, st, (const float*)part2, L.s2,
-                       (long long)n, n, reinterpret_cast<const __nv_bfloat16*>(residual), out, 1));
+    if (norm_out != nullptr) {
+      HY_CUDA(launch_pdl(splitk_sum_rmsnorm_kernel, dim3(rows), dim3(snorm_threads(d)), 0, st, (const float*)part2, L.s2,
+                         (long long)n, d, reinterpret_cast<const __nv_bfloat16*>(residual),
+                         reinterpret_cast<__nv_bfloat16*>(out), norm_gain, norm_eps,
+                         reinterpret_cast<__nv_bfloat16*>(norm_out)));
+    } else {
+      HY_CUDA(launch_pdl(splitk_reduce_kernel, dim3(cdiv(n / 4, 256)), dim3(256), 0, st, (const float*)part2, L.s2,
+                         (long long)n, n, reinterpret_cast<const __nv_bfloat16*>(residual), out, 1));
+    }
     prof_end(st);
   }
   return HYMBA_OK;
+}
+}  // namespace
+
+int hymba_ffn_swiglu_decode(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hymba_f16* w_down, int rows,
+                            int d, int F, const hymba_bf16* residual, hymba_bf16* out, void* ws, size_t ws_bytes,
+                            hymba_stream stream) {
+  return ffn_decode_impl(h, w_gate_up, w_down, rows, d, F, residual, out, nullptr, 0.f, nullptr, ws, ws_bytes, stream);
+}
+
+int hymba_ffn_swiglu_decode_norm(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hymba_f16* w_down, int rows,
+                                 int d, int F, const hymba_bf16* residual, hymba_bf16* out, const float* norm_gain,
+                                 float norm_eps, hymba_bf16* norm_out, void* ws, size_t ws_bytes, hymba_stream stream) {
+  if (norm_gain == nullptr || norm_out == nullptr || !aligned16(norm_gain) || !aligned16(norm_out) || norm_out == out ||
+      norm_out == h)
+    return fail(HYMBA_ERR_INVALID_ARG, "norm gain / output NULL, misaligned, or aliasing out or h");
+  if (d > SNORM_MAX_D) return fail(HYMBA_ERR_UNSUPPORTED, "d %d above %d for the fused norm", d, SNORM_MAX_D);
+  return ffn_decode_impl(h, w_gate_up, w_down, rows, d, F, residual, out, norm_gain, norm_eps, norm_out, ws, ws_bytes,
+                         stream);
 }
 
 int hymba_prepend_meta(const hymba_bf16* meta, const hymba_bf16* x, int batch, int n_meta, int n_tokens, int d,

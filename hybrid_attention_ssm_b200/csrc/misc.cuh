@@ -828,6 +828,61 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// The split-K sum of a decode projection with its residual, followed in the same pass by the
+// RMSNorm of the result (the input norm of the block's next sublayer), one CTA per row and one
+// 16-byte piece of the row per thread (blockDim.x * 4 >= d), the slices' loads 16 at a time:
+//   out_sum[r, :]  = bf16(residual[r, :] + the slices in slice order), exactly as
+//                    splitk_reduce_kernel stores it;
+//   out_norm[r, :] = bf16(s / sqrt(mean(s^2) + eps) * gain) with s = out_sum[r, :] as stored,
+//                    as rmsnorm_kernel computes it from the stored row.
+// d % 4 == 0, d <= 4096.
+constexpr int SNORM_MAX_D = 4096;
+__global__ void __launch_bounds__(1024)
+    splitk_sum_rmsnorm_kernel(const float* __restrict__ part, int n_split, long long stride, int d,
+                              const __nv_bfloat16* __restrict__ residual, __nv_bfloat16* __restrict__ out_sum,
+                              const float* __restrict__ gain, float eps, __nv_bfloat16* __restrict__ out_norm) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float red[32];
+  const int c = threadIdx.x * 4;
+  const size_t i = (size_t)blockIdx.x * d + c;
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (c < d) {
+    __nv_bfloat162 r0, r1;
+    if (residual != nullptr) {
+      r0 = *reinterpret_cast<const __nv_bfloat162*>(residual + i);
+      r1 = *reinterpret_cast<const __nv_bfloat162*>(residual + i + 2);
+    }
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < n_split; s0 += 16) {
+      float4 q[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        q[j] = s0 + j < n_split ? *reinterpret_cast<const float4*>(part + (size_t)(s0 + j) * stride + i)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        acc.x += q[j].x; acc.y += q[j].y; acc.z += q[j].z; acc.w += q[j].w;
+      }
+    }
+    if (residual != nullptr) {
+      acc.x += __low2float(r0); acc.y += __high2float(r0); acc.z += __low2float(r1); acc.w += __high2float(r1);
+    }
+    const uint32_t p0 = pack_bf16x2(acc.x, acc.y), p1 = pack_bf16x2(acc.z, acc.w);
+    *reinterpret_cast<uint2*>(out_sum + i) = make_uint2(p0, p1);
+    const __nv_bfloat162 b0 = *reinterpret_cast<const __nv_bfloat162*>(&p0);
+    const __nv_bfloat162 b1 = *reinterpret_cast<const __nv_bfloat162*>(&p1);
+    v = make_float4(__low2float(b0), __high2float(b0), __low2float(b1), __high2float(b1));
+  }
+  const float ss = block_sum_256(v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w, red);
+  const float r = 1.f / sqrtf(ss / (float)d + eps);
+  if (c < d) {
+    const float4 g = *reinterpret_cast<const float4*>(gain + c);
+    *reinterpret_cast<uint2*>(out_norm + i) =
+        make_uint2(pack_bf16x2(v.x * r * g.x, v.y * r * g.y), pack_bf16x2(v.z * r * g.z, v.w * r * g.w));
+  }
+}
+
 // out[b] = [meta; x[b]] : meta [M, d], x [B, N, d] -> out [B, M+N, d] (16-byte pieces)
 __global__ void prepend_meta_kernel(const __nv_bfloat16* __restrict__ meta, const __nv_bfloat16* __restrict__ x,
                                     int B, int M, int N, int d, __nv_bfloat16* __restrict__ out) {

@@ -111,6 +111,11 @@ def lib():
             "hymba_mixer_prefill_prefix": ([ctypes.POINTER(LayerCfg), ctypes.POINTER(LayerWeights), _vp, _c_int,
                                             _c_int, ctypes.POINTER(MetaPrefix), ctypes.POINTER(KVCache), _vp, _vp,
                                             _vp, _vp, _vp, _c_size, _vp], _c_int),
+            "hymba_mixer_decode_norm": ([ctypes.POINTER(LayerCfg), ctypes.POINTER(LayerWeights), _vp, _c_int,
+                                         _c_int, ctypes.POINTER(KVCache), _vp, _vp, _vp, _vp, _vp, ctypes.c_float,
+                                         _vp, _vp, _c_size, _vp], _c_int),
+            "hymba_ffn_swiglu_decode_norm": ([_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, ctypes.c_float,
+                                              _vp, _vp, _c_size, _vp], _c_int),
             "hymba_mixer_decode_ragged": ([ctypes.POINTER(LayerCfg), ctypes.POINTER(LayerWeights), _vp, _c_int,
                                            _vp, _c_int, ctypes.POINTER(KVCache), _vp, _vp, _vp, _vp, _vp, _c_size,
                                            _vp], _c_int),
@@ -343,6 +348,16 @@ def mixer_decode(dims, dw: DeviceWeights, x, position, kv: Cache, ssm_state, con
                                    ptr(ws), ws.numel(), stream_handle(stream)))
 
 
+def mixer_decode_norm(dims, dw: DeviceWeights, x, position, kv: Cache, ssm_state, conv_state, out, norm_gain,
+                      norm_eps, norm_out, ws, residual=None, stream=None, cfg=None):
+    """hymba_mixer_decode_norm: the decode step, and norm_out = RMSNorm(out) * norm_gain."""
+    cfg = make_cfg(dims) if cfg is None else cfg
+    check(lib().hymba_mixer_decode_norm(ctypes.byref(cfg), ctypes.byref(dw.c), ptr(x), x.shape[0], position,
+                                        ctypes.byref(kv.c), ptr(ssm_state), ptr(conv_state), ptr(residual), ptr(out),
+                                        ptr(norm_gain), norm_eps, ptr(norm_out), ptr(ws), ws.numel(),
+                                        stream_handle(stream)))
+
+
 def mixer_decode_ragged(dims, dw: DeviceWeights, x, positions, max_position, kv: Cache, ssm_state, conv_state, out,
                         ws, residual=None, stream=None, cfg=None):
     """hymba_mixer_decode with a position per sequence: positions is an int32 device tensor [B]."""
@@ -416,6 +431,16 @@ def l2_prefetch(tensors, stream=None):
     ptrs = (_vp * n)(*[t.data_ptr() for t in tensors])
     sizes = (_c_size * n)(*[t.numel() * t.element_size() for t in tensors])
     check(lib().hymba_l2_prefetch(ptrs, sizes, n, stream_handle(stream)))
+
+
+def ffn_swiglu_decode_norm(h, w_gate_up, w_down, out, norm_gain, norm_eps, norm_out, ws, residual=None,
+                           stream=None):
+    """hymba_ffn_swiglu_decode_norm: the decode FFN, and norm_out = RMSNorm(out) * norm_gain."""
+    rows, d = h.shape
+    F = w_down.shape[1]
+    check(lib().hymba_ffn_swiglu_decode_norm(ptr(h), ptr(w_gate_up), ptr(w_down), rows, d, F, ptr(residual), ptr(out),
+                                             ptr(norm_gain), norm_eps, ptr(norm_out), ptr(ws), ws.numel(),
+                                             stream_handle(stream)))
 
 
 def profile_begin(max_records=8192):

@@ -110,6 +110,7 @@ class HymbaStack:
             self.dh = [torch.empty(self.B, dims.d_model, **bf) for _ in range(2)]
             self.dh1 = torch.empty(self.B, dims.d_model, **bf)
             self.dhn = torch.empty(self.B, dims.d_model, **bf)
+            self.dhn2 = torch.empty(self.B, dims.d_model, **bf)
             self.fws = H.alloc_workspace(H.ffn_workspace_size(self.B, dims.d_model, self.F))
 
     def cache_view(self, ptr_value, max_tokens, dl):
@@ -179,23 +180,29 @@ class HymbaStack:
         stream after its mixer and after its FFN."""
         assert self.ssm is not None, "build the stack with decode_room > 0"
         assert self.wl.dims.n_meta < position < self.max_tokens
-        d = self.wl.dims.d_model
         cur = 0
         self.dh[cur].copy_(x)
+        # only the first layer's input norm runs on its own: each later norm is fused into the
+        # last kernel of the sublayer before it (hymba_*_decode_norm)
+        L = len(self.layers)
+        H.rmsnorm(self.dh[cur], self.layers[0][2]["g1"], self.layers[0][0].norm_eps, self.dhn)
         for l, (dl, dw, dev) in enumerate(self.layers):
             hin, hout = self.dh[cur], self.dh[1 - cur]
             kv = self.caches[self.cache_id[l]]
-            H.rmsnorm(hin, dev["g1"], dl.norm_eps, self.dhn)
             if record is not None and l in record:
                 cache = {k: v.float().cpu().numpy() for k, v in self.layer_cache_tensors(l).items()}
                 record[l].update(h_in=hin.float().cpu().numpy(), hn=self.dhn.float().cpu().numpy(), cache=cache,
                                  ssm=self.ssm[l].cpu().numpy(), conv=self.conv[l].cpu().numpy())
-            H.mixer_decode(dl, dw, self.dhn, position, kv, self.ssm[l], self.conv[l], self.dh1, self.dws,
-                           residual=hin)
-            H.rmsnorm(self.dh1, dev["g2"], dl.norm_eps, self.dhn)
-            H.ffn_swiglu_decode(self.dhn, dev["w_gu"], dev["w_down"], hout, self.fws, residual=self.dh1)
+            H.mixer_decode_norm(dl, dw, self.dhn, position, kv, self.ssm[l], self.conv[l], self.dh1, dev["g2"],
+                                dl.norm_eps, self.dhn2, self.dws, residual=hin)
+            if l + 1 < L:
+                ndl, _, ndev = self.layers[l + 1]
+                H.ffn_swiglu_decode_norm(self.dhn2, dev["w_gu"], dev["w_down"], hout, ndev["g1"], ndl.norm_eps,
+                                         self.dhn, self.fws, residual=self.dh1)
+            else:
+                H.ffn_swiglu_decode(self.dhn2, dev["w_gu"], dev["w_down"], hout, self.fws, residual=self.dh1)
             if record is not None and l in record:
-                record[l].update(h_mid=self.dh1.float().cpu().numpy(), hn2=self.dhn.float().cpu().numpy(),
+                record[l].update(h_mid=self.dh1.float().cpu().numpy(), hn2=self.dhn2.float().cpu().numpy(),
                                  h_out=hout.float().cpu().numpy())
             cur = 1 - cur
         return self.dh[cur]

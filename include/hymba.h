@@ -353,6 +353,24 @@ int hymba_ffn_swiglu_decode(const hymba_bf16* h, const hymba_bf16* w_gate_up, co
                             int d, int F, const hymba_bf16* residual, hymba_bf16* out, void* workspace,
                             size_t ws_bytes, hymba_stream stream);
 
+/* The decode steps of a block's two sublayers with the next sublayer's input norm fused into
+ * their last kernel ([JJ] §Hymba 的整体架构: x + mixer(norm(x)), then + FFN(norm(.))): as
+ * hymba_mixer_decode and hymba_ffn_swiglu_decode, and in the same final pass over each row
+ *   norm_out[r, :] = out[r, :] / sqrt(mean(out[r, :]^2) + norm_eps) * norm_gain
+ * (out as stored, bf16; norm_gain [d] fp32, 16-byte aligned; norm_out [rows, d] bf16, not
+ * aliasing out or the input), which is what hymba_rmsnorm computes from out.  out itself is
+ * bit for bit what the plain call writes.  d_model <= 4096.
+ * Errors: as the plain calls; HYMBA_ERR_INVALID_ARG for a NULL, misaligned or aliasing norm
+ * argument, HYMBA_ERR_UNSUPPORTED for d_model above 4096. */
+int hymba_mixer_decode_norm(const hymba_layer_cfg* cfg, const hymba_layer_weights* weights, const hymba_bf16* x,
+                            int batch, int position, hymba_kv_cache* kv, float* ssm_state, float* conv_state,
+                            const hymba_bf16* residual, hymba_bf16* out, const float* norm_gain, float norm_eps,
+                            hymba_bf16* norm_out, void* workspace, size_t ws_bytes, hymba_stream stream);
+int hymba_ffn_swiglu_decode_norm(const hymba_bf16* h, const hymba_bf16* w_gate_up, const hymba_f16* w_down, int rows,
+                                 int d, int F, const hymba_bf16* residual, hymba_bf16* out, const float* norm_gain,
+                                 float norm_eps, hymba_bf16* norm_out, void* workspace, size_t ws_bytes,
+                                 hymba_stream stream);
+
 /* L2 prefetch hint for read-only device ranges that a later kernel on another stream (or
  * later on this one) will stream, e.g. the weights of a decode step's projections while the
  * latency-bound attention and scan kernels before them run.  ranges[i] / bytes[i]: up to 8

@@ -469,6 +469,55 @@ def test_ffn_swiglu_decode(rows):
     assert_rms(to_np(out), to_np(out2), name=f"decode FFN vs prefill FFN ({rows} rows)")
 
 
+@pytest.mark.parametrize("is_global", [False, True])
+def test_decode_norm_variants_equal_the_plain_calls_then_rmsnorm(is_global):
+    """hymba_mixer_decode_norm and hymba_ffn_swiglu_decode_norm: out bit for bit what the plain
+    calls write, and norm_out what hymba_rmsnorm computes from it (the same bf16 row; only the
+    order of the sum of squares differs)."""
+    dims = WL["tiny"].dims.replace(is_global=is_global, window=16)
+    w = _w(dims, seed=31)
+    N = 60
+    X = synth.bf16_round(np.random.default_rng(32).normal(size=(2, N + 1, dims.d_model)).astype(np.float32))
+    T = dims.n_meta + N
+    run = PrefillRun(dims, w, X[:, :N], max_tokens=T + 1)
+    ssm0, conv0 = run.ssm.clone(), run.conv.clone()
+    dw = H.DeviceWeights(w)
+    B, d = 2, dims.d_model
+    x, res = bf16_dev(X[:, N]), bf16_dev(X[:, N - 1])
+    g = torch.from_numpy(np.random.default_rng(33).normal(1.0, 0.1, size=d).astype(np.float32)).cuda()
+    ws = H.alloc_workspace(H.workspace_size(dims, B, T + 1, 0, H.MODE_DECODE))
+    out_a = torch.empty(B, d, dtype=torch.bfloat16, device="cuda")
+    H.mixer_decode(dims, dw, x, T, run.cache, run.ssm, run.conv, out_a, ws, residual=res)
+    norm_a = torch.empty_like(out_a)
+    H.rmsnorm(out_a, g, 1e-6, norm_a)
+    ssm_a = run.ssm.clone()
+    run.ssm.copy_(ssm0)
+    run.conv.copy_(conv0)
+    out_b, norm_b = torch.empty_like(out_a), torch.empty_like(out_a)
+    H.mixer_decode_norm(dims, dw, x, T, run.cache, run.ssm, run.conv, out_b, g, 1e-6, norm_b, ws, residual=res)
+    torch.cuda.synchronize()
+    assert H.status_read(ws) == 0
+    assert torch.equal(out_a, out_b)
+    assert torch.equal(ssm_a, run.ssm)
+    assert_rms(to_np(norm_b), to_np(norm_a), tol=1e-2, name="mixer decode fused norm vs rmsnorm")
+    # the FFN of the same rows (stack sizes d 1600 need not apply: tiny d_model, F a multiple of 64)
+    F = 256
+    bw = synth.block_weights(dims, F, seed=34, layer=0)
+    w_gu = torch.from_numpy(H.interleave_gate_up(bw["w_gate"], bw["w_up"])).cuda().to(torch.bfloat16)
+    w_dn = torch.from_numpy(bw["w_down"]).cuda().to(torch.float16)
+    fws = H.alloc_workspace(H.ffn_workspace_size(B, d, F))
+    f_a, f_b = torch.empty_like(out_a), torch.empty_like(out_a)
+    H.ffn_swiglu_decode(norm_a, w_gu, w_dn, f_a, fws, residual=out_a)
+    fn_a = torch.empty_like(out_a)
+    H.rmsnorm(f_a, g, 1e-6, fn_a)
+    fn_b = torch.empty_like(out_a)
+    H.ffn_swiglu_decode_norm(norm_a, w_gu, w_dn, f_b, g, 1e-6, fn_b, fws, residual=out_a)
+    torch.cuda.synchronize()
+    assert H.status_read(fws) == 0
+    assert torch.equal(f_a, f_b)
+    assert_rms(to_np(fn_b), to_np(fn_a), tol=1e-2, name="FFN decode fused norm vs rmsnorm")
+
+
 def test_l2_prefetch_hint_runs_and_writes_nothing():
     """hymba_l2_prefetch enqueues its bulk L2 prefetches for up to 8 ranges (odd sizes
     included) on a stream and leaves every byte as it was."""
