@@ -1612,9 +1612,14 @@ int hymba_rmsnorm(const hymba_bf16* x, const float* gain, int rows, int d, float
       !aligned16(out))
     return fail(HYMBA_ERR_INVALID_ARG, "rmsnorm arguments");
   prof_begin("rmsnorm", (cudaStream_t)stream);
+  if (d <= 32 * 8 * RMSW_MAXV && aligned16(gain)) {   // a warp per row
+    HY_CUDA(launch_pdl(rmsnorm_warp_kernel, dim3(cdiv(rows, 8)), dim3(256), 0, (cudaStream_t)stream,
+                       reinterpret_cast<const __nv_bfloat16*>(x), gain, rows, d, eps, reinterpret_cast<__nv_bfloat16*>(out)));
+  } else {
     HY_CUDA(launch_pdl(rmsnorm_kernel, dim3(rows), dim3(256), 0, (cudaStream_t)stream, reinterpret_cast<const __nv_bfloat16*>(x), gain, d, eps,
-                                                          reinterpret_cast<__nv_bfloat16*>(out)));
-    prof_end((cudaStream_t)stream);
+                       reinterpret_cast<__nv_bfloat16*>(out)));
+  }
+  prof_end((cudaStream_t)stream);
   HY_CUDA(cudaGetLastError());
   return HYMBA_OK;
 }

@@ -883,6 +883,49 @@ __global__ void __launch_bounds__(1024)
   }
 }
 
+// The same, one warp per row (8 rows per 256-thread CTA), the row held in registers between
+// the sum of squares and the store: for many rows of up to 4096 elements, where one CTA per
+// row leaves each CTA too little work to cover its own memory latency.
+constexpr int RMSW_MAXV = 16;   // 16-byte pieces per lane: d <= 32 * 8 * 16 = 4096
+__global__ void __launch_bounds__(256)
+    rmsnorm_warp_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ gain, int rows, int d,
+                        float eps, __nv_bfloat16* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const __nv_bfloat16* xr = x + row * d;
+  uint4 v[RMSW_MAXV];
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < RMSW_MAXV; ++k) {
+    const int c = (lane + 32 * k) * 8;
+    if (c < d) {
+      v[k] = *reinterpret_cast<const uint4*>(xr + c);
+      float f[8];
+      unpack8(v[k], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss += f[e] * f[e];
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float r = 1.f / sqrtf(ss / (float)d + eps);
+#pragma unroll
+  for (int k = 0; k < RMSW_MAXV; ++k) {
+    const int c = (lane + 32 * k) * 8;
+    if (c < d) {
+      float f[8];
+      unpack8(v[k], f);
+      const float4 g0 = *reinterpret_cast<const float4*>(gain + c), g1 = *reinterpret_cast<const float4*>(gain + c + 4);
+      *reinterpret_cast<uint4*>(out + row * d + c) =
+          make_uint4(pack_bf16x2(f[0] * r * g0.x, f[1] * r * g0.y), pack_bf16x2(f[2] * r * g0.z, f[3] * r * g0.w),
+                     pack_bf16x2(f[4] * r * g1.x, f[5] * r * g1.y), pack_bf16x2(f[6] * r * g1.z, f[7] * r * g1.w));
+    }
+  }
+}
+
 // out[b] = [meta; x[b]] : meta [M, d], x [B, N, d] -> out [B, M+N, d] (16-byte pieces)
 __global__ void prepend_meta_kernel(const __nv_bfloat16* __restrict__ meta, const __nv_bfloat16* __restrict__ x,
                                     int B, int M, int N, int d, __nv_bfloat16* __restrict__ out) {

@@ -469,6 +469,19 @@ def test_ffn_swiglu_decode(rows):
     assert_rms(to_np(out), to_np(out2), name=f"decode FFN vs prefill FFN ({rows} rows)")
 
 
+@pytest.mark.parametrize("rows,d", [(1, 8), (7, 1600), (1000, 1600), (33, 4096), (9, 4104)])
+def test_rmsnorm_against_oracle(rows, d):
+    """hymba_rmsnorm (a warp per row up to d 4096, a CTA per row beyond) against the oracle's
+    RMSNorm of the same bf16 rows, elementwise at the bf16 unit roundoff."""
+    rng = np.random.default_rng(rows + d)
+    x = synth.bf16_round(rng.normal(size=(rows, d)).astype(np.float32) * 3.0)
+    g = rng.normal(1.0, 0.2, size=d).astype(np.float32)
+    out = torch.empty(rows, d, dtype=torch.bfloat16, device="cuda")
+    H.rmsnorm(bf16_dev(x), torch.from_numpy(g).cuda(), 1e-6, out)
+    torch.cuda.synchronize()
+    assert_elem(to_np(out), orc.rmsnorm(x, g, 1e-6), name=f"rmsnorm {rows}x{d}")
+
+
 @pytest.mark.parametrize("is_global", [False, True])
 def test_decode_norm_variants_equal_the_plain_calls_then_rmsnorm(is_global):
     """hymba_mixer_decode_norm and hymba_ffn_swiglu_decode_norm: out bit for bit what the plain
