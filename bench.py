@@ -763,7 +763,7 @@ TRAFFIC = {
     "in_proj": 35381760 + 1385216,
     "conv1d_silu": 13999616 + 0,
     "x_proj": 14809344 + 768,
-    "dt_proj": 2453504 + 0,
+    "dt_proj": 2456576 + 0,
     "attention": 9817344 + 0,
     "scan_chunk_end": 42369280 + 16128,
     "scan_carry": 6089472 + 0,
