@@ -1,5 +1,6 @@
 // SSM branch kernels (prefill): causal depthwise conv1d + SiLU, and the selective scan.
 #pragma once
+#include <type_traits>
 #include "common.cuh"
 
 namespace hymba {
@@ -256,11 +257,15 @@ __global__ void __launch_bounds__(SC_THREADS, SC_PER_SM)
   // one step: decays, h = a h + dx B, and (output pass) y = C . h with two independent
   // accumulators; B and C are read as (state 2q, state 2q+1) pairs straight into 64-bit
   // registers
-  auto step = [&](const ScStage& S, int i, __nv_bfloat16* yp) {
+  // POW: the decay path, a template argument so that a stage's unrolled steps hold no branch
+  // and the scheduler can overlap one step's softplus and decays with the previous step's
+  // state update
+  auto step = [&](auto pow_c, const ScStage& S, int i, __nv_bfloat16* yp) {
+    constexpr bool POW = decltype(pow_c)::value;
     const float d = softplus_sel(S.d[i][tid] + bias);   // delta of this step and channel
     const float dx = d * __bfloat162float(S.x[i][tid]);
     uint64_t a[8];
-    if (pow_path) scan_decays_pow(d, A20, a);
+    if constexpr (POW) scan_decays_pow(d, A20, a);
     else scan_decays_general(d, A2, a);
     const uint64_t dxp = f2_pack(dx, dx);
     const ulonglong2* bc = reinterpret_cast<const ulonglong2*>(&S.bc[i][0]);   // the same address in every lane
@@ -294,11 +299,21 @@ __global__ void __launch_bounds__(SC_THREADS, SC_PER_SM)
       const ScStage& S = sm.st[j % SC_NST];
       __nv_bfloat16* yj = yrow + (size_t)(j * SC_SUB) * p.Di;
       const int n_steps = t1 - t0 - j * SC_SUB;
+      using pow_t = std::integral_constant<bool, true>;
+      using gen_t = std::integral_constant<bool, false>;
       if (n_steps >= SC_SUB) {
+        if (pow_path) {
 #pragma unroll
-        for (int i = 0; i < SC_SUB; ++i) step(S, i, yj + (size_t)i * p.Di);
+          for (int i = 0; i < SC_SUB; ++i) step(pow_t{}, S, i, yj + (size_t)i * p.Di);
+        } else {
+#pragma unroll
+          for (int i = 0; i < SC_SUB; ++i) step(gen_t{}, S, i, yj + (size_t)i * p.Di);
+        }
       } else {
-        for (int i = 0; i < n_steps; ++i) step(S, i, yj + (size_t)i * p.Di);
+        for (int i = 0; i < n_steps; ++i) {
+          if (pow_path) step(pow_t{}, S, i, yj + (size_t)i * p.Di);
+          else step(gen_t{}, S, i, yj + (size_t)i * p.Di);
+        }
       }
     }
     if (__syncthreads_or(ok ? 0 : 1)) break;   // a wait gave up: every thread leaves together
