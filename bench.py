@@ -765,9 +765,9 @@ TRAFFIC = {
     "x_proj": 14809344 + 768,
     "dt_proj": 2456576 + 0,
     "attention": 9817344 + 0,
-    "scan_chunk_end": 42369280 + 16128,
+    "scan_chunk_end": 42719744 + 20224,
     "scan_carry": 6089472 + 0,
-    "selective_scan": 48214272 + 553472,
+    "selective_scan": 48223488 + 587008,
     "norm_avg": 41828864 + 295680,
     "out_proj": 36304640 + 74496,
     "decode_ssm": 16950784 + 0,
