@@ -771,6 +771,8 @@ TRAFFIC = {
     "norm_avg": 41828864 + 295680,
     "out_proj": 36304640 + 74496,
     "decode_ssm": 16950784 + 0,
+    "decode_attn": 94806016 + 3106048,
+    "decode_prep": 5320192 + 0,
 }
 
 
