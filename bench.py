@@ -97,10 +97,10 @@ def scan_chunks(B, Di, T):
 
 
 def scan_bytes(dims, B, T):
-    """Compulsory HBM bytes of the selective scan as a whole: x (bf16), delta (fp32) and
+    """Compulsory HBM bytes of the selective scan as a whole: x (bf16), dt_pre (bf16) and
     B | C (fp32) in, y (bf16) and the final state (fp32) out."""
     rows, Di = B * T, dims.d_inner
-    return rows * Di * (2 + 4 + 2) + rows * 2 * dims.d_state * 4.0 + B * Di * dims.d_state * 4.0
+    return rows * Di * (2 + 2 + 2) + rows * 2 * dims.d_state * 4.0 + B * Di * dims.d_state * 4.0
 
 
 def prefill_work(dims, B, T):
@@ -120,9 +120,9 @@ def prefill_work(dims, B, T):
         "out_proj": ("tensor", 2.0 * rows * d * dims.out_in_width),
         # memory-bound kernels: compulsory bytes
         "conv1d_silu": ("hbm", rows * Di * 2.0 * 2),
-        "scan_chunk_end": ("hbm", rows_a * (Di * (4 + 2) + S * 4.0) + carry),
+        "scan_chunk_end": ("hbm", rows_a * (Di * (2 + 2) + S * 4.0) + carry),
         "scan_carry": ("hbm", 2 * carry),
-        "selective_scan": ("hbm", rows * (Di * (4 + 2 + 2) + 2 * S * 4.0) + B * Di * S * 4.0 + carry),
+        "selective_scan": ("hbm", rows * (Di * (2 + 2 + 2) + 2 * S * 4.0) + B * Di * S * 4.0 + carry),
         "norm_avg": ("hbm", rows * (dims.attn_width * 4.0 + Di * 2 * 2 + dims.out_in_width * 2)),
     }
     # exponentials of the recurrence, one per (row, channel, state) in each pass that walks it
@@ -763,11 +763,8 @@ TRAFFIC = {
     "in_proj": 35381760 + 1385216,
     "conv1d_silu": 13999616 + 0,
     "x_proj": 14809344 + 768,
-    "dt_proj": 2456576 + 0,
     "attention": 9817344 + 0,
-    "scan_chunk_end": 42719744 + 20224,
     "scan_carry": 6089472 + 0,
-    "selective_scan": 48223488 + 587008,
     "norm_avg": 41828864 + 295680,
     "out_proj": 36304640 + 74496,
     "decode_ssm": 16950784 + 0,

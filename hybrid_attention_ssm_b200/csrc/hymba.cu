@@ -303,9 +303,9 @@ template <int ET, int MODE>
 int launch_gemm_bn(int bn, const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& mb, const GemmParams& p,
                    int grid, cudaStream_t st, const char* name) {
   constexpr bool any_bn = MODE == EPI_F32_PART || MODE == EPI_F32_T || MODE == EPI_F32_T_PART;
-  if constexpr (MODE == EPI_F32_ROWS) {   // short K (dt_rank): 4 stages, room for the staging tiles
+  if constexpr (MODE == EPI_F32_ROWS || ET == ET_TF32) {   // short K (dt_rank): 4 stages, room for the staging tiles
     if (bn == 128) return launch_gemm_inst<128, 4, ET, MODE>(m0, m1, mb, p, grid, st, name);
-    return fail(HYMBA_ERR_UNSUPPORTED, "no GEMM instance for tile width %d with the row-store epilogue", bn);
+    return fail(HYMBA_ERR_UNSUPPORTED, "no GEMM instance for tile width %d with tf32 or the row-store epilogue", bn);
   } else {
     if (bn == 256) return launch_gemm_inst<256, 4, ET, MODE>(m0, m1, mb, p, grid, st, name);
     if constexpr (MODE != EPI_PROJ) {
@@ -340,6 +340,7 @@ int launch_gemm_mode(const GemmCall& c, const CUtensorMap& m0, const CUtensorMap
     case EPI_BF16:
       if (c.etype == ET_BF16) return launch_gemm_bn<ET_BF16, EPI_BF16>(c.bn, m0, m1, mb, p, grid, st, c.name);
       if (c.etype == ET_F16) return launch_gemm_bn<ET_F16, EPI_BF16>(c.bn, m0, m1, mb, p, grid, st, c.name);
+      if (c.etype == ET_TF32) return launch_gemm_bn<ET_TF32, EPI_BF16>(c.bn, m0, m1, mb, p, grid, st, c.name);
       break;
     case EPI_SWIGLU:
       if (c.etype == ET_BF16) return launch_gemm_bn<ET_BF16, EPI_SWIGLU>(c.bn, m0, m1, mb, p, grid, st, c.name);
@@ -620,7 +621,7 @@ PrefillWs prefill_layout(const Dims& m, int B, int n_tokens, int x_has_meta, int
   w.xbc = take(rows * m.ld_xbc * 4);
   w.xproj_split = splits_for(cdiv((long long)rows, GEMM_BM), cdiv(m.Di, 64), 16);
   w.xbc_part = take((size_t)w.xproj_split * rows * m.ld_xbc * 4);
-  w.dt_pre = take(rows * m.Di * 4);
+  w.dt_pre = take(rows * m.Di * 2);
   w.y = take(rows * m.Di * 2);
   w.o = take(rows * m.qw * 4);
   w.u = take(rows * m.uw * 2);
@@ -1066,8 +1067,9 @@ static int prefill_impl(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     prof_end(st);
     HY_CUDA(cudaGetLastError());
   }
-  // 4. dt_proj (tf32): dt_pre = dt_low W_dt^T [B*T, Di] fp32 (the scan adds dt_bias and
-  //    applies the softplus as it reads it)
+  // 4. dt_proj (tf32): dt_pre = dt_low W_dt^T [B*T, Di], stored bf16 (the scan adds dt_bias
+  //    and applies the softplus in fp32 as it reads it).  The GEMM is bound by its stores
+  //    (K = dt_rank is short), so the 16-bit rows halve its time and the scan's reads.
   {
     GemmCall c;
     c.etype = ET_TF32;
@@ -1075,8 +1077,8 @@ static int prefill_impl(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     c.b = w->w_dt; c.N = m.Di; c.ldb = w->w_dt_ld; c.K = m.R;
     c.bn = 128;
     c.name = "dt_proj";
-    c.mode = EPI_F32_ROWS;
-    c.p.out = f32(L.dt_pre);
+    c.mode = EPI_BF16;
+    c.p.out = bf(L.dt_pre);
     c.p.ld_out = m.Di;
     c.p.n_valid = m.Di;
     c.p.status = status;
@@ -1117,9 +1119,9 @@ static int prefill_impl(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     CUtensorMap md, mx, mbc;
     {
       const uint64_t dims[2] = {(uint64_t)m.Di, (uint64_t)rows};
-      const uint64_t str[1] = {(uint64_t)m.Di * 4};
+      const uint64_t str[1] = {(uint64_t)m.Di * 2};
       const uint32_t box[2] = {SC_CH, SC_SUB};
-      HY_TRY(make_map(&md, f32(L.dt_pre), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE));
+      HY_TRY(make_map(&md, bf(L.dt_pre), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE));
     }
     {
       const uint64_t dims[2] = {(uint64_t)m.Di, (uint64_t)rows};

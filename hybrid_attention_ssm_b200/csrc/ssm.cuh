@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(256)
 // A lane owns one (sequence, channel, chunk) and the channel's 16 states in registers, so
 // y_t = C_t . h_t is a sum inside the lane and B_t, C_t are the same for every lane of the
 // CTA (shared-memory broadcasts).  CTA = 64 channels (two warps) of one chunk; dt_pre
-// [rows, Di] fp32 (dt_low W_dt^T), x [rows, Di] bf16 and (B | C) [rows, 32] fp32 stream in by
+// [rows, Di] bf16 (dt_low W_dt^T), x [rows, Di] bf16 and (B | C) [rows, 32] fp32 stream in by
 // TMA, 8 steps per stage, all in their row-major producer layouts.  dt_proj's bias and
 // softplus are applied here, as each step is read: delta = softplus(dt_pre + dt_bias), in
 // both passes, instead of a pass of their own over [rows, Di].
@@ -120,11 +120,11 @@ constexpr int SC_THREADS = SC_CH;
 constexpr int SC_PER_SM = 10;  // CTAs resident per SM (the register budget of __launch_bounds__)
 
 struct ScStage {
-  float d[SC_SUB][SC_CH];            // dt_pre rows   (box {64, 8} fp32, 2048 B)
+  __nv_bfloat16 d[SC_SUB][SC_CH];    // dt_pre rows   (box {64, 8} bf16, 1024 B)
   __nv_bfloat16 x[SC_SUB][SC_CH];    // x rows        (box {64, 8} bf16, 1024 B)
   float bc[SC_SUB][32];              // B | C rows    (box {32, 8} fp32, 1024 B)
 };
-static_assert(sizeof(ScStage) == 4096, "stage layout must match the TMA boxes");
+static_assert(sizeof(ScStage) == 3072, "stage layout must match the TMA boxes");
 
 struct ScSmem {
   ScStage st[SC_NST];
@@ -262,7 +262,7 @@ __global__ void __launch_bounds__(SC_THREADS, SC_PER_SM)
   // state update
   auto step = [&](auto pow_c, const ScStage& S, int i, __nv_bfloat16* yp) {
     constexpr bool POW = decltype(pow_c)::value;
-    const float d = softplus_sel(S.d[i][tid] + bias);   // delta of this step and channel
+    const float d = softplus_sel(__bfloat162float(S.d[i][tid]) + bias);   // delta of this step and channel
     const float dx = d * __bfloat162float(S.x[i][tid]);
     uint64_t a[8];
     if constexpr (POW) scan_decays_pow(d, A20, a);

@@ -292,7 +292,7 @@ int hymba_mixer_decode_ragged(const hymba_layer_cfg* cfg, const hymba_layer_weig
  *   xz     [B*T, 2*Di]  bf16  in_proj x | z columns
  *   xc     [B*T, Di]    bf16  SiLU(conv(x))
  *   xbc    [B*T, ld_xbc] fp32 x_proj output: dt_low | B | C
- *   dt_pre [B*T, Di]    fp32  dt_low W_dt^T (the scan applies softplus(. + dt_bias))
+ *   dt_pre [B*T, Di]    bf16  dt_low W_dt^T (the scan applies softplus(. + dt_bias) in fp32)
  *   y      [B*T, Di]    bf16  scan output before the gate
  *   o      [B*T, Hq*D]  fp32  attention output
  *   u      [B*T, Hq*D+Di] fp16 normalised, rescaled, averaged branches (out_proj input)

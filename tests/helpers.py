@@ -97,7 +97,7 @@ class PrefillRun:
             "xz": (L.xz, (B, T, 2 * d.d_inner), torch.bfloat16),
             "xc": (L.xc, (B, T, d.d_inner), torch.bfloat16),
             "xbc": (L.xbc, (B, T, L.ld_xbc), torch.float32),
-            "dt_pre": (L.dt_pre, (B, T, d.d_inner), torch.float32),
+            "dt_pre": (L.dt_pre, (B, T, d.d_inner), torch.bfloat16),
             "y": (L.y, (B, T, d.d_inner), torch.bfloat16),
             "o": (L.o, (B, T, d.n_q_heads * d.head_dim), torch.float32),
             "u": (L.u, (B, T, d.attn_width + d.d_inner), torch.float16),
