@@ -764,7 +764,9 @@ TRAFFIC = {
     "conv1d_silu": 13999616 + 0,
     "x_proj": 14809344 + 768,
     "attention": 9817344 + 0,
+    "scan_chunk_end": 28550400 + 256,
     "scan_carry": 6089472 + 0,
+    "selective_scan": 34297856 + 210688,
     "norm_avg": 41828864 + 295680,
     "out_proj": 36304640 + 74496,
     "decode_ssm": 16950784 + 0,

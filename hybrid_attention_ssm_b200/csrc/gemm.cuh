@@ -28,7 +28,7 @@ enum EpiMode : int {
   EPI_PROJ = 0,         // segmented bf16/fp16 stores with RoPE on marked segments (in_proj)
   EPI_BF16 = 1,         // bf16 store, optional bf16 residual add
   EPI_SWIGLU = 2,       // columns interleaved [gate(32) | up(32)] -> fp16 SiLU(gate)*up
-  EPI_F32_ROWS = 3,     // fp32 row-major store out[row * ld_out + col], 128-byte rows per store
+  // 3: unused (formerly an fp32 row store)
   EPI_F32_T = 4,        // transposed fp32 store: out[n][m] (weights as the M operand)
   EPI_F32_PART = 5,     // fp32 store of split ks's partial sum at out + ks*split_stride (row-major)
   EPI_F32_T_PART = 6,   // the same, transposed
@@ -96,16 +96,13 @@ constexpr int GEMM_EPI_WARPS = 8;
 constexpr int GEMM_THREADS = 64 + 32 * GEMM_EPI_WARPS;
 constexpr int GEMM_BM = 128;
 
-// Shared memory an epilogue stages its output through: EPI_F32_ROWS transposes each warp's
-// 32 x 32 fp32 block (rows padded to 36 words) so that every store writes four whole rows;
-// EPI_BF16 exchanges each warp's 32 x 32 bf16 block (rows of 64 bytes padded to 80) so that
-// four lanes load or store one row's 64 bytes (two whole 32-byte sectors) instead of each lane
-// touching 16 bytes of its own row.
+// Shared memory an epilogue stages its output through: EPI_BF16 exchanges each warp's
+// 32 x 32 bf16 block (rows of 64 bytes padded to 80) so that four lanes load or store one
+// row's 64 bytes (two whole 32-byte sectors) instead of each lane touching 16 bytes of its
+// own row.
 constexpr int GEMM_BF16_TILE_WORDS = 20;   // words per staged row
 __host__ __device__ constexpr int gemm_epi_bytes(int mode) {
-  return mode == 3 /* EPI_F32_ROWS */ ? GEMM_EPI_WARPS * 32 * 36 * 4
-         : mode == 1 /* EPI_BF16 */   ? GEMM_EPI_WARPS * 32 * GEMM_BF16_TILE_WORDS * 4
-                                      : 0;
+  return mode == 1 /* EPI_BF16 */ ? GEMM_EPI_WARPS * 32 * GEMM_BF16_TILE_WORDS * 4 : 0;
 }
 
 template <int BN, int STAGES, int EPI_BYTES = 0, bool PAIR = false>
@@ -463,38 +460,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
               const int orow_t = gc + e;
               if (orow_t < p.n_valid) outf[(size_t)orow_t * p.ld_out + rr] = v[e];
             }
-            return;
-          }
-          if constexpr (MODE == EPI_F32_ROWS) {
-            // the warp's 32 rows x 32 columns, transposed through this warp's shared tile
-            // (rows padded to 36 words, so that 16-byte writes by row and 16-byte reads by
-            // quarter row are both conflict-free): each store instruction writes four whole
-            // 128-byte rows, eight lanes per row
-            if (gc >= p.n_valid) return;          // the same for the whole warp
-            float* tile = reinterpret_cast<float*>(smem + L::EPI_OFFSET) + (warp - 2) * (32 * 36);
-#pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              *reinterpret_cast<float4*>(tile + lane * 36 + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-            __syncwarp();
-            const int rows_valid = src0 ? p.rows0 : p.rows1;
-            const int rr0 = rr - lane;            // accumulator row of lane 0
-            float* dst0 = reinterpret_cast<float*>(p.out) + ((size_t)b1 * p.rows1 + rr0) * p.ld_out + gc;
-            if (gc + 32 <= p.n_valid && (p.ld_out & 3) == 0) {
-              const int r4 = lane >> 3, c4 = (lane & 7) * 4;
-#pragma unroll
-              for (int q = 0; q < 32; q += 4) {
-                const int row = q + r4;
-                if (rr0 + row < rows_valid)
-                  *reinterpret_cast<float4*>(dst0 + (size_t)row * p.ld_out + c4) =
-                      *reinterpret_cast<const float4*>(tile + row * 36 + c4);
-              }
-            } else {
-              const bool col_ok = gc + lane < p.n_valid;
-#pragma unroll 4
-              for (int q = 0; q < 32; ++q)
-                if (rr0 + q < rows_valid && col_ok) dst0[(size_t)q * p.ld_out + lane] = tile[q * 36 + lane];
-            }
-            __syncwarp();
             return;
           }
           if constexpr (MODE == EPI_BF16) {
