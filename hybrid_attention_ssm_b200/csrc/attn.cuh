@@ -3,7 +3,8 @@
 // finer than bf16), fp32 scores and accumulators.
 //
 // Persistent: two CTAs per SM (256 TMEM columns and 113 KB of shared memory each) loop over
-// the (query tile of 128 rows, query head, sequence) work items, heaviest first, so one
+// the (query tile of 128 rows, query head, sequence) work items, heaviest first in a snake
+// order over the CTAs (attn_slot_item), so one
 // CTA's softmax overlaps the other's MMAs and no wave is left half empty.  The TMA warp
 // prefetches the next item's Q and K/V while the current item finishes.  The key tiles a CTA visits are the meta-token tiles plus the tiles that
 // intersect the sliding window of its rows (every causal tile for a global layer): block
@@ -151,6 +152,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// The work item a CTA takes on its k-th pass over the grid: passes go through the items in
+// order (longest query tiles first), the odd passes in reverse CTA order, so the CTAs whose
+// first item was among the shortest of its pass get the longest of the next (a snake order).
+// Item indices grow with k for every CTA, so the first index past the end ends the loop.
+__device__ __forceinline__ int attn_slot_item(int k, int grid, int cta) {
+  return k * grid + ((k & 1) ? grid - 1 - cta : cta);
+}
+
 // work item w -> (query tile, head, sequence); longest query tiles first
 __device__ __forceinline__ void attn_item(const AttnParams& p, int w, int B, int& qt, int& h, int& b) {
   const int per_qt = p.Hq * B;
@@ -222,7 +231,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       tma_prefetch_desc(&mapV);
       int gi = 0, it = 0;                    // tiles and items issued by this CTA
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x, ++it) {
+      for (int k = 0, w = attn_slot_item(0, gridDim.x, blockIdx.x); ok && w < p.n_items;
+           ++k, w = attn_slot_item(k, gridDim.x, blockIdx.x), ++it) {
         int qt, h, b;
         attn_item(p, w, B, qt, h, b);
         const int g = (h * p.Hkv) / p.Hq;
@@ -270,7 +280,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       };
       int gi = 0, it = 0;
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x, ++it) {
+      for (int k = 0, w = attn_slot_item(0, gridDim.x, blockIdx.x); ok && w < p.n_items;
+           ++k, w = attn_slot_item(k, gridDim.x, blockIdx.x), ++it) {
         int qt, h, b;
         attn_item(p, w, B, qt, h, b);
         const int n_tiles = key_tiles(p, qt).count();
@@ -310,7 +321,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
 
     int gi = 0;
     bool ok = true;
-    for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
+    for (int k = 0, w = attn_slot_item(0, gridDim.x, blockIdx.x); ok && w < p.n_items;
+         ++k, w = attn_slot_item(k, gridDim.x, blockIdx.x)) {
       int qt, h, b;
       attn_item(p, w, B, qt, h, b);
       const KeyTiles kts = key_tiles(p, qt);
