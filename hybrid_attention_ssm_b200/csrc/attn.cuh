@@ -2,14 +2,14 @@
 // Q/K/V/P (keys, values and probabilities sit far inside fp16's range, where it rounds 8x
 // finer than bf16), fp32 scores and accumulators.
 //
-// Persistent: two CTAs per SM (256 TMEM columns and 113 KB of shared memory each) loop over
-// the (query tile of 128 rows, query head, sequence) work items, heaviest first in a snake
-// order over the CTAs (attn_slot_item), so one
-// CTA's softmax overlaps the other's MMAs and no wave is left half empty.  The TMA warp
-// prefetches the next item's Q and K/V while the current item finishes.  The key tiles a CTA visits are the meta-token tiles plus the tiles that
-// intersect the sliding window of its rows (every causal tile for a global layer): block
-// skipping, no dense mask.  Only tiles that straddle the causal diagonal or the window
-// edge apply an element mask.
+// Persistent: two CTAs per SM (256 TMEM columns and 113 KB of shared memory each), so one
+// CTA's softmax overlaps the other's MMAs, loop over the (query tile of 128 rows, query head,
+// sequence) work items, heaviest first and dealt in a snake order over the CTAs
+// (attn_slot_item), so that no CTA is left with a much longer list than the rest.  The TMA
+// warp prefetches the next item's Q and K/V while the current item finishes.  The key tiles
+// a CTA visits are the meta-token tiles plus the tiles that intersect the sliding window of
+// its rows (every causal tile for a global layer): block skipping, no dense mask.  Only
+// tiles that straddle the causal diagonal or the window edge apply an element mask.
 //
 // 192 threads:
 //   warp 0      TMA: Q once, K/V tiles through a 3-stage ring
