@@ -396,7 +396,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
           rsp[(e >> 1) & 7] += p0 + p1;
           pk[e >> 1] = pack_f16x2(p0, p1);
         }
-        l_run += ((rsp[0] + rsp[1]) + (rsp[2] + rsp[3])) + ((rsp[4] + rsp[5]) + (rsp[6] + rsp[7]));
+        // the sum so far was taken against the old maximum: rescale it before this tile's
+        // terms (taken against the new one) are added (alpha = 1 without a rescale)
+        l_run = fmaf(l_run, alpha, ((rsp[0] + rsp[1]) + (rsp[2] + rsp[3])) + ((rsp[4] + rsp[5]) + (rsp[6] + rsp[7])));
         // PV of the previous tile must be done before P is replaced and O rescaled
         if (i >= 1 && !wait_bar(o_done, gi - 1, 207)) { ok = false; break; }
         if (__any_sync(0xffffffffu, resc)) {
@@ -408,7 +410,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
             for (int d = 0; d < 32; ++d) o[d] *= alpha;
             tmem_st32(TM_O + lane_off + hcol, reinterpret_cast<const uint32_t*>(o));
           }
-          l_run *= alpha;
         }
         tmem_st32(TM_P + lane_off, pk);
         tmem_st32(TM_P + lane_off + 32, pk + 32);

@@ -145,6 +145,42 @@ def test_prefill_edge_shapes(kw):
     _check_stages(run, ref, dims, w)
 
 
+@pytest.mark.parametrize("is_global,window", [(1, 32), (0, 200)])
+def test_attention_running_max_growth(is_global, window):
+    """Scores that grow along each row, so the running maximum of the online softmax rises
+    by more than the kernel's lazy-rescale threshold (2^8) from one key tile to the next: the
+    attention output, fed the GPU's own Q, K, V, against the oracle's dense softmax.  The
+    test checks on the CPU that its inputs do reach that path."""
+    dims = WL["tiny"].dims.replace(is_global=is_global, window=window)
+    w = _w(dims, seed=61)
+    qk = dims.attn_width + 2 * dims.n_kv_heads * dims.head_dim     # Q and K rows of W_in
+    w_in = w["w_in"].copy()
+    w_in[:qk] = synth.bf16_round(w_in[:qk] * 10.0)
+    w = dict(w, w_in=w_in)
+    N = 500
+    T = dims.n_meta + N
+    rng = np.random.default_rng(62)
+    grow = (0.5 + 3.0 * np.arange(N) / N)[None, :, None]            # later rows larger
+    X = synth.bf16_round((rng.normal(size=(1, N, dims.d_model)) * grow).astype(np.float32))
+    run = PrefillRun(dims, w, X)
+    q, o = run.stage("q")[0], run.stage("o")[0]
+    k, v = run.kv()
+    k, v = k[0], v[0]
+    pos = np.arange(T)
+    o_ref = orc.attention(q, k, v, pos, pos, dims.n_meta, dims.window, dims.is_global)
+    assert_rms(o, o_ref.reshape(T, -1), name="attention, growing scores")
+    # the case is the intended one: some row's running max (log2 units, per 128-key tile in
+    # the order the kernel visits them) grows by more than 8 at some tile
+    g = dims.n_q_heads // dims.n_kv_heads
+    vis = orc.visibility_mask(pos, pos, dims.n_meta, dims.window, dims.is_global)
+    s = np.einsum("thd,shd->hts", q, np.repeat(k, g, axis=1)) * (np.log2(np.e) / np.sqrt(dims.head_dim))
+    s = np.where(vis[None], s, -np.inf)
+    tile_max = np.stack([s[:, :, j:j + 128].max(axis=2) for j in range(0, T, 128)], axis=2)
+    run_max = np.maximum.accumulate(tile_max, axis=2)
+    jumps = np.diff(np.where(np.isfinite(run_max), run_max, np.nan), axis=2)
+    assert np.nanmax(jumps) > 8.0, f"largest running-max step {np.nanmax(jumps):.1f} (log2 units)"
+
+
 def test_prefill_with_meta_in_input_and_residual():
     wl = WL["tiny"]
     dims = wl.dims
