@@ -763,7 +763,6 @@ TRAFFIC = {
     "in_proj": 35381760 + 1385216,
     "conv1d_silu": 13999616 + 0,
     "x_proj": 14809344 + 768,
-    "attention": 9818112 + 768,
     "scan_chunk_end": 28550400 + 256,
     "scan_carry": 6089472 + 0,
     "selective_scan": 34297856 + 210688,
