@@ -876,7 +876,7 @@ def main():
         line = {"impl": "reference", "metric": metric, "value": round(rate, 2), "unit": "tokens/s",
                 "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) inputs, N(0,0.02) weights)",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) inputs, N(0,0.02) weights, dt logits N(-4,1))",
                 "config": cfg,
                 "cpu_baseline": {"value": round(rate, 2), "unit": "tokens/s", "cores": oracle_threads(),
                                  "kind": "oracle",
