@@ -54,6 +54,18 @@ def test_scan_chunking_matches_bench_accounting(B, N, Di):
     assert dec > 0
 
 
+@pytest.mark.parametrize("T,M,W,is_global", [(2176, 128, 1024, 0), (300, 8, 32, 1), (270, 130, 100, 0),
+                                               (308, 8, 1, 0), (140, 0, 64, 0)])
+def test_bench_visible_pairs_equal_the_oracle_mask(T, M, W, is_global):
+    """The attention FLOPs in bench.py's roofline count the (query, key) pairs the oracle's
+    visibility mask allows (the SWA layer: 1,843,776 per head)."""
+    import bench
+    pos = np.arange(T)
+    assert bench.visible_pairs(T, M, W, is_global) == int(orc.visibility_mask(pos, pos, M, W, is_global).sum())
+    if (T, M, W) == (2176, 128, 1024):
+        assert bench.visible_pairs(T, M, W, is_global) == 1843776
+
+
 @pytest.mark.parametrize("field,value,code", [("head_dim", 32, H.ERR_UNSUPPORTED),
                                               ("d_state", 8, H.ERR_UNSUPPORTED),
                                               ("d_inner", 100, H.ERR_UNSUPPORTED),
